@@ -1,0 +1,342 @@
+/*
+ * bsa_oracle.c -- plain CPU oracle for block-sparse compressed-key decode attention.
+ *
+ * TEST INFRASTRUCTURE. Only the tests, the package's smoke check and the benchmark's CPU-baseline
+ * leg may load this library; the CUDA library shares no code with it. Each function follows one
+ * step of the method in double precision; the sources and the readings of the pages are listed in
+ * bsa_oracle.h. Build: gcc -O2 -std=c11 -fopenmp -ffp-contract=off -shared -fPIC.
+ */
+#include "bsa_oracle.h"
+
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+double bsa_oracle_load(const void* base, int dtype, int64_t i) {
+    if (dtype == ORC_F32) return (double)((const float*)base)[i];
+    /* bf16 is the upper half of an IEEE binary32 pattern */
+    uint32_t bits = (uint32_t)((const uint16_t*)base)[i] << 16;
+    float f;
+    memcpy(&f, &bits, sizeof f);
+    return (double)f;
+}
+
+double bsa_oracle_round(double x, int dtype) {
+    if (dtype == ORC_F32) return (double)(float)x; /* C conversion: nearest, ties to even */
+    if (x == 0.0 || isnan(x) || isinf(x)) return x;
+    /* bf16: 8 significant bits, binary32 exponent range (normal from 2^-126, subnormal step 2^-133) */
+    int e;
+    frexp(x, &e); /* |x| in [2^(e-1), 2^e) */
+    int lead = e - 1;
+    if (lead < -126) lead = -126;
+    double quantum = ldexp(1.0, lead - 7);
+    double r = rint(x / quantum) * quantum; /* rint: nearest, ties to even (default mode) */
+    if (fabs(r) >= ldexp(1.0, 128)) r = copysign(INFINITY, x);
+    return r;
+}
+
+void bsa_oracle_round_array(const double* x, int64_t n, int dtype, double* y) {
+    for (int64_t i = 0; i < n; ++i) y[i] = bsa_oracle_round(x[i], dtype);
+}
+
+int64_t bsa_oracle_num_windows(int64_t T, int l, int s) {
+    if (T < l) return 0;
+    return (T - l) / s + 1;
+}
+
+int64_t bsa_oracle_num_blocks(int64_t T, int block_size) {
+    return (T + block_size - 1) / block_size;
+}
+
+/* Theoretical Foundation, Eq. (2): K~_j = Mean(K[j*s : j*s + l]). */
+int64_t bsa_oracle_compress(const void* k, int dtype, int64_t T, int d, int l, int s,
+                            int round_dtype, double* ck) {
+    int64_t nc = bsa_oracle_num_windows(T, l, s);
+    for (int64_t j = 0; j < nc; ++j) {
+        for (int c = 0; c < d; ++c) {
+            double sum = 0.0;
+            for (int r = 0; r < l; ++r) sum += bsa_oracle_load(k, dtype, (j * s + r) * (int64_t)d + c);
+            double mean = sum / (double)l;
+            ck[j * d + c] = (round_dtype == ORC_NO_ROUND) ? mean : bsa_oracle_round(mean, round_dtype);
+        }
+    }
+    return nc;
+}
+
+/* Indexer Training, Eq. (6), target side: S = sum over the group's heads of softmax(q_h K~^T / tau). */
+void bsa_oracle_group_scores(const double* q, const double* ck, int64_t nc, int G, int d,
+                             double tau, double* S) {
+    for (int64_t j = 0; j < nc; ++j) S[j] = 0.0;
+    if (nc <= 0) return;
+    double* x = (double*)malloc((size_t)nc * sizeof(double));
+    for (int h = 0; h < G; ++h) {
+        double m = -INFINITY;
+        for (int64_t j = 0; j < nc; ++j) {
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) dot += q[h * d + c] * ck[j * d + c];
+            x[j] = dot / tau;
+            if (x[j] > m) m = x[j];
+        }
+        double z = 0.0;
+        for (int64_t j = 0; j < nc; ++j) z += exp(x[j] - m);
+        for (int64_t j = 0; j < nc; ++j) S[j] += exp(x[j] - m) / z;
+    }
+    free(x);
+}
+
+/* Fine-grained supervision: scores max-pooled down to the standard block grid. A window overlaps
+ * block b when it shares at least one token with [BS*b, BS*(b+1)). */
+void bsa_oracle_block_scores(const double* S, int64_t nc, int64_t nb, int l, int s,
+                             int block_size, double* sb) {
+    for (int64_t b = 0; b < nb; ++b) {
+        double best = -INFINITY;
+        for (int64_t j = 0; j < nc; ++j) {
+            int64_t first = j * s, end = j * s + l; /* tokens [first, end) */
+            if (first < (int64_t)block_size * (b + 1) && end > (int64_t)block_size * b) {
+                if (S[j] > best) best = S[j];
+            }
+        }
+        sb[b] = best;
+    }
+}
+
+typedef struct {
+    double score;
+    int64_t block;
+} orc_cand_t;
+
+/* Higher score first; equal scores: lower block index first. */
+static int orc_cand_cmp(const void* pa, const void* pb) {
+    const orc_cand_t* a = (const orc_cand_t*)pa;
+    const orc_cand_t* b = (const orc_cand_t*)pb;
+    if (a->score > b->score) return -1;
+    if (a->score < b->score) return 1;
+    return (a->block < b->block) ? -1 : (a->block > b->block);
+}
+
+/* Theoretical Foundation, Eq. (1), with SparDA Architecture, Eq. (4)'s f_top(., k). */
+int bsa_oracle_select(const double* sb, int64_t nb, int n_init, int n_local, int top_k,
+                      int32_t* idx, double* boundary) {
+    boundary[0] = NAN;
+    boundary[1] = NAN;
+    if (nb <= 0) return 0;
+    char* chosen = (char*)calloc((size_t)nb, 1);
+    int64_t init_end = n_init < nb ? n_init : nb;
+    int64_t local_begin = nb - n_local > 0 ? nb - n_local : 0;
+    for (int64_t b = 0; b < init_end; ++b) chosen[b] = 1;
+    for (int64_t b = local_begin; b < nb; ++b) chosen[b] = 1;
+
+    orc_cand_t* cand = (orc_cand_t*)malloc((size_t)nb * sizeof(orc_cand_t));
+    int64_t nc = 0;
+    for (int64_t b = 0; b < nb; ++b) {
+        if (!chosen[b]) {
+            cand[nc].score = sb[b];
+            cand[nc].block = b;
+            ++nc;
+        }
+    }
+    qsort(cand, (size_t)nc, sizeof(orc_cand_t), orc_cand_cmp);
+    int64_t take = top_k < nc ? top_k : nc;
+    for (int64_t i = 0; i < take; ++i) chosen[cand[i].block] = 1;
+    if (take > 0) boundary[0] = cand[take - 1].score;
+    if (take < nc) boundary[1] = cand[take].score;
+
+    int n = 0;
+    for (int64_t b = 0; b < nb; ++b)
+        if (chosen[b]) idx[n++] = (int32_t)b;
+    free(cand);
+    free(chosen);
+    return n;
+}
+
+/* SparDA Architecture, Eq. (5): O = Attn(Q, K[B], V[B]) over the tokens of the selected blocks. */
+void bsa_oracle_attend(const double* q, const void* k, const void* v, int dtype, int64_t T, int d,
+                       int G, const int32_t* idx, int n_sel, int block_size, double scale,
+                       double* out, double* lse) {
+    /* list the attended tokens */
+    int64_t n_tok = 0;
+    for (int i = 0; i < n_sel; ++i) {
+        if (idx[i] < 0) continue; /* -1 marks an unused slot */
+        int64_t lo = (int64_t)idx[i] * block_size, hi = lo + block_size;
+        if (hi > T) hi = T;
+        if (hi > lo) n_tok += hi - lo;
+    }
+    int64_t* tok = (int64_t*)malloc((size_t)(n_tok > 0 ? n_tok : 1) * sizeof(int64_t));
+    double* x = (double*)malloc((size_t)(n_tok > 0 ? n_tok : 1) * sizeof(double));
+    int64_t n = 0;
+    for (int i = 0; i < n_sel; ++i) {
+        if (idx[i] < 0) continue;
+        int64_t lo = (int64_t)idx[i] * block_size, hi = lo + block_size;
+        if (hi > T) hi = T;
+        for (int64_t t = lo; t < hi; ++t) tok[n++] = t;
+    }
+    for (int h = 0; h < G; ++h) {
+        double* o = out + (int64_t)h * d;
+        for (int c = 0; c < d; ++c) o[c] = 0.0;
+        if (n_tok == 0) {
+            lse[h] = -INFINITY;
+            continue;
+        }
+        double m = -INFINITY;
+        for (int64_t i = 0; i < n_tok; ++i) {
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c) dot += q[h * d + c] * bsa_oracle_load(k, dtype, tok[i] * d + c);
+            x[i] = dot * scale;
+            if (x[i] > m) m = x[i];
+        }
+        double z = 0.0;
+        for (int64_t i = 0; i < n_tok; ++i) z += exp(x[i] - m);
+        for (int64_t i = 0; i < n_tok; ++i) {
+            double w = exp(x[i] - m) / z;
+            for (int c = 0; c < d; ++c) o[c] += w * bsa_oracle_load(v, dtype, tok[i] * d + c);
+        }
+        lse[h] = m + log(z);
+    }
+    free(tok);
+    free(x);
+}
+
+static int orc_problem_ok(const orc_problem_t* P) {
+    if (!P) return 0;
+    if (P->batch < 1 || P->num_kv_heads < 1 || P->num_q_heads < 1) return 0;
+    if (P->num_q_heads % P->num_kv_heads) return 0;
+    if (P->head_dim < 1 || P->cmp_kernel < 1 || P->cmp_stride < 1 || P->block_size < 1) return 0;
+    if (P->n_init < 0 || P->n_local < 0 || P->top_k < 0 || P->max_seq_len < 1) return 0;
+    if (P->dtype != ORC_F32 && P->dtype != ORC_BF16) return 0;
+    return 1;
+}
+
+static size_t orc_elem_size(int dtype) { return dtype == ORC_F32 ? 4 : 2; }
+
+/* q rows of one group as doubles: heads kvh*G .. kvh*G + G - 1 of batch b. */
+static void orc_group_q(const orc_problem_t* P, const void* q, int b, int kvh, double* qg) {
+    int G = P->num_q_heads / P->num_kv_heads, d = P->head_dim;
+    for (int h = 0; h < G; ++h)
+        for (int c = 0; c < d; ++c)
+            qg[h * d + c] = bsa_oracle_load(
+                q, P->dtype, ((int64_t)b * P->num_q_heads + (int64_t)kvh * G + h) * d + c);
+}
+
+static const void* orc_pair_rows(const orc_problem_t* P, const void* cache, int pair) {
+    size_t off = (size_t)pair * (size_t)P->max_seq_len * (size_t)P->head_dim * orc_elem_size(P->dtype);
+    return (const char*)cache + off;
+}
+
+int bsa_oracle_decode(const orc_problem_t* P, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seq_lens, const int32_t* pairs,
+                      int n_pairs, const int32_t* given_idx, const int32_t* given_n_sel,
+                      int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary,
+                      double* out, double* lse) {
+    if (!orc_problem_ok(P) || n_pairs < 0) return -1;
+    const int G = P->num_q_heads / P->num_kv_heads, d = P->head_dim;
+    const int sel_cap = P->n_init + P->n_local + P->top_k;
+    const int64_t nb_cap = bsa_oracle_num_blocks(P->max_seq_len, P->block_size);
+    for (int i = 0; i < n_pairs; ++i) {
+        if (pairs[i] < 0 || pairs[i] >= P->batch * P->num_kv_heads) return -1;
+        int64_t T = seq_lens[pairs[i] / P->num_kv_heads];
+        if (T < 0 || T > P->max_seq_len) return -1;
+    }
+    int bad = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : bad)
+    for (int i = 0; i < n_pairs; ++i) {
+        const int pair = pairs[i], b = pair / P->num_kv_heads, kvh = pair % P->num_kv_heads;
+        const int64_t T = seq_lens[b];
+        const int64_t nb = bsa_oracle_num_blocks(T, P->block_size);
+        const void* kp = orc_pair_rows(P, k_cache, pair);
+        const void* vp = orc_pair_rows(P, v_cache, pair);
+        double* qg = (double*)malloc((size_t)G * d * sizeof(double));
+        orc_group_q(P, q, b, kvh, qg);
+        int32_t* my_idx = idx + (int64_t)i * sel_cap;
+        for (int r = 0; r < sel_cap; ++r) my_idx[r] = -1;
+        int ns;
+        double* bs = block_scores ? block_scores + (int64_t)i * nb_cap : NULL;
+        if (bs)
+            for (int64_t r = 0; r < nb_cap; ++r) bs[r] = -INFINITY;
+        if (boundary) {
+            boundary[2 * i] = NAN;
+            boundary[2 * i + 1] = NAN;
+        }
+        if (given_idx) {
+            ns = given_n_sel[i];
+            if (ns < 0 || ns > sel_cap) {
+                bad |= 1;
+                ns = 0;
+            }
+            for (int r = 0; r < ns; ++r) my_idx[r] = given_idx[(int64_t)i * sel_cap + r];
+        } else {
+            int64_t nc = bsa_oracle_num_windows(T, P->cmp_kernel, P->cmp_stride);
+            double* ck = (double*)malloc((size_t)(nc > 0 ? nc : 1) * d * sizeof(double));
+            double* S = (double*)malloc((size_t)(nc > 0 ? nc : 1) * sizeof(double));
+            double* sb = (double*)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(double));
+            double bnd[2];
+            bsa_oracle_compress(kp, P->dtype, T, d, P->cmp_kernel, P->cmp_stride, P->dtype, ck);
+            bsa_oracle_group_scores(qg, ck, nc, G, d, P->tau, S);
+            bsa_oracle_block_scores(S, nc, nb, P->cmp_kernel, P->cmp_stride, P->block_size, sb);
+            ns = bsa_oracle_select(sb, nb, P->n_init, P->n_local, P->top_k, my_idx, bnd);
+            if (bs)
+                for (int64_t r = 0; r < nb; ++r) bs[r] = sb[r];
+            if (boundary) {
+                boundary[2 * i] = bnd[0];
+                boundary[2 * i + 1] = bnd[1];
+            }
+            free(ck);
+            free(S);
+            free(sb);
+        }
+        n_sel[i] = ns;
+        bsa_oracle_attend(qg, kp, vp, P->dtype, T, d, G, my_idx, ns, P->block_size, P->scale,
+                          out + (int64_t)i * G * d, lse + (int64_t)i * G);
+        free(qg);
+    }
+    return bad ? -1 : 0;
+}
+
+int bsa_oracle_attend_pairs(const orc_problem_t* P, const void* q, const void* k_cache,
+                            const void* v_cache, const int32_t* seq_lens, const int32_t* pairs,
+                            int n_pairs, const int32_t* idx, const int32_t* n_sel, double* out,
+                            double* lse) {
+    if (!orc_problem_ok(P) || n_pairs < 0) return -1;
+    const int sel_cap = P->n_init + P->n_local + P->top_k;
+    /* the decode driver copies the given indices into its idx output; give it scratch for that */
+    int32_t* idx_copy = (int32_t*)malloc((size_t)(n_pairs > 0 ? n_pairs : 1) * sel_cap * sizeof(int32_t) + 4);
+    int32_t* nsel_copy = (int32_t*)malloc((size_t)(n_pairs > 0 ? n_pairs : 1) * sizeof(int32_t));
+    int rc = bsa_oracle_decode(P, q, k_cache, v_cache, seq_lens, pairs, n_pairs, idx, n_sel,
+                               idx_copy, nsel_copy, NULL, NULL, out, lse);
+    free(idx_copy);
+    free(nsel_copy);
+    return rc;
+}
+
+int bsa_oracle_compress_cache(const orc_problem_t* P, const void* k_cache,
+                              const int32_t* seq_lens, const int32_t* pairs, int n_pairs,
+                              double* ck) {
+    if (!orc_problem_ok(P) || n_pairs < 0) return -1;
+    const int d = P->head_dim;
+    const int64_t nc_cap = bsa_oracle_num_windows(P->max_seq_len, P->cmp_kernel, P->cmp_stride);
+    for (int i = 0; i < n_pairs; ++i) {
+        if (pairs[i] < 0 || pairs[i] >= P->batch * P->num_kv_heads) return -1;
+        int64_t T = seq_lens[pairs[i] / P->num_kv_heads];
+        if (T < 0 || T > P->max_seq_len) return -1;
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n_pairs; ++i) {
+        const int pair = pairs[i];
+        const int64_t T = seq_lens[pair / P->num_kv_heads];
+        double* dst = ck + (int64_t)i * nc_cap * d;
+        for (int64_t r = 0; r < nc_cap * d; ++r) dst[r] = 0.0;
+        bsa_oracle_compress(orc_pair_rows(P, k_cache, pair), P->dtype, T, d, P->cmp_kernel,
+                            P->cmp_stride, P->dtype, dst);
+    }
+    return 0;
+}
+
+int bsa_oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
