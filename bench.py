@@ -1,0 +1,561 @@
+"""Decode-step benchmark of the B200 block-sparse compressed-key attention library.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl bsa|reference] [--workload NAME]
+
+One step = one decode step of the workload: group scoring of q against the compressed keys,
+block reduction, top-k + init/local selection and sparse attention over the selected blocks, for
+all sequences of the batch (shared-index workload: selection on layer 0, attention on every layer;
+growing-cache workload: the token append with its compressed-key update first).
+
+Prints one JSON line. ``value`` is decode steps/s over all ranks (weak scaling: every rank runs its
+own copy of the workload on its own GPU, no collective on the data path), device-timed with CUDA
+events between barriers + synchronizes, max over ranks. ``e2e`` is the same metric through the
+Python binding with q copied in from pinned host memory and the output copied back every step.
+``roofline`` is for the kernel with the largest share of the step, from a second, identical pass
+that brackets every kernel with CUDA events. ``cpu_baseline`` (rank 0, one GPU only) and
+``--impl reference`` time the CPU oracle on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import datetime
+import hashlib
+import io
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "block-sparse decode steps/s & achieved HBM GB/s (select+attn) at 128K ctx"
+L2_BYTES = 126 * 1024 * 1024
+NOMINAL_HBM_GBS = 8000.0
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="bsa", choices=["bsa", "reference"])
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--no-graph", action="store_true", help="launch steps directly (no CUDA graph)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------------------------ distributed
+def dist_init(args):
+    import torch
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local) if backend == "nccl" else None)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    """Max of a host float over ranks (timing only; not on the data path)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# -------------------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled every 200 ms while the timed region runs."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.text = ""
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}", "--format=csv",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.text, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.text, _ = self.proc.communicate()
+
+    def summary(self) -> dict:
+        rows = []
+        for row in csv.reader(io.StringIO(self.text or "")):
+            if not row or row[0].strip() == "index":
+                continue
+            rows.append([c.strip() for c in row])
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(s):
+            m = re.match(r"([\d.]+)", s)
+            return float(m.group(1)) if m else None
+
+        sm = [num(r[1]) for r in rows if len(r) > 1 and num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if len(r) > 2 and num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for r in rows:
+            for i, n in enumerate(names):
+                if len(r) > 5 + i and r[5 + i].lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [x for x in sm if mx and x > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": sorted(reasons),
+                "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------------- workload run
+class Bench:
+    def __init__(self, w, device, seed_offset: int, steps_total: int):
+        import torch
+        import block_sparse_attention_compressed_b200 as bsa
+        from block_sparse_attention_compressed_b200.workloads import generate
+        self.torch, self.bsa, self.w, self.dev = torch, bsa, w, device
+        ws_ = w.replace(seed=w.seed + seed_offset)
+        self.append = w.append_steps > 0
+        steps = max(steps_total, w.append_steps) if self.append else 0
+        self.data = generate(ws_, device=device, steps=steps)
+        self.T_cap = self.data["seq_cap"]
+        self.p = bsa.make_params(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, self.T_cap,
+                                 w.dtype, w.n_init, w.n_local, w.top_k, w.cmp_kernel, w.cmp_stride,
+                                 w.block_size, num_layers=w.layers)
+        s = bsa.bsa_get_sizes(self.p)
+        self.sizes = s
+        dt = w.torch_dtype
+        B, Hkv, d = w.batch, w.num_kv_heads, w.head_dim
+        self.ck = torch.zeros(B, Hkv, s.nc_cap, d, dtype=dt, device=device)
+        bsa.bsa_compress_keys(self.p, self.data["k"][0], self.data["seq_lens"], self.ck)
+        self.ws = bsa.alloc_workspace(self.p, device)
+        bsa.bsa_workspace_init(self.p, self.ws)
+        self.block_idx = torch.zeros(B, Hkv, s.sel_cap, dtype=torch.int32, device=device)
+        self.n_sel = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
+        self.out = [torch.zeros(B, w.num_q_heads, d, dtype=dt, device=device)
+                    for _ in range(w.layers)]
+        self.lse = [torch.zeros(B, w.num_q_heads, dtype=torch.float32, device=device)
+                    for _ in range(w.layers)]
+        self.seq0 = self.data["seq_lens"].clone()
+        torch.cuda.synchronize()
+
+    def q_of(self, i):
+        return self.data["q_steps"][i] if self.append else self.data["q"][0]
+
+    # the library calls of one step, on `stream`; `events` (optional) brackets every launch
+    def step(self, i, stream=None, events=None, q=None):
+        bsa, d = self.bsa, self.data
+        q = self.q_of(i) if q is None else q
+        ev = (lambda k: events[k].record(stream)) if events is not None else (lambda k: None)
+        if self.w.layers > 1:
+            ev(0)
+            bsa.bsa_select_blocks(self.p, q, self.ck, d["seq_lens"], self.block_idx, self.n_sel,
+                                  None, self.ws, stream=stream)
+            ev(1)
+            bsa.bsa_sparse_decode_layers(self.p, [q] + [d["q"][L] for L in range(1, self.w.layers)],
+                                         d["k"], d["v"], d["seq_lens"], self.block_idx, self.n_sel,
+                                         self.out, self.lse, self.ws, stream=stream)
+            ev(2)
+            return
+        if events is None:
+            bsa.bsa_decode_step(self.p, q, d["k"][0], d["v"][0], self.ck,
+                                d["k_new"][i] if self.append else None,
+                                d["v_new"][i] if self.append else None, d["seq_lens"],
+                                self.block_idx, self.n_sel, None, self.out[0], self.lse[0], self.ws,
+                                stream=stream)
+            return
+        k = 0
+        if self.append:
+            ev(k); k += 1
+            bsa.bsa_compress_append(self.p, d["k"][0], d["v"][0], d["k_new"][i], d["v_new"][i],
+                                    d["seq_lens"], self.ck, self.ws, stream=stream)
+        ev(k)
+        bsa.bsa_select_blocks(self.p, q, self.ck, d["seq_lens"], self.block_idx, self.n_sel, None,
+                              self.ws, stream=stream)
+        ev(k + 1)
+        bsa.bsa_sparse_decode(self.p, q, d["k"][0], d["v"][0], d["seq_lens"], self.block_idx,
+                              self.n_sel, self.out[0], self.lse[0], self.ws, stream=stream)
+        ev(k + 2)
+
+    def kernel_names(self):
+        names = ["select", "decode"]
+        return (["append"] + names) if (self.append and self.w.layers == 1) else names
+
+    def launches_per_step(self):
+        return len(self.kernel_names())
+
+    def reset_lengths(self):
+        self.data["seq_lens"].copy_(self.seq0)
+
+
+def algorithmic(w, T):
+    from block_sparse_attention_compressed_b200.workloads import algorithmic_bytes
+    return algorithmic_bytes(w, T)
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 6650.0, "fallback"
+
+
+def kernel_source_hash() -> str:
+    import glob
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "block_sparse_attention_compressed_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def profile_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel
+    sources (the summary records the sources' hash)."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m = re.search(r"dram_bytes_per_launch:\s*([\d.eE+]+)", text)
+    hm = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
+    if not m or not hm or hm.group(1) != kernel_source_hash():
+        return None
+    return float(m.group(1))
+
+
+# ------------------------------------------------------------------------------- CPU (oracle) leg
+def cpu_oracle_sample(w, data, seconds: float):
+    """Time the CPU oracle on a bounded sample of (batch, kv-head) pairs of the same workload:
+    selection + attention on the first layer, attention with that selection on the others.
+    Returns (steps/s scaled to the whole batch, threads, description)."""
+    import torch
+    import oracle
+    G, Hkv = w.group, w.num_kv_heads
+    total = w.batch * Hkv
+    T_cap = data["seq_cap"]
+    seq = data["seq_lens"].cpu().tolist()
+    threads = oracle.num_threads()
+    n0 = min(max(threads, 1), total)
+    pairs = [divmod(p, Hkv) for p in range(n0)]
+
+    def layer_arrays(L):
+        q = data["q_steps"][0] if ("q_steps" in data and L == 0) else data["q"][L]
+        qs = torch.stack([q[b, h * G:(h + 1) * G] for b, h in pairs])
+        ks = torch.stack([data["k"][L][b, h:h + 1] for b, h in pairs])
+        vs = torch.stack([data["v"][L][b, h:h + 1] for b, h in pairs])
+        return oracle.raw(qs)[0], oracle.raw(ks)[0], oracle.raw(vs)[0]
+
+    arrays = [layer_arrays(L) for L in range(w.layers)]
+    lens = [seq[b] for b, _ in pairs]
+    P = oracle.make_problem(n0, G, 1, w.head_dim, T_cap,
+                            oracle.F32 if w.dtype == "f32" else oracle.BF16, w.n_init, w.n_local,
+                            w.top_k, w.cmp_kernel, w.cmp_stride, w.block_size)
+
+    def one():
+        r = oracle.decode(P, *arrays[0], lens)
+        for L in range(1, w.layers):
+            oracle.attend_pairs(P, *arrays[L], lens, r["idx"], r["n_sel"])
+
+    t0 = time.perf_counter()
+    one()
+    dt0 = time.perf_counter() - t0
+    reps = max(1, int(seconds / max(dt0, 1e-6)))
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        one()
+    dt = (time.perf_counter() - t0) / reps
+    step_s = dt * (total / n0)
+    desc = (f"CPU oracle (fp64; its selection recomputes each pair's compressed keys) on {n0} of "
+            f"{total} (batch, kv-head) pairs" + (f" x {w.layers} layers" if w.layers > 1 else "")
+            + f", {reps} repetitions, time scaled by {total}/{n0} to a full step")
+    return 1.0 / step_s, threads, desc
+
+
+# -------------------------------------------------------------------------------------------- main
+def run_bsa(args, w, world, rank, local):
+    import torch
+    import block_sparse_attention_compressed_b200 as bsa  # noqa: F401  (fails loudly if unbuilt)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    K, W = args.steps, args.warmup
+    bench = Bench(w, dev, seed_offset=10000 * rank, steps_total=K + W + 1)
+    T_run = w.seq_len
+    ab = algorithmic(w, T_run)
+    stream = torch.cuda.Stream(device=dev)
+    per_step_bytes = ab["total"]
+    flush = per_step_bytes < 4 * L2_BYTES
+    flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if flush else None
+    use_graph = not args.no_graph and not bench.append
+
+    graph = None
+    with torch.cuda.stream(stream):
+        for i in range(W):
+            bench.step(i, stream)
+        if use_graph:
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                bench.step(0, stream)
+            graph.replay()
+    stream.synchronize()
+
+    def run_step(i):
+        if graph is not None:
+            graph.replay()
+        else:
+            bench.step(W + i, stream)
+
+    # ---- pass A: the headline
+    if bench.append:
+        bench.reset_lengths()
+        with torch.cuda.stream(stream):
+            for i in range(W):
+                bench.step(i, stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            if flush:
+                starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+                ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+                for i in range(K):
+                    flush_buf.fill_(i & 0xff)
+                    starts[i].record(stream)
+                    run_step(i)
+                    ends[i].record(stream)
+            else:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                for i in range(K):
+                    run_step(i)
+                e1.record(stream)
+        stream.synchronize()
+        torch.cuda.synchronize()
+    barrier(world)
+    if flush:
+        local_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    else:
+        local_ms = e0.elapsed_time(e1)
+    total_ms = max_over_ranks(local_ms, world)
+    ms_per_step = total_ms / K
+    clocks = clk.summary()
+
+    # ---- pass B: per-kernel breakdown (same work, every launch bracketed by events)
+    names = bench.kernel_names()
+    nk = len(names)
+    if bench.append:
+        bench.reset_lengths()
+        with torch.cuda.stream(stream):
+            for i in range(W):
+                bench.step(i, stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nk + 1)] for _ in range(K)]
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for i in range(K):
+            if flush:
+                flush_buf.fill_(i & 0xff)
+            bench.step(W + i if bench.append else 0, stream, events=evs[i])
+    stream.synchronize()
+    kern_ms = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
+               for j, n in enumerate(names)}
+
+    # ---- e2e: through the binding, q from pinned host memory in, output back out, every step
+    q_host = [bench.q_of(W + i if bench.append else 0).cpu().pin_memory() for i in range(K)]
+    q_dev = torch.empty_like(bench.q_of(0))
+    out_host = torch.empty(bench.out[0].shape, dtype=bench.out[0].dtype).pin_memory()
+    if bench.append:
+        bench.reset_lengths()
+        with torch.cuda.stream(stream):
+            for i in range(W):
+                bench.step(i, stream)
+        kn_host = [bench.data["k_new"][W + i].cpu().pin_memory() for i in range(K)]
+        vn_host = [bench.data["v_new"][W + i].cpu().pin_memory() for i in range(K)]
+        kn_dev, vn_dev = torch.empty_like(bench.data["k_new"][0]), torch.empty_like(bench.data["v_new"][0])
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_e2e0 = time.perf_counter()
+    with torch.cuda.stream(stream):
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for i in range(K):
+            q_dev.copy_(q_host[i], non_blocking=True)
+            if bench.append:
+                kn_dev.copy_(kn_host[i], non_blocking=True)
+                vn_dev.copy_(vn_host[i], non_blocking=True)
+                d = bench.data
+                bsa_ = bench.bsa
+                bsa_.bsa_decode_step(bench.p, q_dev, d["k"][0], d["v"][0], bench.ck, kn_dev,
+                                     vn_dev, d["seq_lens"], bench.block_idx, bench.n_sel, None,
+                                     bench.out[0], bench.lse[0], bench.ws, stream=stream)
+            else:
+                bench.step(0, stream, q=q_dev)
+            out_host.copy_(bench.out[0], non_blocking=True)
+        a1.record(stream)
+    stream.synchronize()
+    e2e_local = a0.elapsed_time(a1)
+    e2e_ms = max_over_ranks(e2e_local, world)
+    wall_e2e = time.perf_counter() - t_e2e0
+    h2d = q_host[0].numel() * q_host[0].element_size()
+    if bench.append:
+        h2d += 2 * kn_host[0].numel() * kn_host[0].element_size()
+    d2h = out_host.numel() * out_host.element_size()
+
+    err = bench.bsa.bsa_read_device_error(bench.ws)
+    if err:
+        raise RuntimeError(f"device error flags set during the benchmark: {err:#x}")
+
+    # ---- roofline of the dominant kernel
+    peak, peak_kind = load_peaks()
+    q_bytes = w.batch * w.num_q_heads * w.head_dim * w.elem_bytes
+    kbytes = {"select": ab["ck"] + q_bytes,          # compressed keys of the scored layer + q
+              "decode": ab["kv"] + ab["qo"],         # selected K/V rows + q + out, every layer
+              "append": ab["append"]}
+    dom = max(kern_ms, key=kern_ms.get)
+    achieved = kbytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
+    traffic = profile_traffic(dom, w.name)
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "peak_kind": peak_kind + " copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "traffic": traffic, "algorithmic_bytes_per_launch": kbytes[dom],
+                "kernel_ms": round(kern_ms[dom], 5)}
+
+    steps_per_s = world * K / (total_ms * 1e-3)
+    gbs = per_step_bytes * world * K / (total_ms * 1e-3) / 1e9
+    result = {
+        "metric": METRIC,
+        "value": round(steps_per_s, 2),
+        "unit": "steps/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": W,
+        "ms_per_step": round(ms_per_step, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) q/K/V with planted needle blocks)",
+        "config": {
+            "workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "q_heads": w.num_q_heads,
+            "kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "n_init": w.n_init,
+            "n_local": w.n_local, "top_k": w.top_k, "block_size": w.block_size,
+            "cmp_kernel": w.cmp_kernel, "cmp_stride": w.cmp_stride, "layers": w.layers,
+            "append": bool(bench.append), "parallelism": f"replicas x{world} (batch-sharded)",
+            "l2": ("L2 flushed (256 MB write) between timed steps" if flush else
+                   f"inputs larger than L2: {per_step_bytes / 1e6:.0f} MB read per step vs 126 MB L2"),
+            "cuda_graph": graph is not None,
+        },
+        "tokens_per_s": round(steps_per_s * w.batch, 1),
+        "hbm_gbs": round(gbs / world, 1),
+        "frac_of_8tbs": round(gbs / world / NOMINAL_HBM_GBS, 4),
+        "algorithmic_bytes_per_step": per_step_bytes,
+        "kernels_ms": {k: round(v, 5) for k, v in kern_ms.items()},
+        "roofline": roofline,
+        "e2e": {"value": round(world * K / (e2e_ms * 1e-3), 2), "unit": "steps/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "wall_s": round(wall_e2e, 4), "l2_flush": False},
+        "gpu_launches": K * bench.launches_per_step(),
+        "clocks": clocks,
+        "kernel_sources_sha256_16": kernel_source_hash(),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, cores, desc = cpu_oracle_sample(w, bench.data, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": round(v, 4), "unit": "steps/s", "cores": cores,
+                                  "kind": "oracle", "sample": desc}
+    return result
+
+
+def run_reference(args, w, world, rank):
+    """The reference arm: the CPU oracle, as it stands, on the host cores."""
+    import torch
+    from block_sparse_attention_compressed_b200.workloads import generate
+    if rank != 0:
+        return None
+    per_step = max(1.0, args.cpu_seconds / max(args.steps + args.warmup, 1))
+    w_small = w
+    data = generate(w_small, device="cuda" if torch.cuda.is_available() else "cpu",
+                    steps=1 if w.append_steps else 0)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, data, per_step / 4)
+    vals = []
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        v, cores, desc = cpu_oracle_sample(w, data, per_step)
+        vals.append(v)
+    wall = time.perf_counter() - t0
+    value = statistics.median(vals)
+    return {
+        "metric": METRIC, "value": round(value, 4), "unit": "steps/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 / value, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic (seeded N(0,1) q/K/V with planted needle blocks)",
+        "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len},
+        "impl": "reference",
+        "cpu_baseline": {"value": round(value, 4), "unit": "steps/s", "cores": cores,
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 4), "unit": "steps/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "wall_s": round(wall, 2),
+    }
+
+
+def main():
+    args = parse()
+    from block_sparse_attention_compressed_b200.workloads import DEFAULT_WORKLOAD, WORKLOADS
+    w = WORKLOADS[args.workload or DEFAULT_WORKLOAD]
+    world, rank, local = dist_init(args)
+    if args.impl == "reference":
+        res = run_reference(args, w, world, rank)
+    else:
+        res = run_bsa(args, w, world, rank, local)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,404 @@
+// Host side of libbsa: parameter validation, launch planning, workspace layout and the C ABI
+// declared in include/bsa.h. Nothing here allocates device memory or synchronizes (except
+// bsa_read_device_error, which is documented to).
+#include <math.h>
+#include <string.h>
+
+#include "bsa_internal.cuh"
+
+namespace bsa {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kNumSMs = 148;  // B200; only used to size work splits, never for correctness
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int64_t num_windows(int64_t T, int l, int s) { return T < l ? 0 : (T - l) / s + 1; }
+
+bool is_aligned(const void* p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
+    if (!prm || !p) return BSA_ERR_INVALID_ARG;
+    const bsa_params_t& q = *prm;
+    if (q.batch < 1 || q.num_q_heads < 1 || q.num_kv_heads < 1) return BSA_ERR_INVALID_ARG;
+    if (q.num_q_heads % q.num_kv_heads != 0) return BSA_ERR_INVALID_ARG;
+    if (q.cmp_kernel < 1 || q.cmp_stride < 1 || q.block_size < 1) return BSA_ERR_INVALID_ARG;
+    if (q.n_init < 0 || q.n_local < 0 || q.top_k < 0) return BSA_ERR_INVALID_ARG;
+    if (q.max_seq_len < 1 || q.max_seq_len > ((int64_t)1 << 31) - 1) return BSA_ERR_INVALID_ARG;
+    if (q.num_layers < 1) return BSA_ERR_INVALID_ARG;
+    if (!(q.scale >= 0.f) || isinf(q.scale) || !(q.score_tau >= 0.f) || isinf(q.score_tau))
+        return BSA_ERR_INVALID_ARG;
+    if (q.dtype != BSA_F32 && q.dtype != BSA_BF16) return BSA_ERR_UNSUPPORTED;
+    if (q.head_dim != 64 && q.head_dim != 128) return BSA_ERR_UNSUPPORTED;
+    const int G = q.num_q_heads / q.num_kv_heads;
+    if (G > kMaxG) return BSA_ERR_UNSUPPORTED;
+    if (q.block_size % 16 != 0 || q.block_size > 256) return BSA_ERR_UNSUPPORTED;
+    if (q.num_layers > BSA_MAX_LAYERS) return BSA_ERR_UNSUPPORTED;
+    const int64_t sel = (int64_t)q.n_init + q.n_local + q.top_k;
+    if (sel < 1 || sel > 65536) return BSA_ERR_INVALID_ARG;
+    const int64_t pairs = (int64_t)q.batch * q.num_kv_heads;
+    if (pairs > (1 << 24)) return BSA_ERR_UNSUPPORTED;
+
+    Plan& P = *p;
+    memset(&P, 0, sizeof P);
+    P.B = q.batch;
+    P.Hq = q.num_q_heads;
+    P.Hkv = q.num_kv_heads;
+    P.G = G;
+    P.Gp = 1;
+    while (P.Gp < G) P.Gp <<= 1;
+    P.D = q.head_dim;
+    P.l = q.cmp_kernel;
+    P.s = q.cmp_stride;
+    P.BS = q.block_size;
+    P.n_init = q.n_init;
+    P.n_local = q.n_local;
+    P.top_k = q.top_k;
+    P.sel_cap = (int)sel;
+    P.layers = q.num_layers;
+    P.dtype = q.dtype;
+    P.T_cap = q.max_seq_len;
+    P.nc_cap = num_windows(P.T_cap, P.l, P.s);
+    P.nb_cap = (P.T_cap + P.BS - 1) / P.BS;
+    if (P.nb_cap > kMaxNbCap) return BSA_ERR_UNSUPPORTED;
+    P.pairs = (int)pairs;
+    const double log2e = 1.4426950408889634;
+    const double scale = q.scale > 0.f ? (double)q.scale : 1.0 / sqrt((double)P.D);
+    const double tau = q.score_tau > 0.f ? (double)q.score_tau : sqrt((double)P.D);
+    P.scale_log2 = (float)(scale * log2e);
+    P.score_log2 = (float)(log2e / tau);
+
+    // Scoring split: enough CTAs to cover the GPU twice when the problem allows it, with slices
+    // that are whole 16-row tiles per warp.
+    {
+        const int64_t nc = P.nc_cap > 0 ? P.nc_cap : 1;
+        int64_t items = (nc + 1023) / 1024;
+        const int64_t want = (2 * kNumSMs + P.pairs - 1) / P.pairs;
+        const int64_t most = (nc + 16 * kScoreWarps - 1) / (16 * kScoreWarps);
+        if (items < want) items = want < most ? want : most;
+        if (items < 1) items = 1;
+        const int64_t rows_item = (nc + items - 1) / items;
+        int64_t rpw = (rows_item + kScoreWarps - 1) / kScoreWarps;
+        rpw = (rpw + 15) / 16 * 16;
+        P.score_rows_per_warp = (int)rpw;
+        P.score_items = (int)((nc + rpw * kScoreWarps - 1) / (rpw * kScoreWarps));
+        if ((int64_t)P.pairs * P.score_items > 0x7fffffff) return BSA_ERR_UNSUPPORTED;
+        P.score_smem = (size_t)P.nb_cap * sizeof(uint32_t);
+    }
+    // Decode split: about eight blocks per SM slot in flight, whole blocks per CTA.
+    {
+        const int64_t total = (int64_t)P.layers * P.pairs * P.sel_cap;
+        int64_t bpc = total / (kNumSMs * 8);
+        if (bpc < 1) bpc = 1;
+        if (bpc > 16) bpc = 16;
+        if (bpc > P.sel_cap) bpc = P.sel_cap;
+        const int64_t splits = (P.sel_cap + bpc - 1) / bpc;
+        P.dec_splits = (int)splits;
+        P.dec_bpc = (int)((P.sel_cap + splits - 1) / splits);
+    }
+    // Workspace
+    size_t off = 0;
+    P.off_err = off;
+    off = align_up(off + sizeof(uint32_t));
+    P.off_score_cnt = off;
+    off = align_up(off + (size_t)P.pairs * sizeof(int));
+    P.off_dec_cnt = off;
+    off = align_up(off + (size_t)P.layers * P.pairs * sizeof(int));
+    P.off_logits = off;
+    off = align_up(off + (size_t)P.pairs * P.nc_cap * P.Gp * sizeof(float));
+    P.off_stats = off;
+    off = align_up(off + (size_t)P.pairs * P.score_items * P.Gp * sizeof(float2));
+    P.off_part_ml = off;
+    off = align_up(off + (size_t)P.layers * P.pairs * P.dec_splits * P.Gp * sizeof(float2));
+    P.off_part_acc = off;
+    off = align_up(off + (size_t)P.layers * P.pairs * P.dec_splits * P.Gp * P.D * sizeof(float));
+    P.ws_bytes = off;
+    return BSA_OK;
+}
+
+template <typename T>
+T* ws_at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+bsa_status_t check_ws(const Plan& P, void* ws, size_t bytes) {
+    if (!ws || bytes < P.ws_bytes || !is_aligned(ws, kAlign)) return BSA_ERR_WORKSPACE;
+    return BSA_OK;
+}
+
+bsa_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? BSA_OK : BSA_ERR_CUDA; }
+
+bool ok16(const void* p) { return p && is_aligned(p, 16); }
+bool ok4(const void* p) { return p && is_aligned(p, 4); }
+
+ScoreArgs score_args(const Plan& P, const void* q, const void* ck, const int32_t* seq_lens,
+                     int32_t* block_idx, int32_t* n_sel, float* block_scores, void* ws) {
+    ScoreArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = q;
+    a.ck = ck;
+    a.seq_lens = seq_lens;
+    a.block_idx = block_idx;
+    a.n_sel = n_sel;
+    a.block_scores = block_scores;
+    a.err = ws_at<uint32_t>(ws, P.off_err);
+    a.cnt = ws_at<int>(ws, P.off_score_cnt);
+    a.logits = ws_at<float>(ws, P.off_logits);
+    a.stats = ws_at<float2>(ws, P.off_stats);
+    a.Hq = P.Hq;
+    a.Hkv = P.Hkv;
+    a.G = P.G;
+    a.Gp = P.Gp;
+    a.l = P.l;
+    a.s = P.s;
+    a.BS = P.BS;
+    a.n_init = P.n_init;
+    a.n_local = P.n_local;
+    a.top_k = P.top_k;
+    a.sel_cap = P.sel_cap;
+    a.T_cap = P.T_cap;
+    a.nc_cap = P.nc_cap;
+    a.nb_cap = P.nb_cap;
+    a.items = P.score_items;
+    a.rows_per_warp = P.score_rows_per_warp;
+    a.score_log2 = P.score_log2;
+    return a;
+}
+
+DecodeArgs decode_args(const Plan& P, const int32_t* seq_lens, const int32_t* block_idx,
+                       const int32_t* n_sel, void* ws) {
+    DecodeArgs a;
+    memset(&a, 0, sizeof a);
+    a.seq_lens = seq_lens;
+    a.block_idx = block_idx;
+    a.n_sel = n_sel;
+    a.err = ws_at<uint32_t>(ws, P.off_err);
+    a.cnt = ws_at<int>(ws, P.off_dec_cnt);
+    a.part_ml = ws_at<float2>(ws, P.off_part_ml);
+    a.part_acc = ws_at<float>(ws, P.off_part_acc);
+    a.Hq = P.Hq;
+    a.Hkv = P.Hkv;
+    a.G = P.G;
+    a.Gp = P.Gp;
+    a.BS = P.BS;
+    a.sel_cap = P.sel_cap;
+    a.pairs = P.pairs;
+    a.T_cap = P.T_cap;
+    a.splits = P.dec_splits;
+    a.bpc = P.dec_bpc;
+    a.scale_log2 = P.scale_log2;
+    return a;
+}
+
+bsa_status_t do_append(const Plan& P, void* k_cache, void* v_cache, const void* k_new,
+                       const void* v_new, int32_t* seq_lens, void* ck, void* ws, cudaStream_t st) {
+    AppendArgs a;
+    memset(&a, 0, sizeof a);
+    a.k = k_cache;
+    a.v = v_cache;
+    a.k_new = k_new;
+    a.v_new = v_new;
+    a.seq_lens = seq_lens;
+    a.ck = ck;
+    a.err = ws ? ws_at<uint32_t>(ws, P.off_err) : nullptr;
+    a.Hkv = P.Hkv;
+    a.D = P.D;
+    a.l = P.l;
+    a.s = P.s;
+    a.T_cap = P.T_cap;
+    a.nc_cap = P.nc_cap;
+    return from_cuda(launch_append(P, a, st));
+}
+
+}  // namespace
+}  // namespace bsa
+
+using namespace bsa;
+
+extern "C" {
+
+const char* bsa_status_string(bsa_status_t s) {
+    switch (s) {
+        case BSA_OK: return "BSA_OK";
+        case BSA_ERR_INVALID_ARG: return "BSA_ERR_INVALID_ARG";
+        case BSA_ERR_UNSUPPORTED: return "BSA_ERR_UNSUPPORTED";
+        case BSA_ERR_WORKSPACE: return "BSA_ERR_WORKSPACE";
+        case BSA_ERR_CUDA: return "BSA_ERR_CUDA";
+        case BSA_ERR_DEVICE_CHECK: return "BSA_ERR_DEVICE_CHECK";
+    }
+    return "BSA_ERR_UNKNOWN";
+}
+
+int32_t bsa_abi_version(void) { return BSA_ABI_VERSION; }
+
+bsa_status_t bsa_check_params(const bsa_params_t* params) {
+    Plan P;
+    return make_plan(params, &P);
+}
+
+bsa_status_t bsa_get_sizes(const bsa_params_t* params, bsa_sizes_t* sizes) {
+    if (!sizes) return BSA_ERR_INVALID_ARG;
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    sizes->nc_cap = P.nc_cap;
+    sizes->nb_cap = P.nb_cap;
+    sizes->sel_cap = P.sel_cap;
+    sizes->group = P.G;
+    sizes->workspace_bytes = P.ws_bytes;
+    return BSA_OK;
+}
+
+size_t bsa_workspace_size(const bsa_params_t* params) {
+    Plan P;
+    return make_plan(params, &P) == BSA_OK ? P.ws_bytes : 0;
+}
+
+bsa_status_t bsa_workspace_init(const bsa_params_t* params, void* ws, size_t ws_bytes,
+                                cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if ((st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
+    // error word and both counter arrays are contiguous at the front
+    return from_cuda(cudaMemsetAsync(ws, 0, P.off_logits, stream));
+}
+
+bsa_status_t bsa_compress_keys(const bsa_params_t* params, const void* k_cache,
+                               const int32_t* seq_lens, void* ck, cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if (!ok16(k_cache) || !ok4(seq_lens) || !ok16(ck)) return BSA_ERR_INVALID_ARG;
+    CompressArgs a;
+    memset(&a, 0, sizeof a);
+    a.k = k_cache;
+    a.ck = ck;
+    a.seq_lens = seq_lens;
+    a.err = nullptr;
+    a.Hkv = P.Hkv;
+    a.D = P.D;
+    a.l = P.l;
+    a.s = P.s;
+    a.T_cap = P.T_cap;
+    a.nc_cap = P.nc_cap;
+    if (P.nc_cap == 0) return BSA_OK;
+    return from_cuda(launch_compress_keys(P, a, stream));
+}
+
+bsa_status_t bsa_compress_append(const bsa_params_t* params, void* k_cache, void* v_cache,
+                                 const void* k_new, const void* v_new, int32_t* seq_lens, void* ck,
+                                 void* ws, size_t ws_bytes, cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if (!ok16(k_cache) || !ok16(v_cache) || !ok16(k_new) || !ok16(v_new) || !ok4(seq_lens))
+        return BSA_ERR_INVALID_ARG;
+    if (P.nc_cap > 0 && !ok16(ck)) return BSA_ERR_INVALID_ARG;
+    if (ws && (st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
+    return do_append(P, k_cache, v_cache, k_new, v_new, seq_lens, ck, ws, stream);
+}
+
+bsa_status_t bsa_select_blocks(const bsa_params_t* params, const void* q, const void* ck,
+                               const int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                               float* block_scores, void* ws, size_t ws_bytes,
+                               cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if (!ok16(q) || !ok4(seq_lens) || !ok4(block_idx) || !ok4(n_sel)) return BSA_ERR_INVALID_ARG;
+    if (P.nc_cap > 0 && !ok16(ck)) return BSA_ERR_INVALID_ARG;
+    if (block_scores && !ok4(block_scores)) return BSA_ERR_INVALID_ARG;
+    if ((st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
+    ScoreArgs a = score_args(P, q, ck, seq_lens, block_idx, n_sel, block_scores, ws);
+    return from_cuda(launch_score_select(P, a, stream));
+}
+
+bsa_status_t bsa_sparse_decode_layers(const bsa_params_t* params, int32_t num_layers,
+                                      const void* const* q, const void* const* k_caches,
+                                      const void* const* v_caches, const int32_t* seq_lens,
+                                      const int32_t* block_idx, const int32_t* n_sel,
+                                      void* const* outs, float* const* lses, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if (num_layers < 1 || num_layers > P.layers) return BSA_ERR_INVALID_ARG;
+    if (!q || !k_caches || !v_caches || !outs) return BSA_ERR_INVALID_ARG;
+    if (!ok4(seq_lens) || !ok4(block_idx) || !ok4(n_sel)) return BSA_ERR_INVALID_ARG;
+    if ((st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
+    DecodeArgs a = decode_args(P, seq_lens, block_idx, n_sel, ws);
+    for (int i = 0; i < num_layers; ++i) {
+        if (!ok16(q[i]) || !ok16(k_caches[i]) || !ok16(v_caches[i]) || !ok16(outs[i]))
+            return BSA_ERR_INVALID_ARG;
+        float* lse = lses ? lses[i] : nullptr;
+        if (lse && !ok4(lse)) return BSA_ERR_INVALID_ARG;
+        a.q[i] = q[i];
+        a.k[i] = k_caches[i];
+        a.v[i] = v_caches[i];
+        a.out[i] = outs[i];
+        a.lse[i] = lse;
+    }
+    return from_cuda(launch_decode(P, a, num_layers, stream));
+}
+
+bsa_status_t bsa_sparse_decode(const bsa_params_t* params, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* seq_lens,
+                               const int32_t* block_idx, const int32_t* n_sel, void* out,
+                               float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    const void* qs[1] = {q};
+    const void* ks[1] = {k_cache};
+    const void* vs[1] = {v_cache};
+    void* os[1] = {out};
+    float* ls[1] = {lse};
+    return bsa_sparse_decode_layers(params, 1, qs, ks, vs, seq_lens, block_idx, n_sel, os, ls, ws,
+                                    ws_bytes, stream);
+}
+
+bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_cache,
+                             void* v_cache, void* ck, const void* k_new, const void* v_new,
+                             int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                             float* block_scores, void* out, float* lse, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    const bool append = k_new != nullptr && v_new != nullptr;
+    if ((k_new == nullptr) != (v_new == nullptr)) return BSA_ERR_INVALID_ARG;
+    if (!ok16(q) || !ok16(k_cache) || !ok16(v_cache) || !ok16(out) || !ok4(seq_lens) ||
+        !ok4(block_idx) || !ok4(n_sel))
+        return BSA_ERR_INVALID_ARG;
+    if (P.nc_cap > 0 && !ok16(ck)) return BSA_ERR_INVALID_ARG;
+    if (append && (!ok16(k_new) || !ok16(v_new))) return BSA_ERR_INVALID_ARG;
+    if ((block_scores && !ok4(block_scores)) || (lse && !ok4(lse))) return BSA_ERR_INVALID_ARG;
+    if ((st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
+    if (append) {
+        st = do_append(P, k_cache, v_cache, k_new, v_new, seq_lens, ck, ws, stream);
+        if (st != BSA_OK) return st;
+    }
+    ScoreArgs sa = score_args(P, q, ck, seq_lens, block_idx, n_sel, block_scores, ws);
+    if ((st = from_cuda(launch_score_select(P, sa, stream))) != BSA_OK) return st;
+    DecodeArgs da = decode_args(P, seq_lens, block_idx, n_sel, ws);
+    da.q[0] = q;
+    da.k[0] = k_cache;
+    da.v[0] = v_cache;
+    da.out[0] = out;
+    da.lse[0] = lse;
+    return from_cuda(launch_decode(P, da, 1, stream));
+}
+
+bsa_status_t bsa_read_device_error(void* ws, size_t ws_bytes, uint32_t* flags,
+                                   cudaStream_t stream) {
+    if (!flags) return BSA_ERR_INVALID_ARG;
+    if (!ws || ws_bytes < sizeof(uint32_t) || !is_aligned(ws, kAlign)) return BSA_ERR_WORKSPACE;
+    uint32_t v = 0;
+    if (cudaMemcpyAsync(&v, ws, sizeof v, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    if (cudaMemsetAsync(ws, 0, sizeof v, stream) != cudaSuccess) return BSA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return BSA_ERR_CUDA;
+    *flags = v;
+    return v ? BSA_ERR_DEVICE_CHECK : BSA_OK;
+}
+
+}  // extern "C"

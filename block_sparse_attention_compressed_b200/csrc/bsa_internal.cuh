@@ -1,0 +1,209 @@
+// Internal declarations of libbsa: launch plan, workspace layout, kernel argument blocks and
+// small PTX helpers for sm_100a. Nothing here is part of the C ABI (include/bsa.h is).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <utility>
+
+#include "bsa.h"
+
+namespace bsa {
+
+constexpr int kMaxG = 8;         // query heads per kv head handled by one mma tile (N = 8)
+constexpr int kScoreWarps = 8;   // warps per scoring CTA
+constexpr int kDecodeWarps = 4;  // warps per decode CTA
+constexpr int kMaxNbCap = 32768; // selection blocks per sequence (shared-memory key array)
+
+// ------------------------------------------------------------------------------------------------
+// Launch plan: every size and workspace offset derived from bsa_params_t. The same function feeds
+// bsa_workspace_size and the launches, so the two always agree.
+struct Plan {
+    int B, Hq, Hkv, G, Gp, D, l, s, BS, n_init, n_local, top_k, sel_cap, layers, dtype;
+    int64_t T_cap, nc_cap, nb_cap;
+    int pairs;
+    float scale_log2;  // attention scale * log2(e): softmax evaluated with exp2
+    float score_log2;  // (1 / tau) * log2(e)
+    // scoring: grid = pairs * score_items CTAs of kScoreWarps warps, score_rows_per_warp rows each
+    int score_items, score_rows_per_warp;
+    size_t score_smem;  // dynamic shared memory of the selection phase (block keys)
+    // decode: grid = layers * pairs * dec_splits CTAs of kDecodeWarps warps, dec_bpc blocks each
+    int dec_splits, dec_bpc;
+    // workspace layout (bytes)
+    size_t off_err, off_score_cnt, off_dec_cnt, off_logits, off_stats, off_part_ml, off_part_acc;
+    size_t ws_bytes;
+};
+
+// ------------------------------------------------------------------------------------------------
+struct CompressArgs {
+    const void* k;
+    void* ck;
+    const int32_t* seq_lens;
+    uint32_t* err;  // may be null
+    int Hkv, D, l, s, windows_per_cta;
+    int64_t T_cap, nc_cap;
+};
+
+struct AppendArgs {
+    void* k;
+    void* v;
+    const void* k_new;
+    const void* v_new;
+    int32_t* seq_lens;
+    void* ck;
+    uint32_t* err;  // may be null
+    int Hkv, D, l, s;
+    int64_t T_cap, nc_cap;
+};
+
+struct ScoreArgs {
+    const void* q;
+    const void* ck;
+    const int32_t* seq_lens;
+    int32_t* block_idx;
+    int32_t* n_sel;
+    float* block_scores;  // may be null
+    uint32_t* err;
+    int* cnt;             // [pairs] completion counters
+    float* logits;        // [pairs][nc_cap][Gp], log2 units
+    float2* stats;        // [pairs][items][Gp] (max, sum of exp2(x - max)) per item and head
+    int Hq, Hkv, G, Gp, l, s, BS, n_init, n_local, top_k, sel_cap;
+    int64_t T_cap, nc_cap, nb_cap;
+    int items, rows_per_warp;
+    float score_log2;
+};
+
+struct DecodeArgs {
+    const void* q[BSA_MAX_LAYERS];
+    const void* k[BSA_MAX_LAYERS];
+    const void* v[BSA_MAX_LAYERS];
+    void* out[BSA_MAX_LAYERS];
+    float* lse[BSA_MAX_LAYERS];
+    const int32_t* seq_lens;
+    const int32_t* block_idx;
+    const int32_t* n_sel;
+    uint32_t* err;
+    int* cnt;           // [layers * pairs]
+    float2* part_ml;    // [layers * pairs][splits][Gp] (max, denominator) in log2 units
+    float* part_acc;    // [layers * pairs][splits][Gp][D] unnormalised numerators
+    int Hq, Hkv, G, Gp, BS, sel_cap, pairs;
+    int64_t T_cap;
+    int splits, bpc;
+    float scale_log2;
+};
+
+// Launchers (one per kernel family); they pick the template instance from the plan's dtype/D.
+cudaError_t launch_compress_keys(const Plan& p, const CompressArgs& a, cudaStream_t st);
+cudaError_t launch_append(const Plan& p, const AppendArgs& a, cudaStream_t st);
+cudaError_t launch_score_select(const Plan& p, const ScoreArgs& a, cudaStream_t st);
+cudaError_t launch_decode(const Plan& p, const DecodeArgs& a, int layers, cudaStream_t st);
+
+// Launch with programmatic dependent launch allowed: the kernel may start while the previous
+// kernel in the stream drains; every kernel here waits (griddepcontrol.wait) before touching
+// memory that an earlier kernel writes.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t st, Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Device helpers
+#ifdef __CUDACC__
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// 128-bit streaming load: read-only for the kernel's lifetime, no L1 allocation, 256-byte L2
+// prefetch granule (rows of the caches are 256 bytes at d = 128 bf16).
+__device__ __forceinline__ uint4 ld_stream(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// Loads that bypass L1 (data written by other CTAs of the same grid).
+__device__ __forceinline__ float ld_cg(const float* p) { return __ldcg(p); }
+__device__ __forceinline__ float2 ld_cg(const float2* p) { return __ldcg(p); }
+__device__ __forceinline__ float4 ld_cg(const float4* p) { return __ldcg(p); }
+__device__ __forceinline__ int ld_cg(const int* p) { return __ldcg(p); }
+
+__device__ __forceinline__ uint32_t u4_get(const uint4& v, int i) {
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// D[16x8] += A[16x16] * B[16x8], bf16 inputs, fp32 accumulate (warp-wide).
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+        "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Transpose an 8x8 matrix of 16-bit elements held one 32-bit register per lane.
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
+
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t d;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+    return d;
+}
+
+// Two floats -> packed bf16x2 (lo in the low half), round to nearest even.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
+
+// Running (max, sum exp2(x - max)) of a stream of log2-domain values.
+__device__ __forceinline__ void online_add(float& m, float& s, float x) {
+    float mn = fmaxf(m, x);
+    s = s * exp2f(m - mn) + exp2f(x - mn);
+    m = mn;
+}
+__device__ __forceinline__ void online_merge(float& m, float& s, float m2, float s2) {
+    float mn = fmaxf(m, m2);
+    if (mn == -INFINITY) {
+        m = mn;
+        s = 0.f;
+        return;
+    }
+    s = s * exp2f(m - mn) + s2 * exp2f(m2 - mn);
+    m = mn;
+}
+
+// Order-preserving map of an fp32 score onto uint32 (larger float -> larger key).
+__device__ __forceinline__ uint32_t order_key(float f) {
+    uint32_t u = __float_as_uint(f);
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+#endif  // __CUDACC__
+
+}  // namespace bsa

@@ -1,0 +1,200 @@
+/*
+ * bsa.h -- C ABI of the B200 block-sparse compressed-key decode attention library (libbsa.so).
+ *
+ * The method (InfLLM-V2 style block-sparse decode, as summarised on the page
+ * "SparDA: Sparse Decoupled Attention for Efficient Long-Context LLM Inference"):
+ *   1. compressed keys: K~_j = mean of K over rows [s*j, s*j + l), l = 32, s = 16
+ *      (Theoretical Foundation, Eq. 2);
+ *   2. group scoring: per GQA group, S[j] = sum over the group's query heads of
+ *      softmax_j(q_h . K~_j / tau) (Indexer Training, Eq. 6, the original selector's distribution);
+ *   3. block reduction: the score of a 64-token block is the maximum of S over the complete windows
+ *      that overlap it (Indexer Training, "Fine-grained supervision": max-pooled to the block grid);
+ *   4. selection: top-k blocks by that score, ties to the lower block index, united with the first
+ *      n_init and last n_local blocks (Theoretical Foundation, Eq. 1; SparDA Architecture, Eq. 4);
+ *   5. attention: exact softmax attention of every query head over the tokens of its group's
+ *      selected blocks (SparDA Architecture, Eq. 5).
+ * A shared-index mode reuses one layer's selection for several layers (page "HySparse2: Hybrid
+ * Sparse Attention with Two-Level KV Sharing", first abstract; page "CoSA: Accelerating
+ * Long-Context Inference via Proxy-Kernel Co-Designed Sparse Attention", second abstract).
+ *
+ * Conventions for every entry point:
+ *   - All tensors are dense, row-major, on the current CUDA device, owned by the caller. The
+ *     library allocates no memory and keeps no state between calls except inside the caller's
+ *     workspace. Pointers must be 16-byte aligned.
+ *   - Every call is asynchronous on `stream` (cudaStream_t; 0 = legacy default stream) and does
+ *     not synchronize, except bsa_read_device_error.
+ *   - Arguments are validated on the host before anything is launched; a rejected call returns a
+ *     status other than BSA_OK, launches nothing and leaves all buffers untouched.
+ *   - Conditions that only the device can see (a sequence length above the capacity, a block
+ *     index out of range) set a bit in the workspace's error word (bsa_device_error_t), skip the
+ *     affected (batch, kv-head) pair and never trap; read it with bsa_read_device_error.
+ *   - Kernels that use the workspace need it zero-filled once before first use
+ *     (bsa_workspace_init); they leave it ready for the next call. Calls that share a workspace
+ *     must not overlap on the GPU (same stream, or ordered by events).
+ *
+ * Tensor layouts (B = batch, Hq / Hkv = query / kv heads, G = Hq / Hkv, d = head_dim,
+ * T_cap = max_seq_len, NC_cap = number of windows in T_cap rows, NB_cap = ceil(T_cap / BS),
+ * SEL_cap = n_init + n_local + top_k; "elem" is fp32 or bf16 per bsa_params_t.dtype):
+ *   q            [B][Hq][d]          elem   query head h belongs to kv head h / G
+ *   k_cache      [B][Hkv][T_cap][d]  elem   rows >= seq_lens[b] are never read for attention
+ *   v_cache      [B][Hkv][T_cap][d]  elem
+ *   ck           [B][Hkv][NC_cap][d] elem   compressed keys (rounded to nearest even from fp64)
+ *   seq_lens     [B]                 int32  tokens in each sequence (incl. the current one)
+ *   block_idx    [B][Hkv][SEL_cap]   int32  selected blocks, ascending, then -1 padding
+ *   n_sel        [B][Hkv]            int32  number of valid entries in block_idx
+ *   block_scores [B][Hkv][NB_cap]    fp32   max-pooled group score per block, -inf where no
+ *                                           complete window overlaps the block and past the end
+ *   out          [B][Hq][d]          elem   attention output
+ *   lse          [B][Hq]             fp32   natural log of each head's softmax denominator
+ */
+#ifndef BSA_H
+#define BSA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define BSA_ABI_VERSION 1
+#define BSA_MAX_LAYERS 16
+
+typedef enum {
+    BSA_OK = 0,
+    BSA_ERR_INVALID_ARG = 1, /* a null/misaligned pointer, bad shape or inconsistent parameter */
+    BSA_ERR_UNSUPPORTED = 2, /* valid but not implemented (head_dim, group size, dtype, sizes) */
+    BSA_ERR_WORKSPACE = 3,   /* workspace missing or smaller than bsa_workspace_size() */
+    BSA_ERR_CUDA = 4,        /* a CUDA runtime call failed (launch or memset) */
+    BSA_ERR_DEVICE_CHECK = 5 /* bsa_read_device_error found a device-side error bit set */
+} bsa_status_t;
+
+typedef enum { BSA_F32 = 0, BSA_BF16 = 1 } bsa_dtype_t;
+
+/* Bits of the device error word (bsa_read_device_error). */
+typedef enum {
+    BSA_DEVERR_SEQ_LEN = 1u << 0,   /* seq_lens[b] < 0 or > max_seq_len: pair skipped */
+    BSA_DEVERR_CAPACITY = 1u << 1,  /* bsa_compress_append with seq_lens[b] == max_seq_len */
+    BSA_DEVERR_BLOCK_IDX = 1u << 2, /* block index outside [0, ceil(T/BS)): entry skipped */
+    BSA_DEVERR_N_SEL = 1u << 3      /* n_sel outside [0, SEL_cap]: clamped */
+} bsa_device_error_t;
+
+/* Problem shape and method parameters. Supported: dtype fp32 or bf16; head_dim 64 or 128;
+ * G = Hq / Hkv in 1..8; block_size a multiple of 16 in 16..256; cmp_kernel, cmp_stride >= 1;
+ * n_init + n_local + top_k >= 1; NB_cap <= 32768; num_layers in 1..BSA_MAX_LAYERS. */
+typedef struct {
+    int32_t batch;        /* B */
+    int32_t num_q_heads;  /* Hq */
+    int32_t num_kv_heads; /* Hkv */
+    int32_t head_dim;     /* d */
+    int32_t cmp_kernel;   /* l, compression window length (32 in Eq. 2) */
+    int32_t cmp_stride;   /* s, compression window stride (16 in Eq. 2) */
+    int32_t block_size;   /* BS, tokens per selection block (64) */
+    int32_t n_init;       /* first blocks always selected */
+    int32_t n_local;      /* last blocks always selected (sliding window) */
+    int32_t top_k;        /* blocks chosen by score among the others */
+    int64_t max_seq_len;  /* T_cap, rows allocated per (batch, kv head) in the caches */
+    int32_t num_layers;   /* layers attended with one selection (shared-index mode); sizes ws */
+    int32_t dtype;        /* bsa_dtype_t of q, caches, ck and out */
+    float scale;          /* attention scale of Eq. 5; 0 selects 1/sqrt(head_dim) */
+    float score_tau;      /* tau of Eq. 6; 0 selects sqrt(head_dim) */
+} bsa_params_t;
+
+/* Derived sizes of a parameter set. */
+typedef struct {
+    int64_t nc_cap;          /* NC_cap: windows in max_seq_len rows */
+    int64_t nb_cap;          /* NB_cap: blocks in max_seq_len rows */
+    int32_t sel_cap;         /* SEL_cap: n_init + n_local + top_k */
+    int32_t group;           /* G */
+    size_t workspace_bytes;  /* what bsa_workspace_size returns */
+} bsa_sizes_t;
+
+/* Human-readable name of a status. Never NULL. */
+const char* bsa_status_string(bsa_status_t status);
+
+/* Library ABI version (BSA_ABI_VERSION at build time). */
+int32_t bsa_abi_version(void);
+
+/* Validate a parameter set (host only; no CUDA call). */
+bsa_status_t bsa_check_params(const bsa_params_t* params);
+
+/* Fill *sizes for a valid parameter set (host only). */
+bsa_status_t bsa_get_sizes(const bsa_params_t* params, bsa_sizes_t* sizes);
+
+/* Bytes of device workspace that bsa_select_blocks, bsa_sparse_decode(_layers) and
+ * bsa_decode_step need for these parameters; 0 for invalid parameters. Holds the error word,
+ * per-pair completion counters, fp32 window logits [B*Hkv][NC_cap][G] and attention partials. */
+size_t bsa_workspace_size(const bsa_params_t* params);
+
+/* Zero the workspace's error word and counters (cudaMemsetAsync on `stream`). Call once after
+ * allocating a workspace, or after a call was aborted. */
+bsa_status_t bsa_workspace_init(const bsa_params_t* params, void* workspace, size_t workspace_bytes,
+                                cudaStream_t stream);
+
+/* Eq. 2 over whole caches (prefill): ck[b][h][j] = mean(k_cache[b][h][s*j : s*j + l]) for every
+ * complete window j of sequence b (s*j + l <= seq_lens[b]); other rows of ck are not written.
+ * Sums are formed in fp64 and rounded once to the element type. No workspace. */
+bsa_status_t bsa_compress_keys(const bsa_params_t* params, const void* k_cache,
+                               const int32_t* seq_lens, void* ck, cudaStream_t stream);
+
+/* Decode-time append of one token per sequence: writes k_new[b][h] / v_new[b][h] ([B][Hkv][d])
+ * into row seq_lens[b] of the caches, increments seq_lens[b], and when that completes a window
+ * (new length T >= l and (T - l) % s == 0) writes ck row (T - l) / s as in bsa_compress_keys.
+ * A sequence already at max_seq_len is left unchanged and sets BSA_DEVERR_CAPACITY in the
+ * workspace error word when a workspace is given (workspace may be NULL). */
+bsa_status_t bsa_compress_append(const bsa_params_t* params, void* k_cache, void* v_cache,
+                                 const void* k_new, const void* v_new, int32_t* seq_lens, void* ck,
+                                 void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Steps 2-4: score q against ck per GQA group (Eq. 6), reduce the window scores onto blocks
+ * (max over overlapping complete windows), pick top_k blocks among those that are neither init
+ * nor local (ties to the lower index) and write the union with the init and local blocks in
+ * ascending order to block_idx (-1 padded) with its count in n_sel. block_scores (optional, may be
+ * NULL) receives the per-block scores. Uses the workspace. */
+bsa_status_t bsa_select_blocks(const bsa_params_t* params, const void* q, const void* ck,
+                               const int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                               float* block_scores, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/* Step 5 (Eq. 5): for every query head, softmax attention (scale params->scale) over the tokens
+ * t < seq_lens[b] of the first n_sel[b][kvh] blocks listed in block_idx[b][kvh] (any order; -1
+ * entries are skipped). Writes out and, if not NULL, lse. A pair with no attended token gets a
+ * zero output and lse = -inf. Uses the workspace for split partials. */
+bsa_status_t bsa_sparse_decode(const bsa_params_t* params, const void* q, const void* k_cache,
+                               const void* v_cache, const int32_t* seq_lens,
+                               const int32_t* block_idx, const int32_t* n_sel, void* out,
+                               float* lse, void* workspace, size_t workspace_bytes,
+                               cudaStream_t stream);
+
+/* Shared-index mode: bsa_sparse_decode for num_layers layers at once, all with the same
+ * block_idx / n_sel / seq_lens. q, k_caches, v_caches, outs and lses are HOST arrays of
+ * num_layers device pointers (lses may be NULL, or contain NULLs). num_layers must not exceed
+ * params->num_layers. One launch covers all layers. */
+bsa_status_t bsa_sparse_decode_layers(const bsa_params_t* params, int32_t num_layers,
+                                      const void* const* q, const void* const* k_caches,
+                                      const void* const* v_caches, const int32_t* seq_lens,
+                                      const int32_t* block_idx, const int32_t* n_sel,
+                                      void* const* outs, float* const* lses, void* workspace,
+                                      size_t workspace_bytes, cudaStream_t stream);
+
+/* One decode step of one layer, as launches chained on `stream` with programmatic dependent
+ * launch: optional append (when k_new and v_new are both non-NULL), then bsa_select_blocks, then
+ * bsa_sparse_decode with the fresh selection. block_idx / n_sel receive the selection;
+ * block_scores and lse may be NULL. */
+bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_cache,
+                             void* v_cache, void* ck, const void* k_new, const void* v_new,
+                             int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                             float* block_scores, void* out, float* lse, void* workspace,
+                             size_t workspace_bytes, cudaStream_t stream);
+
+/* Copy the workspace error word to *flags (bits of bsa_device_error_t), clear it, and
+ * synchronize `stream`. Returns BSA_ERR_DEVICE_CHECK when a bit was set, BSA_OK otherwise. */
+bsa_status_t bsa_read_device_error(void* workspace, size_t workspace_bytes, uint32_t* flags,
+                                   cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* BSA_H */
