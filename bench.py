@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="bsa", choices=["bsa", "reference"])
     ap.add_argument("--workload", default=None)
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the workload's batch (small cases for profiling only)")
     ap.add_argument("--no-graph", action="store_true", help="launch steps directly (no CUDA graph)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
@@ -220,7 +222,8 @@ class Bench:
         return (["append"] + names) if (self.append and self.w.layers == 1) else names
 
     def launches_per_step(self):
-        return len(self.kernel_names())
+        # bsa_select_blocks launches two kernels (scoring, selection); the others one each
+        return len(self.kernel_names()) + 1
 
     def reset_lengths(self):
         self.data["seq_lens"].copy_(self.seq0)
@@ -545,6 +548,8 @@ def main():
     args = parse()
     from block_sparse_attention_compressed_b200.workloads import DEFAULT_WORKLOAD, WORKLOADS
     w = WORKLOADS[args.workload or DEFAULT_WORKLOAD]
+    if args.batch:
+        w = w.replace(batch=args.batch, name=f"{w.name}@batch{args.batch}")
     world, rank, local = dist_init(args)
     if args.impl == "reference":
         res = run_reference(args, w, world, rank)

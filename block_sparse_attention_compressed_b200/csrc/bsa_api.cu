@@ -36,7 +36,8 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
     if (q.block_size % 16 != 0 || q.block_size > 256) return BSA_ERR_UNSUPPORTED;
     if (q.num_layers > BSA_MAX_LAYERS) return BSA_ERR_UNSUPPORTED;
     const int64_t sel = (int64_t)q.n_init + q.n_local + q.top_k;
-    if (sel < 1 || sel > 65536) return BSA_ERR_INVALID_ARG;
+    if (sel < 1) return BSA_ERR_INVALID_ARG;
+    if (sel > 4096) return BSA_ERR_UNSUPPORTED;
     const int64_t pairs = (int64_t)q.batch * q.num_kv_heads;
     if (pairs > (1 << 24)) return BSA_ERR_UNSUPPORTED;
 
@@ -69,22 +70,27 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
     P.scale_log2 = (float)(scale * log2e);
     P.score_log2 = (float)(log2e / tau);
 
-    // Scoring split: enough CTAs to cover the GPU twice when the problem allows it, with slices
-    // that are whole 16-row tiles per warp.
+    // Scoring: 64-row chunks, spread evenly over a persistent grid at launch time.
+    P.nchunk = (P.nc_cap + 63) / 64;
+    P.total_chunks = (int64_t)P.pairs * P.nchunk;
+    // Selection: one CTA per pair when there are enough pairs to fill the GPU in one wave,
+    // otherwise the pairs' windows are split into parts of at least 256 windows.
     {
         const int64_t nc = P.nc_cap > 0 ? P.nc_cap : 1;
-        int64_t items = (nc + 1023) / 1024;
-        const int64_t want = (2 * kNumSMs + P.pairs - 1) / P.pairs;
-        const int64_t most = (nc + 16 * kScoreWarps - 1) / (16 * kScoreWarps);
-        if (items < want) items = want < most ? want : most;
-        if (items < 1) items = 1;
-        const int64_t rows_item = (nc + items - 1) / items;
-        int64_t rpw = (rows_item + kScoreWarps - 1) / kScoreWarps;
-        rpw = (rpw + 15) / 16 * 16;
-        P.score_rows_per_warp = (int)rpw;
-        P.score_items = (int)((nc + rpw * kScoreWarps - 1) / (rpw * kScoreWarps));
-        if ((int64_t)P.pairs * P.score_items > 0x7fffffff) return BSA_ERR_UNSUPPORTED;
-        P.score_smem = (size_t)P.nb_cap * sizeof(uint32_t);
+        int64_t parts = kNumSMs / P.pairs;
+        const int64_t most = (nc + 255) / 256;
+        if (parts > most) parts = most;
+        if (parts < 1) parts = 1;
+        const int64_t pw = (nc + parts - 1) / parts;
+        P.select_part_windows = (int)pw;
+        P.select_parts = (int)((nc + pw - 1) / pw);
+        if ((int64_t)P.pairs * P.select_parts > 0x7fffffff) return BSA_ERR_UNSUPPORTED;
+        const int64_t wmax = (P.BS + P.l - 2) / P.s + 2;  // windows overlapping one block, bound
+        // the key array also stages the chunk statistics (2 words per float2)
+        P.select_keys = (size_t)P.nb_cap > (size_t)(2 * P.nchunk * P.Gp)
+                            ? (size_t)P.nb_cap : (size_t)(2 * P.nchunk * P.Gp);
+        P.select_smem = (P.select_keys + (size_t)pw + (size_t)wmax) * sizeof(uint32_t);
+        if (P.select_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
     }
     // Decode split: about eight blocks per SM slot in flight, whole blocks per CTA.
     {
@@ -93,7 +99,8 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
         if (bpc < 1) bpc = 1;
         if (bpc > 16) bpc = 16;
         if (bpc > P.sel_cap) bpc = P.sel_cap;
-        const int64_t splits = (P.sel_cap + bpc - 1) / bpc;
+        int64_t splits = (P.sel_cap + bpc - 1) / bpc;
+        if (splits * P.Gp > kMaxCombineSlots) splits = kMaxCombineSlots / P.Gp;
         P.dec_splits = (int)splits;
         P.dec_bpc = (int)((P.sel_cap + splits - 1) / splits);
     }
@@ -101,14 +108,16 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
     size_t off = 0;
     P.off_err = off;
     off = align_up(off + sizeof(uint32_t));
-    P.off_score_cnt = off;
+    P.off_sel_cnt = off;
     off = align_up(off + (size_t)P.pairs * sizeof(int));
     P.off_dec_cnt = off;
     off = align_up(off + (size_t)P.layers * P.pairs * sizeof(int));
     P.off_logits = off;
     off = align_up(off + (size_t)P.pairs * P.nc_cap * P.Gp * sizeof(float));
     P.off_stats = off;
-    off = align_up(off + (size_t)P.pairs * P.score_items * P.Gp * sizeof(float2));
+    off = align_up(off + (size_t)P.pairs * P.nchunk * P.Gp * sizeof(float2));
+    P.off_bscores = off;
+    off = align_up(off + (size_t)P.pairs * P.nb_cap * sizeof(float));
     P.off_part_ml = off;
     off = align_up(off + (size_t)P.layers * P.pairs * P.dec_splits * P.Gp * sizeof(float2));
     P.off_part_acc = off;
@@ -133,20 +142,43 @@ bool ok16(const void* p) { return p && is_aligned(p, 16); }
 bool ok4(const void* p) { return p && is_aligned(p, 4); }
 
 ScoreArgs score_args(const Plan& P, const void* q, const void* ck, const int32_t* seq_lens,
-                     int32_t* block_idx, int32_t* n_sel, float* block_scores, void* ws) {
+                     void* ws) {
     ScoreArgs a;
     memset(&a, 0, sizeof a);
     a.q = q;
     a.ck = ck;
     a.seq_lens = seq_lens;
-    a.block_idx = block_idx;
-    a.n_sel = n_sel;
-    a.block_scores = block_scores;
     a.err = ws_at<uint32_t>(ws, P.off_err);
-    a.cnt = ws_at<int>(ws, P.off_score_cnt);
     a.logits = ws_at<float>(ws, P.off_logits);
     a.stats = ws_at<float2>(ws, P.off_stats);
+    a.B = P.B;
     a.Hq = P.Hq;
+    a.Hkv = P.Hkv;
+    a.G = P.G;
+    a.Gp = P.Gp;
+    a.l = P.l;
+    a.s = P.s;
+    a.T_cap = P.T_cap;
+    a.nc_cap = P.nc_cap;
+    a.nchunk = P.nchunk;
+    a.total_chunks = P.total_chunks;
+    a.score_log2 = P.score_log2;
+    return a;
+}
+
+SelectArgs select_args(const Plan& P, const int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                       float* block_scores, void* ws) {
+    SelectArgs a;
+    memset(&a, 0, sizeof a);
+    a.seq_lens = seq_lens;
+    a.logits = ws_at<float>(ws, P.off_logits);
+    a.stats = ws_at<float2>(ws, P.off_stats);
+    a.bscores = ws_at<float>(ws, P.off_bscores);
+    a.block_scores = block_scores;
+    a.block_idx = block_idx;
+    a.n_sel = n_sel;
+    a.err = ws_at<uint32_t>(ws, P.off_err);
+    a.cnt = ws_at<int>(ws, P.off_sel_cnt);
     a.Hkv = P.Hkv;
     a.G = P.G;
     a.Gp = P.Gp;
@@ -160,10 +192,22 @@ ScoreArgs score_args(const Plan& P, const void* q, const void* ck, const int32_t
     a.T_cap = P.T_cap;
     a.nc_cap = P.nc_cap;
     a.nb_cap = P.nb_cap;
-    a.items = P.score_items;
-    a.rows_per_warp = P.score_rows_per_warp;
-    a.score_log2 = P.score_log2;
+    a.nchunk = P.nchunk;
+    a.key_words = (int64_t)P.select_keys;
+    a.parts = P.select_parts;
+    a.part_windows = P.select_part_windows;
     return a;
+}
+
+// Scoring then selection, chained on the stream.
+bsa_status_t do_select(const Plan& P, const void* q, const void* ck, const int32_t* seq_lens,
+                       int32_t* block_idx, int32_t* n_sel, float* block_scores, void* ws,
+                       cudaStream_t st) {
+    ScoreArgs sa = score_args(P, q, ck, seq_lens, ws);
+    cudaError_t e = launch_score(P, sa, st);
+    if (e != cudaSuccess) return BSA_ERR_CUDA;
+    SelectArgs la = select_args(P, seq_lens, block_idx, n_sel, block_scores, ws);
+    return from_cuda(launch_select(P, la, st));
 }
 
 DecodeArgs decode_args(const Plan& P, const int32_t* seq_lens, const int32_t* block_idx,
@@ -261,7 +305,7 @@ bsa_status_t bsa_workspace_init(const bsa_params_t* params, void* ws, size_t ws_
     bsa_status_t st = make_plan(params, &P);
     if (st != BSA_OK) return st;
     if ((st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
-    // error word and both counter arrays are contiguous at the front
+    // the error word and both counter arrays are contiguous at the front
     return from_cuda(cudaMemsetAsync(ws, 0, P.off_logits, stream));
 }
 
@@ -270,7 +314,8 @@ bsa_status_t bsa_compress_keys(const bsa_params_t* params, const void* k_cache,
     Plan P;
     bsa_status_t st = make_plan(params, &P);
     if (st != BSA_OK) return st;
-    if (!ok16(k_cache) || !ok4(seq_lens) || !ok16(ck)) return BSA_ERR_INVALID_ARG;
+    if (!ok16(k_cache) || !ok4(seq_lens)) return BSA_ERR_INVALID_ARG;
+    if (P.nc_cap > 0 && !ok16(ck)) return BSA_ERR_INVALID_ARG;  // no window fits: ck may be empty
     CompressArgs a;
     memset(&a, 0, sizeof a);
     a.k = k_cache;
@@ -311,8 +356,7 @@ bsa_status_t bsa_select_blocks(const bsa_params_t* params, const void* q, const 
     if (P.nc_cap > 0 && !ok16(ck)) return BSA_ERR_INVALID_ARG;
     if (block_scores && !ok4(block_scores)) return BSA_ERR_INVALID_ARG;
     if ((st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
-    ScoreArgs a = score_args(P, q, ck, seq_lens, block_idx, n_sel, block_scores, ws);
-    return from_cuda(launch_score_select(P, a, stream));
+    return do_select(P, q, ck, seq_lens, block_idx, n_sel, block_scores, ws, stream);
 }
 
 bsa_status_t bsa_sparse_decode_layers(const bsa_params_t* params, int32_t num_layers,
@@ -377,8 +421,8 @@ bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_
         st = do_append(P, k_cache, v_cache, k_new, v_new, seq_lens, ck, ws, stream);
         if (st != BSA_OK) return st;
     }
-    ScoreArgs sa = score_args(P, q, ck, seq_lens, block_idx, n_sel, block_scores, ws);
-    if ((st = from_cuda(launch_score_select(P, sa, stream))) != BSA_OK) return st;
+    if ((st = do_select(P, q, ck, seq_lens, block_idx, n_sel, block_scores, ws, stream)) != BSA_OK)
+        return st;
     DecodeArgs da = decode_args(P, seq_lens, block_idx, n_sel, ws);
     da.q[0] = q;
     da.k[0] = k_cache;

@@ -16,6 +16,7 @@ constexpr int kMaxG = 8;         // query heads per kv head handled by one mma t
 constexpr int kScoreWarps = 8;   // warps per scoring CTA
 constexpr int kDecodeWarps = 4;  // warps per decode CTA
 constexpr int kMaxNbCap = 32768; // selection blocks per sequence (shared-memory key array)
+constexpr int kMaxCombineSlots = 1024;  // splits * Gp handled by the decode combine
 
 // ------------------------------------------------------------------------------------------------
 // Launch plan: every size and workspace offset derived from bsa_params_t. The same function feeds
@@ -26,17 +27,20 @@ struct Plan {
     int pairs;
     float scale_log2;  // attention scale * log2(e): softmax evaluated with exp2
     float score_log2;  // (1 / tau) * log2(e)
-    // scoring: grid = pairs * score_items CTAs of kScoreWarps warps, score_rows_per_warp rows each
-    int score_items, score_rows_per_warp;
-    size_t score_smem;  // dynamic shared memory of the selection phase (block keys)
+    // scoring: 64-row chunks of compressed keys, spread evenly over a persistent grid
+    int64_t nchunk, total_chunks;
+    // selection: pairs * select_parts CTAs, each scoring select_part_windows windows
+    int select_parts, select_part_windows;
+    size_t select_keys;  // words of the block-key array at the front of its shared memory
+    size_t select_smem;  // dynamic shared memory of the selection kernel
     // decode: grid = layers * pairs * dec_splits CTAs of kDecodeWarps warps, dec_bpc blocks each
     int dec_splits, dec_bpc;
     // workspace layout (bytes)
-    size_t off_err, off_score_cnt, off_dec_cnt, off_logits, off_stats, off_part_ml, off_part_acc;
+    size_t off_err, off_sel_cnt, off_dec_cnt, off_logits, off_stats, off_bscores, off_part_ml,
+        off_part_acc;
     size_t ws_bytes;
 };
 
-// ------------------------------------------------------------------------------------------------
 struct CompressArgs {
     const void* k;
     void* ck;
@@ -62,17 +66,27 @@ struct ScoreArgs {
     const void* q;
     const void* ck;
     const int32_t* seq_lens;
+    uint32_t* err;
+    float* logits;        // [pairs][nc_cap][Gp], log2 units
+    float2* stats;        // [pairs][nchunk][Gp] (max, sum of exp2(x - max)) per chunk and head
+    int B, Hq, Hkv, G, Gp, l, s;
+    int64_t T_cap, nc_cap, nchunk, total_chunks;
+    float score_log2;
+};
+
+struct SelectArgs {
+    const int32_t* seq_lens;
+    const float* logits;
+    const float2* stats;
+    float* bscores;       // [pairs][nb_cap] block scores (workspace)
+    float* block_scores;  // caller's copy, may be null
     int32_t* block_idx;
     int32_t* n_sel;
-    float* block_scores;  // may be null
     uint32_t* err;
     int* cnt;             // [pairs] completion counters
-    float* logits;        // [pairs][nc_cap][Gp], log2 units
-    float2* stats;        // [pairs][items][Gp] (max, sum of exp2(x - max)) per item and head
-    int Hq, Hkv, G, Gp, l, s, BS, n_init, n_local, top_k, sel_cap;
-    int64_t T_cap, nc_cap, nb_cap;
-    int items, rows_per_warp;
-    float score_log2;
+    int Hkv, G, Gp, l, s, BS, n_init, n_local, top_k, sel_cap;
+    int64_t T_cap, nc_cap, nb_cap, nchunk, key_words;
+    int parts, part_windows;
 };
 
 struct DecodeArgs {
@@ -97,7 +111,8 @@ struct DecodeArgs {
 // Launchers (one per kernel family); they pick the template instance from the plan's dtype/D.
 cudaError_t launch_compress_keys(const Plan& p, const CompressArgs& a, cudaStream_t st);
 cudaError_t launch_append(const Plan& p, const AppendArgs& a, cudaStream_t st);
-cudaError_t launch_score_select(const Plan& p, const ScoreArgs& a, cudaStream_t st);
+cudaError_t launch_score(const Plan& p, const ScoreArgs& a, cudaStream_t st);
+cudaError_t launch_select(const Plan& p, const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_decode(const Plan& p, const DecodeArgs& a, int layers, cudaStream_t st);
 
 // Launch with programmatic dependent launch allowed: the kernel may start while the previous

@@ -78,26 +78,51 @@ __device__ void finish_split(const DecodeArgs& a, int layer, int pair, int lp, i
     __syncthreads();
     if (!s_last) return;
     __threadfence();
+    // Combine the splits: per head the global max M and denominator, per split a scale factor
+    // exp2(m_s - M) (shared memory), then every (head, d) element sums its scaled numerators with
+    // the loads of kU splits in flight.
+    __shared__ float2 s_ml[kMaxCombineSlots];
+    __shared__ float s_M[kMaxG], s_den[kMaxG];
+    const int S = a.splits;
+    const float2* ml0 = a.part_ml + (size_t)lp * S * a.Gp;
+    const float* acc0 = a.part_acc + (size_t)lp * S * a.Gp * D;
+    for (int e = threadIdx.x; e < S * a.Gp; e += NT) s_ml[e] = ld_cg(ml0 + e);  // one round
+    __syncthreads();
+    if (threadIdx.x < G) {
+        const int h = threadIdx.x;
+        float M = -INFINITY;
+        for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, s_ml[s2 * a.Gp + h].x);
+        float den = 0.f;
+        for (int s2 = 0; s2 < S; ++s2) {
+            const float2 ml = s_ml[s2 * a.Gp + h];
+            const float f = M == -INFINITY ? 0.f : exp2f(ml.x - M);
+            den = fmaf(f, ml.y, den);
+            s_ml[s2 * a.Gp + h].x = f;  // becomes the split's scale factor
+        }
+        s_M[h] = M;
+        s_den[h] = den;
+    }
+    __syncthreads();
     const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
-    const float2* ml0 = a.part_ml + (size_t)lp * a.splits * a.Gp;
-    const float* acc0 = a.part_acc + (size_t)lp * a.splits * a.Gp * D;
     T* out = reinterpret_cast<T*>(a.out[layer]) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
     float* lse = a.lse[layer] ? a.lse[layer] + (size_t)b * a.Hq + (size_t)kvh * G : nullptr;
+    constexpr int kU = 8;
     for (int e = threadIdx.x; e < G * D; e += NT) {
         const int h = e / D, dd = e - h * D;
-        float M = -INFINITY;
-        for (int s = 0; s < a.splits; ++s) M = fmaxf(M, ld_cg(ml0 + (size_t)s * a.Gp + h).x);
-        float num = 0.f, den = 0.f;
-        if (M != -INFINITY) {
-            for (int s = 0; s < a.splits; ++s) {
-                const float2 ml = ld_cg(ml0 + (size_t)s * a.Gp + h);
-                const float f = exp2f(ml.x - M);
-                num = fmaf(f, ld_cg(acc0 + ((size_t)s * a.Gp + h) * D + dd), num);
-                den = fmaf(f, ml.y, den);
-            }
+        float num = 0.f;
+        for (int s0 = 0; s0 < S; s0 += kU) {
+            float v[kU];
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                v[u] = s0 + u < S ? ld_cg(acc0 + ((size_t)(s0 + u) * a.Gp + h) * D + dd) : 0.f;
+#pragma unroll
+            for (int u = 0; u < kU; ++u)
+                if (s0 + u < S) num = fmaf(s_ml[(s0 + u) * a.Gp + h].x, v[u], num);
         }
+        const float den = s_den[h];
         store_out<T>(out + h * D + dd, den > 0.f ? num / den : 0.f);
-        if (dd == 0 && lse) lse[h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+        if (dd == 0 && lse)
+            lse[h] = den > 0.f ? (s_M[h] + log2f(den)) * 0.69314718055994531f : -INFINITY;
     }
 }
 
@@ -275,18 +300,19 @@ __global__ void __launch_bounds__(kDecodeThreads, 2) decode_bf16_kernel(DecodeAr
         }
         return n_units;
     };
-    int64_t base = -1;
-    int u = next_unit(-1, base);
-    KVTile<D> cur, nxt;
-    if (u < n_units) load_kvtile<D>(cur, kp, vp, base, si.T, g, tq);
-    while (u < n_units) {
-        int64_t nbase = -1;
-        const int un = next_unit(u, nbase);
-        if (un < n_units) load_kvtile<D>(nxt, kp, vp, nbase, si.T, g, tq);
-        attend_tile<D>(cur, qf, base, si.T, a.scale_log2, g, m, lsum, acc);
-        cur = nxt;
-        u = un;
-        base = nbase;
+    // Two tile buffers in ping-pong (no register copy waits on a pending load).
+    KVTile<D> ta, tb;
+    int64_t base_a = -1, base_b = -1;
+    int ua = next_unit(-1, base_a);
+    if (ua < n_units) load_kvtile<D>(ta, kp, vp, base_a, si.T, g, tq);
+    while (ua < n_units) {
+        const int ub = next_unit(ua, base_b);
+        if (ub < n_units) load_kvtile<D>(tb, kp, vp, base_b, si.T, g, tq);
+        attend_tile<D>(ta, qf, base_a, si.T, a.scale_log2, g, m, lsum, acc);
+        if (ub >= n_units) break;
+        ua = next_unit(ub, base_a);
+        if (ua < n_units) load_kvtile<D>(ta, kp, vp, base_a, si.T, g, tq);
+        attend_tile<D>(tb, qf, base_b, si.T, a.scale_log2, g, m, lsum, acc);
     }
 
 #pragma unroll

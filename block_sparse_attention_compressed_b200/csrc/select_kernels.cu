@@ -3,23 +3,30 @@
 // GQA group; "Fine-grained supervision" for the max-pool onto the block grid; Theoretical
 // Foundation, Eq. 1 and SparDA Architecture, Eq. 4 for the union with init/local blocks and f_top).
 //
-// One kernel, grid = pairs * items CTAs (pair-major). Each CTA scores a contiguous slice of the
-// pair's compressed keys against the group's G query heads and writes log2-domain logits plus the
-// slice's per-head (max, sum exp2) to the workspace. The last CTA of a pair to finish (completion
-// counter, no waiting) merges the per-slice statistics into each head's softmax normaliser,
-// evaluates S[j] = sum_h softmax_h[j] on the fly, max-pools onto blocks and runs the selection.
+// Two kernels chained with programmatic dependent launch:
 //
-// bf16 path: the contraction q . K~_j runs on the tensor cores with mma.m16n8k16: compressed-key
-// rows are the M dimension (16 per tile), the group's heads are N (padded to 8), head_dim is K.
-// Because a dot product does not care about the order of its terms, each lane feeds the A operand
-// straight from its own 16-byte global loads (no shared-memory staging, no shuffles) and the q
-// operand is permuted the same way once per CTA.
+// score (persistent): every warp owns a contiguous, equal share of the 64-row chunks of all pairs'
+//   compressed keys, so all warps finish together (no partial last wave). It streams 16-row tiles,
+//   computes the group's logits x[j][h] = q_h . K~_j / tau (log2 units) and writes them to the
+//   workspace together with each chunk's per-head (max, sum exp2(x - max)).
+//   bf16: the contraction runs on the tensor cores with mma.m16n8k16 -- rows are M, the G heads
+//   (padded to 8) are N, head_dim is K. A dot product does not depend on the order of its terms,
+//   so each lane feeds the A operand straight from its own 16-byte global loads and q's operand is
+//   permuted the same way. fp32: FMA dot products, one warp per row.
+//
+// select (pairs x parts CTAs): merges the chunk statistics into each head's softmax normaliser,
+//   turns the logits of its part of the windows into S[j] = sum_h softmax_h[j], max-pools S onto
+//   the blocks it owns and writes the block scores. The last part of a pair to finish (completion
+//   counter, no waiting) runs the top-k: an 8-bit radix select over order-preserving uint32 keys,
+//   ties resolved toward the lower block index by an ordered scan, then the ascending union with
+//   the init and local blocks.
 #include "bsa_internal.cuh"
 
 namespace bsa {
 namespace {
 
 constexpr int kScoreThreads = kScoreWarps * 32;
+constexpr int kSelectThreads = 512;
 
 // Block-wide exclusive scan of one int per thread (contiguous, in thread order).
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total) {
@@ -48,72 +55,404 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
     return base + x - v;
 }
 
-// Selection for one pair, run by a whole CTA after every slice of the pair is scored.
-__device__ void select_pair(const ScoreArgs& a, int pair, int64_t T, int64_t nc, bool ok,
-                            uint32_t* keys) {
-    __shared__ float sM[kMaxG], sInvZ[kMaxG];
+__device__ __forceinline__ int64_t num_windows(int64_t T, int l, int s) {
+    return T < l ? 0 : (T - l) / s + 1;
+}
+// Last window overlapping block b (before clamping to the window count).
+__device__ __forceinline__ int64_t last_window(int64_t b, int BS, int s) {
+    return (b * BS + BS - 1) / s;
+}
+// Smallest block whose first overlapping window is >= j.
+__device__ __forceinline__ int64_t first_block_from(int64_t j, int BS, int l, int s) {
+    return j <= 0 ? 0 : ((int64_t)s * (j - 1) + l + BS - 1) / BS;
+}
+// First and last window overlapping block b, in 32 bits (token indices stay below 2^31).
+__device__ __forceinline__ uint32_t first_window32(uint32_t b, uint32_t BS, uint32_t l, uint32_t s) {
+    const uint32_t tok0 = b * BS;
+    return tok0 >= l ? (tok0 - l) / s + 1 : 0;
+}
+__device__ __forceinline__ uint32_t last_window32(uint32_t b, uint32_t BS, uint32_t s) {
+    return (b * BS + BS - 1) / s;
+}
+
+__device__ __forceinline__ void report_lengths(const ScoreArgs& a) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) {
+        for (int b = 0; b < a.B; ++b) {
+            const int T = a.seq_lens[b];
+            if (T < 0 || T > a.T_cap) atomicOr(a.err, (uint32_t)BSA_DEVERR_SEQ_LEN);
+        }
+    }
+}
+
+// ================================================================================ score kernels
+__device__ __forceinline__ void flush_stats(float2* dst, float m0, float s0, float m1, float s1,
+                                            int g, int tq, int G) {
+    // combine the 8 row groups (lanes with equal tq), then lanes g == 0 publish heads 2tq, 2tq+1
+#pragma unroll
+    for (int off = 4; off < 32; off <<= 1) {
+        float mo = __shfl_xor_sync(0xffffffffu, m0, off), so = __shfl_xor_sync(0xffffffffu, s0, off);
+        online_merge(m0, s0, mo, so);
+        mo = __shfl_xor_sync(0xffffffffu, m1, off);
+        so = __shfl_xor_sync(0xffffffffu, s1, off);
+        online_merge(m1, s1, mo, so);
+    }
+    if (g == 0) {
+        if (2 * tq < G) dst[2 * tq] = make_float2(m0, s0);
+        if (2 * tq + 1 < G) dst[2 * tq + 1] = make_float2(m1, s1);
+    }
+}
+
+template <int D>
+struct KTile {
+    static constexpr int NI = D / 32;  // 16-byte chunks a lane holds per row (chunks tq + 4i)
+    uint4 a[NI], b[NI];                // rows r+g and r+g+8 of the tile
+};
+
+template <int D>
+__device__ __forceinline__ void load_ktile(KTile<D>& t, const uint16_t* ckp, int64_t r, int64_t r1,
+                                           int g, int tq) {
+    const int64_t ra = r + g, rb = r + g + 8;
+#pragma unroll
+    for (int i = 0; i < KTile<D>::NI; ++i) {
+        const int col = (tq + 4 * i) * 8;
+        t.a[i] = ra < r1 ? ld_stream(ckp + ra * D + col) : make_uint4(0, 0, 0, 0);
+        t.b[i] = rb < r1 ? ld_stream(ckp + rb * D + col) : make_uint4(0, 0, 0, 0);
+    }
+}
+
+// A warp's share of the tile stream: slot u covers tile (u % 4) of chunk c_lo + u / 4.
+struct TileCursor {
+    int64_t c_lo, n_slots;
+    int cached_pair;
+    int64_t cached_nc;
+};
+
+__device__ __forceinline__ int64_t pair_windows(const ScoreArgs& a, int pair, TileCursor& tc) {
+    if (pair != tc.cached_pair) {
+        tc.cached_pair = pair;
+        const int64_t T = a.seq_lens[pair / a.Hkv];
+        tc.cached_nc = (T >= 0 && T <= a.T_cap) ? num_windows(T, a.l, a.s) : 0;
+    }
+    return tc.cached_nc;
+}
+
+// First slot >= u whose tile holds at least one window; n_slots when there is none.
+__device__ __forceinline__ int64_t next_slot(const ScoreArgs& a, TileCursor& tc, int64_t u) {
+    while (u < tc.n_slots) {
+        const int64_t chunk = tc.c_lo + (u >> 2);
+        const int pair = (int)(chunk / a.nchunk);
+        const int64_t row = (chunk - (int64_t)pair * a.nchunk) * 64 + (u & 3) * 16;
+        if (row < pair_windows(a, pair, tc)) return u;
+        u = (u | 3) + 1;  // the rest of this chunk is past the sequence: next chunk
+    }
+    return tc.n_slots;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads, 2) score_bf16_kernel(ScoreArgs a) {
+    constexpr int NI = D / 32;
+    const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const int64_t W = (int64_t)gridDim.x * kScoreWarps;
+    const int64_t w = (int64_t)blockIdx.x * kScoreWarps + (threadIdx.x >> 5);
+    TileCursor tc;
+    tc.c_lo = w * a.total_chunks / W;
+    tc.n_slots = ((w + 1) * a.total_chunks / W - tc.c_lo) * 4;
+    tc.cached_pair = -1;
+    tc.cached_nc = 0;
+    pdl_trigger();
+    pdl_wait();
+    report_lengths(a);
+    const bool h0 = 2 * tq < a.G, h1 = 2 * tq + 1 < a.G;
+    int cur_pair = -1;
+    uint32_t qf[NI][4];
+    float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
+
+    KTile<D> ta, tb;
+    auto load_slot = [&](KTile<D>& t, int64_t u) {
+        const int64_t chunk = tc.c_lo + (u >> 2);
+        const int pair = (int)(chunk / a.nchunk);
+        const int64_t row = (chunk - (int64_t)pair * a.nchunk) * 64 + (u & 3) * 16;
+        const int64_t r1 = min(row + 16, pair_windows(a, pair, tc));
+        load_ktile<D>(t, reinterpret_cast<const uint16_t*>(a.ck) + (size_t)pair * a.nc_cap * D, row,
+                      r1, g, tq);
+    };
+    auto compute_slot = [&](const KTile<D>& t, int64_t u, int64_t u_next) {
+        const int64_t chunk = tc.c_lo + (u >> 2);
+        const int pair = (int)(chunk / a.nchunk);
+        const int64_t ci = chunk - (int64_t)pair * a.nchunk;
+        const int64_t row = ci * 64 + (u & 3) * 16;
+        const int64_t r1 = min(row + 16, pair_windows(a, pair, tc));
+        if (pair != cur_pair) {
+            // q as the B operand: lane (g, tq) holds head g at chunks tq + 4i, the d positions its
+            // own key loads cover (heads >= G are zero)
+            cur_pair = pair;
+            const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
+            const uint16_t* qh = reinterpret_cast<const uint16_t*>(a.q) +
+                                 ((size_t)b * a.Hq + (size_t)kvh * a.G + g) * D;
+#pragma unroll
+            for (int i = 0; i < NI; ++i) {
+                uint4 v = g < a.G ? *reinterpret_cast<const uint4*>(qh + (tq + 4 * i) * 8)
+                                  : make_uint4(0, 0, 0, 0);
+                qf[i][0] = v.x;
+                qf[i][1] = v.y;
+                qf[i][2] = v.z;
+                qf[i][3] = v.w;
+            }
+        }
+        float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                mma_bf16_16816(c, u4_get(t.a[i], 2 * hh), u4_get(t.b[i], 2 * hh),
+                               u4_get(t.a[i], 2 * hh + 1), u4_get(t.b[i], 2 * hh + 1),
+                               qf[i][2 * hh], qf[i][2 * hh + 1]);
+            }
+        }
+        float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
+        const float x0 = c[0] * a.score_log2, x1 = c[1] * a.score_log2;
+        const float x2 = c[2] * a.score_log2, x3 = c[3] * a.score_log2;
+        const int64_t ra = row + g, rb = row + g + 8;
+        if (ra < r1) {
+            if (h1) *reinterpret_cast<float2*>(lg + ra * a.Gp + 2 * tq) = make_float2(x0, x1);
+            else if (h0) lg[ra * a.Gp + 2 * tq] = x0;
+            if (h0) online_add(m0, s0, x0);
+            if (h1) online_add(m1, s1, x1);
+        }
+        if (rb < r1) {
+            if (h1) *reinterpret_cast<float2*>(lg + rb * a.Gp + 2 * tq) = make_float2(x2, x3);
+            else if (h0) lg[rb * a.Gp + 2 * tq] = x2;
+            if (h0) online_add(m0, s0, x2);
+            if (h1) online_add(m1, s1, x3);
+        }
+        // last tile of its chunk in this warp's stream: publish the chunk's statistics
+        if (u_next >= tc.n_slots || (u_next >> 2) != (u >> 2)) {
+            flush_stats(a.stats + ((size_t)pair * a.nchunk + ci) * a.Gp, m0, s0, m1, s1, g, tq, a.G);
+            m0 = m1 = -INFINITY;
+            s0 = s1 = 0.f;
+        }
+    };
+    // ping-pong: the next tile's loads are in flight while the current tile is computed
+    int64_t ua = next_slot(a, tc, 0);
+    if (ua < tc.n_slots) load_slot(ta, ua);
+    while (ua < tc.n_slots) {
+        const int64_t ub = next_slot(a, tc, ua + 1);
+        if (ub < tc.n_slots) load_slot(tb, ub);
+        compute_slot(ta, ua, ub);
+        if (ub >= tc.n_slots) break;
+        ua = next_slot(a, tc, ub + 1);
+        if (ua < tc.n_slots) load_slot(ta, ua);
+        compute_slot(tb, ub, ua);
+    }
+}
+
+// fp32: plain FMA dot products (fp32 inputs keep fp32 accuracy); one warp per row, lanes split d.
+template <int D>
+__global__ void __launch_bounds__(kScoreThreads, 2) score_f32_kernel(ScoreArgs a) {
+    constexpr int E = D / 32;
+    const int lane = threadIdx.x & 31;
+    const int64_t W = (int64_t)gridDim.x * kScoreWarps;
+    const int64_t w = (int64_t)blockIdx.x * kScoreWarps + (threadIdx.x >> 5);
+    const int64_t c_lo = w * a.total_chunks / W, c_hi = (w + 1) * a.total_chunks / W;
+    pdl_trigger();
+    pdl_wait();
+    report_lengths(a);
+    int cur_pair = -1;
+    int64_t nc = 0;
+    float qv[kMaxG][E];
+    for (int64_t chunk = c_lo; chunk < c_hi; ++chunk) {
+        const int pair = (int)(chunk / a.nchunk);
+        const int64_t ci = chunk - (int64_t)pair * a.nchunk;
+        if (pair != cur_pair) {
+            cur_pair = pair;
+            const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
+            const int64_t T = a.seq_lens[b];
+            nc = (T >= 0 && T <= a.T_cap) ? num_windows(T, a.l, a.s) : 0;
+            const float* qb = reinterpret_cast<const float*>(a.q) + ((size_t)b * a.Hq + (size_t)kvh * a.G) * D;
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h)
+#pragma unroll
+                for (int e = 0; e < E; ++e) qv[h][e] = h < a.G ? qb[h * D + lane * E + e] : 0.f;
+        }
+        const int64_t r0 = ci * 64, r1 = min(r0 + 64, nc);
+        if (r0 >= r1) continue;
+        const float* ckp = reinterpret_cast<const float*>(a.ck) + (size_t)pair * a.nc_cap * D;
+        float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
+        float m[kMaxG], s[kMaxG];
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h) {
+            m[h] = -INFINITY;
+            s[h] = 0.f;
+        }
+        for (int64_t r = r0; r < r1; ++r) {
+            float kv[E];
+#pragma unroll
+            for (int e = 0; e < E; ++e) kv[e] = __ldg(ckp + r * D + lane * E + e);
+#pragma unroll
+            for (int h = 0; h < kMaxG; ++h) {
+                if (h >= a.G) break;
+                float p = 0.f;
+#pragma unroll
+                for (int e = 0; e < E; ++e) p = fmaf(qv[h][e], kv[e], p);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
+                const float x = p * a.score_log2;
+                if (lane == h) lg[r * a.Gp + h] = x;
+                online_add(m[h], s[h], x);
+            }
+        }
+        float2* st = a.stats + ((size_t)pair * a.nchunk + ci) * a.Gp;
+#pragma unroll
+        for (int h = 0; h < kMaxG; ++h)
+            if (h < a.G && lane == h) st[h] = make_float2(m[h], s[h]);
+    }
+}
+
+// ============================================================================== select kernel
+template <int GP>
+struct LogitRow {
+    float v[GP];
+};
+template <int GP>
+__device__ __forceinline__ LogitRow<GP> load_row(const float* p) {
+    LogitRow<GP> r;
+    if constexpr (GP == 1) {
+        r.v[0] = __ldcg(p);
+    } else if constexpr (GP == 2) {
+        const float2 t = __ldcg(reinterpret_cast<const float2*>(p));
+        r.v[0] = t.x;
+        r.v[1] = t.y;
+    } else {
+#pragma unroll
+        for (int q = 0; q < GP / 4; ++q) {
+            const float4 t = __ldcg(reinterpret_cast<const float4*>(p) + q);
+            r.v[4 * q] = t.x;
+            r.v[4 * q + 1] = t.y;
+            r.v[4 * q + 2] = t.z;
+            r.v[4 * q + 3] = t.w;
+        }
+    }
+    return r;
+}
+
+// S[j - j0] = sum over the group's heads of exp2(x[j][h] - M_h) / Z_h for windows j in [j0, j1),
+// kU rows per thread in flight.
+template <int GP>
+__device__ void window_scores(const float* lg, int64_t j0, int64_t j1, int G, const float* sM,
+                              const float* sInvZ, float* S) {
+    constexpr int kU = GP <= 4 ? 16 : 8;
+    const int tid = threadIdx.x, NT = blockDim.x;
+    for (int64_t base = j0; base < j1; base += (int64_t)NT * kU) {
+        LogitRow<GP> r[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int64_t j = base + (int64_t)u * NT + tid;
+            if (j < j1) r[u] = load_row<GP>(lg + j * GP);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int64_t j = base + (int64_t)u * NT + tid;
+            if (j < j1) {
+                float acc = 0.f;
+#pragma unroll
+                for (int h = 0; h < GP; ++h)
+                    if (h < G) acc += exp2f(r[u].v[h] - sM[h]) * sInvZ[h];
+                S[j - j0] = acc;
+            }
+        }
+    }
+}
+
+// Top-k of the candidate blocks [init_end, local_begin) by score (ties: lower index first), united
+// with the init and local blocks, written ascending. keys[] (shared) holds the nb block keys and
+// is overwritten. Each thread keeps its contiguous segment of up to kKeysPerThread candidate keys
+// in registers for the radix passes (larger candidate sets are streamed from shared memory).
+constexpr int kKeysPerThread = 8;
+
+__device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys) {
     __shared__ int s_warp[32];
     __shared__ int hist[256];
     __shared__ uint32_t s_prefix;
     __shared__ int s_need;
-    const int tid = threadIdx.x, NT = blockDim.x;
-    const int64_t nb = ok ? (T + a.BS - 1) / a.BS : 0;
-
-    // 1. softmax normaliser of every head from the per-slice (max, sum) pairs
-    if (tid < a.G) {
-        const float2* st = a.stats + (size_t)pair * a.items * a.Gp + tid;
-        float M = -INFINITY;
-        for (int it = 0; it < a.items; ++it) M = fmaxf(M, ld_cg(st + (size_t)it * a.Gp).x);
-        float Z = 0.f;
-        if (M != -INFINITY) {
-            for (int it = 0; it < a.items; ++it) {
-                float2 ms = ld_cg(st + (size_t)it * a.Gp);
-                if (ms.x != -INFINITY) Z += ms.y * exp2f(ms.x - M);
-            }
-        }
-        sM[tid] = M;
-        sInvZ[tid] = Z > 0.f ? 1.f / Z : 0.f;
-    }
-    __syncthreads();
-
-    // 2. block scores: max over the complete windows overlapping the block of sum_h p_h[j]
-    const float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
-    for (int64_t bb = tid; bb < a.nb_cap; bb += NT) {
-        float best = -INFINITY;
-        if (bb < nb && nc > 0) {
-            const int64_t tok0 = bb * a.BS;
-            const int64_t jlo = tok0 >= a.l ? (tok0 - a.l) / a.s + 1 : 0;
-            const int64_t jhi = min((tok0 + a.BS - 1) / a.s, nc - 1);
-            for (int64_t j = jlo; j <= jhi; ++j) {
-                const float* row = lg + j * a.Gp;
-                float S = 0.f;
-                for (int h = 0; h < a.G; ++h) S += exp2f(ld_cg(row + h) - sM[h]) * sInvZ[h];
-                best = fmaxf(best, S);
-            }
-        }
-        if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + bb] = best;
-        keys[bb] = order_key(best);
-    }
-    __syncthreads();
-
-    // 3. top-k among the candidates [init_end, local_begin): radix select of the k-th key
-    const int64_t init_end = min((int64_t)a.n_init, nb);
-    const int64_t local_begin = max(nb - (int64_t)a.n_local, (int64_t)0);
-    const int64_t clo = init_end, chi = max(local_begin, init_end);
-    const int64_t ncand = chi - clo;
-    const int kk = (int)min((int64_t)a.top_k, ncand);
+    __shared__ uint32_t s_and[32], s_or[32];
+    const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31;
+    const int init_end = min(a.n_init, nb);
+    const int local_begin = max(nb - a.n_local, 0);
+    const int clo = init_end, chi = max(local_begin, init_end);
+    const int ncand = chi - clo;
+    const int kk = min(a.top_k, ncand);
     const bool take_all = (kk == ncand);
+    const int per = (ncand + NT - 1) / NT;  // contiguous segment of each thread
+    const int seg_lo = clo + tid * per, seg_hi = min(seg_lo + per, chi);
+    const bool in_regs = per <= kKeysPerThread;
+    uint32_t kr[kKeysPerThread];
+#pragma unroll
+    for (int e = 0; e < kKeysPerThread; ++e) kr[e] = (in_regs && seg_lo + e < seg_hi) ? keys[seg_lo + e] : 0u;
+
     uint32_t thr = 0xffffffffu;  // keys > thr are taken, plus the first `need` keys == thr
     int need = 0;
     if (kk > 0 && !take_all) {
-        uint32_t prefix = 0, mask = 0;
+        // bytes that every candidate shares need no histogram pass: start at the first byte in
+        // which two candidates differ (block-wide AND / OR of the keys)
+        uint32_t kand = 0xffffffffu, kor = 0u;
+        if (in_regs) {
+#pragma unroll
+            for (int e = 0; e < kKeysPerThread; ++e) {
+                if (seg_lo + e < seg_hi) {
+                    kand &= kr[e];
+                    kor |= kr[e];
+                }
+            }
+        } else {
+            for (int i = seg_lo; i < seg_hi; ++i) {
+                kand &= keys[i];
+                kor |= keys[i];
+            }
+        }
+        kand = __reduce_and_sync(0xffffffffu, kand);
+        kor = __reduce_or_sync(0xffffffffu, kor);
+        if (lane == 0) {
+            s_and[tid >> 5] = kand;
+            s_or[tid >> 5] = kor;
+        }
+        __syncthreads();
+        kand = 0xffffffffu;
+        kor = 0u;
+        for (int w = 0; w < (NT >> 5); ++w) {
+            kand &= s_and[w];
+            kor |= s_or[w];
+        }
+        const uint32_t diff = kand ^ kor;  // bits in which some candidates differ
+        int top = 24;
+        while (top > 0 && (diff >> top) == 0u) top -= 8;
+        uint32_t prefix = top < 24 ? (kand & (0xffffffffu << (top + 8))) : 0u;
+        uint32_t mask = top < 24 ? (0xffffffffu << (top + 8)) : 0u;
         need = kk;
-        for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int shift = top; shift >= 0; shift -= 8) {
             for (int i = tid; i < 256; i += NT) hist[i] = 0;
             __syncthreads();
-            for (int64_t i = clo + tid; i < chi; i += NT) {
-                const uint32_t u = keys[i];
-                if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & 255u], 1);
+            // warp-aggregated histogram (keys of a warp often share a digit): one atomic per
+            // distinct digit per warp; all of a thread's keys are processed independently
+            if (in_regs) {
+                uint32_t dg[kKeysPerThread];
+#pragma unroll
+                for (int e = 0; e < kKeysPerThread; ++e) {
+                    const bool live = seg_lo + e < seg_hi && (kr[e] & mask) == prefix;
+                    dg[e] = live ? ((kr[e] >> shift) & 255u) : 256u;
+                }
+#pragma unroll
+                for (int e = 0; e < kKeysPerThread; ++e) {
+                    const uint32_t peers = __match_any_sync(0xffffffffu, dg[e]);
+                    if (dg[e] < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[dg[e]], __popc(peers));
+                }
+            } else {
+                for (int i0 = 0; i0 < per; ++i0) {
+                    const int i = seg_lo + i0;
+                    const uint32_t u = i < seg_hi ? keys[i] : 0u;
+                    const uint32_t d = (i < seg_hi && (u & mask) == prefix) ? ((u >> shift) & 255u) : 256u;
+                    const uint32_t peers = __match_any_sync(0xffffffffu, d);
+                    if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
+                }
             }
             __syncthreads();
             if (tid < 32) {
@@ -150,265 +489,191 @@ __device__ void select_pair(const ScoreArgs& a, int pair, int64_t T, int64_t nc,
         }
         thr = prefix;
     }
-
-    // 4. mark the taken candidates in index order (equal keys: lowest block first)
+    // mark the taken candidates in index order (equal keys: lowest block first)
     {
-        const int64_t per = (ncand + NT - 1) / NT;
-        const int64_t lo = clo + tid * per, hi = min(lo + per, chi);
         int cnt = 0;
-        for (int64_t i = lo; i < hi; ++i) cnt += (keys[i] == thr);
+        if (in_regs) {
+#pragma unroll
+            for (int e = 0; e < kKeysPerThread; ++e) cnt += (seg_lo + e < seg_hi && kr[e] == thr);
+        } else {
+            for (int i = seg_lo; i < seg_hi; ++i) cnt += (keys[i] == thr);
+        }
         int tot;
         int r = block_exclusive_scan(cnt, s_warp, &tot);
-        for (int64_t i = lo; i < hi; ++i) {
-            const uint32_t u = keys[i];
-            const bool take = take_all || u > thr || (u == thr && r < need);
-            r += (u == thr);
-            keys[i] = take ? 1u : 0u;
+        if (in_regs) {
+#pragma unroll
+            for (int e = 0; e < kKeysPerThread; ++e) {
+                if (seg_lo + e < seg_hi) {
+                    const uint32_t u = kr[e];
+                    const bool take = take_all || u > thr || (u == thr && r < need);
+                    r += (u == thr);
+                    keys[seg_lo + e] = take ? 1u : 0u;
+                }
+            }
+        } else {
+            for (int i = seg_lo; i < seg_hi; ++i) {
+                const uint32_t u = keys[i];
+                const bool take = take_all || u > thr || (u == thr && r < need);
+                r += (u == thr);
+                keys[i] = take ? 1u : 0u;
+            }
         }
     }
     __syncthreads();
-
-    // 5. union with init and local blocks, emitted in ascending block order
+    // union with init and local blocks, emitted in ascending block order
     int32_t* out = a.block_idx + (size_t)pair * a.sel_cap;
     {
-        const int64_t per = (nb + NT - 1) / NT;
-        const int64_t lo = tid * per, hi = min(lo + per, nb);
+        const int per2 = (nb + NT - 1) / NT;
+        const int lo = tid * per2, hi = min(lo + per2, nb);
         int cnt = 0;
-        for (int64_t i = lo; i < hi; ++i)
-            cnt += (i < init_end || i >= local_begin || keys[i] != 0u);
+        for (int i = lo; i < hi; ++i) cnt += (i < init_end || i >= local_begin || keys[i] != 0u);
         int total;
         int pos = block_exclusive_scan(cnt, s_warp, &total);
-        for (int64_t i = lo; i < hi; ++i)
-            if (i < init_end || i >= local_begin || keys[i] != 0u) out[pos++] = (int32_t)i;
+        for (int i = lo; i < hi; ++i)
+            if (i < init_end || i >= local_begin || keys[i] != 0u) out[pos++] = i;
         for (int i = total + tid; i < a.sel_cap; i += NT) out[i] = -1;
         if (tid == 0) a.n_sel[pair] = total;
     }
 }
 
-// Merge the warps' (max, sum) per head, publish the slice statistics, and let the last CTA of the
-// pair run the selection.
-__device__ void finish_slice(const ScoreArgs& a, int pair, int item, int64_t T, int64_t nc, bool ok,
-                             float (*s_wm)[kMaxG], float (*s_ws)[kMaxG], uint32_t* keys) {
+// grid = pairs * parts. Part p of a pair scores windows [p*PW, p*PW + PW) and owns the blocks whose
+// first overlapping window falls in that range (the last part with windows also owns the blocks
+// past the last window, which score -inf).
+__global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a) {
+    extern __shared__ uint32_t s_dyn[];  // [key_words] keys, then [PW + W_max] window scores
+    __shared__ float sM[kMaxG], sInvZ[kMaxG];
     __shared__ int s_last;
-    __syncthreads();
-    if (threadIdx.x < a.G) {
-        float m = -INFINITY, s = 0.f;
-        for (int w = 0; w < kScoreWarps; ++w) online_merge(m, s, s_wm[w][threadIdx.x], s_ws[w][threadIdx.x]);
-        a.stats[((size_t)pair * a.items + item) * a.Gp + threadIdx.x] = make_float2(m, s);
+    const int pair = blockIdx.x / a.parts, part = blockIdx.x - pair * a.parts;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float* S = reinterpret_cast<float*>(s_dyn + a.key_words);
+    pdl_trigger();
+    pdl_wait();
+    const int64_t T = a.seq_lens[pair / a.Hkv];
+    const bool ok = T >= 0 && T <= a.T_cap;
+    const int64_t nc = ok ? num_windows(T, a.l, a.s) : 0;
+    const int64_t nb = ok ? (T + a.BS - 1) / a.BS : 0;
+    const int64_t parts_used = nc > 0 ? (nc + a.part_windows - 1) / a.part_windows : 1;
+    float* bs = a.bscores + (size_t)pair * a.nb_cap;
+
+    if (part < parts_used) {
+        // softmax normaliser of every head from the chunk statistics: one parallel round of
+        // loads into shared memory (aliasing the key array, unused until the top-k), then warp h
+        // merges head h
+        {
+            const int64_t nch = (nc + 63) / 64;
+            float2* s_st = reinterpret_cast<float2*>(s_dyn);  // 2 * nchunk * Gp <= key_words
+            const float2* st = a.stats + (size_t)pair * a.nchunk * a.Gp;
+            for (int64_t e = tid; e < nch * a.Gp; e += kSelectThreads) s_st[e] = ld_cg(st + e);
+            __syncthreads();
+            if (warp < a.G) {
+                float m = -INFINITY, s = 0.f;
+                for (int64_t c = lane; c < nch; c += 32) {
+                    const float2 v = s_st[c * a.Gp + warp];
+                    online_merge(m, s, v.x, v.y);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) {
+                    const float mo = __shfl_xor_sync(0xffffffffu, m, off);
+                    const float so = __shfl_xor_sync(0xffffffffu, s, off);
+                    online_merge(m, s, mo, so);
+                }
+                if (lane == 0) {
+                    sM[warp] = m;
+                    sInvZ[warp] = s > 0.f ? 1.f / s : 0.f;
+                }
+            }
+            __syncthreads();
+        }
+        const int64_t j0 = (int64_t)part * a.part_windows;
+        const int64_t j1 = min(j0 + a.part_windows, nc);
+        const int64_t b_lo = first_block_from(j0, a.BS, a.l, a.s);
+        const int64_t b_hi =
+            part == parts_used - 1 ? nb : min(first_block_from(j1, a.BS, a.l, a.s), nb);
+        const int64_t jend = b_hi > b_lo ? min(last_window(b_hi - 1, a.BS, a.s) + 1, nc) : j0;
+        if (jend > j0) {
+            const float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
+            switch (a.Gp) {
+                case 1: window_scores<1>(lg, j0, jend, a.G, sM, sInvZ, S); break;
+                case 2: window_scores<2>(lg, j0, jend, a.G, sM, sInvZ, S); break;
+                case 4: window_scores<4>(lg, j0, jend, a.G, sM, sInvZ, S); break;
+                default: window_scores<8>(lg, j0, jend, a.G, sM, sInvZ, S); break;
+            }
+        }
+        __syncthreads();
+        const int j0i = (int)j0, nci = (int)nc;
+        for (int b = (int)b_lo + tid; b < (int)b_hi; b += kSelectThreads) {
+            float best = -INFINITY;
+            const int jlo = (int)first_window32(b, a.BS, a.l, a.s);
+            const int jhi = min((int)last_window32(b, a.BS, a.s), nci - 1);
+            for (int j = jlo; j <= jhi; ++j) best = fmaxf(best, S[j - j0i]);
+            bs[b] = best;
+            if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + b] = best;
+        }
     }
+    if (part == 0 && a.block_scores)
+        for (int64_t b = nb + tid; b < a.nb_cap; b += kSelectThreads)
+            a.block_scores[(size_t)pair * a.nb_cap + b] = -INFINITY;
+
+    // the last part of the pair runs the top-k over all its block scores
     __threadfence();
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         const int prev = atomicAdd(a.cnt + pair, 1);
-        s_last = (prev == a.items - 1);
+        s_last = (prev == a.parts - 1);
         if (s_last) atomicExch(a.cnt + pair, 0);  // ready for the next launch
     }
     __syncthreads();
     if (!s_last) return;
     __threadfence();
-    select_pair(a, pair, T, nc, ok, keys);
+    for (int64_t b = tid; b < nb; b += kSelectThreads) s_dyn[b] = order_key(ld_cg(bs + b));
+    __syncthreads();
+    topk_union(a, pair, (int)nb, s_dyn);
 }
 
-__device__ __forceinline__ void seq_info(const ScoreArgs& a, int b, int pair, int item, int64_t& T,
-                                         int64_t& nc, bool& ok) {
-    T = a.seq_lens[b];
-    ok = T >= 0 && T <= a.T_cap;
-    if (!ok && item == 0 && threadIdx.x == 0 && pair % a.Hkv == 0)
-        atomicOr(a.err, (uint32_t)BSA_DEVERR_SEQ_LEN);
-    nc = (ok && T >= a.l) ? (T - a.l) / a.s + 1 : 0;
-}
-
-// ---------------------------------------------------------------------------------- bf16 path
-template <int D>
-struct KTile {
-    static constexpr int NI = D / 32;  // 16-byte chunks a lane holds per row (chunks tq + 4i)
-    uint4 a[NI], b[NI];                // rows r+g and r+g+8 of the tile
-};
-
-template <int D>
-__device__ __forceinline__ void load_ktile(KTile<D>& t, const uint16_t* ckp, int64_t r, int64_t r1,
-                                           int g, int tq) {
-    const int64_t ra = r + g, rb = r + g + 8;
-#pragma unroll
-    for (int i = 0; i < KTile<D>::NI; ++i) {
-        const int col = (tq + 4 * i) * 8;
-        t.a[i] = ra < r1 ? ld_stream(ckp + ra * D + col) : make_uint4(0, 0, 0, 0);
-        t.b[i] = rb < r1 ? ld_stream(ckp + rb * D + col) : make_uint4(0, 0, 0, 0);
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0)
+            n = 148;
+        cached[dev] = n;
     }
-}
-
-template <int D>
-__global__ void __launch_bounds__(kScoreThreads, 2) score_select_bf16_kernel(ScoreArgs a) {
-    extern __shared__ uint32_t s_keys[];
-    __shared__ float s_wm[kScoreWarps][kMaxG], s_ws[kScoreWarps][kMaxG];
-    constexpr int NI = D / 32;
-    const int pair = blockIdx.x / a.items, item = blockIdx.x - pair * a.items;
-    const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-
-    // q as the B operand: lane (g, tq) holds head g, chunks tq + 4i -- the same d positions its
-    // own key loads cover. q is never written by this library, so it is read before the wait.
-    uint32_t qf[NI][4];
-    {
-        const uint16_t* qh =
-            reinterpret_cast<const uint16_t*>(a.q) + ((size_t)b * a.Hq + (size_t)kvh * a.G + g) * D;
-#pragma unroll
-        for (int i = 0; i < NI; ++i) {
-            uint4 v = g < a.G ? *reinterpret_cast<const uint4*>(qh + (tq + 4 * i) * 8)
-                              : make_uint4(0, 0, 0, 0);
-            qf[i][0] = v.x;
-            qf[i][1] = v.y;
-            qf[i][2] = v.z;
-            qf[i][3] = v.w;
-        }
-    }
-    pdl_trigger();
-    pdl_wait();
-    int64_t T, nc;
-    bool ok;
-    seq_info(a, b, pair, item, T, nc, ok);
-
-    const int64_t r0 = ((int64_t)item * kScoreWarps + warp) * a.rows_per_warp;
-    const int64_t r1 = min(r0 + (int64_t)a.rows_per_warp, nc);
-    const uint16_t* ckp = reinterpret_cast<const uint16_t*>(a.ck) + (size_t)pair * a.nc_cap * D;
-    float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
-    const bool h0 = 2 * tq < a.G, h1 = 2 * tq + 1 < a.G;
-    float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
-
-    KTile<D> cur, nxt;
-    if (r0 < r1) load_ktile<D>(cur, ckp, r0, r1, g, tq);
-    for (int64_t r = r0; r < r1; r += 16) {
-        if (r + 16 < r1) load_ktile<D>(nxt, ckp, r + 16, r1, g, tq);
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < NI; ++i) {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                mma_bf16_16816(c, u4_get(cur.a[i], 2 * hh), u4_get(cur.b[i], 2 * hh),
-                               u4_get(cur.a[i], 2 * hh + 1), u4_get(cur.b[i], 2 * hh + 1),
-                               qf[i][2 * hh], qf[i][2 * hh + 1]);
-            }
-        }
-        const float x0 = c[0] * a.score_log2, x1 = c[1] * a.score_log2;
-        const float x2 = c[2] * a.score_log2, x3 = c[3] * a.score_log2;
-        const int64_t ra = r + g, rb = r + g + 8;
-        if (ra < r1) {
-            if (h1) *reinterpret_cast<float2*>(lg + ra * a.Gp + 2 * tq) = make_float2(x0, x1);
-            else if (h0) lg[ra * a.Gp + 2 * tq] = x0;
-            if (h0) online_add(m0, s0, x0);
-            if (h1) online_add(m1, s1, x1);
-        }
-        if (rb < r1) {
-            if (h1) *reinterpret_cast<float2*>(lg + rb * a.Gp + 2 * tq) = make_float2(x2, x3);
-            else if (h0) lg[rb * a.Gp + 2 * tq] = x2;
-            if (h0) online_add(m0, s0, x2);
-            if (h1) online_add(m1, s1, x3);
-        }
-        cur = nxt;
-    }
-    // combine the 8 row-groups (lanes with equal tq)
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        float mo = __shfl_xor_sync(0xffffffffu, m0, off), so = __shfl_xor_sync(0xffffffffu, s0, off);
-        online_merge(m0, s0, mo, so);
-        mo = __shfl_xor_sync(0xffffffffu, m1, off);
-        so = __shfl_xor_sync(0xffffffffu, s1, off);
-        online_merge(m1, s1, mo, so);
-    }
-    if (g == 0) {
-        if (h0) {
-            s_wm[warp][2 * tq] = m0;
-            s_ws[warp][2 * tq] = s0;
-        }
-        if (h1) {
-            s_wm[warp][2 * tq + 1] = m1;
-            s_ws[warp][2 * tq + 1] = s1;
-        }
-    }
-    finish_slice(a, pair, item, T, nc, ok, s_wm, s_ws, s_keys);
-}
-
-// ---------------------------------------------------------------------------------- fp32 path
-// Plain FMA dot products (fp32 inputs keep fp32 accuracy); one warp per row, lanes split d.
-template <int D>
-__global__ void __launch_bounds__(kScoreThreads, 2) score_select_f32_kernel(ScoreArgs a) {
-    extern __shared__ uint32_t s_keys[];
-    __shared__ float s_wm[kScoreWarps][kMaxG], s_ws[kScoreWarps][kMaxG];
-    constexpr int E = D / 32;
-    const int pair = blockIdx.x / a.items, item = blockIdx.x - pair * a.items;
-    const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-
-    float qv[kMaxG][E];
-    const float* qbase = reinterpret_cast<const float*>(a.q) + ((size_t)b * a.Hq + (size_t)kvh * a.G) * D;
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h)
-#pragma unroll
-        for (int e = 0; e < E; ++e) qv[h][e] = h < a.G ? qbase[h * D + lane * E + e] : 0.f;
-    pdl_trigger();
-    pdl_wait();
-    int64_t T, nc;
-    bool ok;
-    seq_info(a, b, pair, item, T, nc, ok);
-
-    const int64_t r0 = ((int64_t)item * kScoreWarps + warp) * a.rows_per_warp;
-    const int64_t r1 = min(r0 + (int64_t)a.rows_per_warp, nc);
-    const float* ckp = reinterpret_cast<const float*>(a.ck) + (size_t)pair * a.nc_cap * D;
-    float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
-    float m[kMaxG], s[kMaxG];
-#pragma unroll
-    for (int h = 0; h < kMaxG; ++h) {
-        m[h] = -INFINITY;
-        s[h] = 0.f;
-    }
-    for (int64_t r = r0; r < r1; ++r) {
-        float kv[E];
-#pragma unroll
-        for (int e = 0; e < E; ++e) kv[e] = __ldg(ckp + r * D + lane * E + e);
-#pragma unroll
-        for (int h = 0; h < kMaxG; ++h) {
-            if (h >= a.G) break;
-            float p = 0.f;
-#pragma unroll
-            for (int e = 0; e < E; ++e) p = fmaf(qv[h][e], kv[e], p);
-#pragma unroll
-            for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-            const float x = p * a.score_log2;
-            if (lane == h) lg[r * a.Gp + h] = x;
-            online_add(m[h], s[h], x);
-        }
-    }
-    if (lane == 0) {
-#pragma unroll
-        for (int h = 0; h < kMaxG; ++h) {
-            if (h < a.G) {
-                s_wm[warp][h] = m[h];
-                s_ws[warp][h] = s[h];
-            }
-        }
-    }
-    finish_slice(a, pair, item, T, nc, ok, s_wm, s_ws, s_keys);
+    return cached[dev];
 }
 
 template <typename K>
-cudaError_t launch_with_smem(K kernel, const Plan& p, const ScoreArgs& a, cudaStream_t st) {
-    if (p.score_smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)p.score_smem);
-        if (e != cudaSuccess) return e;
-    }
-    return launch_pdl(kernel, dim3((unsigned)(p.pairs * p.score_items)), dim3(kScoreThreads),
-                      p.score_smem, st, a);
+cudaError_t launch_score_k(K kernel, const ScoreArgs& a, cudaStream_t st) {
+    if (a.total_chunks == 0) return cudaSuccess;
+    int per_sm = 0;
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kScoreThreads, 0);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) per_sm = 1;
+    int64_t grid = (int64_t)per_sm * sm_count();
+    const int64_t need = (a.total_chunks + kScoreWarps - 1) / kScoreWarps;  // >= 1 chunk per warp
+    if (grid > need) grid = need;
+    return launch_pdl(kernel, dim3((unsigned)grid), dim3(kScoreThreads), 0, st, a);
 }
 
 }  // namespace
 
-cudaError_t launch_score_select(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
+cudaError_t launch_score(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
     if (p.dtype == BSA_BF16)
-        return p.D == 128 ? launch_with_smem(score_select_bf16_kernel<128>, p, a, st)
-                          : launch_with_smem(score_select_bf16_kernel<64>, p, a, st);
-    return p.D == 128 ? launch_with_smem(score_select_f32_kernel<128>, p, a, st)
-                      : launch_with_smem(score_select_f32_kernel<64>, p, a, st);
+        return p.D == 128 ? launch_score_k(score_bf16_kernel<128>, a, st)
+                          : launch_score_k(score_bf16_kernel<64>, a, st);
+    return p.D == 128 ? launch_score_k(score_f32_kernel<128>, a, st)
+                      : launch_score_k(score_f32_kernel<64>, a, st);
+}
+
+cudaError_t launch_select(const Plan& p, const SelectArgs& a, cudaStream_t st) {
+    if (p.select_smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)p.select_smem);
+        if (e != cudaSuccess) return e;
+    }
+    return launch_pdl(select_kernel, dim3((unsigned)(p.pairs * p.select_parts)),
+                      dim3(kSelectThreads), p.select_smem, st, a);
 }
 
 }  // namespace bsa

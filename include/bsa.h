@@ -83,7 +83,7 @@ typedef enum {
 
 /* Problem shape and method parameters. Supported: dtype fp32 or bf16; head_dim 64 or 128;
  * G = Hq / Hkv in 1..8; block_size a multiple of 16 in 16..256; cmp_kernel, cmp_stride >= 1;
- * n_init + n_local + top_k >= 1; NB_cap <= 32768; num_layers in 1..BSA_MAX_LAYERS. */
+ * 1 <= n_init + n_local + top_k <= 4096; NB_cap <= 32768; num_layers in 1..BSA_MAX_LAYERS. */
 typedef struct {
     int32_t batch;        /* B */
     int32_t num_q_heads;  /* Hq */

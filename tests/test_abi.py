@@ -73,6 +73,7 @@ def _p(**kw):
     (dict(cmp_stride=0), bsa.BSA_ERR_INVALID_ARG),
     (dict(n_init=0, n_local=0, top_k=0), bsa.BSA_ERR_INVALID_ARG),
     (dict(top_k=-1), bsa.BSA_ERR_INVALID_ARG),
+    (dict(top_k=5000), bsa.BSA_ERR_UNSUPPORTED),                       # SEL_cap > 4096
     (dict(max_seq_len=0), bsa.BSA_ERR_INVALID_ARG),
     (dict(max_seq_len=64 * 32768 + 1), bsa.BSA_ERR_UNSUPPORTED),       # nb_cap > 32768
     (dict(num_layers=0), bsa.BSA_ERR_INVALID_ARG),
