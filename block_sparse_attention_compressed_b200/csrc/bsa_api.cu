@@ -103,6 +103,20 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
         if (splits * P.Gp > kMaxCombineSlots) splits = kMaxCombineSlots / P.Gp;
         P.dec_splits = (int)splits;
         P.dec_bpc = (int)((P.sel_cap + splits - 1) / splits);
+        // bf16: C persistent CTAs, each an equal contiguous share of the layers * pairs * SEL_cap
+        // block slots; a (layer, pair) then spans at most ceil(SEL_cap / per_cta) + 1 CTAs
+        const int64_t slots_total = (int64_t)P.layers * P.pairs * P.sel_cap;
+        int64_t ctas = 2 * kNumSMs;
+        if (ctas > (slots_total + 1) / 2) ctas = (slots_total + 1) / 2;
+        if (ctas < 1) ctas = 1;
+        P.dec_ctas = (int)ctas;
+        const int64_t per_cta = slots_total / ctas > 0 ? slots_total / ctas : 1;
+        P.dec_slots = P.dtype == BSA_BF16 ? (int)((P.sel_cap + per_cta - 1) / per_cta + 2) : P.dec_splits;
+        if ((int64_t)P.dec_slots * P.Gp > kMaxCombineSlots) return BSA_ERR_UNSUPPORTED;
+        P.stage_tokens = P.BS % 64 == 0 ? 64 : (P.BS % 32 == 0 ? 32 : 16);
+        // TMA row coordinates are 32-bit: every cache row must be addressable
+        if (P.dtype == BSA_BF16 && (int64_t)P.pairs * P.T_cap > 0x7fffffffLL)
+            return BSA_ERR_UNSUPPORTED;
     }
     // Workspace
     size_t off = 0;
@@ -119,9 +133,9 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
     P.off_bscores = off;
     off = align_up(off + (size_t)P.pairs * P.nb_cap * sizeof(float));
     P.off_part_ml = off;
-    off = align_up(off + (size_t)P.layers * P.pairs * P.dec_splits * P.Gp * sizeof(float2));
+    off = align_up(off + (size_t)P.layers * P.pairs * P.dec_slots * P.Gp * sizeof(float2));
     P.off_part_acc = off;
-    off = align_up(off + (size_t)P.layers * P.pairs * P.dec_splits * P.Gp * P.D * sizeof(float));
+    off = align_up(off + (size_t)P.layers * P.pairs * P.dec_slots * P.Gp * P.D * sizeof(float));
     P.ws_bytes = off;
     return BSA_OK;
 }
@@ -231,8 +245,23 @@ DecodeArgs decode_args(const Plan& P, const int32_t* seq_lens, const int32_t* bl
     a.T_cap = P.T_cap;
     a.splits = P.dec_splits;
     a.bpc = P.dec_bpc;
+    a.slots = P.dec_slots;
+    a.ctas = P.dec_ctas;
+    a.stage_tokens = P.stage_tokens;
     a.scale_log2 = P.scale_log2;
     return a;
+}
+
+// TMA descriptors of the layers' caches (bf16 path only).
+bsa_status_t make_maps(const Plan& P, const DecodeArgs& a, int layers, KVMaps* maps) {
+    if (P.dtype != BSA_BF16) return BSA_OK;
+    const uint64_t rows = (uint64_t)P.pairs * (uint64_t)P.T_cap;
+    for (int i = 0; i < layers; ++i) {
+        if (!encode_kv_map(&maps->k[i], a.k[i], rows, P.D, P.stage_tokens) ||
+            !encode_kv_map(&maps->v[i], a.v[i], rows, P.D, P.stage_tokens))
+            return BSA_ERR_CUDA;
+    }
+    return BSA_OK;
 }
 
 bsa_status_t do_append(const Plan& P, void* k_cache, void* v_cache, const void* k_new,
@@ -384,7 +413,9 @@ bsa_status_t bsa_sparse_decode_layers(const bsa_params_t* params, int32_t num_la
         a.out[i] = outs[i];
         a.lse[i] = lse;
     }
-    return from_cuda(launch_decode(P, a, num_layers, stream));
+    static thread_local KVMaps maps;
+    if ((st = make_maps(P, a, num_layers, &maps)) != BSA_OK) return st;
+    return from_cuda(launch_decode(P, a, &maps, num_layers, stream));
 }
 
 bsa_status_t bsa_sparse_decode(const bsa_params_t* params, const void* q, const void* k_cache,
@@ -429,7 +460,9 @@ bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_
     da.v[0] = v_cache;
     da.out[0] = out;
     da.lse[0] = lse;
-    return from_cuda(launch_decode(P, da, 1, stream));
+    static thread_local KVMaps maps;
+    if ((st = make_maps(P, da, 1, &maps)) != BSA_OK) return st;
+    return from_cuda(launch_decode(P, da, &maps, 1, stream));
 }
 
 bsa_status_t bsa_read_device_error(void* ws, size_t ws_bytes, uint32_t* flags,

@@ -2,6 +2,7 @@
 // small PTX helpers for sm_100a. Nothing here is part of the C ABI (include/bsa.h is).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -35,6 +36,8 @@ struct Plan {
     size_t select_smem;  // dynamic shared memory of the selection kernel
     // decode: grid = layers * pairs * dec_splits CTAs of kDecodeWarps warps, dec_bpc blocks each
     int dec_splits, dec_bpc;
+    int dec_ctas, dec_slots;  // bf16: persistent CTAs; partial slots per (layer, pair)
+    int stage_tokens;  // bf16 decode pipeline stage: 64, 32 or 16 tokens (divides BS)
     // workspace layout (bytes)
     size_t off_err, off_sel_cnt, off_dec_cnt, off_logits, off_stats, off_bscores, off_part_ml,
         off_part_acc;
@@ -89,6 +92,13 @@ struct SelectArgs {
     int parts, part_windows;
 };
 
+// TMA descriptors of the K and V caches of every layer (bf16 path): 2-D views
+// [B*Hkv*T_cap rows][D columns], boxes of 64 columns x stage_tokens rows, 128-byte swizzle.
+struct alignas(64) KVMaps {
+    CUtensorMap k[BSA_MAX_LAYERS];
+    CUtensorMap v[BSA_MAX_LAYERS];
+};
+
 struct DecodeArgs {
     const void* q[BSA_MAX_LAYERS];
     const void* k[BSA_MAX_LAYERS];
@@ -104,7 +114,10 @@ struct DecodeArgs {
     float* part_acc;    // [layers * pairs][splits][Gp][D] unnormalised numerators
     int Hq, Hkv, G, Gp, BS, sel_cap, pairs;
     int64_t T_cap;
-    int splits, bpc;
+    int splits, bpc;   // fp32 path: CTA = (layer, pair, split) of bpc blocks
+    int slots;         // partial slots per (layer, pair) in the workspace
+    int ctas;          // bf16 path: persistent CTAs sharing the (layer, pair, block) slots evenly
+    int stage_tokens;  // tokens per pipeline stage (bf16 path): 64, 32 or 16, dividing BS
     float scale_log2;
 };
 
@@ -113,7 +126,10 @@ cudaError_t launch_compress_keys(const Plan& p, const CompressArgs& a, cudaStrea
 cudaError_t launch_append(const Plan& p, const AppendArgs& a, cudaStream_t st);
 cudaError_t launch_score(const Plan& p, const ScoreArgs& a, cudaStream_t st);
 cudaError_t launch_select(const Plan& p, const SelectArgs& a, cudaStream_t st);
-cudaError_t launch_decode(const Plan& p, const DecodeArgs& a, int layers, cudaStream_t st);
+cudaError_t launch_decode(const Plan& p, const DecodeArgs& a, const KVMaps* maps, int layers,
+                          cudaStream_t st);
+// Encode a 2-D bf16 TMA descriptor over rows x D elements (128-byte swizzle, box 64 x box_rows).
+bool encode_kv_map(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows);
 
 // Launch with programmatic dependent launch allowed: the kernel may start while the previous
 // kernel in the stream drains; every kernel here waits (griddepcontrol.wait) before touching
@@ -211,6 +227,69 @@ __device__ __forceinline__ void online_merge(float& m, float& s, float m2, float
     }
     s = s * exp2f(m - mn) + s2 * exp2f(m2 - mn);
     m = mn;
+}
+
+// ---- shared-memory barriers and TMA (sm_90+ instructions, used on sm_100a)
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_fence_init() {
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+// Wait for the phase with the given parity to complete; gives up after `limit` polls (returns
+// false) so that no wait can run forever.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint32_t limit) {
+    for (uint32_t it = 0; it < limit; ++it) {
+        uint32_t done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            " selp.u32 %0, 1, 0, p;\n}\n"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+// 2-D tiled TMA load of one box into shared memory, completing on `bar` (transaction bytes).
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, int x, int y,
+                                            uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(map), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+// 1-D bulk copy global -> shared (16-byte aligned addresses, size a multiple of 16).
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void ldmatrix_x4(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t addr) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                 : "r"(addr));
 }
 
 // Order-preserving map of an fp32 score onto uint32 (larger float -> larger key).

@@ -5,19 +5,21 @@
 // Sparse Attention" (second abstract): several layers attended with one layer's selection.
 //
 // Split-KV flash decoding. grid = layers * pairs * splits CTAs; CTA `split` of a (layer, pair)
-// owns blocks [split*bpc, (split+1)*bpc) of the pair's selection, its warps take those blocks
-// round-robin and run an online softmax (fp32, exp2 domain) over 16-token sub-tiles. The warps'
-// partial states are merged in shared memory and written to the workspace; the last CTA of the
-// (layer, pair) to finish (completion counter, no waiting) combines all splits into O and LSE.
+// owns blocks [split*bpc, (split+1)*bpc) of the pair's selection. The warps' partial softmax
+// states (fp32, exp2 domain) are merged in shared memory and written to the workspace; the last CTA
+// of the (layer, pair) to finish (completion counter, no waiting) combines all splits into O, LSE.
 //
-// bf16 path, per 16-token sub-tile, all on the tensor cores with mma.m16n8k16:
-//   S^T[tok][head] = K_tile[tok][:] . q^T   (tokens are M, the G heads padded to 8 are N); each
-//       lane feeds the A operand from its own 16-byte global loads, q permuted to match;
-//   O^T[d][head] += V_tile^T[d][tok] . P^T[tok][head]   (d is M, tokens are K): the V operand is
-//       built from two token rows per register with PRMT, P^T comes from the S^T accumulators via
-//       movmatrix.trans. P is split as P_hi + P_lo (both bf16) so that the products keep ~16
-//       significant bits of the fp32 probabilities.
-// K and V rows at or past the sequence length are never loaded (zero fill) and masked to -inf.
+// bf16 path (TMA pipeline): one producer warp walks the CTA's selected blocks and issues 2-D TMA
+// tensor copies (128-byte swizzle) of each 16..64-token stage of K and V into a ring of shared-
+// memory stages, completing on per-stage mbarriers; four consumer warps each take 16 tokens of a
+// stage and run, on the tensor cores (mma.m16n8k16, operands from ldmatrix):
+//   S^T[tok][head] = K[tok][:] . q^T          (tokens are M, the G heads padded to 8 are N)
+//   O^T[d][head] += V^T[d][tok] . P^T[tok][head]  (d is M; V^T via ldmatrix.trans; P^T from the
+//       S^T accumulators via movmatrix.trans, split as bf16 hi + lo so the products keep ~16
+//       significant bits of the fp32 probabilities)
+// then release the stage. Bytes in flight are set by the ring size, not by registers. Tokens at or
+// past the sequence length are masked to -inf and their V rows zeroed in shared memory.
+// fp32 path: one token at a time per warp, FMA dot products and warp reductions.
 #include "bsa_internal.cuh"
 
 namespace bsa {
@@ -25,13 +27,18 @@ namespace {
 
 constexpr int kDecodeThreads = kDecodeWarps * 32;
 
-// Shared-memory image of the warps' states, merged by the whole CTA.
-template <int D>
-struct DecodeSmem {
-    float m[kDecodeWarps][kMaxG];
-    float l[kDecodeWarps][kMaxG];
-    float acc[kDecodeWarps][kMaxG][D];
+// Shared-memory image of the warps' states: m and l per (warp, head), numerators per
+// (warp, head, d) packed for the problem's G heads.
+struct MergeView {
+    float* m;    // [kDecodeWarps][kMaxG]
+    float* l;    // [kDecodeWarps][kMaxG]
+    float* acc;  // [kDecodeWarps][G][D]
+    __device__ __forceinline__ float& M(int w, int h) const { return m[w * kMaxG + h]; }
+    __device__ __forceinline__ float& L(int w, int h) const { return l[w * kMaxG + h]; }
 };
+__host__ __device__ constexpr size_t merge_bytes(int G, int D) {
+    return sizeof(float) * (2 * kDecodeWarps * kMaxG + (size_t)kDecodeWarps * G * D);
+}
 
 template <typename T>
 __device__ __forceinline__ void store_out(T* p, float v);
@@ -42,54 +49,64 @@ __device__ __forceinline__ void store_out<__nv_bfloat16>(__nv_bfloat16* p, float
     *p = __float2bfloat16_rn(v);
 }
 
-// CTA merge of the warp states, split partial write, and the cross-split combine by the last CTA.
+// The threads that merge a split: the whole CTA (bar_id 0, __syncthreads) or a named-barrier
+// group of `nthreads` threads (the consumer warps of the persistent kernel).
+struct Group {
+    int tid, nthreads, bar_id;
+    __device__ __forceinline__ void sync() const {
+        if (bar_id == 0) __syncthreads();
+        else asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "r"(nthreads) : "memory");
+    }
+};
+
+// Merge of the warp states, split partial write, and the cross-split combine by the last split of
+// the (layer, pair) to finish.
 template <typename T, int D>
-__device__ void finish_split(const DecodeArgs& a, int layer, int pair, int lp, int split,
-                             DecodeSmem<D>& sm) {
+__device__ void finish_split(const DecodeArgs& a, int layer, int pair, int lp, int slot, int nslots,
+                             const MergeView sm, float2* s_ml /* nslots * Gp */, const Group gp) {
     __shared__ int s_last;
-    __syncthreads();
-    const int G = a.G, NT = blockDim.x;
-    float2* pml = a.part_ml + ((size_t)lp * a.splits + split) * a.Gp;
-    float* pacc = a.part_acc + ((size_t)lp * a.splits + split) * a.Gp * D;
-    for (int e = threadIdx.x; e < G * D; e += NT) {
+    gp.sync();
+    const int G = a.G, NT = gp.nthreads;
+    float2* pml = a.part_ml + ((size_t)lp * a.slots + slot) * a.Gp;
+    float* pacc = a.part_acc + ((size_t)lp * a.slots + slot) * a.Gp * D;
+    for (int e = gp.tid; e < G * D; e += NT) {
         const int h = e / D, dd = e - h * D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, sm.m[w][h]);
+        for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, sm.M(w, h));
         float num = 0.f, den = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < kDecodeWarps; ++w) {
-                const float f = exp2f(sm.m[w][h] - M);
-                num = fmaf(f, sm.acc[w][h][dd], num);
-                den = fmaf(f, sm.l[w][h], den);
+                const float f = exp2f(sm.M(w, h) - M);
+                num = fmaf(f, sm.acc[(w * G + h) * D + dd], num);
+                den = fmaf(f, sm.L(w, h), den);
             }
         }
         pacc[h * D + dd] = num;
         if (dd == 0) pml[h] = make_float2(M, den);
     }
     __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
+    gp.sync();
+    if (gp.tid == 0) {
         const int prev = atomicAdd(a.cnt + lp, 1);
-        s_last = (prev == a.splits - 1);
+        s_last = (prev == nslots - 1);
         if (s_last) atomicExch(a.cnt + lp, 0);
     }
-    __syncthreads();
+    gp.sync();
     if (!s_last) return;
     __threadfence();
     // Combine the splits: per head the global max M and denominator, per split a scale factor
     // exp2(m_s - M) (shared memory), then every (head, d) element sums its scaled numerators with
     // the loads of kU splits in flight.
-    __shared__ float2 s_ml[kMaxCombineSlots];
     __shared__ float s_M[kMaxG], s_den[kMaxG];
-    const int S = a.splits;
-    const float2* ml0 = a.part_ml + (size_t)lp * S * a.Gp;
-    const float* acc0 = a.part_acc + (size_t)lp * S * a.Gp * D;
-    for (int e = threadIdx.x; e < S * a.Gp; e += NT) s_ml[e] = ld_cg(ml0 + e);  // one round
-    __syncthreads();
-    if (threadIdx.x < G) {
-        const int h = threadIdx.x;
+    const int S = nslots;
+    const float2* ml0 = a.part_ml + (size_t)lp * a.slots * a.Gp;
+    const float* acc0 = a.part_acc + (size_t)lp * a.slots * a.Gp * D;
+    for (int e = gp.tid; e < S * a.Gp; e += NT) s_ml[e] = ld_cg(ml0 + e);  // one round
+    gp.sync();
+    if (gp.tid < G) {
+        const int h = gp.tid;
         float M = -INFINITY;
         for (int s2 = 0; s2 < S; ++s2) M = fmaxf(M, s_ml[s2 * a.Gp + h].x);
         float den = 0.f;
@@ -102,12 +119,12 @@ __device__ void finish_split(const DecodeArgs& a, int layer, int pair, int lp, i
         s_M[h] = M;
         s_den[h] = den;
     }
-    __syncthreads();
+    gp.sync();
     const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
     T* out = reinterpret_cast<T*>(a.out[layer]) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
     float* lse = a.lse[layer] ? a.lse[layer] + (size_t)b * a.Hq + (size_t)kvh * G : nullptr;
     constexpr int kU = 8;
-    for (int e = threadIdx.x; e < G * D; e += NT) {
+    for (int e = gp.tid; e < G * D; e += NT) {
         const int h = e / D, dd = e - h * D;
         float num = 0.f;
         for (int s0 = 0; s0 < S; s0 += kU) {
@@ -129,16 +146,19 @@ __device__ void finish_split(const DecodeArgs& a, int layer, int pair, int lp, i
 // Which blocks this CTA owns, and the sequence facts every warp needs.
 struct SplitInfo {
     int64_t T, nb;
-    int beg, end;
+    int ns;        // selected blocks of the pair (clamped to [0, SEL_cap]; 0 for a bad length)
+    int beg, end;  // this split's blocks [beg, end) (fp32 path)
     bool ok;
 };
 
-__device__ __forceinline__ SplitInfo split_info(const DecodeArgs& a, int layer, int pair, int split) {
+// `lead` is true for exactly one thread of the CTA that handles the split (it reports errors).
+__device__ __forceinline__ SplitInfo split_info(const DecodeArgs& a, int layer, int pair, int split,
+                                                bool lead) {
     SplitInfo si;
     const int b = pair / a.Hkv;
     si.T = a.seq_lens[b];
     si.ok = si.T >= 0 && si.T <= a.T_cap;
-    const bool reporter = layer == 0 && split == 0 && threadIdx.x == 0;
+    const bool reporter = layer == 0 && split == 0 && lead;
     if (!si.ok && reporter && pair % a.Hkv == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_SEQ_LEN);
     int ns = a.n_sel[pair];
     if (ns < 0 || ns > a.sel_cap) {
@@ -146,6 +166,7 @@ __device__ __forceinline__ SplitInfo split_info(const DecodeArgs& a, int layer, 
         ns = ns < 0 ? 0 : a.sel_cap;
     }
     if (!si.ok) ns = 0;
+    si.ns = ns;
     si.nb = si.ok ? (si.T + a.BS - 1) / a.BS : 0;
     si.beg = split * a.bpc;
     si.end = min(si.beg + a.bpc, ns);
@@ -153,205 +174,315 @@ __device__ __forceinline__ SplitInfo split_info(const DecodeArgs& a, int layer, 
 }
 
 // -------------------------------------------------------------------------------------- bf16 path
-template <int D>
-struct KVTile {
-    static constexpr int NI = D / 32;   // key chunks per lane per row (chunks tq + 4i)
-    static constexpr int NCV = D / 64;  // value chunks per lane per token (chunks g, g + 8)
-    uint4 ka[NI], kb[NI];               // key rows base+g, base+g+8
-    uint4 v[4][NCV];                    // value rows base+2tq, +2tq+1, +2tq+8, +2tq+9
+constexpr int kConsumerWarps = 4;
+constexpr int kTmaThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
+constexpr int kMaxStages = 8;
+constexpr uint32_t kWaitPolls = 1u << 26;  // far beyond any legitimate wait; then give up
+constexpr uint32_t kQSlot = 1024;          // bytes per stage for q of the group (G * D * 2 <= 2048)
+
+enum : int { kStageFirst = 1, kStageLast = 2, kStageEnd = 4 };
+
+struct StageMeta {
+    int tok0;    // first token of the stage within the sequence
+    int nvalid;  // tokens of the stage below the sequence length (0: flush-only stage)
+    int lp;      // layer * pairs + pair
+    int seg;     // this CTA's segment of the (layer, pair): partial slot
+    int nseg;    // segments (CTAs) the (layer, pair) spans
+    int flags;   // kStageFirst: q of this pair is in the stage; kStageLast: segment ends; kStageEnd
 };
 
-template <int D>
-__device__ __forceinline__ void load_kvtile(KVTile<D>& t, const uint16_t* kp, const uint16_t* vp,
-                                            int64_t base, int64_t T, int g, int tq) {
-    const int64_t ra = base + g, rb = base + g + 8;
-#pragma unroll
-    for (int i = 0; i < KVTile<D>::NI; ++i) {
-        const int col = (tq + 4 * i) * 8;
-        t.ka[i] = ra < T ? ld_stream(kp + ra * D + col) : make_uint4(0, 0, 0, 0);
-        t.kb[i] = rb < T ? ld_stream(kp + rb * D + col) : make_uint4(0, 0, 0, 0);
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int64_t row = base + 2 * tq + (r & 1) + (r >> 1) * 8;
-#pragma unroll
-        for (int i = 0; i < KVTile<D>::NCV; ++i) {
-            const int col = (g + 8 * i) * 8;
-            t.v[r][i] = row < T ? ld_stream(vp + row * D + col) : make_uint4(0, 0, 0, 0);
-        }
-    }
+// CTA (of C) whose share [c*N/C, (c+1)*N/C) of the N block slots holds slot x.
+__device__ __forceinline__ int cta_of_slot(int64_t x, int64_t N, int C) {
+    return (int)(((x + 1) * C + N - 1) / N - 1);
 }
 
+// Persistent: the N = layers * pairs * SEL_cap block slots are shared evenly by C CTAs; CTA c walks
+// slots [c*N/C, (c+1)*N/C). The producer lane streams every stage of its slots through the ring
+// without draining; where its range crosses from one (layer, pair) to the next, the consumer warps
+// flush the segment (merge, partial, and the combine when it is the pair's last segment) behind a
+// named barrier while the next stages are already loading.
 template <int D>
-__device__ __forceinline__ void attend_tile(const KVTile<D>& t, const uint32_t (&qf)[D / 32][4],
-                                            int64_t base, int64_t T, float sl, int g, float (&m)[2],
-                                            float (&lsum)[2], float (&acc)[D / 16][4]) {
-    constexpr int NI = D / 32, MT = D / 16;
-    float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int i = 0; i < NI; ++i)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-            mma_bf16_16816(c, u4_get(t.ka[i], 2 * hh), u4_get(t.kb[i], 2 * hh),
-                           u4_get(t.ka[i], 2 * hh + 1), u4_get(t.kb[i], 2 * hh + 1),
-                           qf[i][2 * hh], qf[i][2 * hh + 1]);
-    const bool va = base + g < T, vb = base + g + 8 < T;
-    const float x0 = va ? c[0] * sl : -INFINITY, x1 = va ? c[1] * sl : -INFINITY;
-    const float x2 = vb ? c[2] * sl : -INFINITY, x3 = vb ? c[3] * sl : -INFINITY;
-    float t0 = fmaxf(x0, x2), t1 = fmaxf(x1, x3);
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, off));
-        t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, off));
-    }
-    const float mn0 = fmaxf(m[0], t0), mn1 = fmaxf(m[1], t1);
-    const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m[0] - mn0);
-    const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m[1] - mn1);
-    const float ref0 = mn0 == -INFINITY ? 0.f : mn0, ref1 = mn1 == -INFINITY ? 0.f : mn1;
-    const float p0 = exp2f(x0 - ref0), p2 = exp2f(x2 - ref0);
-    const float p1 = exp2f(x1 - ref1), p3 = exp2f(x3 - ref1);
-    m[0] = mn0;
-    m[1] = mn1;
-    lsum[0] = lsum[0] * al0 + (p0 + p2);
-    lsum[1] = lsum[1] * al1 + (p1 + p3);
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        acc[mt][0] *= al0;
-        acc[mt][1] *= al1;
-        acc[mt][2] *= al0;
-        acc[mt][3] *= al1;
-    }
-    // P^T operand: rows of the S^T accumulator are tokens, columns heads; transpose 8x8 pieces
-    const uint32_t hi0 = pack_bf16x2(p0, p1), hi1 = pack_bf16x2(p2, p3);
-    const uint32_t lo0 = pack_bf16x2(p0 - bf16_lo(hi0), p1 - bf16_hi(hi0));
-    const uint32_t lo1 = pack_bf16x2(p2 - bf16_lo(hi1), p3 - bf16_hi(hi1));
-    const uint32_t bh0 = movmatrix_trans(hi0), bh1 = movmatrix_trans(hi1);
-    const uint32_t bl0 = movmatrix_trans(lo0), bl1 = movmatrix_trans(lo1);
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        const int ci = mt / 4, comp = mt % 4;
-        const uint32_t r0 = u4_get(t.v[0][ci], comp), r1 = u4_get(t.v[1][ci], comp);
-        const uint32_t r2 = u4_get(t.v[2][ci], comp), r3 = u4_get(t.v[3][ci], comp);
-        const uint32_t a0 = prmt(r0, r1, 0x5410u), a1 = prmt(r0, r1, 0x7632u);
-        const uint32_t a2 = prmt(r2, r3, 0x5410u), a3 = prmt(r2, r3, 0x7632u);
-        mma_bf16_16816(acc[mt], a0, a1, a2, a3, bh0, bh1);
-        mma_bf16_16816(acc[mt], a0, a1, a2, a3, bl0, bl1);
-    }
-}
+__global__ void __launch_bounds__(kTmaThreads, 2)
+    decode_tma_kernel(const DecodeArgs a, const __grid_constant__ KVMaps maps, const int nstages,
+                      const int64_t n_slots) {
+    extern __shared__ uint8_t dsm_raw[];
+    __shared__ __align__(8) uint64_t full[kMaxStages], empty[kMaxStages];
+    __shared__ StageMeta meta[kMaxStages];
+    constexpr int NB = D / 64;     // 64-column boxes per row
+    constexpr int KS = D / 16;     // k-steps of S^T = K q^T
+    constexpr int MT = D / 16;     // m-tiles of O^T
+    const int ST = a.stage_tokens;
+    const uint32_t box_bytes = (uint32_t)ST * 128u;
+    const uint32_t kv_bytes = 2u * NB * box_bytes;
+    const uint32_t stage_bytes = kv_bytes + kQSlot * ((a.G * D * 2 + kQSlot - 1) / kQSlot);
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    float* mbase = reinterpret_cast<float*>(ring + (size_t)nstages * stage_bytes);
+    const MergeView sm{mbase, mbase + kDecodeWarps * kMaxG, mbase + 2 * kDecodeWarps * kMaxG};
+    float2* s_ml = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(mbase) + merge_bytes(a.G, D));
 
-template <int D>
-__global__ void __launch_bounds__(kDecodeThreads, 2) decode_bf16_kernel(DecodeArgs a) {
-    __shared__ DecodeSmem<D> sm;
-    constexpr int NI = D / 32, MT = D / 16;
-    const int split = blockIdx.x % a.splits, lp = blockIdx.x / a.splits;
-    const int layer = lp / a.pairs, pair = lp - layer * a.pairs;
-    const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const bool producer = warp == kConsumerWarps;
+    const int C = (int)gridDim.x;
+    const int64_t x_lo = (int64_t)blockIdx.x * n_slots / C, x_hi = (int64_t)(blockIdx.x + 1) * n_slots / C;
 
-    uint32_t qf[NI][4];
-    {
-        const uint16_t* qh = reinterpret_cast<const uint16_t*>(a.q[layer]) +
-                             ((size_t)b * a.Hq + (size_t)kvh * a.G + g) * D;
-#pragma unroll
-        for (int i = 0; i < NI; ++i) {
-            uint4 v = g < a.G ? *reinterpret_cast<const uint4*>(qh + (tq + 4 * i) * 8)
-                              : make_uint4(0, 0, 0, 0);
-            qf[i][0] = v.x;
-            qf[i][1] = v.y;
-            qf[i][2] = v.z;
-            qf[i][3] = v.w;
+    if (threadIdx.x == 0) {
+        for (int s2 = 0; s2 < nstages; ++s2) {
+            mbar_init(&full[s2], 1);
+            mbar_init(&empty[s2], kConsumerWarps);
         }
+        mbar_fence_init();
     }
+    __syncthreads();
     pdl_trigger();
     pdl_wait();
-    const SplitInfo si = split_info(a, layer, pair, split);
-    const uint16_t* kp = reinterpret_cast<const uint16_t*>(a.k[layer]) + (size_t)pair * a.T_cap * D;
-    const uint16_t* vp = reinterpret_cast<const uint16_t*>(a.v[layer]) + (size_t)pair * a.T_cap * D;
-    const int32_t* ip = a.block_idx + (size_t)pair * a.sel_cap;
 
-    float m[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
-    float acc[MT][4];
+    if (producer) {
+        if (lane == 0) {
+            const int sub_per_block = a.BS / ST;
+            int k = 0;
+            bool ok = true;
+            // claims ring slot k (waiting for the consumers to release it)
+            auto claim = [&](int kk) -> int {
+                const int st = kk % nstages;
+                if (kk >= nstages && !mbar_wait(&empty[st], ((kk / nstages) - 1) & 1, kWaitPolls)) {
+                    atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                    ok = false;
+                }
+                return st;
+            };
+            int q_lp = -1;  // (layer, pair) whose q the consumers hold
+            for (int64_t x = x_lo; x < x_hi && ok;) {
+                const int lp = (int)(x / a.sel_cap);
+                const int64_t seg_end = min((int64_t)(lp + 1) * a.sel_cap, x_hi);
+                const int layer = lp / a.pairs, pair = lp - layer * a.pairs;
+                const int c_first = cta_of_slot((int64_t)lp * a.sel_cap, n_slots, C);
+                const int c_last = cta_of_slot((int64_t)(lp + 1) * a.sel_cap - 1, n_slots, C);
+                const int seg = (int)blockIdx.x - c_first, nseg = c_last - c_first + 1;
+                // blocks [i_lo, i_hi) of the pair's selection fall in this CTA's share
+                SplitInfo si = split_info(a, layer, pair, 0, seg == 0);
+                const int i_lo = (int)(x - (int64_t)lp * a.sel_cap);
+                const int i_hi = min((int)(seg_end - (int64_t)lp * a.sel_cap), si.ns);
+                x = seg_end;
+                const int64_t row_base = (int64_t)pair * a.T_cap;
+                const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
+                const uint8_t* qsrc = reinterpret_cast<const uint8_t*>(a.q[layer]) +
+                                      ((size_t)b * a.Hq + (size_t)kvh * a.G) * D * 2;
+                bool first = lp != q_lp;
+                int issued = 0;
+                const int32_t* ip = a.block_idx + (size_t)pair * a.sel_cap;
+                for (int i = i_lo; i < i_hi && ok; ++i) {
+                    const int blk = ip[i];
+                    if (blk < 0) continue;
+                    if (blk >= si.nb) {
+                        atomicOr(a.err, (uint32_t)BSA_DEVERR_BLOCK_IDX);
+                        continue;
+                    }
+                    for (int sub = 0; sub < sub_per_block && ok; ++sub) {
+                        const int64_t tok0 = (int64_t)blk * a.BS + (int64_t)sub * ST;
+                        if (tok0 >= si.T) break;
+                        const int st = claim(k);
+                        if (!ok) break;
+                        // is this the segment's last stage? (look ahead for another valid stage)
+                        bool more = tok0 + ST < si.T && sub + 1 < sub_per_block;
+                        for (int i2 = i + 1; i2 < i_hi && !more; ++i2) {
+                            const int b2 = ip[i2];
+                            more = b2 >= 0 && b2 < si.nb;
+                        }
+                        meta[st].tok0 = (int)tok0;
+                        meta[st].nvalid = (int)min((int64_t)ST, si.T - tok0);
+                        meta[st].lp = lp;
+                        meta[st].seg = seg;
+                        meta[st].nseg = nseg;
+                        meta[st].flags = (first ? kStageFirst : 0) | (more ? 0 : kStageLast);
+                        uint8_t* dst = ring + (size_t)st * stage_bytes;
+                        const uint32_t qb = first ? (uint32_t)(a.G * D * 2) : 0u;
+                        mbar_arrive_expect_tx(&full[st], kv_bytes + qb);
+                        const int y = (int)(row_base + tok0);
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
-
-    // The warp's work: its blocks (round-robin within the split) x 16-token sub-tiles, walked
-    // with the next sub-tile's loads in flight while the current one is computed.
-    const int sub_per_block = a.BS / 16;
-    int my_blk = -1;  // lane j holds the warp's j-th block index
-    {
-        const int i = si.beg + warp + lane * kDecodeWarps;
-        if (lane * kDecodeWarps + warp < a.bpc && i < si.end) {
-            const int v = ip[i];
-            if (v >= 0 && v < si.nb) my_blk = v;
-            else if (v >= si.nb) atomicOr(a.err, (uint32_t)BSA_DEVERR_BLOCK_IDX);
-        }
-    }
-    const int n_units = ((a.bpc + kDecodeWarps - 1) / kDecodeWarps) * sub_per_block;
-    auto unit_base = [&](int u) -> int64_t {  // token base of a unit, or -1 when it has no token
-        const int blk = __shfl_sync(0xffffffffu, my_blk, u / sub_per_block);
-        if (blk < 0) return -1;
-        const int64_t base = (int64_t)blk * a.BS + (u % sub_per_block) * 16;
-        return base < si.T ? base : -1;
-    };
-    auto next_unit = [&](int u, int64_t& base) -> int {
-        for (++u; u < n_units; ++u) {
-            base = unit_base(u);
-            if (base >= 0) return u;
-        }
-        return n_units;
-    };
-    // Two tile buffers in ping-pong (no register copy waits on a pending load).
-    KVTile<D> ta, tb;
-    int64_t base_a = -1, base_b = -1;
-    int ua = next_unit(-1, base_a);
-    if (ua < n_units) load_kvtile<D>(ta, kp, vp, base_a, si.T, g, tq);
-    while (ua < n_units) {
-        const int ub = next_unit(ua, base_b);
-        if (ub < n_units) load_kvtile<D>(tb, kp, vp, base_b, si.T, g, tq);
-        attend_tile<D>(ta, qf, base_a, si.T, a.scale_log2, g, m, lsum, acc);
-        if (ub >= n_units) break;
-        ua = next_unit(ub, base_a);
-        if (ua < n_units) load_kvtile<D>(ta, kp, vp, base_a, si.T, g, tq);
-        attend_tile<D>(tb, qf, base_b, si.T, a.scale_log2, g, m, lsum, acc);
-    }
-
+                        for (int bi = 0; bi < NB; ++bi)
+                            tma_load_2d(dst + bi * box_bytes, &maps.k[layer], 64 * bi, y, &full[st]);
 #pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], off);
-        lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], off);
-    }
-    const int h0 = 2 * tq, h1 = 2 * tq + 1;
-    if (g == 0) {
-        if (h0 < a.G) {
-            sm.m[warp][h0] = m[0];
-            sm.l[warp][h0] = lsum[0];
+                        for (int bi = 0; bi < NB; ++bi)
+                            tma_load_2d(dst + (NB + bi) * box_bytes, &maps.v[layer], 64 * bi, y, &full[st]);
+                        if (first) {
+                            bulk_load(dst + kv_bytes, qsrc, qb, &full[st]);
+                            q_lp = lp;
+                        }
+                        first = false;
+                        ++issued;
+                        ++k;
+                    }
+                }
+                if (ok && issued == 0) {
+                    // nothing to attend: a flush-only stage so the consumers publish an empty part
+                    const int st = claim(k);
+                    if (!ok) break;
+                    meta[st].tok0 = 0;
+                    meta[st].nvalid = 0;
+                    meta[st].lp = lp;
+                    meta[st].seg = seg;
+                    meta[st].nseg = nseg;
+                    meta[st].flags = kStageLast;
+                    mbar_arrive(&full[st]);
+                    ++k;
+                }
+            }
+            if (ok) {
+                const int st = claim(k);
+                if (ok) {
+                    meta[st].flags = kStageEnd;
+                    mbar_arrive(&full[st]);
+                }
+            }
         }
-        if (h1 < a.G) {
-            sm.m[warp][h1] = m[1];
-            sm.l[warp][h1] = lsum[1];
-        }
-    }
-    // accumulator (mt, row g / g+8) <-> d = (mt/4)*64 + 8g + 2(mt%4) + {0, 1}
+    } else {
+        const int r0 = 16 * warp;
+        const int mi = lane >> 3, ri = lane & 7;
+        const Group gp{(int)threadIdx.x, kConsumerWarps * 32, 1};
+        uint32_t qf[KS][2];
+        float m[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
+        float acc[MT][4];
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        const int d0 = (mt / 4) * 64 + 8 * g + 2 * (mt % 4);
-        if (h0 < a.G) {
-            sm.acc[warp][h0][d0] = acc[mt][0];
-            sm.acc[warp][h0][d0 + 1] = acc[mt][2];
-        }
-        if (h1 < a.G) {
-            sm.acc[warp][h1][d0] = acc[mt][1];
-            sm.acc[warp][h1][d0 + 1] = acc[mt][3];
+        for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        for (int k = 0;; ++k) {
+            const int st = k % nstages;
+            if (!mbar_wait(&full[st], (k / nstages) & 1, kWaitPolls)) {
+                if (lane == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                break;
+            }
+            const StageMeta md = meta[st];
+            if (md.flags & kStageEnd) break;
+            uint8_t* kst = ring + (size_t)st * stage_bytes;
+            uint8_t* vst = kst + NB * box_bytes;
+            if (md.flags & kStageFirst) {
+                // q as the B operand: lane (g, tq) holds head g, d = 16ks + 2tq (+1, +8, +9)
+                const uint32_t* qs = reinterpret_cast<const uint32_t*>(kst + kv_bytes) + g * (D / 2);
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    qf[ks][0] = g < a.G ? qs[8 * ks + tq] : 0u;
+                    qf[ks][1] = g < a.G ? qs[8 * ks + 4 + tq] : 0u;
+                }
+            }
+            if (r0 < md.nvalid) {
+                if (r0 + 16 > md.nvalid) {
+                    // rows past the sequence may hold anything: zero this warp's V rows there
+                    for (int e = lane; e < 16 * NB * 8; e += 32) {
+                        const int row = r0 + e / (NB * 8), bi = (e / 8) % NB, ch = e % 8;
+                        if (row >= md.nvalid)
+                            *reinterpret_cast<uint4*>(vst + bi * box_bytes + row * 128 + ch * 16) =
+                                make_uint4(0, 0, 0, 0);
+                    }
+                    fence_proxy_async_smem();
+                    __syncwarp();
+                }
+                // S^T = K q^T over this warp's 16 tokens
+                float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    const int row = r0 + ri + 8 * (mi & 1);
+                    const int ch = (ks & 3) * 2 + (mi >> 1);
+                    uint32_t af[4];
+                    ldmatrix_x4(af, smem_u32(kst + (ks >> 2) * box_bytes + row * 128 + ((ch ^ (row & 7)) << 4)));
+                    mma_bf16_16816(c, af[0], af[1], af[2], af[3], qf[ks][0], qf[ks][1]);
+                }
+                const float sl = a.scale_log2;
+                const bool va = r0 + g < md.nvalid, vb = r0 + g + 8 < md.nvalid;
+                const float x0 = va ? c[0] * sl : -INFINITY, x1 = va ? c[1] * sl : -INFINITY;
+                const float x2 = vb ? c[2] * sl : -INFINITY, x3 = vb ? c[3] * sl : -INFINITY;
+                float t0 = fmaxf(x0, x2), t1 = fmaxf(x1, x3);
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, off));
+                    t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, off));
+                }
+                const float mn0 = fmaxf(m[0], t0), mn1 = fmaxf(m[1], t1);
+                const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m[0] - mn0);
+                const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m[1] - mn1);
+                const float ref0 = mn0 == -INFINITY ? 0.f : mn0, ref1 = mn1 == -INFINITY ? 0.f : mn1;
+                const float p0 = exp2f(x0 - ref0), p2 = exp2f(x2 - ref0);
+                const float p1 = exp2f(x1 - ref1), p3 = exp2f(x3 - ref1);
+                m[0] = mn0;
+                m[1] = mn1;
+                lsum[0] = lsum[0] * al0 + (p0 + p2);
+                lsum[1] = lsum[1] * al1 + (p1 + p3);
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    acc[mt][0] *= al0;
+                    acc[mt][1] *= al1;
+                    acc[mt][2] *= al0;
+                    acc[mt][3] *= al1;
+                }
+                // P^T operand from the S^T accumulators (8x8 transposes), hi + lo bf16 parts
+                const uint32_t hi0 = pack_bf16x2(p0, p1), hi1 = pack_bf16x2(p2, p3);
+                const uint32_t lo0 = pack_bf16x2(p0 - bf16_lo(hi0), p1 - bf16_hi(hi0));
+                const uint32_t lo1 = pack_bf16x2(p2 - bf16_lo(hi1), p3 - bf16_hi(hi1));
+                const uint32_t bh0 = movmatrix_trans(hi0), bh1 = movmatrix_trans(hi1);
+                const uint32_t bl0 = movmatrix_trans(lo0), bl1 = movmatrix_trans(lo1);
+                // O^T += V^T P^T: V^T fragments straight from the swizzled stage (ldmatrix.trans)
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const int row = r0 + ri + 8 * (mi >> 1);
+                    const int ch = 2 * mt + (mi & 1);
+                    uint32_t af[4];
+                    ldmatrix_x4_trans(af, smem_u32(vst + (ch >> 3) * box_bytes + row * 128 +
+                                                   (((ch & 7) ^ (row & 7)) << 4)));
+                    mma_bf16_16816(acc[mt], af[0], af[1], af[2], af[3], bh0, bh1);
+                    mma_bf16_16816(acc[mt], af[0], af[1], af[2], af[3], bl0, bl1);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);  // the ring slot may be refilled now
+            if (md.flags & kStageLast) {
+                // publish this warp's state of the item, then merge the item's split as a group
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], off);
+                    lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], off);
+                }
+                const int h0 = 2 * tq, h1 = 2 * tq + 1;
+                if (g == 0) {
+                    if (h0 < a.G) {
+                        sm.M(warp, h0) = m[0];
+                        sm.L(warp, h0) = lsum[0];
+                    }
+                    if (h1 < a.G) {
+                        sm.M(warp, h1) = m[1];
+                        sm.L(warp, h1) = lsum[1];
+                    }
+                }
+                // accumulator (mt, row g / g+8) <-> d = 16 mt + g (+8)
+                float* w0 = sm.acc + (warp * a.G + h0) * D;
+                float* w1 = w0 + D;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) {
+                    const int d0 = 16 * mt + g;
+                    if (h0 < a.G) {
+                        w0[d0] = acc[mt][0];
+                        w0[d0 + 8] = acc[mt][2];
+                    }
+                    if (h1 < a.G) {
+                        w1[d0] = acc[mt][1];
+                        w1[d0 + 8] = acc[mt][3];
+                    }
+                }
+                const int layer = md.lp / a.pairs, pair = md.lp - layer * a.pairs;
+                finish_split<__nv_bfloat16, D>(a, layer, pair, md.lp, md.seg, md.nseg, sm, s_ml, gp);
+                m[0] = m[1] = -INFINITY;
+                lsum[0] = lsum[1] = 0.f;
+#pragma unroll
+                for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+            }
         }
     }
-    finish_split<__nv_bfloat16, D>(a, layer, pair, lp, split, sm);
 }
 
 // -------------------------------------------------------------------------------------- fp32 path
 // One token at a time per warp; lanes split d, warp reductions form the dot products.
 template <int D>
 __global__ void __launch_bounds__(kDecodeThreads) decode_f32_kernel(DecodeArgs a) {
-    __shared__ DecodeSmem<D> sm;
+    __shared__ float s_m[kDecodeWarps * kMaxG], s_l[kDecodeWarps * kMaxG];
+    __shared__ float s_acc[kDecodeWarps * kMaxG * D];
+    const MergeView sm{s_m, s_l, s_acc};
     constexpr int E = D / 32;
     const int split = blockIdx.x % a.splits, lp = blockIdx.x / a.splits;
     const int layer = lp / a.pairs, pair = lp - layer * a.pairs;
@@ -366,7 +497,7 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_f32_kernel(DecodeArgs a
         for (int e = 0; e < E; ++e) qv[h][e] = h < a.G ? qb[h * D + lane * E + e] : 0.f;
     pdl_trigger();
     pdl_wait();
-    const SplitInfo si = split_info(a, layer, pair, split);
+    const SplitInfo si = split_info(a, layer, pair, split, threadIdx.x == 0);
     const float* kp = reinterpret_cast<const float*>(a.k[layer]) + (size_t)pair * a.T_cap * D;
     const float* vp = reinterpret_cast<const float*>(a.v[layer]) + (size_t)pair * a.T_cap * D;
     const int32_t* ip = a.block_idx + (size_t)pair * a.sel_cap;
@@ -417,14 +548,16 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_f32_kernel(DecodeArgs a
     for (int h = 0; h < kMaxG; ++h) {
         if (h < a.G) {
             if (lane == 0) {
-                sm.m[warp][h] = m[h];
-                sm.l[warp][h] = l[h];
+                sm.M(warp, h) = m[h];
+                sm.L(warp, h) = l[h];
             }
 #pragma unroll
-            for (int e = 0; e < E; ++e) sm.acc[warp][h][lane * E + e] = acc[h][e];
+            for (int e = 0; e < E; ++e) sm.acc[(warp * a.G + h) * D + lane * E + e] = acc[h][e];
         }
     }
-    finish_split<float, D>(a, layer, pair, lp, split, sm);
+    __shared__ float2 s_ml[kMaxCombineSlots];
+    finish_split<float, D>(a, layer, pair, lp, split, a.splits, sm, s_ml,
+                           Group{(int)threadIdx.x, (int)blockDim.x, 0});
 }
 
 template <typename K>
@@ -435,14 +568,63 @@ cudaError_t launch_decode_k(K kernel, const Plan& p, const DecodeArgs& a, int la
     return launch_pdl(kernel, dim3((unsigned)grid), dim3(kDecodeThreads), 0, st, a);
 }
 
+template <int D>
+cudaError_t launch_decode_tma(const Plan& p, const DecodeArgs& a, const KVMaps* maps, int layers,
+                              cudaStream_t st) {
+    const int64_t n_slots = (int64_t)layers * p.pairs * p.sel_cap;
+    if (n_slots <= 0) return cudaSuccess;
+    // the plan's CTA count covers num_layers layers; fewer layers get proportionally fewer CTAs
+    int64_t ctas = (int64_t)p.dec_ctas * layers / p.layers;
+    if (ctas < 1) ctas = 1;
+    const size_t qslot = kQSlot * (((size_t)a.G * D * 2 + kQSlot - 1) / kQSlot);
+    const size_t stage_bytes = (size_t)2 * (D / 64) * a.stage_tokens * 128 + qslot;
+    // two CTAs per SM: ~112 KB each, of which the merge and combine scratch take a few KB
+    const size_t scratch = merge_bytes(a.G, D) + sizeof(float2) * (size_t)a.slots * a.Gp;
+    const size_t budget = 112 * 1024 - 1024 - scratch;
+    int nstages = (int)(budget / stage_bytes);
+    if (nstages < 2) nstages = 2;
+    if (nstages > kMaxStages) nstages = kMaxStages;
+    const size_t smem = 1024 + (size_t)nstages * stage_bytes + scratch;
+    cudaError_t e = cudaFuncSetAttribute(decode_tma_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(decode_tma_kernel<D>, dim3((unsigned)ctas), dim3(kTmaThreads), smem, st, a,
+                      *maps, nstages, n_slots);
+}
+
 }  // namespace
 
-cudaError_t launch_decode(const Plan& p, const DecodeArgs& a, int layers, cudaStream_t st) {
+cudaError_t launch_decode(const Plan& p, const DecodeArgs& a, const KVMaps* maps, int layers,
+                          cudaStream_t st) {
     if (p.dtype == BSA_BF16)
-        return p.D == 128 ? launch_decode_k(decode_bf16_kernel<128>, p, a, layers, st)
-                          : launch_decode_k(decode_bf16_kernel<64>, p, a, layers, st);
+        return p.D == 128 ? launch_decode_tma<128>(p, a, maps, layers, st)
+                          : launch_decode_tma<64>(p, a, maps, layers, st);
     return p.D == 128 ? launch_decode_k(decode_f32_kernel<128>, p, a, layers, st)
                       : launch_decode_k(decode_f32_kernel<64>, p, a, layers, st);
+}
+
+bool encode_kv_map(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows) {
+    typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                 const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                 const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                 CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeFn encode = nullptr;
+    if (!encode) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || !fn)
+            return false;
+        encode = reinterpret_cast<EncodeFn>(fn);
+    }
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    const cuuint32_t estr[2] = {1, 1};
+    return encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace bsa

@@ -539,6 +539,7 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
 // grid = pairs * parts. Part p of a pair scores windows [p*PW, p*PW + PW) and owns the blocks whose
 // first overlapping window falls in that range (the last part with windows also owns the blocks
 // past the last window, which score -inf).
+template <int GP>
 __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a) {
     extern __shared__ uint32_t s_dyn[];  // [key_words] keys, then [PW + W_max] window scores
     __shared__ float sM[kMaxG], sInvZ[kMaxG];
@@ -592,12 +593,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
         const int64_t jend = b_hi > b_lo ? min(last_window(b_hi - 1, a.BS, a.s) + 1, nc) : j0;
         if (jend > j0) {
             const float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
-            switch (a.Gp) {
-                case 1: window_scores<1>(lg, j0, jend, a.G, sM, sInvZ, S); break;
-                case 2: window_scores<2>(lg, j0, jend, a.G, sM, sInvZ, S); break;
-                case 4: window_scores<4>(lg, j0, jend, a.G, sM, sInvZ, S); break;
-                default: window_scores<8>(lg, j0, jend, a.G, sM, sInvZ, S); break;
-            }
+            window_scores<GP>(lg, j0, jend, a.G, sM, sInvZ, S);
         }
         __syncthreads();
         const int j0i = (int)j0, nci = (int)nc;
@@ -656,9 +652,7 @@ cudaError_t launch_score_k(K kernel, const ScoreArgs& a, cudaStream_t st) {
     return launch_pdl(kernel, dim3((unsigned)grid), dim3(kScoreThreads), 0, st, a);
 }
 
-}  // namespace
-
-cudaError_t launch_score(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
+cudaError_t launch_score_impl(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
     if (p.dtype == BSA_BF16)
         return p.D == 128 ? launch_score_k(score_bf16_kernel<128>, a, st)
                           : launch_score_k(score_bf16_kernel<64>, a, st);
@@ -666,14 +660,31 @@ cudaError_t launch_score(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
                       : launch_score_k(score_f32_kernel<64>, a, st);
 }
 
-cudaError_t launch_select(const Plan& p, const SelectArgs& a, cudaStream_t st) {
+template <int GP>
+cudaError_t launch_select_k(const Plan& p, const SelectArgs& a, cudaStream_t st) {
     if (p.select_smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaError_t e = cudaFuncSetAttribute(select_kernel<GP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)p.select_smem);
         if (e != cudaSuccess) return e;
     }
-    return launch_pdl(select_kernel, dim3((unsigned)(p.pairs * p.select_parts)),
+    return launch_pdl(select_kernel<GP>, dim3((unsigned)(p.pairs * p.select_parts)),
                       dim3(kSelectThreads), p.select_smem, st, a);
+}
+
+}  // namespace
+
+cudaError_t launch_score(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
+    return launch_score_impl(p, a, st);
+}
+
+cudaError_t launch_select(const Plan& p, const SelectArgs& a, cudaStream_t st) {
+    switch (p.Gp) {
+        case 1: return launch_select_k<1>(p, a, st);
+        case 2: return launch_select_k<2>(p, a, st);
+        case 4: return launch_select_k<4>(p, a, st);
+        default: return launch_select_k<8>(p, a, st);
+    }
 }
 
 }  // namespace bsa

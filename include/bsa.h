@@ -78,7 +78,8 @@ typedef enum {
     BSA_DEVERR_SEQ_LEN = 1u << 0,   /* seq_lens[b] < 0 or > max_seq_len: pair skipped */
     BSA_DEVERR_CAPACITY = 1u << 1,  /* bsa_compress_append with seq_lens[b] == max_seq_len */
     BSA_DEVERR_BLOCK_IDX = 1u << 2, /* block index outside [0, ceil(T/BS)): entry skipped */
-    BSA_DEVERR_N_SEL = 1u << 3      /* n_sel outside [0, SEL_cap]: clamped */
+    BSA_DEVERR_N_SEL = 1u << 3,     /* n_sel outside [0, SEL_cap]: clamped */
+    BSA_DEVERR_TIMEOUT = 1u << 4    /* a pipeline wait gave up (never expected): output invalid */
 } bsa_device_error_t;
 
 /* Problem shape and method parameters. Supported: dtype fp32 or bf16; head_dim 64 or 128;
