@@ -73,6 +73,10 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
     // Scoring: 64-row chunks, spread evenly over a persistent grid at launch time.
     P.nchunk = (P.nc_cap + 63) / 64;
     P.total_chunks = (int64_t)P.pairs * P.nchunk;
+    P.nstat = P.nchunk;  // softmax statistics per 64-row chunk
+    P.score_ctas = (int)(P.total_chunks < 2 * kNumSMs ? (P.total_chunks > 0 ? P.total_chunks : 1)
+                                                       : 2 * kNumSMs);
+    if (P.dtype == BSA_BF16 && (int64_t)P.pairs * P.nc_cap > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
     // Selection: one CTA per pair when there are enough pairs to fill the GPU in one wave,
     // otherwise the pairs' windows are split into parts of at least 256 windows.
     {
@@ -87,8 +91,8 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
         if ((int64_t)P.pairs * P.select_parts > 0x7fffffff) return BSA_ERR_UNSUPPORTED;
         const int64_t wmax = (P.BS + P.l - 2) / P.s + 2;  // windows overlapping one block, bound
         // the key array also stages the chunk statistics (2 words per float2)
-        P.select_keys = (size_t)P.nb_cap > (size_t)(2 * P.nchunk * P.Gp)
-                            ? (size_t)P.nb_cap : (size_t)(2 * P.nchunk * P.Gp);
+        P.select_keys = (size_t)P.nb_cap > (size_t)(2 * P.nstat * P.Gp)
+                            ? (size_t)P.nb_cap : (size_t)(2 * P.nstat * P.Gp);
         P.select_smem = (P.select_keys + (size_t)pw + (size_t)wmax) * sizeof(uint32_t);
         if (P.select_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
     }
@@ -129,7 +133,7 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
     P.off_logits = off;
     off = align_up(off + (size_t)P.pairs * P.nc_cap * P.Gp * sizeof(float));
     P.off_stats = off;
-    off = align_up(off + (size_t)P.pairs * P.nchunk * P.Gp * sizeof(float2));
+    off = align_up(off + (size_t)P.pairs * P.nstat * P.Gp * sizeof(float2));
     P.off_bscores = off;
     off = align_up(off + (size_t)P.pairs * P.nb_cap * sizeof(float));
     P.off_part_ml = off;
@@ -176,6 +180,7 @@ ScoreArgs score_args(const Plan& P, const void* q, const void* ck, const int32_t
     a.nc_cap = P.nc_cap;
     a.nchunk = P.nchunk;
     a.total_chunks = P.total_chunks;
+    a.nstat = P.nstat;
     a.score_log2 = P.score_log2;
     return a;
 }
@@ -206,7 +211,7 @@ SelectArgs select_args(const Plan& P, const int32_t* seq_lens, int32_t* block_id
     a.T_cap = P.T_cap;
     a.nc_cap = P.nc_cap;
     a.nb_cap = P.nb_cap;
-    a.nchunk = P.nchunk;
+    a.nstat = P.nstat;
     a.key_words = (int64_t)P.select_keys;
     a.parts = P.select_parts;
     a.part_windows = P.select_part_windows;
@@ -218,7 +223,11 @@ bsa_status_t do_select(const Plan& P, const void* q, const void* ck, const int32
                        int32_t* block_idx, int32_t* n_sel, float* block_scores, void* ws,
                        cudaStream_t st) {
     ScoreArgs sa = score_args(P, q, ck, seq_lens, ws);
-    cudaError_t e = launch_score(P, sa, st);
+    static thread_local CUtensorMap ck_map;
+    if (P.dtype == BSA_BF16 && P.nc_cap > 0 &&
+        !encode_kv_map(&ck_map, ck, (uint64_t)P.pairs * P.nc_cap, P.D, 64))
+        return BSA_ERR_CUDA;
+    cudaError_t e = launch_score(P, sa, &ck_map, st);
     if (e != cudaSuccess) return BSA_ERR_CUDA;
     SelectArgs la = select_args(P, seq_lens, block_idx, n_sel, block_scores, ws);
     return from_cuda(launch_select(P, la, st));

@@ -28,8 +28,10 @@ struct Plan {
     int pairs;
     float scale_log2;  // attention scale * log2(e): softmax evaluated with exp2
     float score_log2;  // (1 / tau) * log2(e)
-    // scoring: 64-row chunks of compressed keys, spread evenly over a persistent grid
-    int64_t nchunk, total_chunks;
+    // scoring: 64-row chunks of compressed keys spread evenly over a persistent grid; softmax
+    // statistics per chunk
+    int64_t nchunk, total_chunks, nstat;
+    int score_ctas;
     // selection: pairs * select_parts CTAs, each scoring select_part_windows windows
     int select_parts, select_part_windows;
     size_t select_keys;  // words of the block-key array at the front of its shared memory
@@ -71,9 +73,9 @@ struct ScoreArgs {
     const int32_t* seq_lens;
     uint32_t* err;
     float* logits;        // [pairs][nc_cap][Gp], log2 units
-    float2* stats;        // [pairs][nchunk][Gp] (max, sum of exp2(x - max)) per chunk and head
+    float2* stats;        // [pairs][nstat][Gp] (max, sum of exp2(x - max)) per chunk and head
     int B, Hq, Hkv, G, Gp, l, s;
-    int64_t T_cap, nc_cap, nchunk, total_chunks;
+    int64_t T_cap, nc_cap, nchunk, total_chunks, nstat;
     float score_log2;
 };
 
@@ -88,7 +90,7 @@ struct SelectArgs {
     uint32_t* err;
     int* cnt;             // [pairs] completion counters
     int Hkv, G, Gp, l, s, BS, n_init, n_local, top_k, sel_cap;
-    int64_t T_cap, nc_cap, nb_cap, nchunk, key_words;
+    int64_t T_cap, nc_cap, nb_cap, nstat, key_words;
     int parts, part_windows;
 };
 
@@ -124,7 +126,8 @@ struct DecodeArgs {
 // Launchers (one per kernel family); they pick the template instance from the plan's dtype/D.
 cudaError_t launch_compress_keys(const Plan& p, const CompressArgs& a, cudaStream_t st);
 cudaError_t launch_append(const Plan& p, const AppendArgs& a, cudaStream_t st);
-cudaError_t launch_score(const Plan& p, const ScoreArgs& a, cudaStream_t st);
+cudaError_t launch_score(const Plan& p, const ScoreArgs& a, const CUtensorMap* ck_map,
+                         cudaStream_t st);
 cudaError_t launch_select(const Plan& p, const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_decode(const Plan& p, const DecodeArgs& a, const KVMaps* maps, int layers,
                           cudaStream_t st);

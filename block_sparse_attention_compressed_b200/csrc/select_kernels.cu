@@ -5,14 +5,14 @@
 //
 // Two kernels chained with programmatic dependent launch:
 //
-// score (persistent): every warp owns a contiguous, equal share of the 64-row chunks of all pairs'
-//   compressed keys, so all warps finish together (no partial last wave). It streams 16-row tiles,
-//   computes the group's logits x[j][h] = q_h . K~_j / tau (log2 units) and writes them to the
-//   workspace together with each chunk's per-head (max, sum exp2(x - max)).
-//   bf16: the contraction runs on the tensor cores with mma.m16n8k16 -- rows are M, the G heads
-//   (padded to 8) are N, head_dim is K. A dot product does not depend on the order of its terms,
-//   so each lane feeds the A operand straight from its own 16-byte global loads and q's operand is
-//   permuted the same way. fp32: FMA dot products, one warp per row.
+// score (persistent): the 64-row chunks of all pairs' compressed keys are shared evenly by the CTAs,
+//   so all finish together. It computes the group's logits x[j][h] = q_h . K~_j / tau (log2 units)
+//   and writes them to the workspace with each chunk's per-head (max, sum exp2(x - max)).
+//   bf16: a producer warp streams the chunks into a ring of shared-memory stages with 2-D TMA
+//   tensor copies (128-byte swizzle) completing on mbarriers; four consumer warps take whole
+//   chunks in turn and run the contraction on the tensor cores (mma.m16n8k16 with ldmatrix
+//   operands: rows are M, the G heads padded to 8 are N, head_dim is K). fp32: FMA dot products,
+//   one warp per row.
 //
 // select (pairs x parts CTAs): merges the chunk statistics into each head's softmax normaliser,
 //   turns the logits of its part of the windows into S[j] = sum_h softmax_h[j], max-pools S onto
@@ -102,147 +102,159 @@ __device__ __forceinline__ void flush_stats(float2* dst, float m0, float s0, flo
     }
 }
 
-template <int D>
-struct KTile {
-    static constexpr int NI = D / 32;  // 16-byte chunks a lane holds per row (chunks tq + 4i)
-    uint4 a[NI], b[NI];                // rows r+g and r+g+8 of the tile
+constexpr int kScoreConsumers = 4;
+constexpr int kScoreTmaThreads = (kScoreConsumers + 1) * 32;
+constexpr int kScoreMaxStages = 8;
+static_assert(kScoreMaxStages % kScoreConsumers == 0, "slots are owned by one consumer warp each");
+constexpr uint32_t kScoreWaitPolls = 1u << 26;
+
+struct ScoreStage {
+    int pair;
+    int row0;   // first window of the chunk
+    int nrows;  // windows of the chunk below the pair's window count; -1 ends the stream
 };
 
+// Consumer warp w takes stages w, w + 4, ...: a whole 64-row chunk per warp, its four 16-row groups
+// as independent mma chains, so four chunks are in compute at once while the producer keeps the
+// rest of the ring loading. The stage count must be a multiple of the consumer count: then slot
+// st only ever serves warp st % 4, which waits on it one phase at a time. (A slot shared by two
+// warps lets one of them wait two phases ahead, where the parity test cannot tell the phases
+// apart and passes on a slot whose copy is still in flight.)
 template <int D>
-__device__ __forceinline__ void load_ktile(KTile<D>& t, const uint16_t* ckp, int64_t r, int64_t r1,
-                                           int g, int tq) {
-    const int64_t ra = r + g, rb = r + g + 8;
-#pragma unroll
-    for (int i = 0; i < KTile<D>::NI; ++i) {
-        const int col = (tq + 4 * i) * 8;
-        t.a[i] = ra < r1 ? ld_stream(ckp + ra * D + col) : make_uint4(0, 0, 0, 0);
-        t.b[i] = rb < r1 ? ld_stream(ckp + rb * D + col) : make_uint4(0, 0, 0, 0);
+__global__ void __launch_bounds__(kScoreTmaThreads, 2)
+    score_tma_kernel(const ScoreArgs a, const __grid_constant__ CUtensorMap ck_map, const int nstages) {
+    extern __shared__ uint8_t dsm_raw[];
+    __shared__ __align__(8) uint64_t full[kScoreMaxStages], empty[kScoreMaxStages];
+    __shared__ ScoreStage meta[kScoreMaxStages];
+    constexpr int NB = D / 64;  // 64-column boxes per row
+    constexpr int KS = D / 16;  // k-steps
+    const uint32_t box_bytes = 64u * 128u;
+    const uint32_t stage_bytes = NB * box_bytes;
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
+    const int C = (int)gridDim.x;
+    const int64_t c_lo = (int64_t)blockIdx.x * a.total_chunks / C;
+    const int64_t c_hi = (int64_t)(blockIdx.x + 1) * a.total_chunks / C;
+    if (threadIdx.x == 0) {
+        for (int s2 = 0; s2 < nstages; ++s2) {
+            mbar_init(&full[s2], 1);
+            mbar_init(&empty[s2], 1);
+        }
+        mbar_fence_init();
     }
-}
-
-// A warp's share of the tile stream: slot u covers tile (u % 4) of chunk c_lo + u / 4.
-struct TileCursor {
-    int64_t c_lo, n_slots;
-    int cached_pair;
-    int64_t cached_nc;
-};
-
-__device__ __forceinline__ int64_t pair_windows(const ScoreArgs& a, int pair, TileCursor& tc) {
-    if (pair != tc.cached_pair) {
-        tc.cached_pair = pair;
-        const int64_t T = a.seq_lens[pair / a.Hkv];
-        tc.cached_nc = (T >= 0 && T <= a.T_cap) ? num_windows(T, a.l, a.s) : 0;
-    }
-    return tc.cached_nc;
-}
-
-// First slot >= u whose tile holds at least one window; n_slots when there is none.
-__device__ __forceinline__ int64_t next_slot(const ScoreArgs& a, TileCursor& tc, int64_t u) {
-    while (u < tc.n_slots) {
-        const int64_t chunk = tc.c_lo + (u >> 2);
-        const int pair = (int)(chunk / a.nchunk);
-        const int64_t row = (chunk - (int64_t)pair * a.nchunk) * 64 + (u & 3) * 16;
-        if (row < pair_windows(a, pair, tc)) return u;
-        u = (u | 3) + 1;  // the rest of this chunk is past the sequence: next chunk
-    }
-    return tc.n_slots;
-}
-
-template <int D>
-__global__ void __launch_bounds__(kScoreThreads, 2) score_bf16_kernel(ScoreArgs a) {
-    constexpr int NI = D / 32;
-    const int lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
-    const int64_t W = (int64_t)gridDim.x * kScoreWarps;
-    const int64_t w = (int64_t)blockIdx.x * kScoreWarps + (threadIdx.x >> 5);
-    TileCursor tc;
-    tc.c_lo = w * a.total_chunks / W;
-    tc.n_slots = ((w + 1) * a.total_chunks / W - tc.c_lo) * 4;
-    tc.cached_pair = -1;
-    tc.cached_nc = 0;
+    __syncthreads();
     pdl_trigger();
     pdl_wait();
     report_lengths(a);
-    const bool h0 = 2 * tq < a.G, h1 = 2 * tq + 1 < a.G;
-    int cur_pair = -1;
-    uint32_t qf[NI][4];
-    float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
 
-    KTile<D> ta, tb;
-    auto load_slot = [&](KTile<D>& t, int64_t u) {
-        const int64_t chunk = tc.c_lo + (u >> 2);
-        const int pair = (int)(chunk / a.nchunk);
-        const int64_t row = (chunk - (int64_t)pair * a.nchunk) * 64 + (u & 3) * 16;
-        const int64_t r1 = min(row + 16, pair_windows(a, pair, tc));
-        load_ktile<D>(t, reinterpret_cast<const uint16_t*>(a.ck) + (size_t)pair * a.nc_cap * D, row,
-                      r1, g, tq);
-    };
-    auto compute_slot = [&](const KTile<D>& t, int64_t u, int64_t u_next) {
-        const int64_t chunk = tc.c_lo + (u >> 2);
-        const int pair = (int)(chunk / a.nchunk);
-        const int64_t ci = chunk - (int64_t)pair * a.nchunk;
-        const int64_t row = ci * 64 + (u & 3) * 16;
-        const int64_t r1 = min(row + 16, pair_windows(a, pair, tc));
-        if (pair != cur_pair) {
-            // q as the B operand: lane (g, tq) holds head g at chunks tq + 4i, the d positions its
-            // own key loads cover (heads >= G are zero)
-            cur_pair = pair;
-            const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
-            const uint16_t* qh = reinterpret_cast<const uint16_t*>(a.q) +
-                                 ((size_t)b * a.Hq + (size_t)kvh * a.G + g) * D;
+    if (warp == kScoreConsumers) {
+        if (lane == 0) {
+            int k = 0, cur_pair = -1;
+            int64_t nc = 0;
+            bool ok = true;
+            auto claim = [&](int kk) -> int {
+                const int st = kk % nstages;
+                if (kk >= nstages && !mbar_wait(&empty[st], ((kk / nstages) - 1) & 1, kScoreWaitPolls)) {
+                    atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                    ok = false;
+                }
+                return st;
+            };
+            for (int64_t chunk = c_lo; chunk < c_hi && ok; ++chunk) {
+                const int pair = (int)(chunk / a.nchunk);
+                const int64_t row0 = (chunk - (int64_t)pair * a.nchunk) * 64;
+                if (pair != cur_pair) {
+                    cur_pair = pair;
+                    const int64_t T = a.seq_lens[pair / a.Hkv];
+                    nc = (T >= 0 && T <= a.T_cap) ? num_windows(T, a.l, a.s) : 0;
+                }
+                if (row0 >= nc) continue;  // past the sequence: nothing to score
+                const int st = claim(k);
+                if (!ok) break;
+                meta[st].pair = pair;
+                meta[st].row0 = (int)row0;
+                meta[st].nrows = (int)min((int64_t)64, nc - row0);
+                uint8_t* dst = ring + (size_t)st * stage_bytes;
+                mbar_arrive_expect_tx(&full[st], stage_bytes);
+                const int y = (int)((int64_t)pair * a.nc_cap + row0);
 #pragma unroll
-            for (int i = 0; i < NI; ++i) {
-                uint4 v = g < a.G ? *reinterpret_cast<const uint4*>(qh + (tq + 4 * i) * 8)
-                                  : make_uint4(0, 0, 0, 0);
-                qf[i][0] = v.x;
-                qf[i][1] = v.y;
-                qf[i][2] = v.z;
-                qf[i][3] = v.w;
+                for (int bi = 0; bi < NB; ++bi) tma_load_2d(dst + bi * box_bytes, &ck_map, 64 * bi, y, &full[st]);
+                ++k;
+            }
+            // end-of-stream markers, one per consumer warp (each waits on its own stages only)
+            for (int w = 0; w < kScoreConsumers && ok; ++w) {
+                const int st = claim(k);
+                if (!ok) break;
+                meta[st].nrows = -1;
+                mbar_arrive(&full[st]);
+                ++k;
             }
         }
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < NI; ++i) {
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                mma_bf16_16816(c, u4_get(t.a[i], 2 * hh), u4_get(t.b[i], 2 * hh),
-                               u4_get(t.a[i], 2 * hh + 1), u4_get(t.b[i], 2 * hh + 1),
-                               qf[i][2 * hh], qf[i][2 * hh + 1]);
+    } else {
+        const int mi = lane >> 3, ri = lane & 7;
+        const bool h0 = 2 * tq < a.G, h1 = 2 * tq + 1 < a.G;
+        uint32_t qf[KS][2];
+        int q_pair = -1;
+        for (int k = warp;; k += kScoreConsumers) {
+            const int st = k % nstages;
+            if (!mbar_wait(&full[st], (k / nstages) & 1, kScoreWaitPolls)) {
+                if (lane == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                break;
             }
+            const ScoreStage md = meta[st];
+            if (md.nrows < 0) break;
+            if (md.pair != q_pair) {
+                // q as the B operand: lane (g, tq) holds head g, d = 16ks + 2tq (+1, +8, +9)
+                q_pair = md.pair;
+                const int b = md.pair / a.Hkv, kvh = md.pair - b * a.Hkv;
+                const uint32_t* qs = reinterpret_cast<const uint32_t*>(
+                    reinterpret_cast<const uint16_t*>(a.q) + ((size_t)b * a.Hq + (size_t)kvh * a.G + g) * D);
+#pragma unroll
+                for (int ks = 0; ks < KS; ++ks) {
+                    qf[ks][0] = g < a.G ? qs[8 * ks + tq] : 0u;
+                    qf[ks][1] = g < a.G ? qs[8 * ks + 4 + tq] : 0u;
+                }
+            }
+            const uint8_t* cst = ring + (size_t)st * stage_bytes;
+            float c[4][4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) c[r][0] = c[r][1] = c[r][2] = c[r][3] = 0.f;
+#pragma unroll
+            for (int ks = 0; ks < KS; ++ks) {
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {  // four independent 16-row groups
+                    const int row = 16 * r + ri + 8 * (mi & 1);
+                    const int ch = (ks & 3) * 2 + (mi >> 1);
+                    uint32_t af[4];
+                    ldmatrix_x4(af, smem_u32(cst + (ks >> 2) * box_bytes + row * 128 + ((ch ^ (row & 7)) << 4)));
+                    mma_bf16_16816(c[r], af[0], af[1], af[2], af[3], qf[ks][0], qf[ks][1]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[st]);  // the data is in registers: refill the slot
+            float* lg = a.logits + (size_t)md.pair * a.nc_cap * a.Gp;
+            float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const float x0 = c[r][0] * a.score_log2, x1 = c[r][1] * a.score_log2;
+                const float x2 = c[r][2] * a.score_log2, x3 = c[r][3] * a.score_log2;
+                const int lra = 16 * r + g, lrb = lra + 8;
+                const int64_t ra = md.row0 + lra, rb = md.row0 + lrb;
+                if (lra < md.nrows) {
+                    if (h1) *reinterpret_cast<float2*>(lg + ra * a.Gp + 2 * tq) = make_float2(x0, x1);
+                    else if (h0) lg[ra * a.Gp + 2 * tq] = x0;
+                    if (h0) online_add(m0, s0, x0);
+                    if (h1) online_add(m1, s1, x1);
+                }
+                if (lrb < md.nrows) {
+                    if (h1) *reinterpret_cast<float2*>(lg + rb * a.Gp + 2 * tq) = make_float2(x2, x3);
+                    else if (h0) lg[rb * a.Gp + 2 * tq] = x2;
+                    if (h0) online_add(m0, s0, x2);
+                    if (h1) online_add(m1, s1, x3);
+                }
+            }
+            flush_stats(a.stats + ((size_t)md.pair * a.nstat + md.row0 / 64) * a.Gp, m0, s0, m1, s1, g, tq, a.G);
         }
-        float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
-        const float x0 = c[0] * a.score_log2, x1 = c[1] * a.score_log2;
-        const float x2 = c[2] * a.score_log2, x3 = c[3] * a.score_log2;
-        const int64_t ra = row + g, rb = row + g + 8;
-        if (ra < r1) {
-            if (h1) *reinterpret_cast<float2*>(lg + ra * a.Gp + 2 * tq) = make_float2(x0, x1);
-            else if (h0) lg[ra * a.Gp + 2 * tq] = x0;
-            if (h0) online_add(m0, s0, x0);
-            if (h1) online_add(m1, s1, x1);
-        }
-        if (rb < r1) {
-            if (h1) *reinterpret_cast<float2*>(lg + rb * a.Gp + 2 * tq) = make_float2(x2, x3);
-            else if (h0) lg[rb * a.Gp + 2 * tq] = x2;
-            if (h0) online_add(m0, s0, x2);
-            if (h1) online_add(m1, s1, x3);
-        }
-        // last tile of its chunk in this warp's stream: publish the chunk's statistics
-        if (u_next >= tc.n_slots || (u_next >> 2) != (u >> 2)) {
-            flush_stats(a.stats + ((size_t)pair * a.nchunk + ci) * a.Gp, m0, s0, m1, s1, g, tq, a.G);
-            m0 = m1 = -INFINITY;
-            s0 = s1 = 0.f;
-        }
-    };
-    // ping-pong: the next tile's loads are in flight while the current tile is computed
-    int64_t ua = next_slot(a, tc, 0);
-    if (ua < tc.n_slots) load_slot(ta, ua);
-    while (ua < tc.n_slots) {
-        const int64_t ub = next_slot(a, tc, ua + 1);
-        if (ub < tc.n_slots) load_slot(tb, ub);
-        compute_slot(ta, ua, ub);
-        if (ub >= tc.n_slots) break;
-        ua = next_slot(a, tc, ub + 1);
-        if (ua < tc.n_slots) load_slot(ta, ua);
-        compute_slot(tb, ub, ua);
     }
 }
 
@@ -301,7 +313,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_f32_kernel(ScoreArgs a
                 online_add(m[h], s[h], x);
             }
         }
-        float2* st = a.stats + ((size_t)pair * a.nchunk + ci) * a.Gp;
+        float2* st = a.stats + ((size_t)pair * a.nstat + ci) * a.Gp;
 #pragma unroll
         for (int h = 0; h < kMaxG; ++h)
             if (h < a.G && lane == h) st[h] = make_float2(m[h], s[h]);
@@ -562,8 +574,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
         // merges head h
         {
             const int64_t nch = (nc + 63) / 64;
-            float2* s_st = reinterpret_cast<float2*>(s_dyn);  // 2 * nchunk * Gp <= key_words
-            const float2* st = a.stats + (size_t)pair * a.nchunk * a.Gp;
+            float2* s_st = reinterpret_cast<float2*>(s_dyn);  // 2 * nstat * Gp <= key_words
+            const float2* st = a.stats + (size_t)pair * a.nstat * a.Gp;
             for (int64_t e = tid; e < nch * a.Gp; e += kSelectThreads) s_st[e] = ld_cg(st + e);
             __syncthreads();
             if (warp < a.G) {
@@ -640,7 +652,7 @@ int sm_count() {
 }
 
 template <typename K>
-cudaError_t launch_score_k(K kernel, const ScoreArgs& a, cudaStream_t st) {
+cudaError_t launch_score_f32(K kernel, const ScoreArgs& a, cudaStream_t st) {
     if (a.total_chunks == 0) return cudaSuccess;
     int per_sm = 0;
     cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kernel, kScoreThreads, 0);
@@ -652,12 +664,22 @@ cudaError_t launch_score_k(K kernel, const ScoreArgs& a, cudaStream_t st) {
     return launch_pdl(kernel, dim3((unsigned)grid), dim3(kScoreThreads), 0, st, a);
 }
 
-cudaError_t launch_score_impl(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
-    if (p.dtype == BSA_BF16)
-        return p.D == 128 ? launch_score_k(score_bf16_kernel<128>, a, st)
-                          : launch_score_k(score_bf16_kernel<64>, a, st);
-    return p.D == 128 ? launch_score_k(score_f32_kernel<128>, a, st)
-                      : launch_score_k(score_f32_kernel<64>, a, st);
+template <int D>
+cudaError_t launch_score_tma(const Plan& p, const ScoreArgs& a, const CUtensorMap* ck_map,
+                             cudaStream_t st) {
+    if (a.total_chunks == 0) return cudaSuccess;
+    const size_t stage_bytes = (size_t)(D / 64) * 64 * 128;
+    // a multiple of the consumer count, so that every slot belongs to one consumer warp
+    int nstages = (int)((100 * 1024) / stage_bytes);
+    if (nstages > kScoreMaxStages) nstages = kScoreMaxStages;
+    nstages -= nstages % kScoreConsumers;
+    if (nstages < kScoreConsumers) nstages = kScoreConsumers;
+    const size_t smem = 1024 + (size_t)nstages * stage_bytes;
+    cudaError_t e = cudaFuncSetAttribute(score_tma_kernel<D>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(score_tma_kernel<D>, dim3((unsigned)p.score_ctas), dim3(kScoreTmaThreads),
+                      smem, st, a, *ck_map, nstages);
 }
 
 template <int GP>
@@ -674,8 +696,12 @@ cudaError_t launch_select_k(const Plan& p, const SelectArgs& a, cudaStream_t st)
 
 }  // namespace
 
-cudaError_t launch_score(const Plan& p, const ScoreArgs& a, cudaStream_t st) {
-    return launch_score_impl(p, a, st);
+cudaError_t launch_score(const Plan& p, const ScoreArgs& a, const CUtensorMap* ck_map,
+                         cudaStream_t st) {
+    if (p.dtype == BSA_BF16)
+        return p.D == 128 ? launch_score_tma<128>(p, a, ck_map, st) : launch_score_tma<64>(p, a, ck_map, st);
+    return p.D == 128 ? launch_score_f32(score_f32_kernel<128>, a, st)
+                      : launch_score_f32(score_f32_kernel<64>, a, st);
 }
 
 cudaError_t launch_select(const Plan& p, const SelectArgs& a, cudaStream_t st) {

@@ -257,6 +257,35 @@ def test_full_workload(name, cuda_device):
 
 
 @pytest.mark.slow
+def test_back_to_back_calls_are_stable(cuda_device):
+    """Many selections and decodes queued without a host sync between them (the launches overlap
+    through programmatic dependent launch and the persistent rings run at full speed) give the
+    first call's results bit for bit and raise no device error: pipeline races show up here."""
+    w = WORKLOADS["gqa4-bf16-128k-b16"]
+    run = GpuRun(w)
+    run.compress()
+    run.select()
+    run.decode()
+    torch.cuda.synchronize()
+    first = (run.block_idx.clone(), run.n_sel.clone(), run.block_scores.clone(),
+             run.out[0].clone(), run.lse[0].clone())
+    for _ in range(60):
+        run.select()
+    for _ in range(60):
+        run.decode()
+    for _ in range(20):
+        run.select()
+        run.decode()
+    torch.cuda.synchronize()
+    assert run.device_errors() == 0
+    now = (run.block_idx, run.n_sel, run.block_scores, run.out[0], run.lse[0])
+    for a, b in zip(first, now):
+        assert torch.equal(a, b)
+    del run
+    torch.cuda.empty_cache()
+
+
+@pytest.mark.slow
 def test_full_shared_index_workload(cuda_device):
     """Selection on layer 0, reused by the sparse attention of all four layers (one launch)."""
     w, run = _full_run("shared-index-4x64k-b8")
