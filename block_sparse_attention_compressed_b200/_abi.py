@@ -79,6 +79,7 @@ _SIGS = {
     "bsa_decode_step": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                              ctypes.c_size_t, _P]),
     "bsa_read_device_error": (_S, [_P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32), _P]),
+    "bsa_sparse_decode_noalloc": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
 
@@ -244,6 +245,23 @@ def bsa_sparse_decode(p: Params, q, k_cache, v_cache, seq_lens, block_idx, n_sel
         _ptr(lse, "lse", torch.float32, n["lse"], optional=True), _ptr(ws, "workspace"),
         ws.numel() * ws.element_size(), _stream(stream)),
         "bsa_sparse_decode")
+
+
+def bsa_sparse_decode_noalloc(p: Params, q, k_cache, v_cache, seq_lens, block_idx, n_sel, out,
+                              lse=None, device_error=None, stream=None):
+    """bsa_sparse_decode without a workspace, for callers that cannot allocate device memory: the
+    library keeps the split partials in its own fixed per-device scratch. ``device_error`` is an
+    optional int32 tensor of one element that receives the device error bits (OR-ed in)."""
+    import torch
+    n, e = _shapes(p), _elem(p)
+    _check(lib().bsa_sparse_decode_noalloc(
+        ctypes.byref(p), _ptr(q, "q", e, n["q"]), _ptr(k_cache, "k_cache", e, n["cache"]),
+        _ptr(v_cache, "v_cache", e, n["cache"]), _ptr(seq_lens, "seq_lens", torch.int32, p.batch),
+        _ptr(block_idx, "block_idx", torch.int32, n["idx"]),
+        _ptr(n_sel, "n_sel", torch.int32, n["pairs"]), _ptr(out, "out", e, n["q"]),
+        _ptr(lse, "lse", torch.float32, n["lse"], optional=True),
+        _ptr(device_error, "device_error", torch.int32, 1, optional=True), _stream(stream)),
+        "bsa_sparse_decode_noalloc")
 
 
 def bsa_sparse_decode_layers(p: Params, qs, k_caches, v_caches, seq_lens, block_idx, n_sel, outs,

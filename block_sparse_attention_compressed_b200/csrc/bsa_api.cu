@@ -488,3 +488,88 @@ bsa_status_t bsa_read_device_error(void* ws, size_t ws_bytes, uint32_t* flags,
 }
 
 }  // extern "C"
+
+// ============================================================ decode without a caller workspace
+// For callers that cannot allocate device memory: the sparse attention's split partials and
+// completion counters live in a fixed array of this library instead of a caller's workspace.
+#include <mutex>
+
+namespace bsa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;  // BSA_NOALLOC_SCRATCH_BYTES
+static_assert(kNoAllocScratchBytes == BSA_NOALLOC_SCRATCH_BYTES, "header and library agree");
+constexpr int kNoAllocMaxDevices = 64;
+
+// Zero when the library's device code is loaded; every call re-zeroes its counter region.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+std::mutex g_noalloc_mutex;
+void* g_noalloc_ptr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch on the current device, looked up once per device (with that
+// device current: the lookup may load this library's device code onto it).
+bsa_status_t noalloc_scratch(void** out) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return BSA_ERR_CUDA;
+    if (dev < 0 || dev >= kNoAllocMaxDevices) return BSA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress((void**)&p, g_noalloc_scratch) != cudaSuccess || !p)
+            return BSA_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return BSA_OK;
+}
+
+// The decode part of the workspace layout (error word, counters, partials), packed from offset 0.
+Plan noalloc_layout(const Plan& P) {
+    Plan V = P;
+    size_t off = 0;
+    V.off_err = off;
+    off = align_up(off + sizeof(uint32_t));
+    V.off_dec_cnt = off;
+    off = align_up(off + (size_t)P.layers * P.pairs * sizeof(int));
+    V.off_part_ml = off;
+    off = align_up(off + (size_t)P.layers * P.pairs * P.dec_slots * P.Gp * sizeof(float2));
+    V.off_part_acc = off;
+    off = align_up(off + (size_t)P.layers * P.pairs * P.dec_slots * P.Gp * P.D * sizeof(float));
+    V.ws_bytes = off;
+    return V;
+}
+
+}  // namespace
+}  // namespace bsa
+
+extern "C" bsa_status_t bsa_sparse_decode_noalloc(const bsa_params_t* params, const void* q,
+                                                  const void* k_cache, const void* v_cache,
+                                                  const int32_t* seq_lens,
+                                                  const int32_t* block_idx, const int32_t* n_sel,
+                                                  void* out, float* lse, uint32_t* device_error,
+                                                  cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if (!ok16(q) || !ok16(k_cache) || !ok16(v_cache) || !ok16(out) || !ok4(seq_lens) ||
+        !ok4(block_idx) || !ok4(n_sel))
+        return BSA_ERR_INVALID_ARG;
+    if ((lse && !ok4(lse)) || (device_error && !ok4(device_error))) return BSA_ERR_INVALID_ARG;
+    const Plan V = noalloc_layout(P);
+    if (V.ws_bytes > kNoAllocScratchBytes) return BSA_ERR_WORKSPACE;  // before any CUDA call
+    void* scratch = nullptr;
+    if ((st = noalloc_scratch(&scratch)) != BSA_OK) return st;
+    // error word and counters must start at zero: clear them on the stream, ahead of the kernel
+    if (cudaMemsetAsync(scratch, 0, V.off_part_ml, stream) != cudaSuccess) return BSA_ERR_CUDA;
+    DecodeArgs a = decode_args(V, seq_lens, block_idx, n_sel, scratch);
+    if (device_error) a.err = device_error;
+    a.q[0] = q;
+    a.k[0] = k_cache;
+    a.v[0] = v_cache;
+    a.out[0] = out;
+    a.lse[0] = lse;
+    static thread_local KVMaps maps;
+    if ((st = make_maps(P, a, 1, &maps)) != BSA_OK) return st;
+    return from_cuda(launch_decode(P, a, &maps, 1, stream));
+}

@@ -20,7 +20,8 @@
  * Conventions for every entry point:
  *   - All tensors are dense, row-major, on the current CUDA device, owned by the caller. The
  *     library allocates no memory and keeps no state between calls except inside the caller's
- *     workspace. Pointers must be 16-byte aligned.
+ *     workspace (bsa_sparse_decode_noalloc, at the end, uses a fixed scratch array instead).
+ *     Pointers must be 16-byte aligned.
  *   - Every call is asynchronous on `stream` (cudaStream_t; 0 = legacy default stream) and does
  *     not synchronize, except bsa_read_device_error.
  *   - Arguments are validated on the host before anything is launched; a rejected call returns a
@@ -194,6 +195,42 @@ bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_
  * synchronize `stream`. Returns BSA_ERR_DEVICE_CHECK when a bit was set, BSA_OK otherwise. */
 bsa_status_t bsa_read_device_error(void* workspace, size_t workspace_bytes, uint32_t* flags,
                                    cudaStream_t stream);
+
+/* Size of the fixed device scratch of bsa_sparse_decode_noalloc, per device: 4 MiB. */
+#define BSA_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* bsa_sparse_decode for callers that cannot allocate device memory, and so cannot provide a
+ * workspace. Examples are a host runtime whose allocator must not be entered from the calling
+ * thread, and a process with a fixed memory budget that has no room for a second buffer. The
+ * paper has no counterpart: it is a deployment variant of the step 5 entry point. It computes
+ * the same results with the same kernels and allocates nothing: no cudaMalloc, no allocating
+ * library routine.
+ *
+ * Scratch: the split partials and per-pair completion counters live in a fixed array inside
+ * libbsa, BSA_NOALLOC_SCRATCH_BYTES per device.
+ *   - Size limit. A parameter set whose partials do not fit returns BSA_ERR_WORKSPACE before any
+ *     CUDA call and launches nothing. The partials need about
+ *     B*Hkv*num_layers*Gp*(d + 2)*4 bytes per partial slot, where Gp is G rounded up to a power
+ *     of two. For example, B=16, Hkv=8, G=4, d=128 with 69 selected blocks needs 1.3 MiB.
+ *   - First call on a device. It looks up the array's device address (cudaGetSymbolAddress), with
+ *     that device current. The lookup may load the library's device code. Make the first call on
+ *     each device outside any stream capture.
+ *   - Zeroing. The counters and the scratch's error word must start at zero. Every call clears
+ *     them with a cudaMemsetAsync on `stream` ahead of its kernel.
+ *   - Concurrency. All calls on one device share the one array. Calls that overlap on the GPU
+ *     (different streams without an event between them, or several host threads) race on it and
+ *     give wrong results. Calls on one stream are ordered and safe.
+ *
+ * device_error: optional device pointer to a caller-owned, 4-byte aligned word.
+ *   - If it is given, device-side error bits (bsa_device_error_t) are OR-ed into it. The caller
+ *     zeroes the word and reads it back.
+ *   - If it is NULL, they go to the scratch's error word and are not reported.
+ * Other arguments, layouts and results are those of bsa_sparse_decode for one layer. */
+bsa_status_t bsa_sparse_decode_noalloc(const bsa_params_t* params, const void* q,
+                                       const void* k_cache, const void* v_cache,
+                                       const int32_t* seq_lens, const int32_t* block_idx,
+                                       const int32_t* n_sel, void* out, float* lse,
+                                       uint32_t* device_error, cudaStream_t stream);
 
 #ifdef __cplusplus
 }
