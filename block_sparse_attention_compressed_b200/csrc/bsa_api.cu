@@ -62,6 +62,7 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
     P.T_cap = q.max_seq_len;
     P.nc_cap = num_windows(P.T_cap, P.l, P.s);
     P.nb_cap = (P.T_cap + P.BS - 1) / P.BS;
+    P.lg_stride = (P.nc_cap + 3) / 4 * 4;
     if (P.nb_cap > kMaxNbCap) return BSA_ERR_UNSUPPORTED;
     P.pairs = (int)pairs;
     const double log2e = 1.4426950408889634;
@@ -95,6 +96,14 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
                             ? (size_t)P.nb_cap : (size_t)(2 * P.nstat * P.Gp);
         P.select_smem = (P.select_keys + (size_t)pw + (size_t)wmax) * sizeof(uint32_t);
         if (P.select_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
+        // one part per pair: the pair's logits stream through a ring of 16 KB shared-memory stages
+        P.select_ring = 0;
+        if (P.select_parts == 1) {
+            const size_t rest = 1024 + P.select_smem;
+            int64_t ring = ((size_t)220 * 1024 > rest) ? ((size_t)220 * 1024 - rest) / (16 * 1024) : 0;
+            if (ring > 8) ring = 8;
+            if (ring >= 2) P.select_ring = (int)ring;
+        }
     }
     // Decode split: about eight blocks per SM slot in flight, whole blocks per CTA.
     {
@@ -131,7 +140,7 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
     P.off_dec_cnt = off;
     off = align_up(off + (size_t)P.layers * P.pairs * sizeof(int));
     P.off_logits = off;
-    off = align_up(off + (size_t)P.pairs * P.nc_cap * P.Gp * sizeof(float));
+    off = align_up(off + (size_t)P.pairs * P.lg_stride * P.Gp * sizeof(float));
     P.off_stats = off;
     off = align_up(off + (size_t)P.pairs * P.nstat * P.Gp * sizeof(float2));
     P.off_bscores = off;
@@ -178,6 +187,7 @@ ScoreArgs score_args(const Plan& P, const void* q, const void* ck, const int32_t
     a.s = P.s;
     a.T_cap = P.T_cap;
     a.nc_cap = P.nc_cap;
+    a.lg_stride = P.lg_stride;
     a.nchunk = P.nchunk;
     a.total_chunks = P.total_chunks;
     a.nstat = P.nstat;
@@ -211,8 +221,10 @@ SelectArgs select_args(const Plan& P, const int32_t* seq_lens, int32_t* block_id
     a.T_cap = P.T_cap;
     a.nc_cap = P.nc_cap;
     a.nb_cap = P.nb_cap;
+    a.lg_stride = P.lg_stride;
     a.nstat = P.nstat;
     a.key_words = (int64_t)P.select_keys;
+    a.ring = P.select_ring;
     a.parts = P.select_parts;
     a.part_windows = P.select_part_windows;
     return a;

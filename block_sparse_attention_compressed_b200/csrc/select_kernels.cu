@@ -232,7 +232,7 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 2)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);  // the data is in registers: refill the slot
-            float* lg = a.logits + (size_t)md.pair * a.nc_cap * a.Gp;
+            float* lg = a.logits + (size_t)md.pair * a.lg_stride * a.Gp;
             float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
@@ -289,7 +289,7 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_f32_kernel(ScoreArgs a
         const int64_t r0 = ci * 64, r1 = min(r0 + 64, nc);
         if (r0 >= r1) continue;
         const float* ckp = reinterpret_cast<const float*>(a.ck) + (size_t)pair * a.nc_cap * D;
-        float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
+        float* lg = a.logits + (size_t)pair * a.lg_stride * a.Gp;
         float m[kMaxG], s[kMaxG];
 #pragma unroll
         for (int h = 0; h < kMaxG; ++h) {
@@ -604,7 +604,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
             part == parts_used - 1 ? nb : min(first_block_from(j1, a.BS, a.l, a.s), nb);
         const int64_t jend = b_hi > b_lo ? min(last_window(b_hi - 1, a.BS, a.s) + 1, nc) : j0;
         if (jend > j0) {
-            const float* lg = a.logits + (size_t)pair * a.nc_cap * a.Gp;
+            const float* lg = a.logits + (size_t)pair * a.lg_stride * a.Gp;
             window_scores<GP>(lg, j0, jend, a.G, sM, sInvZ, S);
         }
         __syncthreads();
@@ -636,6 +636,135 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
     for (int64_t b = tid; b < nb; b += kSelectThreads) s_dyn[b] = order_key(ld_cg(bs + b));
     __syncthreads();
     topk_union(a, pair, (int)nb, s_dyn);
+}
+
+// One CTA per pair, when there are enough pairs to fill the GPU: the pair's logits stream into a
+// ring of 16 KB shared-memory stages with 1-D bulk copies (all stages in flight at once, while the
+// chunk statistics are merged), S[j] is evaluated from shared memory, the block maxima go straight
+// to the key array and the top-k follows, with no completion counter.
+constexpr int kRingStage = 16 * 1024;
+constexpr int kMaxRing = 8;
+
+template <int GP>
+__global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(SelectArgs a) {
+    extern __shared__ __align__(128) uint8_t s_raw[];
+    __shared__ __align__(8) uint64_t full[kMaxRing];
+    __shared__ float sM[kMaxG], sInvZ[kMaxG];
+    uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_raw) + 127) & ~uintptr_t(127));
+    uint32_t* keys = reinterpret_cast<uint32_t*>(ring + (size_t)a.ring * kRingStage);
+    float* S = reinterpret_cast<float*>(keys + a.key_words);
+    const int pair = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int R = a.ring;
+    if (tid == 0) {
+        for (int r = 0; r < R; ++r) mbar_init(&full[r], 1);
+        mbar_fence_init();
+    }
+    __syncthreads();
+    pdl_trigger();
+    pdl_wait();
+    const int64_t T = a.seq_lens[pair / a.Hkv];
+    const bool ok = T >= 0 && T <= a.T_cap;
+    const int nc = ok ? (int)num_windows(T, a.l, a.s) : 0;
+    const int nb = ok ? (int)((T + a.BS - 1) / a.BS) : 0;
+    constexpr int PW = kRingStage / (GP * 4);  // windows per stage
+    const int npieces = (nc + PW - 1) / PW;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(a.logits + (size_t)pair * a.lg_stride * GP);
+    auto issue = [&](int r) {  // thread 0: stage r of the pair's logits into ring slot r % R
+        const int w0 = r * PW, wn = min(PW, nc - w0);
+        const uint32_t bytes = ((uint32_t)wn * GP * 4 + 15u) & ~15u;  // inside the padded row
+        uint64_t* bar = &full[r % R];
+        mbar_arrive_expect_tx(bar, bytes);
+        bulk_load(ring + (size_t)(r % R) * kRingStage, src + (size_t)w0 * GP * 4, bytes, bar);
+    };
+    if (tid == 0)
+        for (int r = 0; r < npieces && r < R; ++r) issue(r);
+
+    // softmax normaliser of every head from the chunk statistics (staged in the key array)
+    {
+        const int nch = (nc + 63) / 64;
+        float2* s_st = reinterpret_cast<float2*>(keys);  // 2 * nstat * Gp <= key_words
+        const float2* st = a.stats + (size_t)pair * a.nstat * GP;
+        for (int e = tid; e < nch * GP; e += kSelectThreads) s_st[e] = ld_cg(st + e);
+        __syncthreads();
+        if (warp < a.G) {
+            float m = -INFINITY, sum = 0.f;
+            for (int c = lane; c < nch; c += 32) {
+                const float2 v = s_st[c * GP + warp];
+                online_merge(m, sum, v.x, v.y);
+            }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) {
+                const float mo = __shfl_xor_sync(0xffffffffu, m, off);
+                const float so = __shfl_xor_sync(0xffffffffu, sum, off);
+                online_merge(m, sum, mo, so);
+            }
+            if (lane == 0) {
+                sM[warp] = m;
+                sInvZ[warp] = sum > 0.f ? 1.f / sum : 0.f;
+            }
+        }
+        __syncthreads();
+    }
+    float M[GP], iz[GP];
+#pragma unroll
+    for (int h = 0; h < GP; ++h) {
+        M[h] = h < a.G ? sM[h] : 0.f;
+        iz[h] = h < a.G ? sInvZ[h] : 0.f;
+    }
+    // S[j] = sum_h exp2(x[j][h] - M_h) / Z_h, stage by stage
+    for (int r = 0; r < npieces; ++r) {
+        if (!mbar_wait(&full[r % R], (r / R) & 1, kScoreWaitPolls)) {
+            if (tid == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+            break;
+        }
+        const float* lg = reinterpret_cast<const float*>(ring + (size_t)(r % R) * kRingStage);
+        const int w0 = r * PW, wn = min(PW, nc - w0);
+        for (int i = tid; i < wn; i += kSelectThreads) {
+            float x[GP];
+            if constexpr (GP == 1) {
+                x[0] = lg[i];
+            } else if constexpr (GP == 2) {
+                const float2 t = reinterpret_cast<const float2*>(lg)[i];
+                x[0] = t.x;
+                x[1] = t.y;
+            } else {
+#pragma unroll
+                for (int q = 0; q < GP / 4; ++q) {
+                    const float4 t = reinterpret_cast<const float4*>(lg + (size_t)i * GP)[q];
+                    x[4 * q] = t.x;
+                    x[4 * q + 1] = t.y;
+                    x[4 * q + 2] = t.z;
+                    x[4 * q + 3] = t.w;
+                }
+            }
+            float acc = 0.f;
+#pragma unroll
+            for (int h = 0; h < GP; ++h)
+                if (h < a.G) acc += exp2f(x[h] - M[h]) * iz[h];
+            S[w0 + i] = acc;
+        }
+        __syncthreads();  // the slot has been read by everyone
+        if (tid == 0 && r + R < npieces) {
+            fence_proxy_async_smem();
+            issue(r + R);
+        }
+    }
+    __syncthreads();
+    // block scores: the maximum of S over the complete windows overlapping each block
+    for (int b = tid; b < nb; b += kSelectThreads) {
+        float best = -INFINITY;
+        const int jlo = (int)first_window32(b, a.BS, a.l, a.s);
+        const int jhi = min((int)last_window32(b, a.BS, a.s), nc - 1);
+        for (int j = jlo; j <= jhi; ++j) best = fmaxf(best, S[j]);
+        keys[b] = order_key(best);
+        if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + b] = best;
+    }
+    if (a.block_scores)
+        for (int64_t b = nb + tid; b < a.nb_cap; b += kSelectThreads)
+            a.block_scores[(size_t)pair * a.nb_cap + b] = -INFINITY;
+    __syncthreads();
+    topk_union(a, pair, nb, keys);
 }
 
 int sm_count() {
@@ -684,6 +813,15 @@ cudaError_t launch_score_tma(const Plan& p, const ScoreArgs& a, const CUtensorMa
 
 template <int GP>
 cudaError_t launch_select_k(const Plan& p, const SelectArgs& a, cudaStream_t st) {
+    if (p.select_ring > 0) {
+        const size_t smem = 128 + (size_t)p.select_ring * kRingStage +
+                            (p.select_keys + (size_t)p.select_part_windows) * sizeof(uint32_t);
+        cudaError_t e = cudaFuncSetAttribute(select_single_kernel<GP>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(select_single_kernel<GP>, dim3((unsigned)p.pairs), dim3(kSelectThreads),
+                          smem, st, a);
+    }
     if (p.select_smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(select_kernel<GP>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
