@@ -227,8 +227,9 @@ class Bench:
         return (["append"] + names) if (self.append and self.w.layers == 1) else names
 
     def launches_per_step(self):
-        # bsa_select_blocks launches two kernels (scoring, selection); the others one each
-        return len(self.kernel_names()) + 1
+        # bsa_select_blocks launches two kernels (scoring, selection), the bf16 sparse attention two
+        # (attention, combine), the fp32 one one, the append one
+        return len(self.kernel_names()) + 1 + (1 if self.w.dtype == "bf16" else 0)
 
     def reset_lengths(self):
         self.data["seq_lens"].copy_(self.seq0)

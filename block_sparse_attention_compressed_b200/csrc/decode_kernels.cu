@@ -59,8 +59,12 @@ struct Group {
     }
 };
 
+template <typename T, int D>
+__device__ void combine_partials(const DecodeArgs& a, int layer, int pair, int lp, int S,
+                                 float2* s_ml, const Group gp);
+
 // Merge of the warp states, split partial write, and the cross-split combine by the last split of
-// the (layer, pair) to finish.
+// the (layer, pair) to finish (fp32 path).
 template <typename T, int D>
 __device__ void finish_split(const DecodeArgs& a, int layer, int pair, int lp, int slot, int nslots,
                              const MergeView sm, float2* s_ml /* nslots * Gp */, const Group gp) {
@@ -96,11 +100,17 @@ __device__ void finish_split(const DecodeArgs& a, int layer, int pair, int lp, i
     gp.sync();
     if (!s_last) return;
     __threadfence();
-    // Combine the splits: per head the global max M and denominator, per split a scale factor
-    // exp2(m_s - M) (shared memory), then every (head, d) element sums its scaled numerators with
-    // the loads of kU splits in flight.
+    combine_partials<T, D>(a, layer, pair, lp, nslots, s_ml, gp);
+}
+
+// Combine the S partials of a (layer, pair) into O and LSE: per head the global max M and
+// denominator, per partial a scale factor exp2(m_s - M) (shared memory), then every (head, d)
+// element sums its scaled numerators with the loads of kU partials in flight.
+template <typename T, int D>
+__device__ void combine_partials(const DecodeArgs& a, int layer, int pair, int lp, int S,
+                                 float2* s_ml /* S * Gp */, const Group gp) {
     __shared__ float s_M[kMaxG], s_den[kMaxG];
-    const int S = nslots;
+    const int G = a.G, NT = gp.nthreads;
     const float2* ml0 = a.part_ml + (size_t)lp * a.slots * a.Gp;
     const float* acc0 = a.part_acc + (size_t)lp * a.slots * a.Gp * D;
     for (int e = gp.tid; e < S * a.Gp; e += NT) s_ml[e] = ld_cg(ml0 + e);  // one round
@@ -143,6 +153,36 @@ __device__ void finish_split(const DecodeArgs& a, int layer, int pair, int lp, i
     }
 }
 
+// bf16 path: merge of the consumer warps' states into partial `slot` of a (layer, pair). The
+// partials are combined by a second kernel once the whole grid has finished, so no fence or
+// completion count is needed here.
+template <int D>
+__device__ void write_partial(const DecodeArgs& a, int lp, int slot, const MergeView sm,
+                              const Group gp) {
+    gp.sync();
+    const int G = a.G, NT = gp.nthreads;
+    float2* pml = a.part_ml + ((size_t)lp * a.slots + slot) * a.Gp;
+    float* pacc = a.part_acc + ((size_t)lp * a.slots + slot) * a.Gp * D;
+    for (int e = gp.tid; e < G * D; e += NT) {
+        const int h = e / D, dd = e - h * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kDecodeWarps; ++w) M = fmaxf(M, sm.M(w, h));
+        float num = 0.f, den = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < kDecodeWarps; ++w) {
+                const float f = exp2f(sm.M(w, h) - M);
+                num = fmaf(f, sm.acc[(w * G + h) * D + dd], num);
+                den = fmaf(f, sm.L(w, h), den);
+            }
+        }
+        pacc[h * D + dd] = num;
+        if (dd == 0) pml[h] = make_float2(M, den);
+    }
+    gp.sync();  // the merge area is free for the next segment
+}
+
 // Which blocks this CTA owns, and the sequence facts every warp needs.
 struct SplitInfo {
     int64_t T, nb;
@@ -179,6 +219,7 @@ constexpr int kTmaThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kMaxStages = 8;
 constexpr uint32_t kWaitPolls = 1u << 26;  // far beyond any legitimate wait; then give up
 constexpr uint32_t kQSlot = 1024;          // bytes per stage for q of the group (G * D * 2 <= 2048)
+constexpr int kCombineThreads = 128;
 
 enum : int { kStageFirst = 1, kStageLast = 2, kStageEnd = 4 };
 
@@ -199,8 +240,8 @@ __device__ __forceinline__ int cta_of_slot(int64_t x, int64_t N, int C) {
 // Persistent: the N = layers * pairs * SEL_cap block slots are shared evenly by C CTAs; CTA c walks
 // slots [c*N/C, (c+1)*N/C). The producer lane streams every stage of its slots through the ring
 // without draining; where its range crosses from one (layer, pair) to the next, the consumer warps
-// flush the segment (merge, partial, and the combine when it is the pair's last segment) behind a
-// named barrier while the next stages are already loading.
+// flush the segment (merge into the segment's partial) behind a named barrier while the next
+// stages are already loading. combine_kernel then merges each (layer, pair)'s partials.
 template <int D>
 __global__ void __launch_bounds__(kTmaThreads, 2)
     decode_tma_kernel(const DecodeArgs a, const __grid_constant__ KVMaps maps, const int nstages,
@@ -218,7 +259,6 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
     float* mbase = reinterpret_cast<float*>(ring + (size_t)nstages * stage_bytes);
     const MergeView sm{mbase, mbase + kDecodeWarps * kMaxG, mbase + 2 * kDecodeWarps * kMaxG};
-    float2* s_ml = reinterpret_cast<float2*>(reinterpret_cast<uint8_t*>(mbase) + merge_bytes(a.G, D));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, tq = lane & 3;
     const bool producer = warp == kConsumerWarps;
@@ -465,8 +505,7 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
                         w1[d0 + 8] = acc[mt][3];
                     }
                 }
-                const int layer = md.lp / a.pairs, pair = md.lp - layer * a.pairs;
-                finish_split<__nv_bfloat16, D>(a, layer, pair, md.lp, md.seg, md.nseg, sm, s_ml, gp);
+                write_partial<D>(a, md.lp, md.seg, sm, gp);
                 m[0] = m[1] = -INFINITY;
                 lsum[0] = lsum[1] = 0.f;
 #pragma unroll
@@ -568,6 +607,22 @@ cudaError_t launch_decode_k(K kernel, const Plan& p, const DecodeArgs& a, int la
     return launch_pdl(kernel, dim3((unsigned)grid), dim3(kDecodeThreads), 0, st, a);
 }
 
+// bf16 path: one CTA per (layer, pair) merges, in segment order, the partials of the CTAs whose
+// shares cover it, once the attention grid has finished.
+template <int D>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const DecodeArgs a, const int64_t n_slots,
+                                                                  const int C) {
+    __shared__ float2 s_ml[kMaxCombineSlots];
+    pdl_trigger();
+    pdl_wait();
+    const int lp = blockIdx.x;
+    const int layer = lp / a.pairs, pair = lp - layer * a.pairs;
+    const int c_first = cta_of_slot((int64_t)lp * a.sel_cap, n_slots, C);
+    const int c_last = cta_of_slot((int64_t)(lp + 1) * a.sel_cap - 1, n_slots, C);
+    combine_partials<__nv_bfloat16, D>(a, layer, pair, lp, c_last - c_first + 1, s_ml,
+                                       Group{(int)threadIdx.x, (int)blockDim.x, 0});
+}
+
 template <int D>
 cudaError_t launch_decode_tma(const Plan& p, const DecodeArgs& a, const KVMaps* maps, int layers,
                               cudaStream_t st) {
@@ -579,7 +634,7 @@ cudaError_t launch_decode_tma(const Plan& p, const DecodeArgs& a, const KVMaps* 
     const size_t qslot = kQSlot * (((size_t)a.G * D * 2 + kQSlot - 1) / kQSlot);
     const size_t stage_bytes = (size_t)2 * (D / 64) * a.stage_tokens * 128 + qslot;
     // two CTAs per SM: ~112 KB each, of which the merge and combine scratch take a few KB
-    const size_t scratch = merge_bytes(a.G, D) + sizeof(float2) * (size_t)a.slots * a.Gp;
+    const size_t scratch = merge_bytes(a.G, D);
     const size_t budget = 112 * 1024 - 1024 - scratch;
     int nstages = (int)(budget / stage_bytes);
     if (nstages < 2) nstages = 2;
@@ -588,8 +643,12 @@ cudaError_t launch_decode_tma(const Plan& p, const DecodeArgs& a, const KVMaps* 
     cudaError_t e = cudaFuncSetAttribute(decode_tma_kernel<D>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(decode_tma_kernel<D>, dim3((unsigned)ctas), dim3(kTmaThreads), smem, st, a,
-                      *maps, nstages, n_slots);
+    e = launch_pdl(decode_tma_kernel<D>, dim3((unsigned)ctas), dim3(kTmaThreads), smem, st, a, *maps,
+                   nstages, n_slots);
+    if (e != cudaSuccess) return e;
+    const int64_t lps = (int64_t)layers * p.pairs;
+    return launch_pdl(combine_kernel<D>, dim3((unsigned)lps), dim3(kCombineThreads), 0, st, a, n_slots,
+                      (int)ctas);
 }
 
 }  // namespace
