@@ -385,8 +385,10 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
     __shared__ int s_warp[32];
     __shared__ int hist[256];
     __shared__ uint32_t s_prefix;
-    __shared__ int s_need;
+    __shared__ int s_need, s_bcnt, s_bn;
     __shared__ uint32_t s_and[32], s_or[32];
+    __shared__ uint32_t s_bkey[32];
+    __shared__ int s_bidx[32], s_btake[32];
     const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31;
     const int init_end = min(a.n_init, nb);
     const int local_begin = max(nb - a.n_local, 0);
@@ -403,6 +405,12 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
 
     uint32_t thr = 0xffffffffu;  // keys > thr are taken, plus the first `need` keys == thr
     int need = 0;
+    // Early finish: once the digit bucket that holds the k-th key has at most 32 keys, one warp
+    // ranks them exactly (score descending, block ascending); then the candidates taken are those
+    // above the bucket plus the bucket keys ranked below `need`.
+    bool exact = false;
+    uint32_t emask = 0u, eprefix = 0u;
+    int ebn = 0;
     if (kk > 0 && !take_all) {
         // bytes that every candidate shares need no histogram pass: start at the first byte in
         // which two candidates differ (block-wide AND / OR of the keys)
@@ -442,6 +450,7 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
         need = kk;
         for (int shift = top; shift >= 0; shift -= 8) {
             for (int i = tid; i < 256; i += NT) hist[i] = 0;
+            if (tid == 0) s_bn = 0;
             __syncthreads();
             // warp-aggregated histogram (keys of a warp often share a digit): one atomic per
             // distinct digit per warp; all of a thread's keys are processed independently
@@ -489,6 +498,7 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
                         if (acc < need && acc + c[k] >= need) {
                             s_prefix = prefix | ((uint32_t)(255 - 8 * tid - k) << shift);
                             s_need = need - acc;
+                            s_bcnt = c[k];
                         }
                         acc += c[k];
                     }
@@ -498,11 +508,53 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
             prefix = s_prefix;
             need = s_need;
             mask |= 255u << shift;
+            if (in_regs && shift > 0 && s_bcnt <= 32) {
+                exact = true;
+                break;
+            }
         }
         thr = prefix;
+        if (exact) {
+            emask = mask;
+            eprefix = prefix;
+#pragma unroll
+            for (int e = 0; e < kKeysPerThread; ++e) {
+                if (seg_lo + e < seg_hi && (kr[e] & mask) == prefix) {
+                    const int slot = atomicAdd(&s_bn, 1);
+                    s_bkey[slot] = kr[e];
+                    s_bidx[slot] = seg_lo + e;
+                }
+            }
+            __syncthreads();
+            ebn = s_bn;
+            if (tid < 32) {
+                const uint32_t key = tid < ebn ? s_bkey[tid] : 0u;
+                const int idx = tid < ebn ? s_bidx[tid] : 0x7fffffff;
+                int rank = 0;
+                for (int j = 0; j < ebn; ++j) {
+                    const uint32_t kj = s_bkey[j];
+                    const int ij = s_bidx[j];
+                    rank += (kj > key || (kj == key && ij < idx));
+                }
+                if (tid < ebn) s_btake[tid] = rank < need ? idx : -1;
+            }
+            __syncthreads();
+        }
     }
-    // mark the taken candidates in index order (equal keys: lowest block first)
-    {
+    if (exact) {
+        // above the bucket, or ranked within it
+#pragma unroll
+        for (int e = 0; e < kKeysPerThread; ++e) {
+            if (seg_lo + e < seg_hi) {
+                const uint32_t mk = kr[e] & emask;
+                bool take = mk > eprefix;
+                if (mk == eprefix)
+                    for (int j = 0; j < ebn; ++j) take |= s_btake[j] == seg_lo + e;
+                keys[seg_lo + e] = take ? 1u : 0u;
+            }
+        }
+    } else {
+        // mark the taken candidates in index order (equal keys: lowest block first)
         int cnt = 0;
         if (in_regs) {
 #pragma unroll
