@@ -149,6 +149,9 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 2)
 
     if (warp == kScoreConsumers) {
         if (lane == 0) {
+            // the compressed keys are read once: keep the window logits (reread by the
+            // selection) in L2 rather than them
+            const uint64_t ck_policy = l2_evict_first_policy();
             int k = 0, cur_pair = -1;
             int64_t nc = 0;
             bool ok = true;
@@ -178,7 +181,8 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 2)
                 mbar_arrive_expect_tx(&full[st], stage_bytes);
                 const int y = (int)((int64_t)pair * a.nc_cap + row0);
 #pragma unroll
-                for (int bi = 0; bi < NB; ++bi) tma_load_2d(dst + bi * box_bytes, &ck_map, 64 * bi, y, &full[st]);
+                for (int bi = 0; bi < NB; ++bi)
+                    tma_load_2d_hint(dst + bi * box_bytes, &ck_map, 64 * bi, y, &full[st], ck_policy);
                 ++k;
             }
             // end-of-stream markers, one per consumer warp (each waits on its own stages only)
