@@ -278,6 +278,8 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
 
     if (producer) {
         if (lane == 0) {
+            // the selected K/V rows are read once: keep the partials (reread by the combine) in L2
+            const uint64_t kv_policy = l2_evict_first_policy();
             const int sub_per_block = a.BS / ST;
             int k = 0;
             bool ok = true;
@@ -340,10 +342,11 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
                         const int y = (int)(row_base + tok0);
 #pragma unroll
                         for (int bi = 0; bi < NB; ++bi)
-                            tma_load_2d(dst + bi * box_bytes, &maps.k[layer], 64 * bi, y, &full[st]);
+                            tma_load_2d_hint(dst + bi * box_bytes, &maps.k[layer], 64 * bi, y, &full[st], kv_policy);
 #pragma unroll
                         for (int bi = 0; bi < NB; ++bi)
-                            tma_load_2d(dst + (NB + bi) * box_bytes, &maps.v[layer], 64 * bi, y, &full[st]);
+                            tma_load_2d_hint(dst + (NB + bi) * box_bytes, &maps.v[layer], 64 * bi, y, &full[st],
+                                             kv_policy);
                         if (first) {
                             bulk_load(dst + kv_bytes, qsrc, qb, &full[st]);
                             q_lp = lp;
