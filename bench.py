@@ -10,10 +10,12 @@ growing-cache workload: the token append with its compressed-key update first).
 Prints one JSON line. ``value`` is decode steps/s over all ranks (weak scaling: every rank runs its
 own copy of the workload on its own GPU, no collective on the data path), device-timed with CUDA
 events between barriers + synchronizes, max over ranks. ``e2e`` is the same metric through the
-Python binding with q copied in from pinned host memory and the output copied back every step.
+Python binding, with every step's inputs (each layer's q; the new k/v rows when the cache grows)
+copied in from pinned host memory and its outputs (every layer) copied back. The copies are
+double-buffered on two copy streams, so a step's transfers overlap its neighbours' compute.
 ``roofline`` is for the largest single kernel of the step (the sparse attention), from a second,
-identical pass that brackets every library call with CUDA events. ``cpu_baseline`` (rank 0, one GPU only) and
-``--impl reference`` time the CPU oracle on a bounded sample of the same workload.
+identical pass that brackets every library call with CUDA events. ``cpu_baseline`` (rank 0, one
+GPU only) and ``--impl reference`` time the CPU oracle on a bounded sample of the same workload.
 """
 from __future__ import annotations
 
@@ -222,6 +224,19 @@ class Bench:
                               self.n_sel, self.out[0], self.lse[0], self.ws, stream=stream)
         ev(k + 2)
 
+    # one step with caller-given input and output buffers (the end-to-end pass)
+    def step_io(self, qs, outs, lses, stream, k_new=None, v_new=None):
+        bsa, d = self.bsa, self.data
+        if self.w.layers > 1:
+            bsa.bsa_select_blocks(self.p, qs[0], self.ck, d["seq_lens"], self.block_idx, self.n_sel,
+                                  None, self.ws, stream=stream)
+            bsa.bsa_sparse_decode_layers(self.p, qs, d["k"], d["v"], d["seq_lens"], self.block_idx,
+                                         self.n_sel, outs, lses, self.ws, stream=stream)
+            return
+        bsa.bsa_decode_step(self.p, qs[0], d["k"][0], d["v"][0], self.ck, k_new, v_new, d["seq_lens"],
+                            self.block_idx, self.n_sel, None, outs[0], lses[0], self.ws,
+                            stream=stream)
+
     def kernel_names(self):
         names = ["select", "decode"]
         return (["append"] + names) if (self.append and self.w.layers == 1) else names
@@ -410,47 +425,76 @@ def run_bsa(args, w, world, rank, local):
     kern_ms = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
                for j, n in enumerate(names)}
 
-    # ---- e2e: through the binding, q from pinned host memory in, output back out, every step
-    q_host = [bench.q_of(W + i if bench.append else 0).cpu().pin_memory() for i in range(K)]
-    q_dev = torch.empty_like(bench.q_of(0))
-    out_host = torch.empty(bench.out[0].shape, dtype=bench.out[0].dtype).pin_memory()
+    # ---- e2e: through the binding, every step's inputs copied in from pinned host memory and its
+    # outputs (every layer) copied back, double-buffered: step i+1's inputs land and step i's
+    # outputs return on copy streams while step i+1 computes
+    import torch as _t
+    L_ = w.layers
+    NBUF = 2
+    def step_q(i):  # the query of every layer for timed step i
+        return [bench.q_of(W + i if bench.append else 0)] + [bench.data["q"][l] for l in range(1, L_)]
+    q_host = [[t.cpu().pin_memory() for t in step_q(i)] for i in range(K)]
+    q_dev = [[_t.empty_like(t) for t in step_q(0)] for _ in range(NBUF)]
+    out_dev = [[_t.empty_like(bench.out[l]) for l in range(L_)] for _ in range(NBUF)]
+    lse_dev = [[_t.empty_like(bench.lse[l]) for l in range(L_)] for _ in range(NBUF)]
+    out_host = [[_t.empty(bench.out[l].shape, dtype=bench.out[l].dtype).pin_memory() for l in range(L_)]
+                for _ in range(NBUF)]
     if bench.append:
         bench.reset_lengths()
-        with torch.cuda.stream(stream):
+        with _t.cuda.stream(stream):
             for i in range(W):
                 bench.step(i, stream)
         kn_host = [bench.data["k_new"][W + i].cpu().pin_memory() for i in range(K)]
         vn_host = [bench.data["v_new"][W + i].cpu().pin_memory() for i in range(K)]
-        kn_dev, vn_dev = torch.empty_like(bench.data["k_new"][0]), torch.empty_like(bench.data["v_new"][0])
-    torch.cuda.synchronize()
+        kn_dev = [_t.empty_like(bench.data["k_new"][0]) for _ in range(NBUF)]
+        vn_dev = [_t.empty_like(bench.data["v_new"][0]) for _ in range(NBUF)]
+    h2d_stream = _t.cuda.Stream(device=dev)
+    d2h_stream = _t.cuda.Stream(device=dev)
+    ev_in = [_t.cuda.Event() for _ in range(NBUF)]
+    ev_step = [_t.cuda.Event() for _ in range(NBUF)]
+    ev_back = [_t.cuda.Event() for _ in range(NBUF)]
+    _t.cuda.synchronize()
     barrier(world)
-    torch.cuda.synchronize()
+    _t.cuda.synchronize()
     t_e2e0 = time.perf_counter()
-    with torch.cuda.stream(stream):
-        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a0.record(stream)
-        for i in range(K):
-            q_dev.copy_(q_host[i], non_blocking=True)
+    a0, a1 = _t.cuda.Event(enable_timing=True), _t.cuda.Event(enable_timing=True)
+    a0.record(stream)
+    h2d_stream.wait_event(a0)
+    d2h_stream.wait_event(a0)
+    for i in range(K):
+        j = i % NBUF
+        with _t.cuda.stream(h2d_stream):
+            if i >= NBUF:
+                h2d_stream.wait_event(ev_step[j])  # the step that last read buffer j is done
+            for l in range(L_):
+                q_dev[j][l].copy_(q_host[i][l], non_blocking=True)
             if bench.append:
-                kn_dev.copy_(kn_host[i], non_blocking=True)
-                vn_dev.copy_(vn_host[i], non_blocking=True)
-                d = bench.data
-                bsa_ = bench.bsa
-                bsa_.bsa_decode_step(bench.p, q_dev, d["k"][0], d["v"][0], bench.ck, kn_dev,
-                                     vn_dev, d["seq_lens"], bench.block_idx, bench.n_sel, None,
-                                     bench.out[0], bench.lse[0], bench.ws, stream=stream)
-            else:
-                bench.step(0, stream, q=q_dev)
-            out_host.copy_(bench.out[0], non_blocking=True)
-        a1.record(stream)
+                kn_dev[j].copy_(kn_host[i], non_blocking=True)
+                vn_dev[j].copy_(vn_host[i], non_blocking=True)
+            ev_in[j].record(h2d_stream)
+        stream.wait_event(ev_in[j])
+        if i >= NBUF:
+            stream.wait_event(ev_back[j])  # buffer j's outputs have been copied back
+        with _t.cuda.stream(stream):
+            bench.step_io(q_dev[j], out_dev[j], lse_dev[j], stream,
+                          kn_dev[j] if bench.append else None, vn_dev[j] if bench.append else None)
+        ev_step[j].record(stream)
+        with _t.cuda.stream(d2h_stream):
+            d2h_stream.wait_event(ev_step[j])
+            for l in range(L_):
+                out_host[j][l].copy_(out_dev[j][l], non_blocking=True)
+            ev_back[j].record(d2h_stream)
+    stream.wait_stream(h2d_stream)
+    stream.wait_stream(d2h_stream)
+    a1.record(stream)
     stream.synchronize()
     e2e_local = a0.elapsed_time(a1)
     e2e_ms = max_over_ranks(e2e_local, world)
     wall_e2e = time.perf_counter() - t_e2e0
-    h2d = q_host[0].numel() * q_host[0].element_size()
+    h2d = sum(t.numel() * t.element_size() for t in q_host[0])
     if bench.append:
         h2d += 2 * kn_host[0].numel() * kn_host[0].element_size()
-    d2h = out_host.numel() * out_host.element_size()
+    d2h = sum(o.numel() * o.element_size() for o in out_host[0])
 
     err = bench.bsa.bsa_read_device_error(bench.ws)
     if err:
