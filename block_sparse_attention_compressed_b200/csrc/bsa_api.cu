@@ -236,8 +236,9 @@ bsa_status_t do_select(const Plan& P, const void* q, const void* ck, const int32
                        cudaStream_t st) {
     ScoreArgs sa = score_args(P, q, ck, seq_lens, ws);
     static thread_local CUtensorMap ck_map;
+    static thread_local MapKey ck_key;
     if (P.dtype == BSA_BF16 && P.nc_cap > 0 &&
-        !encode_kv_map(&ck_map, ck, (uint64_t)P.pairs * P.nc_cap, P.D, 64))
+        !encode_kv_map_cached(&ck_map, &ck_key, ck, (uint64_t)P.pairs * P.nc_cap, P.D, 64))
         return BSA_ERR_CUDA;
     cudaError_t e = launch_score(P, sa, &ck_map, st);
     if (e != cudaSuccess) return BSA_ERR_CUDA;
@@ -274,12 +275,18 @@ DecodeArgs decode_args(const Plan& P, const int32_t* seq_lens, const int32_t* bl
 }
 
 // TMA descriptors of the layers' caches (bf16 path only).
-bsa_status_t make_maps(const Plan& P, const DecodeArgs& a, int layers, KVMaps* maps) {
+// (Each entry point keeps its descriptors, with the tensors they were encoded for, per thread.)
+struct KVMapCache {
+    KVMaps maps;
+    MapKey k[BSA_MAX_LAYERS], v[BSA_MAX_LAYERS];
+};
+
+bsa_status_t make_maps(const Plan& P, const DecodeArgs& a, int layers, KVMapCache* c) {
     if (P.dtype != BSA_BF16) return BSA_OK;
     const uint64_t rows = (uint64_t)P.pairs * (uint64_t)P.T_cap;
     for (int i = 0; i < layers; ++i) {
-        if (!encode_kv_map(&maps->k[i], a.k[i], rows, P.D, P.stage_tokens) ||
-            !encode_kv_map(&maps->v[i], a.v[i], rows, P.D, P.stage_tokens))
+        if (!encode_kv_map_cached(&c->maps.k[i], &c->k[i], a.k[i], rows, P.D, P.stage_tokens) ||
+            !encode_kv_map_cached(&c->maps.v[i], &c->v[i], a.v[i], rows, P.D, P.stage_tokens))
             return BSA_ERR_CUDA;
     }
     return BSA_OK;
@@ -434,9 +441,9 @@ bsa_status_t bsa_sparse_decode_layers(const bsa_params_t* params, int32_t num_la
         a.out[i] = outs[i];
         a.lse[i] = lse;
     }
-    static thread_local KVMaps maps;
+    static thread_local KVMapCache maps;
     if ((st = make_maps(P, a, num_layers, &maps)) != BSA_OK) return st;
-    return from_cuda(launch_decode(P, a, &maps, num_layers, stream));
+    return from_cuda(launch_decode(P, a, &maps.maps, num_layers, stream));
 }
 
 bsa_status_t bsa_sparse_decode(const bsa_params_t* params, const void* q, const void* k_cache,
@@ -481,9 +488,9 @@ bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_
     da.v[0] = v_cache;
     da.out[0] = out;
     da.lse[0] = lse;
-    static thread_local KVMaps maps;
+    static thread_local KVMapCache maps;
     if ((st = make_maps(P, da, 1, &maps)) != BSA_OK) return st;
-    return from_cuda(launch_decode(P, da, &maps, 1, stream));
+    return from_cuda(launch_decode(P, da, &maps.maps, 1, stream));
 }
 
 bsa_status_t bsa_read_device_error(void* ws, size_t ws_bytes, uint32_t* flags,
@@ -581,7 +588,7 @@ extern "C" bsa_status_t bsa_sparse_decode_noalloc(const bsa_params_t* params, co
     a.v[0] = v_cache;
     a.out[0] = out;
     a.lse[0] = lse;
-    static thread_local KVMaps maps;
+    static thread_local KVMapCache maps;
     if ((st = make_maps(P, a, 1, &maps)) != BSA_OK) return st;
-    return from_cuda(launch_decode(P, a, &maps, 1, stream));
+    return from_cuda(launch_decode(P, a, &maps.maps, 1, stream));
 }

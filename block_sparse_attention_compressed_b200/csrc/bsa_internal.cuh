@@ -137,6 +137,38 @@ cudaError_t launch_decode(const Plan& p, const DecodeArgs& a, const KVMaps* maps
 // Encode a 2-D bf16 TMA descriptor over rows x D elements (128-byte swizzle, box 64 x box_rows).
 bool encode_kv_map(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows);
 
+// The arguments `map` was last encoded for: calls with the same tensor skip the encode.
+struct MapKey {
+    const void* base = nullptr;
+    uint64_t rows = 0;
+    int D = 0, box = 0;
+};
+inline bool encode_kv_map_cached(CUtensorMap* map, MapKey* key, const void* base, uint64_t rows,
+                                 int D, int box_rows) {
+    if (base && key->base == base && key->rows == rows && key->D == D && key->box == box_rows)
+        return true;
+    key->base = nullptr;
+    if (!encode_kv_map(map, base, rows, D, box_rows)) return false;
+    key->base = base;
+    key->rows = rows;
+    key->D = D;
+    key->box = box_rows;
+    return true;
+}
+
+// Raise a kernel's dynamic shared-memory limit once per device (and size), not on every launch.
+template <auto Kernel>
+inline cudaError_t ensure_smem(size_t smem) {
+    static int done[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = -1;
+    if (dev >= 0 && dev < 64 && done[dev] >= (int)smem) return cudaSuccess;
+    const cudaError_t e =
+        cudaFuncSetAttribute(Kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess && dev >= 0 && dev < 64) done[dev] = (int)smem;
+    return e;
+}
+
 // Launch with programmatic dependent launch allowed: the kernel may start while the previous
 // kernel in the stream drains; every kernel here waits (griddepcontrol.wait) before touching
 // memory that an earlier kernel writes.

@@ -643,8 +643,7 @@ cudaError_t launch_decode_tma(const Plan& p, const DecodeArgs& a, const KVMaps* 
     if (nstages < 2) nstages = 2;
     if (nstages > kMaxStages) nstages = kMaxStages;
     const size_t smem = 1024 + (size_t)nstages * stage_bytes + scratch;
-    cudaError_t e = cudaFuncSetAttribute(decode_tma_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem<decode_tma_kernel<D>>(smem);
     if (e != cudaSuccess) return e;
     e = launch_pdl(decode_tma_kernel<D>, dim3((unsigned)ctas), dim3(kTmaThreads), smem, st, a, *maps,
                    nstages, n_slots);

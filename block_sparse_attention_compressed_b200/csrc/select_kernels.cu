@@ -860,8 +860,7 @@ cudaError_t launch_score_tma(const Plan& p, const ScoreArgs& a, const CUtensorMa
     nstages -= nstages % kScoreConsumers;
     if (nstages < kScoreConsumers) nstages = kScoreConsumers;
     const size_t smem = 1024 + (size_t)nstages * stage_bytes;
-    cudaError_t e = cudaFuncSetAttribute(score_tma_kernel<D>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = ensure_smem<score_tma_kernel<D>>(smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(score_tma_kernel<D>, dim3((unsigned)p.score_ctas), dim3(kScoreTmaThreads),
                       smem, st, a, *ck_map, nstages);
@@ -872,16 +871,13 @@ cudaError_t launch_select_k(const Plan& p, const SelectArgs& a, cudaStream_t st)
     if (p.select_ring > 0) {
         const size_t smem = 128 + (size_t)p.select_ring * kRingStage +
                             (p.select_keys + (size_t)p.select_part_windows) * sizeof(uint32_t);
-        cudaError_t e = cudaFuncSetAttribute(select_single_kernel<GP>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaError_t e = ensure_smem<select_single_kernel<GP>>(smem);
         if (e != cudaSuccess) return e;
         return launch_pdl(select_single_kernel<GP>, dim3((unsigned)p.pairs), dim3(kSelectThreads),
                           smem, st, a);
     }
     if (p.select_smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(select_kernel<GP>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             (int)p.select_smem);
+        cudaError_t e = ensure_smem<select_kernel<GP>>(p.select_smem);
         if (e != cudaSuccess) return e;
     }
     return launch_pdl(select_kernel<GP>, dim3((unsigned)(p.pairs * p.select_parts)),
