@@ -612,18 +612,52 @@ cudaError_t launch_decode_k(K kernel, const Plan& p, const DecodeArgs& a, int la
 
 // bf16 path: one CTA per (layer, pair) merges, in segment order, the partials of the CTAs whose
 // shares cover it, once the attention grid has finished.
+// Every thread owns (head, d) elements and merges the partials of each element in segment order,
+// with the (max, sum) and numerator loads of up to kCombineU partials in flight together: one
+// round of memory latency for the usual handful of partials, and no block barrier.
+constexpr int kCombineU = 8;
+
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const DecodeArgs a, const int64_t n_slots,
                                                                   const int C) {
-    __shared__ float2 s_ml[kMaxCombineSlots];
     pdl_trigger();
     pdl_wait();
     const int lp = blockIdx.x;
     const int layer = lp / a.pairs, pair = lp - layer * a.pairs;
     const int c_first = cta_of_slot((int64_t)lp * a.sel_cap, n_slots, C);
     const int c_last = cta_of_slot((int64_t)(lp + 1) * a.sel_cap - 1, n_slots, C);
-    combine_partials<__nv_bfloat16, D>(a, layer, pair, lp, c_last - c_first + 1, s_ml,
-                                       Group{(int)threadIdx.x, (int)blockDim.x, 0});
+    const int S = c_last - c_first + 1;
+    const int G = a.G;
+    const float2* ml0 = a.part_ml + (size_t)lp * a.slots * a.Gp;
+    const float* acc0 = a.part_acc + (size_t)lp * a.slots * a.Gp * D;
+    const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out[layer]) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
+    float* lse = a.lse[layer] ? a.lse[layer] + (size_t)b * a.Hq + (size_t)kvh * G : nullptr;
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+        const int h = e / D, dd = e - h * D;
+        float M = -INFINITY, den = 0.f, num = 0.f;
+        for (int s0 = 0; s0 < S; s0 += kCombineU) {
+            float2 ml[kCombineU];
+            float ac[kCombineU];
+#pragma unroll
+            for (int u = 0; u < kCombineU; ++u) {
+                const bool in = s0 + u < S;
+                ml[u] = in ? ld_cg(ml0 + (size_t)(s0 + u) * a.Gp + h) : make_float2(-INFINITY, 0.f);
+                ac[u] = in ? ld_cg(acc0 + ((size_t)(s0 + u) * a.Gp + h) * D + dd) : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < kCombineU; ++u) {
+                if (ml[u].x == -INFINITY) continue;  // an empty partial
+                const float Mn = fmaxf(M, ml[u].x);
+                const float fo = exp2f(M - Mn), fn = exp2f(ml[u].x - Mn);
+                den = den * fo + ml[u].y * fn;
+                num = num * fo + ac[u] * fn;
+                M = Mn;
+            }
+        }
+        store_out<__nv_bfloat16>(out + h * D + dd, den > 0.f ? num / den : 0.f);
+        if (dd == 0 && lse) lse[h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+    }
 }
 
 template <int D>
