@@ -220,6 +220,7 @@ constexpr int kMaxStages = 8;
 constexpr uint32_t kWaitPolls = 1u << 26;  // far beyond any legitimate wait; then give up
 constexpr uint32_t kQSlot = 1024;          // bytes per stage for q of the group (G * D * 2 <= 2048)
 constexpr int kCombineThreads = 128;
+constexpr int kTokU = 4;  // fp32 path: tokens per warp step (BS is a multiple of 16)
 
 enum : int { kStageFirst = 1, kStageLast = 2, kStageEnd = 4 };
 
@@ -552,38 +553,68 @@ __global__ void __launch_bounds__(kDecodeThreads) decode_f32_kernel(DecodeArgs a
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[h][e] = 0.f;
     }
-    for (int i = si.beg + warp; i < si.end; i += kDecodeWarps) {
+    // The split's tokens, in groups of kTokU consecutive tokens of one block, are dealt to the
+    // warps in turn; a group's K and V rows are loaded together and its softmax update is one step.
+    const int gpb = a.BS / kTokU;  // groups per block
+    const int ngroups = (si.end > si.beg ? si.end - si.beg : 0) * gpb;
+    for (int gi = warp; gi < ngroups; gi += kDecodeWarps) {
+        const int i = si.beg + gi / gpb;
         const int blk = ip[i];
         if (blk < 0) continue;
         if (blk >= si.nb) {
-            if (lane == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_BLOCK_IDX);
+            if (lane == 0 && gi % gpb == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_BLOCK_IDX);
             continue;
         }
-        const int64_t t0 = (int64_t)blk * a.BS, t1 = min(t0 + a.BS, si.T);
-        for (int64_t tok = t0; tok < t1; ++tok) {
-            float kv[E], vv[E];
+        const int64_t t0 = (int64_t)blk * a.BS + (int64_t)(gi % gpb) * kTokU;
+        if (t0 >= si.T) continue;
+        float kv[kTokU][E], vv[kTokU][E];
+#pragma unroll
+        for (int u = 0; u < kTokU; ++u) {
+            const bool in = t0 + u < si.T;
 #pragma unroll
             for (int e = 0; e < E; ++e) {
-                kv[e] = __ldg(kp + tok * D + lane * E + e);
-                vv[e] = __ldg(vp + tok * D + lane * E + e);
+                kv[u][e] = in ? __ldg(kp + (t0 + u) * D + lane * E + e) : 0.f;
+                vv[u][e] = in ? __ldg(vp + (t0 + u) * D + lane * E + e) : 0.f;
             }
+        }
 #pragma unroll
-            for (int h = 0; h < kMaxG; ++h) {
-                if (h >= a.G) break;
+        for (int h = 0; h < kMaxG; ++h) {
+            if (h >= a.G) break;
+            float x[kTokU];
+#pragma unroll
+            for (int u = 0; u < kTokU; ++u) {
                 float p = 0.f;
 #pragma unroll
-                for (int e = 0; e < E; ++e) p = fmaf(qv[h][e], kv[e], p);
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-                const float x = p * a.scale_log2;
-                const float mn = fmaxf(m[h], x);
-                const float al = exp2f(m[h] - mn);
-                const float w = exp2f(x - mn);
-                l[h] = l[h] * al + w;
-#pragma unroll
-                for (int e = 0; e < E; ++e) acc[h][e] = fmaf(w, vv[e], acc[h][e] * al);
-                m[h] = mn;
+                for (int e = 0; e < E; ++e) p = fmaf(qv[h][e], kv[u][e], p);
+                x[u] = p;
             }
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                for (int u = 0; u < kTokU; ++u) x[u] += __shfl_xor_sync(0xffffffffu, x[u], off);
+            float gmax = -INFINITY;
+#pragma unroll
+            for (int u = 0; u < kTokU; ++u) {
+                x[u] = t0 + u < si.T ? x[u] * a.scale_log2 : -INFINITY;
+                gmax = fmaxf(gmax, x[u]);
+            }
+            const float mn = fmaxf(m[h], gmax);
+            const float al = exp2f(m[h] - mn);  // m[h] = -inf first: al = 0
+            float wsum = 0.f, w[kTokU];
+#pragma unroll
+            for (int u = 0; u < kTokU; ++u) {
+                w[u] = exp2f(x[u] - mn);
+                wsum += w[u];
+            }
+            l[h] = l[h] * al + wsum;
+#pragma unroll
+            for (int e = 0; e < E; ++e) {
+                float t = acc[h][e] * al;
+#pragma unroll
+                for (int u = 0; u < kTokU; ++u) t = fmaf(w[u], vv[u][e], t);
+                acc[h][e] = t;
+            }
+            m[h] = mn;
         }
     }
 #pragma unroll

@@ -262,7 +262,9 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 2)
     }
 }
 
-// fp32: plain FMA dot products (fp32 inputs keep fp32 accuracy); one warp per row, lanes split d.
+// fp32: plain FMA dot products (fp32 inputs keep fp32 accuracy); a warp per chunk takes kRowU rows
+// at a time, lanes splitting d.
+constexpr int kRowU = 8;
 template <int D>
 __global__ void __launch_bounds__(kScoreThreads, 2) score_f32_kernel(ScoreArgs a) {
     constexpr int E = D / 32;
@@ -300,21 +302,36 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_f32_kernel(ScoreArgs a
             m[h] = -INFINITY;
             s[h] = 0.f;
         }
-        for (int64_t r = r0; r < r1; ++r) {
-            float kv[E];
+        // rows in groups of kRowU, their loads in flight together
+        for (int64_t rg = r0; rg < r1; rg += kRowU) {
+            float kv[kRowU][E];
 #pragma unroll
-            for (int e = 0; e < E; ++e) kv[e] = __ldg(ckp + r * D + lane * E + e);
+            for (int u = 0; u < kRowU; ++u)
+#pragma unroll
+                for (int e = 0; e < E; ++e)
+                    kv[u][e] = rg + u < r1 ? __ldg(ckp + (rg + u) * D + lane * E + e) : 0.f;
 #pragma unroll
             for (int h = 0; h < kMaxG; ++h) {
                 if (h >= a.G) break;
-                float p = 0.f;
+                float p[kRowU];
 #pragma unroll
-                for (int e = 0; e < E; ++e) p = fmaf(qv[h][e], kv[e], p);
+                for (int u = 0; u < kRowU; ++u) {
+                    p[u] = 0.f;
 #pragma unroll
-                for (int off = 16; off > 0; off >>= 1) p += __shfl_xor_sync(0xffffffffu, p, off);
-                const float x = p * a.score_log2;
-                if (lane == h) lg[r * a.Gp + h] = x;
-                online_add(m[h], s[h], x);
+                    for (int e = 0; e < E; ++e) p[u] = fmaf(qv[h][e], kv[u][e], p[u]);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+                    for (int u = 0; u < kRowU; ++u) p[u] += __shfl_xor_sync(0xffffffffu, p[u], off);
+#pragma unroll
+                for (int u = 0; u < kRowU; ++u) {
+                    if (rg + u < r1) {
+                        const float x = p[u] * a.score_log2;
+                        if (lane == h) lg[(rg + u) * a.Gp + h] = x;
+                        online_add(m[h], s[h], x);
+                    }
+                }
             }
         }
         float2* st = a.stats + ((size_t)pair * a.nstat + ci) * a.Gp;
