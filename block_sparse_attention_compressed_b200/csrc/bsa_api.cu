@@ -79,21 +79,26 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
                                                        : 2 * kNumSMs);
     if (P.dtype == BSA_BF16 && (int64_t)P.pairs * P.nc_cap > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
     // Selection: one CTA per pair when there are enough pairs to fill the GPU in one wave,
-    // otherwise the pairs' windows are split into parts of at least 256 windows.
+    // otherwise the pairs' windows are split into parts of at least 256 windows. A part's window
+    // scores sit in shared memory next to the key array, so very long contexts get more parts.
     {
         const int64_t nc = P.nc_cap > 0 ? P.nc_cap : 1;
-        int64_t parts = kNumSMs / P.pairs;
-        const int64_t most = (nc + 255) / 256;
-        if (parts > most) parts = most;
-        if (parts < 1) parts = 1;
-        const int64_t pw = (nc + parts - 1) / parts;
-        P.select_part_windows = (int)pw;
-        P.select_parts = (int)((nc + pw - 1) / pw);
-        if ((int64_t)P.pairs * P.select_parts > 0x7fffffff) return BSA_ERR_UNSUPPORTED;
         const int64_t wmax = (P.BS + P.l - 2) / P.s + 2;  // windows overlapping one block, bound
         // the key array also stages the chunk statistics (2 words per float2)
         P.select_keys = (size_t)P.nb_cap > (size_t)(2 * P.nstat * P.Gp)
                             ? (size_t)P.nb_cap : (size_t)(2 * P.nstat * P.Gp);
+        const int64_t smem_words = (int64_t)(200 * 1024) / (int64_t)sizeof(uint32_t);
+        const int64_t max_pw = smem_words - (int64_t)P.select_keys - wmax;
+        if (max_pw < 256) return BSA_ERR_UNSUPPORTED;
+        int64_t parts = kNumSMs / P.pairs;
+        const int64_t most = (nc + 255) / 256;
+        if (parts > most) parts = most;
+        if (parts < 1) parts = 1;
+        if ((nc + parts - 1) / parts > max_pw) parts = (nc + max_pw - 1) / max_pw;
+        const int64_t pw = (nc + parts - 1) / parts;
+        P.select_part_windows = (int)pw;
+        P.select_parts = (int)((nc + pw - 1) / pw);
+        if ((int64_t)P.pairs * P.select_parts > 0x7fffffff) return BSA_ERR_UNSUPPORTED;
         P.select_smem = (P.select_keys + (size_t)pw + (size_t)wmax) * sizeof(uint32_t);
         if (P.select_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
         // one part per pair: the pair's logits stream through a ring of 16 KB shared-memory stages

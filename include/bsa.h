@@ -85,7 +85,9 @@ typedef enum {
 
 /* Problem shape and method parameters. Supported: dtype fp32 or bf16; head_dim 64 or 128;
  * G = Hq / Hkv in 1..8; block_size a multiple of 16 in 16..256; cmp_kernel, cmp_stride >= 1;
- * 1 <= n_init + n_local + top_k <= 4096; NB_cap <= 32768; num_layers in 1..BSA_MAX_LAYERS. */
+ * 1 <= n_init + n_local + top_k <= 4096; NB_cap <= 32768; num_layers in 1..BSA_MAX_LAYERS;
+ * bf16: B * Hkv * max_seq_len below 2^31 (cache rows are addressed with 32-bit TMA coordinates).
+ * Parameters outside these limits are reported as BSA_ERR_UNSUPPORTED. */
 typedef struct {
     int32_t batch;        /* B */
     int32_t num_q_heads;  /* Hq */

@@ -87,6 +87,20 @@ def test_invalid_params_rejected(lib, kw, status):
     assert bsa.bsa_workspace_size(p) == 0
 
 
+@pytest.mark.parametrize("batch,kv_heads,T", [(64, 8, 1 << 20), (16, 8, 1 << 21), (1, 1, 1 << 21)])
+def test_long_contexts_supported_at_any_pair_count(lib, batch, kv_heads, T):
+    # up to NB_cap = 32768 blocks, whatever the number of (batch, kv-head) pairs
+    p = _p(batch=batch, num_q_heads=4 * kv_heads, num_kv_heads=kv_heads, max_seq_len=T, top_k=64)
+    assert bsa.bsa_check_params(p) == bsa.BSA_OK
+    assert bsa.bsa_workspace_size(p) > 0
+
+
+def test_cache_rows_beyond_tma_coordinates_rejected(lib):
+    # B * Hkv * T_cap cache rows must stay below 2^31 (32-bit TMA row coordinates)
+    p = _p(batch=128, num_q_heads=32, num_kv_heads=8, max_seq_len=1 << 21, top_k=64)
+    assert bsa.bsa_check_params(p) == bsa.BSA_ERR_UNSUPPORTED
+
+
 def test_unsupported_dtype(lib):
     p = _p()
     p.dtype = 7
