@@ -4,22 +4,27 @@
 // (first abstract) and "CoSA: Accelerating Long-Context Inference via Proxy-Kernel Co-Designed
 // Sparse Attention" (second abstract): several layers attended with one layer's selection.
 //
-// Split-KV flash decoding. grid = layers * pairs * splits CTAs; CTA `split` of a (layer, pair)
-// owns blocks [split*bpc, (split+1)*bpc) of the pair's selection. The warps' partial softmax
-// states (fp32, exp2 domain) are merged in shared memory and written to the workspace; the last CTA
-// of the (layer, pair) to finish (completion counter, no waiting) combines all splits into O, LSE.
+// Split-KV flash decoding: partial softmax states (fp32, exp2 domain; per head the max m, the
+// denominator l and the numerators acc) over disjoint parts of a pair's selected blocks, merged
+// into O and LSE at the end.
 //
-// bf16 path (TMA pipeline): one producer warp walks the CTA's selected blocks and issues 2-D TMA
-// tensor copies (128-byte swizzle) of each 16..64-token stage of K and V into a ring of shared-
-// memory stages, completing on per-stage mbarriers; four consumer warps each take 16 tokens of a
-// stage and run, on the tensor cores (mma.m16n8k16, operands from ldmatrix):
+// bf16 path (TMA pipeline, persistent): the layers * pairs * SEL_cap block slots are shared evenly
+// by the CTAs; a (layer, pair) run inside a CTA's share is a segment with one partial. One producer
+// warp walks the share and issues 2-D TMA tensor copies (128-byte swizzle, L2 evict-first) of each
+// 16..64-token stage of K and V into a ring of shared-memory stages, completing on per-stage
+// mbarriers; four consumer warps each take 16 tokens of a stage and run, on the tensor cores
+// (mma.m16n8k16, operands from ldmatrix):
 //   S^T[tok][head] = K[tok][:] . q^T          (tokens are M, the G heads padded to 8 are N)
 //   O^T[d][head] += V^T[d][tok] . P^T[tok][head]  (d is M; V^T via ldmatrix.trans; P^T from the
 //       S^T accumulators via movmatrix.trans, split as bf16 hi + lo so the products keep ~16
 //       significant bits of the fp32 probabilities)
 // then release the stage. Bytes in flight are set by the ring size, not by registers. Tokens at or
-// past the sequence length are masked to -inf and their V rows zeroed in shared memory.
-// fp32 path: one token at a time per warp, FMA dot products and warp reductions.
+// past the sequence length are masked to -inf and their V rows zeroed in shared memory. At the end
+// of a segment the warps merge their states and write its partial; combine_kernel merges each
+// (layer, pair)'s partials in segment order once the grid has finished.
+// fp32 path: grid = layers * pairs * splits CTAs, a split of bpc blocks each; the warps take groups
+// of consecutive tokens in turn (FMA dot products, warp reductions), merge in shared memory, and
+// the last split of a (layer, pair) to finish (completion counter, no waiting) combines them.
 #include "bsa_internal.cuh"
 
 namespace bsa {
