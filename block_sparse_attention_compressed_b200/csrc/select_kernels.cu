@@ -785,42 +785,54 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
         M[h] = h < a.G ? sM[h] : 0.f;
         iz[h] = h < a.G ? sInvZ[h] : 0.f;
     }
-    // S[j] = sum_h exp2(x[j][h] - M_h) / Z_h, stage by stage
-    for (int r = 0; r < npieces; ++r) {
-        if (!mbar_wait(&full[r % R], (r / R) & 1, kScoreWaitPolls)) {
-            if (tid == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
-            break;
-        }
-        const float* lg = reinterpret_cast<const float*>(ring + (size_t)(r % R) * kRingStage);
-        const int w0 = r * PW, wn = min(PW, nc - w0);
-        for (int i = tid; i < wn; i += kSelectThreads) {
-            float x[GP];
-            if constexpr (GP == 1) {
-                x[0] = lg[i];
-            } else if constexpr (GP == 2) {
-                const float2 t = reinterpret_cast<const float2*>(lg)[i];
-                x[0] = t.x;
-                x[1] = t.y;
-            } else {
+    // S[j] = sum_h exp2(x[j][h] - M_h) / Z_h for window j at index i of the stage in slot `slot`
+    auto window_score = [&](int slot, int i) -> float {
+        const float* lg = reinterpret_cast<const float*>(ring + (size_t)slot * kRingStage);
+        float x[GP];
+        if constexpr (GP == 1) {
+            x[0] = lg[i];
+        } else if constexpr (GP == 2) {
+            const float2 t = reinterpret_cast<const float2*>(lg)[i];
+            x[0] = t.x;
+            x[1] = t.y;
+        } else {
 #pragma unroll
-                for (int q = 0; q < GP / 4; ++q) {
-                    const float4 t = reinterpret_cast<const float4*>(lg + (size_t)i * GP)[q];
-                    x[4 * q] = t.x;
-                    x[4 * q + 1] = t.y;
-                    x[4 * q + 2] = t.z;
-                    x[4 * q + 3] = t.w;
-                }
+            for (int q = 0; q < GP / 4; ++q) {
+                const float4 t = reinterpret_cast<const float4*>(lg + (size_t)i * GP)[q];
+                x[4 * q] = t.x;
+                x[4 * q + 1] = t.y;
+                x[4 * q + 2] = t.z;
+                x[4 * q + 3] = t.w;
             }
-            float acc = 0.f;
-#pragma unroll
-            for (int h = 0; h < GP; ++h)
-                if (h < a.G) acc += exp2f(x[h] - M[h]) * iz[h];
-            S[w0 + i] = acc;
         }
-        __syncthreads();  // the slot has been read by everyone
-        if (tid == 0 && r + R < npieces) {
-            fence_proxy_async_smem();
-            issue(r + R);
+        float acc = 0.f;
+#pragma unroll
+        for (int h = 0; h < GP; ++h)
+            if (h < a.G) acc += exp2f(x[h] - M[h]) * iz[h];
+        return acc;
+    };
+    if (npieces <= R) {
+        // every stage is in flight from the start: wait for all, then one pass over the windows
+        bool waited = true;
+        for (int r = 0; r < npieces && waited; ++r) waited = mbar_wait(&full[r], 0, kScoreWaitPolls);
+        if (!waited) {
+            if (tid == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+        } else {
+            for (int j = tid; j < nc; j += kSelectThreads) S[j] = window_score(j / PW, j % PW);
+        }
+    } else {
+        for (int r = 0; r < npieces; ++r) {
+            if (!mbar_wait(&full[r % R], (r / R) & 1, kScoreWaitPolls)) {
+                if (tid == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                break;
+            }
+            const int w0 = r * PW, wn = min(PW, nc - w0);
+            for (int i = tid; i < wn; i += kSelectThreads) S[w0 + i] = window_score(r % R, i);
+            __syncthreads();  // the slot has been read by everyone
+            if (tid == 0 && r + R < npieces) {
+                fence_proxy_async_smem();
+                issue(r + R);
+            }
         }
     }
     __syncthreads();
