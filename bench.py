@@ -265,18 +265,32 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
-def kernel_source_hash() -> str:
+# The sources that decide a kernel's code and launch plan: its own file, the shared header and the
+# host side that plans the launch.
+KERNEL_SOURCES = {"decode": "decode_kernels.cu", "combine": "decode_kernels.cu",
+                  "score": "select_kernels.cu", "select": "select_kernels.cu",
+                  "compress": "compress_kernels.cu", "append": "compress_kernels.cu"}
+
+
+def kernel_source_hash(kernel: str | None = None) -> str:
+    """sha256 (16 hex digits) of the kernel's sources, or of every kernel source when None."""
     import glob
+    csrc = os.path.join(ROOT, "block_sparse_attention_compressed_b200", "csrc")
+    if kernel is None:
+        paths = sorted(glob.glob(os.path.join(csrc, "*")))
+    else:
+        own = next(f for k, f in KERNEL_SOURCES.items() if kernel.startswith(k))
+        paths = [os.path.join(csrc, n) for n in (own, "bsa_internal.cuh", "bsa_api.cu")]
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "block_sparse_attention_compressed_b200", "csrc", "*"))):
+    for p in paths:
         with open(p, "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
 def profile_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current kernel
-    sources (the summary records the sources' hash)."""
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the kernel's current
+    sources (the summary records their hash: kernel_source_hash(kernel))."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     try:
         text = open(path).read()
@@ -284,7 +298,7 @@ def profile_traffic(kernel: str, workload: str):
         return None
     m = re.search(r"dram_bytes_per_launch:\s*([\d.eE+]+)", text)
     hm = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not hm or hm.group(1) != kernel_source_hash():
+    if not m or not hm or hm.group(1) != kernel_source_hash(kernel):
         return None
     return float(m.group(1))
 
