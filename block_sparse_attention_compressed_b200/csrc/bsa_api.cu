@@ -101,11 +101,13 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
         if ((int64_t)P.pairs * P.select_parts > 0x7fffffff) return BSA_ERR_UNSUPPORTED;
         P.select_smem = (P.select_keys + (size_t)pw + (size_t)wmax) * sizeof(uint32_t);
         if (P.select_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
-        // one part per pair: the pair's logits stream through a ring of 16 KB shared-memory stages
+        // one part per pair: the pair's logits stream through a ring of 16 KB shared-memory stages,
+        // next to the keys, the window scores and one weight per (chunk, head)
         P.select_ring = 0;
         if (P.select_parts == 1) {
-            const size_t rest = 1024 + P.select_smem;
-            int64_t ring = ((size_t)220 * 1024 > rest) ? ((size_t)220 * 1024 - rest) / (16 * 1024) : 0;
+            // 200 KB of dynamic shared memory at most: the top-k's histogram is static (16 KB)
+            const size_t rest = 1024 + P.select_smem + (size_t)P.nstat * P.Gp * sizeof(float);
+            int64_t ring = ((size_t)200 * 1024 > rest) ? ((size_t)200 * 1024 - rest) / (16 * 1024) : 0;
             if (ring > 8) ring = 8;
             if (ring >= 2) P.select_ring = (int)ring;
         }

@@ -224,7 +224,7 @@ constexpr int kTmaThreads = (kConsumerWarps + 1) * 32;  // + one producer warp
 constexpr int kMaxStages = 8;
 constexpr uint32_t kWaitPolls = 1u << 26;  // far beyond any legitimate wait; then give up
 constexpr uint32_t kQSlot = 1024;          // bytes per stage for q of the group (G * D * 2 <= 2048)
-constexpr int kCombineThreads = 128;
+constexpr int kCombineThreads = 256;
 constexpr int kTokU = 4;  // fp32 path: tokens per warp step (BS is a multiple of 16)
 
 enum : int { kStageFirst = 1, kStageLast = 2, kStageEnd = 4 };
@@ -648,51 +648,72 @@ cudaError_t launch_decode_k(K kernel, const Plan& p, const DecodeArgs& a, int la
 
 // bf16 path: one CTA per (layer, pair) merges, in segment order, the partials of the CTAs whose
 // shares cover it, once the attention grid has finished.
-// Every thread owns (head, d) elements and merges the partials of each element in segment order,
-// with the (max, sum) and numerator loads of up to kCombineU partials in flight together: one
-// round of memory latency for the usual handful of partials, and no block barrier.
+// Every thread owns one head and four consecutive d values, and merges their partials in segment
+// order with the (max, sum) and 16-byte numerator loads of up to kCombineU partials in flight
+// together: one round of memory latency for the usual handful of partials, and no block barrier.
 constexpr int kCombineU = 8;
+static_assert(kCombineThreads * 4 >= kMaxG * 128, "one thread per head and four d values");
 
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads) combine_kernel(const DecodeArgs a, const int64_t n_slots,
                                                                   const int C) {
     pdl_trigger();
     pdl_wait();
+    constexpr int Q = D / 4;  // groups of four d values per head
     const int lp = blockIdx.x;
+    const int G = a.G;
+    if ((int)threadIdx.x >= G * Q) return;
+    const int h = (int)threadIdx.x / Q, dd = ((int)threadIdx.x - h * Q) * 4;
     const int layer = lp / a.pairs, pair = lp - layer * a.pairs;
     const int c_first = cta_of_slot((int64_t)lp * a.sel_cap, n_slots, C);
     const int c_last = cta_of_slot((int64_t)(lp + 1) * a.sel_cap - 1, n_slots, C);
     const int S = c_last - c_first + 1;
-    const int G = a.G;
-    const float2* ml0 = a.part_ml + (size_t)lp * a.slots * a.Gp;
-    const float* acc0 = a.part_acc + (size_t)lp * a.slots * a.Gp * D;
+    const float2* ml0 = a.part_ml + (size_t)lp * a.slots * a.Gp + h;
+    const float* acc0 = a.part_acc + (size_t)lp * a.slots * a.Gp * D + (size_t)h * D + dd;
     const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
-    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out[layer]) + ((size_t)b * a.Hq + (size_t)kvh * G) * D;
-    float* lse = a.lse[layer] ? a.lse[layer] + (size_t)b * a.Hq + (size_t)kvh * G : nullptr;
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-        const int h = e / D, dd = e - h * D;
-        float M = -INFINITY, den = 0.f, num = 0.f;
-        for (int s0 = 0; s0 < S; s0 += kCombineU) {
-            float2 ml[kCombineU];
-            float ac[kCombineU];
+    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out[layer]) +
+                         ((size_t)b * a.Hq + (size_t)kvh * G + h) * D + dd;
+    float M = -INFINITY, den = 0.f;
+    float num[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int s0 = 0; s0 < S; s0 += kCombineU) {
+        float2 ml[kCombineU];
+        float4 ac[kCombineU];
 #pragma unroll
-            for (int u = 0; u < kCombineU; ++u) {
-                const bool in = s0 + u < S;
-                ml[u] = in ? ld_cg(ml0 + (size_t)(s0 + u) * a.Gp + h) : make_float2(-INFINITY, 0.f);
-                ac[u] = in ? ld_cg(acc0 + ((size_t)(s0 + u) * a.Gp + h) * D + dd) : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < kCombineU; ++u) {
-                if (ml[u].x == -INFINITY) continue;  // an empty partial
-                const float Mn = fmaxf(M, ml[u].x);
-                const float fo = exp2f(M - Mn), fn = exp2f(ml[u].x - Mn);
-                den = den * fo + ml[u].y * fn;
-                num = num * fo + ac[u] * fn;
-                M = Mn;
-            }
+        for (int u = 0; u < kCombineU; ++u) {
+            const bool in = s0 + u < S;
+            const size_t slot = (size_t)(s0 + u) * a.Gp;
+            ml[u] = in ? ld_cg(ml0 + slot) : make_float2(-INFINITY, 0.f);
+            ac[u] = in ? ld_cg(reinterpret_cast<const float4*>(acc0 + slot * D)) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
-        store_out<__nv_bfloat16>(out + h * D + dd, den > 0.f ? num / den : 0.f);
-        if (dd == 0 && lse) lse[h] = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
+#pragma unroll
+        for (int u = 0; u < kCombineU; ++u) {
+            if (ml[u].x == -INFINITY) continue;  // an empty partial
+            const float Mn = fmaxf(M, ml[u].x);
+            const float fo = exp2f(M - Mn), fn = exp2f(ml[u].x - Mn);
+            den = den * fo + ml[u].y * fn;
+            num[0] = num[0] * fo + ac[u].x * fn;
+            num[1] = num[1] * fo + ac[u].y * fn;
+            num[2] = num[2] * fo + ac[u].z * fn;
+            num[3] = num[3] * fo + ac[u].w * fn;
+            M = Mn;
+        }
+    }
+    float o[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) o[k] = den > 0.f ? num[k] / den : 0.f;
+    if ((reinterpret_cast<uintptr_t>(out) & 7u) == 0u) {
+        __nv_bfloat162 lo = __floats2bfloat162_rn(o[0], o[1]), hi = __floats2bfloat162_rn(o[2], o[3]);
+        uint2 v;
+        v.x = *reinterpret_cast<uint32_t*>(&lo);
+        v.y = *reinterpret_cast<uint32_t*>(&hi);
+        *reinterpret_cast<uint2*>(out) = v;
+    } else {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) store_out<__nv_bfloat16>(out + k, o[k]);
+    }
+    if (dd == 0 && a.lse[layer]) {
+        float* lse = a.lse[layer] + (size_t)b * a.Hq + (size_t)kvh * G + h;
+        *lse = den > 0.f ? (M + log2f(den)) * 0.69314718055994531f : -INFINITY;
     }
 }
 

@@ -28,8 +28,9 @@ namespace {
 constexpr int kScoreThreads = kScoreWarps * 32;
 constexpr int kSelectThreads = 512;
 
-// Block-wide exclusive scan of one int per thread (contiguous, in thread order).
-__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total) {
+// Block-wide exclusive scan of one int per thread (contiguous, in thread order). With `reuse`,
+// s_warp may be written again as soon as it returns.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total, bool reuse = true) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     int x = v;
 #pragma unroll
@@ -51,7 +52,7 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
     __syncthreads();
     const int base = warp > 0 ? s_warp[warp - 1] : 0;
     *total = s_warp[nwarps - 1];
-    __syncthreads();  // s_warp may be reused right after
+    if (reuse) __syncthreads();
     return base + x - v;
 }
 
@@ -85,23 +86,6 @@ __device__ __forceinline__ void report_lengths(const ScoreArgs& a) {
 }
 
 // ================================================================================ score kernels
-__device__ __forceinline__ void flush_stats(float2* dst, float m0, float s0, float m1, float s1,
-                                            int g, int tq, int G) {
-    // combine the 8 row groups (lanes with equal tq), then lanes g == 0 publish heads 2tq, 2tq+1
-#pragma unroll
-    for (int off = 4; off < 32; off <<= 1) {
-        float mo = __shfl_xor_sync(0xffffffffu, m0, off), so = __shfl_xor_sync(0xffffffffu, s0, off);
-        online_merge(m0, s0, mo, so);
-        mo = __shfl_xor_sync(0xffffffffu, m1, off);
-        so = __shfl_xor_sync(0xffffffffu, s1, off);
-        online_merge(m1, s1, mo, so);
-    }
-    if (g == 0) {
-        if (2 * tq < G) dst[2 * tq] = make_float2(m0, s0);
-        if (2 * tq + 1 < G) dst[2 * tq + 1] = make_float2(m1, s1);
-    }
-}
-
 constexpr int kScoreConsumers = 4;
 constexpr int kScoreTmaThreads = (kScoreConsumers + 1) * 32;
 constexpr int kScoreMaxStages = 8;
@@ -236,28 +220,59 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 2)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);  // the data is in registers: refill the slot
-            float* lg = a.logits + (size_t)md.pair * a.lg_stride * a.Gp;
-            float m0 = -INFINITY, s0 = 0.f, m1 = -INFINITY, s1 = 0.f;
+            // the chunk's maximum per head first, then e = exp2(x - max) is stored and summed: the
+            // selection only rescales each chunk's e by one weight per head
+            float x[4][4];
+            float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
-                const float x0 = c[r][0] * a.score_log2, x1 = c[r][1] * a.score_log2;
-                const float x2 = c[r][2] * a.score_log2, x3 = c[r][3] * a.score_log2;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) x[r][e] = c[r][e] * a.score_log2;
+                if (16 * r + g < md.nrows) {
+                    m0 = fmaxf(m0, x[r][0]);
+                    m1 = fmaxf(m1, x[r][1]);
+                }
+                if (16 * r + g + 8 < md.nrows) {
+                    m0 = fmaxf(m0, x[r][2]);
+                    m1 = fmaxf(m1, x[r][3]);
+                }
+            }
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {  // over the 8 row groups (lanes with equal tq)
+                m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
+                m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
+            }
+            float* lg = a.logits + (size_t)md.pair * a.lg_stride * a.Gp;
+            float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
                 const int lra = 16 * r + g, lrb = lra + 8;
                 const int64_t ra = md.row0 + lra, rb = md.row0 + lrb;
                 if (lra < md.nrows) {
-                    if (h1) *reinterpret_cast<float2*>(lg + ra * a.Gp + 2 * tq) = make_float2(x0, x1);
-                    else if (h0) lg[ra * a.Gp + 2 * tq] = x0;
-                    if (h0) online_add(m0, s0, x0);
-                    if (h1) online_add(m1, s1, x1);
+                    const float e0 = exp2f(x[r][0] - m0), e1 = exp2f(x[r][1] - m1);
+                    if (h1) *reinterpret_cast<float2*>(lg + ra * a.Gp + 2 * tq) = make_float2(e0, e1);
+                    else if (h0) lg[ra * a.Gp + 2 * tq] = e0;
+                    s0 += e0;
+                    s1 += e1;
                 }
                 if (lrb < md.nrows) {
-                    if (h1) *reinterpret_cast<float2*>(lg + rb * a.Gp + 2 * tq) = make_float2(x2, x3);
-                    else if (h0) lg[rb * a.Gp + 2 * tq] = x2;
-                    if (h0) online_add(m0, s0, x2);
-                    if (h1) online_add(m1, s1, x3);
+                    const float e2 = exp2f(x[r][2] - m0), e3 = exp2f(x[r][3] - m1);
+                    if (h1) *reinterpret_cast<float2*>(lg + rb * a.Gp + 2 * tq) = make_float2(e2, e3);
+                    else if (h0) lg[rb * a.Gp + 2 * tq] = e2;
+                    s0 += e2;
+                    s1 += e3;
                 }
             }
-            flush_stats(a.stats + ((size_t)md.pair * a.nstat + md.row0 / 64) * a.Gp, m0, s0, m1, s1, g, tq, a.G);
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                s0 += __shfl_xor_sync(0xffffffffu, s0, off);
+                s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+            }
+            if (g == 0) {
+                float2* dst = a.stats + ((size_t)md.pair * a.nstat + md.row0 / 64) * a.Gp;
+                if (h0) dst[2 * tq] = make_float2(m0, s0);
+                if (h1) dst[2 * tq + 1] = make_float2(m1, s1);
+            }
         }
     }
 }
@@ -335,9 +350,16 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_f32_kernel(ScoreArgs a
             }
         }
         float2* st = a.stats + ((size_t)pair * a.nstat + ci) * a.Gp;
+        float mh = 0.f;
 #pragma unroll
         for (int h = 0; h < kMaxG; ++h)
-            if (h < a.G && lane == h) st[h] = make_float2(m[h], s[h]);
+            if (h < a.G && lane == h) {
+                st[h] = make_float2(m[h], s[h]);
+                mh = m[h];
+            }
+        // the chunk's e = exp2(x - max) replaces the logits that lane h stored above
+        if (lane < a.G)
+            for (int64_t r = r0; r < r1; ++r) lg[r * a.Gp + lane] = exp2f(lg[r * a.Gp + lane] - mh);
     }
 }
 
@@ -368,11 +390,11 @@ __device__ __forceinline__ LogitRow<GP> load_row(const float* p) {
     return r;
 }
 
-// S[j - j0] = sum over the group's heads of exp2(x[j][h] - M_h) / Z_h for windows j in [j0, j1),
-// kU rows per thread in flight.
+// S[j - j0] = sum over the group's heads of e[j][h] * w[j / 64][h] for windows j in [j0, j1), where
+// e = exp2(x - chunk max) is what the scorer stored and w[c][h] = exp2(chunk max - M_h) / Z_h (the
+// .x of the chunk's staged statistics), kU rows per thread in flight.
 template <int GP>
-__device__ void window_scores(const float* lg, int64_t j0, int64_t j1, int G, const float* sM,
-                              const float* sInvZ, float* S) {
+__device__ void window_scores(const float* lg, int64_t j0, int64_t j1, int G, const float2* wt, float* S) {
     constexpr int kU = GP <= 4 ? 16 : 8;
     const int tid = threadIdx.x, NT = blockDim.x;
     for (int64_t base = j0; base < j1; base += (int64_t)NT * kU) {
@@ -386,10 +408,11 @@ __device__ void window_scores(const float* lg, int64_t j0, int64_t j1, int G, co
         for (int u = 0; u < kU; ++u) {
             const int64_t j = base + (int64_t)u * NT + tid;
             if (j < j1) {
+                const float2* w = wt + (j >> 6) * GP;
                 float acc = 0.f;
 #pragma unroll
                 for (int h = 0; h < GP; ++h)
-                    if (h < G) acc += exp2f(r[u].v[h] - sM[h]) * sInvZ[h];
+                    if (h < G) acc += r[u].v[h] * w[h].x;
                 S[j - j0] = acc;
             }
         }
@@ -398,18 +421,90 @@ __device__ void window_scores(const float* lg, int64_t j0, int64_t j1, int G, co
 
 // Top-k of the candidate blocks [init_end, local_begin) by score (ties: lower index first), united
 // with the init and local blocks, written ascending. keys[] (shared) holds the nb block keys and
-// is overwritten. Each thread keeps its contiguous segment of up to kKeysPerThread candidate keys
-// in registers for the radix passes (larger candidate sets are streamed from shared memory).
+// may be overwritten. Each thread owns a contiguous segment of the candidates, kept in registers
+// when it has at most kKeysPerThread of them (larger candidate sets are streamed from shared
+// memory).
+//
+// The k-th largest key is located by radix digits below the bits that all candidates share: a
+// first digit of up to kFirstDigitBits bits (one histogram bin per value, found with a two-level
+// descending scan), then 8-bit digits. As soon as the digit bucket holding the k-th key has at
+// most kExactMax keys, the owners of those keys rank them exactly among themselves (score
+// descending, block ascending); the taken candidates are those above the bucket plus the bucket
+// keys ranked below the number still needed. Otherwise the ties at the final key value are taken
+// in block order.
 constexpr int kKeysPerThread = 8;
+constexpr int kFirstDigitBits = 12;
+constexpr int kExactMax = 128;
+constexpr int kHistBins = 1 << kFirstDigitBits;
+
+// Bin d* (scanning digits from the top) at which the running count of hist reaches `need`; the
+// winning thread publishes the digit, the count still needed inside it and the bin's size.
+__device__ __forceinline__ void find_digit_from_top(const int* hist, int nbins, int need, int* s_warp,
+                                                    int* s_digit, int* s_need, int* s_bcnt) {
+    const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    const int per_t = (nbins + NT - 1) / NT;  // bins per thread, descending from the top
+    int c = 0, h8[8];
+    const bool vec = per_t == 8 && nbins == 8 * NT;  // bins [nbins - 8(t+1), nbins - 8t), 2 x 16 B
+    if (vec) {
+        const int4* p = reinterpret_cast<const int4*>(hist + nbins - 8 * (tid + 1));
+        const int4 lo = p[0], hi = p[1];
+        h8[0] = hi.w; h8[1] = hi.z; h8[2] = hi.y; h8[3] = hi.x;
+        h8[4] = lo.w; h8[5] = lo.z; h8[6] = lo.y; h8[7] = lo.x;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) c += h8[k];
+    } else {
+        for (int k = 0; k < per_t; ++k) {
+            const int d = nbins - 1 - (tid * per_t + k);
+            if (d >= 0) c += hist[d];
+        }
+    }
+    int incl = c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+    }
+    if (lane == 31) s_warp[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; ++w) base += s_warp[w];
+    const int excl = base + incl - c;
+    if (excl < need && need <= excl + c) {
+        int acc = excl;
+        if (vec) {
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                if (acc < need && acc + h8[k] >= need) {
+                    *s_digit = nbins - 1 - (tid * 8 + k);
+                    *s_need = need - acc;
+                    *s_bcnt = h8[k];
+                }
+                acc += h8[k];
+            }
+        } else {
+            for (int k = 0; k < per_t; ++k) {
+                const int d = nbins - 1 - (tid * per_t + k);
+                if (d < 0) break;
+                const int cd = hist[d];
+                if (acc < need && acc + cd >= need) {
+                    *s_digit = d;
+                    *s_need = need - acc;
+                    *s_bcnt = cd;
+                }
+                acc += cd;
+            }
+        }
+    }
+    __syncthreads();
+}
 
 __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys) {
     __shared__ int s_warp[32];
-    __shared__ int hist[256];
-    __shared__ uint32_t s_prefix;
-    __shared__ int s_need, s_bcnt, s_bn;
+    __shared__ __align__(16) int hist[kHistBins];
+    __shared__ int s_digit, s_need, s_bcnt, s_bn;
     __shared__ uint32_t s_and[32], s_or[32];
-    __shared__ uint32_t s_bkey[32];
-    __shared__ int s_bidx[32], s_btake[32];
+    __shared__ __align__(16) uint32_t s_bkey[kExactMax];  // 0 pads: below every real key
+    __shared__ __align__(16) int s_bidx[kExactMax];
     const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31;
     const int init_end = min(a.n_init, nb);
     const int local_begin = max(nb - a.n_local, 0);
@@ -423,18 +518,16 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
     uint32_t kr[kKeysPerThread];
 #pragma unroll
     for (int e = 0; e < kKeysPerThread; ++e) kr[e] = (in_regs && seg_lo + e < seg_hi) ? keys[seg_lo + e] : 0u;
+    for (int i = tid; i < kHistBins / 4; i += NT) reinterpret_cast<int4*>(hist)[i] = make_int4(0, 0, 0, 0);
+    for (int i = tid; i < kExactMax; i += NT) s_bkey[i] = 0u;
+    if (tid == 0) s_bn = 0;
 
     uint32_t thr = 0xffffffffu;  // keys > thr are taken, plus the first `need` keys == thr
     int need = 0;
-    // Early finish: once the digit bucket that holds the k-th key has at most 32 keys, one warp
-    // ranks them exactly (score descending, block ascending); then the candidates taken are those
-    // above the bucket plus the bucket keys ranked below `need`.
     bool exact = false;
     uint32_t emask = 0u, eprefix = 0u;
-    int ebn = 0;
     if (kk > 0 && !take_all) {
-        // bytes that every candidate shares need no histogram pass: start at the first byte in
-        // which two candidates differ (block-wide AND / OR of the keys)
+        // bits that every candidate shares need no histogram pass (block-wide AND / OR)
         uint32_t kand = 0xffffffffu, kor = 0u;
         if (in_regs) {
 #pragma unroll
@@ -464,158 +557,154 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
             kor |= s_or[w];
         }
         const uint32_t diff = kand ^ kor;  // bits in which some candidates differ
-        int top = 24;
-        while (top > 0 && (diff >> top) == 0u) top -= 8;
-        uint32_t prefix = top < 24 ? (kand & (0xffffffffu << (top + 8))) : 0u;
-        uint32_t mask = top < 24 ? (0xffffffffu << (top + 8)) : 0u;
+        uint32_t prefix = kand, mask = 0xffffffffu;
         need = kk;
-        for (int shift = top; shift >= 0; shift -= 8) {
-            for (int i = tid; i < 256; i += NT) hist[i] = 0;
-            if (tid == 0) s_bn = 0;
-            __syncthreads();
-            // warp-aggregated histogram (keys of a warp often share a digit): one atomic per
-            // distinct digit per warp; all of a thread's keys are processed independently
-            if (in_regs) {
-                uint32_t dg[kKeysPerThread];
-#pragma unroll
-                for (int e = 0; e < kKeysPerThread; ++e) {
-                    const bool live = seg_lo + e < seg_hi && (kr[e] & mask) == prefix;
-                    dg[e] = live ? ((kr[e] >> shift) & 255u) : 256u;
+        if (diff != 0u) {
+            int hi = 31 - __clz(diff);
+            mask = hi < 31 ? (0xffffffffu << (hi + 1)) : 0u;
+            prefix = kand & mask;
+            int width = min(kFirstDigitBits, hi + 1);
+            for (bool first = true;; first = false) {
+                const int shift = hi - width + 1;
+                const int nbins = 1 << width;
+                const uint32_t dmask = (uint32_t)nbins - 1u;
+                if (!first) {
+                    for (int i = tid; i < nbins; i += NT) hist[i] = 0;
+                    __syncthreads();
                 }
+                if (in_regs) {
 #pragma unroll
-                for (int e = 0; e < kKeysPerThread; ++e) {
-                    const uint32_t peers = __match_any_sync(0xffffffffu, dg[e]);
-                    if (dg[e] < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[dg[e]], __popc(peers));
-                }
-            } else {
-                for (int i0 = 0; i0 < per; ++i0) {
-                    const int i = seg_lo + i0;
-                    const uint32_t u = i < seg_hi ? keys[i] : 0u;
-                    const uint32_t d = (i < seg_hi && (u & mask) == prefix) ? ((u >> shift) & 255u) : 256u;
-                    const uint32_t peers = __match_any_sync(0xffffffffu, d);
-                    if (d < 256u && lane == __ffs(peers) - 1) atomicAdd(&hist[d], __popc(peers));
-                }
-            }
-            __syncthreads();
-            if (tid < 32) {
-                // lane L owns digits 255-8L .. 248-8L, scanned from the top
-                int c[8], sum = 0;
-#pragma unroll
-                for (int k = 0; k < 8; ++k) {
-                    c[k] = hist[255 - 8 * tid - k];
-                    sum += c[k];
-                }
-                int incl = sum;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    int y = __shfl_up_sync(0xffffffffu, incl, off);
-                    if (tid >= off) incl += y;
-                }
-                const int excl = incl - sum;
-                if (excl < need && need <= incl) {
-                    int acc = excl;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        if (acc < need && acc + c[k] >= need) {
-                            s_prefix = prefix | ((uint32_t)(255 - 8 * tid - k) << shift);
-                            s_need = need - acc;
-                            s_bcnt = c[k];
-                        }
-                        acc += c[k];
+                    for (int e = 0; e < kKeysPerThread; ++e)
+                        if (seg_lo + e < seg_hi && (kr[e] & mask) == prefix) atomicAdd(&hist[(kr[e] >> shift) & dmask], 1);
+                } else {
+                    for (int i = seg_lo; i < seg_hi; ++i) {
+                        const uint32_t u = keys[i];
+                        if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1);
                     }
                 }
-            }
-            __syncthreads();
-            prefix = s_prefix;
-            need = s_need;
-            mask |= 255u << shift;
-            if (in_regs && shift > 0 && s_bcnt <= 32) {
-                exact = true;
-                break;
+                __syncthreads();
+                find_digit_from_top(hist, nbins, need, s_warp, &s_digit, &s_need, &s_bcnt);
+                prefix |= (uint32_t)s_digit << shift;
+                need = s_need;
+                mask |= dmask << shift;
+                if (shift == 0) break;  // every bit decided: the bucket's keys are all equal
+                if (in_regs && s_bcnt <= kExactMax) {
+                    exact = true;
+                    break;
+                }
+                __syncthreads();  // everyone has read the bins before they are cleared
+                hi = shift - 1;
+                width = min(8, hi + 1);
             }
         }
         thr = prefix;
         if (exact) {
             emask = mask;
             eprefix = prefix;
+        }
+    }
+
+    int32_t* out = a.block_idx + (size_t)pair * a.sel_cap;
+    if (in_regs) {
+        // taken flags of the thread's own candidates
+        bool fl[kKeysPerThread];
+        if (exact) {
 #pragma unroll
             for (int e = 0; e < kKeysPerThread; ++e) {
-                if (seg_lo + e < seg_hi && (kr[e] & mask) == prefix) {
+                if (seg_lo + e < seg_hi && (kr[e] & emask) == eprefix) {
                     const int slot = atomicAdd(&s_bn, 1);
                     s_bkey[slot] = kr[e];
                     s_bidx[slot] = seg_lo + e;
                 }
             }
             __syncthreads();
-            ebn = s_bn;
-            if (tid < 32) {
-                const uint32_t key = tid < ebn ? s_bkey[tid] : 0u;
-                const int idx = tid < ebn ? s_bidx[tid] : 0x7fffffff;
-                int rank = 0;
-                for (int j = 0; j < ebn; ++j) {
-                    const uint32_t kj = s_bkey[j];
-                    const int ij = s_bidx[j];
-                    rank += (kj > key || (kj == key && ij < idx));
-                }
-                if (tid < ebn) s_btake[tid] = rank < need ? idx : -1;
-            }
-            __syncthreads();
-        }
-    }
-    if (exact) {
-        // above the bucket, or ranked within it
-#pragma unroll
-        for (int e = 0; e < kKeysPerThread; ++e) {
-            if (seg_lo + e < seg_hi) {
-                const uint32_t mk = kr[e] & emask;
-                bool take = mk > eprefix;
-                if (mk == eprefix)
-                    for (int j = 0; j < ebn; ++j) take |= s_btake[j] == seg_lo + e;
-                keys[seg_lo + e] = take ? 1u : 0u;
-            }
-        }
-    } else {
-        // mark the taken candidates in index order (equal keys: lowest block first)
-        int cnt = 0;
-        if (in_regs) {
-#pragma unroll
-            for (int e = 0; e < kKeysPerThread; ++e) cnt += (seg_lo + e < seg_hi && kr[e] == thr);
-        } else {
-            for (int i = seg_lo; i < seg_hi; ++i) cnt += (keys[i] == thr);
-        }
-        int tot;
-        int r = block_exclusive_scan(cnt, s_warp, &tot);
-        if (in_regs) {
+            const int ebn = s_bn;
 #pragma unroll
             for (int e = 0; e < kKeysPerThread; ++e) {
+                fl[e] = false;
                 if (seg_lo + e < seg_hi) {
-                    const uint32_t u = kr[e];
-                    const bool take = take_all || u > thr || (u == thr && r < need);
-                    r += (u == thr);
-                    keys[seg_lo + e] = take ? 1u : 0u;
+                    const uint32_t u = kr[e], mk = u & emask;
+                    if (mk > eprefix) {
+                        fl[e] = true;
+                    } else if (mk == eprefix) {
+                        // four bucket entries per 16-byte read; the zero pads never count
+                        const int idx = seg_lo + e;
+                        const uint4* bk4 = reinterpret_cast<const uint4*>(s_bkey);
+                        const int4* bi4 = reinterpret_cast<const int4*>(s_bidx);
+                        int rank = 0;
+#pragma unroll 4
+                        for (int q = 0; q < (ebn + 3) / 4; ++q) {
+                            const uint4 kq = bk4[q];
+                            const int4 iq = bi4[q];
+                            rank += (kq.x > u || (kq.x == u && iq.x < idx)) + (kq.y > u || (kq.y == u && iq.y < idx)) +
+                                    (kq.z > u || (kq.z == u && iq.z < idx)) + (kq.w > u || (kq.w == u && iq.w < idx));
+                        }
+                        fl[e] = rank < need;
+                    }
                 }
             }
+        } else if (take_all || kk == 0) {
+#pragma unroll
+            for (int e = 0; e < kKeysPerThread; ++e) fl[e] = take_all && seg_lo + e < seg_hi;
         } else {
-            for (int i = seg_lo; i < seg_hi; ++i) {
-                const uint32_t u = keys[i];
-                const bool take = take_all || u > thr || (u == thr && r < need);
-                r += (u == thr);
-                keys[i] = take ? 1u : 0u;
+            // keys above thr, and the first `need` keys equal to thr in block order
+            int cnt = 0;
+#pragma unroll
+            for (int e = 0; e < kKeysPerThread; ++e) cnt += (seg_lo + e < seg_hi && kr[e] == thr);
+            int tot;
+            int r = block_exclusive_scan(cnt, s_warp, &tot);
+#pragma unroll
+            for (int e = 0; e < kKeysPerThread; ++e) {
+                fl[e] = false;
+                if (seg_lo + e < seg_hi) {
+                    const uint32_t u = kr[e];
+                    fl[e] = u > thr || (u == thr && r < need);
+                    r += (u == thr);
+                }
             }
+        }
+        // union: init blocks, the taken candidates in block order, then the local blocks
+        int cnt = 0;
+#pragma unroll
+        for (int e = 0; e < kKeysPerThread; ++e) cnt += fl[e];
+        int taken;
+        int pos = init_end + block_exclusive_scan(cnt, s_warp, &taken, false);
+#pragma unroll
+        for (int e = 0; e < kKeysPerThread; ++e)
+            if (fl[e]) out[pos++] = seg_lo + e;
+        for (int i = tid; i < init_end; i += NT) out[i] = i;
+        const int n_loc = nb - chi;
+        for (int i = tid; i < n_loc; i += NT) out[init_end + taken + i] = chi + i;
+        const int total = init_end + taken + n_loc;
+        for (int i = total + tid; i < a.sel_cap; i += NT) out[i] = -1;
+        if (tid == 0) a.n_sel[pair] = total;
+        return;
+    }
+
+    // streamed candidates: mark the taken ones in keys[] (1 / 0), ties at thr in block order
+    {
+        int cnt = 0;
+        for (int i = seg_lo; i < seg_hi; ++i) cnt += (keys[i] == thr);
+        int tot;
+        int r = block_exclusive_scan(cnt, s_warp, &tot);
+        for (int i = seg_lo; i < seg_hi; ++i) {
+            const uint32_t u = keys[i];
+            const bool take = kk > 0 && (take_all || u > thr || (u == thr && r < need));
+            r += (u == thr);
+            keys[i] = take ? 1u : 0u;
         }
     }
     __syncthreads();
     // union with init and local blocks, emitted in ascending block order
-    int32_t* out = a.block_idx + (size_t)pair * a.sel_cap;
     {
         const int per2 = (nb + NT - 1) / NT;
         const int lo = tid * per2, hi = min(lo + per2, nb);
         int cnt = 0;
-        for (int i = lo; i < hi; ++i) cnt += (i < init_end || i >= local_begin || keys[i] != 0u);
+        for (int i = lo; i < hi; ++i) cnt += (i < init_end || i >= chi || keys[i] != 0u);
         int total;
         int pos = block_exclusive_scan(cnt, s_warp, &total);
         for (int i = lo; i < hi; ++i)
-            if (i < init_end || i >= local_begin || keys[i] != 0u) out[pos++] = i;
+            if (i < init_end || i >= chi || keys[i] != 0u) out[pos++] = i;
         for (int i = total + tid; i < a.sel_cap; i += NT) out[i] = -1;
         if (tid == 0) a.n_sel[pair] = total;
     }
@@ -644,10 +733,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
     if (part < parts_used) {
         // softmax normaliser of every head from the chunk statistics: one parallel round of
         // loads into shared memory (aliasing the key array, unused until the top-k), then warp h
-        // merges head h
+        // merges head h, and every chunk's weight per head replaces its maximum
+        float2* s_st = reinterpret_cast<float2*>(s_dyn);  // 2 * nstat * Gp <= key_words
         {
             const int64_t nch = (nc + 63) / 64;
-            float2* s_st = reinterpret_cast<float2*>(s_dyn);  // 2 * nstat * Gp <= key_words
             const float2* st = a.stats + (size_t)pair * a.nstat * a.Gp;
             for (int64_t e = tid; e < nch * a.Gp; e += kSelectThreads) s_st[e] = ld_cg(st + e);
             __syncthreads();
@@ -669,6 +758,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
                 }
             }
             __syncthreads();
+            for (int64_t e = tid; e < nch * a.Gp; e += kSelectThreads) {
+                const int h = (int)(e % a.Gp);
+                s_st[e].x = h < a.G ? exp2f(s_st[e].x - sM[h]) * sInvZ[h] : 0.f;
+            }
+            __syncthreads();
         }
         const int64_t j0 = (int64_t)part * a.part_windows;
         const int64_t j1 = min(j0 + a.part_windows, nc);
@@ -678,7 +772,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
         const int64_t jend = b_hi > b_lo ? min(last_window(b_hi - 1, a.BS, a.s) + 1, nc) : j0;
         if (jend > j0) {
             const float* lg = a.logits + (size_t)pair * a.lg_stride * a.Gp;
-            window_scores<GP>(lg, j0, jend, a.G, sM, sInvZ, S);
+            window_scores<GP>(lg, j0, jend, a.G, s_st, S);
         }
         __syncthreads();
         const int j0i = (int)j0, nci = (int)nc;
@@ -711,10 +805,13 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
     topk_union(a, pair, (int)nb, s_dyn);
 }
 
-// One CTA per pair, when there are enough pairs to fill the GPU: the pair's logits stream into a
-// ring of 16 KB shared-memory stages with 1-D bulk copies (all stages in flight at once, while the
-// chunk statistics are merged), S[j] is evaluated from shared memory, the block maxima go straight
-// to the key array and the top-k follows, with no completion counter.
+// One CTA per pair, when there are enough pairs to fill the GPU: the pair's stored e rows stream
+// into a ring of 16 KB shared-memory stages with 1-D bulk copies (the first stages are issued as
+// soon as the scores are complete, before the sequence length is read, sized by the row capacity),
+// while the chunk statistics turn into one weight per (chunk, head). S[j] is then evaluated from
+// shared memory; when the whole row fits the ring and blocks start on window boundaries, the block
+// maxima are taken with warp shuffles in the same pass, straight into the key array. The top-k
+// follows, with no completion counter.
 constexpr int kRingStage = 16 * 1024;
 constexpr int kMaxRing = 8;
 
@@ -726,6 +823,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_raw) + 127) & ~uintptr_t(127));
     uint32_t* keys = reinterpret_cast<uint32_t*>(ring + (size_t)a.ring * kRingStage);
     float* S = reinterpret_cast<float*>(keys + a.key_words);
+    float* wt = S + a.part_windows;  // [nstat][GP] chunk weights
     const int pair = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int R = a.ring;
@@ -736,69 +834,87 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     __syncthreads();
     pdl_trigger();
     pdl_wait();
-    const int64_t T = a.seq_lens[pair / a.Hkv];
-    const bool ok = T >= 0 && T <= a.T_cap;
-    const int nc = ok ? (int)num_windows(T, a.l, a.s) : 0;
-    const int nb = ok ? (int)((T + a.BS - 1) / a.BS) : 0;
     constexpr int PW = kRingStage / (GP * 4);  // windows per stage
-    const int npieces = (nc + PW - 1) / PW;
     const uint8_t* src = reinterpret_cast<const uint8_t*>(a.logits + (size_t)pair * a.lg_stride * GP);
-    auto issue = [&](int r) {  // thread 0: stage r of the pair's logits into ring slot r % R
-        const int w0 = r * PW, wn = min(PW, nc - w0);
+    // thread 0: windows [r*PW, r*PW + PW) below `limit` into ring slot r % R
+    auto issue = [&](int r, int64_t limit) {
+        const int64_t w0 = (int64_t)r * PW;
+        const int64_t wn = min((int64_t)PW, limit - w0);
         const uint32_t bytes = ((uint32_t)wn * GP * 4 + 15u) & ~15u;  // inside the padded row
         uint64_t* bar = &full[r % R];
         mbar_arrive_expect_tx(bar, bytes);
         bulk_load(ring + (size_t)(r % R) * kRingStage, src + (size_t)w0 * GP * 4, bytes, bar);
     };
+    // the sequence length and the chunk statistics (for the row capacity) in one round of loads,
+    // requested before the bulk copies so that they do not queue behind them; the statistics are
+    // staged in the key array
+    constexpr int kStatU = 4;
+    float2* s_st = reinterpret_cast<float2*>(keys);  // 2 * nstat * Gp <= key_words
+    const float2* st = a.stats + (size_t)pair * a.nstat * GP;
+    const int64_t n_st = a.nstat * GP;
+    float2 sv[kStatU];
+#pragma unroll
+    for (int u = 0; u < kStatU; ++u) {
+        const int64_t e = tid + (int64_t)u * kSelectThreads;
+        if (e < n_st) sv[u] = ld_cg(st + e);
+    }
+    const int64_t T = a.seq_lens[pair / a.Hkv];
+    __syncthreads();  // every load above has been issued
+    const int cap_pieces = (int)((a.lg_stride + PW - 1) / PW);
+    const int n_pre = min(cap_pieces, R);
     if (tid == 0)
-        for (int r = 0; r < npieces && r < R; ++r) issue(r);
-
-    // softmax normaliser of every head from the chunk statistics (staged in the key array)
-    {
-        const int nch = (nc + 63) / 64;
-        float2* s_st = reinterpret_cast<float2*>(keys);  // 2 * nstat * Gp <= key_words
-        const float2* st = a.stats + (size_t)pair * a.nstat * GP;
-        for (int e = tid; e < nch * GP; e += kSelectThreads) s_st[e] = ld_cg(st + e);
-        __syncthreads();
-        if (warp < a.G) {
-            float m = -INFINITY, sum = 0.f;
-            for (int c = lane; c < nch; c += 32) {
-                const float2 v = s_st[c * GP + warp];
-                online_merge(m, sum, v.x, v.y);
-            }
+        for (int r = 0; r < n_pre; ++r) issue(r, a.lg_stride);
 #pragma unroll
-            for (int off = 16; off > 0; off >>= 1) {
-                const float mo = __shfl_xor_sync(0xffffffffu, m, off);
-                const float so = __shfl_xor_sync(0xffffffffu, sum, off);
-                online_merge(m, sum, mo, so);
-            }
-            if (lane == 0) {
-                sM[warp] = m;
-                sInvZ[warp] = sum > 0.f ? 1.f / sum : 0.f;
-            }
+    for (int u = 0; u < kStatU; ++u) {
+        const int64_t e = tid + (int64_t)u * kSelectThreads;
+        if (e < n_st) s_st[e] = sv[u];
+    }
+    for (int64_t e = tid + (int64_t)kStatU * kSelectThreads; e < n_st; e += kSelectThreads) s_st[e] = ld_cg(st + e);
+    const bool ok = T >= 0 && T <= a.T_cap;
+    const int nc = ok ? (int)num_windows(T, a.l, a.s) : 0;
+    const int nb = ok ? (int)((T + a.BS - 1) / a.BS) : 0;
+    const int npieces = (nc + PW - 1) / PW;
+    const int nch = (nc + 63) / 64;
+    __syncthreads();
+    // softmax normaliser of every head (warp h merges head h), then each chunk's weight per head
+    if (warp < a.G) {
+        float m = -INFINITY, sum = 0.f;
+        for (int c = lane; c < nch; c += 32) {
+            const float2 v = s_st[c * GP + warp];
+            online_merge(m, sum, v.x, v.y);
         }
-        __syncthreads();
-    }
-    float M[GP], iz[GP];
 #pragma unroll
-    for (int h = 0; h < GP; ++h) {
-        M[h] = h < a.G ? sM[h] : 0.f;
-        iz[h] = h < a.G ? sInvZ[h] : 0.f;
+        for (int off = 16; off > 0; off >>= 1) {
+            const float mo = __shfl_xor_sync(0xffffffffu, m, off);
+            const float so = __shfl_xor_sync(0xffffffffu, sum, off);
+            online_merge(m, sum, mo, so);
+        }
+        if (lane == 0) {
+            sM[warp] = m;
+            sInvZ[warp] = sum > 0.f ? 1.f / sum : 0.f;
+        }
     }
-    // S[j] = sum_h exp2(x[j][h] - M_h) / Z_h for window j at index i of the stage in slot `slot`
-    auto window_score = [&](int slot, int i) -> float {
-        const float* lg = reinterpret_cast<const float*>(ring + (size_t)slot * kRingStage);
+    __syncthreads();
+    for (int e = tid; e < nch * GP; e += kSelectThreads) {
+        const int h = e % GP;
+        wt[e] = h < a.G ? exp2f(s_st[e].x - sM[h]) * sInvZ[h] : 0.f;
+    }
+    __syncthreads();
+    // S[j] = sum_h e[j][h] * w[j / 64][h], for window j at index i of the stage in slot `slot`
+    auto window_score = [&](int slot, int i, int j) -> float {
+        const float* lg = reinterpret_cast<const float*>(ring + (size_t)slot * kRingStage) + (size_t)i * GP;
+        const float* w = wt + (j >> 6) * GP;
         float x[GP];
         if constexpr (GP == 1) {
-            x[0] = lg[i];
+            x[0] = lg[0];
         } else if constexpr (GP == 2) {
-            const float2 t = reinterpret_cast<const float2*>(lg)[i];
+            const float2 t = *reinterpret_cast<const float2*>(lg);
             x[0] = t.x;
             x[1] = t.y;
         } else {
 #pragma unroll
             for (int q = 0; q < GP / 4; ++q) {
-                const float4 t = reinterpret_cast<const float4*>(lg + (size_t)i * GP)[q];
+                const float4 t = reinterpret_cast<const float4*>(lg)[q];
                 x[4 * q] = t.x;
                 x[4 * q + 1] = t.y;
                 x[4 * q + 2] = t.z;
@@ -808,17 +924,63 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
         float acc = 0.f;
 #pragma unroll
         for (int h = 0; h < GP; ++h)
-            if (h < a.G) acc += exp2f(x[h] - M[h]) * iz[h];
+            if (h < a.G) acc += x[h] * w[h];
         return acc;
     };
+    // blocks start on window boundaries: block b's windows are [rb - (L - 1), rb + r - 1], with
+    // r = BS / s a power of two up to 32 and L = l / s in {1, 2}
+    const int r_w = a.BS / a.s, L_w = a.l / a.s;
+    const bool shuffle_max = a.BS % a.s == 0 && a.l % a.s == 0 && r_w >= 1 && r_w <= 32 &&
+                             (r_w & (r_w - 1)) == 0 && (L_w == 1 || L_w == 2) && nc > 0;
+    bool keys_done = false;
     if (npieces <= R) {
-        // every stage is in flight from the start: wait for all, then one pass over the windows
+        // every stage needed is in flight from the start: wait for all that were issued
         bool waited = true;
-        for (int r = 0; r < npieces && waited; ++r) waited = mbar_wait(&full[r], 0, kScoreWaitPolls);
+        for (int r = 0; r < n_pre && waited; ++r) waited = mbar_wait(&full[r], 0, kScoreWaitPolls);
         if (!waited) {
             if (tid == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+        } else if (shuffle_max) {
+            // warp w takes a contiguous run of 32-window tiles: lane l scores window 32t + l (the
+            // stages are contiguous in shared memory, so window j sits at index j of slot 0); the
+            // lanes then take running maxima over groups of r lanes, and lane r*i adds window
+            // 32t + r*i - 1 when L = 2 (lane 31 of the previous tile for i = 0)
+            const int bpt = 32 / r_w;  // blocks per tile
+            const int tiles = (nb + bpt - 1) / bpt;
+            const int nw = kSelectThreads / 32;
+            const int t_lo = (int)((int64_t)warp * tiles / nw), t_hi = (int)((int64_t)(warp + 1) * tiles / nw);
+            auto S_at = [&](int j) -> float {
+                const float v = window_score(0, min(j, nc - 1), min(j, nc - 1));
+                return j < nc ? v : -INFINITY;
+            };
+            // four tiles at a time, their shared-memory reads in flight together
+            constexpr int kTileU = 4;
+            float prev = t_lo > 0 ? S_at(32 * t_lo - 32 + lane) : -INFINITY;
+            for (int t0 = t_lo; t0 < t_hi; t0 += kTileU) {
+                float cur[kTileU];
+#pragma unroll
+                for (int u = 0; u < kTileU; ++u) cur[u] = t0 + u < t_hi ? S_at(32 * (t0 + u) + lane) : -INFINITY;
+#pragma unroll
+                for (int u = 0; u < kTileU; ++u) {
+                    const int t = t0 + u;
+                    if (t >= t_hi) break;  // warp-uniform
+                    float m = cur[u];
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1)
+                        if (off < r_w) m = fmaxf(m, __shfl_down_sync(0xffffffffu, m, off));
+                    const float before = __shfl_up_sync(0xffffffffu, cur[u], 1);
+                    const float last_prev = __shfl_sync(0xffffffffu, u == 0 ? prev : cur[u > 0 ? u - 1 : 0], 31);
+                    if (L_w == 2) m = fmaxf(m, lane == 0 ? last_prev : before);
+                    const int b = t * bpt + lane / r_w;
+                    if ((lane & (r_w - 1)) == 0 && b < nb) {
+                        keys[b] = order_key(m);
+                        if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + b] = m;
+                    }
+                }
+                prev = cur[kTileU - 1];
+            }
+            keys_done = true;
         } else {
-            for (int j = tid; j < nc; j += kSelectThreads) S[j] = window_score(j / PW, j % PW);
+            for (int j = tid; j < nc; j += kSelectThreads) S[j] = window_score(0, j, j);
         }
     } else {
         for (int r = 0; r < npieces; ++r) {
@@ -827,23 +989,25 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
                 break;
             }
             const int w0 = r * PW, wn = min(PW, nc - w0);
-            for (int i = tid; i < wn; i += kSelectThreads) S[w0 + i] = window_score(r % R, i);
+            for (int i = tid; i < wn; i += kSelectThreads) S[w0 + i] = window_score(r % R, i, w0 + i);
             __syncthreads();  // the slot has been read by everyone
             if (tid == 0 && r + R < npieces) {
                 fence_proxy_async_smem();
-                issue(r + R);
+                issue(r + R, nc);
             }
         }
     }
     __syncthreads();
-    // block scores: the maximum of S over the complete windows overlapping each block
-    for (int b = tid; b < nb; b += kSelectThreads) {
-        float best = -INFINITY;
-        const int jlo = (int)first_window32(b, a.BS, a.l, a.s);
-        const int jhi = min((int)last_window32(b, a.BS, a.s), nc - 1);
-        for (int j = jlo; j <= jhi; ++j) best = fmaxf(best, S[j]);
-        keys[b] = order_key(best);
-        if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + b] = best;
+    if (!keys_done) {
+        // block scores: the maximum of S over the complete windows overlapping each block
+        for (int b = tid; b < nb; b += kSelectThreads) {
+            float best = -INFINITY;
+            const int jlo = (int)first_window32(b, a.BS, a.l, a.s);
+            const int jhi = min((int)last_window32(b, a.BS, a.s), nc - 1);
+            for (int j = jlo; j <= jhi; ++j) best = fmaxf(best, S[j]);
+            keys[b] = order_key(best);
+            if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + b] = best;
+        }
     }
     if (a.block_scores)
         for (int64_t b = nb + tid; b < a.nb_cap; b += kSelectThreads)
@@ -899,7 +1063,8 @@ template <int GP>
 cudaError_t launch_select_k(const Plan& p, const SelectArgs& a, cudaStream_t st) {
     if (p.select_ring > 0) {
         const size_t smem = 128 + (size_t)p.select_ring * kRingStage +
-                            (p.select_keys + (size_t)p.select_part_windows) * sizeof(uint32_t);
+                            (p.select_keys + (size_t)p.select_part_windows + (size_t)p.nstat * p.Gp) *
+                                sizeof(uint32_t);
         cudaError_t e = ensure_smem<select_single_kernel<GP>>(smem);
         if (e != cudaSuccess) return e;
         return launch_pdl(select_single_kernel<GP>, dim3((unsigned)p.pairs), dim3(kSelectThreads),

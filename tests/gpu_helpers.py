@@ -168,7 +168,22 @@ def check_selection(run: GpuRun, pairs: list[int], orc: dict) -> list[int]:
             assert idx[pr, :n_o].tolist() == orc["idx"][i, :n_o].tolist(), \
                 f"pair {pr}: idx {idx[pr, :n_o].tolist()} vs oracle {orc['idx'][i, :n_o].tolist()}"
         assert np.all(idx[pr, n_o:] == -1), f"pair {pr}: padding"
+        # the selection is exactly the top-k of the kernel's own block scores (ties: lower block)
+        want_idx = topk_union_of(sc[pr, :nb].astype(np.float32), nb, w.n_init, w.n_local, w.top_k)
+        assert idx[pr, :int(ns[pr])].tolist() == want_idx, \
+            f"pair {pr}: selection is not the top-k of the returned block scores"
     return ties
+
+
+def topk_union_of(scores: np.ndarray, nb: int, n_init: int, n_local: int, top_k: int) -> list[int]:
+    """Init blocks, the top_k candidates by score (ties: lower block first) and the local blocks,
+    ascending: the selection rule applied to given block scores."""
+    init_end = min(n_init, nb)
+    chi = max(nb - n_local, init_end)
+    cand = np.arange(init_end, chi)
+    kk = min(top_k, len(cand))
+    order = cand[np.lexsort((cand, -scores[cand].astype(np.float64)))] if len(cand) else cand
+    return list(range(init_end)) + sorted(order[:kk].tolist()) + list(range(chi, nb))
 
 
 def check_output(run: GpuRun, pairs: list[int], orc: dict, layer=0, skip=()):

@@ -84,6 +84,44 @@ def test_ragged_batch_lengths(cuda_device):
     assert (run.out[0][3] == 0).all() and torch.isneginf(run.lse[0][3]).all()
 
 
+def test_equal_scores_take_lowest_blocks(cuda_device):
+    """q = 0: every window has the same score, so every candidate block ties and the lowest
+    candidate blocks are taken."""
+    w = BASE.replace(name="x", batch=1, num_q_heads=4, num_kv_heads=1, seq_len=5000, top_k=8,
+                     needles=0)
+    run = GpuRun(w)
+    run.data["q"][0].zero_()
+    run.compress()
+    run.select()
+    run.decode()
+    assert run.device_errors() == 0
+    nb = -(-5000 // w.block_size)
+    init_end, chi = w.n_init, nb - w.n_local
+    want = list(range(init_end)) + list(range(init_end, init_end + w.top_k)) + list(range(chi, nb))
+    assert run.n_sel[0, 0].item() == len(want)
+    assert run.block_idx[0, 0, :len(want)].tolist() == want
+    full_check(run, [0])
+
+
+@pytest.mark.parametrize("seq_len", [20000, 40000])
+def test_periodic_keys_many_ties(seq_len, cuda_device):
+    """Keys that repeat every 256 tokens give block scores that repeat every four blocks: the k-th
+    largest sits in a group of equal scores (about 80 or 160 of them), ranked by block index."""
+    w = BASE.replace(name="x", batch=1, num_q_heads=8, num_kv_heads=2, seq_len=seq_len, top_k=50,
+                     needles=0)
+    run = GpuRun(w)
+    k = run.data["k"][0]
+    period = 256
+    reps = -(-seq_len // period)
+    tiled = k[:, :, :period].repeat(1, 1, reps, 1)[:, :, :seq_len]
+    k[:, :, :seq_len] = tiled
+    run.compress()
+    run.select()
+    run.decode()
+    assert run.device_errors() == 0
+    full_check(run, [0, 1])
+
+
 def test_long_context_large_block_count(cuda_device):
     """nb_cap = 16384 blocks: the selection keeps 64 KB of keys in shared memory."""
     w = BASE.replace(name="x", batch=1, num_q_heads=4, num_kv_heads=1, seq_len=300000, top_k=40,
