@@ -498,17 +498,51 @@ __device__ __forceinline__ void find_digit_from_top(const int* hist, int nbins, 
     __syncthreads();
 }
 
-__device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys) {
-    __shared__ int s_warp[32];
-    __shared__ __align__(16) int hist[kHistBins];
-    __shared__ int s_digit, s_need, s_bcnt, s_bn;
-    __shared__ uint32_t s_and[32], s_or[32];
-    __shared__ __align__(16) uint32_t s_bkey[kExactMax];  // 0 pads: below every real key
-    __shared__ __align__(16) int s_bidx[kExactMax];
+// The top-k's shared memory, declared by each selection kernel.
+struct TopkSmem {
+    int warp[32];
+    __align__(16) int hist[kHistBins];
+    int digit, need, bcnt, bn;
+    uint32_t kand[32], kor[32];                 // each warp's AND / OR of candidate keys
+    __align__(16) uint32_t bkey[kExactMax];     // 0 pads: below every real key
+    __align__(16) int bidx[kExactMax];
+};
+
+// Candidate blocks [init_end(nb), cand_end(nb)): neither init nor local.
+__device__ __forceinline__ int cand_begin(const SelectArgs& a, int nb) { return min(a.n_init, nb); }
+__device__ __forceinline__ int cand_end(const SelectArgs& a, int nb) {
+    return max(max(nb - a.n_local, 0), min(a.n_init, nb));
+}
+
+// Clears the first digit's bins and the exact bucket; a barrier must follow before topk_union.
+__device__ __forceinline__ void topk_prepare(TopkSmem& t) {
+    for (int i = threadIdx.x; i < kHistBins / 4; i += blockDim.x)
+        reinterpret_cast<int4*>(t.hist)[i] = make_int4(0, 0, 0, 0);
+    for (int i = threadIdx.x; i < kExactMax; i += blockDim.x) t.bkey[i] = 0u;
+    if (threadIdx.x == 0) t.bn = 0;
+}
+
+// Publishes a warp's AND / OR of the candidate keys it wrote (identity values when none).
+__device__ __forceinline__ void publish_andor(TopkSmem& t, uint32_t kand, uint32_t kor) {
+    kand = __reduce_and_sync(0xffffffffu, kand);
+    kor = __reduce_or_sync(0xffffffffu, kor);
+    if ((threadIdx.x & 31) == 0) {
+        t.kand[threadIdx.x >> 5] = kand;
+        t.kor[threadIdx.x >> 5] = kor;
+    }
+}
+
+// `andor_ready`: every warp has published the AND / OR of the candidate keys it wrote (then no
+// pass over the keys is needed for them). topk_prepare and a barrier come before the call.
+__device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys, TopkSmem& t,
+                           bool andor_ready) {
+    int* s_warp = t.warp;
+    int* hist = t.hist;
+    uint32_t* s_bkey = t.bkey;
+    int* s_bidx = t.bidx;
     const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31;
-    const int init_end = min(a.n_init, nb);
-    const int local_begin = max(nb - a.n_local, 0);
-    const int clo = init_end, chi = max(local_begin, init_end);
+    const int init_end = cand_begin(a, nb);
+    const int clo = init_end, chi = cand_end(a, nb);
     const int ncand = chi - clo;
     const int kk = min(a.top_k, ncand);
     const bool take_all = (kk == ncand);
@@ -518,9 +552,6 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
     uint32_t kr[kKeysPerThread];
 #pragma unroll
     for (int e = 0; e < kKeysPerThread; ++e) kr[e] = (in_regs && seg_lo + e < seg_hi) ? keys[seg_lo + e] : 0u;
-    for (int i = tid; i < kHistBins / 4; i += NT) reinterpret_cast<int4*>(hist)[i] = make_int4(0, 0, 0, 0);
-    for (int i = tid; i < kExactMax; i += NT) s_bkey[i] = 0u;
-    if (tid == 0) s_bn = 0;
 
     uint32_t thr = 0xffffffffu;  // keys > thr are taken, plus the first `need` keys == thr
     int need = 0;
@@ -528,33 +559,29 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
     uint32_t emask = 0u, eprefix = 0u;
     if (kk > 0 && !take_all) {
         // bits that every candidate shares need no histogram pass (block-wide AND / OR)
-        uint32_t kand = 0xffffffffu, kor = 0u;
-        if (in_regs) {
+        if (!andor_ready) {
+            uint32_t kand = 0xffffffffu, kor = 0u;
+            if (in_regs) {
 #pragma unroll
-            for (int e = 0; e < kKeysPerThread; ++e) {
-                if (seg_lo + e < seg_hi) {
-                    kand &= kr[e];
-                    kor |= kr[e];
+                for (int e = 0; e < kKeysPerThread; ++e) {
+                    if (seg_lo + e < seg_hi) {
+                        kand &= kr[e];
+                        kor |= kr[e];
+                    }
+                }
+            } else {
+                for (int i = seg_lo; i < seg_hi; ++i) {
+                    kand &= keys[i];
+                    kor |= keys[i];
                 }
             }
-        } else {
-            for (int i = seg_lo; i < seg_hi; ++i) {
-                kand &= keys[i];
-                kor |= keys[i];
-            }
+            publish_andor(t, kand, kor);
+            __syncthreads();
         }
-        kand = __reduce_and_sync(0xffffffffu, kand);
-        kor = __reduce_or_sync(0xffffffffu, kor);
-        if (lane == 0) {
-            s_and[tid >> 5] = kand;
-            s_or[tid >> 5] = kor;
-        }
-        __syncthreads();
-        kand = 0xffffffffu;
-        kor = 0u;
+        uint32_t kand = 0xffffffffu, kor = 0u;
         for (int w = 0; w < (NT >> 5); ++w) {
-            kand &= s_and[w];
-            kor |= s_or[w];
+            kand &= t.kand[w];
+            kor |= t.kor[w];
         }
         const uint32_t diff = kand ^ kor;  // bits in which some candidates differ
         uint32_t prefix = kand, mask = 0xffffffffu;
@@ -583,12 +610,12 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
                     }
                 }
                 __syncthreads();
-                find_digit_from_top(hist, nbins, need, s_warp, &s_digit, &s_need, &s_bcnt);
-                prefix |= (uint32_t)s_digit << shift;
-                need = s_need;
+                find_digit_from_top(hist, nbins, need, s_warp, &t.digit, &t.need, &t.bcnt);
+                prefix |= (uint32_t)t.digit << shift;
+                need = t.need;
                 mask |= dmask << shift;
                 if (shift == 0) break;  // every bit decided: the bucket's keys are all equal
-                if (in_regs && s_bcnt <= kExactMax) {
+                if (in_regs && t.bcnt <= kExactMax) {
                     exact = true;
                     break;
                 }
@@ -612,13 +639,13 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
 #pragma unroll
             for (int e = 0; e < kKeysPerThread; ++e) {
                 if (seg_lo + e < seg_hi && (kr[e] & emask) == eprefix) {
-                    const int slot = atomicAdd(&s_bn, 1);
+                    const int slot = atomicAdd(&t.bn, 1);
                     s_bkey[slot] = kr[e];
                     s_bidx[slot] = seg_lo + e;
                 }
             }
             __syncthreads();
-            const int ebn = s_bn;
+            const int ebn = t.bn;
 #pragma unroll
             for (int e = 0; e < kKeysPerThread; ++e) {
                 fl[e] = false;
@@ -717,6 +744,7 @@ template <int GP>
 __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a) {
     extern __shared__ uint32_t s_dyn[];  // [key_words] keys, then [PW + W_max] window scores
     __shared__ float sM[kMaxG], sInvZ[kMaxG];
+    __shared__ TopkSmem tk;
     __shared__ int s_last;
     const int pair = blockIdx.x / a.parts, part = blockIdx.x - pair * a.parts;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -801,8 +829,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
     if (!s_last) return;
     __threadfence();
     for (int64_t b = tid; b < nb; b += kSelectThreads) s_dyn[b] = order_key(ld_cg(bs + b));
+    topk_prepare(tk);
     __syncthreads();
-    topk_union(a, pair, (int)nb, s_dyn);
+    topk_union(a, pair, (int)nb, s_dyn, tk, false);
 }
 
 // One CTA per pair, when there are enough pairs to fill the GPU: the pair's stored e rows stream
@@ -819,7 +848,7 @@ template <int GP>
 __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(SelectArgs a) {
     extern __shared__ __align__(128) uint8_t s_raw[];
     __shared__ __align__(8) uint64_t full[kMaxRing];
-    __shared__ float sM[kMaxG], sInvZ[kMaxG];
+    __shared__ TopkSmem tk;
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_raw) + 127) & ~uintptr_t(127));
     uint32_t* keys = reinterpret_cast<uint32_t*>(ring + (size_t)a.ring * kRingStage);
     float* S = reinterpret_cast<float*>(keys + a.key_words);
@@ -876,7 +905,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     const int npieces = (nc + PW - 1) / PW;
     const int nch = (nc + 63) / 64;
     __syncthreads();
-    // softmax normaliser of every head (warp h merges head h), then each chunk's weight per head
+    // warp h merges head h's chunk statistics into its normaliser (M_h, Z_h), which every lane
+    // then holds, and weighs the head's chunks: w[c][h] = exp2(m_c - M_h) / Z_h
     if (warp < a.G) {
         float m = -INFINITY, sum = 0.f;
         for (int c = lane; c < nch; c += 32) {
@@ -889,15 +919,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
             const float so = __shfl_xor_sync(0xffffffffu, sum, off);
             online_merge(m, sum, mo, so);
         }
-        if (lane == 0) {
-            sM[warp] = m;
-            sInvZ[warp] = sum > 0.f ? 1.f / sum : 0.f;
-        }
-    }
-    __syncthreads();
-    for (int e = tid; e < nch * GP; e += kSelectThreads) {
-        const int h = e % GP;
-        wt[e] = h < a.G ? exp2f(s_st[e].x - sM[h]) * sInvZ[h] : 0.f;
+        const float iz = sum > 0.f ? 1.f / sum : 0.f;
+        for (int c = lane; c < nch; c += 32) wt[c * GP + warp] = exp2f(s_st[c * GP + warp].x - m) * iz;
     }
     __syncthreads();
     // S[j] = sum_h e[j][h] * w[j / 64][h], for window j at index i of the stage in slot `slot`
@@ -933,6 +956,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     const bool shuffle_max = a.BS % a.s == 0 && a.l % a.s == 0 && r_w >= 1 && r_w <= 32 &&
                              (r_w & (r_w - 1)) == 0 && (L_w == 1 || L_w == 2) && nc > 0;
     bool keys_done = false;
+    uint32_t kand = 0xffffffffu, kor = 0u;  // over the candidate keys this thread writes
     if (npieces <= R) {
         // every stage needed is in flight from the start: wait for all that were issued
         bool waited = true;
@@ -955,6 +979,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
             // four tiles at a time, their shared-memory reads in flight together
             constexpr int kTileU = 4;
             float prev = t_lo > 0 ? S_at(32 * t_lo - 32 + lane) : -INFINITY;
+            const int clo = cand_begin(a, nb), chi = cand_end(a, nb);
             for (int t0 = t_lo; t0 < t_hi; t0 += kTileU) {
                 float cur[kTileU];
 #pragma unroll
@@ -972,7 +997,12 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
                     if (L_w == 2) m = fmaxf(m, lane == 0 ? last_prev : before);
                     const int b = t * bpt + lane / r_w;
                     if ((lane & (r_w - 1)) == 0 && b < nb) {
-                        keys[b] = order_key(m);
+                        const uint32_t key = order_key(m);
+                        keys[b] = key;
+                        if (b >= clo && b < chi) {
+                            kand &= key;
+                            kor |= key;
+                        }
                         if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + b] = m;
                     }
                 }
@@ -1000,20 +1030,28 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     __syncthreads();
     if (!keys_done) {
         // block scores: the maximum of S over the complete windows overlapping each block
+        const int clo = cand_begin(a, nb), chi = cand_end(a, nb);
         for (int b = tid; b < nb; b += kSelectThreads) {
             float best = -INFINITY;
             const int jlo = (int)first_window32(b, a.BS, a.l, a.s);
             const int jhi = min((int)last_window32(b, a.BS, a.s), nc - 1);
             for (int j = jlo; j <= jhi; ++j) best = fmaxf(best, S[j]);
-            keys[b] = order_key(best);
+            const uint32_t key = order_key(best);
+            keys[b] = key;
+            if (b >= clo && b < chi) {
+                kand &= key;
+                kor |= key;
+            }
             if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + b] = best;
         }
     }
     if (a.block_scores)
         for (int64_t b = nb + tid; b < a.nb_cap; b += kSelectThreads)
             a.block_scores[(size_t)pair * a.nb_cap + b] = -INFINITY;
+    publish_andor(tk, kand, kor);
+    topk_prepare(tk);
     __syncthreads();
-    topk_union(a, pair, nb, keys);
+    topk_union(a, pair, nb, keys, tk, true);
 }
 
 int sm_count() {
