@@ -290,6 +290,11 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_f32_kernel(ScoreArgs a
     pdl_trigger();
     pdl_wait();
     report_lengths(a);
+    // the warp's chunk: x staged in shared memory, written out as e = exp2(x - max) at the end
+    __shared__ float s_x[kScoreWarps][64 * kMaxG];
+    __shared__ float s_m[kScoreWarps][kMaxG];
+    float* sx = s_x[threadIdx.x >> 5];
+    float* sm = s_m[threadIdx.x >> 5];
     int cur_pair = -1;
     int64_t nc = 0;
     float qv[kMaxG][E];
@@ -343,23 +348,27 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_f32_kernel(ScoreArgs a
                 for (int u = 0; u < kRowU; ++u) {
                     if (rg + u < r1) {
                         const float x = p[u] * a.score_log2;
-                        if (lane == h) lg[(rg + u) * a.Gp + h] = x;
+                        if (lane == h) sx[(rg + u - r0) * a.Gp + h] = x;
                         online_add(m[h], s[h], x);
                     }
                 }
             }
         }
         float2* st = a.stats + ((size_t)pair * a.nstat + ci) * a.Gp;
-        float mh = 0.f;
 #pragma unroll
         for (int h = 0; h < kMaxG; ++h)
             if (h < a.G && lane == h) {
                 st[h] = make_float2(m[h], s[h]);
-                mh = m[h];
+                sm[h] = m[h];
             }
-        // the chunk's e = exp2(x - max) replaces the logits that lane h stored above
-        if (lane < a.G)
-            for (int64_t r = r0; r < r1; ++r) lg[r * a.Gp + lane] = exp2f(lg[r * a.Gp + lane] - mh);
+        __syncwarp();
+        // the chunk's rows, coalesced: e = exp2(x - max) (0 in the padding heads)
+        const int nvals = (int)(r1 - r0) * a.Gp;
+        for (int e = lane; e < nvals; e += 32) {
+            const int h = e % a.Gp;
+            lg[r0 * a.Gp + e] = h < a.G ? exp2f(sx[e] - sm[h]) : 0.f;
+        }
+        __syncwarp();
     }
 }
 
