@@ -83,12 +83,15 @@ def _bind(path: str):
         "bsa_oracle_num_blocks": (_I64, [_I64, _INT]),
         "bsa_oracle_compress": (_I64, [_P, _INT, _I64, _INT, _INT, _INT, _INT, _P]),
         "bsa_oracle_group_scores": (None, [_P, _P, _I64, _INT, _INT, _D, _P]),
+        "bsa_oracle_forecast_scores": (None, [_P, _P, _I64, _INT, _P]),
         "bsa_oracle_block_scores": (None, [_P, _I64, _I64, _INT, _INT, _INT, _P]),
         "bsa_oracle_select": (_INT, [_P, _I64, _INT, _INT, _INT, _P, _P]),
         "bsa_oracle_attend": (None, [_P, _P, _P, _INT, _I64, _INT, _INT, _P, _INT, _INT,
                                      _D, _P, _P]),
         "bsa_oracle_decode": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _INT,
                                      _P, _P, _P, _P, _P, _P, _P, _P]),
+        "bsa_oracle_decode_forecast": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P,
+                                              _INT, _P, _P, _P, _P, _P, _P]),
         "bsa_oracle_attend_pairs": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P,
                                            _INT, _P, _P, _P, _P]),
         "bsa_oracle_compress_cache": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _INT,
@@ -201,6 +204,15 @@ def group_scores(q, ck, tau: float) -> np.ndarray:
     return S
 
 
+def forecast_scores(f, ck) -> np.ndarray:
+    """Eq. (4) with the Compact Forecast Indexer: f [d], ck [nc][d] -> S [nc] = f . ck_j."""
+    f, ck = _f64(f), _f64(ck)
+    nc, d = ck.shape
+    S = np.zeros(nc, dtype=np.float64)
+    _load().bsa_oracle_forecast_scores(_ptr(f), _ptr(ck), nc, d, _ptr(S))
+    return S
+
+
 def block_scores(S, nb: int, l: int = 32, s: int = 16, block_size: int = 64) -> np.ndarray:
     S = _f64(S)
     sb = np.zeros(nb, dtype=np.float64)
@@ -284,6 +296,35 @@ def decode(P: Problem, q, k_cache, v_cache, seq_lens, pairs=None, given_idx=None
         _ptr(res["block_scores"]), _ptr(res["boundary"]), _ptr(res["out"]), _ptr(res["lse"]))
     if rc != 0:
         raise ValueError("bsa_oracle_decode rejected its arguments")
+    return res
+
+
+def decode_forecast(P: Problem, f, q, k_cache, v_cache, seq_lens, pairs=None) -> dict:
+    """As ``decode``, with the blocks selected from the Forecast vectors f [B][Hkv][d] (storage
+    array of the problem's dtype) instead of the queries; q attends them."""
+    f = _raw_check(f, P.dtype)
+    q = _raw_check(q, P.dtype)
+    k_cache, v_cache = _raw_check(k_cache, P.dtype), _raw_check(v_cache, P.dtype)
+    seq_lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    if pairs is None:
+        pairs = np.arange(P.batch * P.num_kv_heads, dtype=np.int32)
+    pairs = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32))
+    n = pairs.size
+    G, sel_cap, nb_cap = _sizes(P)
+    res = dict(
+        idx=np.full((n, sel_cap), -1, dtype=np.int32),
+        n_sel=np.zeros(n, dtype=np.int32),
+        block_scores=np.full((n, nb_cap), -np.inf, dtype=np.float64),
+        boundary=np.full((n, 2), np.nan, dtype=np.float64),
+        out=np.zeros((n, G, P.head_dim), dtype=np.float64),
+        lse=np.zeros((n, G), dtype=np.float64),
+    )
+    rc = _load().bsa_oracle_decode_forecast(
+        ctypes.byref(P), _ptr(f), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+        _ptr(pairs), n, _ptr(res["idx"]), _ptr(res["n_sel"]), _ptr(res["block_scores"]),
+        _ptr(res["boundary"]), _ptr(res["out"]), _ptr(res["lse"]))
+    if rc != 0:
+        raise ValueError("bsa_oracle_decode_forecast rejected its arguments")
     return res
 
 

@@ -87,6 +87,16 @@ void bsa_oracle_group_scores(const double* q, const double* ck, int64_t nc, int 
     free(x);
 }
 
+/* SparDA Architecture, Eq. (4), with the Compact Forecast Indexer: one Forecast vector f per GQA
+ * group scores every compressed key as f . K~_j, with no softmax. */
+void bsa_oracle_forecast_scores(const double* f, const double* ck, int64_t nc, int d, double* S) {
+    for (int64_t j = 0; j < nc; ++j) {
+        double dot = 0.0;
+        for (int c = 0; c < d; ++c) dot += f[c] * ck[j * d + c];
+        S[j] = dot;
+    }
+}
+
 /* Fine-grained supervision: scores max-pooled down to the standard block grid. A window overlaps
  * block b when it shares at least one token with [BS*b, BS*(b+1)). */
 void bsa_oracle_block_scores(const double* S, int64_t nc, int64_t nb, int l, int s,
@@ -225,7 +235,8 @@ static const void* orc_pair_rows(const orc_problem_t* P, const void* cache, int 
     return (const char*)cache + off;
 }
 
-int bsa_oracle_decode(const orc_problem_t* P, const void* q, const void* k_cache,
+/* Select (from q, or from the Forecast vectors f when given) and attend, per listed pair. */
+static int orc_decode(const orc_problem_t* P, const void* f, const void* q, const void* k_cache,
                       const void* v_cache, const int32_t* seq_lens, const int32_t* pairs,
                       int n_pairs, const int32_t* given_idx, const int32_t* given_n_sel,
                       int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary,
@@ -273,7 +284,14 @@ int bsa_oracle_decode(const orc_problem_t* P, const void* q, const void* k_cache
             double* sb = (double*)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(double));
             double bnd[2];
             bsa_oracle_compress(kp, P->dtype, T, d, P->cmp_kernel, P->cmp_stride, P->dtype, ck);
-            bsa_oracle_group_scores(qg, ck, nc, G, d, P->tau, S);
+            if (f) {
+                double* fv = (double*)malloc((size_t)d * sizeof(double));
+                for (int c = 0; c < d; ++c) fv[c] = bsa_oracle_load(f, P->dtype, (int64_t)pair * d + c);
+                bsa_oracle_forecast_scores(fv, ck, nc, d, S);
+                free(fv);
+            } else {
+                bsa_oracle_group_scores(qg, ck, nc, G, d, P->tau, S);
+            }
             bsa_oracle_block_scores(S, nc, nb, P->cmp_kernel, P->cmp_stride, P->block_size, sb);
             ns = bsa_oracle_select(sb, nb, P->n_init, P->n_local, P->top_k, my_idx, bnd);
             if (bs)
@@ -292,6 +310,26 @@ int bsa_oracle_decode(const orc_problem_t* P, const void* q, const void* k_cache
         free(qg);
     }
     return bad ? -1 : 0;
+}
+
+int bsa_oracle_decode(const orc_problem_t* P, const void* q, const void* k_cache,
+                      const void* v_cache, const int32_t* seq_lens, const int32_t* pairs,
+                      int n_pairs, const int32_t* given_idx, const int32_t* given_n_sel,
+                      int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary,
+                      double* out, double* lse) {
+    return orc_decode(P, NULL, q, k_cache, v_cache, seq_lens, pairs, n_pairs, given_idx,
+                      given_n_sel, idx, n_sel, block_scores, boundary, out, lse);
+}
+
+/* SparDA Architecture: the blocks of Eq. (4), selected with the Forecast vectors f [B][Hkv][d]
+ * (one per GQA group), attended by the queries q as in Eq. (5). */
+int bsa_oracle_decode_forecast(const orc_problem_t* P, const void* f, const void* q,
+                               const void* k_cache, const void* v_cache, const int32_t* seq_lens,
+                               const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel,
+                               double* block_scores, double* boundary, double* out, double* lse) {
+    if (!f) return -1;
+    return orc_decode(P, f, q, k_cache, v_cache, seq_lens, pairs, n_pairs, NULL, NULL, idx, n_sel,
+                      block_scores, boundary, out, lse);
 }
 
 int bsa_oracle_attend_pairs(const orc_problem_t* P, const void* q, const void* k_cache,

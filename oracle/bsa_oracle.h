@@ -15,7 +15,10 @@
  *       - Theoretical Foundation, Eq. (1): block set = init blocks U local blocks U top-k blocks.
  *       - Theoretical Foundation, Eq. (2): compressed key = mean of K over a window of
  *         l = 32 rows starting at stride s = 16.
- *       - SparDA Architecture, Eq. (4): f_top, the top-k of the block scores.
+ *       - SparDA Architecture, Eq. (4): f_top, the top-k of the block scores; the Forecast F_l of
+ *         layer l scores the compressed keys of layer l + 1 (F_l K~^T).
+ *       - SparDA Architecture, "Compact Forecast Indexer": one Forecast head per GQA group, and no
+ *         softmax normalisation of its scores.
  *       - SparDA Architecture, Eq. (5): exact attention over the selected blocks only.
  *       - Indexer Training, Eq. (6): the original selector's score of a GQA group is the sum over the
  *         group's heads of softmax(q_h K~^T / tau).
@@ -79,6 +82,10 @@ int64_t bsa_oracle_compress(const void* k, int dtype, int64_t T, int d, int l, i
 void bsa_oracle_group_scores(const double* q, const double* ck, int64_t nc, int G, int d,
                              double tau, double* S);
 
+/* Eq. (4) with the Compact Forecast Indexer: S[j] = f . ck_j for one group's Forecast vector
+ * f [d] (no softmax). ck is [nc][d]. */
+void bsa_oracle_forecast_scores(const double* f, const double* ck, int64_t nc, int d, double* S);
+
 /* Max of S over the complete windows overlapping each block, -inf where there is none. */
 void bsa_oracle_block_scores(const double* S, int64_t nc, int64_t nb, int l, int s,
                              int block_size, double* sb);
@@ -120,6 +127,14 @@ int bsa_oracle_decode(const orc_problem_t* P, const void* q, const void* k_cache
                       int n_pairs, const int32_t* given_idx, const int32_t* given_n_sel,
                       int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary,
                       double* out, double* lse);
+
+/* As bsa_oracle_decode, but the blocks are selected from the Forecast vectors f [B][Hkv][d]
+ * (type dtype, one per GQA group) with bsa_oracle_forecast_scores in place of the group scores;
+ * q still attends them. block_scores hold the max-pooled raw forecast scores. */
+int bsa_oracle_decode_forecast(const orc_problem_t* P, const void* f, const void* q,
+                               const void* k_cache, const void* v_cache, const int32_t* seq_lens,
+                               const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel,
+                               double* block_scores, double* boundary, double* out, double* lse);
 
 /* [CLSA]/[Kascade] shared index: attend one layer's q/K/V with block indices computed elsewhere
  * (by bsa_oracle_decode on the anchor layer). Same layouts as bsa_oracle_decode. */

@@ -166,6 +166,23 @@ def pin_scores_closed_form():
     np.testing.assert_allclose(S, [2.0 / 3.0, 4.0 / 3.0], rtol=1e-15)
 
 
+def pin_forecast_scores_closed_form():
+    """Compact Forecast Indexer: one vector per group, raw dot products, no softmax."""
+    f = np.array([1.0, 2.0, -1.0])
+    ck = np.array([[3.0, 4.0, 0.0], [-1.0, 0.5, 2.0], [0.0, 0.0, 0.0]])
+    np.testing.assert_array_equal(oracle.forecast_scores(f, ck), [11.0, -2.0, 0.0])
+
+
+def pin_forecast_scores_unit_vectors():
+    """f = e_t reads coordinate t of every compressed key."""
+    d, nc = 16, 23
+    ck = _randn((nc, d), 24).double().numpy()
+    for t in range(d):
+        f = np.zeros(d)
+        f[t] = 1.0
+        np.testing.assert_array_equal(oracle.forecast_scores(f, ck), ck[:, t])
+
+
 # ------------------------------------------------------------------------------- block reduction
 def pin_block_scores_match_max_pool():
     """With l=32, s=16, BS=64 the overlapping windows of block b are 4b-1 .. 4b+3: a max pool of
@@ -389,15 +406,60 @@ def pin_shared_index_identical_layers():
     np.testing.assert_allclose(r2["out"][0], ro, rtol=1e-12, atol=1e-13)
 
 
+def pin_forecast_decode_composes():
+    """The forecast driver selects each pair with its own Forecast vector f[b][kvh]: compress ->
+    forecast scores -> block scores -> select, then q attends the selected blocks."""
+    B, Hq, Hkv, d, T = 2, 4, 2, 16, 64 * 20
+    q, k, v = _randn((B, Hq, d), 90), _randn((B, Hkv, T, d), 91), _randn((B, Hkv, T, d), 92)
+    f = _randn((B, Hkv, d), 93)
+    qb, kb, vb, fb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v), _bf16_bits(f)
+    P = oracle.make_problem(B, Hq, Hkv, d, T, oracle.BF16, 1, 2, 3)
+    lens = [T, T - 100]
+    res = oracle.decode_forecast(P, fb, qb, kb, vb, lens)
+    G = Hq // Hkv
+    for b in range(B):
+        for kvh in range(Hkv):
+            i = b * Hkv + kvh
+            Tb = lens[b]
+            ck = oracle.compress(kb[b, kvh, :Tb].copy(), oracle.BF16)
+            S = oracle.forecast_scores(oracle.widen(fb[b, kvh], oracle.BF16), ck)
+            sb = oracle.block_scores(S, oracle.num_blocks(Tb, 64))
+            idx, _ = oracle.select(sb, 1, 2, 3)
+            assert res["idx"][i, :res["n_sel"][i]].tolist() == idx.tolist()
+            np.testing.assert_array_equal(res["block_scores"][i, :sb.size], sb)
+            qg = oracle.widen(qb[b, kvh * G:(kvh + 1) * G], oracle.BF16)
+            out, _ = oracle.attend(qg, kb[b, kvh].copy(), vb[b, kvh].copy(), oracle.BF16, Tb, idx)
+            np.testing.assert_array_equal(res["out"][i], out)
+
+
+def pin_forecast_one_head_matches_base_selector():
+    """With one query head per group, the base selector's softmax is monotone in q . K~, so a
+    Forecast vector equal to q selects the same blocks (and q attends them identically); doubling
+    f doubles every block score exactly and keeps the selection."""
+    B, Hq, Hkv, d, T = 1, 3, 3, 16, 64 * 24
+    q, k, v = _randn((B, Hq, d), 94), _randn((B, Hkv, T, d), 95), _randn((B, Hkv, T, d), 96)
+    P = oracle.make_problem(B, Hq, Hkv, d, T, oracle.F32, 1, 2, 5)
+    qn, kn, vn = q.numpy(), k.numpy(), v.numpy()
+    base = oracle.decode(P, qn, kn, vn, [T])
+    fc = oracle.decode_forecast(P, qn.reshape(B, Hkv, d), qn, kn, vn, [T])
+    assert np.array_equal(base["idx"], fc["idx"]) and np.array_equal(base["n_sel"], fc["n_sel"])
+    np.testing.assert_array_equal(base["out"], fc["out"])
+    fc2 = oracle.decode_forecast(P, (2.0 * qn).reshape(B, Hkv, d), qn, kn, vn, [T])
+    assert np.array_equal(fc2["idx"], fc["idx"])
+    np.testing.assert_array_equal(fc2["block_scores"], 2.0 * fc["block_scores"])
+
+
 ALL_PINS = [
     pin_round_bf16_matches_torch, pin_round_ties_even, pin_round_f32_matches_numpy,
     pin_compress_matches_avg_pool, pin_compress_constant_windows, pin_window_and_block_counts,
     pin_compress_cache_matches_per_pair,
     pin_scores_single_head_is_softmax, pin_scores_group_sum_of_softmaxes, pin_scores_closed_form,
+    pin_forecast_scores_closed_form, pin_forecast_scores_unit_vectors,
     pin_block_scores_match_max_pool, pin_block_scores_brute_force_overlap,
     pin_select_brute_force, pin_select_invariants, pin_select_closed_form_ties,
     pin_attend_all_blocks_is_dense, pin_attend_subset_is_gathered_dense,
     pin_attend_identical_keys_mean_of_v,
     pin_decode_full_coverage_is_dense_gqa, pin_decode_selection_composes,
     pin_shared_index_identical_layers,
+    pin_forecast_decode_composes, pin_forecast_one_head_matches_base_selector,
 ]

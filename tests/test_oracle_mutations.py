@@ -36,6 +36,11 @@ MUTANTS = {
     "lse_drops_max": ("lse[h] = m + log(z);", "lse[h] = log(z);"),
     "head_group_interleaved": ("(int64_t)kvh * G + h) * d + c", "(int64_t)h * P->num_kv_heads + kvh) * d + c"),
     "keys_values_swapped": ("bsa_oracle_attend(qg, kp, vp,", "bsa_oracle_attend(qg, vp, kp,"),
+    "forecast_drops_last_coordinate": ("for (int c = 0; c < d; ++c) dot += f[c] * ck[j * d + c];",
+                                       "for (int c = 0; c < d - 1; ++c) dot += f[c] * ck[j * d + c];"),
+    "forecast_vector_of_batch_row": ("bsa_oracle_load(f, P->dtype, (int64_t)pair * d + c)",
+                                     "bsa_oracle_load(f, P->dtype, (int64_t)b * d + c)"),
+    "forecast_scores_negated": ("        S[j] = dot;\n", "        S[j] = -dot;\n"),
 }
 
 
