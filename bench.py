@@ -184,6 +184,8 @@ class Bench:
         self.lse = [torch.zeros(B, w.num_q_heads, dtype=torch.float32, device=device)
                     for _ in range(w.layers)]
         self.seq0 = self.data["seq_lens"].clone()
+        if w.forecast and (w.layers > 1 or self.append):
+            raise ValueError("the Forecast-indexer workloads are single-layer, fixed-length")
         torch.cuda.synchronize()
 
     def q_of(self, i):
@@ -194,6 +196,15 @@ class Bench:
         bsa, d = self.bsa, self.data
         q = self.q_of(i) if q is None else q
         ev = (lambda k: events[k].record(stream)) if events is not None else (lambda k: None)
+        if self.w.forecast:
+            ev(0)
+            bsa.bsa_select_blocks_forecast(self.p, d["f"], self.ck, d["seq_lens"], self.block_idx,
+                                           self.n_sel, None, self.ws, stream=stream)
+            ev(1)
+            bsa.bsa_sparse_decode(self.p, q, d["k"][0], d["v"][0], d["seq_lens"], self.block_idx,
+                                  self.n_sel, self.out[0], self.lse[0], self.ws, stream=stream)
+            ev(2)
+            return
         if self.w.layers > 1:
             ev(0)
             bsa.bsa_select_blocks(self.p, q, self.ck, d["seq_lens"], self.block_idx, self.n_sel,
@@ -224,9 +235,16 @@ class Bench:
                               self.n_sel, self.out[0], self.lse[0], self.ws, stream=stream)
         ev(k + 2)
 
-    # one step with caller-given input and output buffers (the end-to-end pass)
+    # one step with caller-given input and output buffers (the end-to-end pass); for the
+    # Forecast-indexer workloads qs is [q, f]
     def step_io(self, qs, outs, lses, stream, k_new=None, v_new=None):
         bsa, d = self.bsa, self.data
+        if self.w.forecast:
+            bsa.bsa_select_blocks_forecast(self.p, qs[1], self.ck, d["seq_lens"], self.block_idx,
+                                           self.n_sel, None, self.ws, stream=stream)
+            bsa.bsa_sparse_decode(self.p, qs[0], d["k"][0], d["v"][0], d["seq_lens"], self.block_idx,
+                                  self.n_sel, outs[0], lses[0], self.ws, stream=stream)
+            return
         if self.w.layers > 1:
             bsa.bsa_select_blocks(self.p, qs[0], self.ck, d["seq_lens"], self.block_idx, self.n_sel,
                                   None, self.ws, stream=stream)
@@ -331,7 +349,13 @@ def cpu_oracle_sample(w, data, seconds: float):
                             oracle.F32 if w.dtype == "f32" else oracle.BF16, w.n_init, w.n_local,
                             w.top_k, w.cmp_kernel, w.cmp_stride, w.block_size)
 
+    f_arr = (oracle.raw(torch.stack([data["f"][b, h:h + 1] for b, h in pairs]))[0]
+             if w.forecast else None)
+
     def one():
+        if w.forecast:
+            oracle.decode_forecast(P, f_arr, *arrays[0], lens)
+            return
         r = oracle.decode(P, *arrays[0], lens)
         for L in range(1, w.layers):
             oracle.attend_pairs(P, *arrays[L], lens, r["idx"], r["n_sel"])
@@ -445,8 +469,9 @@ def run_bsa(args, w, world, rank, local):
     import torch as _t
     L_ = w.layers
     NBUF = 2
-    def step_q(i):  # the query of every layer for timed step i
-        return [bench.q_of(W + i if bench.append else 0)] + [bench.data["q"][l] for l in range(1, L_)]
+    def step_q(i):  # the query of every layer for timed step i (then the Forecast vectors)
+        return ([bench.q_of(W + i if bench.append else 0)] + [bench.data["q"][l] for l in range(1, L_)]
+                + ([bench.data["f"]] if w.forecast else []))
     q_host = [[t.cpu().pin_memory() for t in step_q(i)] for i in range(K)]
     q_dev = [[_t.empty_like(t) for t in step_q(0)] for _ in range(NBUF)]
     out_dev = [[_t.empty_like(bench.out[l]) for l in range(L_)] for _ in range(NBUF)]
@@ -480,7 +505,7 @@ def run_bsa(args, w, world, rank, local):
         with _t.cuda.stream(h2d_stream):
             if i >= NBUF:
                 h2d_stream.wait_event(ev_step[j])  # the step that last read buffer j is done
-            for l in range(L_):
+            for l in range(len(q_host[i])):
                 q_dev[j][l].copy_(q_host[i][l], non_blocking=True)
             if bench.append:
                 kn_dev[j].copy_(kn_host[i], non_blocking=True)
@@ -517,7 +542,7 @@ def run_bsa(args, w, world, rank, local):
     # ---- roofline of the dominant kernel
     peak, peak_kind = load_peaks()
     q_bytes = w.batch * w.num_q_heads * w.head_dim * w.elem_bytes
-    kbytes = {"select": ab["ck"] + q_bytes,          # compressed keys of the scored layer + q
+    kbytes = {"select": ab["ck"] + (ab["f"] if w.forecast else q_bytes),  # compressed keys + q (or f)
               "decode": ab["kv"] + ab["qo"],         # selected K/V rows + q + out, every layer
               "append": ab["append"]}
     # the selection phase is two launches (scoring, then selection); the others are one each, so
@@ -547,13 +572,15 @@ def run_bsa(args, w, world, rank, local):
         "scaling": "weak",
         "vs_baseline": None,
         "dtype": w.dtype,
-        "data": "synthetic (seeded N(0,1) q/K/V with planted needle blocks)",
+        "data": "synthetic (seeded N(0,1) q/K/V with planted needle blocks)"
+                + ("; Forecast vectors = each GQA group's mean query" if w.forecast else ""),
         "config": {
             "workload": w.name, "batch": w.batch, "seq_len": w.seq_len, "q_heads": w.num_q_heads,
             "kv_heads": w.num_kv_heads, "head_dim": w.head_dim, "n_init": w.n_init,
             "n_local": w.n_local, "top_k": w.top_k, "block_size": w.block_size,
             "cmp_kernel": w.cmp_kernel, "cmp_stride": w.cmp_stride, "layers": w.layers,
-            "append": bool(bench.append), "parallelism": f"replicas x{world} (batch-sharded)",
+            "append": bool(bench.append), "forecast_indexer": bool(w.forecast),
+            "parallelism": f"replicas x{world} (batch-sharded)",
             "l2": ("L2 flushed (256 MB write) between timed steps" if flush else
                    f"inputs larger than L2: {per_step_bytes / 1e6:.0f} MB read per step vs 126 MB L2"),
             "cuda_graph": graph is not None,

@@ -73,6 +73,7 @@ _SIGS = {
     "bsa_compress_keys": (_S, [_PP, _P, _P, _P, _P]),
     "bsa_compress_append": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "bsa_select_blocks": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "bsa_select_blocks_forecast": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "bsa_sparse_decode": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "bsa_sparse_decode_layers": (_S, [_PP, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_size_t, _P]),
@@ -231,6 +232,21 @@ def bsa_select_blocks(p: Params, q, ck, seq_lens, block_idx, n_sel, block_scores
         _ptr(block_scores, "block_scores", torch.float32, n["scores"], optional=True),
         _ptr(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
         "bsa_select_blocks")
+
+
+def bsa_select_blocks_forecast(p: Params, f, ck, seq_lens, block_idx, n_sel, block_scores, ws,
+                               stream=None):
+    """Selection from one Forecast vector per (batch, kv head), f [B][Hkv][d]."""
+    import torch
+    n, e = _shapes(p), _elem(p)
+    _check(lib().bsa_select_blocks_forecast(
+        ctypes.byref(p), _ptr(f, "f", e, n["pairs"] * p.head_dim), _ptr(ck, "ck", e, n["ck"]),
+        _ptr(seq_lens, "seq_lens", torch.int32, p.batch),
+        _ptr(block_idx, "block_idx", torch.int32, n["idx"]),
+        _ptr(n_sel, "n_sel", torch.int32, n["pairs"]),
+        _ptr(block_scores, "block_scores", torch.float32, n["scores"], optional=True),
+        _ptr(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
+        "bsa_select_blocks_forecast")
 
 
 def bsa_sparse_decode(p: Params, q, k_cache, v_cache, seq_lens, block_idx, n_sel, out, lse, ws,

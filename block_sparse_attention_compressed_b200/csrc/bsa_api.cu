@@ -423,6 +423,38 @@ bsa_status_t bsa_select_blocks(const bsa_params_t* params, const void* q, const 
     return do_select(P, q, ck, seq_lens, block_idx, n_sel, block_scores, ws, stream);
 }
 
+bsa_status_t bsa_select_blocks_forecast(const bsa_params_t* params, const void* f, const void* ck,
+                                        const int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                                        float* block_scores, void* ws, size_t ws_bytes,
+                                        cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if (!ok16(f) || !ok4(seq_lens) || !ok4(block_idx) || !ok4(n_sel)) return BSA_ERR_INVALID_ARG;
+    if (P.nc_cap > 0 && !ok16(ck)) return BSA_ERR_INVALID_ARG;
+    if (block_scores && !ok4(block_scores)) return BSA_ERR_INVALID_ARG;
+    if ((st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
+    // one scoring head per group: the plan of a problem with Hq = Hkv, whose workspace is a prefix
+    // of this one's (same counters, smaller score and partial arrays)
+    bsa_params_t pf = *params;
+    pf.num_q_heads = pf.num_kv_heads;
+    Plan F;
+    if ((st = make_plan(&pf, &F)) != BSA_OK) return st;
+    if (F.ws_bytes > P.ws_bytes || F.off_logits != P.off_logits) return BSA_ERR_UNSUPPORTED;
+    ScoreArgs sa = score_args(F, f, ck, seq_lens, ws);
+    sa.raw = 1;
+    sa.score_log2 = 1.f;  // the raw dot products
+    static thread_local CUtensorMap ck_map;
+    static thread_local MapKey ck_key;
+    if (F.dtype == BSA_BF16 && F.nc_cap > 0 &&
+        !encode_kv_map_cached(&ck_map, &ck_key, ck, (uint64_t)F.pairs * F.nc_cap, F.D, 64))
+        return BSA_ERR_CUDA;
+    if (launch_score(F, sa, &ck_map, stream) != cudaSuccess) return BSA_ERR_CUDA;
+    SelectArgs la = select_args(F, seq_lens, block_idx, n_sel, block_scores, ws);
+    la.raw = 1;
+    return from_cuda(launch_select(F, la, stream));
+}
+
 bsa_status_t bsa_sparse_decode_layers(const bsa_params_t* params, int32_t num_layers,
                                       const void* const* q, const void* const* k_caches,
                                       const void* const* v_caches, const int32_t* seq_lens,

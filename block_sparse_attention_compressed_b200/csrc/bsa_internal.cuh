@@ -79,6 +79,7 @@ struct ScoreArgs {
     int B, Hq, Hkv, G, Gp, l, s;
     int64_t T_cap, nc_cap, lg_stride, nchunk, total_chunks, nstat;
     float score_log2;
+    int raw;  // Forecast indexer: store the raw scores x (no exp2, no statistics)
 };
 
 struct SelectArgs {
@@ -95,6 +96,7 @@ struct SelectArgs {
     int64_t T_cap, nc_cap, nb_cap, lg_stride, nstat, key_words;
     int parts, part_windows;
     int ring;  // one-part kernel: logits stages in flight
+    int raw;   // Forecast indexer: the stored scores are the window scores (weight 1, no statistics)
 };
 
 // TMA descriptors of the K and V caches of every layer (bf16 path): 2-D views

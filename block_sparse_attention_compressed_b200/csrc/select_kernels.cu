@@ -220,6 +220,27 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 2)
             }
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);  // the data is in registers: refill the slot
+            if (a.raw) {
+                // Forecast indexer: the raw scores are the window scores
+                float* lgr = a.logits + (size_t)md.pair * a.lg_stride * a.Gp;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int lra = 16 * r + g, lrb = lra + 8;
+                    if (lra < md.nrows) {
+                        const int64_t ra = md.row0 + lra;
+                        if (h1) *reinterpret_cast<float2*>(lgr + ra * a.Gp + 2 * tq) =
+                            make_float2(c[r][0] * a.score_log2, c[r][1] * a.score_log2);
+                        else if (h0) lgr[ra * a.Gp + 2 * tq] = c[r][0] * a.score_log2;
+                    }
+                    if (lrb < md.nrows) {
+                        const int64_t rb = md.row0 + lrb;
+                        if (h1) *reinterpret_cast<float2*>(lgr + rb * a.Gp + 2 * tq) =
+                            make_float2(c[r][2] * a.score_log2, c[r][3] * a.score_log2);
+                        else if (h0) lgr[rb * a.Gp + 2 * tq] = c[r][2] * a.score_log2;
+                    }
+                }
+                continue;
+            }
             // the chunk's maximum per head first, then e = exp2(x - max) is stored and summed: the
             // selection only rescales each chunk's e by one weight per head
             float x[4][4];
@@ -362,11 +383,12 @@ __global__ void __launch_bounds__(kScoreThreads, 2) score_f32_kernel(ScoreArgs a
                 sm[h] = m[h];
             }
         __syncwarp();
-        // the chunk's rows, coalesced: e = exp2(x - max) (0 in the padding heads)
+        // the chunk's rows, coalesced: e = exp2(x - max) (0 in the padding heads), or the raw
+        // scores x for the Forecast indexer
         const int nvals = (int)(r1 - r0) * a.Gp;
         for (int e = lane; e < nvals; e += 32) {
             const int h = e % a.Gp;
-            lg[r0 * a.Gp + e] = h < a.G ? exp2f(sx[e] - sm[h]) : 0.f;
+            lg[r0 * a.Gp + e] = h < a.G ? (a.raw ? sx[e] : exp2f(sx[e] - sm[h])) : 0.f;
         }
         __syncwarp();
     }
@@ -797,7 +819,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
             __syncthreads();
             for (int64_t e = tid; e < nch * a.Gp; e += kSelectThreads) {
                 const int h = (int)(e % a.Gp);
-                s_st[e].x = h < a.G ? exp2f(s_st[e].x - sM[h]) * sInvZ[h] : 0.f;
+                s_st[e].x = h < a.G ? (a.raw ? 1.f : exp2f(s_st[e].x - sM[h]) * sInvZ[h]) : 0.f;
             }
             __syncthreads();
         }
@@ -917,19 +939,24 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     // warp h merges head h's chunk statistics into its normaliser (M_h, Z_h), which every lane
     // then holds, and weighs the head's chunks: w[c][h] = exp2(m_c - M_h) / Z_h
     if (warp < a.G) {
-        float m = -INFINITY, sum = 0.f;
-        for (int c = lane; c < nch; c += 32) {
-            const float2 v = s_st[c * GP + warp];
-            online_merge(m, sum, v.x, v.y);
-        }
+        if (a.raw) {
+            // Forecast indexer: the stored raw scores are the window scores
+            for (int c = lane; c < nch; c += 32) wt[c * GP + warp] = 1.f;
+        } else {
+            float m = -INFINITY, sum = 0.f;
+            for (int c = lane; c < nch; c += 32) {
+                const float2 v = s_st[c * GP + warp];
+                online_merge(m, sum, v.x, v.y);
+            }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-            const float mo = __shfl_xor_sync(0xffffffffu, m, off);
-            const float so = __shfl_xor_sync(0xffffffffu, sum, off);
-            online_merge(m, sum, mo, so);
+            for (int off = 16; off > 0; off >>= 1) {
+                const float mo = __shfl_xor_sync(0xffffffffu, m, off);
+                const float so = __shfl_xor_sync(0xffffffffu, sum, off);
+                online_merge(m, sum, mo, so);
+            }
+            const float iz = sum > 0.f ? 1.f / sum : 0.f;
+            for (int c = lane; c < nch; c += 32) wt[c * GP + warp] = exp2f(s_st[c * GP + warp].x - m) * iz;
         }
-        const float iz = sum > 0.f ? 1.f / sum : 0.f;
-        for (int c = lane; c < nch; c += 32) wt[c * GP + warp] = exp2f(s_st[c * GP + warp].x - m) * iz;
     }
     __syncthreads();
     // S[j] = sum_h e[j][h] * w[j / 64][h], for window j at index i of the stage in slot `slot`

@@ -46,6 +46,7 @@ class Workload:
     cmp_stride: int = 16
     block_size: int = 64
     needle_shift: float = 2.0
+    forecast: bool = False  # select with one Forecast vector per GQA group (f = the group's mean q)
 
     @property
     def group(self) -> int:
@@ -63,7 +64,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The five decode workloads: one small parity case and four throughput cases.
+# The decode workloads: one small parity case and five throughput cases.
 WORKLOADS: dict[str, Workload] = {
     w.name: w
     for w in [
@@ -80,6 +81,9 @@ WORKLOADS: dict[str, Workload] = {
         Workload("append-bf16-16k-b128", batch=128, num_q_heads=32, num_kv_heads=8, head_dim=128,
                  seq_len=16384, dtype="bf16", n_init=1, n_local=2, top_k=16, needles=4, seed=1005,
                  append_steps=64),
+        Workload("forecast-bf16-128k-b16", batch=16, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                 seq_len=131072, dtype="bf16", n_init=1, n_local=4, top_k=64, needles=16,
+                 seed=1006, forecast=True),
     ]
 }
 DEFAULT_WORKLOAD = "gqa4-bf16-128k-b16"
@@ -122,6 +126,8 @@ def generate(w: Workload, device="cpu", seq_cap: int | None = None, steps: int |
       k, v     [L][B][Hkv][T_cap][d]  caches, zero at rows >= seq_len
       seq_lens [B] int32              (on ``device``)
       needles  [B][Hkv][n] numpy      needle block positions
+      f        [B][Hkv][d]            Forecast vectors (forecast workloads): the mean of each
+                                      group's query vectors of the first layer, in the cache type
     and, when ``steps`` > 0 (growing-cache workload):
       q_steps  [steps][B][Hq][d], k_new / v_new [steps][B][Hkv][d]
     ``seq_cap`` is the cache capacity T_cap (default: seq_len + steps).
@@ -166,6 +172,9 @@ def generate(w: Workload, device="cpu", seq_cap: int | None = None, steps: int |
         seq_lens=torch.full((w.batch,), T, dtype=torch.int32, device=device),
         needles=blocks, seq_cap=T_cap,
     )
+    if w.forecast:
+        q0 = res["q"][0].float().view(w.batch, w.num_kv_heads, w.group, w.head_dim)
+        res["f"] = q0.mean(dim=2).to(dt).contiguous()
     res.update(extra)
     return res
 
@@ -190,4 +199,5 @@ def algorithmic_bytes(w: Workload, T: int | None = None) -> dict:
     app = 0
     if w.append_steps:
         app = pairs * d * e * 4 + pairs * (w.cmp_kernel + 1) * d * e / w.cmp_stride
-    return dict(ck=ck, kv=kv, qo=qo, append=app, total=ck + kv + qo + app)
+    fv = pairs * d * e if w.forecast else 0   # the Forecast vectors read by the scoring
+    return dict(ck=ck, kv=kv, qo=qo, append=app, f=fv, total=ck + kv + qo + app + fv)

@@ -162,6 +162,20 @@ bsa_status_t bsa_select_blocks(const bsa_params_t* params, const void* q, const 
                                float* block_scores, void* workspace, size_t workspace_bytes,
                                cudaStream_t stream);
 
+/* SparDA Architecture, Eq. (4), with the "Compact Forecast Indexer": the same selection as
+ * bsa_select_blocks, but each (batch, kv head) pair is scored by ONE Forecast vector
+ * f[b][kvh] (params->head_dim elements of params->dtype, [batch][num_kv_heads][head_dim],
+ * 16-byte aligned, caller-owned) instead of its group's query heads, with no softmax: the window
+ * score is the raw dot product f . ck_j (fp32 accumulation of exact products), the block score
+ * its maximum over the block's complete windows (-inf when there is none; written to
+ * block_scores when that is not NULL). top_k, init and local blocks, tie rule, outputs and
+ * workspace (bsa_workspace_size(params)) are those of bsa_select_blocks; q then attends the
+ * blocks through bsa_sparse_decode. Errors as bsa_select_blocks. */
+bsa_status_t bsa_select_blocks_forecast(const bsa_params_t* params, const void* f, const void* ck,
+                                        const int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                                        float* block_scores, void* workspace,
+                                        size_t workspace_bytes, cudaStream_t stream);
+
 /* Step 5 (Eq. 5): for every query head, softmax attention (scale params->scale) over the tokens
  * t < seq_lens[b] of the first n_sel[b][kvh] blocks listed in block_idx[b][kvh] (any order; -1
  * entries are skipped). Writes out and, if not NULL, lse. A pair with no attended token gets a

@@ -10,8 +10,8 @@ import torch
 import block_sparse_attention_compressed_b200 as bsa
 import oracle
 from block_sparse_attention_compressed_b200.workloads import WORKLOADS, Workload
-from gpu_helpers import (GpuRun, check_output, check_selection, full_check, oracle_on_pairs,
-                         sample_pairs)
+from gpu_helpers import (GpuRun, check_output, check_selection, forecast_check, full_check,
+                         oracle_on_pairs, sample_pairs)
 
 pytestmark = pytest.mark.gpu
 
@@ -379,3 +379,69 @@ def test_full_append_workload(cuda_device):
     check_output(run, pairs, orc, skip=set(ties))
     del run
     torch.cuda.empty_cache()
+
+
+# ------------------------------------------------------------------ Forecast indexer (SparDA Eq. 4)
+FORECAST = {
+    # few pairs: the selection splits each pair's windows over several CTAs
+    "bf16-g4-d128-ragged": BASE.replace(name="x", batch=2, seq_len=4096 + 37, top_k=8, needles=4,
+                                        forecast=True),
+    "bf16-g8-d64": BASE.replace(name="x", batch=2, num_q_heads=16, num_kv_heads=2, head_dim=64,
+                                seq_len=3000, top_k=6, needles=3, forecast=True),
+    "f32-g4-d128": BASE.replace(name="x", dtype="f32", batch=1, seq_len=2500, top_k=6, needles=2,
+                                forecast=True),
+    "bf16-bs32-l16s8": BASE.replace(name="x", batch=1, num_q_heads=4, num_kv_heads=2, head_dim=64,
+                                    seq_len=2000, block_size=32, cmp_kernel=16, cmp_stride=8,
+                                    top_k=10, needles=3, forecast=True),
+    # enough pairs for one CTA per pair (the shared-memory ring and shuffle block maxima)
+    "bf16-256-pairs": BASE.replace(name="x", batch=32, seq_len=6000, top_k=12, needles=3,
+                                   forecast=True),
+}
+
+
+@pytest.mark.parametrize("case", sorted(FORECAST))
+def test_forecast_select_and_decode(case, cuda_device):
+    """Blocks chosen by one Forecast vector per group (raw scores f . K~, no softmax), attended by
+    the group's queries."""
+    w = FORECAST[case]
+    run = GpuRun(w)
+    run.compress()
+    f = run.data["f"]
+    bsa.bsa_select_blocks_forecast(run.p, f, run.ck[0], run.data["seq_lens"], run.block_idx,
+                                   run.n_sel, run.block_scores, run.ws)
+    run.decode()
+    assert run.device_errors() == 0
+    forecast_check(run, sample_pairs(w, 48), f)
+
+
+def test_forecast_ragged_lengths(cuda_device):
+    """Different lengths in one batch, down to no window and an empty sequence."""
+    w = BASE.replace(name="x", batch=5, seq_len=5000, top_k=9, needles=3, forecast=True)
+    run = GpuRun(w, seq_lens=[5000, 64, 31, 0, 4097])
+    run.compress()
+    bsa.bsa_select_blocks_forecast(run.p, run.data["f"], run.ck[0], run.data["seq_lens"],
+                                   run.block_idx, run.n_sel, run.block_scores, run.ws)
+    run.decode()
+    assert run.device_errors() == 0
+    forecast_check(run, list(range(w.batch * w.num_kv_heads)), run.data["f"])
+
+
+@pytest.mark.slow
+def test_forecast_full_workload(cuda_device):
+    w = WORKLOADS["forecast-bf16-128k-b16"]
+    run = GpuRun(w)
+    run.compress()
+    bsa.bsa_select_blocks_forecast(run.p, run.data["f"], run.ck[0], run.data["seq_lens"],
+                                   run.block_idx, run.n_sel, run.block_scores, run.ws)
+    run.decode()
+    assert run.device_errors() == 0
+    forecast_check(run, sample_pairs(w, 12, seed=2), run.data["f"])
+    # the needles lie along each group's mean query, which is the Forecast vector here
+    nd = run.data["needles"]
+    idx = run.block_idx.cpu().numpy()
+    hit = np.mean([np.isin(nd[b, h], idx[b, h]).mean() for b in range(w.batch)
+                   for h in range(w.num_kv_heads)])
+    assert hit > 0.9, hit
+    del run
+    torch.cuda.empty_cache()
+
