@@ -175,10 +175,18 @@ class Bench:
         B, Hkv, d = w.batch, w.num_kv_heads, w.head_dim
         self.ck = torch.zeros(B, Hkv, s.nc_cap, d, dtype=dt, device=device)
         bsa.bsa_compress_keys(self.p, self.data["k"][0], self.data["seq_lens"], self.ck)
+        # anchored index reuse: compressed keys of every anchor layer, one selection per anchor
+        self.anchored = len(w.anchors) > 1
+        self.cks = [self.ck if L == 0 else None for L in range(w.layers)]
+        for L in w.anchors[1:]:
+            self.cks[L] = torch.zeros_like(self.ck)
+            bsa.bsa_compress_keys(self.p, self.data["k"][L], self.data["seq_lens"], self.cks[L])
         self.ws = bsa.alloc_workspace(self.p, device)
         bsa.bsa_workspace_init(self.p, self.ws)
-        self.block_idx = torch.zeros(B, Hkv, s.sel_cap, dtype=torch.int32, device=device)
-        self.n_sel = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
+        A = len(w.anchors)
+        self.block_idx_all = torch.zeros(A, B, Hkv, s.sel_cap, dtype=torch.int32, device=device)
+        self.n_sel_all = torch.zeros(A, B, Hkv, dtype=torch.int32, device=device)
+        self.block_idx, self.n_sel = self.block_idx_all[0], self.n_sel_all[0]
         self.out = [torch.zeros(B, w.num_q_heads, d, dtype=dt, device=device)
                     for _ in range(w.layers)]
         self.lse = [torch.zeros(B, w.num_q_heads, dtype=torch.float32, device=device)
@@ -206,14 +214,27 @@ class Bench:
             ev(2)
             return
         if self.w.layers > 1:
-            ev(0)
-            bsa.bsa_select_blocks(self.p, q, self.ck, d["seq_lens"], self.block_idx, self.n_sel,
-                                  None, self.ws, stream=stream)
-            ev(1)
-            bsa.bsa_sparse_decode_layers(self.p, [q] + [d["q"][L] for L in range(1, self.w.layers)],
-                                         d["k"], d["v"], d["seq_lens"], self.block_idx, self.n_sel,
-                                         self.out, self.lse, self.ws, stream=stream)
-            ev(2)
+            qs = [q] + [d["q"][L] for L in range(1, self.w.layers)]
+            if self.anchored and events is None:
+                bsa.bsa_decode_step_anchored(self.p, self.w.anchors, qs, d["k"], d["v"], self.cks,
+                                             d["seq_lens"], self.block_idx_all, self.n_sel_all,
+                                             self.out, self.lse, self.ws, stream=stream)
+                return
+            # one selection per anchor (the calls bsa_decode_step_anchored chains), each reused
+            # by the layers up to the next anchor
+            anchors = list(self.w.anchors) + [self.w.layers]
+            for i in range(len(anchors) - 1):
+                a0, a1 = anchors[i], anchors[i + 1]
+                ev(2 * i)
+                bsa.bsa_select_blocks(self.p, qs[a0], self.cks[a0], d["seq_lens"],
+                                      self.block_idx_all[i], self.n_sel_all[i], None, self.ws,
+                                      stream=stream)
+                ev(2 * i + 1)
+                bsa.bsa_sparse_decode_layers(self.p, qs[a0:a1], d["k"][a0:a1], d["v"][a0:a1],
+                                             d["seq_lens"], self.block_idx_all[i],
+                                             self.n_sel_all[i], self.out[a0:a1], self.lse[a0:a1],
+                                             self.ws, stream=stream)
+            ev(2 * (len(anchors) - 1))
             return
         if events is None:
             bsa.bsa_decode_step(self.p, q, d["k"][0], d["v"][0], self.ck,
@@ -246,6 +267,11 @@ class Bench:
                                   self.n_sel, outs[0], lses[0], self.ws, stream=stream)
             return
         if self.w.layers > 1:
+            if self.anchored:
+                bsa.bsa_decode_step_anchored(self.p, self.w.anchors, qs, d["k"], d["v"], self.cks,
+                                             d["seq_lens"], self.block_idx_all, self.n_sel_all,
+                                             outs, lses, self.ws, stream=stream)
+                return
             bsa.bsa_select_blocks(self.p, qs[0], self.ck, d["seq_lens"], self.block_idx, self.n_sel,
                                   None, self.ws, stream=stream)
             bsa.bsa_sparse_decode_layers(self.p, qs, d["k"], d["v"], d["seq_lens"], self.block_idx,
@@ -256,13 +282,14 @@ class Bench:
                             stream=stream)
 
     def kernel_names(self):
-        names = ["select", "decode"]
+        names = ["select", "decode"] * (len(self.w.anchors) if self.w.layers > 1 else 1)
         return (["append"] + names) if (self.append and self.w.layers == 1) else names
 
     def launches_per_step(self):
         # bsa_select_blocks launches two kernels (scoring, selection), the bf16 sparse attention two
         # (attention, combine), the fp32 one one, the append one
-        return len(self.kernel_names()) + 1 + (1 if self.w.dtype == "bf16" else 0)
+        n = self.kernel_names()
+        return len(n) + n.count("select") + (n.count("decode") if self.w.dtype == "bf16" else 0)
 
     def reset_lengths(self):
         self.data["seq_lens"].copy_(self.seq0)
@@ -356,9 +383,12 @@ def cpu_oracle_sample(w, data, seconds: float):
         if w.forecast:
             oracle.decode_forecast(P, f_arr, *arrays[0], lens)
             return
-        r = oracle.decode(P, *arrays[0], lens)
-        for L in range(1, w.layers):
-            oracle.attend_pairs(P, *arrays[L], lens, r["idx"], r["n_sel"])
+        r = None
+        for L in range(w.layers):
+            if L in w.anchors:
+                r = oracle.decode(P, *arrays[L], lens)   # select + attend on an anchor layer
+            else:
+                oracle.attend_pairs(P, *arrays[L], lens, r["idx"], r["n_sel"])
 
     t0 = time.perf_counter()
     one()
@@ -460,8 +490,9 @@ def run_bsa(args, w, world, rank, local):
                 flush_buf.fill_(i & 0xff)
             bench.step(W + i if bench.append else 0, stream, events=evs[i])
     stream.synchronize()
-    kern_ms = {n: sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
-               for j, n in enumerate(names)}
+    kern_ms = {}  # per phase, summed over the phase's calls in a step (one per anchor)
+    for j, n in enumerate(names):
+        kern_ms[n] = kern_ms.get(n, 0.0) + sum(evs[i][j].elapsed_time(evs[i][j + 1]) for i in range(K)) / K
 
     # ---- e2e: through the binding, every step's inputs copied in from pinned host memory and its
     # outputs (every layer) copied back, double-buffered: step i+1's inputs land and step i's
@@ -550,13 +581,14 @@ def run_bsa(args, w, world, rank, local):
     single = {n: t for n, t in kern_ms.items() if n != "select"} or kern_ms
     dom = max(single, key=single.get)
     kname = KERNEL_OF_PHASE[dom][w.dtype]
+    n_calls = names.count(dom)  # launches of that kernel per step (one per anchor)
     achieved = kbytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
     traffic = profile_traffic(kname, w.name)
     roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
                 "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                 "peak_kind": peak_kind + " copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                "traffic": traffic, "algorithmic_bytes_per_launch": kbytes[dom],
-                "kernel_ms": round(kern_ms[dom], 5)}
+                "traffic": traffic, "algorithmic_bytes_per_launch": kbytes[dom] / n_calls,
+                "kernel_ms": round(kern_ms[dom] / n_calls, 5)}
 
     steps_per_s = world * K / (total_ms * 1e-3)
     gbs = per_step_bytes * world * K / (total_ms * 1e-3) / 1e9
@@ -580,6 +612,7 @@ def run_bsa(args, w, world, rank, local):
             "n_local": w.n_local, "top_k": w.top_k, "block_size": w.block_size,
             "cmp_kernel": w.cmp_kernel, "cmp_stride": w.cmp_stride, "layers": w.layers,
             "append": bool(bench.append), "forecast_indexer": bool(w.forecast),
+            "anchors": list(w.anchors),
             "parallelism": f"replicas x{world} (batch-sharded)",
             "l2": ("L2 flushed (256 MB write) between timed steps" if flush else
                    f"inputs larger than L2: {per_step_bytes / 1e6:.0f} MB read per step vs 126 MB L2"),

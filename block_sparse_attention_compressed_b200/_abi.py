@@ -79,6 +79,8 @@ _SIGS = {
                                       ctypes.c_size_t, _P]),
     "bsa_decode_step": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                              ctypes.c_size_t, _P]),
+    "bsa_decode_step_anchored": (_S, [_PP, ctypes.c_int32, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
+                                      _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "bsa_read_device_error": (_S, [_P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32), _P]),
     "bsa_sparse_decode_noalloc": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
@@ -300,6 +302,36 @@ def bsa_sparse_decode_layers(p: Params, qs, k_caches, v_caches, seq_lens, block_
         _ptr(n_sel, "n_sel", torch.int32, n["pairs"]), o_a, l_a, _ptr(ws, "workspace"),
         ws.numel() * ws.element_size(), _stream(stream)),
         "bsa_sparse_decode_layers")
+
+
+def bsa_decode_step_anchored(p: Params, anchors, qs, k_caches, v_caches, cks, seq_lens, block_idx,
+                             n_sel, outs, lses, ws, stream=None):
+    """Anchored index reuse: one selection per anchor layer, reused by the layers up to the next
+    anchor. block_idx is [num_anchors][B][Hkv][SEL_cap], n_sel [num_anchors][B][Hkv]; cks lists one
+    compressed-key tensor per layer (None where the layer is not an anchor)."""
+    import torch
+    n, e = _shapes(p), _elem(p)
+    L, A = len(qs), len(anchors)
+    if not (len(k_caches) == len(v_caches) == len(outs) == len(cks) == L) or \
+            (lses is not None and len(lses) != L):
+        raise ValueError("per-layer lists must have the same length")
+    arr = ctypes.c_void_p * L
+    anc = set(int(a) for a in anchors)
+    q_a = arr(*[_ptr(t, "q", e, n["q"]) for t in qs])
+    k_a = arr(*[_ptr(t, "k_cache", e, n["cache"]) for t in k_caches])
+    v_a = arr(*[_ptr(t, "v_cache", e, n["cache"]) for t in v_caches])
+    c_a = arr(*[_ptr(t, "ck", e, n["ck"]) if i in anc else None for i, t in enumerate(cks)])
+    o_a = arr(*[_ptr(t, "out", e, n["q"]) for t in outs])
+    l_a = None if lses is None else arr(*[_ptr(t, "lse", torch.float32, n["lse"], optional=True)
+                                          for t in lses])
+    a_a = (ctypes.c_int32 * A)(*[int(a) for a in anchors])
+    _check(lib().bsa_decode_step_anchored(
+        ctypes.byref(p), L, a_a, A, q_a, k_a, v_a, c_a,
+        _ptr(seq_lens, "seq_lens", torch.int32, p.batch),
+        _ptr(block_idx, "block_idx", torch.int32, n["idx"] * A),
+        _ptr(n_sel, "n_sel", torch.int32, n["pairs"] * A), o_a, l_a, _ptr(ws, "workspace"),
+        ws.numel() * ws.element_size(), _stream(stream)),
+        "bsa_decode_step_anchored")
 
 
 def bsa_decode_step(p: Params, q, k_cache, v_cache, ck, k_new, v_new, seq_lens, block_idx, n_sel,

@@ -238,16 +238,22 @@ SelectArgs select_args(const Plan& P, const int32_t* seq_lens, int32_t* block_id
 }
 
 // Scoring then selection, chained on the stream.
+// The TMA descriptor of a compressed-key array, re-encoded only when the array changes.
+struct CkMapCache {
+    CUtensorMap map;
+    MapKey key;
+};
+
 bsa_status_t do_select(const Plan& P, const void* q, const void* ck, const int32_t* seq_lens,
                        int32_t* block_idx, int32_t* n_sel, float* block_scores, void* ws,
-                       cudaStream_t st) {
+                       cudaStream_t st, CkMapCache* cache = nullptr) {
     ScoreArgs sa = score_args(P, q, ck, seq_lens, ws);
-    static thread_local CUtensorMap ck_map;
-    static thread_local MapKey ck_key;
+    static thread_local CkMapCache own;
+    CkMapCache& c = cache ? *cache : own;
     if (P.dtype == BSA_BF16 && P.nc_cap > 0 &&
-        !encode_kv_map_cached(&ck_map, &ck_key, ck, (uint64_t)P.pairs * P.nc_cap, P.D, 64))
+        !encode_kv_map_cached(&c.map, &c.key, ck, (uint64_t)P.pairs * P.nc_cap, P.D, 64))
         return BSA_ERR_CUDA;
-    cudaError_t e = launch_score(P, sa, &ck_map, st);
+    cudaError_t e = launch_score(P, sa, &c.map, st);
     if (e != cudaSuccess) return BSA_ERR_CUDA;
     SelectArgs la = select_args(P, seq_lens, block_idx, n_sel, block_scores, ws);
     return from_cuda(launch_select(P, la, st));
@@ -483,6 +489,57 @@ bsa_status_t bsa_sparse_decode_layers(const bsa_params_t* params, int32_t num_la
     static thread_local KVMapCache maps;
     if ((st = make_maps(P, a, num_layers, &maps)) != BSA_OK) return st;
     return from_cuda(launch_decode(P, a, &maps.maps, num_layers, stream));
+}
+
+bsa_status_t bsa_decode_step_anchored(const bsa_params_t* params, int32_t num_layers,
+                                      const int32_t* anchors, int32_t num_anchors,
+                                      const void* const* q, const void* const* k_caches,
+                                      const void* const* v_caches, const void* const* cks,
+                                      const int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                                      void* const* outs, float* const* lses, void* ws,
+                                      size_t ws_bytes, cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if (num_layers < 1 || num_layers > P.layers) return BSA_ERR_INVALID_ARG;
+    if (!anchors || num_anchors < 1 || num_anchors > num_layers || anchors[0] != 0)
+        return BSA_ERR_INVALID_ARG;
+    for (int i = 1; i < num_anchors; ++i)
+        if (anchors[i] <= anchors[i - 1] || anchors[i] >= num_layers) return BSA_ERR_INVALID_ARG;
+    if (!q || !k_caches || !v_caches || !cks || !outs) return BSA_ERR_INVALID_ARG;
+    if (!ok4(seq_lens) || !ok4(block_idx) || !ok4(n_sel)) return BSA_ERR_INVALID_ARG;
+    for (int l = 0; l < num_layers; ++l) {
+        if (!ok16(q[l]) || !ok16(k_caches[l]) || !ok16(v_caches[l]) || !ok16(outs[l]))
+            return BSA_ERR_INVALID_ARG;
+        if (lses && lses[l] && !ok4(lses[l])) return BSA_ERR_INVALID_ARG;
+    }
+    for (int i = 0; i < num_anchors; ++i)
+        if (P.nc_cap > 0 && !ok16(cks[anchors[i]])) return BSA_ERR_INVALID_ARG;
+    if ((st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
+    // one descriptor cache per anchor position, so a steady schedule never re-encodes
+    static thread_local CkMapCache ck_cache[BSA_MAX_LAYERS];
+    static thread_local KVMapCache kv_cache[BSA_MAX_LAYERS];
+    const size_t idx_stride = (size_t)P.pairs * P.sel_cap;
+    for (int i = 0; i < num_anchors; ++i) {
+        const int a0 = anchors[i], a1 = i + 1 < num_anchors ? anchors[i + 1] : num_layers;
+        int32_t* bi = block_idx + (size_t)i * idx_stride;
+        int32_t* ns = n_sel + (size_t)i * P.pairs;
+        if ((st = do_select(P, q[a0], cks[a0], seq_lens, bi, ns, nullptr, ws, stream, &ck_cache[i])) !=
+            BSA_OK)
+            return st;
+        DecodeArgs da = decode_args(P, seq_lens, bi, ns, ws);
+        for (int l = a0; l < a1; ++l) {
+            da.q[l - a0] = q[l];
+            da.k[l - a0] = k_caches[l];
+            da.v[l - a0] = v_caches[l];
+            da.out[l - a0] = outs[l];
+            da.lse[l - a0] = lses ? lses[l] : nullptr;
+        }
+        if ((st = make_maps(P, da, a1 - a0, &kv_cache[i])) != BSA_OK) return st;
+        if ((st = from_cuda(launch_decode(P, da, &kv_cache[i].maps, a1 - a0, stream))) != BSA_OK)
+            return st;
+    }
+    return BSA_OK;
 }
 
 bsa_status_t bsa_sparse_decode(const bsa_params_t* params, const void* q, const void* k_cache,

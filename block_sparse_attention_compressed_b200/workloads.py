@@ -47,6 +47,7 @@ class Workload:
     block_size: int = 64
     needle_shift: float = 2.0
     forecast: bool = False  # select with one Forecast vector per GQA group (f = the group's mean q)
+    anchors: tuple = (0,)   # multi-layer: layers that select; the others reuse the last anchor's
 
     @property
     def group(self) -> int:
@@ -64,7 +65,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The decode workloads: one small parity case and five throughput cases.
+# The decode workloads: one small parity case and six throughput cases.
 WORKLOADS: dict[str, Workload] = {
     w.name: w
     for w in [
@@ -84,6 +85,9 @@ WORKLOADS: dict[str, Workload] = {
         Workload("forecast-bf16-128k-b16", batch=16, num_q_heads=32, num_kv_heads=8, head_dim=128,
                  seq_len=131072, dtype="bf16", n_init=1, n_local=4, top_k=64, needles=16,
                  seed=1006, forecast=True),
+        Workload("anchors-2of4-64k-b8", batch=8, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                 seq_len=65536, dtype="bf16", n_init=1, n_local=2, top_k=48, needles=8, seed=1007,
+                 layers=4, anchors=(0, 2)),
     ]
 }
 DEFAULT_WORKLOAD = "gqa4-bf16-128k-b16"
@@ -193,7 +197,7 @@ def algorithmic_bytes(w: Workload, T: int | None = None) -> dict:
     sel_tokens = n_sel * w.block_size
     if w.n_local > 0 or n_sel == nb:          # the last (possibly partial) block is selected
         sel_tokens -= nb * w.block_size - T
-    ck = pairs * nc * d * e
+    ck = pairs * nc * d * e * len(w.anchors)   # every anchor layer scores its compressed keys
     kv = w.layers * pairs * sel_tokens * d * e * 2
     qo = w.layers * w.batch * w.num_q_heads * d * e * 2
     app = 0

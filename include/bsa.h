@@ -197,6 +197,26 @@ bsa_status_t bsa_sparse_decode_layers(const bsa_params_t* params, int32_t num_la
                                       void* const* outs, float* const* lses, void* workspace,
                                       size_t workspace_bytes, cudaStream_t stream);
 
+/* Anchored index reuse ([CoSA] Kascade abstract: exact top-k indices computed in a few anchor
+ * layers and reused, head by head, by the layers that follow; [HySparse2] CLSA abstract: one
+ * routing index shared across layers). anchors is a HOST array of num_anchors layer numbers,
+ * ascending, anchors[0] == 0, each < num_layers <= params->num_layers. For anchor i this runs
+ * bsa_select_blocks on q[anchors[i]] and cks[anchors[i]], writing its selection to
+ * block_idx + i * (batch * num_kv_heads * (n_init + n_local + top_k)) and
+ * n_sel + i * (batch * num_kv_heads) (per kv head, so the reuse is head-aware), then
+ * bsa_sparse_decode_layers on layers [anchors[i], anchors[i+1]) (the last group runs to
+ * num_layers) with that selection. q, k_caches, v_caches, cks, outs and lses are HOST arrays of
+ * num_layers device pointers (cks is read at the anchors only; lses may be NULL or contain NULLs).
+ * Everything is queued on `stream` with no host synchronisation. Errors as the two calls it
+ * chains; an invalid schedule is BSA_ERR_INVALID_ARG. */
+bsa_status_t bsa_decode_step_anchored(const bsa_params_t* params, int32_t num_layers,
+                                      const int32_t* anchors, int32_t num_anchors,
+                                      const void* const* q, const void* const* k_caches,
+                                      const void* const* v_caches, const void* const* cks,
+                                      const int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                                      void* const* outs, float* const* lses, void* workspace,
+                                      size_t workspace_bytes, cudaStream_t stream);
+
 /* One decode step of one layer, as launches chained on `stream` with programmatic dependent
  * launch: optional append (when k_new and v_new are both non-NULL), then bsa_select_blocks, then
  * bsa_sparse_decode with the fresh selection. block_idx / n_sel receive the selection;

@@ -164,6 +164,31 @@ def test_entry_points_reject_bad_arguments_before_launch(lib):
     assert lib.bsa_read_device_error(A, 4, None, S0) == bsa.BSA_ERR_INVALID_ARG
 
 
+def test_anchored_schedule_validated_before_launch(lib):
+    """bsa_decode_step_anchored: the anchor list must start at layer 0, ascend and stay below
+    num_layers; the Forecast selection validates like bsa_select_blocks."""
+    p = _p(num_layers=4)
+    P = ctypes.byref(p)
+    ws_need = bsa.bsa_workspace_size(p)
+    N = None
+    arr = (ctypes.c_void_p * 4)(A, A, A, A)
+
+    def run(anchors, layers=4, ws=ws_need):
+        a = (ctypes.c_int32 * len(anchors))(*anchors)
+        return lib.bsa_decode_step_anchored(P, layers, a, len(anchors), arr, arr, arr, arr, A, A, A,
+                                            arr, N, A, ws, S0)
+    for bad in ([1], [0, 0], [0, 3, 2], [0, 4], [0, 1, 2, 3, 3]):
+        assert run(bad) == bsa.BSA_ERR_INVALID_ARG, bad
+    assert run([0, 2], layers=5) == bsa.BSA_ERR_INVALID_ARG       # more layers than planned
+    assert run([0, 2], ws=ws_need - 1) == bsa.BSA_ERR_WORKSPACE
+    assert lib.bsa_decode_step_anchored(P, 4, N, 1, arr, arr, arr, arr, A, A, A, arr, N, A,
+                                        ws_need, S0) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_select_blocks_forecast(P, N, A, A, A, A, N, A, ws_need, S0) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_select_blocks_forecast(P, MIS, A, A, A, A, N, A, ws_need, S0) == bsa.BSA_ERR_INVALID_ARG
+    assert lib.bsa_select_blocks_forecast(P, A, A, A, A, A, N, A, ws_need - 1,
+                                          S0) == bsa.BSA_ERR_WORKSPACE
+
+
 def test_binding_rejects_host_tensors(lib):
     import torch
     p = _p()

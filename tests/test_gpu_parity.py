@@ -11,7 +11,7 @@ import block_sparse_attention_compressed_b200 as bsa
 import oracle
 from block_sparse_attention_compressed_b200.workloads import WORKLOADS, Workload
 from gpu_helpers import (GpuRun, check_output, check_selection, forecast_check, full_check,
-                         oracle_on_pairs, sample_pairs)
+                         near_tie, oracle_on_pairs, sample_pairs)
 
 pytestmark = pytest.mark.gpu
 
@@ -442,6 +442,69 @@ def test_forecast_full_workload(cuda_device):
     hit = np.mean([np.isin(nd[b, h], idx[b, h]).mean() for b in range(w.batch)
                    for h in range(w.num_kv_heads)])
     assert hit > 0.9, hit
+    del run
+    torch.cuda.empty_cache()
+
+
+# ----------------------------------------------------------- anchored index reuse (Kascade, CLSA)
+@pytest.mark.parametrize("anchors", [(0, 2), (0, 1, 3)])
+def test_anchored_reuse(anchors, cuda_device):
+    """Each anchor layer selects its own blocks per kv head; the layers up to the next anchor
+    attend those blocks."""
+    w = BASE.replace(name="x", batch=2, seq_len=3000 + 29, top_k=6, needles=3, layers=4,
+                     anchors=anchors)
+    run = GpuRun(w)
+    run.compress()
+    A, s = len(anchors), run.sizes
+    idx = torch.full((A, w.batch, w.num_kv_heads, s.sel_cap), -7, dtype=torch.int32, device="cuda")
+    ns = torch.full((A, w.batch, w.num_kv_heads), -7, dtype=torch.int32, device="cuda")
+    bsa.bsa_decode_step_anchored(run.p, anchors, [run.q[L] for L in range(w.layers)], run.data["k"],
+                                 run.data["v"], run.ck, run.data["seq_lens"], idx, ns, run.out,
+                                 run.lse, run.ws)
+    assert run.device_errors() == 0
+    pairs = list(range(w.batch * w.num_kv_heads))
+    bounds = list(anchors) + [w.layers]
+    for i in range(A):
+        a0, a1 = bounds[i], bounds[i + 1]
+        orc = oracle_on_pairs(run, pairs, a0)           # the anchor layer's own selection
+        gi, gn = idx[i].view(len(pairs), -1).cpu().numpy(), ns[i].view(-1).cpu().numpy()
+        for j, pr in enumerate(pairs):
+            n_o = int(orc["n_sel"][j])
+            assert int(gn[pr]) == n_o
+            if not near_tie(orc["boundary"][j]):
+                assert gi[pr, :n_o].tolist() == orc["idx"][j, :n_o].tolist(), (i, pr)
+        # every layer of the group attends the anchor's (GPU) selection
+        for L in range(a0, a1):
+            ref = oracle_on_pairs(run, pairs, L, given_idx=gi, given_n_sel=gn)
+            check_output(run, pairs, ref, L)
+
+
+@pytest.mark.slow
+def test_full_anchored_workload(cuda_device):
+    """The 4 x 64K x 8 workload with anchors at layers 0 and 2, in the bench's launch
+    configuration (one anchored call), checked on sampled pairs."""
+    w, run = _full_run("anchors-2of4-64k-b8")
+    A, s = len(w.anchors), run.sizes
+    idx = torch.full((A, w.batch, w.num_kv_heads, s.sel_cap), -7, dtype=torch.int32, device="cuda")
+    ns = torch.full((A, w.batch, w.num_kv_heads), -7, dtype=torch.int32, device="cuda")
+    bsa.bsa_decode_step_anchored(run.p, w.anchors, [run.q[L] for L in range(w.layers)],
+                                 run.data["k"], run.data["v"], run.ck, run.data["seq_lens"], idx, ns,
+                                 run.out, run.lse, run.ws)
+    assert run.device_errors() == 0
+    pairs = sample_pairs(w, 6, seed=3)
+    bounds = list(w.anchors) + [w.layers]
+    for i in range(A):
+        orc = oracle_on_pairs(run, pairs, bounds[i])
+        gi = idx[i].view(-1, s.sel_cap).cpu().numpy()
+        gn = ns[i].view(-1).cpu().numpy()
+        for j, pr in enumerate(pairs):
+            n_o = int(orc["n_sel"][j])
+            assert int(gn[pr]) == n_o
+            if not near_tie(orc["boundary"][j]):
+                assert gi[pr, :n_o].tolist() == orc["idx"][j, :n_o].tolist(), (i, pr)
+        for L in range(bounds[i], bounds[i + 1]):
+            ref = oracle_on_pairs(run, pairs, L, given_idx=gi[pairs], given_n_sel=gn[pairs])
+            check_output(run, pairs, ref, L)
     del run
     torch.cuda.empty_cache()
 
