@@ -75,8 +75,9 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
     P.nchunk = (P.nc_cap + 63) / 64;
     P.total_chunks = (int64_t)P.pairs * P.nchunk;
     P.nstat = P.nchunk;  // softmax statistics per 64-row chunk
-    P.score_ctas = (int)(P.total_chunks < 2 * kNumSMs ? (P.total_chunks > 0 ? P.total_chunks : 1)
-                                                       : 2 * kNumSMs);
+    // three CTAs per SM: 3 x 64 KB of compressed-key stages in flight per SM
+    P.score_ctas = (int)(P.total_chunks < 3 * kNumSMs ? (P.total_chunks > 0 ? P.total_chunks : 1)
+                                                       : 3 * kNumSMs);
     if (P.dtype == BSA_BF16 && (int64_t)P.pairs * P.nc_cap > 0x7fffffffLL) return BSA_ERR_UNSUPPORTED;
     // Selection: one CTA per pair when there are enough pairs to fill the GPU in one wave,
     // otherwise the pairs' windows are split into parts of at least 256 windows. A part's window

@@ -105,7 +105,7 @@ struct ScoreStage {
 // warps lets one of them wait two phases ahead, where the parity test cannot tell the phases
 // apart and passes on a slot whose copy is still in flight.)
 template <int D>
-__global__ void __launch_bounds__(kScoreTmaThreads, 2)
+__global__ void __launch_bounds__(kScoreTmaThreads, 3)
     score_tma_kernel(const ScoreArgs a, const __grid_constant__ CUtensorMap ck_map, const int nstages) {
     extern __shared__ uint8_t dsm_raw[];
     __shared__ __align__(8) uint64_t full[kScoreMaxStages], empty[kScoreMaxStages];
@@ -1004,8 +1004,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
             // stages are contiguous in shared memory, so window j sits at index j of slot 0); the
             // lanes then take running maxima over groups of r lanes, and lane r*i adds window
             // 32t + r*i - 1 when L = 2 (lane 31 of the previous tile for i = 0)
-            const int bpt = 32 / r_w;  // blocks per tile
-            const int tiles = (nb + bpt - 1) / bpt;
+            const int lsh = __ffs(r_w) - 1;  // log2(r)
+            const int bsh = 5 - lsh;          // log2(blocks per tile)
+            const int bpt = 1 << bsh;
+            const int tiles = (nb + bpt - 1) >> bsh;
             const int nw = kSelectThreads / 32;
             const int t_lo = (int)((int64_t)warp * tiles / nw), t_hi = (int)((int64_t)(warp + 1) * tiles / nw);
             auto S_at = [&](int j) -> float {
@@ -1017,29 +1019,39 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
             float prev = t_lo > 0 ? S_at(32 * t_lo - 32 + lane) : -INFINITY;
             const int clo = cand_begin(a, nb), chi = cand_end(a, nb);
             for (int t0 = t_lo; t0 < t_hi; t0 += kTileU) {
-                float cur[kTileU];
-#pragma unroll
-                for (int u = 0; u < kTileU; ++u) cur[u] = t0 + u < t_hi ? S_at(32 * (t0 + u) + lane) : -INFINITY;
+                // the tiles' chains side by side: reads, then each shuffle step for all tiles
+                float cur[kTileU], m[kTileU];
 #pragma unroll
                 for (int u = 0; u < kTileU; ++u) {
-                    const int t = t0 + u;
-                    if (t >= t_hi) break;  // warp-uniform
-                    float m = cur[u];
+                    cur[u] = t0 + u < t_hi ? S_at(32 * (t0 + u) + lane) : -INFINITY;
+                    m[u] = cur[u];
+                }
 #pragma unroll
-                    for (int off = 1; off < 32; off <<= 1)
-                        if (off < r_w) m = fmaxf(m, __shfl_down_sync(0xffffffffu, m, off));
-                    const float before = __shfl_up_sync(0xffffffffu, cur[u], 1);
-                    const float last_prev = __shfl_sync(0xffffffffu, u == 0 ? prev : cur[u > 0 ? u - 1 : 0], 31);
-                    if (L_w == 2) m = fmaxf(m, lane == 0 ? last_prev : before);
-                    const int b = t * bpt + lane / r_w;
-                    if ((lane & (r_w - 1)) == 0 && b < nb) {
-                        const uint32_t key = order_key(m);
+                for (int off = 1; off < 32; off <<= 1) {
+                    if (off < r_w) {
+#pragma unroll
+                        for (int u = 0; u < kTileU; ++u) m[u] = fmaxf(m[u], __shfl_down_sync(0xffffffffu, m[u], off));
+                    }
+                }
+                if (L_w == 2) {
+#pragma unroll
+                    for (int u = 0; u < kTileU; ++u) {
+                        const float before = __shfl_up_sync(0xffffffffu, cur[u], 1);
+                        const float last_prev = __shfl_sync(0xffffffffu, u == 0 ? prev : cur[u > 0 ? u - 1 : 0], 31);
+                        m[u] = fmaxf(m[u], lane == 0 ? last_prev : before);
+                    }
+                }
+#pragma unroll
+                for (int u = 0; u < kTileU; ++u) {
+                    const int b = ((t0 + u) << bsh) + (lane >> lsh);
+                    if ((lane & (r_w - 1)) == 0 && t0 + u < t_hi && b < nb) {
+                        const uint32_t key = order_key(m[u]);
                         keys[b] = key;
                         if (b >= clo && b < chi) {
                             kand &= key;
                             kor |= key;
                         }
-                        if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + b] = m;
+                        if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + b] = m[u];
                     }
                 }
                 prev = cur[kTileU - 1];
