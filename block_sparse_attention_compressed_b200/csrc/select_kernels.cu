@@ -497,8 +497,14 @@ __device__ __forceinline__ void find_digit_from_top(const int* hist, int nbins, 
     }
     if (lane == 31) s_warp[warp] = incl;
     __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; ++w) base += s_warp[w];
+    // totals of the warps before this one (a warp scan over the per-warp totals)
+    int wt = lane < (NT >> 5) ? s_warp[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, wt, off);
+        if (lane >= off) wt += y;
+    }
+    const int base = __shfl_sync(0xffffffffu, wt, (warp + 31) & 31) * (warp > 0);
     const int excl = base + incl - c;
     if (excl < need && need <= excl + c) {
         int acc = excl;
@@ -571,7 +577,7 @@ __device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys
     int* hist = t.hist;
     uint32_t* s_bkey = t.bkey;
     int* s_bidx = t.bidx;
-    const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31;
+    const int tid = threadIdx.x, NT = blockDim.x;
     const int init_end = cand_begin(a, nb);
     const int clo = init_end, chi = cand_end(a, nb);
     const int ncand = chi - clo;
