@@ -447,12 +447,12 @@ def test_forecast_full_workload(cuda_device):
 
 
 # ----------------------------------------------------------- anchored index reuse (Kascade, CLSA)
-@pytest.mark.parametrize("anchors", [(0, 2), (0, 1, 3)])
-def test_anchored_reuse(anchors, cuda_device):
+@pytest.mark.parametrize("anchors,dtype", [((0, 2), "bf16"), ((0, 1, 3), "bf16"), ((0, 2), "f32")])
+def test_anchored_reuse(anchors, dtype, cuda_device):
     """Each anchor layer selects its own blocks per kv head; the layers up to the next anchor
     attend those blocks."""
     w = BASE.replace(name="x", batch=2, seq_len=3000 + 29, top_k=6, needles=3, layers=4,
-                     anchors=anchors)
+                     anchors=anchors, dtype=dtype)
     run = GpuRun(w)
     run.compress()
     A, s = len(anchors), run.sizes
