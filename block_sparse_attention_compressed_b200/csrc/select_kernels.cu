@@ -28,8 +28,9 @@ namespace {
 constexpr int kScoreThreads = kScoreWarps * 32;
 constexpr int kSelectThreads = 512;
 
-// Block-wide exclusive scan of one int per thread (contiguous, in thread order). With `reuse`,
-// s_warp may be written again as soon as it returns.
+// Block-wide exclusive scan of one int per thread (contiguous, in thread order), with one barrier:
+// every warp scans its own values, publishes its total, and then scans all the warps' totals
+// itself. With `reuse`, s_warp may be written again as soon as it returns.
 __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total, bool reuse = true) {
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
     int x = v;
@@ -40,18 +41,14 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
     }
     if (lane == 31) s_warp[warp] = x;
     __syncthreads();
-    if (warp == 0) {
-        int w = lane < nwarps ? s_warp[lane] : 0;
+    int w = lane < nwarps ? s_warp[lane] : 0;
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            int y = __shfl_up_sync(0xffffffffu, w, off);
-            if (lane >= off) w += y;
-        }
-        if (lane < nwarps) s_warp[lane] = w;
+    for (int off = 1; off < 32; off <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, w, off);
+        if (lane >= off) w += y;
     }
-    __syncthreads();
-    const int base = warp > 0 ? s_warp[warp - 1] : 0;
-    *total = s_warp[nwarps - 1];
+    const int base = warp > 0 ? __shfl_sync(0xffffffffu, w, warp - 1) : 0;
+    *total = __shfl_sync(0xffffffffu, w, nwarps - 1);
     if (reuse) __syncthreads();
     return base + x - v;
 }
@@ -1001,11 +998,12 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     uint32_t kand = 0xffffffffu, kor = 0u;  // over the candidate keys this thread writes
     if (npieces <= R) {
         // every stage needed is in flight from the start: wait for all that were issued
+        // (a wait that runs out is reported; the pass then reads whatever the ring holds, so that
+        // every thread takes the same path to the barriers below)
         bool waited = true;
         for (int r = 0; r < n_pre && waited; ++r) waited = mbar_wait(&full[r], 0, kScoreWaitPolls);
-        if (!waited) {
-            if (tid == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
-        } else if (shuffle_max) {
+        if (!waited) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+        if (shuffle_max) {
             // warp w takes a contiguous run of 32-window tiles: lane l scores window 32t + l (the
             // stages are contiguous in shared memory, so window j sits at index j of slot 0); the
             // lanes then take running maxima over groups of r lanes, and lane r*i adds window
@@ -1081,8 +1079,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
             }
         }
     }
-    __syncthreads();
-    if (!keys_done) {
+    if (!keys_done) {  // uniform: the window scores S are complete once every thread is here
+        __syncthreads();
         // block scores: the maximum of S over the complete windows overlapping each block
         const int clo = cand_begin(a, nb), chi = cand_end(a, nb);
         for (int b = tid; b < nb; b += kSelectThreads) {
