@@ -908,18 +908,18 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
         mbar_arrive_expect_tx(bar, bytes);
         bulk_load(ring + (size_t)(r % R) * kRingStage, src + (size_t)w0 * GP * 4, bytes, bar);
     };
-    // the sequence length and the chunk statistics (for the row capacity) in one round of loads,
-    // requested before the bulk copies so that they do not queue behind them; the statistics are
-    // staged in the key array
+    // the sequence length and, in warp h < G, head h's chunk statistics (lane l: chunks l + 32u of
+    // the row capacity) in one round of loads, requested before the bulk copies so that they do not
+    // queue behind them
     constexpr int kStatU = 4;
-    float2* s_st = reinterpret_cast<float2*>(keys);  // 2 * nstat * Gp <= key_words
-    const float2* st = a.stats + (size_t)pair * a.nstat * GP;
-    const int64_t n_st = a.nstat * GP;
+    const float2* sth = a.stats + (size_t)pair * a.nstat * GP + warp;  // [chunk][GP], head `warp`
     float2 sv[kStatU];
+    if (warp < a.G && !a.raw) {
 #pragma unroll
-    for (int u = 0; u < kStatU; ++u) {
-        const int64_t e = tid + (int64_t)u * kSelectThreads;
-        if (e < n_st) sv[u] = ld_cg(st + e);
+        for (int u = 0; u < kStatU; ++u) {
+            const int64_t c = lane + 32 * u;
+            if (c < a.nstat) sv[u] = ld_cg(sth + c * GP);
+        }
     }
     const int64_t T = a.seq_lens[pair / a.Hkv];
     __syncthreads();  // every load above has been issued
@@ -927,18 +927,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     const int n_pre = min(cap_pieces, R);
     if (tid == 0)
         for (int r = 0; r < n_pre; ++r) issue(r, a.lg_stride);
-#pragma unroll
-    for (int u = 0; u < kStatU; ++u) {
-        const int64_t e = tid + (int64_t)u * kSelectThreads;
-        if (e < n_st) s_st[e] = sv[u];
-    }
-    for (int64_t e = tid + (int64_t)kStatU * kSelectThreads; e < n_st; e += kSelectThreads) s_st[e] = ld_cg(st + e);
     const bool ok = T >= 0 && T <= a.T_cap;
     const int nc = ok ? (int)num_windows(T, a.l, a.s) : 0;
     const int nb = ok ? (int)((T + a.BS - 1) / a.BS) : 0;
     const int npieces = (nc + PW - 1) / PW;
     const int nch = (nc + 63) / 64;
-    __syncthreads();
     // warp h merges head h's chunk statistics into its normaliser (M_h, Z_h), which every lane
     // then holds, and weighs the head's chunks: w[c][h] = exp2(m_c - M_h) / Z_h
     if (warp < a.G) {
@@ -947,8 +940,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
             for (int c = lane; c < nch; c += 32) wt[c * GP + warp] = 1.f;
         } else {
             float m = -INFINITY, sum = 0.f;
-            for (int c = lane; c < nch; c += 32) {
-                const float2 v = s_st[c * GP + warp];
+#pragma unroll
+            for (int u = 0; u < kStatU; ++u)
+                if (lane + 32 * u < nch) online_merge(m, sum, sv[u].x, sv[u].y);
+            for (int c = lane + 32 * kStatU; c < nch; c += 32) {  // rows longer than 8192 windows
+                const float2 v = ld_cg(sth + (int64_t)c * GP);
                 online_merge(m, sum, v.x, v.y);
             }
 #pragma unroll
@@ -958,7 +954,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
                 online_merge(m, sum, mo, so);
             }
             const float iz = sum > 0.f ? 1.f / sum : 0.f;
-            for (int c = lane; c < nch; c += 32) wt[c * GP + warp] = exp2f(s_st[c * GP + warp].x - m) * iz;
+#pragma unroll
+            for (int u = 0; u < kStatU; ++u)
+                if (lane + 32 * u < nch) wt[(lane + 32 * u) * GP + warp] = exp2f(sv[u].x - m) * iz;
+            for (int c = lane + 32 * kStatU; c < nch; c += 32)
+                wt[c * GP + warp] = exp2f(ld_cg(sth + (int64_t)c * GP).x - m) * iz;
         }
     }
     __syncthreads();
