@@ -1066,7 +1066,9 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
         }
     } else {
         for (int r = 0; r < npieces; ++r) {
-            if (!mbar_wait(&full[r % R], (r / R) & 1, kScoreWaitPolls)) {
+            // every thread leaves the loop together when a wait runs out (barriers follow)
+            const bool got = mbar_wait(&full[r % R], (r / R) & 1, kScoreWaitPolls);
+            if (!__syncthreads_and(got)) {
                 if (tid == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
                 break;
             }

@@ -134,6 +134,21 @@ def test_long_context_large_block_count(cuda_device):
     full_check(run, [0])
 
 
+@pytest.mark.slow
+def test_select_streams_rows_longer_than_the_ring(cuda_device):
+    """80 pairs get one selection CTA each; at T = 150000 a pair's 9374 windows of window terms
+    (150 KB) exceed the 128 KB shared-memory ring, so the stages are refilled as they are read."""
+    w = BASE.replace(name="x", batch=10, seq_len=150000, top_k=16, needles=4)
+    run = GpuRun(w)
+    run.compress()
+    run.select()
+    run.decode()
+    assert run.device_errors() == 0
+    full_check(run, sample_pairs(w, 4, seed=4))
+    del run
+    torch.cuda.empty_cache()
+
+
 def test_decode_with_given_indices_any_order(cuda_device):
     """Eq. 5 only depends on the set of blocks: shuffled indices and -1 holes give the same
     output as the oracle on the same set."""
