@@ -317,19 +317,45 @@ KERNEL_SOURCES = {"decode": "decode_kernels.cu", "combine": "decode_kernels.cu",
                   "compress": "compress_kernels.cu", "append": "compress_kernels.cu"}
 
 
+def _code_only(text: str) -> str:
+    """C/C++/CUDA source without its comments and with whitespace runs collapsed, so that a
+    comment edit does not count as a change of the compiled code."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"' or c == "'":          # string or char literal, kept whole
+            j = i + 1
+            while j < n and text[j] != c:
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash(kernel: str | None = None) -> str:
-    """sha256 (16 hex digits) of the kernel's sources, or of every kernel source when None."""
+    """sha256 (16 hex digits) of the kernel's sources with comments removed (see _code_only), or
+    of every kernel source when None."""
     import glob
     csrc = os.path.join(ROOT, "block_sparse_attention_compressed_b200", "csrc")
     if kernel is None:
-        paths = sorted(glob.glob(os.path.join(csrc, "*")))
+        paths = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")))
     else:
         own = next(f for k, f in KERNEL_SOURCES.items() if kernel.startswith(k))
         paths = [os.path.join(csrc, n) for n in (own, "bsa_internal.cuh", "bsa_api.cu")]
     h = hashlib.sha256()
     for p in paths:
-        with open(p, "rb") as f:
-            h.update(f.read())
+        with open(p, encoding="utf-8") as f:
+            h.update(_code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -102,7 +102,7 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
         if ((int64_t)P.pairs * P.select_parts > 0x7fffffff) return BSA_ERR_UNSUPPORTED;
         P.select_smem = (P.select_keys + (size_t)pw + (size_t)wmax) * sizeof(uint32_t);
         if (P.select_smem > 200 * 1024) return BSA_ERR_UNSUPPORTED;
-        // one part per pair: the pair's logits stream through a ring of 16 KB shared-memory stages,
+        // one part per pair: the pair's window terms stream through a ring of 16 KB shared-memory stages,
         // next to the keys, the window scores and one weight per (chunk, head)
         P.select_ring = 0;
         if (P.select_parts == 1) {

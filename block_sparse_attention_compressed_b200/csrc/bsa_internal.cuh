@@ -25,7 +25,7 @@ constexpr int kMaxCombineSlots = 1024;  // splits * Gp handled by the decode com
 struct Plan {
     int B, Hq, Hkv, G, Gp, D, l, s, BS, n_init, n_local, top_k, sel_cap, layers, dtype;
     int64_t T_cap, nc_cap, nb_cap;
-    int64_t lg_stride;  // windows per pair in the logits array (nc_cap rounded up to 4: 16 B)
+    int64_t lg_stride;  // windows per pair in the window-term array (nc_cap rounded up to 4: 16 B)
     int pairs;
     float scale_log2;  // attention scale * log2(e): softmax evaluated with exp2
     float score_log2;  // (1 / tau) * log2(e)
@@ -37,7 +37,7 @@ struct Plan {
     int select_parts, select_part_windows;
     size_t select_keys;  // words of the block-key array at the front of its shared memory
     size_t select_smem;  // dynamic shared memory of the selection kernel
-    int select_ring;     // one-part selection: 16 KB logits stages in flight (0: general kernel)
+    int select_ring;     // one-part selection: 16 KB window-term stages in flight (0: general kernel)
     // decode: grid = layers * pairs * dec_splits CTAs of kDecodeWarps warps, dec_bpc blocks each
     int dec_splits, dec_bpc;
     int dec_ctas, dec_slots;  // bf16: persistent CTAs; partial slots per (layer, pair)
@@ -74,7 +74,7 @@ struct ScoreArgs {
     const void* ck;
     const int32_t* seq_lens;
     uint32_t* err;
-    float* logits;        // [pairs][nc_cap][Gp], log2 units
+    float* logits;        // [pairs][lg_stride][Gp] window terms: exp2(x - chunk max), or raw x
     float2* stats;        // [pairs][nstat][Gp] (max, sum of exp2(x - max)) per chunk and head
     int B, Hq, Hkv, G, Gp, l, s;
     int64_t T_cap, nc_cap, lg_stride, nchunk, total_chunks, nstat;
@@ -95,7 +95,7 @@ struct SelectArgs {
     int Hkv, G, Gp, l, s, BS, n_init, n_local, top_k, sel_cap;
     int64_t T_cap, nc_cap, nb_cap, lg_stride, nstat, key_words;
     int parts, part_windows;
-    int ring;  // one-part kernel: logits stages in flight
+    int ring;  // one-part kernel: window-term stages in flight
     int raw;   // Forecast indexer: the stored scores are the window scores (weight 1, no statistics)
 };
 

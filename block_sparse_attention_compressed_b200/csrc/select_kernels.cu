@@ -1,25 +1,30 @@
 // Block selection: group scoring, block reduction and top-k (page "SparDA: Sparse Decoupled
 // Attention for Efficient Long-Context LLM Inference": Indexer Training, Eq. 6 for the score of a
 // GQA group; "Fine-grained supervision" for the max-pool onto the block grid; Theoretical
-// Foundation, Eq. 1 and SparDA Architecture, Eq. 4 for the union with init/local blocks and f_top).
+// Foundation, Eq. 1 and SparDA Architecture, Eq. 4 for the union with init/local blocks and f_top;
+// SparDA Architecture, "Compact Forecast Indexer" for the raw-score mode).
 //
 // Two kernels chained with programmatic dependent launch:
 //
 // score (persistent): the 64-row chunks of all pairs' compressed keys are shared evenly by the CTAs,
-//   so all finish together. It computes the group's logits x[j][h] = q_h . K~_j / tau (log2 units)
-//   and writes them to the workspace with each chunk's per-head (max, sum exp2(x - max)).
+//   so all finish together. For each chunk it computes the group's logits x[j][h] = q_h . K~_j / tau
+//   (log2 units), takes the chunk's maximum m per head and writes e = exp2(x - m) to the workspace
+//   with the chunk's per-head (m, sum e). (Raw-score mode, one Forecast vector per group: x itself.)
 //   bf16: a producer warp streams the chunks into a ring of shared-memory stages with 2-D TMA
 //   tensor copies (128-byte swizzle) completing on mbarriers; four consumer warps take whole
 //   chunks in turn and run the contraction on the tensor cores (mma.m16n8k16 with ldmatrix
 //   operands: rows are M, the G heads padded to 8 are N, head_dim is K). fp32: FMA dot products,
 //   one warp per row.
 //
-// select (pairs x parts CTAs): merges the chunk statistics into each head's softmax normaliser,
-//   turns the logits of its part of the windows into S[j] = sum_h softmax_h[j], max-pools S onto
-//   the blocks it owns and writes the block scores. The last part of a pair to finish (completion
-//   counter, no waiting) runs the top-k: an 8-bit radix select over order-preserving uint32 keys,
-//   ties resolved toward the lower block index by an ordered scan, then the ascending union with
-//   the init and local blocks.
+// select: merges the chunk statistics into each head's softmax normaliser (M, Z) and one weight per
+//   (chunk, head), w = exp2(m - M) / Z, so that S[j] = sum_h e[j][h] w[c(j)][h] = sum_h softmax_h[j];
+//   max-pools S onto the blocks and runs the top-k: radix digits over order-preserving uint32 keys
+//   (a wide first digit, then 8 bits), an exact ranking of the k-th key's bucket, ties toward the
+//   lower block index, then the ascending union with the init and local blocks.
+//   select_single_kernel (one CTA per pair) streams the pair's e rows into a shared-memory ring
+//   with 1-D bulk copies and takes the block maxima with warp shuffles; select_kernel (pairs x
+//   parts CTAs, for few pairs) splits the windows, and the last part of a pair to finish
+//   (completion counter, no waiting) runs the top-k.
 #include "bsa_internal.cuh"
 
 namespace bsa {
@@ -130,7 +135,7 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 3)
 
     if (warp == kScoreConsumers) {
         if (lane == 0) {
-            // the compressed keys are read once: keep the window logits (reread by the
+            // the compressed keys are read once: keep the window terms (reread by the
             // selection) in L2 rather than them
             const uint64_t ck_policy = l2_evict_first_policy();
             int k = 0, cur_pair = -1;

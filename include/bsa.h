@@ -129,7 +129,8 @@ bsa_status_t bsa_get_sizes(const bsa_params_t* params, bsa_sizes_t* sizes);
 
 /* Bytes of device workspace that bsa_select_blocks, bsa_sparse_decode(_layers) and
  * bsa_decode_step need for these parameters; 0 for invalid parameters. Holds the error word,
- * per-pair completion counters, fp32 window logits [B*Hkv][NC_cap][G] and attention partials. */
+ * per-pair completion counters, fp32 window terms [B*Hkv][NC_cap][G] with per-chunk statistics,
+ * block scores and attention partials. */
 size_t bsa_workspace_size(const bsa_params_t* params);
 
 /* Zero the workspace's error word and counters (cudaMemsetAsync on `stream`). Call once after
