@@ -1,0 +1,55 @@
+"""Host-side pieces of bench.py (no GPU): the source fingerprint that ties an ncu summary in
+profiles/ to the code it was taken on, and the byte model of every workload."""
+import os
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+import bench  # noqa: E402
+from block_sparse_attention_compressed_b200.workloads import WORKLOADS, algorithmic_bytes  # noqa: E402
+
+
+def test_code_only_drops_comments_and_keeps_literals():
+    src = 'int a = 1;  // note\n/* block\n comment */ const char* s = "// kept /* too */";\nfloat  b;'
+    assert bench._code_only(src) == 'int a = 1; const char* s = "// kept /* too */"; float b;'
+    # a comment edit does not change the fingerprint input, a code edit does
+    assert bench._code_only(src.replace("note", "other note")) == bench._code_only(src)
+    assert bench._code_only(src.replace("a = 1", "a = 2")) != bench._code_only(src)
+
+
+def test_kernel_source_hash_covers_each_kernel():
+    for k in ("decode_tma_kernel", "combine_kernel", "score_tma_kernel", "select_single_kernel",
+              "compress_keys_kernel", "append_kernel"):
+        h = bench.kernel_source_hash(k)
+        assert len(h) == 16 and int(h, 16) >= 0
+    assert bench.kernel_source_hash("decode_tma_kernel") != bench.kernel_source_hash("score_tma_kernel")
+
+
+def test_profile_summaries_parse():
+    """Every committed DRAM summary states its bytes per launch and a source fingerprint."""
+    import re
+    pdir = os.path.join(ROOT, "profiles")
+    names = [n for n in os.listdir(pdir) if n.endswith(".md") and "kernel_" in n]
+    assert names
+    for n in names:
+        text = open(os.path.join(pdir, n)).read()
+        assert re.search(r"kernel_sources_sha256_16:\s*[0-9a-f]{16}", text), n
+        if n.startswith(("decode_tma_kernel", "score_tma_kernel")):
+            assert re.search(r"dram_bytes_per_launch:\s*\d+", text), n
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_algorithmic_bytes(name):
+    """The byte model: compressed keys of every scoring layer, the selected K/V rows of every
+    layer, q and out, the appended rows and the Forecast vectors, summed."""
+    w = WORKLOADS[name]
+    ab = algorithmic_bytes(w)
+    assert ab["total"] == pytest.approx(ab["ck"] + ab["kv"] + ab["qo"] + ab["append"] + ab["f"])
+    pairs, e, d = w.batch * w.num_kv_heads, w.elem_bytes, w.head_dim
+    nc = (w.seq_len - w.cmp_kernel) // w.cmp_stride + 1
+    assert ab["ck"] == pairs * nc * d * e * len(w.anchors)
+    assert ab["f"] == (pairs * d * e if w.forecast else 0)
+    if name == "gqa4-bf16-128k-b16":
+        assert ab["total"] == 558071808   # 268.40 MB of compressed keys + 289.41 MB of K/V + q, out
