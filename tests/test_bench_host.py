@@ -53,3 +53,15 @@ def test_algorithmic_bytes(name):
     assert ab["f"] == (pairs * d * e if w.forecast else 0)
     if name == "gqa4-bf16-128k-b16":
         assert ab["total"] == 558071808   # 268.40 MB of compressed keys + 289.41 MB of K/V + q, out
+
+
+@pytest.mark.parametrize("name", ["forecast-bf16-128k-b16", "anchors-2of4-64k-b8", "gqa4-bf16-32k-b1"])
+def test_cpu_oracle_leg_runs(name):
+    """The bench's CPU-baseline / reference leg (the oracle on a bounded sample of pairs) for the
+    Forecast-indexer, anchored and plain workloads, on a shortened copy of each."""
+    from block_sparse_attention_compressed_b200.workloads import generate
+    w = WORKLOADS[name].replace(batch=1, seq_len=4096, needles=2)
+    data = generate(w, device="cpu")
+    steps_per_s, threads, desc = bench.cpu_oracle_sample(w, data, seconds=0.05)
+    assert steps_per_s > 0 and threads >= 1
+    assert "pairs" in desc
