@@ -15,7 +15,10 @@
  *      selected blocks (SparDA Architecture, Eq. 5).
  * A shared-index mode reuses one layer's selection for several layers (page "HySparse2: Hybrid
  * Sparse Attention with Two-Level KV Sharing", first abstract; page "CoSA: Accelerating
- * Long-Context Inference via Proxy-Kernel Co-Designed Sparse Attention", second abstract).
+ * Long-Context Inference via Proxy-Kernel Co-Designed Sparse Attention", second abstract), also
+ * with several anchor layers (bsa_decode_step_anchored). A Forecast-indexer selection scores with
+ * one given vector per GQA group instead of the query heads (SparDA Architecture, Eq. 4 and
+ * "Compact Forecast Indexer"; bsa_select_blocks_forecast).
  *
  * Conventions for every entry point:
  *   - All tensors are dense, row-major, on the current CUDA device, owned by the caller. The
