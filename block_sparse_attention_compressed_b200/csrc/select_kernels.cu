@@ -891,7 +891,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     uint8_t* ring = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(s_raw) + 127) & ~uintptr_t(127));
     uint32_t* keys = reinterpret_cast<uint32_t*>(ring + (size_t)a.ring * kRingStage);
     float* S = reinterpret_cast<float*>(keys + a.key_words);
-    float* wt = S + a.part_windows;  // [nstat][GP] chunk weights
+    // [nstat][GP] chunk weights, 16-byte aligned (one vector per chunk when GP = 4)
+    float* wt = reinterpret_cast<float*>((reinterpret_cast<uintptr_t>(S + a.part_windows) + 15) & ~uintptr_t(15));
     const int pair = blockIdx.x;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int R = a.ring;
@@ -1019,8 +1020,21 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
             const int tiles = (nb + bpt - 1) >> bsh;
             const int nw = kSelectThreads / 32;
             const int t_lo = (int)((int64_t)warp * tiles / nw), t_hi = (int)((int64_t)(warp + 1) * tiles / nw);
+            // S of window j = 32t + lane (the tile's windows share one chunk, so GP = 4 reads its
+            // weights as one broadcast vector)
             auto S_at = [&](int j) -> float {
-                const float v = window_score(0, min(j, nc - 1), min(j, nc - 1));
+                const int jj = min(j, nc - 1);
+                float v;
+                if constexpr (GP == 4) {
+                    const float4 e = reinterpret_cast<const float4*>(ring)[jj];
+                    const float4 w = reinterpret_cast<const float4*>(wt)[jj >> 6];
+                    v = e.x * w.x;
+                    if (a.G > 1) v += e.y * w.y;
+                    if (a.G > 2) v += e.z * w.z;
+                    if (a.G > 3) v += e.w * w.w;
+                } else {
+                    v = window_score(0, jj, jj);
+                }
                 return j < nc ? v : -INFINITY;
             };
             // four tiles at a time, their shared-memory reads in flight together
@@ -1160,7 +1174,7 @@ template <int GP>
 cudaError_t launch_select_k(const Plan& p, const SelectArgs& a, cudaStream_t st) {
     if (p.select_ring > 0) {
         const size_t smem = 128 + (size_t)p.select_ring * kRingStage +
-                            (p.select_keys + (size_t)p.select_part_windows + (size_t)p.nstat * p.Gp) *
+                            (p.select_keys + (size_t)p.select_part_windows + 4 + (size_t)p.nstat * p.Gp) *
                                 sizeof(uint32_t);
         cudaError_t e = ensure_smem<select_single_kernel<GP>>(smem);
         if (e != cudaSuccess) return e;
