@@ -134,6 +134,22 @@ def test_long_context_large_block_count(cuda_device):
     full_check(run, [0])
 
 
+@pytest.mark.parametrize("q_heads,kv_heads,d", [(16, 2, 64), (16, 8, 128), (8, 8, 64)])
+def test_one_cta_per_pair_selection_every_group_size(q_heads, kv_heads, d, cuda_device):
+    """Enough pairs (>= 75) for one selection CTA per pair, with groups of 8, 2 and 1 query heads:
+    the shared-memory ring, the shuffle block maxima and the top-k of select_single_kernel for
+    every padded group size."""
+    B = -(-80 // kv_heads)
+    w = BASE.replace(name="x", batch=B, num_q_heads=q_heads, num_kv_heads=kv_heads, head_dim=d,
+                     seq_len=3000 + 11, top_k=9, needles=3)
+    run = GpuRun(w)
+    run.compress()
+    run.select()
+    run.decode()
+    assert run.device_errors() == 0
+    full_check(run, sample_pairs(w, 24))
+
+
 @pytest.mark.slow
 def test_select_streams_rows_longer_than_the_ring(cuda_device):
     """80 pairs get one selection CTA each; at T = 150000 a pair's 9374 windows of window terms
