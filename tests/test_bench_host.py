@@ -65,3 +65,17 @@ def test_cpu_oracle_leg_runs(name):
     steps_per_s, threads, desc = bench.cpu_oracle_sample(w, data, seconds=0.05)
     assert steps_per_s > 0 and threads >= 1
     assert "pairs" in desc
+
+
+def test_forecast_vectors_are_group_mean_queries():
+    """The synthetic Forecast vector of each (batch, kv head) is the mean of the group's query
+    vectors of the first layer, stored in the cache type; other workloads carry none."""
+    import torch
+    from block_sparse_attention_compressed_b200.workloads import generate
+    w = WORKLOADS["forecast-bf16-128k-b16"].replace(batch=2, seq_len=2048, needles=2)
+    d = generate(w, device="cpu")
+    f = d["f"]
+    assert f.shape == (w.batch, w.num_kv_heads, w.head_dim) and f.dtype == w.torch_dtype
+    q = d["q"][0].float().view(w.batch, w.num_kv_heads, w.group, w.head_dim)
+    assert torch.equal(f, q.mean(dim=2).to(w.torch_dtype))
+    assert "f" not in generate(WORKLOADS["gqa4-bf16-32k-b1"].replace(seq_len=1024, needles=0))
