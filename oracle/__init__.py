@@ -97,6 +97,9 @@ def _bind(path: str):
         "bsa_oracle_compress_cache": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _INT,
                                              _P]),
         "bsa_oracle_num_threads": (_INT, []),
+        "bsa_oracle_set_num_threads": (None, [_INT]),
+        "bsa_oracle_decode_ck": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P, _INT,
+                                        _P, _P, _P, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -164,6 +167,18 @@ def widen(a: np.ndarray, dtype: int) -> np.ndarray:
 
 def num_threads() -> int:
     return _load().bsa_oracle_num_threads()
+
+
+@contextlib.contextmanager
+def threads(n: int):
+    """Run the OpenMP loops over pairs on n threads inside the block (timing only)."""
+    lib = _load()
+    saved = lib.bsa_oracle_num_threads()
+    lib.bsa_oracle_set_num_threads(n)
+    try:
+        yield
+    finally:
+        lib.bsa_oracle_set_num_threads(saved)
 
 
 def round_to(x, dtype: int) -> np.ndarray:
@@ -263,12 +278,14 @@ def _sizes(P: Problem):
 
 
 def decode(P: Problem, q, k_cache, v_cache, seq_lens, pairs=None, given_idx=None,
-           given_n_sel=None) -> dict:
+           given_n_sel=None, ck=None) -> dict:
     """Select + attend for the listed (batch, kv-head) pairs (all pairs by default).
 
     q/k_cache/v_cache are storage arrays ([B][Hq][d], [B][Hkv][T_cap][d]); returns a dict with
     idx [n][sel_cap], n_sel [n], block_scores [n][nb_cap], boundary [n][2], out [n][G][d],
-    lse [n][G]. With ``given_idx`` the selection is skipped and those blocks are attended.
+    lse [n][G]. With ``given_idx`` the selection is skipped and those blocks are attended. With
+    ``ck`` (float64 [n][nc_cap][d], as ``compress_cache`` returns for the same pairs) the
+    compressed keys are taken from it instead of being formed from the cache.
     """
     q = _raw_check(q, P.dtype)
     k_cache, v_cache = _raw_check(k_cache, P.dtype), _raw_check(v_cache, P.dtype)
@@ -290,10 +307,22 @@ def decode(P: Problem, q, k_cache, v_cache, seq_lens, pairs=None, given_idx=None
         out=np.zeros((n, G, d), dtype=np.float64),
         lse=np.zeros((n, G), dtype=np.float64),
     )
-    rc = _load().bsa_oracle_decode(
-        ctypes.byref(P), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), _ptr(pairs), n,
-        _ptr(given_idx), _ptr(given_n_sel), _ptr(res["idx"]), _ptr(res["n_sel"]),
-        _ptr(res["block_scores"]), _ptr(res["boundary"]), _ptr(res["out"]), _ptr(res["lse"]))
+    if ck is not None:
+        if given_idx is not None:
+            raise ValueError("given compressed keys are for a selection, not given indices")
+        nc_cap = num_windows(P.max_seq_len, P.cmp_kernel, P.cmp_stride)
+        ck = np.ascontiguousarray(np.asarray(ck, dtype=np.float64))
+        if ck.shape != (n, max(nc_cap, 0), d):
+            raise ValueError(f"ck must be [{n}][{nc_cap}][{d}] float64")
+        rc = _load().bsa_oracle_decode_ck(
+            ctypes.byref(P), _ptr(q), _ptr(ck), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+            _ptr(pairs), n, _ptr(res["idx"]), _ptr(res["n_sel"]), _ptr(res["block_scores"]),
+            _ptr(res["boundary"]), _ptr(res["out"]), _ptr(res["lse"]))
+    else:
+        rc = _load().bsa_oracle_decode(
+            ctypes.byref(P), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens), _ptr(pairs), n,
+            _ptr(given_idx), _ptr(given_n_sel), _ptr(res["idx"]), _ptr(res["n_sel"]),
+            _ptr(res["block_scores"]), _ptr(res["boundary"]), _ptr(res["out"]), _ptr(res["lse"]))
     if rc != 0:
         raise ValueError("bsa_oracle_decode rejected its arguments")
     return res

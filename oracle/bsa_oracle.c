@@ -235,12 +235,14 @@ static const void* orc_pair_rows(const orc_problem_t* P, const void* cache, int 
     return (const char*)cache + off;
 }
 
-/* Select (from q, or from the Forecast vectors f when given) and attend, per listed pair. */
+/* Select (from q, or from the Forecast vectors f when given) and attend, per listed pair. The
+ * compressed keys are formed from the cache (Eq. 2), or taken from ck_given [n_pairs][nc_cap][d]
+ * (already rounded, as bsa_oracle_compress_cache writes them) when that is not NULL. */
 static int orc_decode(const orc_problem_t* P, const void* f, const void* q, const void* k_cache,
-                      const void* v_cache, const int32_t* seq_lens, const int32_t* pairs,
-                      int n_pairs, const int32_t* given_idx, const int32_t* given_n_sel,
-                      int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary,
-                      double* out, double* lse) {
+                      const void* v_cache, const double* ck_given, const int32_t* seq_lens,
+                      const int32_t* pairs, int n_pairs, const int32_t* given_idx,
+                      const int32_t* given_n_sel, int32_t* idx, int32_t* n_sel,
+                      double* block_scores, double* boundary, double* out, double* lse) {
     if (!orc_problem_ok(P) || n_pairs < 0) return -1;
     const int G = P->num_q_heads / P->num_kv_heads, d = P->head_dim;
     const int sel_cap = P->n_init + P->n_local + P->top_k;
@@ -279,11 +281,13 @@ static int orc_decode(const orc_problem_t* P, const void* f, const void* q, cons
             for (int r = 0; r < ns; ++r) my_idx[r] = given_idx[(int64_t)i * sel_cap + r];
         } else {
             int64_t nc = bsa_oracle_num_windows(T, P->cmp_kernel, P->cmp_stride);
-            double* ck = (double*)malloc((size_t)(nc > 0 ? nc : 1) * d * sizeof(double));
+            const int64_t nc_cap = bsa_oracle_num_windows(P->max_seq_len, P->cmp_kernel, P->cmp_stride);
+            double* ck_own = ck_given ? NULL : (double*)malloc((size_t)(nc > 0 ? nc : 1) * d * sizeof(double));
+            const double* ck = ck_given ? ck_given + (int64_t)i * nc_cap * d : ck_own;
             double* S = (double*)malloc((size_t)(nc > 0 ? nc : 1) * sizeof(double));
             double* sb = (double*)malloc((size_t)(nb > 0 ? nb : 1) * sizeof(double));
             double bnd[2];
-            bsa_oracle_compress(kp, P->dtype, T, d, P->cmp_kernel, P->cmp_stride, P->dtype, ck);
+            if (!ck_given) bsa_oracle_compress(kp, P->dtype, T, d, P->cmp_kernel, P->cmp_stride, P->dtype, ck_own);
             if (f) {
                 double* fv = (double*)malloc((size_t)d * sizeof(double));
                 for (int c = 0; c < d; ++c) fv[c] = bsa_oracle_load(f, P->dtype, (int64_t)pair * d + c);
@@ -300,7 +304,7 @@ static int orc_decode(const orc_problem_t* P, const void* f, const void* q, cons
                 boundary[2 * i] = bnd[0];
                 boundary[2 * i + 1] = bnd[1];
             }
-            free(ck);
+            free(ck_own);
             free(S);
             free(sb);
         }
@@ -317,8 +321,20 @@ int bsa_oracle_decode(const orc_problem_t* P, const void* q, const void* k_cache
                       int n_pairs, const int32_t* given_idx, const int32_t* given_n_sel,
                       int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary,
                       double* out, double* lse) {
-    return orc_decode(P, NULL, q, k_cache, v_cache, seq_lens, pairs, n_pairs, given_idx,
+    return orc_decode(P, NULL, q, k_cache, v_cache, NULL, seq_lens, pairs, n_pairs, given_idx,
                       given_n_sel, idx, n_sel, block_scores, boundary, out, lse);
+}
+
+/* bsa_oracle_decode with the compressed keys of the listed pairs given (ck [n_pairs][nc_cap][d],
+ * e.g. from bsa_oracle_compress_cache): a decode step on a cache whose keys were compressed
+ * beforehand, as at decode time. */
+int bsa_oracle_decode_ck(const orc_problem_t* P, const void* q, const double* ck,
+                         const void* k_cache, const void* v_cache, const int32_t* seq_lens,
+                         const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel,
+                         double* block_scores, double* boundary, double* out, double* lse) {
+    if (!ck) return -1;
+    return orc_decode(P, NULL, q, k_cache, v_cache, ck, seq_lens, pairs, n_pairs, NULL, NULL, idx,
+                      n_sel, block_scores, boundary, out, lse);
 }
 
 /* SparDA Architecture: the blocks of Eq. (4), selected with the Forecast vectors f [B][Hkv][d]
@@ -328,8 +344,8 @@ int bsa_oracle_decode_forecast(const orc_problem_t* P, const void* f, const void
                                const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel,
                                double* block_scores, double* boundary, double* out, double* lse) {
     if (!f) return -1;
-    return orc_decode(P, f, q, k_cache, v_cache, seq_lens, pairs, n_pairs, NULL, NULL, idx, n_sel,
-                      block_scores, boundary, out, lse);
+    return orc_decode(P, f, q, k_cache, v_cache, NULL, seq_lens, pairs, n_pairs, NULL, NULL, idx,
+                      n_sel, block_scores, boundary, out, lse);
 }
 
 int bsa_oracle_attend_pairs(const orc_problem_t* P, const void* q, const void* k_cache,
@@ -369,6 +385,15 @@ int bsa_oracle_compress_cache(const orc_problem_t* P, const void* k_cache,
                             P->cmp_stride, P->dtype, dst);
     }
     return 0;
+}
+
+/* Threads of the OpenMP loops over pairs (n >= 1); timing only, no effect on the results. */
+void bsa_oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+    if (n >= 1) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
 }
 
 int bsa_oracle_num_threads(void) {

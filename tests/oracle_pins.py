@@ -388,6 +388,24 @@ def pin_decode_selection_composes():
         np.testing.assert_array_equal(res["out"][kvh], out)
 
 
+def pin_decode_given_compressed_keys_composes():
+    """A decode step on keys compressed beforehand (compress_cache, then decode with ck) gives the
+    selection, block scores and output of the driver that compresses on its own, bit for bit, on
+    ragged lengths and a pair subset; the thread count changes nothing."""
+    B, Hq, Hkv, d, Tc = 2, 6, 3, 16, 64 * 18
+    q, k, v = _randn((B, Hq, d), 86), _randn((B, Hkv, Tc, d), 87), _randn((B, Hkv, Tc, d), 88)
+    qb, kb, vb = _bf16_bits(q), _bf16_bits(k), _bf16_bits(v)
+    P = oracle.make_problem(B, Hq, Hkv, d, Tc, oracle.BF16, 1, 2, 4)
+    lens, pairs = [Tc, 64 * 11 + 23], [0, 2, 4, 5]
+    ref = oracle.decode(P, qb, kb, vb, lens, pairs=pairs)
+    ck = oracle.compress_cache(P, kb, lens, pairs=pairs)
+    for n in (1, 3):
+        with oracle.threads(n):
+            got = oracle.decode(P, qb, kb, vb, lens, pairs=pairs, ck=ck)
+        for key in ("idx", "n_sel", "block_scores", "out", "lse"):
+            np.testing.assert_array_equal(got[key], ref[key])
+
+
 def pin_shared_index_identical_layers():
     """[CLSA]/[Kascade] reuse: attending an identical layer with layer 0's index reproduces layer
     0's output; a different layer gives its own dense-over-selected result."""
@@ -460,6 +478,7 @@ ALL_PINS = [
     pin_attend_all_blocks_is_dense, pin_attend_subset_is_gathered_dense,
     pin_attend_identical_keys_mean_of_v,
     pin_decode_full_coverage_is_dense_gqa, pin_decode_selection_composes,
+    pin_decode_given_compressed_keys_composes,
     pin_shared_index_identical_layers,
     pin_forecast_decode_composes, pin_forecast_one_head_matches_base_selector,
 ]
