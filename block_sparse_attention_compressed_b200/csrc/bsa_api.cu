@@ -139,6 +139,33 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
         if (P.dtype == BSA_BF16 && (int64_t)P.pairs * P.T_cap > 0x7fffffffLL)
             return BSA_ERR_UNSUPPORTED;
     }
+    // Fused step (bf16): blocks start on window boundaries (BS / s a power of two up to 32, l / s
+    // 1 or 2, BS a multiple of the 64-token attention unit), the pair's window terms fit tensor
+    // memory (512 columns: 4 chunks of 64 windows per 2 * Gp columns, plus the slack of one
+    // block-maximum load of up to 4 chunks) and the rest fits one CTA.
+    {
+        P.step_fused = 0;
+        const int r_w = P.s > 0 ? P.BS / P.s : 0;
+        const bool geo = P.BS % P.s == 0 && P.l % P.s == 0 && r_w >= 1 && r_w <= 32 &&
+                         (r_w & (r_w - 1)) == 0 && (P.l / P.s == 1 || P.l / P.s == 2) && P.BS % 64 == 0;
+        if (P.dtype == BSA_BF16 && geo && P.nc_cap > 0 && P.nb_cap <= 16384) {
+            P.step_sgp = P.Gp;
+            P.step_nch_cap = (int)((P.nc_cap + 63) / 64);
+            const int64_t nbc_cap = (P.nb_cap * r_w + 63) / 64;  // chunks holding block starts
+            const int64_t chunk_cols = (nbc_cap > P.step_nch_cap ? nbc_cap : P.step_nch_cap);
+            const int per_load = 16 / P.Gp < 4 ? 16 / P.Gp : 4;
+            const int64_t cols = ((chunk_cols + 3) / 4 + per_load) * 2 * P.Gp;
+            uint32_t tc = 32;
+            while ((int64_t)tc < cols) tc <<= 1;
+            P.step_key_words = (int)((P.nb_cap + 3) / 4 * 4);
+            P.step_smem = step_smem_bytes(P.D, P.Gp, P.G, P.step_nch_cap, P.step_key_words, P.sel_cap);
+            if (tc <= 512 && P.step_smem > 0) {
+                P.step_tmem_cols = tc;
+                P.step_ctas = P.pairs < kNumSMs ? P.pairs : kNumSMs;
+                P.step_fused = 1;
+            }
+        }
+    }
     // Workspace
     size_t off = 0;
     P.off_err = off;
@@ -304,6 +331,60 @@ bsa_status_t make_maps(const Plan& P, const DecodeArgs& a, int layers, KVMapCach
             return BSA_ERR_CUDA;
     }
     return BSA_OK;
+}
+
+// TMA descriptors of the fused step: compressed keys, K and V in boxes of 64 rows.
+struct StepMapCache {
+    StepMaps maps;
+    MapKey ck, k, v;
+};
+
+StepArgs step_args(const Plan& P, const void* q, const void* f, const int32_t* seq_lens,
+                   int32_t* block_idx, int32_t* n_sel, float* block_scores, void* out, float* lse,
+                   void* ws) {
+    StepArgs a;
+    memset(&a, 0, sizeof a);
+    a.q = q;
+    a.f = f;
+    a.seq_lens = seq_lens;
+    a.block_idx = block_idx;
+    a.n_sel = n_sel;
+    a.block_scores = block_scores;
+    a.out = out;
+    a.lse = lse;
+    a.err = ws_at<uint32_t>(ws, P.off_err);
+    a.Hq = P.Hq;
+    a.Hkv = P.Hkv;
+    a.G = P.G;
+    a.l = P.l;
+    a.s = P.s;
+    a.BS = P.BS;
+    a.n_init = P.n_init;
+    a.n_local = P.n_local;
+    a.top_k = P.top_k;
+    a.sel_cap = P.sel_cap;
+    a.pairs = P.pairs;
+    a.T_cap = P.T_cap;
+    a.nc_cap = P.nc_cap;
+    a.nb_cap = P.nb_cap;
+    a.nch_cap = P.step_nch_cap;
+    a.key_words = P.step_key_words;
+    a.tmem_cols = P.step_tmem_cols;
+    a.score_log2 = P.score_log2;
+    a.scale_log2 = P.scale_log2;
+    return a;
+}
+
+bsa_status_t do_step_fused(const Plan& P, const void* q, const void* k_cache, const void* v_cache,
+                           const void* ck, const int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                           float* block_scores, void* out, float* lse, void* ws, cudaStream_t st) {
+    static thread_local StepMapCache c;
+    if (!encode_kv_map_cached(&c.maps.ck, &c.ck, ck, (uint64_t)P.pairs * P.nc_cap, P.D, 64) ||
+        !encode_kv_map_cached(&c.maps.k, &c.k, k_cache, (uint64_t)P.pairs * P.T_cap, P.D, 64) ||
+        !encode_kv_map_cached(&c.maps.v, &c.v, v_cache, (uint64_t)P.pairs * P.T_cap, P.D, 64))
+        return BSA_ERR_CUDA;
+    const StepArgs a = step_args(P, q, nullptr, seq_lens, block_idx, n_sel, block_scores, out, lse, ws);
+    return from_cuda(launch_step(P, a, &c.maps, st));
 }
 
 bsa_status_t do_append(const Plan& P, void* k_cache, void* v_cache, const void* k_new,
@@ -577,6 +658,9 @@ bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_
         st = do_append(P, k_cache, v_cache, k_new, v_new, seq_lens, ck, ws, stream);
         if (st != BSA_OK) return st;
     }
+    if (P.step_fused)
+        return do_step_fused(P, q, k_cache, v_cache, ck, seq_lens, block_idx, n_sel, block_scores, out,
+                             lse, ws, stream);
     if ((st = do_select(P, q, ck, seq_lens, block_idx, n_sel, block_scores, ws, stream)) != BSA_OK)
         return st;
     DecodeArgs da = decode_args(P, seq_lens, block_idx, n_sel, ws);
@@ -665,8 +749,12 @@ extern "C" bsa_status_t bsa_sparse_decode_noalloc(const bsa_params_t* params, co
                                                   const int32_t* block_idx, const int32_t* n_sel,
                                                   void* out, float* lse, uint32_t* device_error,
                                                   cudaStream_t stream) {
+    // one layer is attended: the scratch is laid out for one, whatever num_layers says
+    if (!params) return BSA_ERR_INVALID_ARG;
+    bsa_params_t one = *params;
+    one.num_layers = 1;
     Plan P;
-    bsa_status_t st = make_plan(params, &P);
+    bsa_status_t st = make_plan(&one, &P);
     if (st != BSA_OK) return st;
     if (!ok16(q) || !ok16(k_cache) || !ok16(v_cache) || !ok16(out) || !ok4(seq_lens) ||
         !ok4(block_idx) || !ok4(n_sel))
@@ -674,6 +762,13 @@ extern "C" bsa_status_t bsa_sparse_decode_noalloc(const bsa_params_t* params, co
     if ((lse && !ok4(lse)) || (device_error && !ok4(device_error))) return BSA_ERR_INVALID_ARG;
     const Plan V = noalloc_layout(P);
     if (V.ws_bytes > kNoAllocScratchBytes) return BSA_ERR_WORKSPACE;  // before any CUDA call
+    // the scratch used is the current device's: the stream must belong to that device
+    if (stream != 0 && stream != cudaStreamLegacy && stream != cudaStreamPerThread) {
+        int cur = -1, sdev = -1;
+        if (cudaGetDevice(&cur) != cudaSuccess || cudaStreamGetDevice(stream, &sdev) != cudaSuccess)
+            return BSA_ERR_CUDA;
+        if (sdev != cur) return BSA_ERR_INVALID_ARG;
+    }
     void* scratch = nullptr;
     if ((st = noalloc_scratch(&scratch)) != BSA_OK) return st;
     // error word and counters must start at zero: clear them on the stream, ahead of the kernel

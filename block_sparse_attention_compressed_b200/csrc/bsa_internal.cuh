@@ -42,6 +42,11 @@ struct Plan {
     int dec_splits, dec_bpc;
     int dec_ctas, dec_slots;  // bf16: persistent CTAs; partial slots per (layer, pair)
     int stage_tokens;  // bf16 decode pipeline stage: 64, 32 or 16 tokens (divides BS)
+    // fused step (bf16): one CTA per pair (a persistent grid walks the pairs); 0 when the shape is
+    // outside what that kernel handles, and the step then chains the separate kernels
+    int step_fused, step_ctas, step_sgp, step_nch_cap, step_key_words;
+    uint32_t step_tmem_cols;
+    size_t step_smem;
     // workspace layout (bytes)
     size_t off_err, off_sel_cnt, off_dec_cnt, off_logits, off_stats, off_bscores, off_part_ml,
         off_part_acc;
@@ -128,6 +133,29 @@ struct DecodeArgs {
     float scale_log2;
 };
 
+// The fused step: scoring, block reduction, top-k and attention of each (batch, kv head) pair in
+// one CTA, its window terms held in tensor memory.
+struct StepArgs {
+    const void* q;         // [B][Hq][D] queries: the attention heads, and the scoring heads unless f
+    const void* f;         // Forecast indexer: [B][Hkv][D] scoring vectors (raw scores), or null
+    const int32_t* seq_lens;
+    int32_t* block_idx;    // [pairs][sel_cap]
+    int32_t* n_sel;        // [pairs]
+    float* block_scores;   // [pairs][nb_cap] or null
+    void* out;             // [B][Hq][D]
+    float* lse;            // [B][Hq] or null
+    uint32_t* err;
+    int Hq, Hkv, G, l, s, BS, n_init, n_local, top_k, sel_cap, pairs;
+    int64_t T_cap, nc_cap, nb_cap;
+    int nch_cap, key_words;
+    uint32_t tmem_cols;
+    float score_log2, scale_log2;
+};
+// TMA descriptors of the step: compressed keys (boxes of 64 rows), K and V (boxes of 32 rows).
+struct alignas(64) StepMaps {
+    CUtensorMap ck, k, v;
+};
+
 // Launchers (one per kernel family); they pick the template instance from the plan's dtype/D.
 cudaError_t launch_compress_keys(const Plan& p, const CompressArgs& a, cudaStream_t st);
 cudaError_t launch_append(const Plan& p, const AppendArgs& a, cudaStream_t st);
@@ -136,6 +164,10 @@ cudaError_t launch_score(const Plan& p, const ScoreArgs& a, const CUtensorMap* c
 cudaError_t launch_select(const Plan& p, const SelectArgs& a, cudaStream_t st);
 cudaError_t launch_decode(const Plan& p, const DecodeArgs& a, const KVMaps* maps, int layers,
                           cudaStream_t st);
+cudaError_t launch_step(const Plan& p, const StepArgs& a, const StepMaps* maps, cudaStream_t st);
+// Shared-memory bytes of the fused step kernel (dynamic part) for a parameter set, or 0 when its
+// layout does not fit one CTA.
+size_t step_smem_bytes(int D, int sgp, int G, int nch_cap, int key_words, int sel_cap);
 // Encode a 2-D bf16 TMA descriptor over rows x D elements (128-byte swizzle, box 64 x box_rows).
 bool encode_kv_map(CUtensorMap* map, const void* base, uint64_t rows, int D, int box_rows);
 
@@ -193,6 +225,16 @@ inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 // ------------------------------------------------------------------------------------------------
 // Device helpers
 #ifdef __CUDACC__
+
+// A thread group that synchronises as one: the whole CTA (bar 0: __syncthreads) or the first `nt`
+// threads of the CTA behind named barrier `bar`. tid is the thread's index inside the group.
+struct Grp {
+    int tid, nt, bar;
+    __device__ __forceinline__ void sync() const {
+        if (bar == 0) __syncthreads();
+        else asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(nt) : "memory");
+    }
+};
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() {
@@ -252,10 +294,12 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xffff0000u); }
 
-// Running (max, sum exp2(x - max)) of a stream of log2-domain values.
+// Running (max, sum exp2(x - max)) of a stream of log2-domain values. The roundings are spelled
+// out (explicit mul / fma) so that every kernel merging the same statistics in the same order gets
+// the same bits, whatever contraction the compiler would pick in each context.
 __device__ __forceinline__ void online_add(float& m, float& s, float x) {
     float mn = fmaxf(m, x);
-    s = s * exp2f(m - mn) + exp2f(x - mn);
+    s = __fadd_rn(__fmul_rn(s, exp2f(m - mn)), exp2f(x - mn));
     m = mn;
 }
 __device__ __forceinline__ void online_merge(float& m, float& s, float m2, float s2) {
@@ -265,8 +309,19 @@ __device__ __forceinline__ void online_merge(float& m, float& s, float m2, float
         s = 0.f;
         return;
     }
-    s = s * exp2f(m - mn) + s2 * exp2f(m2 - mn);
+    s = __fmaf_rn(s2, exp2f(m2 - mn), __fmul_rn(s, exp2f(m - mn)));
     m = mn;
+}
+
+// A window's group score S = sum over the group's heads h < G of e[h] * w[h], in head order, with
+// the roundings spelled out: the selection kernels and the fused step give the same bits.
+template <int GP>
+__device__ __forceinline__ float group_sum(const float* e, const float* w, int G) {
+    float acc = __fmul_rn(e[0], w[0]);
+#pragma unroll
+    for (int h = 1; h < GP; ++h)
+        if (h < G) acc = __fmaf_rn(e[h], w[h], acc);
+    return acc;
 }
 
 // ---- shared-memory barriers and TMA (sm_90+ instructions, used on sm_100a)
@@ -282,6 +337,10 @@ __device__ __forceinline__ void mbar_fence_init() {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                  : "memory");
+}
+// Arrival that counts `count` times (one warp standing for several expected arrivals).
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
@@ -345,6 +404,92 @@ __device__ __forceinline__ void ldmatrix_x4_trans(uint32_t (&r)[4], uint32_t add
     asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                  : "r"(addr));
+}
+
+// ---- tensor memory (TMEM, 512 columns x 128 lanes of 32 bits per SM), used here as storage
+// next to shared memory. Warp w of a CTA reaches lanes 32 * (w % 4) .. 32 * (w % 4) + 31; an address
+// is (lane << 16) | column. Allocation is per CTA by one warp, in powers of two of >= 32 columns.
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(dst_smem)),
+                 "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_fence_before_sync() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_fence_after_sync() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+// Lane i of the warp stores v[0..N) to columns taddr.col .. +N of TMEM lane taddr.lane + i (warp-wide).
+template <int N>
+__device__ __forceinline__ void tmem_st(uint32_t taddr, const float (&v)[N]) {
+    static_assert(N == 2 || N == 4 || N == 8 || N == 16, "x2, x4, x8 or x16");
+    const uint32_t* u = reinterpret_cast<const uint32_t*>(v);
+    if constexpr (N == 2) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x2.b32 [%0], {%1, %2};" ::"r"(taddr), "r"(u[0]), "r"(u[1])
+                     : "memory");
+    } else if constexpr (N == 4) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1, %2, %3, %4};" ::"r"(taddr), "r"(u[0]),
+                     "r"(u[1]), "r"(u[2]), "r"(u[3])
+                     : "memory");
+    } else if constexpr (N == 8) {
+        asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+                     "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7])
+                     : "memory");
+    } else {
+        asm volatile(
+            "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, "
+            "%13, %14, %15, %16};" ::"r"(taddr),
+            "r"(u[0]), "r"(u[1]), "r"(u[2]), "r"(u[3]), "r"(u[4]), "r"(u[5]), "r"(u[6]), "r"(u[7]), "r"(u[8]),
+            "r"(u[9]), "r"(u[10]), "r"(u[11]), "r"(u[12]), "r"(u[13]), "r"(u[14]), "r"(u[15])
+            : "memory");
+    }
+}
+// Lane i of the warp loads columns taddr.col .. +N of TMEM lane taddr.lane + i into v (warp-wide;
+// complete after tmem_wait_ld).
+template <int N>
+__device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
+    static_assert(N == 2 || N == 4 || N == 8 || N == 16 || N == 32, "x2, x4, x8, x16 or x32");
+    uint32_t* u = reinterpret_cast<uint32_t*>(v);
+    if constexpr (N == 2) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0, %1}, [%2];" : "=r"(u[0]), "=r"(u[1]) : "r"(taddr)
+                     : "memory");
+    } else if constexpr (N == 4) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0, %1, %2, %3}, [%4];"
+                     : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3])
+                     : "r"(taddr)
+                     : "memory");
+    } else if constexpr (N == 8) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                     : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]),
+                       "=r"(u[7])
+                     : "r"(taddr)
+                     : "memory");
+    } else if constexpr (N == 16) {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15}, [%16];"
+            : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+              "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15])
+            : "r"(taddr)
+            : "memory");
+    } else {
+        asm volatile(
+            "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+            "%14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+            : "=r"(u[0]), "=r"(u[1]), "=r"(u[2]), "=r"(u[3]), "=r"(u[4]), "=r"(u[5]), "=r"(u[6]), "=r"(u[7]),
+              "=r"(u[8]), "=r"(u[9]), "=r"(u[10]), "=r"(u[11]), "=r"(u[12]), "=r"(u[13]), "=r"(u[14]), "=r"(u[15]),
+              "=r"(u[16]), "=r"(u[17]), "=r"(u[18]), "=r"(u[19]), "=r"(u[20]), "=r"(u[21]), "=r"(u[22]), "=r"(u[23]),
+              "=r"(u[24]), "=r"(u[25]), "=r"(u[26]), "=r"(u[27]), "=r"(u[28]), "=r"(u[29]), "=r"(u[30]), "=r"(u[31])
+            : "r"(taddr)
+            : "memory");
+    }
 }
 
 // Order-preserving map of an fp32 score onto uint32 (larger float -> larger key).

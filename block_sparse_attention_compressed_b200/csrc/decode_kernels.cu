@@ -26,6 +26,7 @@
 // of consecutive tokens in turn (FMA dot products, warp reductions), merge in shared memory, and
 // the last split of a (layer, pair) to finish (completion counter, no waiting) combines them.
 #include "bsa_internal.cuh"
+#include "tiles.cuh"
 
 namespace bsa {
 namespace {
@@ -386,13 +387,10 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
         }
     } else {
         const int r0 = 16 * warp;
-        const int mi = lane >> 3, ri = lane & 7;
         const Group gp{(int)threadIdx.x, kConsumerWarps * 32, 1};
         uint32_t qf[KS][2];
-        float m[2] = {-INFINITY, -INFINITY}, lsum[2] = {0.f, 0.f};
-        float acc[MT][4];
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+        AttnState<D> as;
+        as.reset();
         for (int k = 0;; ++k) {
             const int st = k % nstages;
             if (!mbar_wait(&full[st], (k / nstages) & 1, kWaitPolls)) {
@@ -405,98 +403,27 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
             uint8_t* vst = kst + NB * box_bytes;
             if (md.flags & kStageFirst) {
                 // q as the B operand: lane (g, tq) holds head g, d = 16ks + 2tq (+1, +8, +9)
-                const uint32_t* qs = reinterpret_cast<const uint32_t*>(kst + kv_bytes) + g * (D / 2);
-#pragma unroll
-                for (int ks = 0; ks < KS; ++ks) {
-                    qf[ks][0] = g < a.G ? qs[8 * ks + tq] : 0u;
-                    qf[ks][1] = g < a.G ? qs[8 * ks + 4 + tq] : 0u;
-                }
+                load_q_frag<D>(qf, reinterpret_cast<const uint32_t*>(kst + kv_bytes) + g * (D / 2), g < a.G, tq);
             }
-            if (r0 < md.nvalid) {
-                if (r0 + 16 > md.nvalid) {
-                    // rows past the sequence may hold anything: zero this warp's V rows there
-                    for (int e = lane; e < 16 * NB * 8; e += 32) {
-                        const int row = r0 + e / (NB * 8), bi = (e / 8) % NB, ch = e % 8;
-                        if (row >= md.nvalid)
-                            *reinterpret_cast<uint4*>(vst + bi * box_bytes + row * 128 + ch * 16) =
-                                make_uint4(0, 0, 0, 0);
-                    }
-                    fence_proxy_async_smem();
-                    __syncwarp();
-                }
-                // S^T = K q^T over this warp's 16 tokens
-                float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-                for (int ks = 0; ks < KS; ++ks) {
-                    const int row = r0 + ri + 8 * (mi & 1);
-                    const int ch = (ks & 3) * 2 + (mi >> 1);
-                    uint32_t af[4];
-                    ldmatrix_x4(af, smem_u32(kst + (ks >> 2) * box_bytes + row * 128 + ((ch ^ (row & 7)) << 4)));
-                    mma_bf16_16816(c, af[0], af[1], af[2], af[3], qf[ks][0], qf[ks][1]);
-                }
-                const float sl = a.scale_log2;
-                const bool va = r0 + g < md.nvalid, vb = r0 + g + 8 < md.nvalid;
-                const float x0 = va ? c[0] * sl : -INFINITY, x1 = va ? c[1] * sl : -INFINITY;
-                const float x2 = vb ? c[2] * sl : -INFINITY, x3 = vb ? c[3] * sl : -INFINITY;
-                float t0 = fmaxf(x0, x2), t1 = fmaxf(x1, x3);
-#pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    t0 = fmaxf(t0, __shfl_xor_sync(0xffffffffu, t0, off));
-                    t1 = fmaxf(t1, __shfl_xor_sync(0xffffffffu, t1, off));
-                }
-                const float mn0 = fmaxf(m[0], t0), mn1 = fmaxf(m[1], t1);
-                const float al0 = mn0 == -INFINITY ? 1.f : exp2f(m[0] - mn0);
-                const float al1 = mn1 == -INFINITY ? 1.f : exp2f(m[1] - mn1);
-                const float ref0 = mn0 == -INFINITY ? 0.f : mn0, ref1 = mn1 == -INFINITY ? 0.f : mn1;
-                const float p0 = exp2f(x0 - ref0), p2 = exp2f(x2 - ref0);
-                const float p1 = exp2f(x1 - ref1), p3 = exp2f(x3 - ref1);
-                m[0] = mn0;
-                m[1] = mn1;
-                lsum[0] = lsum[0] * al0 + (p0 + p2);
-                lsum[1] = lsum[1] * al1 + (p1 + p3);
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    acc[mt][0] *= al0;
-                    acc[mt][1] *= al1;
-                    acc[mt][2] *= al0;
-                    acc[mt][3] *= al1;
-                }
-                // P^T operand from the S^T accumulators (8x8 transposes), hi + lo bf16 parts
-                const uint32_t hi0 = pack_bf16x2(p0, p1), hi1 = pack_bf16x2(p2, p3);
-                const uint32_t lo0 = pack_bf16x2(p0 - bf16_lo(hi0), p1 - bf16_hi(hi0));
-                const uint32_t lo1 = pack_bf16x2(p2 - bf16_lo(hi1), p3 - bf16_hi(hi1));
-                const uint32_t bh0 = movmatrix_trans(hi0), bh1 = movmatrix_trans(hi1);
-                const uint32_t bl0 = movmatrix_trans(lo0), bl1 = movmatrix_trans(lo1);
-                // O^T += V^T P^T: V^T fragments straight from the swizzled stage (ldmatrix.trans)
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    const int row = r0 + ri + 8 * (mi >> 1);
-                    const int ch = 2 * mt + (mi & 1);
-                    uint32_t af[4];
-                    ldmatrix_x4_trans(af, smem_u32(vst + (ch >> 3) * box_bytes + row * 128 +
-                                                   (((ch & 7) ^ (row & 7)) << 4)));
-                    mma_bf16_16816(acc[mt], af[0], af[1], af[2], af[3], bh0, bh1);
-                    mma_bf16_16816(acc[mt], af[0], af[1], af[2], af[3], bl0, bl1);
-                }
-            }
+            if (r0 < md.nvalid) attend16<D>(kst, vst, box_bytes, r0, md.nvalid, qf, a.scale_log2, as, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);  // the ring slot may be refilled now
             if (md.flags & kStageLast) {
                 // publish this warp's state of the item, then merge the item's split as a group
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1) {
-                    lsum[0] += __shfl_xor_sync(0xffffffffu, lsum[0], off);
-                    lsum[1] += __shfl_xor_sync(0xffffffffu, lsum[1], off);
+                    as.lsum[0] += __shfl_xor_sync(0xffffffffu, as.lsum[0], off);
+                    as.lsum[1] += __shfl_xor_sync(0xffffffffu, as.lsum[1], off);
                 }
                 const int h0 = 2 * tq, h1 = 2 * tq + 1;
                 if (g == 0) {
                     if (h0 < a.G) {
-                        sm.M(warp, h0) = m[0];
-                        sm.L(warp, h0) = lsum[0];
+                        sm.M(warp, h0) = as.m[0];
+                        sm.L(warp, h0) = as.lsum[0];
                     }
                     if (h1 < a.G) {
-                        sm.M(warp, h1) = m[1];
-                        sm.L(warp, h1) = lsum[1];
+                        sm.M(warp, h1) = as.m[1];
+                        sm.L(warp, h1) = as.lsum[1];
                     }
                 }
                 // accumulator (mt, row g / g+8) <-> d = 16 mt + g (+8)
@@ -506,19 +433,16 @@ __global__ void __launch_bounds__(kTmaThreads, 2)
                 for (int mt = 0; mt < MT; ++mt) {
                     const int d0 = 16 * mt + g;
                     if (h0 < a.G) {
-                        w0[d0] = acc[mt][0];
-                        w0[d0 + 8] = acc[mt][2];
+                        w0[d0] = as.acc[mt][0];
+                        w0[d0 + 8] = as.acc[mt][2];
                     }
                     if (h1 < a.G) {
-                        w1[d0] = acc[mt][1];
-                        w1[d0 + 8] = acc[mt][3];
+                        w1[d0] = as.acc[mt][1];
+                        w1[d0 + 8] = as.acc[mt][3];
                     }
                 }
                 write_partial<D>(a, md.lp, md.seg, sm, gp);
-                m[0] = m[1] = -INFINITY;
-                lsum[0] = lsum[1] = 0.f;
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) acc[mt][0] = acc[mt][1] = acc[mt][2] = acc[mt][3] = 0.f;
+                as.reset();
             }
         }
     }

@@ -26,6 +26,8 @@
 //   parts CTAs, for few pairs) splits the windows, and the last part of a pair to finish
 //   (completion counter, no waiting) runs the top-k.
 #include "bsa_internal.cuh"
+#include "tiles.cuh"
+#include "topk.cuh"
 
 namespace bsa {
 namespace {
@@ -33,30 +35,6 @@ namespace {
 constexpr int kScoreThreads = kScoreWarps * 32;
 constexpr int kSelectThreads = 512;
 
-// Block-wide exclusive scan of one int per thread (contiguous, in thread order), with one barrier:
-// every warp scans its own values, publishes its total, and then scans all the warps' totals
-// itself. With `reuse`, s_warp may be written again as soon as it returns.
-__device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* total, bool reuse = true) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-    int x = v;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, x, off);
-        if (lane >= off) x += y;
-    }
-    if (lane == 31) s_warp[warp] = x;
-    __syncthreads();
-    int w = lane < nwarps ? s_warp[lane] : 0;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        int y = __shfl_up_sync(0xffffffffu, w, off);
-        if (lane >= off) w += y;
-    }
-    const int base = warp > 0 ? __shfl_sync(0xffffffffu, w, warp - 1) : 0;
-    *total = __shfl_sync(0xffffffffu, w, nwarps - 1);
-    if (reuse) __syncthreads();
-    return base + x - v;
-}
 
 __device__ __forceinline__ int64_t num_windows(int64_t T, int l, int s) {
     return T < l ? 0 : (T - l) / s + 1;
@@ -181,7 +159,6 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 3)
             }
         }
     } else {
-        const int mi = lane >> 3, ri = lane & 7;
         const bool h0 = 2 * tq < a.G, h1 = 2 * tq + 1 < a.G;
         uint32_t qf[KS][2];
         int q_pair = -1;
@@ -197,29 +174,12 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 3)
                 // q as the B operand: lane (g, tq) holds head g, d = 16ks + 2tq (+1, +8, +9)
                 q_pair = md.pair;
                 const int b = md.pair / a.Hkv, kvh = md.pair - b * a.Hkv;
-                const uint32_t* qs = reinterpret_cast<const uint32_t*>(
-                    reinterpret_cast<const uint16_t*>(a.q) + ((size_t)b * a.Hq + (size_t)kvh * a.G + g) * D);
-#pragma unroll
-                for (int ks = 0; ks < KS; ++ks) {
-                    qf[ks][0] = g < a.G ? qs[8 * ks + tq] : 0u;
-                    qf[ks][1] = g < a.G ? qs[8 * ks + 4 + tq] : 0u;
-                }
+                load_q_frag<D>(qf, reinterpret_cast<const uint32_t*>(reinterpret_cast<const uint16_t*>(a.q) +
+                                                                     ((size_t)b * a.Hq + (size_t)kvh * a.G + g) * D),
+                               g < a.G, tq);
             }
-            const uint8_t* cst = ring + (size_t)st * stage_bytes;
             float c[4][4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) c[r][0] = c[r][1] = c[r][2] = c[r][3] = 0.f;
-#pragma unroll
-            for (int ks = 0; ks < KS; ++ks) {
-#pragma unroll
-                for (int r = 0; r < 4; ++r) {  // four independent 16-row groups
-                    const int row = 16 * r + ri + 8 * (mi & 1);
-                    const int ch = (ks & 3) * 2 + (mi >> 1);
-                    uint32_t af[4];
-                    ldmatrix_x4(af, smem_u32(cst + (ks >> 2) * box_bytes + row * 128 + ((ch ^ (row & 7)) << 4)));
-                    mma_bf16_16816(c[r], af[0], af[1], af[2], af[3], qf[ks][0], qf[ks][1]);
-                }
-            }
+            score_chunk<D>(ring + (size_t)st * stage_bytes, qf, c, lane);
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[st]);  // the data is in registers: refill the slot
             if (a.raw) {
@@ -250,7 +210,7 @@ __global__ void __launch_bounds__(kScoreTmaThreads, 3)
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
 #pragma unroll
-                for (int e = 0; e < 4; ++e) x[r][e] = c[r][e] * a.score_log2;
+                for (int e = 0; e < 4; ++e) x[r][e] = __fmul_rn(c[r][e], a.score_log2);  // rounded here in every kernel
                 if (16 * r + g < md.nrows) {
                     m0 = fmaxf(m0, x[r][0]);
                     m1 = fmaxf(m1, x[r][1]);
@@ -442,339 +402,15 @@ __device__ void window_scores(const float* lg, int64_t j0, int64_t j1, int G, co
             const int64_t j = base + (int64_t)u * NT + tid;
             if (j < j1) {
                 const float2* w = wt + (j >> 6) * GP;
-                float acc = 0.f;
+                float wx[GP];
 #pragma unroll
-                for (int h = 0; h < GP; ++h)
-                    if (h < G) acc += r[u].v[h] * w[h].x;
-                S[j - j0] = acc;
+                for (int h = 0; h < GP; ++h) wx[h] = w[h].x;
+                S[j - j0] = group_sum<GP>(r[u].v, wx, G);
             }
         }
     }
 }
 
-// Top-k of the candidate blocks [init_end, local_begin) by score (ties: lower index first), united
-// with the init and local blocks, written ascending. keys[] (shared) holds the nb block keys and
-// may be overwritten. Each thread owns a contiguous segment of the candidates, kept in registers
-// when it has at most kKeysPerThread of them (larger candidate sets are streamed from shared
-// memory).
-//
-// The k-th largest key is located by radix digits below the bits that all candidates share: a
-// first digit of up to kFirstDigitBits bits (one histogram bin per value, found with a two-level
-// descending scan), then 8-bit digits. As soon as the digit bucket holding the k-th key has at
-// most kExactMax keys, the owners of those keys rank them exactly among themselves (score
-// descending, block ascending); the taken candidates are those above the bucket plus the bucket
-// keys ranked below the number still needed. Otherwise the ties at the final key value are taken
-// in block order.
-constexpr int kKeysPerThread = 8;
-constexpr int kFirstDigitBits = 12;
-constexpr int kExactMax = 128;
-constexpr int kHistBins = 1 << kFirstDigitBits;
-
-// Bin d* (scanning digits from the top) at which the running count of hist reaches `need`; the
-// winning thread publishes the digit, the count still needed inside it and the bin's size.
-__device__ __forceinline__ void find_digit_from_top(const int* hist, int nbins, int need, int* s_warp,
-                                                    int* s_digit, int* s_need, int* s_bcnt) {
-    const int tid = threadIdx.x, NT = blockDim.x, lane = tid & 31, warp = tid >> 5;
-    const int per_t = (nbins + NT - 1) / NT;  // bins per thread, descending from the top
-    int c = 0, h8[8];
-    const bool vec = per_t == 8 && nbins == 8 * NT;  // bins [nbins - 8(t+1), nbins - 8t), 2 x 16 B
-    if (vec) {
-        const int4* p = reinterpret_cast<const int4*>(hist + nbins - 8 * (tid + 1));
-        const int4 lo = p[0], hi = p[1];
-        h8[0] = hi.w; h8[1] = hi.z; h8[2] = hi.y; h8[3] = hi.x;
-        h8[4] = lo.w; h8[5] = lo.z; h8[6] = lo.y; h8[7] = lo.x;
-#pragma unroll
-        for (int k = 0; k < 8; ++k) c += h8[k];
-    } else {
-        for (int k = 0; k < per_t; ++k) {
-            const int d = nbins - 1 - (tid * per_t + k);
-            if (d >= 0) c += hist[d];
-        }
-    }
-    int incl = c;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-    }
-    if (lane == 31) s_warp[warp] = incl;
-    __syncthreads();
-    // totals of the warps before this one (a warp scan over the per-warp totals)
-    int wt = lane < (NT >> 5) ? s_warp[lane] : 0;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, wt, off);
-        if (lane >= off) wt += y;
-    }
-    const int base = __shfl_sync(0xffffffffu, wt, (warp + 31) & 31) * (warp > 0);
-    const int excl = base + incl - c;
-    if (excl < need && need <= excl + c) {
-        int acc = excl;
-        if (vec) {
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                if (acc < need && acc + h8[k] >= need) {
-                    *s_digit = nbins - 1 - (tid * 8 + k);
-                    *s_need = need - acc;
-                    *s_bcnt = h8[k];
-                }
-                acc += h8[k];
-            }
-        } else {
-            for (int k = 0; k < per_t; ++k) {
-                const int d = nbins - 1 - (tid * per_t + k);
-                if (d < 0) break;
-                const int cd = hist[d];
-                if (acc < need && acc + cd >= need) {
-                    *s_digit = d;
-                    *s_need = need - acc;
-                    *s_bcnt = cd;
-                }
-                acc += cd;
-            }
-        }
-    }
-    __syncthreads();
-}
-
-// The top-k's shared memory, declared by each selection kernel.
-struct TopkSmem {
-    int warp[32];
-    __align__(16) int hist[kHistBins];
-    int digit, need, bcnt, bn;
-    uint32_t kand[32], kor[32];                 // each warp's AND / OR of candidate keys
-    __align__(16) uint32_t bkey[kExactMax];     // 0 pads: below every real key
-    __align__(16) int bidx[kExactMax];
-};
-
-// Candidate blocks [init_end(nb), cand_end(nb)): neither init nor local.
-__device__ __forceinline__ int cand_begin(const SelectArgs& a, int nb) { return min(a.n_init, nb); }
-__device__ __forceinline__ int cand_end(const SelectArgs& a, int nb) {
-    return max(max(nb - a.n_local, 0), min(a.n_init, nb));
-}
-
-// Clears the first digit's bins and the exact bucket; a barrier must follow before topk_union.
-__device__ __forceinline__ void topk_prepare(TopkSmem& t) {
-    for (int i = threadIdx.x; i < kHistBins / 4; i += blockDim.x)
-        reinterpret_cast<int4*>(t.hist)[i] = make_int4(0, 0, 0, 0);
-    for (int i = threadIdx.x; i < kExactMax; i += blockDim.x) t.bkey[i] = 0u;
-    if (threadIdx.x == 0) t.bn = 0;
-}
-
-// Publishes a warp's AND / OR of the candidate keys it wrote (identity values when none).
-__device__ __forceinline__ void publish_andor(TopkSmem& t, uint32_t kand, uint32_t kor) {
-    kand = __reduce_and_sync(0xffffffffu, kand);
-    kor = __reduce_or_sync(0xffffffffu, kor);
-    if ((threadIdx.x & 31) == 0) {
-        t.kand[threadIdx.x >> 5] = kand;
-        t.kor[threadIdx.x >> 5] = kor;
-    }
-}
-
-// `andor_ready`: every warp has published the AND / OR of the candidate keys it wrote (then no
-// pass over the keys is needed for them). topk_prepare and a barrier come before the call.
-__device__ void topk_union(const SelectArgs& a, int pair, int nb, uint32_t* keys, TopkSmem& t,
-                           bool andor_ready) {
-    int* s_warp = t.warp;
-    int* hist = t.hist;
-    uint32_t* s_bkey = t.bkey;
-    int* s_bidx = t.bidx;
-    const int tid = threadIdx.x, NT = blockDim.x;
-    const int init_end = cand_begin(a, nb);
-    const int clo = init_end, chi = cand_end(a, nb);
-    const int ncand = chi - clo;
-    const int kk = min(a.top_k, ncand);
-    const bool take_all = (kk == ncand);
-    const int per = (ncand + NT - 1) / NT;  // contiguous segment of each thread
-    const int seg_lo = clo + tid * per, seg_hi = min(seg_lo + per, chi);
-    const bool in_regs = per <= kKeysPerThread;
-    uint32_t kr[kKeysPerThread];
-#pragma unroll
-    for (int e = 0; e < kKeysPerThread; ++e) kr[e] = (in_regs && seg_lo + e < seg_hi) ? keys[seg_lo + e] : 0u;
-
-    uint32_t thr = 0xffffffffu;  // keys > thr are taken, plus the first `need` keys == thr
-    int need = 0;
-    bool exact = false;
-    uint32_t emask = 0u, eprefix = 0u;
-    if (kk > 0 && !take_all) {
-        // bits that every candidate shares need no histogram pass (block-wide AND / OR)
-        if (!andor_ready) {
-            uint32_t kand = 0xffffffffu, kor = 0u;
-            if (in_regs) {
-#pragma unroll
-                for (int e = 0; e < kKeysPerThread; ++e) {
-                    if (seg_lo + e < seg_hi) {
-                        kand &= kr[e];
-                        kor |= kr[e];
-                    }
-                }
-            } else {
-                for (int i = seg_lo; i < seg_hi; ++i) {
-                    kand &= keys[i];
-                    kor |= keys[i];
-                }
-            }
-            publish_andor(t, kand, kor);
-            __syncthreads();
-        }
-        uint32_t kand = 0xffffffffu, kor = 0u;
-        for (int w = 0; w < (NT >> 5); ++w) {
-            kand &= t.kand[w];
-            kor |= t.kor[w];
-        }
-        const uint32_t diff = kand ^ kor;  // bits in which some candidates differ
-        uint32_t prefix = kand, mask = 0xffffffffu;
-        need = kk;
-        if (diff != 0u) {
-            int hi = 31 - __clz(diff);
-            mask = hi < 31 ? (0xffffffffu << (hi + 1)) : 0u;
-            prefix = kand & mask;
-            int width = min(kFirstDigitBits, hi + 1);
-            for (bool first = true;; first = false) {
-                const int shift = hi - width + 1;
-                const int nbins = 1 << width;
-                const uint32_t dmask = (uint32_t)nbins - 1u;
-                if (!first) {
-                    for (int i = tid; i < nbins; i += NT) hist[i] = 0;
-                    __syncthreads();
-                }
-                if (in_regs) {
-#pragma unroll
-                    for (int e = 0; e < kKeysPerThread; ++e)
-                        if (seg_lo + e < seg_hi && (kr[e] & mask) == prefix) atomicAdd(&hist[(kr[e] >> shift) & dmask], 1);
-                } else {
-                    for (int i = seg_lo; i < seg_hi; ++i) {
-                        const uint32_t u = keys[i];
-                        if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1);
-                    }
-                }
-                __syncthreads();
-                find_digit_from_top(hist, nbins, need, s_warp, &t.digit, &t.need, &t.bcnt);
-                prefix |= (uint32_t)t.digit << shift;
-                need = t.need;
-                mask |= dmask << shift;
-                if (shift == 0) break;  // every bit decided: the bucket's keys are all equal
-                if (in_regs && t.bcnt <= kExactMax) {
-                    exact = true;
-                    break;
-                }
-                __syncthreads();  // everyone has read the bins before they are cleared
-                hi = shift - 1;
-                width = min(8, hi + 1);
-            }
-        }
-        thr = prefix;
-        if (exact) {
-            emask = mask;
-            eprefix = prefix;
-        }
-    }
-
-    int32_t* out = a.block_idx + (size_t)pair * a.sel_cap;
-    if (in_regs) {
-        // taken flags of the thread's own candidates
-        bool fl[kKeysPerThread];
-        if (exact) {
-#pragma unroll
-            for (int e = 0; e < kKeysPerThread; ++e) {
-                if (seg_lo + e < seg_hi && (kr[e] & emask) == eprefix) {
-                    const int slot = atomicAdd(&t.bn, 1);
-                    s_bkey[slot] = kr[e];
-                    s_bidx[slot] = seg_lo + e;
-                }
-            }
-            __syncthreads();
-            const int ebn = t.bn;
-#pragma unroll
-            for (int e = 0; e < kKeysPerThread; ++e) {
-                fl[e] = false;
-                if (seg_lo + e < seg_hi) {
-                    const uint32_t u = kr[e], mk = u & emask;
-                    if (mk > eprefix) {
-                        fl[e] = true;
-                    } else if (mk == eprefix) {
-                        // four bucket entries per 16-byte read; the zero pads never count
-                        const int idx = seg_lo + e;
-                        const uint4* bk4 = reinterpret_cast<const uint4*>(s_bkey);
-                        const int4* bi4 = reinterpret_cast<const int4*>(s_bidx);
-                        int rank = 0;
-#pragma unroll 4
-                        for (int q = 0; q < (ebn + 3) / 4; ++q) {
-                            const uint4 kq = bk4[q];
-                            const int4 iq = bi4[q];
-                            rank += (kq.x > u || (kq.x == u && iq.x < idx)) + (kq.y > u || (kq.y == u && iq.y < idx)) +
-                                    (kq.z > u || (kq.z == u && iq.z < idx)) + (kq.w > u || (kq.w == u && iq.w < idx));
-                        }
-                        fl[e] = rank < need;
-                    }
-                }
-            }
-        } else if (take_all || kk == 0) {
-#pragma unroll
-            for (int e = 0; e < kKeysPerThread; ++e) fl[e] = take_all && seg_lo + e < seg_hi;
-        } else {
-            // keys above thr, and the first `need` keys equal to thr in block order
-            int cnt = 0;
-#pragma unroll
-            for (int e = 0; e < kKeysPerThread; ++e) cnt += (seg_lo + e < seg_hi && kr[e] == thr);
-            int tot;
-            int r = block_exclusive_scan(cnt, s_warp, &tot);
-#pragma unroll
-            for (int e = 0; e < kKeysPerThread; ++e) {
-                fl[e] = false;
-                if (seg_lo + e < seg_hi) {
-                    const uint32_t u = kr[e];
-                    fl[e] = u > thr || (u == thr && r < need);
-                    r += (u == thr);
-                }
-            }
-        }
-        // union: init blocks, the taken candidates in block order, then the local blocks
-        int cnt = 0;
-#pragma unroll
-        for (int e = 0; e < kKeysPerThread; ++e) cnt += fl[e];
-        int taken;
-        int pos = init_end + block_exclusive_scan(cnt, s_warp, &taken, false);
-#pragma unroll
-        for (int e = 0; e < kKeysPerThread; ++e)
-            if (fl[e]) out[pos++] = seg_lo + e;
-        for (int i = tid; i < init_end; i += NT) out[i] = i;
-        const int n_loc = nb - chi;
-        for (int i = tid; i < n_loc; i += NT) out[init_end + taken + i] = chi + i;
-        const int total = init_end + taken + n_loc;
-        for (int i = total + tid; i < a.sel_cap; i += NT) out[i] = -1;
-        if (tid == 0) a.n_sel[pair] = total;
-        return;
-    }
-
-    // streamed candidates: mark the taken ones in keys[] (1 / 0), ties at thr in block order
-    {
-        int cnt = 0;
-        for (int i = seg_lo; i < seg_hi; ++i) cnt += (keys[i] == thr);
-        int tot;
-        int r = block_exclusive_scan(cnt, s_warp, &tot);
-        for (int i = seg_lo; i < seg_hi; ++i) {
-            const uint32_t u = keys[i];
-            const bool take = kk > 0 && (take_all || u > thr || (u == thr && r < need));
-            r += (u == thr);
-            keys[i] = take ? 1u : 0u;
-        }
-    }
-    __syncthreads();
-    // union with init and local blocks, emitted in ascending block order
-    {
-        const int per2 = (nb + NT - 1) / NT;
-        const int lo = tid * per2, hi = min(lo + per2, nb);
-        int cnt = 0;
-        for (int i = lo; i < hi; ++i) cnt += (i < init_end || i >= chi || keys[i] != 0u);
-        int total;
-        int pos = block_exclusive_scan(cnt, s_warp, &total);
-        for (int i = lo; i < hi; ++i)
-            if (i < init_end || i >= chi || keys[i] != 0u) out[pos++] = i;
-        for (int i = total + tid; i < a.sel_cap; i += NT) out[i] = -1;
-        if (tid == 0) a.n_sel[pair] = total;
-    }
-}
 
 // grid = pairs * parts. Part p of a pair scores windows [p*PW, p*PW + PW) and owns the blocks whose
 // first overlapping window falls in that range (the last part with windows also owns the blocks
@@ -868,9 +504,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_kernel(SelectArgs a)
     if (!s_last) return;
     __threadfence();
     for (int64_t b = tid; b < nb; b += kSelectThreads) s_dyn[b] = order_key(ld_cg(bs + b));
-    topk_prepare(tk);
+    const Grp cta{(int)threadIdx.x, (int)blockDim.x, 0};
+    topk_prepare(tk, cta);
     __syncthreads();
-    topk_union(a, pair, (int)nb, s_dyn, tk, false);
+    topk_union(a, (int)nb, s_dyn, tk, false, cta, a.block_idx + (size_t)pair * a.sel_cap, a.n_sel + pair);
 }
 
 // One CTA per pair, when there are enough pairs to fill the GPU: the pair's stored e rows stream
@@ -959,6 +596,10 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
                 const float so = __shfl_xor_sync(0xffffffffu, sum, off);
                 online_merge(m, sum, mo, so);
             }
+            // the lanes' merges round in different orders: every lane takes lane 0's (M, Z), as
+            // the multi-part kernel does
+            m = __shfl_sync(0xffffffffu, m, 0);
+            sum = __shfl_sync(0xffffffffu, sum, 0);
             const float iz = sum > 0.f ? 1.f / sum : 0.f;
 #pragma unroll
             for (int u = 0; u < kStatU; ++u)
@@ -989,11 +630,7 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
                 x[4 * q + 3] = t.w;
             }
         }
-        float acc = 0.f;
-#pragma unroll
-        for (int h = 0; h < GP; ++h)
-            if (h < a.G) acc += x[h] * w[h];
-        return acc;
+        return group_sum<GP>(x, w, a.G);
     };
     // blocks start on window boundaries: block b's windows are [rb - (L - 1), rb + r - 1], with
     // r = BS / s a power of two up to 32 and L = l / s in {1, 2}
@@ -1028,10 +665,8 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
                 if constexpr (GP == 4) {
                     const float4 e = reinterpret_cast<const float4*>(ring)[jj];
                     const float4 w = reinterpret_cast<const float4*>(wt)[jj >> 6];
-                    v = e.x * w.x;
-                    if (a.G > 1) v += e.y * w.y;
-                    if (a.G > 2) v += e.z * w.z;
-                    if (a.G > 3) v += e.w * w.w;
+                    const float ev[4] = {e.x, e.y, e.z, e.w}, wv[4] = {w.x, w.y, w.z, w.w};
+                    v = group_sum<4>(ev, wv, a.G);
                 } else {
                     v = window_score(0, jj, jj);
                 }
@@ -1121,10 +756,11 @@ __global__ void __launch_bounds__(kSelectThreads, 1) select_single_kernel(Select
     if (a.block_scores)
         for (int64_t b = nb + tid; b < a.nb_cap; b += kSelectThreads)
             a.block_scores[(size_t)pair * a.nb_cap + b] = -INFINITY;
-    publish_andor(tk, kand, kor);
-    topk_prepare(tk);
+    const Grp cta{(int)threadIdx.x, (int)blockDim.x, 0};
+    publish_andor(tk, kand, kor, cta);
+    topk_prepare(tk, cta);
     __syncthreads();
-    topk_union(a, pair, nb, keys, tk, true);
+    topk_union(a, nb, keys, tk, true, cta, a.block_idx + (size_t)pair * a.sel_cap, a.n_sel + pair);
 }
 
 int sm_count() {

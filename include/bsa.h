@@ -249,9 +249,12 @@ bsa_status_t bsa_read_device_error(void* workspace, size_t workspace_bytes, uint
  * Scratch: the split partials and per-pair completion counters live in a fixed array inside
  * libbsa, BSA_NOALLOC_SCRATCH_BYTES per device.
  *   - Size limit. A parameter set whose partials do not fit returns BSA_ERR_WORKSPACE before any
- *     CUDA call and launches nothing. The partials need about
- *     B*Hkv*num_layers*Gp*(d + 2)*4 bytes per partial slot, where Gp is G rounded up to a power
- *     of two. For example, B=16, Hkv=8, G=4, d=128 with 69 selected blocks needs 1.3 MiB.
+ *     CUDA call and launches nothing. The call attends one layer, so params->num_layers plays no
+ *     part in the size: the partials need about B*Hkv*Gp*(d + 2)*4 bytes per partial slot, where
+ *     Gp is G rounded up to a power of two. For example, B=16, Hkv=8, G=4, d=128 with 69 selected
+ *     blocks needs 1.3 MiB.
+ *   - Device. The scratch used is the current device's, so `stream` must belong to the current
+ *     device (or be a default stream); a stream of another device is BSA_ERR_INVALID_ARG.
  *   - First call on a device. It looks up the array's device address (cudaGetSymbolAddress), with
  *     that device current. The lookup may load the library's device code. Make the first call on
  *     each device outside any stream capture.

@@ -34,10 +34,15 @@ def test_noalloc_matches_workspace_decode(name, cuda_device):
     err = torch.zeros(1, dtype=torch.int32, device=cuda_device)
     outs = [torch.full_like(ref_out, 77.0) for _ in range(2)]
     lses = [torch.full_like(ref_lse, 77.0) for _ in range(2)]
-    # two calls in a row on the stream, no host sync between them; the second reports no errors
+    # two calls in a row on the stream, no host sync between them; the second reports no errors.
+    # The second call's parameters name four layers: the call attends one, and its scratch is
+    # sized for one (at 128K x 16, four layers' partials would not fit the scratch).
+    p4 = bsa.make_params(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, run.T_cap, w.dtype,
+                         w.n_init, w.n_local, w.top_k, w.cmp_kernel, w.cmp_stride, w.block_size,
+                         num_layers=4)
     for i in range(2):
-        bsa.bsa_sparse_decode_noalloc(run.p, run.q[0], d["k"][0], d["v"][0], d["seq_lens"],
-                                      run.block_idx, run.n_sel, outs[i], lses[i],
+        bsa.bsa_sparse_decode_noalloc(run.p if i == 0 else p4, run.q[0], d["k"][0], d["v"][0],
+                                      d["seq_lens"], run.block_idx, run.n_sel, outs[i], lses[i],
                                       device_error=err if i == 0 else None)
     torch.cuda.synchronize()
     assert int(err.item()) == 0
@@ -63,3 +68,19 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     st = bsa.lib().bsa_sparse_decode_noalloc(ctypes.byref(p), ctypes.c_void_p(0x10002), A, A, A,
                                              A, A, A, None, None, ctypes.c_void_p(0))
     assert st == bsa.BSA_ERR_INVALID_ARG
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="host-side check with fake device addresses")
+def test_noalloc_scratch_is_sized_for_one_layer():
+    """The call attends one layer: a parameter set naming more layers is not refused for the size
+    of partials it will never write. (On a machine without a GPU the call then stops at its first
+    CUDA call, which is all this host-side check needs.)"""
+    bsa.lib()
+    w = WORKLOADS["gqa4-bf16-128k-b16"]  # 1.3 MiB of partials for one layer, 5.3 MiB for four
+    A = ctypes.c_void_p(0x10000)
+    for layers in (1, 4, 16):
+        p = bsa.make_params(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.seq_len, w.dtype,
+                            w.n_init, w.n_local, w.top_k, num_layers=layers)
+        st = bsa.lib().bsa_sparse_decode_noalloc(ctypes.byref(p), A, A, A, A, A, A, A, None, None,
+                                                 ctypes.c_void_p(0))
+        assert st not in (bsa.BSA_OK, bsa.BSA_ERR_WORKSPACE), (layers, st)
