@@ -139,22 +139,20 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
         if (P.dtype == BSA_BF16 && (int64_t)P.pairs * P.T_cap > 0x7fffffffLL)
             return BSA_ERR_UNSUPPORTED;
     }
-    // Fused step (bf16): blocks start on window boundaries (BS / s a power of two up to 32, l / s
-    // 1 or 2, BS a multiple of the 64-token attention unit), the pair's window terms fit tensor
-    // memory (512 columns: 4 chunks of 64 windows per 2 * Gp columns, plus the slack of one
-    // block-maximum load of up to 4 chunks) and the rest fits one CTA.
+    // Fused step (bf16): blocks of four windows (BS = 4s, l = s or 2s; the paper's 64 / 16 / 32),
+    // BS a multiple of the 64-token attention unit, the pair's window terms in tensor memory (512
+    // columns: tiles of 32 blocks, four per 4 * Gp columns, plus the slack of one block-maximum load
+    // of up to two tiles) and the rest in one CTA.
     {
         P.step_fused = 0;
-        const int r_w = P.s > 0 ? P.BS / P.s : 0;
-        const bool geo = P.BS % P.s == 0 && P.l % P.s == 0 && r_w >= 1 && r_w <= 32 &&
-                         (r_w & (r_w - 1)) == 0 && (P.l / P.s == 1 || P.l / P.s == 2) && P.BS % 64 == 0;
+        const bool geo = P.BS == 4 * P.s && (P.l == P.s || P.l == 2 * P.s) && P.BS % 64 == 0;
         if (P.dtype == BSA_BF16 && geo && P.nc_cap > 0 && P.nb_cap <= 16384) {
             P.step_sgp = P.Gp;
             P.step_nch_cap = (int)((P.nc_cap + 63) / 64);
-            const int64_t nbc_cap = (P.nb_cap * r_w + 63) / 64;  // chunks holding block starts
-            const int64_t chunk_cols = (nbc_cap > P.step_nch_cap ? nbc_cap : P.step_nch_cap);
-            const int per_load = 16 / P.Gp < 4 ? 16 / P.Gp : 4;
-            const int64_t cols = ((chunk_cols + 3) / 4 + per_load) * 2 * P.Gp;
+            const int64_t tiles = (P.step_nch_cap + 1) / 2;
+            const int64_t block_tiles = (P.nb_cap + 31) / 32;
+            const int64_t t_max = tiles > block_tiles ? tiles : block_tiles;
+            const int64_t cols = ((t_max + 3) / 4 + 2) * 4 * P.Gp;
             uint32_t tc = 32;
             while ((int64_t)tc < cols) tc <<= 1;
             P.step_key_words = (int)((P.nb_cap + 3) / 4 * 4);

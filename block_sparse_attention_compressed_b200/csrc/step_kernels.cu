@@ -20,11 +20,11 @@
 // no combine pass.
 //
 // Stage bookkeeping: a global stage counter k runs over the CTA's lifetime on every warp; stage k
-// uses slot k % 8 and is issued by producer k % 2. Scoring stage k is consumed by warp k % 8 (its
-// TMEM lane quarter is k % 4, the chunk's); attention unit i of a pair (stages kd + 2i for K and
-// kd + 2i + 1 for V) by the four warps of group i % 2, 16 tokens each. Slots therefore have one
-// consumer per phase, and a CTA-wide barrier separates the phases, so no warp waits on a slot two
-// phases ahead of its last use.
+// uses slot k % 8 and is issued by producer k % 2. Chunk c of a pair (stage k0 + c) is scored by
+// warp (c / 2) % 4 + 4 (c % 2): the two warps of TMEM lane quarter (c / 2) % 4 write the tile of
+// chunks 2p, 2p + 1 there, one block per lane; attention unit i (stages kd + 2i for K and kd + 2i + 1 for V) is consumed by the four
+// warps of group i % 2, 16 tokens each. Slots therefore have one consumer per phase, and a CTA-wide
+// barrier separates the phases, so no warp waits on a slot two phases ahead of its last use.
 #include "bsa_internal.cuh"
 #include "tiles.cuh"
 #include "topk.cuh"
@@ -33,6 +33,7 @@ namespace bsa {
 namespace {
 
 constexpr int kStepConsumers = 8;
+constexpr int kStepScorers = 4;  // TMEM lane quarters: tile p of a pair goes to quarter p % 4
 constexpr int kStepProducers = 2;
 constexpr int kStepThreads = (kStepConsumers + kStepProducers) * 32;
 constexpr int kStepSlots = 8;
@@ -42,8 +43,9 @@ constexpr uint32_t kBox = 64 * 128;             // one 64-row, 64-column box (co
 constexpr uint32_t kEmptyCount = 4;             // arrivals that free a slot: an attention unit's warps
 constexpr int kConsumerBar = 1;               // named barrier of the consumer warps
 constexpr int kHandBar = 2;                   // consumers + producers: the selection is handed over
+constexpr int kPairBar0 = 3;                  // 3..6: the two scoring warps of a TMEM lane quarter
 constexpr uint32_t kStepWaitPolls = 1u << 26;
-static_assert(kStepSlots % kStepConsumers == 0, "a scoring slot serves one consumer warp");
+static_assert(kStepSlots % (2 * kStepScorers) == 0, "a scoring slot serves one consumer warp");
 static_assert(kStepSlots % 4 == 0, "an attention slot serves one group of four warps");
 static_assert(kStepSlots % kStepProducers == 0, "a slot is refilled by one producer");
 
@@ -114,7 +116,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     float* lastE = reinterpret_cast<float*>(p);
     p += (size_t)a.nch_cap * SGP * sizeof(float);
     float* staging = reinterpret_cast<float*>(p);
-    p += (size_t)kStepConsumers * 64 * SGP * sizeof(float);
+    p += (size_t)kStepScorers * 2 * 128 * SGP * sizeof(float);
     int32_t* sel = reinterpret_cast<int32_t*>(p);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -229,7 +231,6 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         const Grp grp{(int)threadIdx.x, kStepConsumers * 32, kConsumerBar};
         const int g = lane >> 2, tq = lane & 3;
         const int GS = RAW ? 1 : a.G;  // scoring heads
-        float* stg = staging + w * 64 * SGP;
         const uint32_t tq_addr = tbase + ((32u * (uint32_t)(w & 3)) << 16);  // this warp's TMEM lanes
         SelectArgs sa;
         memset(&sa, 0, sizeof sa);
@@ -237,8 +238,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
         sa.n_local = a.n_local;
         sa.top_k = a.top_k;
         sa.sel_cap = a.sel_cap;
-        const int r_w = a.BS / a.s, L_w = a.l / a.s;
-        const int lsh = __ffs(r_w) - 1;
+        const int L_w = a.l / a.s;  // windows of one block: BS = 4s, l = s or 2s
         // waits for stage kk's data; after a wait that runs out the CTA finishes without waiting
         auto await_stage = [&](int64_t kk) -> int {
             const int slot = (int)(kk % kStepSlots);
@@ -265,97 +265,102 @@ __global__ void __launch_bounds__(kStepThreads, 1)
             // scoring B operand: the group's query heads, or the Forecast vector
             const uint32_t(&qs)[KS][2] = *reinterpret_cast<const uint32_t(*)[KS][2]>(RAW ? &qf_raw[0][0] : &qa[0][0]);
 
-            // ---- scoring: chunks w, w + 8, ... of the pair
+            topk_prepare(tk, grp);  // the top-k's bins, cleared while the first chunks load
+            // ---- scoring: tiles of two 64-window chunks. Chunk 2p of tile p is scored by warp p % 4 and
+            // chunk 2p + 1 by warp p % 4 + 4, the two warps of TMEM lane quarter p % 4; they meet at a
+            // named barrier and the first stores the tile, one block per lane: lane i holds block
+            // 32p + i, its four windows 128p + 4i .. + 3 with every head (4 * SGP columns).
             const bool h0 = 2 * tq < GS, h1 = 2 * tq + 1 < GS;
-            for (int c = w; c < pg.nch; c += kStepConsumers) {
-                const int slot = await_stage(k + c);
-                float cc[4][4];
-                score_chunk<D>(ring + (size_t)slot * kSlotBytes, qs, cc, lane);
-                __syncwarp();
-                if (lane == 0) mbar_arrive_cnt(&empty[slot], kEmptyCount);  // one warp stands for four
-                const int nrows = min(64, pg.nc - 64 * c);
-                float x[4][4];
+            const int qd = w & 3, half = w >> 2;
+            for (int p = qd; 2 * p < pg.nch; p += kStepScorers) {
+                float* stg = staging + (qd * 2 + ((p / kStepScorers) & 1)) * 128 * SGP;  // double-buffered
+                const int c = 2 * p + half;
+                if (c < pg.nch) {
+                    const int slot = await_stage(k + c);
+                    float cc[4][4];
+                    score_chunk<D>(ring + (size_t)slot * kSlotBytes, qs, cc, lane);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive_cnt(&empty[slot], kEmptyCount);  // one warp stands for four
+                    const int nrows = min(64, pg.nc - 64 * c);
+                    float x[4][4];
 #pragma unroll
-                for (int r = 0; r < 4; ++r)
+                    for (int r = 0; r < 4; ++r)
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) x[r][e] = __fmul_rn(cc[r][e], a.score_log2);  // rounded here in every kernel
-                if constexpr (!RAW) {
-                    // the chunk's maximum per head, then e = exp2(x - max) and its sum
-                    float m0 = -INFINITY, m1 = -INFINITY;
+                        for (int e = 0; e < 4; ++e) x[r][e] = __fmul_rn(cc[r][e], a.score_log2);  // rounded here in every kernel
+                    if constexpr (!RAW) {
+                        // the chunk's maximum per head, then e = exp2(x - max) and its sum
+                        float m0 = -INFINITY, m1 = -INFINITY;
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            if (16 * r + g < nrows) {
+                                m0 = fmaxf(m0, x[r][0]);
+                                m1 = fmaxf(m1, x[r][1]);
+                            }
+                            if (16 * r + g + 8 < nrows) {
+                                m0 = fmaxf(m0, x[r][2]);
+                                m1 = fmaxf(m1, x[r][3]);
+                            }
+                        }
+#pragma unroll
+                        for (int off = 4; off < 32; off <<= 1) {
+                            m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
+                            m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
+                        }
+                        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const int lra = 16 * r + g, lrb = lra + 8;
+                            if (lra < nrows) {
+                                x[r][0] = exp2f(x[r][0] - m0);
+                                x[r][1] = exp2f(x[r][1] - m1);
+                                s0 += x[r][0];
+                                s1 += x[r][1];
+                            } else {
+                                x[r][0] = x[r][1] = 0.f;
+                            }
+                            if (lrb < nrows) {
+                                x[r][2] = exp2f(x[r][2] - m0);
+                                x[r][3] = exp2f(x[r][3] - m1);
+                                s0 += x[r][2];
+                                s1 += x[r][3];
+                            } else {
+                                x[r][2] = x[r][3] = 0.f;
+                            }
+                        }
+#pragma unroll
+                        for (int off = 4; off < 32; off <<= 1) {
+                            s0 += __shfl_xor_sync(0xffffffffu, s0, off);
+                            s1 += __shfl_xor_sync(0xffffffffu, s1, off);
+                        }
+                        if (g == 0) {
+                            if (h0) stats[c * SGP + 2 * tq] = make_float2(m0, s0);
+                            if (h1) stats[c * SGP + 2 * tq + 1] = make_float2(m1, s1);
+                        }
+                    }
+                    // the chunk's rows into the tile's staging rows 64 * half ..
 #pragma unroll
                     for (int r = 0; r < 4; ++r) {
-                        if (16 * r + g < nrows) {
-                            m0 = fmaxf(m0, x[r][0]);
-                            m1 = fmaxf(m1, x[r][1]);
+                        const int lra = 64 * half + 16 * r + g, lrb = lra + 8;
+                        if (2 * tq < SGP) {
+                            stg[lra * SGP + 2 * tq] = x[r][0];
+                            stg[lrb * SGP + 2 * tq] = x[r][2];
                         }
-                        if (16 * r + g + 8 < nrows) {
-                            m0 = fmaxf(m0, x[r][2]);
-                            m1 = fmaxf(m1, x[r][3]);
-                        }
-                    }
-#pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
-                        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
-                    }
-                    float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const int lra = 16 * r + g, lrb = lra + 8;
-                        if (lra < nrows) {
-                            x[r][0] = exp2f(x[r][0] - m0);
-                            x[r][1] = exp2f(x[r][1] - m1);
-                            s0 += x[r][0];
-                            s1 += x[r][1];
-                        } else {
-                            x[r][0] = x[r][1] = 0.f;
-                        }
-                        if (lrb < nrows) {
-                            x[r][2] = exp2f(x[r][2] - m0);
-                            x[r][3] = exp2f(x[r][3] - m1);
-                            s0 += x[r][2];
-                            s1 += x[r][3];
-                        } else {
-                            x[r][2] = x[r][3] = 0.f;
+                        if (2 * tq + 1 < SGP) {
+                            stg[lra * SGP + 2 * tq + 1] = x[r][1];
+                            stg[lrb * SGP + 2 * tq + 1] = x[r][3];
                         }
                     }
-#pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        s0 += __shfl_xor_sync(0xffffffffu, s0, off);
-                        s1 += __shfl_xor_sync(0xffffffffu, s1, off);
-                    }
-                    if (g == 0) {
-                        if (h0) stats[c * SGP + 2 * tq] = make_float2(m0, s0);
-                        if (h1) stats[c * SGP + 2 * tq + 1] = make_float2(m1, s1);
-                    }
+                    __syncwarp();
+                    if (lane < SGP) lastE[c * SGP + lane] = stg[(64 * half + 63) * SGP + lane];
                 }
-                // rows into TMEM lanes: through a per-warp staging tile, lane i takes windows
-                // 64c + i and 64c + 32 + i with all their heads
+                asm volatile("bar.sync %0, %1;" ::"r"(kPairBar0 + qd), "r"(64) : "memory");
+                if (half == 0) {
+                    // lane i: rows 4i .. 4i + 3 of the tile (block 32p + i), all heads
+                    float v[4 * SGP];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) {
-                    const int lra = 16 * r + g, lrb = lra + 8;
-                    if (2 * tq < SGP) {
-                        stg[lra * SGP + 2 * tq] = x[r][0];
-                        stg[lrb * SGP + 2 * tq] = x[r][2];
-                    }
-                    if (2 * tq + 1 < SGP) {
-                        stg[lra * SGP + 2 * tq + 1] = x[r][1];
-                        stg[lrb * SGP + 2 * tq + 1] = x[r][3];
-                    }
+                    for (int e = 0; e < 4 * SGP; ++e) v[e] = stg[4 * lane * SGP + e];
+                    tmem_st<4 * SGP>(tq_addr + (uint32_t)((p / kStepScorers) * 4 * SGP), v);
                 }
-                __syncwarp();
-                float v[2 * SGP];
-#pragma unroll
-                for (int h = 0; h < SGP; ++h) {
-                    v[h] = stg[lane * SGP + h];
-                    v[SGP + h] = stg[(32 + lane) * SGP + h];
-                }
-                tmem_st<2 * SGP>(tq_addr + (uint32_t)((c >> 2) * 2 * SGP), v);
-                if (lane == 31) {
-#pragma unroll
-                    for (int h = 0; h < SGP; ++h) lastE[c * SGP + h] = v[SGP + h];
-                }
-                __syncwarp();
             }
             k += pg.nch;
             tmem_wait_st();
@@ -390,64 +395,57 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                 for (int c = grp.tid; c < pg.nch; c += grp.nt) wt[c] = 1.f;
             }
             grp.sync();
-            // block b's windows are [b*r - (L - 1), b*r + r - 1] (r = BS / s, L = l / s): lane i of a
-            // 32-window tile holds window 32t + i, the maxima run over groups of r lanes, plus the
-            // window before the group when L = 2
+            // block maxima, one block per lane: tile p of quarter p % 4 (warps w and w + 4 split the
+            // quarter's tiles, TB tiles per TMEM load). Block b = 32p + i covers windows 4b .. 4b + 3,
+            // and 4b - 1 when l = 2s: the previous lane's last window (lane 0: the previous tile's,
+            // from the chunk's last terms).
             uint32_t kand = 0xffffffffu, kor = 0u;
-            // chunks c = q + 4i of TMEM lane quarter q: warp w takes the first half of them, w + 4
-            // the second, CPL chunks (LW columns) per load, their maxima chains side by side
-            constexpr int CPL = 32 / (2 * SGP) < 2 ? 32 / (2 * SGP) : 2;
-            constexpr int LW = CPL * 2 * SGP;
-            const int nbc = (int)(((int64_t)pg.nb * r_w + 63) / 64);  // chunks holding block starts
+            constexpr int TB = 32 / (4 * SGP) < 2 ? 1 : 2;
+            constexpr int LW = TB * 4 * SGP;
+            const int nbt = (pg.nb + 31) / 32;  // tiles holding blocks
             const int qq = w & 3;
-            const int nq = nbc > qq ? (nbc - qq + 3) / 4 : 0;
+            const int nq = nbt > qq ? (nbt - qq + 3) / 4 : 0;
             const int i_lo = w < 4 ? 0 : (nq + 1) / 2, i_hi = w < 4 ? (nq + 1) / 2 : nq;
-            for (int i0 = i_lo; i0 < i_hi; i0 += CPL) {
+            for (int i0 = i_lo; i0 < i_hi; i0 += TB) {
                 float v[LW];
-                if (qq + 4 * i0 < pg.nch) {
-                    tmem_ld<LW>(tq_addr + (uint32_t)(i0 * 2 * SGP), v);
+                if (2 * (qq + 4 * i0) < pg.nch) {
+                    tmem_ld<LW>(tq_addr + (uint32_t)(i0 * 4 * SGP), v);
                     tmem_wait_ld();
                 }
-                float cur[2 * CPL], m[2 * CPL], sp[CPL];
 #pragma unroll
-                for (int u = 0; u < CPL; ++u) {
-                    const int c = qq + 4 * (i0 + u);
-                    cur[2 * u] = cur[2 * u + 1] = sp[u] = -INFINITY;
-                    if (i0 + u < i_hi && c < pg.nch) {
-                        const float* wc = wt + c * SGP;
-                        if (64 * c + lane < pg.nc) cur[2 * u] = group_sum<SGP>(v + u * 2 * SGP, wc, GS);
-                        if (64 * c + 32 + lane < pg.nc) cur[2 * u + 1] = group_sum<SGP>(v + u * 2 * SGP + SGP, wc, GS);
+                for (int u = 0; u < TB; ++u) {
+                    if (i0 + u >= i_hi) break;
+                    const int p = qq + 4 * (i0 + u);
+                    const int j0 = 128 * p + 4 * lane;  // the lane's first window
+                    float mx = -INFINITY, last = -INFINITY;
+                    if (j0 < pg.nc) {
+                        float wc[SGP];  // the chunk's weights, loaded once
+#pragma unroll
+                        for (int h = 0; h < SGP; ++h) wc[h] = wt[(j0 >> 6) * SGP + h];
+#pragma unroll
+                        for (int jj = 0; jj < 4; ++jj) {
+                            const float sv = j0 + jj < pg.nc ? group_sum<SGP>(v + u * 4 * SGP + jj * SGP, wc, GS) : -INFINITY;
+                            mx = fmaxf(mx, sv);
+                            if (jj == 3) last = sv;
+                        }
                     }
-                    // window 64c - 1, the last of the previous chunk (another quarter's)
-                    if (L_w == 2 && i0 + u < i_hi && c > 0 && 64 * c - 1 < pg.nc)
-                        sp[u] = group_sum<SGP>(lastE + (c - 1) * SGP, wt + (c - 1) * SGP, GS);
-                }
-#pragma unroll
-                for (int t = 0; t < 2 * CPL; ++t) m[t] = cur[t];
-                for (int off = 1; off < r_w; off <<= 1) {
-#pragma unroll
-                    for (int t = 0; t < 2 * CPL; ++t) m[t] = fmaxf(m[t], __shfl_down_sync(0xffffffffu, m[t], off));
-                }
-                if (L_w == 2) {
-#pragma unroll
-                    for (int t = 0; t < 2 * CPL; ++t) {
-                        const float before = __shfl_up_sync(0xffffffffu, cur[t], 1);
-                        const float last_prev = (t & 1) ? __shfl_sync(0xffffffffu, cur[t - 1 + ((t & 1) ^ 1)], 31) : sp[t >> 1];
-                        m[t] = fmaxf(m[t], lane == 0 ? last_prev : before);
+                    if (L_w == 2) {
+                        float prev = __shfl_up_sync(0xffffffffu, last, 1);
+                        if (lane == 0)
+                            prev = p > 0 && 128 * p - 1 < pg.nc
+                                       ? group_sum<SGP>(lastE + (2 * p - 1) * SGP, wt + (2 * p - 1) * SGP, GS)
+                                       : -INFINITY;
+                        mx = fmaxf(mx, prev);
                     }
-                }
-#pragma unroll
-                for (int t = 0; t < 2 * CPL; ++t) {
-                    const int c = qq + 4 * (i0 + (t >> 1));
-                    const int blk = (64 * c + 32 * (t & 1) + lane) >> lsh;
-                    if (i0 + (t >> 1) < i_hi && (lane & (r_w - 1)) == 0 && blk < pg.nb) {
-                        const uint32_t key = order_key(m[t]);
+                    const int blk = 32 * p + lane;
+                    if (blk < pg.nb) {
+                        const uint32_t key = order_key(mx);
                         keys[blk] = key;
                         if (blk >= pg.init_end && blk < pg.chi) {
                             kand &= key;
                             kor |= key;
                         }
-                        if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + blk] = m[t];
+                        if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + blk] = mx;
                     }
                 }
             }
@@ -455,7 +453,6 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                 for (int64_t blk = pg.nb + grp.tid; blk < a.nb_cap; blk += grp.nt)
                     a.block_scores[(size_t)pair * a.nb_cap + blk] = -INFINITY;
             publish_andor(tk, kand, kor, grp);
-            topk_prepare(tk, grp);
             grp.sync();
             topk_union(sa, pg.nb, keys, tk, true, grp, sel, &s_nsel);
             grp.sync();
@@ -586,7 +583,7 @@ size_t step_smem_bytes(int D, int sgp, int G, int nch_cap, int key_words, int se
     const size_t region = keys_bytes > merge_bytes ? keys_bytes : merge_bytes;
     size_t bytes = 1024 + (size_t)kStepSlots * kSlotBytes + ((region + 15) & ~size_t(15));
     bytes += (size_t)nch_cap * sgp * (sizeof(float2) + 2 * sizeof(float));
-    bytes += (size_t)kStepConsumers * 64 * sgp * sizeof(float);
+    bytes += (size_t)kStepScorers * 2 * 128 * sgp * sizeof(float);
     bytes += (size_t)sel_cap * sizeof(int32_t);
     // the static part (ring barriers, stage records, top-k scratch) shares the 227 KB of a CTA
     const size_t limit = 227 * 1024 - sizeof(TopkSmem) - 1024;

@@ -61,15 +61,26 @@ __device__ __forceinline__ void find_digit_from_top(const int* hist, int nbins, 
                                                     int* s_digit, int* s_need, int* s_bcnt, const Grp& gp) {
     const int tid = gp.tid, NT = gp.nt, lane = tid & 31, warp = tid >> 5;
     const int per_t = (nbins + NT - 1) / NT;  // bins per thread, descending from the top
-    int c = 0, h8[8];
-    const bool vec = per_t == 8 && nbins == 8 * NT;  // bins [nbins - 8(t+1), nbins - 8t), 2 x 16 B
+    int c = 0, h8[16];
+    // 8 or 16 bins per thread: bins [nbins - P(t+1), nbins - Pt) in 16-byte loads, top bin first
+    const int P = (per_t == 16 && nbins == 16 * NT) ? 16 : ((per_t == 8 && nbins == 8 * NT) ? 8 : 0);
+    const bool vec = P != 0;
     if (vec) {
-        const int4* p = reinterpret_cast<const int4*>(hist + nbins - 8 * (tid + 1));
-        const int4 lo = p[0], hi = p[1];
-        h8[0] = hi.w; h8[1] = hi.z; h8[2] = hi.y; h8[3] = hi.x;
-        h8[4] = lo.w; h8[5] = lo.z; h8[6] = lo.y; h8[7] = lo.x;
+        const int4* p = reinterpret_cast<const int4*>(hist + nbins - P * (tid + 1));
 #pragma unroll
-        for (int k = 0; k < 8; ++k) c += h8[k];
+        for (int q = 0; q < 4; ++q) {
+            if (q < P / 4) {
+                const int4 v = p[P / 4 - 1 - q];
+                h8[4 * q] = v.w;
+                h8[4 * q + 1] = v.z;
+                h8[4 * q + 2] = v.y;
+                h8[4 * q + 3] = v.x;
+            } else {
+                h8[4 * q] = h8[4 * q + 1] = h8[4 * q + 2] = h8[4 * q + 3] = 0;
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) c += h8[k];
     } else {
         for (int k = 0; k < per_t; ++k) {
             const int d = nbins - 1 - (tid * per_t + k);
@@ -104,9 +115,9 @@ __device__ __forceinline__ void find_digit_from_top(const int* hist, int nbins, 
         int acc = excl;
         if (vec) {
 #pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                if (acc < need && acc + h8[k] >= need) {
-                    *s_digit = nbins - 1 - (tid * 8 + k);
+            for (int k = 0; k < 16; ++k) {
+                if (k < P && acc < need && acc + h8[k] >= need) {
+                    *s_digit = nbins - 1 - (tid * P + k);
                     *s_need = need - acc;
                     *s_bcnt = h8[k];
                 }

@@ -1,12 +1,14 @@
 """The fused decode step, vs the CPU oracle, through the C ABI.
 
-For bf16 caches bsa_decode_step runs one kernel in which a CTA takes a whole (batch, kv-head) pair:
-it scores the pair's compressed keys (window terms kept in tensor memory), selects its blocks and
-attends them. These cases cover the shapes that kernel handles: every padded group size, both head
-dims, block sizes 32..256 with windows of one or two strides, ragged lengths (down to no window and
-an empty sequence), last blocks cut inside either 32-token half, more pairs than SMs (the persistent
-loop over pairs) and the selection edge cases (top-k covering every candidate, k = 0, no init or
-local blocks).
+For bf16 caches whose blocks are four windows long (BS = 4s, l = s or 2s, BS a multiple of 64; the
+paper's 64 / 16 / 32), bsa_decode_step runs one kernel in which a CTA takes a whole (batch, kv-head)
+pair: it scores the pair's compressed keys (window terms kept in tensor memory), selects its blocks
+and attends them. Other geometries chain the separate kernels behind the same entry point. These
+cases cover every padded group size, both head dims, both window lengths, blocks of 64 and 128
+tokens, ragged lengths (down to no window and an empty sequence), last blocks cut inside either
+32-token half, more pairs than SMs (the persistent loop over pairs) and the selection edge cases
+(top-k covering every candidate, k = 0, no init or local blocks), plus geometries of the chained
+path.
 """
 import numpy as np
 import pytest
@@ -31,6 +33,8 @@ STEP = {
                                        top_k=10, needles=3), None),
     "g4-bs128": (BASE.replace(name="x", batch=1, seq_len=5000, block_size=128, top_k=7, needles=2),
                  None),
+    "g4-bs128-l64s32": (BASE.replace(name="x", batch=2, seq_len=7000 + 45, block_size=128,
+                                     cmp_kernel=64, cmp_stride=32, top_k=6, needles=2), None),
     "g4-bs256-l32s16": (BASE.replace(name="x", batch=2, seq_len=9000, block_size=256, top_k=5,
                                      needles=2), None),
     "g4-l16s16": (BASE.replace(name="x", batch=2, seq_len=6100, cmp_kernel=16, cmp_stride=16,
@@ -74,7 +78,8 @@ def test_step_matches_oracle(case, cuda_device):
 
 
 @pytest.mark.parametrize("case", ["g4-d128-ragged", "g8-d64", "g2-d64-bs32-l16s8", "ragged",
-                                  "more-pairs-than-sms", "no-local-partial-last"])
+                                  "more-pairs-than-sms", "no-local-partial-last", "g4-l16s16",
+                                  "g4-bs128-l64s32", "g3-padded-heads"])
 def test_step_selection_equals_separate_selection(case, cuda_device):
     """The step's block scores and selection are those of bsa_select_blocks, bit for bit: both
     weigh the same stored window terms by the same per-chunk softmax weights."""
