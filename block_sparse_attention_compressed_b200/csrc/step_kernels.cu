@@ -400,18 +400,14 @@ __global__ void __launch_bounds__(kStepThreads, 1)
             // and 4b - 1 when l = 2s: the previous lane's last window (lane 0: the previous tile's,
             // from the chunk's last terms).
             uint32_t kand = 0xffffffffu, kor = 0u;
-            constexpr int TB = 32 / (4 * SGP) < 2 ? 1 : 2;
+            constexpr int TB = 1;  // tiles per TMEM load (two loads in flight)
             constexpr int LW = TB * 4 * SGP;
             const int nbt = (pg.nb + 31) / 32;  // tiles holding blocks
             const int qq = w & 3;
             const int nq = nbt > qq ? (nbt - qq + 3) / 4 : 0;
             const int i_lo = w < 4 ? 0 : (nq + 1) / 2, i_hi = w < 4 ? (nq + 1) / 2 : nq;
-            for (int i0 = i_lo; i0 < i_hi; i0 += TB) {
-                float v[LW];
-                if (2 * (qq + 4 * i0) < pg.nch) {
-                    tmem_ld<LW>(tq_addr + (uint32_t)(i0 * 4 * SGP), v);
-                    tmem_wait_ld();
-                }
+            // one tile group's maxima from its TMEM terms
+            auto tile_maxima = [&](const float (&v)[LW], int i0) {
 #pragma unroll
                 for (int u = 0; u < TB; ++u) {
                     if (i0 + u >= i_hi) break;
@@ -448,7 +444,22 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                         if (a.block_scores) a.block_scores[(size_t)pair * a.nb_cap + blk] = mx;
                     }
                 }
+            };
+            // TMEM loads double-buffered: the next group's load is in flight while this one's
+            // maxima are taken (only tiles that hold scored windows are loaded)
+            auto scored = [&](int i0) { return i0 < i_hi && 2 * (qq + 4 * i0) < pg.nch; };
+            float va[LW], vb[LW];
+            if (scored(i_lo)) tmem_ld<LW>(tq_addr + (uint32_t)(i_lo * 4 * SGP), va);
+            for (int i0 = i_lo; i0 < i_hi; i0 += 2 * TB) {
+                tmem_wait_ld();
+                if (scored(i0 + TB)) tmem_ld<LW>(tq_addr + (uint32_t)((i0 + TB) * 4 * SGP), vb);
+                tile_maxima(va, i0);
+                if (i0 + TB >= i_hi) break;
+                tmem_wait_ld();
+                if (scored(i0 + 2 * TB)) tmem_ld<LW>(tq_addr + (uint32_t)((i0 + 2 * TB) * 4 * SGP), va);
+                tile_maxima(vb, i0 + TB);
             }
+            tmem_wait_ld();
             if (a.block_scores)
                 for (int64_t blk = pg.nb + grp.tid; blk < a.nb_cap; blk += grp.nt)
                     a.block_scores[(size_t)pair * a.nb_cap + blk] = -INFINITY;

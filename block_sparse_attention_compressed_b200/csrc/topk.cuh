@@ -45,11 +45,12 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 //
 // The k-th largest key is located by radix digits below the bits that all candidates share: a
 // first digit of up to kFirstDigitBits bits (one histogram bin per value, found with a two-level
-// descending scan), then 8-bit digits. As soon as the digit bucket holding the k-th key has at
-// most kExactMax keys, the owners of those keys rank them exactly among themselves (score
-// descending, block ascending); the taken candidates are those above the bucket plus the bucket
-// keys ranked below the number still needed. Otherwise the ties at the final key value are taken
-// in block order.
+// descending scan), then 8-bit digits. When that bucket holds exactly the number of keys still
+// needed, all of them are taken with those above it. Otherwise, as soon as the bucket has at most
+// kExactMax keys, the owners of those keys rank them exactly among themselves (score descending,
+// block ascending); the taken candidates are those above the bucket plus the bucket keys ranked
+// below the number still needed. Otherwise the ties at the final key value are taken in block
+// order.
 constexpr int kKeysPerThread = 8;
 constexpr int kFirstDigitBits = 12;
 constexpr int kExactMax = 128;
@@ -197,7 +198,7 @@ __device__ void topk_union(const SelectArgs& a, int nb, uint32_t* keys, TopkSmem
 
     uint32_t thr = 0xffffffffu;  // keys > thr are taken, plus the first `need` keys == thr
     int need = 0;
-    bool exact = false;
+    bool exact = false, whole = false;
     uint32_t emask = 0u, eprefix = 0u;
     if (kk > 0 && !take_all) {
         // bits that every candidate shares need no histogram pass (block-wide AND / OR)
@@ -256,6 +257,10 @@ __device__ void topk_union(const SelectArgs& a, int nb, uint32_t* keys, TopkSmem
                 prefix |= (uint32_t)t.digit << shift;
                 need = t.need;
                 mask |= dmask << shift;
+                if (in_regs && t.bcnt == need) {
+                    whole = true;  // the bucket holds exactly the keys still needed: all are taken
+                    break;
+                }
                 if (shift == 0) break;  // every bit decided: the bucket's keys are all equal
                 if (in_regs && t.bcnt <= kExactMax) {
                     exact = true;
@@ -267,7 +272,7 @@ __device__ void topk_union(const SelectArgs& a, int nb, uint32_t* keys, TopkSmem
             }
         }
         thr = prefix;
-        if (exact) {
+        if (exact || whole) {
             emask = mask;
             eprefix = prefix;
         }
@@ -276,7 +281,11 @@ __device__ void topk_union(const SelectArgs& a, int nb, uint32_t* keys, TopkSmem
     if (in_regs) {
         // taken flags of the thread's own candidates
         bool fl[kKeysPerThread];
-        if (exact) {
+        if (whole) {
+            // the keys above the k-th key's bucket, and the whole bucket
+#pragma unroll
+            for (int e = 0; e < kKeysPerThread; ++e) fl[e] = seg_lo + e < seg_hi && (kr[e] & emask) >= eprefix;
+        } else if (exact) {
 #pragma unroll
             for (int e = 0; e < kKeysPerThread; ++e) {
                 if (seg_lo + e < seg_hi && (kr[e] & emask) == eprefix) {
