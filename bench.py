@@ -13,9 +13,15 @@ events between barriers + synchronizes, max over ranks. ``e2e`` is the same metr
 Python binding, with every step's inputs (each layer's q; the new k/v rows when the cache grows)
 copied in from pinned host memory and its outputs (every layer) copied back. The copies are
 double-buffered on two copy streams, so a step's transfers overlap its neighbours' compute.
-``roofline`` is for the largest single kernel of the step (the sparse attention), from a second,
-identical pass that brackets every library call with CUDA events. ``cpu_baseline`` (rank 0, one
-GPU only) and ``--impl reference`` time the CPU oracle on a bounded sample of the same workload.
+``roofline`` is for the largest single launch of the step (the fused step kernel where
+bsa_decode_step runs one, else the sparse attention with its combine), from a second, identical pass
+that brackets every library call with CUDA events; the benchmark spec is the whole step's algorithmic
+bytes over 8 TB/s against the 0.70 target. ``cpu_baseline`` (rank 0, one GPU only) and ``--impl
+reference`` time the CPU oracle's decode step (keys compressed beforehand, as at decode time) on a
+bounded sample of the same workload, on all host cores and on one.
+
+With ``--gpus N`` and no WORLD_SIZE in the environment, the script starts the N ranks itself
+(torch.distributed.run on 127.0.0.1); under a launcher it checks that WORLD_SIZE is N.
 """
 from __future__ import annotations
 
@@ -37,10 +43,12 @@ sys.path.insert(0, ROOT)
 
 METRIC = "block-sparse decode steps/s & achieved HBM GB/s (select+attn) at 128K ctx"
 # the library kernel behind each single-launch phase of a step, by dtype
-KERNEL_OF_PHASE = {"decode": {"bf16": "decode_tma_kernel", "f32": "decode_f32_kernel"},
+KERNEL_OF_PHASE = {"step": {"bf16": "step_kernel"},
+                   "decode": {"bf16": "decode_tma_kernel+combine_kernel", "f32": "decode_f32_kernel"},
                    "append": {"bf16": "append_kernel", "f32": "append_kernel"},
                    "select": {"bf16": "score_tma_kernel+select_kernel",
                               "f32": "score_f32_kernel+select_kernel"}}
+NORTH_STAR_FRAC = 0.70  # of 8 TB/s, for the fused select + sparse attention at 128K
 L2_BYTES = 126 * 1024 * 1024
 NOMINAL_HBM_GBS = 8000.0
 
@@ -55,6 +63,9 @@ def parse():
     ap.add_argument("--batch", type=int, default=None,
                     help="override the workload's batch (small cases for profiling only)")
     ap.add_argument("--no-graph", action="store_true", help="launch steps directly (no CUDA graph)")
+    ap.add_argument("--path", default="auto", choices=["auto", "fused", "chained"],
+                    help="single-layer steps: bsa_decode_step's own choice, the fused one-kernel step "
+                         "(bsa_decode_step_fused), or the chained selection and attention kernels")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
@@ -156,7 +167,7 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------------------- workload run
 class Bench:
-    def __init__(self, w, device, seed_offset: int, steps_total: int):
+    def __init__(self, w, device, seed_offset: int, steps_total: int, path: str = "auto"):
         import torch
         import block_sparse_attention_compressed_b200 as bsa
         from block_sparse_attention_compressed_b200.workloads import generate
@@ -192,6 +203,11 @@ class Bench:
         self.lse = [torch.zeros(B, w.num_q_heads, dtype=torch.float32, device=device)
                     for _ in range(w.layers)]
         self.seq0 = self.data["seq_lens"].clone()
+        # one kernel per step (the fused path) for the single-layer workloads: bsa_decode_step's
+        # own choice, or the path asked for
+        single = w.layers == 1 and not w.forecast
+        self.path = path if single else "auto"
+        self.fused = single and (path == "fused" or (path == "auto" and bsa.bsa_decode_step_info(self.p)[0]))
         if w.forecast and (w.layers > 1 or self.append):
             raise ValueError("the Forecast-indexer workloads are single-layer, fixed-length")
         torch.cuda.synchronize()
@@ -236,18 +252,26 @@ class Bench:
                                              self.ws, stream=stream)
             ev(2 * (len(anchors) - 1))
             return
-        if events is None:
+        if events is None and self.path != "chained":
             bsa.bsa_decode_step(self.p, q, d["k"][0], d["v"][0], self.ck,
                                 d["k_new"][i] if self.append else None,
                                 d["v_new"][i] if self.append else None, d["seq_lens"],
                                 self.block_idx, self.n_sel, None, self.out[0], self.lse[0], self.ws,
-                                stream=stream)
+                                stream=stream, fused=self.fused)
             return
         k = 0
         if self.append:
             ev(k); k += 1
             bsa.bsa_compress_append(self.p, d["k"][0], d["v"][0], d["k_new"][i], d["v_new"][i],
                                     d["seq_lens"], self.ck, self.ws, stream=stream)
+        if self.fused:
+            # the step kernel alone (the append, if any, was bracketed above)
+            ev(k)
+            bsa.bsa_decode_step(self.p, q, d["k"][0], d["v"][0], self.ck, None, None, d["seq_lens"],
+                                self.block_idx, self.n_sel, None, self.out[0], self.lse[0], self.ws,
+                                stream=stream, fused=True)
+            ev(k + 1)
+            return
         ev(k)
         bsa.bsa_select_blocks(self.p, q, self.ck, d["seq_lens"], self.block_idx, self.n_sel, None,
                               self.ws, stream=stream)
@@ -277,17 +301,31 @@ class Bench:
             bsa.bsa_sparse_decode_layers(self.p, qs, d["k"], d["v"], d["seq_lens"], self.block_idx,
                                          self.n_sel, outs, lses, self.ws, stream=stream)
             return
+        if self.path == "chained":
+            if k_new is not None:
+                bsa.bsa_compress_append(self.p, d["k"][0], d["v"][0], k_new, v_new, d["seq_lens"],
+                                        self.ck, self.ws, stream=stream)
+            bsa.bsa_select_blocks(self.p, qs[0], self.ck, d["seq_lens"], self.block_idx, self.n_sel,
+                                  None, self.ws, stream=stream)
+            bsa.bsa_sparse_decode(self.p, qs[0], d["k"][0], d["v"][0], d["seq_lens"], self.block_idx,
+                                  self.n_sel, outs[0], lses[0], self.ws, stream=stream)
+            return
         bsa.bsa_decode_step(self.p, qs[0], d["k"][0], d["v"][0], self.ck, k_new, v_new, d["seq_lens"],
                             self.block_idx, self.n_sel, None, outs[0], lses[0], self.ws,
-                            stream=stream)
+                            stream=stream, fused=self.fused)
 
     def kernel_names(self):
+        """The phases pass B brackets with events, in launch order."""
+        if self.fused:
+            return (["append"] if self.append else []) + ["step"]
         names = ["select", "decode"] * (len(self.w.anchors) if self.w.layers > 1 else 1)
         return (["append"] + names) if (self.append and self.w.layers == 1) else names
 
     def launches_per_step(self):
+        if self.fused:
+            return 1 + (1 if self.append else 0)
         # bsa_select_blocks launches two kernels (scoring, selection), the bf16 sparse attention two
-        # (attention, combine), the fp32 one one, the append one
+        # (attention, combine), the fp32 one one
         n = self.kernel_names()
         return len(n) + n.count("select") + (n.count("decode") if self.w.dtype == "bf16" else 0)
 
@@ -310,9 +348,9 @@ def load_peaks():
         return 6650.0, "fallback"
 
 
-# The sources that decide a kernel's code and launch plan: its own file, the shared header and the
-# host side that plans the launch.
-KERNEL_SOURCES = {"decode": "decode_kernels.cu", "combine": "decode_kernels.cu",
+# The sources that decide a kernel's code and launch plan: its own file, the shared headers and
+# the host side that plans the launch.
+KERNEL_SOURCES = {"step": "step_kernels.cu", "decode": "decode_kernels.cu", "combine": "decode_kernels.cu",
                   "score": "select_kernels.cu", "select": "select_kernels.cu",
                   "compress": "compress_kernels.cu", "append": "compress_kernels.cu"}
 
@@ -351,7 +389,8 @@ def kernel_source_hash(kernel: str | None = None) -> str:
         paths = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")))
     else:
         own = next(f for k, f in KERNEL_SOURCES.items() if kernel.startswith(k))
-        paths = [os.path.join(csrc, n) for n in (own, "bsa_internal.cuh", "bsa_api.cu")]
+        paths = [os.path.join(csrc, n) for n in (own, "bsa_internal.cuh", "bsa_api.cu", "tiles.cuh",
+                                                 "topk.cuh")]
     h = hashlib.sha256()
     for p in paths:
         with open(p, encoding="utf-8") as f:
@@ -376,9 +415,11 @@ def profile_traffic(kernel: str, workload: str):
 
 # ------------------------------------------------------------------------------- CPU (oracle) leg
 def cpu_oracle_sample(w, data, seconds: float):
-    """Time the CPU oracle on a bounded sample of (batch, kv-head) pairs of the same workload:
-    selection + attention on the first layer, attention with that selection on the others.
-    Returns (steps/s scaled to the whole batch, threads, description)."""
+    """The CPU oracle's decode step on a bounded sample of the workload's (batch, kv-head) pairs:
+    group scoring, block reduction, top-k and attention on the scoring layers (the compressed keys
+    formed beforehand, as at decode time), attention with their selection on the other layers.
+    Returns a dict: steps/s scaled to the whole batch on all host threads and on one, the threads,
+    the compression's CPU time per step-equivalent cache (reported apart), and a description."""
     import torch
     import oracle
     G, Hkv = w.group, w.num_kv_heads
@@ -401,34 +442,52 @@ def cpu_oracle_sample(w, data, seconds: float):
     P = oracle.make_problem(n0, G, 1, w.head_dim, T_cap,
                             oracle.F32 if w.dtype == "f32" else oracle.BF16, w.n_init, w.n_local,
                             w.top_k, w.cmp_kernel, w.cmp_stride, w.block_size)
-
     f_arr = (oracle.raw(torch.stack([data["f"][b, h:h + 1] for b, h in pairs]))[0]
              if w.forecast else None)
+    # A1, the compression of every scoring layer's keys (once per cache; timed apart)
+    t0 = time.perf_counter()
+    cks = {L: oracle.compress_cache(P, arrays[L][1], lens) for L in w.anchors}
+    compress_s = (time.perf_counter() - t0) * (total / n0)
 
-    def one():
-        if w.forecast:
-            oracle.decode_forecast(P, f_arr, *arrays[0], lens)
-            return
+    def one(sub=None):
+        idx = slice(None) if sub is None else slice(0, sub)
         r = None
         for L in range(w.layers):
-            if L in w.anchors:
-                r = oracle.decode(P, *arrays[L], lens)   # select + attend on an anchor layer
+            q_, k_, v_ = arrays[L]
+            if sub is not None:
+                q_, k_, v_ = q_[idx], k_[idx], v_[idx]
+            Ps = P if sub is None else oracle.make_problem(
+                sub, G, 1, w.head_dim, T_cap, P.dtype, w.n_init, w.n_local, w.top_k, w.cmp_kernel,
+                w.cmp_stride, w.block_size)
+            ln = lens if sub is None else lens[:sub]
+            if w.forecast:
+                oracle.decode_forecast(Ps, f_arr[idx], q_, k_, v_, ln, ck=cks[0][idx])
+            elif L in w.anchors:
+                r = oracle.decode(Ps, q_, k_, v_, ln, ck=cks[L][idx])  # select + attend
             else:
-                oracle.attend_pairs(P, *arrays[L], lens, r["idx"], r["n_sel"])
+                oracle.attend_pairs(Ps, q_, k_, v_, ln, r["idx"], r["n_sel"])
 
-    t0 = time.perf_counter()
-    one()
-    dt0 = time.perf_counter() - t0
-    reps = max(1, int(seconds / max(dt0, 1e-6)))
-    t0 = time.perf_counter()
-    for _ in range(reps):
-        one()
-    dt = (time.perf_counter() - t0) / reps
-    step_s = dt * (total / n0)
-    desc = (f"CPU oracle (fp64; its selection recomputes each pair's compressed keys) on {n0} of "
-            f"{total} (batch, kv-head) pairs" + (f" x {w.layers} layers" if w.layers > 1 else "")
-            + f", {reps} repetitions, time scaled by {total}/{n0} to a full step")
-    return 1.0 / step_s, threads, desc
+    def timed(fn, budget):
+        t0 = time.perf_counter()
+        fn()
+        dt0 = time.perf_counter() - t0
+        reps = max(1, int(budget / max(dt0, 1e-6)))
+        t0 = time.perf_counter()
+        for _ in range(reps):
+            fn()
+        return (time.perf_counter() - t0) / reps, reps
+
+    dt, reps = timed(one, seconds)
+    with oracle.threads(1):
+        dt1, reps1 = timed(lambda: one(1), seconds / 4)   # one pair on one thread
+    layers = f" x {w.layers} layers" if w.layers > 1 else ""
+    desc = (f"CPU oracle (fp64) decode step on {n0} of {total} (batch, kv-head) pairs{layers}: "
+            f"scoring, block reduction, top-k and attention with the keys compressed beforehand "
+            f"(their compression, {compress_s:.2f} s per full cache, is timed apart), "
+            f"{reps} repetitions on {threads} threads scaled by {total}/{n0}, and one pair on one "
+            f"thread ({reps1} repetitions) scaled by {total}")
+    return {"value": 1.0 / (dt * total / n0), "single_thread_value": 1.0 / (dt1 * total),
+            "cores": threads, "compress_s_per_cache": compress_s, "sample": desc}
 
 
 # -------------------------------------------------------------------------------------------- main
@@ -438,7 +497,7 @@ def run_bsa(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     K, W = args.steps, args.warmup
-    bench = Bench(w, dev, seed_offset=10000 * rank, steps_total=K + W + 1)
+    bench = Bench(w, dev, seed_offset=10000 * rank, steps_total=K + W + 1, path=args.path)
     T_run = w.seq_len
     ab = algorithmic(w, T_run)
     stream = torch.cuda.Stream(device=dev)
@@ -596,25 +655,29 @@ def run_bsa(args, w, world, rank, local):
     if err:
         raise RuntimeError(f"device error flags set during the benchmark: {err:#x}")
 
-    # ---- roofline of the dominant kernel
+    # ---- roofline of the largest single launch, and the spec fraction of the whole step
     peak, peak_kind = load_peaks()
     q_bytes = w.batch * w.num_q_heads * w.head_dim * w.elem_bytes
-    kbytes = {"select": ab["ck"] + (ab["f"] if w.forecast else q_bytes),  # compressed keys + q (or f)
+    fv = ab["f"] if w.forecast else 0
+    kbytes = {"select": ab["ck"] + (fv if w.forecast else q_bytes),  # compressed keys + q (or f)
               "decode": ab["kv"] + ab["qo"],         # selected K/V rows + q + out, every layer
+              "step": ab["ck"] + ab["kv"] + ab["qo"] + fv,  # the fused step: all of them
               "append": ab["append"]}
-    # the selection phase is two launches (scoring, then selection); the others are one each, so
-    # the roofline is taken on the largest single-launch phase: the sparse attention
+    # the selection phase is two launches (scoring, then selection): the roofline is taken on the
+    # largest phase that is one launch, or one launch and its combine
     single = {n: t for n, t in kern_ms.items() if n != "select"} or kern_ms
     dom = max(single, key=single.get)
     kname = KERNEL_OF_PHASE[dom][w.dtype]
-    n_calls = names.count(dom)  # launches of that kernel per step (one per anchor)
+    n_calls = names.count(dom)  # launches of that phase per step (one per anchor)
     achieved = kbytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
     traffic = profile_traffic(kname, w.name)
     roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
                 "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
                 "peak_kind": peak_kind + " copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
                 "traffic": traffic, "algorithmic_bytes_per_launch": kbytes[dom] / n_calls,
-                "kernel_ms": round(kern_ms[dom] / n_calls, 5)}
+                "kernel_ms": round(kern_ms[dom] / n_calls, 5),
+                "launches_timed": "one" if "+" not in kname else "the attention kernel and its combine"}
 
     steps_per_s = world * K / (total_ms * 1e-3)
     gbs = per_step_bytes * world * K / (total_ms * 1e-3) / 1e9
@@ -643,10 +706,16 @@ def run_bsa(args, w, world, rank, local):
             "l2": ("L2 flushed (256 MB write) between timed steps" if flush else
                    f"inputs larger than L2: {per_step_bytes / 1e6:.0f} MB read per step vs 126 MB L2"),
             "cuda_graph": graph is not None,
+            "step_path": "fused" if bench.fused else "chained",
         },
         "tokens_per_s": round(steps_per_s * w.batch, 1),
         "hbm_gbs": round(gbs / world, 1),
         "frac_of_8tbs": round(gbs / world / NOMINAL_HBM_GBS, 4),
+        "north_star": {"basis": "compressed keys + selected K/V + q + out bytes of the whole step "
+                                "over 8 TB/s, device-timed step", "frac_of_8tbs":
+                       round(gbs / world / NOMINAL_HBM_GBS, 4), "target": NORTH_STAR_FRAC,
+                       "met": bool(gbs / world / NOMINAL_HBM_GBS >= NORTH_STAR_FRAC)},
+        "fused_step": bool(bench.fused),
         "algorithmic_bytes_per_step": per_step_bytes,
         "kernels_ms": {k: round(v, 5) for k, v in kern_ms.items()},
         "roofline": roofline,
@@ -658,9 +727,12 @@ def run_bsa(args, w, world, rank, local):
         "kernel_sources_sha256_16": kernel_source_hash(),
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        v, cores, desc = cpu_oracle_sample(w, bench.data, args.cpu_seconds)
-        result["cpu_baseline"] = {"value": round(v, 4), "unit": "steps/s", "cores": cores,
-                                  "kind": "oracle", "sample": desc}
+        c = cpu_oracle_sample(w, bench.data, args.cpu_seconds)
+        result["cpu_baseline"] = {"value": round(c["value"], 4), "unit": "steps/s",
+                                  "cores": c["cores"], "kind": "oracle",
+                                  "single_thread_value": round(c["single_thread_value"], 5),
+                                  "compress_s_per_cache": round(c["compress_s_per_cache"], 3),
+                                  "sample": c["sample"]}
     return result
 
 
@@ -679,8 +751,9 @@ def run_reference(args, w, world, rank):
     vals = []
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        v, cores, desc = cpu_oracle_sample(w, data, per_step)
-        vals.append(v)
+        c = cpu_oracle_sample(w, data, per_step)
+        vals.append(c["value"])
+    cores, desc = c["cores"], c["sample"]
     wall = time.perf_counter() - t0
     value = statistics.median(vals)
     return {
@@ -691,15 +764,35 @@ def run_reference(args, w, world, rank):
         "config": {"workload": w.name, "batch": w.batch, "seq_len": w.seq_len},
         "impl": "reference",
         "cpu_baseline": {"value": round(value, 4), "unit": "steps/s", "cores": cores,
-                         "kind": "oracle", "sample": desc},
+                         "kind": "oracle", "single_thread_value": round(c["single_thread_value"], 5),
+                         "sample": desc},
         "e2e": {"value": round(value, 4), "unit": "steps/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
         "wall_s": round(wall, 2),
     }
 
 
+def relaunch(n: int) -> int:
+    """Start n ranks of this script on this node (torch.distributed.run, rendezvous on
+    127.0.0.1, a free port) with the same arguments; rank 0 prints the JSON line."""
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), os.path.abspath(__file__),
+           *sys.argv[1:]]
+    return subprocess.call(cmd)
+
+
 def main():
     args = parse()
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        sys.exit(relaunch(args.gpus))
+    if world_env is not None and int(world_env) != args.gpus:
+        raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world_env}; "
+                         "start one rank per GPU with the same N")
     from block_sparse_attention_compressed_b200.workloads import DEFAULT_WORKLOAD, WORKLOADS
     w = WORKLOADS[args.workload or DEFAULT_WORKLOAD]
     if args.batch:

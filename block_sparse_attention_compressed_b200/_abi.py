@@ -79,9 +79,13 @@ _SIGS = {
                                       ctypes.c_size_t, _P]),
     "bsa_decode_step": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                              ctypes.c_size_t, _P]),
+    "bsa_decode_step_fused": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                   ctypes.c_size_t, _P]),
     "bsa_decode_step_anchored": (_S, [_PP, ctypes.c_int32, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
                                       _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "bsa_read_device_error": (_S, [_P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32), _P]),
+    "bsa_decode_step_info": (_S, [_PP, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32),
+                                  ctypes.POINTER(ctypes.c_int32)]),
     "bsa_sparse_decode_noalloc": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]),
 }
 
@@ -334,11 +338,22 @@ def bsa_decode_step_anchored(p: Params, anchors, qs, k_caches, v_caches, cks, se
         "bsa_decode_step_anchored")
 
 
+def bsa_decode_step_info(p: Params, append: bool = False) -> tuple[bool, int]:
+    """(fused, launches) of bsa_decode_step for these parameters: whether one kernel runs the
+    whole step, and the kernel launches of one call (with the append when ``append``)."""
+    fused, launches = ctypes.c_int32(), ctypes.c_int32()
+    _check(lib().bsa_decode_step_info(ctypes.byref(p), int(bool(append)), ctypes.byref(fused),
+                                      ctypes.byref(launches)), "bsa_decode_step_info")
+    return bool(fused.value), int(launches.value)
+
+
 def bsa_decode_step(p: Params, q, k_cache, v_cache, ck, k_new, v_new, seq_lens, block_idx, n_sel,
-                    block_scores, out, lse, ws, stream=None):
+                    block_scores, out, lse, ws, stream=None, fused=False):
+    """bsa_decode_step (or, with ``fused``, bsa_decode_step_fused)."""
     import torch
     n, e = _shapes(p), _elem(p)
-    _check(lib().bsa_decode_step(
+    name = "bsa_decode_step_fused" if fused else "bsa_decode_step"
+    _check(getattr(lib(), name)(
         ctypes.byref(p), _ptr(q, "q", e, n["q"]), _ptr(k_cache, "k_cache", e, n["cache"]),
         _ptr(v_cache, "v_cache", e, n["cache"]), _ptr(ck, "ck", e, n["ck"]),
         _ptr(k_new, "k_new", e, n["new"], optional=True),
@@ -349,7 +364,7 @@ def bsa_decode_step(p: Params, q, k_cache, v_cache, ck, k_new, v_new, seq_lens, 
         _ptr(block_scores, "block_scores", torch.float32, n["scores"], optional=True),
         _ptr(out, "out", e, n["q"]), _ptr(lse, "lse", torch.float32, n["lse"], optional=True),
         _ptr(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
-        "bsa_decode_step")
+        name)
 
 
 def bsa_read_device_error(ws, stream=None) -> int:

@@ -161,6 +161,9 @@ bsa_status_t make_plan(const bsa_params_t* prm, Plan* p) {
                 P.step_tmem_cols = tc;
                 P.step_ctas = P.pairs < kNumSMs ? P.pairs : kNumSMs;
                 P.step_fused = 1;
+                // one CTA per pair streams at most ~50 GB/s: with fewer pairs than about two thirds
+                // of the SMs, the chained kernels (spread over every SM) are faster
+                P.step_preferred = 3 * P.pairs >= 2 * kNumSMs;
             }
         }
     }
@@ -635,14 +638,19 @@ bsa_status_t bsa_sparse_decode(const bsa_params_t* params, const void* q, const 
                                     ws_bytes, stream);
 }
 
-bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_cache,
-                             void* v_cache, void* ck, const void* k_new, const void* v_new,
-                             int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
-                             float* block_scores, void* out, float* lse, void* ws,
-                             size_t ws_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace bsa {
+namespace {
+// bsa_decode_step and bsa_decode_step_fused: `mode` 0 picks the path, 1 requires the fused one.
+bsa_status_t decode_step(int mode, const bsa_params_t* params, const void* q, void* k_cache,
+                         void* v_cache, void* ck, const void* k_new, const void* v_new,
+                         int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel, float* block_scores,
+                         void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
     Plan P;
     bsa_status_t st = make_plan(params, &P);
     if (st != BSA_OK) return st;
+    if (mode == 1 && !P.step_fused) return BSA_ERR_UNSUPPORTED;
     const bool append = k_new != nullptr && v_new != nullptr;
     if ((k_new == nullptr) != (v_new == nullptr)) return BSA_ERR_INVALID_ARG;
     if (!ok16(q) || !ok16(k_cache) || !ok16(v_cache) || !ok16(out) || !ok4(seq_lens) ||
@@ -656,7 +664,7 @@ bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_
         st = do_append(P, k_cache, v_cache, k_new, v_new, seq_lens, ck, ws, stream);
         if (st != BSA_OK) return st;
     }
-    if (P.step_fused)
+    if (mode == 1 || P.step_preferred)
         return do_step_fused(P, q, k_cache, v_cache, ck, seq_lens, block_idx, n_sel, block_scores, out,
                              lse, ws, stream);
     if ((st = do_select(P, q, ck, seq_lens, block_idx, n_sel, block_scores, ws, stream)) != BSA_OK)
@@ -670,6 +678,40 @@ bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_
     static thread_local KVMapCache maps;
     if ((st = make_maps(P, da, 1, &maps)) != BSA_OK) return st;
     return from_cuda(launch_decode(P, da, &maps.maps, 1, stream));
+}
+}  // namespace
+}  // namespace bsa
+
+extern "C" {
+
+bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_cache,
+                             void* v_cache, void* ck, const void* k_new, const void* v_new,
+                             int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                             float* block_scores, void* out, float* lse, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+    return decode_step(0, params, q, k_cache, v_cache, ck, k_new, v_new, seq_lens, block_idx, n_sel,
+                       block_scores, out, lse, ws, ws_bytes, stream);
+}
+
+bsa_status_t bsa_decode_step_fused(const bsa_params_t* params, const void* q, void* k_cache,
+                                   void* v_cache, void* ck, const void* k_new, const void* v_new,
+                                   int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                                   float* block_scores, void* out, float* lse, void* ws,
+                                   size_t ws_bytes, cudaStream_t stream) {
+    return decode_step(1, params, q, k_cache, v_cache, ck, k_new, v_new, seq_lens, block_idx, n_sel,
+                       block_scores, out, lse, ws, ws_bytes, stream);
+}
+
+bsa_status_t bsa_decode_step_info(const bsa_params_t* params, int32_t append, int32_t* fused,
+                                  int32_t* launches) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if (fused) *fused = P.step_preferred;
+    // fused: the step kernel; chained: scoring, selection, attention (+ combine for bf16)
+    const int32_t n = P.step_preferred ? 1 : (P.dtype == BSA_BF16 ? 4 : 3);
+    if (launches) *launches = n + (append ? 1 : 0);
+    return BSA_OK;
 }
 
 bsa_status_t bsa_read_device_error(void* ws, size_t ws_bytes, uint32_t* flags,

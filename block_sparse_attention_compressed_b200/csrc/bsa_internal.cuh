@@ -45,6 +45,7 @@ struct Plan {
     // fused step (bf16): one CTA per pair (a persistent grid walks the pairs); 0 when the shape is
     // outside what that kernel handles, and the step then chains the separate kernels
     int step_fused, step_ctas, step_sgp, step_nch_cap, step_key_words;
+    int step_preferred;  // bsa_decode_step takes the fused path (enough pairs to fill the SMs)
     uint32_t step_tmem_cols;
     size_t step_smem;
     // workspace layout (bytes)

@@ -221,15 +221,41 @@ bsa_status_t bsa_decode_step_anchored(const bsa_params_t* params, int32_t num_la
                                       void* const* outs, float* const* lses, void* workspace,
                                       size_t workspace_bytes, cudaStream_t stream);
 
-/* One decode step of one layer, as launches chained on `stream` with programmatic dependent
- * launch: optional append (when k_new and v_new are both non-NULL), then bsa_select_blocks, then
- * bsa_sparse_decode with the fresh selection. block_idx / n_sel receive the selection;
- * block_scores and lse may be NULL. */
+/* One decode step of one layer (steps 2-5, after an optional append when k_new and v_new are both
+ * non-NULL), queued on `stream` with no host synchronisation. block_idx / n_sel receive the
+ * selection; block_scores and lse may be NULL. It runs the fused step (as bsa_decode_step_fused)
+ * when that is possible and there are enough (batch, kv head) pairs to keep most SMs streaming
+ * (at least two thirds of the SM count), else the chained launches of bsa_select_blocks and
+ * bsa_sparse_decode with programmatic dependent launch; bsa_decode_step_info tells which. The
+ * selection is the same bit for bit either way. */
 bsa_status_t bsa_decode_step(const bsa_params_t* params, const void* q, void* k_cache,
                              void* v_cache, void* ck, const void* k_new, const void* v_new,
                              int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
                              float* block_scores, void* out, float* lse, void* workspace,
                              size_t workspace_bytes, cudaStream_t stream);
+
+/* bsa_decode_step as one kernel (after the optional append's): a CTA per (batch, kv head) pair,
+ * one per SM (a persistent grid walks the pairs when there are more pairs than SMs), scores the
+ * pair's compressed keys with the group's query heads, keeps the window terms in the SM's tensor
+ * memory, takes the block maxima and the top-k there and in shared memory, and attends the
+ * selected blocks, writing out and lse directly (no split partials, no combine pass). Same
+ * arguments, results and selection as bsa_decode_step; the workspace holds only the error word.
+ * Supported: bf16, blocks of four compression strides (BS = 4s, l = s or 2s, BS a multiple of 64),
+ * max_seq_len of at least one window (l) and window terms within 512 tensor-memory columns (about
+ * 260K tokens at G = 4); other parameter sets return BSA_ERR_UNSUPPORTED. Each SM streams at most ~50 GB/s, so with few pairs the chained
+ * kernels of bsa_decode_step are faster. */
+bsa_status_t bsa_decode_step_fused(const bsa_params_t* params, const void* q, void* k_cache,
+                                   void* v_cache, void* ck, const void* k_new, const void* v_new,
+                                   int32_t* seq_lens, int32_t* block_idx, int32_t* n_sel,
+                                   float* block_scores, void* out, float* lse, void* workspace,
+                                   size_t workspace_bytes, cudaStream_t stream);
+
+/* How bsa_decode_step runs for these parameters (host only, no CUDA call): *fused is 1 when it
+ * runs the one-kernel step of bsa_decode_step_fused, 0 when it chains the scoring, selection,
+ * attention and combine kernels; *launches is the number of kernel launches of one call, counting
+ * the append when `append` is non-zero. Either output pointer may be NULL. */
+bsa_status_t bsa_decode_step_info(const bsa_params_t* params, int32_t append, int32_t* fused,
+                                  int32_t* launches);
 
 /* Copy the workspace error word to *flags (bits of bsa_device_error_t), clear it, and
  * synchronize `stream`. Returns BSA_ERR_DEVICE_CHECK when a bit was set, BSA_OK otherwise. */

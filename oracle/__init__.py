@@ -100,6 +100,8 @@ def _bind(path: str):
         "bsa_oracle_set_num_threads": (None, [_INT]),
         "bsa_oracle_decode_ck": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P, _INT,
                                         _P, _P, _P, _P, _P, _P]),
+        "bsa_oracle_decode_forecast_ck": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P, _P,
+                                                 _INT, _P, _P, _P, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -328,9 +330,9 @@ def decode(P: Problem, q, k_cache, v_cache, seq_lens, pairs=None, given_idx=None
     return res
 
 
-def decode_forecast(P: Problem, f, q, k_cache, v_cache, seq_lens, pairs=None) -> dict:
+def decode_forecast(P: Problem, f, q, k_cache, v_cache, seq_lens, pairs=None, ck=None) -> dict:
     """As ``decode``, with the blocks selected from the Forecast vectors f [B][Hkv][d] (storage
-    array of the problem's dtype) instead of the queries; q attends them."""
+    array of the problem's dtype) instead of the queries; q attends them. ``ck`` as in ``decode``."""
     f = _raw_check(f, P.dtype)
     q = _raw_check(q, P.dtype)
     k_cache, v_cache = _raw_check(k_cache, P.dtype), _raw_check(v_cache, P.dtype)
@@ -348,10 +350,20 @@ def decode_forecast(P: Problem, f, q, k_cache, v_cache, seq_lens, pairs=None) ->
         out=np.zeros((n, G, P.head_dim), dtype=np.float64),
         lse=np.zeros((n, G), dtype=np.float64),
     )
-    rc = _load().bsa_oracle_decode_forecast(
-        ctypes.byref(P), _ptr(f), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
-        _ptr(pairs), n, _ptr(res["idx"]), _ptr(res["n_sel"]), _ptr(res["block_scores"]),
-        _ptr(res["boundary"]), _ptr(res["out"]), _ptr(res["lse"]))
+    if ck is not None:
+        nc_cap = num_windows(P.max_seq_len, P.cmp_kernel, P.cmp_stride)
+        ck = np.ascontiguousarray(np.asarray(ck, dtype=np.float64))
+        if ck.shape != (n, max(nc_cap, 0), P.head_dim):
+            raise ValueError(f"ck must be [{n}][{nc_cap}][{P.head_dim}] float64")
+        rc = _load().bsa_oracle_decode_forecast_ck(
+            ctypes.byref(P), _ptr(f), _ptr(q), _ptr(ck), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+            _ptr(pairs), n, _ptr(res["idx"]), _ptr(res["n_sel"]), _ptr(res["block_scores"]),
+            _ptr(res["boundary"]), _ptr(res["out"]), _ptr(res["lse"]))
+    else:
+        rc = _load().bsa_oracle_decode_forecast(
+            ctypes.byref(P), _ptr(f), _ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seq_lens),
+            _ptr(pairs), n, _ptr(res["idx"]), _ptr(res["n_sel"]), _ptr(res["block_scores"]),
+            _ptr(res["boundary"]), _ptr(res["out"]), _ptr(res["lse"]))
     if rc != 0:
         raise ValueError("bsa_oracle_decode_forecast rejected its arguments")
     return res

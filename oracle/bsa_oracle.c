@@ -348,6 +348,16 @@ int bsa_oracle_decode_forecast(const orc_problem_t* P, const void* f, const void
                       n_sel, block_scores, boundary, out, lse);
 }
 
+/* bsa_oracle_decode_forecast with the listed pairs' compressed keys given, as bsa_oracle_decode_ck. */
+int bsa_oracle_decode_forecast_ck(const orc_problem_t* P, const void* f, const void* q, const double* ck,
+                                  const void* k_cache, const void* v_cache, const int32_t* seq_lens,
+                                  const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel,
+                                  double* block_scores, double* boundary, double* out, double* lse) {
+    if (!f || !ck) return -1;
+    return orc_decode(P, f, q, k_cache, v_cache, ck, seq_lens, pairs, n_pairs, NULL, NULL, idx, n_sel,
+                      block_scores, boundary, out, lse);
+}
+
 int bsa_oracle_attend_pairs(const orc_problem_t* P, const void* q, const void* k_cache,
                             const void* v_cache, const int32_t* seq_lens, const int32_t* pairs,
                             int n_pairs, const int32_t* idx, const int32_t* n_sel, double* out,

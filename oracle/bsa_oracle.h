@@ -154,6 +154,10 @@ int bsa_oracle_num_threads(void);
 void bsa_oracle_set_num_threads(int n);
 /* bsa_oracle_decode with the listed pairs' compressed keys given ([n_pairs][nc_cap][d], rounded to
  * the cache type, as bsa_oracle_compress_cache writes them) instead of formed from the cache. */
+int bsa_oracle_decode_forecast_ck(const orc_problem_t* P, const void* f, const void* q, const double* ck,
+                                  const void* k_cache, const void* v_cache, const int32_t* seq_lens,
+                                  const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel,
+                                  double* block_scores, double* boundary, double* out, double* lse);
 int bsa_oracle_decode_ck(const orc_problem_t* P, const void* q, const double* ck,
                          const void* k_cache, const void* v_cache, const int32_t* seq_lens,
                          const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel,

@@ -82,12 +82,13 @@ class GpuRun:
                               self.n_sel if n_sel is None else n_sel, self.out[layer],
                               self.lse[layer], self.ws)
 
-    def step(self, q=None, block_scores=True):
-        """bsa_decode_step on layer 0 (no append): selection and attention in one call."""
+    def step(self, q=None, block_scores=True, fused=False):
+        """bsa_decode_step on layer 0 (no append): selection and attention in one call; with
+        ``fused``, bsa_decode_step_fused (the one-kernel step, whatever the number of pairs)."""
         bsa.bsa_decode_step(self.p, self.q[0] if q is None else q, self.data["k"][0],
                             self.data["v"][0], self.ck[0], None, None, self.data["seq_lens"],
                             self.block_idx, self.n_sel, self.block_scores if block_scores else None,
-                            self.out[0], self.lse[0], self.ws)
+                            self.out[0], self.lse[0], self.ws, fused=fused)
 
     def decode_layers(self, block_idx=None, n_sel=None):
         L = self.w.layers

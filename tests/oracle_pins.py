@@ -404,6 +404,12 @@ def pin_decode_given_compressed_keys_composes():
             got = oracle.decode(P, qb, kb, vb, lens, pairs=pairs, ck=ck)
         for key in ("idx", "n_sel", "block_scores", "out", "lse"):
             np.testing.assert_array_equal(got[key], ref[key])
+    # the Forecast driver too
+    f = _bf16_bits(_randn((B, Hkv, d), 89))
+    ref_f = oracle.decode_forecast(P, f, qb, kb, vb, lens, pairs=pairs)
+    got_f = oracle.decode_forecast(P, f, qb, kb, vb, lens, pairs=pairs, ck=ck)
+    for key in ("idx", "n_sel", "block_scores", "out", "lse"):
+        np.testing.assert_array_equal(got_f[key], ref_f[key])
 
 
 def pin_shared_index_identical_layers():

@@ -20,8 +20,8 @@ def test_code_only_drops_comments_and_keeps_literals():
 
 
 def test_kernel_source_hash_covers_each_kernel():
-    for k in ("decode_tma_kernel", "combine_kernel", "score_tma_kernel", "select_single_kernel",
-              "compress_keys_kernel", "append_kernel"):
+    for k in ("step_kernel", "decode_tma_kernel", "combine_kernel", "score_tma_kernel",
+              "select_single_kernel", "compress_keys_kernel", "append_kernel"):
         h = bench.kernel_source_hash(k)
         assert len(h) == 16 and int(h, 16) >= 0
     assert bench.kernel_source_hash("decode_tma_kernel") != bench.kernel_source_hash("score_tma_kernel")
@@ -62,9 +62,38 @@ def test_cpu_oracle_leg_runs(name):
     from block_sparse_attention_compressed_b200.workloads import generate
     w = WORKLOADS[name].replace(batch=1, seq_len=4096, needles=2)
     data = generate(w, device="cpu")
-    steps_per_s, threads, desc = bench.cpu_oracle_sample(w, data, seconds=0.05)
-    assert steps_per_s > 0 and threads >= 1
-    assert "pairs" in desc
+    c = bench.cpu_oracle_sample(w, data, seconds=0.05)
+    assert c["value"] > 0 and c["single_thread_value"] > 0 and c["cores"] >= 1
+    assert c["compress_s_per_cache"] >= 0
+    assert "pairs" in c["sample"] and "compressed beforehand" in c["sample"]
+
+
+def test_bench_starts_its_own_ranks():
+    """`bench.py --gpus 2` without a launcher starts two ranks itself (gloo here, no GPU): the
+    reference arm prints one JSON line, from rank 0, with n_gpus 2."""
+    import json
+    import subprocess
+    env = dict(os.environ)
+    env.pop("WORLD_SIZE", None)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl",
+                        "reference", "--workload", "tiny-f32-2k", "--steps", "1", "--warmup", "0",
+                        "--cpu-seconds", "0.2"], capture_output=True, text=True, timeout=600,
+                       cwd=ROOT, env=env)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [ln for ln in r.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, r.stdout
+    d = json.loads(lines[0])
+    assert d["n_gpus"] == 2 and d["impl"] == "reference"
+
+
+def test_bench_refuses_a_mismatched_world():
+    """Under a launcher whose WORLD_SIZE differs from --gpus the script stops at once."""
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl",
+                        "reference", "--workload", "tiny-f32-2k"], capture_output=True, text=True,
+                       timeout=300, cwd=ROOT, env=env)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr
 
 
 def test_forecast_vectors_are_group_mean_queries():

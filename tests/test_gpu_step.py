@@ -1,14 +1,15 @@
-"""The fused decode step, vs the CPU oracle, through the C ABI.
+"""The fused decode step (bsa_decode_step_fused), vs the CPU oracle, through the C ABI.
 
 For bf16 caches whose blocks are four windows long (BS = 4s, l = s or 2s, BS a multiple of 64; the
-paper's 64 / 16 / 32), bsa_decode_step runs one kernel in which a CTA takes a whole (batch, kv-head)
-pair: it scores the pair's compressed keys (window terms kept in tensor memory), selects its blocks
-and attends them. Other geometries chain the separate kernels behind the same entry point. These
-cases cover every padded group size, both head dims, both window lengths, blocks of 64 and 128
-tokens, ragged lengths (down to no window and an empty sequence), last blocks cut inside either
-32-token half, more pairs than SMs (the persistent loop over pairs) and the selection edge cases
-(top-k covering every candidate, k = 0, no init or local blocks), plus geometries of the chained
-path.
+paper's 64 / 16 / 32), bsa_decode_step_fused runs one kernel in which a CTA takes a whole
+(batch, kv-head) pair: it scores the pair's compressed keys (window terms kept in tensor memory),
+selects its blocks and attends them. bsa_decode_step takes that path when there are enough pairs to
+keep most SMs streaming, else it chains the separate kernels. These cases cover every padded group
+size, both head dims, both window lengths, blocks of 64 and 128 tokens, ragged lengths (down to no
+window and an empty sequence), last blocks cut inside either 32-token half, more pairs than SMs
+(the persistent loop over pairs) and the selection edge cases (top-k covering every candidate,
+k = 0, no init or local blocks); geometries the fused kernel does not take run through
+bsa_decode_step's chained path.
 """
 import numpy as np
 import pytest
@@ -68,11 +69,18 @@ def _run(case):
     return w, run
 
 
+def _fused_ok(w) -> bool:
+    """The fused kernel's geometry (bf16, BS = 4s, l = s or 2s, BS a multiple of 64, a cache of at
+    least one window)."""
+    return (w.dtype == "bf16" and w.block_size == 4 * w.cmp_stride and w.block_size % 64 == 0
+            and w.cmp_kernel in (w.cmp_stride, 2 * w.cmp_stride) and w.seq_len >= w.cmp_kernel)
+
+
 @pytest.mark.parametrize("case", sorted(STEP))
 def test_step_matches_oracle(case, cuda_device):
     w, run = _run(case)
     assert bsa.bsa_get_sizes(run.p).workspace_bytes > 0
-    run.step()
+    run.step(fused=_fused_ok(w))
     assert run.device_errors() == 0
     full_check(run, sample_pairs(w, 48))
 
@@ -84,7 +92,7 @@ def test_step_selection_equals_separate_selection(case, cuda_device):
     """The step's block scores and selection are those of bsa_select_blocks, bit for bit: both
     weigh the same stored window terms by the same per-chunk softmax weights."""
     w, run = _run(case)
-    run.step()
+    run.step(fused=_fused_ok(w))
     got = (run.block_idx.clone(), run.n_sel.clone(), run.block_scores.clone())
     run.select()
     assert torch.equal(got[0], run.block_idx)
@@ -95,7 +103,7 @@ def test_step_selection_equals_separate_selection(case, cuda_device):
 def test_step_empty_sequence_outputs(cuda_device):
     """A sequence of length 0 selects nothing and attends nothing: zero output, -inf LSE."""
     w, run = _run("ragged")
-    run.step()
+    run.step(fused=True)
     Hkv = w.num_kv_heads
     assert (run.n_sel.view(-1)[3 * Hkv:4 * Hkv] == 0).all()
     assert (run.block_idx[3] == -1).all()
@@ -105,12 +113,53 @@ def test_step_empty_sequence_outputs(cuda_device):
 def test_step_repeats_bit_for_bit(cuda_device):
     """Queued steps without a host sync give the first step's results bit for bit."""
     w, run = _run("more-pairs-than-sms")
-    run.step()
+    run.step(fused=True)
     torch.cuda.synchronize()
     first = (run.block_idx.clone(), run.out[0].clone(), run.lse[0].clone())
     for _ in range(30):
-        run.step()
+        run.step(fused=True)
     torch.cuda.synchronize()
     assert run.device_errors() == 0
     for a, b in zip(first, (run.block_idx, run.out[0], run.lse[0])):
+        assert torch.equal(a, b)
+
+
+def test_step_path_choice_and_unsupported_geometry(cuda_device):
+    """bsa_decode_step takes the fused kernel only with enough pairs to fill most SMs; the fused
+    entry point refuses a geometry it does not handle (blocks of eight strides) on the host."""
+    small, _ = STEP["g4-d128-ragged"]
+    big, _ = STEP["more-pairs-than-sms"]
+    for w, want in ((small, False), (big, True)):
+        p = bsa.make_params(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, w.seq_len, w.dtype,
+                            w.n_init, w.n_local, w.top_k, w.cmp_kernel, w.cmp_stride, w.block_size)
+        assert bsa.bsa_decode_step_info(p)[0] is want
+    w, run = _run("g4-bs128")
+    with pytest.raises(bsa.BsaError) as e:
+        run.step(fused=True)
+    assert e.value.status == bsa.BSA_ERR_UNSUPPORTED
+
+
+def test_fused_step_graph_replay(cuda_device):
+    """The fused step captured in a CUDA graph (its launch attributes included) and replayed gives
+    the eager call's results bit for bit."""
+    w, run = _run("more-pairs-than-sms")
+    run.step(fused=True)
+    torch.cuda.synchronize()
+    ref = (run.block_idx.clone(), run.out[0].clone(), run.lse[0].clone())
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(graph, stream=s):
+            bsa.bsa_decode_step(run.p, run.q[0], run.data["k"][0], run.data["v"][0], run.ck[0],
+                                None, None, run.data["seq_lens"], run.block_idx, run.n_sel, None,
+                                run.out[0], run.lse[0], run.ws, stream=s, fused=True)
+    torch.cuda.current_stream().wait_stream(s)
+    run.out[0].fill_(0)
+    run.block_idx.fill_(-5)
+    for _ in range(3):
+        graph.replay()
+    torch.cuda.synchronize()
+    assert run.device_errors() == 0
+    for a, b in zip(ref, (run.block_idx, run.out[0], run.lse[0])):
         assert torch.equal(a, b)
