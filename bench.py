@@ -389,8 +389,8 @@ def kernel_source_hash(kernel: str | None = None) -> str:
         paths = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")))
     else:
         own = next(f for k, f in KERNEL_SOURCES.items() if kernel.startswith(k))
-        paths = [os.path.join(csrc, n) for n in (own, "bsa_internal.cuh", "bsa_api.cu", "tiles.cuh",
-                                                 "topk.cuh")]
+        # the kernel's own file and the device headers (the host-side launch code is left out)
+        paths = [os.path.join(csrc, n) for n in (own, "bsa_internal.cuh", "tiles.cuh", "topk.cuh")]
     h = hashlib.sha256()
     for p in paths:
         with open(p, encoding="utf-8") as f:
@@ -399,18 +399,28 @@ def kernel_source_hash(kernel: str | None = None) -> str:
 
 
 def profile_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on the kernel's current
-    sources (the summary records their hash: kernel_source_hash(kernel))."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
-    try:
+    """DRAM bytes per launch from the committed ncu summaries of the workload, if they were taken on
+    the kernel's current sources (each summary records their hash: kernel_source_hash(kernel)).
+
+    A summary ``profiles/<name>_<workload>.md`` gives, per kernel, the lines
+    ``dram_bytes_per_launch[<kernel>]: N`` and ``kernel_sources_sha256_16[<kernel>]: H`` (or, in
+    ``profiles/<kernel>_<workload>.md``, the same two lines without the bracket). A phase of two
+    kernels ("a+b") adds up both kernels' bytes."""
+    if "+" in kernel:
+        parts = [profile_traffic(k, workload) for k in kernel.split("+")]
+        return None if any(v is None for v in parts) else sum(parts)
+    import glob
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", f"*_{workload}.md"))):
         text = open(path).read()
-    except OSError:
-        return None
-    m = re.search(r"dram_bytes_per_launch:\s*([\d.eE+]+)", text)
-    hm = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
-    if not m or not hm or hm.group(1) != kernel_source_hash(kernel):
-        return None
-    return float(m.group(1))
+        tag = re.escape(f"[{kernel}]")
+        m = re.search(r"dram_bytes_per_launch" + tag + r":\s*([\d.eE+]+)", text)
+        hm = re.search(r"kernel_sources_sha256_16" + tag + r":\s*([0-9a-f]+)", text)
+        if not m and os.path.basename(path) == f"{kernel}_{workload}.md":
+            m = re.search(r"dram_bytes_per_launch:\s*([\d.eE+]+)", text)
+            hm = re.search(r"kernel_sources_sha256_16:\s*([0-9a-f]+)", text)
+        if m and hm:
+            return float(m.group(1)) if hm.group(1) == kernel_source_hash(kernel) else None
+    return None
 
 
 # ------------------------------------------------------------------------------- CPU (oracle) leg

@@ -28,16 +28,25 @@ def test_kernel_source_hash_covers_each_kernel():
 
 
 def test_profile_summaries_parse():
-    """Every committed DRAM summary states its bytes per launch and a source fingerprint."""
+    """Every committed DRAM summary states, per kernel, its bytes per launch and a source
+    fingerprint, and the bench finds the figure of the kernel it reports for each summarised
+    workload (when the summary's fingerprint is the kernel's current one)."""
     import re
+    import bench
     pdir = os.path.join(ROOT, "profiles")
-    names = [n for n in os.listdir(pdir) if n.endswith(".md") and "kernel_" in n]
+    names = [n for n in os.listdir(pdir) if n.endswith(".md") and not n.startswith("launches_")]
     assert names
     for n in names:
         text = open(os.path.join(pdir, n)).read()
-        assert re.search(r"kernel_sources_sha256_16:\s*[0-9a-f]{16}", text), n
-        if n.startswith(("decode_tma_kernel", "score_tma_kernel")):
-            assert re.search(r"dram_bytes_per_launch:\s*\d+", text), n
+        tagged = re.findall(r"dram_bytes_per_launch\[(\w+)\]:\s*\d+", text)
+        assert tagged, n
+        for k in tagged:
+            assert re.search(r"kernel_sources_sha256_16\[" + k + r"\]:\s*[0-9a-f]{16}", text), (n, k)
+        for wl in WORKLOADS:
+            if n.endswith(f"_{wl}.md"):
+                for k in tagged:
+                    got = bench.profile_traffic(k, wl)
+                    assert got is None or got > 0, (n, k)
 
 
 @pytest.mark.parametrize("name", sorted(WORKLOADS))
