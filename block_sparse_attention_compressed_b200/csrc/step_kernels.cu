@@ -45,6 +45,7 @@ constexpr int kConsumerBar = 1;               // named barrier of the consumer w
 constexpr int kHandBar = 2;                   // consumers + producers: the selection is handed over
 constexpr int kPairBar0 = 3;                  // 3..6: the two scoring warps of a TMEM lane quarter
 constexpr uint32_t kStepWaitPolls = 1u << 26;
+constexpr int kPrefetchChunks = 16;           // compressed-key chunks prefetched into L2 at start-up
 static_assert(kStepSlots % (2 * kStepScorers) == 0, "a scoring slot serves one consumer warp");
 static_assert(kStepSlots % 4 == 0, "an attention slot serves one group of four warps");
 static_assert(kStepSlots % kStepProducers == 0, "a slot is refilled by one producer");
@@ -134,6 +135,14 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     tmem_fence_after_sync();
     const uint32_t tbase = s_tmem;
     pdl_trigger();
+    if (warp >= kStepConsumers && (int)blockIdx.x < a.pairs) {
+        // while the previous kernel finishes, the first compressed-key chunks of this CTA's first
+        // pair stream into L2 (a prefetch reads nothing into the CTA, so it needs no dependency;
+        // the chunk count comes from the capacity, since the sequence lengths may not be final)
+        const int nbox = min(kPrefetchChunks, (int)((a.nc_cap + 63) / 64)) * NB;
+        for (int e = (warp - kStepConsumers) * 32 + lane; e < nbox; e += kStepProducers * 32)
+            tma_prefetch_2d(&maps.ck, 64 * (e % NB), (int)((int64_t)blockIdx.x * a.nc_cap + 64 * (e / NB)));
+    }
     pdl_wait();
 
     if (warp >= kStepConsumers) {

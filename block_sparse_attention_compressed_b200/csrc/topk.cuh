@@ -47,10 +47,10 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 // first digit of up to kFirstDigitBits bits (one histogram bin per value, found with a two-level
 // descending scan), then 8-bit digits. When that bucket holds exactly the number of keys still
 // needed, all of them are taken with those above it. Otherwise, as soon as the bucket has at most
-// kExactMax keys, the owners of those keys rank them exactly among themselves (score descending,
-// block ascending); the taken candidates are those above the bucket plus the bucket keys ranked
-// below the number still needed. Otherwise the ties at the final key value are taken in block
-// order.
+// kExactMax keys, they are gathered and each is ranked exactly against the others (score
+// descending, block ascending) by its own team of threads; the taken candidates are those above
+// the bucket plus the bucket keys ranked below the number still needed. Otherwise the ties at the
+// final key value are taken in block order. Thread groups have kExactMax threads or more.
 constexpr int kKeysPerThread = 8;
 constexpr int kFirstDigitBits = 12;
 constexpr int kExactMax = 128;
@@ -298,27 +298,35 @@ __device__ void topk_union(const SelectArgs& a, int nb, uint32_t* keys, TopkSmem
             }
             gp.sync();
             const int ebn = min(t.bn, kExactMax);
+            const uint4* bk4 = reinterpret_cast<const uint4*>(s_bkey);
+            const int4* bi4 = reinterpret_cast<const int4*>(s_bidx);
+            // entries of the bucket ahead of key u at block idx (four per 16-byte read; the zero
+            // pads never count), over the quads q0, q0 + dq, ...
+            auto ahead = [&](uint32_t u, int idx, int q0, int dq) {
+                int rank = 0;
+                for (int q = q0; q < (ebn + 3) / 4; q += dq) {
+                    const uint4 kq = bk4[q];
+                    const int4 iq = bi4[q];
+                    rank += (kq.x > u || (kq.x == u && iq.x < idx)) + (kq.y > u || (kq.y == u && iq.y < idx)) +
+                            (kq.z > u || (kq.z == u && iq.z < idx)) + (kq.w > u || (kq.w == u && iq.w < idx));
+                }
+                return rank;
+            };
+            {
+                // each entry is ranked by a team of NT / kExactMax consecutive lanes, which marks it
+                // taken or not in keys[] at its block (its owner may hold several entries)
+                const int team = NT / kExactMax;  // 1, 2, 4 or 8 (NT = 128 .. 1024)
+                const int j = tid / team, r = tid - j * team;
+                int rank = j < ebn ? ahead(s_bkey[j], s_bidx[j], r, team) : 0;
+                for (int off = 1; off < team; off <<= 1) rank += __shfl_xor_sync(0xffffffffu, rank, off);
+                if (j < ebn && r == 0) keys[s_bidx[j]] = rank < need ? 1u : 0u;
+                gp.sync();
 #pragma unroll
-            for (int e = 0; e < kKeysPerThread; ++e) {
-                fl[e] = false;
-                if (seg_lo + e < seg_hi) {
-                    const uint32_t u = kr[e], mk = u & emask;
-                    if (mk > eprefix) {
-                        fl[e] = true;
-                    } else if (mk == eprefix) {
-                        // four bucket entries per 16-byte read; the zero pads never count
-                        const int idx = seg_lo + e;
-                        const uint4* bk4 = reinterpret_cast<const uint4*>(s_bkey);
-                        const int4* bi4 = reinterpret_cast<const int4*>(s_bidx);
-                        int rank = 0;
-#pragma unroll 4
-                        for (int q = 0; q < (ebn + 3) / 4; ++q) {
-                            const uint4 kq = bk4[q];
-                            const int4 iq = bi4[q];
-                            rank += (kq.x > u || (kq.x == u && iq.x < idx)) + (kq.y > u || (kq.y == u && iq.y < idx)) +
-                                    (kq.z > u || (kq.z == u && iq.z < idx)) + (kq.w > u || (kq.w == u && iq.w < idx));
-                        }
-                        fl[e] = rank < need;
+                for (int e = 0; e < kKeysPerThread; ++e) {
+                    fl[e] = false;
+                    if (seg_lo + e < seg_hi) {
+                        const uint32_t mk = kr[e] & emask;
+                        fl[e] = mk > eprefix || (mk == eprefix && keys[seg_lo + e] == 1u);
                     }
                 }
             }
