@@ -102,6 +102,8 @@ def _bind(path: str):
                                         _P, _P, _P, _P, _P, _P]),
         "bsa_oracle_decode_forecast_ck": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _P, _P, _P,
                                                  _INT, _P, _P, _P, _P, _P, _P]),
+        "bsa_oracle_select_forecast_ck": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _INT,
+                                                 _P, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -367,6 +369,44 @@ def decode_forecast(P: Problem, f, q, k_cache, v_cache, seq_lens, pairs=None, ck
     if rc != 0:
         raise ValueError("bsa_oracle_decode_forecast rejected its arguments")
     return res
+
+
+def select_forecast(P: Problem, f, ck, seq_lens, pairs=None) -> dict:
+    """The Forecast selection alone (SparDA Architecture, Eq. 4): the blocks that f [B][Hkv][d]
+    (storage array of the problem's dtype) chooses among the compressed keys ck (float64
+    [n][nc_cap][d], as ``compress_cache`` returns them for the same pairs). Returns idx, n_sel,
+    block_scores and boundary as ``decode``."""
+    f = _raw_check(f, P.dtype)
+    seq_lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    if pairs is None:
+        pairs = np.arange(P.batch * P.num_kv_heads, dtype=np.int32)
+    pairs = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32))
+    n = pairs.size
+    G, sel_cap, nb_cap = _sizes(P)
+    nc_cap = num_windows(P.max_seq_len, P.cmp_kernel, P.cmp_stride)
+    ck = np.ascontiguousarray(np.asarray(ck, dtype=np.float64))
+    if ck.shape != (n, max(nc_cap, 0), P.head_dim):
+        raise ValueError(f"ck must be [{n}][{nc_cap}][{P.head_dim}] float64")
+    res = dict(idx=np.full((n, sel_cap), -1, dtype=np.int32), n_sel=np.zeros(n, dtype=np.int32),
+               block_scores=np.full((n, nb_cap), -np.inf, dtype=np.float64),
+               boundary=np.full((n, 2), np.nan, dtype=np.float64))
+    rc = _load().bsa_oracle_select_forecast_ck(
+        ctypes.byref(P), _ptr(f), _ptr(ck), _ptr(seq_lens), _ptr(pairs), n, _ptr(res["idx"]),
+        _ptr(res["n_sel"]), _ptr(res["block_scores"]), _ptr(res["boundary"]))
+    if rc != 0:
+        raise ValueError("bsa_oracle_select_forecast_ck rejected its arguments")
+    return res
+
+
+def lookahead_step(P: Problem, q, k_cache, v_cache, idx, n_sel, f, ck_next, seq_lens,
+                   pairs=None) -> dict:
+    """One layer l of one-layer-lookahead decoding (SparDA Architecture, Eqs. 4 and 5): layer l's
+    queries attend the blocks chosen for it beforehand (idx, n_sel), and layer l + 1's blocks are
+    chosen from layer l's Forecast vectors f against layer l + 1's compressed keys ck_next.
+    Returns out, lse (layer l) and idx, n_sel, block_scores, boundary (layer l + 1)."""
+    att = attend_pairs(P, q, k_cache, v_cache, seq_lens, idx, n_sel, pairs)
+    nxt = select_forecast(P, f, ck_next, seq_lens, pairs)
+    return dict(out=att["out"], lse=att["lse"], **nxt)
 
 
 def attend_pairs(P: Problem, q, k_cache, v_cache, seq_lens, idx, n_sel, pairs=None) -> dict:

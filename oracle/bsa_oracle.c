@@ -237,7 +237,8 @@ static const void* orc_pair_rows(const orc_problem_t* P, const void* cache, int 
 
 /* Select (from q, or from the Forecast vectors f when given) and attend, per listed pair. The
  * compressed keys are formed from the cache (Eq. 2), or taken from ck_given [n_pairs][nc_cap][d]
- * (already rounded, as bsa_oracle_compress_cache writes them) when that is not NULL. */
+ * (already rounded, as bsa_oracle_compress_cache writes them) when that is not NULL. With out ==
+ * NULL (and f and ck_given given) only the selection runs: q, k_cache and v_cache are not read. */
 static int orc_decode(const orc_problem_t* P, const void* f, const void* q, const void* k_cache,
                       const void* v_cache, const double* ck_given, const int32_t* seq_lens,
                       const int32_t* pairs, int n_pairs, const int32_t* given_idx,
@@ -258,10 +259,11 @@ static int orc_decode(const orc_problem_t* P, const void* f, const void* q, cons
         const int pair = pairs[i], b = pair / P->num_kv_heads, kvh = pair % P->num_kv_heads;
         const int64_t T = seq_lens[b];
         const int64_t nb = bsa_oracle_num_blocks(T, P->block_size);
-        const void* kp = orc_pair_rows(P, k_cache, pair);
-        const void* vp = orc_pair_rows(P, v_cache, pair);
+        const int attend = out != NULL;
+        const void* kp = attend || !ck_given ? orc_pair_rows(P, k_cache, pair) : NULL;
+        const void* vp = attend ? orc_pair_rows(P, v_cache, pair) : NULL;
         double* qg = (double*)malloc((size_t)G * d * sizeof(double));
-        orc_group_q(P, q, b, kvh, qg);
+        if (attend || !f) orc_group_q(P, q, b, kvh, qg);
         int32_t* my_idx = idx + (int64_t)i * sel_cap;
         for (int r = 0; r < sel_cap; ++r) my_idx[r] = -1;
         int ns;
@@ -309,8 +311,9 @@ static int orc_decode(const orc_problem_t* P, const void* f, const void* q, cons
             free(sb);
         }
         n_sel[i] = ns;
-        bsa_oracle_attend(qg, kp, vp, P->dtype, T, d, G, my_idx, ns, P->block_size, P->scale,
-                          out + (int64_t)i * G * d, lse + (int64_t)i * G);
+        if (attend)
+            bsa_oracle_attend(qg, kp, vp, P->dtype, T, d, G, my_idx, ns, P->block_size, P->scale,
+                              out + (int64_t)i * G * d, lse + (int64_t)i * G);
         free(qg);
     }
     return bad ? -1 : 0;
@@ -356,6 +359,17 @@ int bsa_oracle_decode_forecast_ck(const orc_problem_t* P, const void* f, const v
     if (!f || !ck) return -1;
     return orc_decode(P, f, q, k_cache, v_cache, ck, seq_lens, pairs, n_pairs, NULL, NULL, idx, n_sel,
                       block_scores, boundary, out, lse);
+}
+
+/* The selection of bsa_oracle_decode_forecast_ck alone (SparDA Architecture, Eq. 4): the blocks
+ * that the Forecast vectors f choose among the given compressed keys ck; with one-layer lookahead
+ * (the abstract's lookahead selection) f is layer l's and ck layer l + 1's. */
+int bsa_oracle_select_forecast_ck(const orc_problem_t* P, const void* f, const double* ck,
+                                  const int32_t* seq_lens, const int32_t* pairs, int n_pairs,
+                                  int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary) {
+    if (!f || !ck) return -1;
+    return orc_decode(P, f, NULL, NULL, NULL, ck, seq_lens, pairs, n_pairs, NULL, NULL, idx, n_sel,
+                      block_scores, boundary, NULL, NULL);
 }
 
 int bsa_oracle_attend_pairs(const orc_problem_t* P, const void* q, const void* k_cache,

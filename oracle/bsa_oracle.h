@@ -162,6 +162,12 @@ int bsa_oracle_decode_ck(const orc_problem_t* P, const void* q, const double* ck
                          const void* k_cache, const void* v_cache, const int32_t* seq_lens,
                          const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel,
                          double* block_scores, double* boundary, double* out, double* lse);
+/* The Forecast selection of bsa_oracle_decode_forecast_ck alone (no attention): f [B][Hkv][d]
+ * against the given compressed keys ck [n_pairs][nc_cap][d] (for one-layer lookahead, f of layer
+ * l and ck of layer l + 1). */
+int bsa_oracle_select_forecast_ck(const orc_problem_t* P, const void* f, const double* ck,
+                                  const int32_t* seq_lens, const int32_t* pairs, int n_pairs,
+                                  int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary);
 
 #ifdef __cplusplus
 }

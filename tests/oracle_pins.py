@@ -473,6 +473,45 @@ def pin_forecast_one_head_matches_base_selector():
     np.testing.assert_array_equal(fc2["block_scores"], 2.0 * fc["block_scores"])
 
 
+def pin_lookahead_step_brute_force():
+    """One-layer lookahead (SparDA Architecture, Eqs. 4-5): layer 0 attends the blocks given for it
+    (the gathered tokens through torch's SDPA, in float64), and layer 1's blocks are those whose
+    raw Forecast score f . K~_j (numpy dot products over the windows of each block) rank highest,
+    ties to the lower block, from a plain sort, united with the init and local blocks."""
+    B, Hq, Hkv, d, Tc = 1, 4, 2, 16, 64 * 14
+    q, k0, v0 = _randn((B, Hq, d), 97), _randn((B, Hkv, Tc, d), 98), _randn((B, Hkv, Tc, d), 99)
+    k1, f = _randn((B, Hkv, Tc, d), 100), _randn((B, Hkv, d), 101)
+    P = oracle.make_problem(B, Hq, Hkv, d, Tc, oracle.F32, 1, 2, 3)
+    T = 64 * 11 + 40
+    qn, k0n, v0n, k1n, fn = (x.numpy() for x in (q, k0, v0, k1, f))
+    idx0 = np.array([[0, 4, 5, 9, 11, -1], [0, 2, 7, 8, 10, 11]], dtype=np.int32)
+    nsel0 = np.array([5, 6], dtype=np.int32)
+    ck1 = oracle.compress_cache(P, k1n, [T])
+    res = oracle.lookahead_step(P, qn, k0n, v0n, idx0, nsel0, fn, ck1, [T])
+    G = Hq // Hkv
+    nb = -(-T // 64)
+    nc = (T - 32) // 16 + 1
+    for kvh in range(Hkv):
+        toks = [t for b in idx0[kvh, :nsel0[kvh]] for t in range(b * 64, min(b * 64 + 64, T))]
+        ro, rl = _sdpa(qn[0, kvh * G:(kvh + 1) * G].astype(np.float64), k0n[0, kvh, toks].astype(np.float64),
+                       v0n[0, kvh, toks].astype(np.float64), 1.0 / math.sqrt(d))
+        np.testing.assert_allclose(res["out"][kvh], ro, rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(res["lse"][kvh], rl, rtol=1e-12, atol=1e-13)
+        # layer 1: windows j cover tokens [16j, 16j + 32); block b takes the max over the windows
+        # that overlap its tokens
+        kk = k1n[0, kvh].astype(np.float64)
+        win = np.array([kk[16 * j:16 * j + 32].mean(0) for j in range(nc)])
+        win = win.astype(np.float32).astype(np.float64)  # the cache dtype (fp32) rounding
+        raw = win @ fn[0, kvh].astype(np.float64)
+        sb = [max(raw[j] for j in range(nc) if 16 * j < 64 * (b + 1) and 16 * j + 32 > 64 * b)
+              for b in range(nb)]
+        fixed = {0} | {nb - 2, nb - 1}
+        cand = sorted((b for b in range(nb) if b not in fixed), key=lambda b: (-sb[b], b))
+        want = sorted(fixed | set(cand[:3]))
+        assert res["idx"][kvh, :res["n_sel"][kvh]].tolist() == want
+        np.testing.assert_allclose(res["block_scores"][kvh, :nb], sb, rtol=1e-12, atol=1e-12)
+
+
 ALL_PINS = [
     pin_round_bf16_matches_torch, pin_round_ties_even, pin_round_f32_matches_numpy,
     pin_compress_matches_avg_pool, pin_compress_constant_windows, pin_window_and_block_counts,
@@ -487,4 +526,5 @@ ALL_PINS = [
     pin_decode_given_compressed_keys_composes,
     pin_shared_index_identical_layers,
     pin_forecast_decode_composes, pin_forecast_one_head_matches_base_selector,
+    pin_lookahead_step_brute_force,
 ]
