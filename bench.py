@@ -208,7 +208,18 @@ class Bench:
         single = w.layers == 1 and not w.forecast
         self.path = path if single else "auto"
         self.fused = single and (path == "fused" or (path == "auto" and bsa.bsa_decode_step_info(self.p)[0]))
-        if w.forecast and (w.layers > 1 or self.append):
+        self.lookahead = bool(w.lookahead)
+        if self.lookahead:
+            # layer 0 attends blocks chosen beforehand (here by its own queries, outside the timed
+            # region) while layer 1's are chosen from the Forecast vectors: one kernel per step
+            self.ck_next = torch.zeros_like(self.ck)
+            bsa.bsa_compress_keys(self.p, self.data["k"][1], self.data["seq_lens"], self.ck_next)
+            bsa.bsa_select_blocks(self.p, self.data["q"][0], self.ck, self.data["seq_lens"], self.block_idx,
+                                  self.n_sel, None, self.ws)
+            self.idx_next = torch.zeros_like(self.block_idx)
+            self.n_sel_next = torch.zeros_like(self.n_sel)
+            self.fused = True
+        elif w.forecast and (w.layers > 1 or self.append):
             raise ValueError("the Forecast-indexer workloads are single-layer, fixed-length")
         torch.cuda.synchronize()
 
@@ -220,6 +231,14 @@ class Bench:
         bsa, d = self.bsa, self.data
         q = self.q_of(i) if q is None else q
         ev = (lambda k: events[k].record(stream)) if events is not None else (lambda k: None)
+        if self.lookahead:
+            ev(0)
+            bsa.bsa_decode_step_lookahead(self.p, q, d["k"][0], d["v"][0], self.block_idx, self.n_sel,
+                                          d["f"], self.ck_next, d["seq_lens"], self.idx_next,
+                                          self.n_sel_next, None, self.out[0], self.lse[0], self.ws,
+                                          stream=stream)
+            ev(1)
+            return
         if self.w.forecast:
             ev(0)
             bsa.bsa_select_blocks_forecast(self.p, d["f"], self.ck, d["seq_lens"], self.block_idx,
@@ -284,6 +303,11 @@ class Bench:
     # Forecast-indexer workloads qs is [q, f]
     def step_io(self, qs, outs, lses, stream, k_new=None, v_new=None):
         bsa, d = self.bsa, self.data
+        if self.lookahead:
+            bsa.bsa_decode_step_lookahead(self.p, qs[0], d["k"][0], d["v"][0], self.block_idx, self.n_sel,
+                                          qs[1], self.ck_next, d["seq_lens"], self.idx_next,
+                                          self.n_sel_next, None, outs[0], lses[0], self.ws, stream=stream)
+            return
         if self.w.forecast:
             bsa.bsa_select_blocks_forecast(self.p, qs[1], self.ck, d["seq_lens"], self.block_idx,
                                            self.n_sel, None, self.ws, stream=stream)
@@ -455,9 +479,12 @@ def cpu_oracle_sample(w, data, seconds: float):
     f_arr = (oracle.raw(torch.stack([data["f"][b, h:h + 1] for b, h in pairs]))[0]
              if w.forecast else None)
     # A1, the compression of every scoring layer's keys (once per cache; timed apart)
+    scored = [1] if w.lookahead else list(w.anchors)
     t0 = time.perf_counter()
-    cks = {L: oracle.compress_cache(P, arrays[L][1], lens) for L in w.anchors}
-    compress_s = (time.perf_counter() - t0) * (total / n0)
+    cks = {L: oracle.compress_cache(P, arrays[L][1], lens) for L in scored}
+    compress_s = (time.perf_counter() - t0) * (total / n0) / len(scored)
+    # lookahead: layer 0's blocks, chosen beforehand (by its own queries; untimed)
+    sel0 = oracle.decode(P, *arrays[0], lens) if w.lookahead else None
 
     def one(sub=None):
         idx = slice(None) if sub is None else slice(0, sub)
@@ -470,6 +497,11 @@ def cpu_oracle_sample(w, data, seconds: float):
                 sub, G, 1, w.head_dim, T_cap, P.dtype, w.n_init, w.n_local, w.top_k, w.cmp_kernel,
                 w.cmp_stride, w.block_size)
             ln = lens if sub is None else lens[:sub]
+            if w.lookahead:
+                # layer 0 attends its blocks, layer 1's are chosen from the Forecast vectors
+                oracle.lookahead_step(Ps, q_, k_, v_, sel0["idx"][idx], sel0["n_sel"][idx], f_arr[idx],
+                                      cks[1][idx], ln)
+                return
             if w.forecast:
                 oracle.decode_forecast(Ps, f_arr[idx], q_, k_, v_, ln, ck=cks[0][idx])
             elif L in w.anchors:
@@ -490,7 +522,7 @@ def cpu_oracle_sample(w, data, seconds: float):
     dt, reps = timed(one, seconds)
     with oracle.threads(1):
         dt1, reps1 = timed(lambda: one(1), seconds / 4)   # one pair on one thread
-    layers = f" x {w.layers} layers" if w.layers > 1 else ""
+    layers = f" x {w.layers} layers" if w.layers > 1 and not w.lookahead else ""
     desc = (f"CPU oracle (fp64) decode step on {n0} of {total} (batch, kv-head) pairs{layers}: "
             f"scoring, block reduction, top-k and attention with the keys compressed beforehand "
             f"(their compression, {compress_s:.2f} s per full cache, is timed apart), "
@@ -621,7 +653,7 @@ def run_bsa(args, w, world, rank, local):
     # outputs (every layer) copied back, double-buffered: step i+1's inputs land and step i's
     # outputs return on copy streams while step i+1 computes
     import torch as _t
-    L_ = w.layers
+    L_ = 1 if w.lookahead else w.layers  # lookahead: one layer attends per step
     NBUF = 2
     def step_q(i):  # the query of every layer for timed step i (then the Forecast vectors)
         return ([bench.q_of(W + i if bench.append else 0)] + [bench.data["q"][l] for l in range(1, L_)]

@@ -81,6 +81,8 @@ _SIGS = {
                              ctypes.c_size_t, _P]),
     "bsa_decode_step_fused": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                    ctypes.c_size_t, _P]),
+    "bsa_decode_step_lookahead": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                       ctypes.c_size_t, _P]),
     "bsa_decode_step_anchored": (_S, [_PP, ctypes.c_int32, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
                                       _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "bsa_read_device_error": (_S, [_P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32), _P]),
@@ -365,6 +367,28 @@ def bsa_decode_step(p: Params, q, k_cache, v_cache, ck, k_new, v_new, seq_lens, 
         _ptr(out, "out", e, n["q"]), _ptr(lse, "lse", torch.float32, n["lse"], optional=True),
         _ptr(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
         name)
+
+
+def bsa_decode_step_lookahead(p: Params, q, k_cache, v_cache, block_idx, n_sel, f, ck_next, seq_lens,
+                              block_idx_next, n_sel_next, block_scores_next, out, lse, ws,
+                              stream=None):
+    """bsa_decode_step_lookahead: this layer attends block_idx / n_sel while the next layer's
+    blocks are chosen from f (one Forecast vector per (batch, kv head)) against ck_next."""
+    import torch
+    n, e = _shapes(p), _elem(p)
+    _check(lib().bsa_decode_step_lookahead(
+        ctypes.byref(p), _ptr(q, "q", e, n["q"]), _ptr(k_cache, "k_cache", e, n["cache"]),
+        _ptr(v_cache, "v_cache", e, n["cache"]),
+        _ptr(block_idx, "block_idx", torch.int32, n["idx"]),
+        _ptr(n_sel, "n_sel", torch.int32, n["pairs"]),
+        _ptr(f, "f", e, n["pairs"] * p.head_dim), _ptr(ck_next, "ck_next", e, n["ck"]),
+        _ptr(seq_lens, "seq_lens", torch.int32, p.batch),
+        _ptr(block_idx_next, "block_idx_next", torch.int32, n["idx"]),
+        _ptr(n_sel_next, "n_sel_next", torch.int32, n["pairs"]),
+        _ptr(block_scores_next, "block_scores_next", torch.float32, n["scores"], optional=True),
+        _ptr(out, "out", e, n["q"]), _ptr(lse, "lse", torch.float32, n["lse"], optional=True),
+        _ptr(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
+        "bsa_decode_step_lookahead")
 
 
 def bsa_read_device_error(ws, stream=None) -> int:

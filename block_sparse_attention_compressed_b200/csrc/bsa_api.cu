@@ -702,6 +702,42 @@ bsa_status_t bsa_decode_step_fused(const bsa_params_t* params, const void* q, vo
                        block_scores, out, lse, ws, ws_bytes, stream);
 }
 
+bsa_status_t bsa_decode_step_lookahead(const bsa_params_t* params, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* block_idx,
+                                       const int32_t* n_sel, const void* f, const void* ck_next,
+                                       const int32_t* seq_lens, int32_t* block_idx_next,
+                                       int32_t* n_sel_next, float* block_scores_next, void* out,
+                                       float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    Plan P;
+    bsa_status_t st = make_plan(params, &P);
+    if (st != BSA_OK) return st;
+    if (!P.step_fused) return BSA_ERR_UNSUPPORTED;
+    if (!ok16(q) || !ok16(k_cache) || !ok16(v_cache) || !ok16(f) || !ok16(ck_next) || !ok16(out) ||
+        !ok4(seq_lens) || !ok4(block_idx) || !ok4(n_sel) || !ok4(block_idx_next) || !ok4(n_sel_next))
+        return BSA_ERR_INVALID_ARG;
+    if ((block_scores_next && !ok4(block_scores_next)) || (lse && !ok4(lse))) return BSA_ERR_INVALID_ARG;
+    // the next layer's selection must not overwrite the blocks this layer reads
+    const size_t idx_bytes = (size_t)P.pairs * P.sel_cap * sizeof(int32_t), ns_bytes = (size_t)P.pairs * sizeof(int32_t);
+    auto overlap = [](const void* a, size_t na, const void* b, size_t nb) {
+        const char *x = static_cast<const char*>(a), *y = static_cast<const char*>(b);
+        return x < y + nb && y < x + na;
+    };
+    if (overlap(block_idx, idx_bytes, block_idx_next, idx_bytes) || overlap(block_idx, idx_bytes, n_sel_next, ns_bytes) ||
+        overlap(n_sel, ns_bytes, block_idx_next, idx_bytes) || overlap(n_sel, ns_bytes, n_sel_next, ns_bytes))
+        return BSA_ERR_INVALID_ARG;
+    if ((st = check_ws(P, ws, ws_bytes)) != BSA_OK) return st;
+    static thread_local StepMapCache c;
+    if (!encode_kv_map_cached(&c.maps.ck, &c.ck, ck_next, (uint64_t)P.pairs * P.nc_cap, P.D, 64) ||
+        !encode_kv_map_cached(&c.maps.k, &c.k, k_cache, (uint64_t)P.pairs * P.T_cap, P.D, 64) ||
+        !encode_kv_map_cached(&c.maps.v, &c.v, v_cache, (uint64_t)P.pairs * P.T_cap, P.D, 64))
+        return BSA_ERR_CUDA;
+    StepArgs a = step_args(P, q, f, seq_lens, block_idx_next, n_sel_next, block_scores_next, out, lse, ws);
+    a.in_idx = block_idx;
+    a.in_nsel = n_sel;
+    a.score_log2 = 1.f;  // the raw dot products
+    return from_cuda(launch_step(P, a, &c.maps, stream));
+}
+
 bsa_status_t bsa_decode_step_info(const bsa_params_t* params, int32_t append, int32_t* fused,
                                   int32_t* launches) {
     Plan P;

@@ -139,6 +139,10 @@ struct DecodeArgs {
 struct StepArgs {
     const void* q;         // [B][Hq][D] queries: the attention heads, and the scoring heads unless f
     const void* f;         // Forecast indexer: [B][Hkv][D] scoring vectors (raw scores), or null
+    // lookahead (with f): this layer's blocks, chosen beforehand ([pairs][sel_cap], [pairs]); the
+    // selection then goes to the next layer (block_idx, n_sel, from the next layer's compressed keys)
+    const int32_t* in_idx;
+    const int32_t* in_nsel;
     const int32_t* seq_lens;
     int32_t* block_idx;    // [pairs][sel_cap]
     int32_t* n_sel;        // [pairs]

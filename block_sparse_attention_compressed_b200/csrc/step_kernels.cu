@@ -44,6 +44,7 @@ constexpr uint32_t kEmptyCount = 4;             // arrivals that free a slot: an
 constexpr int kConsumerBar = 1;               // named barrier of the consumer warps
 constexpr int kHandBar = 2;                   // consumers + producers: the selection is handed over
 constexpr int kPairBar0 = 3;                  // 3..6: the two scoring warps of a TMEM lane quarter
+constexpr int kTopkBar = 7;                   // lookahead: the four warps that select the next layer's blocks
 constexpr uint32_t kStepWaitPolls = 1u << 26;
 constexpr int kPrefetchChunks = 16;           // compressed-key chunks prefetched into L2 at start-up
 static_assert(kStepSlots % (2 * kStepScorers) == 0, "a scoring slot serves one consumer warp");
@@ -80,13 +81,30 @@ __device__ __forceinline__ int block_units(int64_t T, int b, int BS) {
     return (int)((n + kUnitTokens - 1) / kUnitTokens);
 }
 
+// Lookahead: the attention units of the blocks given for this layer (entries outside [0, nb), such
+// as the -1 padding, are skipped).
+__device__ __forceinline__ int given_units(const StepArgs& a, const PairGeo& pg, int pair) {
+    const int nin = min(max(a.in_nsel[pair], 0), a.sel_cap);
+    int nu = 0;
+    for (int i = 0; i < nin; ++i) {
+        const int blk = a.in_idx[(size_t)pair * a.sel_cap + i];
+        if (blk >= 0 && blk < pg.nb) nu += block_units(pg.T, blk, a.BS);
+    }
+    return nu;
+}
+
 __device__ __forceinline__ bool aborted(const volatile int* s_abort) { return *s_abort != 0; }
 
 // SGP: scoring heads padded to a power of two (1 for the Forecast indexer's one vector); RAW: the
-// stored window terms are the raw scores (no softmax, weight 1).
-template <int D, int SGP, bool RAW>
+// stored window terms are the raw scores (no softmax, weight 1). LA (lookahead, with RAW): the
+// Forecast vectors score the NEXT layer's compressed keys (maps.ck) and choose that layer's blocks
+// (into block_idx / n_sel), while this layer attends the blocks chosen for it beforehand (in_idx /
+// in_nsel, maps.k / maps.v): those stream right behind the chunks, and once the block maxima are
+// taken four warps run the top-k while the other four attend.
+template <int D, int SGP, bool RAW, bool LA>
 __global__ void __launch_bounds__(kStepThreads, 1)
     step_kernel(const StepArgs a, const __grid_constant__ StepMaps maps) {
+    static_assert(!LA || (RAW && SGP == 1), "lookahead selection scores one Forecast vector");
     extern __shared__ uint8_t dsm_raw[];
     __shared__ __align__(8) uint64_t full[kStepSlots], empty[kStepSlots];
     __shared__ StepStage meta[kStepSlots];
@@ -206,24 +224,37 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                         tma_load_2d_hint(dst + bi * kBox, &maps.ck, 64 * bi, y, &full[slot], pol);
                     last_k[slot] = kk + 1;
                 }
-                // the init and local blocks are in every selection: their first stages load while
-                // the consumers select (as many as the ring holds without waiting for them)
                 int j = 0;
-                for (int b = 0; b < pg.init_end; ++b) issue_block(b, j, 0, kStepSlots);
-                for (int b = pg.chi; b < pg.nb; ++b) issue_block(b, j, 0, kStepSlots);
+                if constexpr (LA) {
+                    // this layer's blocks are known: all their stages follow the chunks
+                    const int nin = min(max(a.in_nsel[pair], 0), a.sel_cap);
+                    for (int i = 0; i < nin; ++i) {
+                        const int blk = a.in_idx[(size_t)pair * a.sel_cap + i];
+                        if (blk >= 0 && blk < pg.nb) issue_block(blk, j, 0, INT32_MAX);
+                    }
+                } else {
+                    // the init and local blocks are in every selection: their first stages load
+                    // while the consumers select (as many as the ring holds without waiting for them)
+                    for (int b = 0; b < pg.init_end; ++b) issue_block(b, j, 0, kStepSlots);
+                    for (int b = pg.chi; b < pg.nb; ++b) issue_block(b, j, 0, kStepSlots);
+                }
             }
             __syncwarp();
-            asm volatile("bar.sync %0, %1;" ::"r"(kHandBar), "r"(kStepThreads) : "memory");
-            if (lane == 0) {
-                // the rest: init / local stages beyond the ring, then the top-k blocks
-                int j = 0;
-                for (int b = 0; b < pg.init_end; ++b) issue_block(b, j, kStepSlots, INT32_MAX);
-                for (int b = pg.chi; b < pg.nb; ++b) issue_block(b, j, kStepSlots, INT32_MAX);
-                const int top_end = s_nsel - (pg.nb - pg.chi);
-                for (int i = pg.init_end; i < top_end; ++i) issue_block(sel[i], j, 0, INT32_MAX);
+            if constexpr (!LA) {
+                asm volatile("bar.sync %0, %1;" ::"r"(kHandBar), "r"(kStepThreads) : "memory");
+                if (lane == 0) {
+                    // the rest: init / local stages beyond the ring, then the top-k blocks
+                    int j = 0;
+                    for (int b = 0; b < pg.init_end; ++b) issue_block(b, j, kStepSlots, INT32_MAX);
+                    for (int b = pg.chi; b < pg.nb; ++b) issue_block(b, j, kStepSlots, INT32_MAX);
+                    const int top_end = s_nsel - (pg.nb - pg.chi);
+                    for (int i = pg.init_end; i < top_end; ++i) issue_block(sel[i], j, 0, INT32_MAX);
+                }
+                __syncwarp();
+                k = kd + s_ndec;
+            } else {
+                k = kd + 2 * given_units(a, pg, pair);
             }
-            __syncwarp();
-            k = kd + s_ndec;
         }
         // copies still in flight land before the CTA exits (all of them, on the normal path, have
         // been consumed already)
@@ -275,6 +306,7 @@ __global__ void __launch_bounds__(kStepThreads, 1)
             const uint32_t(&qs)[KS][2] = *reinterpret_cast<const uint32_t(*)[KS][2]>(RAW ? &qf_raw[0][0] : &qa[0][0]);
 
             topk_prepare(tk, grp);  // the top-k's bins, cleared while the first chunks load
+            if (LA && grp.tid == 0) s_ndec = 2 * given_units(a, pg, pair);  // read after the scoring's barrier
             // ---- scoring: tiles of two 64-window chunks. Chunk 2p of tile p is scored by warp p % 4 and
             // chunk 2p + 1 by warp p % 4 + 4, the two warps of TMEM lane quarter p % 4; they meet at a
             // named barrier and the first stores the tile, one block per lane: lane i holds block
@@ -474,47 +506,69 @@ __global__ void __launch_bounds__(kStepThreads, 1)
                     a.block_scores[(size_t)pair * a.nb_cap + blk] = -INFINITY;
             publish_andor(tk, kand, kor, grp);
             grp.sync();
-            topk_union(sa, pg.nb, keys, tk, true, grp, sel, &s_nsel);
-            grp.sync();
-            for (int i = grp.tid; i < a.sel_cap; i += grp.nt) a.block_idx[(size_t)pair * a.sel_cap + i] = sel[i];
-            if (grp.tid == 0) {
-                const int nsel = s_nsel;
-                a.n_sel[pair] = nsel;
-                // attention units: one per selected block at BS = 64, else counted block by block
-                int nu = nsel;
-                if (a.BS != kUnitTokens) {
-                    nu = 0;
-                    for (int blk = 0; blk < pg.init_end; ++blk) nu += block_units(pg.T, blk, a.BS);
-                    for (int blk = pg.chi; blk < pg.nb; ++blk) nu += block_units(pg.T, blk, a.BS);
-                    for (int i = pg.init_end; i < nsel - (pg.nb - pg.chi); ++i) nu += block_units(pg.T, sel[i], a.BS);
-                }
-                s_ndec = 2 * nu;
-            }
-            asm volatile("bar.sync %0, %1;" ::"r"(kHandBar), "r"(kStepThreads) : "memory");
 
-            // ---- attention: units i of group i % 2, 16 tokens per warp: the K stage gives the
-            // scores and probabilities, the V stage the numerators
-            const int n_dec = s_ndec;
-            const int64_t kd = k;
-            const int r0 = 16 * (w & 3);
+            // attention: units i0, i0 + di, ... of this pair's blocks (stages kd + 2i for the K rows
+            // and kd + 2i + 1 for the V rows), 16 tokens per warp: the K stage gives the scores and
+            // probabilities, the V stage the numerators
             AttnState<D> as;
             as.reset();
-            for (int i = w >> 2; 2 * i < n_dec; i += 2) {
-                const int ks_ = await_stage(kd + 2 * i);
-                const StepStage md = meta[ks_];
-                PFrag pf;
-                if (r0 < md.nvalid)
-                    pf = attn_scores16<D>(ring + (size_t)ks_ * kSlotBytes, kBox, r0, md.nvalid, qa, a.scale_log2, as, lane);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[ks_]);
-                const int vs_ = await_stage(kd + 2 * i + 1);
-                if (r0 < md.nvalid) attn_accum16<D>(ring + (size_t)vs_ * kSlotBytes, kBox, r0, md.nvalid, pf, as, lane);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&empty[vs_]);
+            auto attend_units = [&](int64_t kd, int n_dec, int i0, int di) {
+                const int r0 = 16 * (w & 3);
+                for (int i = i0; 2 * i < n_dec; i += di) {
+                    const int ks_ = await_stage(kd + 2 * i);
+                    const StepStage md = meta[ks_];
+                    PFrag pf;
+                    if (r0 < md.nvalid)
+                        pf = attn_scores16<D>(ring + (size_t)ks_ * kSlotBytes, kBox, r0, md.nvalid, qa, a.scale_log2, as, lane);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[ks_]);
+                    const int vs_ = await_stage(kd + 2 * i + 1);
+                    if (r0 < md.nvalid) attn_accum16<D>(ring + (size_t)vs_ * kSlotBytes, kBox, r0, md.nvalid, pf, as, lane);
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&empty[vs_]);
+                }
+            };
+            if constexpr (LA) {
+                // warps 0-3 choose the next layer's blocks while warps 4-7 attend this layer's
+                // (all its units, in order: a slot is always refilled for the same four warps)
+                const int n_dec = s_ndec;
+                if (w < 4) {
+                    const Grp ga{(int)threadIdx.x, 4 * 32, kTopkBar};
+                    topk_union(sa, pg.nb, keys, tk, false, ga, sel, &s_nsel);
+                    ga.sync();
+                    for (int i = ga.tid; i < a.sel_cap; i += ga.nt) a.block_idx[(size_t)pair * a.sel_cap + i] = sel[i];
+                    if (ga.tid == 0) a.n_sel[pair] = s_nsel;
+                } else {
+                    attend_units(k, n_dec, 0, 1);
+                }
+                k += n_dec;
+            } else {
+                topk_union(sa, pg.nb, keys, tk, true, grp, sel, &s_nsel);
+                grp.sync();
+                for (int i = grp.tid; i < a.sel_cap; i += grp.nt) a.block_idx[(size_t)pair * a.sel_cap + i] = sel[i];
+                if (grp.tid == 0) {
+                    const int nsel = s_nsel;
+                    a.n_sel[pair] = nsel;
+                    // attention units: one per selected block at BS = 64, else counted block by block
+                    int nu = nsel;
+                    if (a.BS != kUnitTokens) {
+                        nu = 0;
+                        for (int blk = 0; blk < pg.init_end; ++blk) nu += block_units(pg.T, blk, a.BS);
+                        for (int blk = pg.chi; blk < pg.nb; ++blk) nu += block_units(pg.T, blk, a.BS);
+                        for (int i = pg.init_end; i < nsel - (pg.nb - pg.chi); ++i) nu += block_units(pg.T, sel[i], a.BS);
+                    }
+                    s_ndec = 2 * nu;
+                }
+                asm volatile("bar.sync %0, %1;" ::"r"(kHandBar), "r"(kStepThreads) : "memory");
+                // units i of group i % 2
+                const int n_dec = s_ndec;
+                attend_units(k, n_dec, w >> 2, 2);
+                k += n_dec;
             }
-            k = kd + n_dec;
 
-            // ---- the eight warps' states merge into O and LSE
+            // ---- the eight warps' states merge into O and LSE (the merge area lies over the keys,
+            // which the lookahead's top-k may still be using)
+            if constexpr (LA) grp.sync();
 #pragma unroll
             for (int off = 4; off < 32; off <<= 1) {
                 as.lsum[0] += __shfl_xor_sync(0xffffffffu, as.lsum[0], off);
@@ -575,23 +629,24 @@ __global__ void __launch_bounds__(kStepThreads, 1)
     if (warp == 0) tmem_dealloc(tbase, a.tmem_cols);
 }
 
-template <int D, int SGP, bool RAW>
+template <int D, int SGP, bool RAW, bool LA>
 cudaError_t launch_step_k(const Plan& p, const StepArgs& a, const StepMaps* maps, cudaStream_t st) {
     if (a.pairs <= 0) return cudaSuccess;
-    cudaError_t e = ensure_smem<step_kernel<D, SGP, RAW>>(p.step_smem);
+    cudaError_t e = ensure_smem<step_kernel<D, SGP, RAW, LA>>(p.step_smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(step_kernel<D, SGP, RAW>, dim3((unsigned)p.step_ctas), dim3(kStepThreads), p.step_smem, st,
-                      a, *maps);
+    return launch_pdl(step_kernel<D, SGP, RAW, LA>, dim3((unsigned)p.step_ctas), dim3(kStepThreads), p.step_smem,
+                      st, a, *maps);
 }
 
 template <int D>
 cudaError_t launch_step_d(const Plan& p, const StepArgs& a, const StepMaps* maps, cudaStream_t st) {
-    if (a.f) return launch_step_k<D, 1, true>(p, a, maps, st);
+    if (a.in_idx) return launch_step_k<D, 1, true, true>(p, a, maps, st);
+    if (a.f) return launch_step_k<D, 1, true, false>(p, a, maps, st);
     switch (p.step_sgp) {
-        case 1: return launch_step_k<D, 1, false>(p, a, maps, st);
-        case 2: return launch_step_k<D, 2, false>(p, a, maps, st);
-        case 4: return launch_step_k<D, 4, false>(p, a, maps, st);
-        default: return launch_step_k<D, 8, false>(p, a, maps, st);
+        case 1: return launch_step_k<D, 1, false, false>(p, a, maps, st);
+        case 2: return launch_step_k<D, 2, false, false>(p, a, maps, st);
+        case 4: return launch_step_k<D, 4, false, false>(p, a, maps, st);
+        default: return launch_step_k<D, 8, false, false>(p, a, maps, st);
     }
 }
 

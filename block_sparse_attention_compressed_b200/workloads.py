@@ -47,6 +47,7 @@ class Workload:
     block_size: int = 64
     needle_shift: float = 2.0
     forecast: bool = False  # select with one Forecast vector per GQA group (f = the group's mean q)
+    lookahead: bool = False  # (two layers, forecast) layer 0 attends given blocks and selects layer 1's
     anchors: tuple = (0,)   # multi-layer: layers that select; the others reuse the last anchor's
 
     @property
@@ -65,7 +66,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The decode workloads: one small parity case and six throughput cases.
+# The decode workloads: one small parity case and seven throughput cases.
 WORKLOADS: dict[str, Workload] = {
     w.name: w
     for w in [
@@ -88,6 +89,9 @@ WORKLOADS: dict[str, Workload] = {
         Workload("anchors-2of4-64k-b8", batch=8, num_q_heads=32, num_kv_heads=8, head_dim=128,
                  seq_len=65536, dtype="bf16", n_init=1, n_local=2, top_k=48, needles=8, seed=1007,
                  layers=4, anchors=(0, 2)),
+        Workload("lookahead-bf16-128k-b16", batch=16, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                 seq_len=131072, dtype="bf16", n_init=1, n_local=4, top_k=64, needles=16,
+                 seed=1008, layers=2, forecast=True, lookahead=True),
     ]
 }
 DEFAULT_WORKLOAD = "gqa4-bf16-128k-b16"
@@ -132,6 +136,7 @@ def generate(w: Workload, device="cpu", seq_cap: int | None = None, steps: int |
       needles  [B][Hkv][n] numpy      needle block positions
       f        [B][Hkv][d]            Forecast vectors (forecast workloads): the mean of each
                                       group's query vectors of the first layer, in the cache type
+                                      (lookahead: of the second layer, the one f selects for)
     and, when ``steps`` > 0 (growing-cache workload):
       q_steps  [steps][B][Hq][d], k_new / v_new [steps][B][Hkv][d]
     ``seq_cap`` is the cache capacity T_cap (default: seq_len + steps).
@@ -177,7 +182,8 @@ def generate(w: Workload, device="cpu", seq_cap: int | None = None, steps: int |
         needles=blocks, seq_cap=T_cap,
     )
     if w.forecast:
-        q0 = res["q"][0].float().view(w.batch, w.num_kv_heads, w.group, w.head_dim)
+        qf = res["q"][1 if w.lookahead and len(out_q) > 1 else 0]
+        q0 = qf.float().view(w.batch, w.num_kv_heads, w.group, w.head_dim)
         res["f"] = q0.mean(dim=2).to(dt).contiguous()
     res.update(extra)
     return res
@@ -198,8 +204,9 @@ def algorithmic_bytes(w: Workload, T: int | None = None) -> dict:
     if w.n_local > 0 or n_sel == nb:          # the last (possibly partial) block is selected
         sel_tokens -= nb * w.block_size - T
     ck = pairs * nc * d * e * len(w.anchors)   # every anchor layer scores its compressed keys
-    kv = w.layers * pairs * sel_tokens * d * e * 2
-    qo = w.layers * w.batch * w.num_q_heads * d * e * 2
+    attended = 1 if w.lookahead else w.layers  # lookahead: one layer attends, the next one is scored
+    kv = attended * pairs * sel_tokens * d * e * 2
+    qo = attended * w.batch * w.num_q_heads * d * e * 2
     app = 0
     if w.append_steps:
         app = pairs * d * e * 4 + pairs * (w.cmp_kernel + 1) * d * e / w.cmp_stride

@@ -250,6 +250,33 @@ bsa_status_t bsa_decode_step_fused(const bsa_params_t* params, const void* q, vo
                                    float* block_scores, void* out, float* lse, void* workspace,
                                    size_t workspace_bytes, cudaStream_t stream);
 
+/* One layer l of one-layer-lookahead decoding (page "SparDA: Sparse Decoupled Attention for
+ * Efficient Long-Context LLM Inference", SparDA Architecture, Eqs. 4 and 5, and the lookahead
+ * selection of its abstract): layer l attends the blocks chosen for it beforehand while layer
+ * l + 1's blocks are chosen from layer l's Forecast vectors, in the same kernel.
+ *   attention (Eq. 5): q (this layer's queries, [batch][num_q_heads][head_dim]) over the tokens of
+ *     the blocks in block_idx / n_sel ([batch][num_kv_heads][n_init + n_local + top_k] and
+ *     [batch][num_kv_heads], as bsa_select_blocks writes them; entries outside the sequence's
+ *     blocks, such as the -1 padding, are skipped) of k_cache / v_cache -> out, lse (may be NULL);
+ *   selection (Eq. 4): f ([batch][num_kv_heads][head_dim], one Forecast vector per GQA group)
+ *     against ck_next (the NEXT layer's compressed keys, [batch][num_kv_heads][nc_cap][head_dim])
+ *     exactly as bsa_select_blocks_forecast -> block_idx_next, n_sel_next, block_scores_next (may
+ *     be NULL).
+ * The blocks of this layer stream while the next layer's are being chosen (the kernel has no
+ * selection-to-attention dependency). block_idx_next / n_sel_next must not overlap block_idx /
+ * n_sel. The first layer's blocks come from bsa_select_blocks (its own queries) or
+ * bsa_select_blocks_forecast; the last layer attends with bsa_sparse_decode. All device pointers
+ * are caller-owned, 16-byte aligned (4-byte for the int32 / fp32 arrays); seq_lens as
+ * bsa_decode_step (not modified); the workspace holds the error word. Runs the fused step kernel,
+ * so the parameter sets of bsa_decode_step_fused only; others return BSA_ERR_UNSUPPORTED. */
+bsa_status_t bsa_decode_step_lookahead(const bsa_params_t* params, const void* q, const void* k_cache,
+                                       const void* v_cache, const int32_t* block_idx,
+                                       const int32_t* n_sel, const void* f, const void* ck_next,
+                                       const int32_t* seq_lens, int32_t* block_idx_next,
+                                       int32_t* n_sel_next, float* block_scores_next, void* out,
+                                       float* lse, void* workspace, size_t workspace_bytes,
+                                       cudaStream_t stream);
+
 /* How bsa_decode_step runs for these parameters (host only, no CUDA call): *fused is 1 when it
  * runs the one-kernel step of bsa_decode_step_fused, 0 when it chains the scoring, selection,
  * attention and combine kernels; *launches is the number of kernel launches of one call, counting

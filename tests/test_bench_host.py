@@ -64,7 +64,8 @@ def test_algorithmic_bytes(name):
         assert ab["total"] == 558071808   # 268.40 MB of compressed keys + 289.41 MB of K/V + q, out
 
 
-@pytest.mark.parametrize("name", ["forecast-bf16-128k-b16", "anchors-2of4-64k-b8", "gqa4-bf16-32k-b1"])
+@pytest.mark.parametrize("name", ["forecast-bf16-128k-b16", "anchors-2of4-64k-b8", "gqa4-bf16-32k-b1",
+                                  "lookahead-bf16-128k-b16"])
 def test_cpu_oracle_leg_runs(name):
     """The bench's CPU-baseline / reference leg (the oracle on a bounded sample of pairs) for the
     Forecast-indexer, anchored and plain workloads, on a shortened copy of each."""
