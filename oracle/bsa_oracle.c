@@ -372,6 +372,92 @@ int bsa_oracle_select_forecast_ck(const orc_problem_t* P, const void* f, const d
                       block_scores, boundary, NULL, NULL);
 }
 
+/* Block-sparse prefill of a chunk (page "SparDA: Sparse Decoupled Attention for Efficient
+ * Long-Context LLM Inference", Theoretical Foundation, Eq. 1, with the selection made per query
+ * tile as in the tile-level operations of the page "CoSA: Accelerating Long-Context Inference via
+ * Proxy-Kernel Co-Designed Sparse Attention", Kascade abstract). The chunk's C queries of sequence b
+ * sit at positions T - C .. T - 1 (T = seq_lens[b], the chunk's keys and values already in the
+ * cache). Query tile r holds the chunk's positions inside block r; for each (tile, kv head):
+ *   scores: S[j] = sum over the tile's positions and the group's heads of softmax_j(q . K~_j / tau),
+ *           over the windows complete before the tile's block begins (s j + l <= BS r), Eq. 6;
+ *   blocks: the maximum of S over the windows overlapping each block, blocks 0 .. r ("Fine-grained
+ *           supervision"), and the selection of Eq. 1 among those r + 1 blocks (init, local = the
+ *           last n_local of them, top-k by score with ties to the lower block);
+ *   attention: the query at position p attends the selected blocks' tokens u <= p (Eq. 5).
+ * q is [B][C][Hq][d]; idx [n][tiles_cap][sel_cap], n_sel [n][tiles_cap] (tile i of pair i0 is
+ * block (T - C) / BS + i; tiles past the chunk are -1 / 0); out [n][C][G][d], lse [n][C][G] for the
+ * listed pairs. Returns 0, or -1 on an invalid argument. */
+int bsa_oracle_prefill(const orc_problem_t* P, const void* q, const void* k_cache, const void* v_cache,
+                       const int32_t* seq_lens, int chunk, const int32_t* pairs, int n_pairs, int tiles_cap,
+                       int32_t* idx, int32_t* n_sel, double* out, double* lse) {
+    if (!orc_problem_ok(P) || n_pairs < 0 || chunk < 1 || tiles_cap < 1) return -1;
+    const int G = P->num_q_heads / P->num_kv_heads, d = P->head_dim, BS = P->block_size;
+    const int sel_cap = P->n_init + P->n_local + P->top_k;
+    for (int i = 0; i < n_pairs; ++i) {
+        if (pairs[i] < 0 || pairs[i] >= P->batch * P->num_kv_heads) return -1;
+        const int64_t T = seq_lens[pairs[i] / P->num_kv_heads];
+        if (T < chunk || T > P->max_seq_len) return -1;
+        if ((T - 1) / BS - (T - chunk) / BS + 1 > tiles_cap) return -1;
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n_pairs; ++i) {
+        const int pair = pairs[i], b = pair / P->num_kv_heads, kvh = pair % P->num_kv_heads;
+        const int64_t T = seq_lens[b], t0 = T - chunk;
+        const void* kp = orc_pair_rows(P, k_cache, pair);
+        const void* vp = orc_pair_rows(P, v_cache, pair);
+        const int64_t nc_all = bsa_oracle_num_windows(T, P->cmp_kernel, P->cmp_stride);
+        double* ck = (double*)malloc((size_t)(nc_all > 0 ? nc_all : 1) * d * sizeof(double));
+        bsa_oracle_compress(kp, P->dtype, T, d, P->cmp_kernel, P->cmp_stride, P->dtype, ck);
+        double* qg = (double*)malloc((size_t)G * d * sizeof(double));
+        double* S = (double*)malloc((size_t)(nc_all > 0 ? nc_all : 1) * sizeof(double));
+        double* St = (double*)malloc((size_t)(nc_all > 0 ? nc_all : 1) * sizeof(double));
+        const int64_t r_lo = t0 / BS, r_hi = (T - 1) / BS;
+        double* sb = (double*)malloc((size_t)(r_hi + 1) * sizeof(double));
+        for (int ti = 0; ti < tiles_cap; ++ti) {
+            int32_t* my_idx = idx + ((int64_t)i * tiles_cap + ti) * sel_cap;
+            for (int r = 0; r < sel_cap; ++r) my_idx[r] = -1;
+            n_sel[(int64_t)i * tiles_cap + ti] = 0;
+        }
+        for (int64_t r = r_lo; r <= r_hi; ++r) {
+            /* windows complete before block r begins: s j + l <= BS r */
+            int64_t nc = bsa_oracle_num_windows(BS * r, P->cmp_kernel, P->cmp_stride);
+            if (nc > nc_all) nc = nc_all;
+            const int64_t p_lo = t0 > BS * r ? t0 : BS * r, p_hi = T < BS * (r + 1) ? T : BS * (r + 1);
+            for (int64_t j = 0; j < nc; ++j) S[j] = 0.0;
+            for (int64_t p = p_lo; p < p_hi; ++p) {
+                for (int h = 0; h < G; ++h)
+                    for (int c = 0; c < d; ++c)
+                        qg[h * d + c] = bsa_oracle_load(q, P->dtype,
+                                                        (((int64_t)b * chunk + (p - t0)) * P->num_q_heads + (int64_t)kvh * G + h) * d + c);
+                bsa_oracle_group_scores(qg, ck, nc, G, d, P->tau, St);
+                for (int64_t j = 0; j < nc; ++j) S[j] += St[j];
+            }
+            const int64_t nb = r + 1;
+            bsa_oracle_block_scores(S, nc, nb, P->cmp_kernel, P->cmp_stride, BS, sb);
+            int32_t* my_idx = idx + ((int64_t)i * tiles_cap + (r - r_lo)) * sel_cap;
+            double bnd[2];
+            const int ns = bsa_oracle_select(sb, nb, P->n_init, P->n_local, P->top_k, my_idx, bnd);
+            n_sel[(int64_t)i * tiles_cap + (r - r_lo)] = ns;
+            for (int64_t p = p_lo; p < p_hi; ++p) {
+                for (int h = 0; h < G; ++h)
+                    for (int c = 0; c < d; ++c)
+                        qg[h * d + c] = bsa_oracle_load(q, P->dtype,
+                                                        (((int64_t)b * chunk + (p - t0)) * P->num_q_heads + (int64_t)kvh * G + h) * d + c);
+                /* causal: the tokens of the selected blocks before and at p */
+                bsa_oracle_attend(qg, kp, vp, P->dtype, p + 1, d, G, my_idx, ns, BS, P->scale,
+                                  out + (((int64_t)i * chunk + (p - t0)) * G) * d,
+                                  lse + ((int64_t)i * chunk + (p - t0)) * G);
+            }
+        }
+        free(ck);
+        free(qg);
+        free(S);
+        free(St);
+        free(sb);
+    }
+    return 0;
+}
+
 int bsa_oracle_attend_pairs(const orc_problem_t* P, const void* q, const void* k_cache,
                             const void* v_cache, const int32_t* seq_lens, const int32_t* pairs,
                             int n_pairs, const int32_t* idx, const int32_t* n_sel, double* out,

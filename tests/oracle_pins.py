@@ -512,6 +512,81 @@ def pin_lookahead_step_brute_force():
         np.testing.assert_allclose(res["block_scores"][kvh, :nb], sb, rtol=1e-12, atol=1e-12)
 
 
+def pin_prefill_single_position_is_decode():
+    """A prefill chunk of one query at the first position of a block is a decode step at that
+    length: the windows complete before the block are those complete one token later, the tile's
+    score is that one query's, and it attends tokens up to itself, so selection and output agree
+    bit for bit."""
+    B, Hq, Hkv, d, Tc = 1, 6, 2, 16, 64 * 16
+    k, v = _randn((B, Hkv, Tc, d), 102), _randn((B, Hkv, Tc, d), 103)
+    kb, vb = _bf16_bits(k), _bf16_bits(v)
+    P = oracle.make_problem(B, Hq, Hkv, d, Tc, oracle.BF16, 1, 2, 4)
+    for r in (0, 1, 5, 13):
+        T = 64 * r + 1
+        q = _bf16_bits(_randn((B, 1, Hq, d), 104 + r))
+        pre = oracle.prefill(P, q, kb, vb, [T], 1)
+        dec = oracle.decode(P, q[:, 0], kb, vb, [T])
+        for i in range(Hkv):
+            n = int(dec["n_sel"][i])
+            assert int(pre["n_sel"][i, 0]) == n and pre["idx"][i, 0, :n].tolist() == dec["idx"][i, :n].tolist()
+            assert (pre["n_sel"][i, 1:] == 0).all()
+            np.testing.assert_array_equal(pre["out"][i, 0], dec["out"][i])
+            np.testing.assert_array_equal(pre["lse"][i, 0], dec["lse"][i])
+
+
+def pin_prefill_all_blocks_is_causal_dense():
+    """With top-k covering every candidate each query attends every earlier token and itself:
+    causal dense attention (torch SDPA in float64 with a causal mask), for a chunk that starts and
+    ends inside blocks."""
+    B, Hq, Hkv, d = 1, 4, 2, 16
+    T, C = 64 * 5 + 20, 100
+    q, k, v = _randn((B, C, Hq, d), 105), _randn((B, Hkv, T, d), 106), _randn((B, Hkv, T, d), 107)
+    P = oracle.make_problem(B, Hq, Hkv, d, T, oracle.F32, 1, 1, 64)
+    res = oracle.prefill(P, q.numpy(), k.numpy(), v.numpy(), [T], C)
+    G = Hq // Hkv
+    for kvh in range(Hkv):
+        for c in range(C):
+            pos = T - C + c
+            ro, rl = _sdpa(q[0, c, kvh * G:(kvh + 1) * G].double().numpy(), k[0, kvh, :pos + 1].double().numpy(),
+                           v[0, kvh, :pos + 1].double().numpy(), 1.0 / math.sqrt(d))
+            np.testing.assert_allclose(res["out"][kvh, c], ro, rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(res["lse"][kvh, c], rl, rtol=1e-12, atol=1e-13)
+
+
+def pin_prefill_tile_selection_brute_force():
+    """Each query tile's blocks by brute force: per position and head a softmax (torch) over the
+    windows complete before the tile's block, summed; the block score the largest over the
+    overlapping windows (plain loops); the top-k from a plain sort, ties to the lower block."""
+    B, Hq, Hkv, d = 1, 4, 1, 8
+    T, C = 64 * 9 + 37, 64 * 3 + 5
+    q, k, v = _randn((B, C, Hq, d), 108), _randn((B, Hkv, T, d), 109), _randn((B, Hkv, T, d), 110)
+    n_init, n_local, top_k = 1, 2, 3
+    P = oracle.make_problem(B, Hq, Hkv, d, T, oracle.F32, n_init, n_local, top_k)
+    res = oracle.prefill(P, q.numpy(), k.numpy(), v.numpy(), [T], C)
+    kk = k[0, 0].double()
+    t0 = T - C
+    r_lo, r_hi = t0 // 64, (T - 1) // 64
+    assert res["idx"].shape[1] == oracle.prefill_tiles_cap(C) and (res["n_sel"][0, r_hi - r_lo + 1:] == 0).all()
+    for r in range(r_lo, r_hi + 1):
+        nc = max((64 * r - 32) // 16 + 1, 0) if 64 * r >= 32 else 0
+        win = torch.stack([kk[16 * j:16 * j + 32].mean(0) for j in range(nc)]) if nc else torch.zeros(0, d, dtype=torch.float64)
+        win = win.float().double()  # the cache dtype (fp32)
+        S = torch.zeros(nc, dtype=torch.float64)
+        for pos in range(max(t0, 64 * r), min(T, 64 * r + 64)):
+            for h in range(Hq):
+                if nc:
+                    S += torch.softmax(win @ q[0, pos - t0, h].double() / math.sqrt(d), dim=0)
+        nb = r + 1
+        sb = [max([float(S[j]) for j in range(nc) if 16 * j < 64 * (b + 1) and 16 * j + 32 > 64 * b], default=-math.inf)
+              for b in range(nb)]
+        fixed = set(range(min(n_init, nb))) | set(range(max(nb - n_local, min(n_init, nb)), nb))
+        cand = sorted((b for b in range(nb) if b not in fixed), key=lambda b: (-sb[b], b))
+        want = sorted(fixed | set(cand[:top_k]))
+        ti = r - r_lo
+        got = res["idx"][0, ti, :res["n_sel"][0, ti]].tolist()
+        assert got == want, (r, got, want)
+
+
 ALL_PINS = [
     pin_round_bf16_matches_torch, pin_round_ties_even, pin_round_f32_matches_numpy,
     pin_compress_matches_avg_pool, pin_compress_constant_windows, pin_window_and_block_counts,
@@ -527,4 +602,6 @@ ALL_PINS = [
     pin_shared_index_identical_layers,
     pin_forecast_decode_composes, pin_forecast_one_head_matches_base_selector,
     pin_lookahead_step_brute_force,
+    pin_prefill_single_position_is_decode, pin_prefill_all_blocks_is_causal_dense,
+    pin_prefill_tile_selection_brute_force,
 ]
