@@ -105,7 +105,7 @@ def _bind(path: str):
         "bsa_oracle_select_forecast_ck": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _INT,
                                                  _P, _P, _P, _P]),
         "bsa_oracle_prefill": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _INT, _P, _INT, _INT,
-                                      _P, _P, _P, _P]),
+                                      _P, _P, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -420,7 +420,8 @@ def prefill(P: Problem, q, k_cache, v_cache, seq_lens, chunk: int, pairs=None) -
     """Block-sparse prefill of the last ``chunk`` positions of each sequence (see
     ``bsa_oracle_prefill``): q is the chunk's queries [B][C][Hq][d] (storage array of the
     problem's dtype). Returns idx [n][tiles][sel_cap], n_sel [n][tiles] (tile i covers block
-    (T - C) // BS + i), out [n][C][G][d] and lse [n][C][G]."""
+    (T - C) // BS + i), boundary [n][tiles][2] (the k-th taken and best rejected block score),
+    out [n][C][G][d] and lse [n][C][G]."""
     q = _raw_check(q, P.dtype)
     k_cache, v_cache = _raw_check(k_cache, P.dtype), _raw_check(v_cache, P.dtype)
     seq_lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
@@ -432,11 +433,13 @@ def prefill(P: Problem, q, k_cache, v_cache, seq_lens, chunk: int, pairs=None) -
     tiles = prefill_tiles_cap(chunk, P.block_size)
     res = dict(idx=np.full((n, tiles, sel_cap), -1, dtype=np.int32),
                n_sel=np.zeros((n, tiles), dtype=np.int32),
+               boundary=np.full((n, tiles, 2), np.nan, dtype=np.float64),
                out=np.zeros((n, chunk, G, P.head_dim), dtype=np.float64),
                lse=np.zeros((n, chunk, G), dtype=np.float64))
     rc = _load().bsa_oracle_prefill(ctypes.byref(P), _ptr(q), _ptr(k_cache), _ptr(v_cache),
                                     _ptr(seq_lens), chunk, _ptr(pairs), n, tiles, _ptr(res["idx"]),
-                                    _ptr(res["n_sel"]), _ptr(res["out"]), _ptr(res["lse"]))
+                                    _ptr(res["n_sel"]), _ptr(res["boundary"]), _ptr(res["out"]),
+                                    _ptr(res["lse"]))
     if rc != 0:
         raise ValueError("bsa_oracle_prefill rejected its arguments")
     return res

@@ -385,11 +385,12 @@ int bsa_oracle_select_forecast_ck(const orc_problem_t* P, const void* f, const d
  *           last n_local of them, top-k by score with ties to the lower block);
  *   attention: the query at position p attends the selected blocks' tokens u <= p (Eq. 5).
  * q is [B][C][Hq][d]; idx [n][tiles_cap][sel_cap], n_sel [n][tiles_cap] (tile i of pair i0 is
- * block (T - C) / BS + i; tiles past the chunk are -1 / 0); out [n][C][G][d], lse [n][C][G] for the
- * listed pairs. Returns 0, or -1 on an invalid argument. */
+ * block (T - C) / BS + i; tiles past the chunk are -1 / 0), boundary [n][tiles_cap][2] (as in the
+ * decode driver: the k-th taken and the best rejected block score; may be NULL); out [n][C][G][d],
+ * lse [n][C][G] for the listed pairs. Returns 0, or -1 on an invalid argument. */
 int bsa_oracle_prefill(const orc_problem_t* P, const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* seq_lens, int chunk, const int32_t* pairs, int n_pairs, int tiles_cap,
-                       int32_t* idx, int32_t* n_sel, double* out, double* lse) {
+                       int32_t* idx, int32_t* n_sel, double* boundary, double* out, double* lse) {
     if (!orc_problem_ok(P) || n_pairs < 0 || chunk < 1 || tiles_cap < 1) return -1;
     const int G = P->num_q_heads / P->num_kv_heads, d = P->head_dim, BS = P->block_size;
     const int sel_cap = P->n_init + P->n_local + P->top_k;
@@ -417,6 +418,7 @@ int bsa_oracle_prefill(const orc_problem_t* P, const void* q, const void* k_cach
             int32_t* my_idx = idx + ((int64_t)i * tiles_cap + ti) * sel_cap;
             for (int r = 0; r < sel_cap; ++r) my_idx[r] = -1;
             n_sel[(int64_t)i * tiles_cap + ti] = 0;
+            if (boundary) boundary[2 * ((int64_t)i * tiles_cap + ti)] = boundary[2 * ((int64_t)i * tiles_cap + ti) + 1] = NAN;
         }
         for (int64_t r = r_lo; r <= r_hi; ++r) {
             /* windows complete before block r begins: s j + l <= BS r */
@@ -438,6 +440,10 @@ int bsa_oracle_prefill(const orc_problem_t* P, const void* q, const void* k_cach
             double bnd[2];
             const int ns = bsa_oracle_select(sb, nb, P->n_init, P->n_local, P->top_k, my_idx, bnd);
             n_sel[(int64_t)i * tiles_cap + (r - r_lo)] = ns;
+            if (boundary) {
+                boundary[2 * ((int64_t)i * tiles_cap + (r - r_lo))] = bnd[0];
+                boundary[2 * ((int64_t)i * tiles_cap + (r - r_lo)) + 1] = bnd[1];
+            }
             for (int64_t p = p_lo; p < p_hi; ++p) {
                 for (int h = 0; h < G; ++h)
                     for (int c = 0; c < d; ++c)

@@ -169,10 +169,10 @@ int bsa_oracle_decode_ck(const orc_problem_t* P, const void* q, const double* ck
  * seq_lens[b] - C .. seq_lens[b] - 1), one selection per query tile (the chunk's positions inside
  * one block) and kv head from the windows complete before that block, causal attention per query;
  * see bsa_oracle.c for the definition. Outputs per listed pair i: idx [n][tiles_cap][sel_cap],
- * n_sel [n][tiles_cap], out [n][C][G][d], lse [n][C][G]. */
+ * n_sel [n][tiles_cap], boundary [n][tiles_cap][2] (may be NULL), out [n][C][G][d], lse [n][C][G]. */
 int bsa_oracle_prefill(const orc_problem_t* P, const void* q, const void* k_cache, const void* v_cache,
                        const int32_t* seq_lens, int chunk, const int32_t* pairs, int n_pairs, int tiles_cap,
-                       int32_t* idx, int32_t* n_sel, double* out, double* lse);
+                       int32_t* idx, int32_t* n_sel, double* boundary, double* out, double* lse);
 int bsa_oracle_select_forecast_ck(const orc_problem_t* P, const void* f, const double* ck,
                                   const int32_t* seq_lens, const int32_t* pairs, int n_pairs,
                                   int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary);
