@@ -11,7 +11,8 @@ from ._abi import (  # noqa: F401
     BSA_ERR_WORKSPACE, BSA_F32, BSA_MAX_LAYERS, BSA_OK, DEVERR_BLOCK_IDX, DEVERR_CAPACITY,
     DEVERR_N_SEL, DEVERR_SEQ_LEN, LIB_PATH, BsaError, Params, Sizes, alloc_workspace,
     bsa_abi_version, bsa_check_params, bsa_compress_append, bsa_compress_keys, bsa_decode_step,
-    bsa_decode_step_anchored, bsa_decode_step_info, bsa_decode_step_lookahead,
+    bsa_decode_step_anchored, bsa_decode_step_info, bsa_decode_step_lookahead, bsa_prefill,
+    bsa_prefill_attend, bsa_prefill_tiles,
     bsa_get_sizes, bsa_read_device_error, bsa_select_blocks, bsa_select_blocks_forecast,
     bsa_sparse_decode, bsa_sparse_decode_layers, bsa_sparse_decode_noalloc, bsa_workspace_init,
     bsa_workspace_size, lib, make_params, status_string,

@@ -83,6 +83,10 @@ _SIGS = {
                                    ctypes.c_size_t, _P]),
     "bsa_decode_step_lookahead": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                        ctypes.c_size_t, _P]),
+    "bsa_prefill": (_S, [_PP, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "bsa_prefill_attend": (_S, [_PP, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
+                                _P]),
+    "bsa_prefill_tiles": (ctypes.c_int32, [ctypes.c_int32, ctypes.c_int32]),
     "bsa_decode_step_anchored": (_S, [_PP, ctypes.c_int32, _P, ctypes.c_int32, _P, _P, _P, _P, _P,
                                       _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "bsa_read_device_error": (_S, [_P, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32), _P]),
@@ -389,6 +393,46 @@ def bsa_decode_step_lookahead(p: Params, q, k_cache, v_cache, block_idx, n_sel, 
         _ptr(out, "out", e, n["q"]), _ptr(lse, "lse", torch.float32, n["lse"], optional=True),
         _ptr(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
         "bsa_decode_step_lookahead")
+
+
+def bsa_prefill_tiles(chunk: int, block_size: int = 64) -> int:
+    """Query tiles per (batch, kv head) pair of a prefill chunk."""
+    return int(lib().bsa_prefill_tiles(int(chunk), int(block_size)))
+
+
+def _prefill_ptrs(p: Params, chunk, q, seq_lens, block_idx, n_sel, out, lse):
+    import torch
+    e = _elem(p)
+    pairs = p.batch * p.num_kv_heads
+    tiles = bsa_prefill_tiles(chunk, p.block_size)
+    sel_cap = p.n_init + p.n_local + p.top_k
+    qn = p.batch * chunk * p.num_q_heads * p.head_dim
+    return (_ptr(q, "q", e, qn), _ptr(seq_lens, "seq_lens", torch.int32, p.batch),
+            _ptr(block_idx, "block_idx", torch.int32, pairs * tiles * sel_cap),
+            _ptr(n_sel, "n_sel", torch.int32, pairs * tiles), _ptr(out, "out", e, qn),
+            _ptr(lse, "lse", torch.float32, p.batch * chunk * p.num_q_heads, optional=True))
+
+
+def bsa_prefill(p: Params, chunk: int, q, k_cache, v_cache, ck, seq_lens, block_idx, n_sel, out, lse, ws,
+                stream=None):
+    """bsa_prefill: the last `chunk` positions of every sequence, one selection per query tile."""
+    n, e = _shapes(p), _elem(p)
+    qp, sp, ip, np_, op, lp = _prefill_ptrs(p, chunk, q, seq_lens, block_idx, n_sel, out, lse)
+    _check(lib().bsa_prefill(ctypes.byref(p), int(chunk), qp, _ptr(k_cache, "k_cache", e, n["cache"]),
+                             _ptr(v_cache, "v_cache", e, n["cache"]), _ptr(ck, "ck", e, n["ck"]), sp, ip, np_,
+                             op, lp, _ptr(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
+           "bsa_prefill")
+
+
+def bsa_prefill_attend(p: Params, chunk: int, q, k_cache, v_cache, seq_lens, block_idx, n_sel, out, lse, ws,
+                       stream=None):
+    """bsa_prefill_attend: the prefill attention with the tiles' blocks given."""
+    n, e = _shapes(p), _elem(p)
+    qp, sp, ip, np_, op, lp = _prefill_ptrs(p, chunk, q, seq_lens, block_idx, n_sel, out, lse)
+    _check(lib().bsa_prefill_attend(ctypes.byref(p), int(chunk), qp, _ptr(k_cache, "k_cache", e, n["cache"]),
+                                    _ptr(v_cache, "v_cache", e, n["cache"]), sp, ip, np_, op, lp,
+                                    _ptr(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
+           "bsa_prefill_attend")
 
 
 def bsa_read_device_error(ws, stream=None) -> int:

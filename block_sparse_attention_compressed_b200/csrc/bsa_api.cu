@@ -738,6 +738,109 @@ bsa_status_t bsa_decode_step_lookahead(const bsa_params_t* params, const void* q
     return from_cuda(launch_step(P, a, &c.maps, stream));
 }
 
+}  // extern "C"
+
+namespace bsa {
+namespace {
+// Prefill: argument checks and the kernels' arguments; `select` also checks the selection
+// kernel's shared memory.
+bsa_status_t prefill_args(const bsa_params_t* params, int32_t chunk, const void* q, const int32_t* seq_lens,
+                          const int32_t* block_idx, const int32_t* n_sel, void* out, float* lse, void* ws,
+                          size_t ws_bytes, bool select, Plan* P, PrefillArgs* a, size_t* smem) {
+    bsa_status_t st = make_plan(params, P);
+    if (st != BSA_OK) return st;
+    if (P->dtype != BSA_BF16 || P->D != 128 || (P->G != 2 && P->G != 4) || P->BS != 64 || P->l != 32 ||
+        P->s != 16)
+        return BSA_ERR_UNSUPPORTED;
+    if (chunk < 1 || chunk > P->T_cap) return BSA_ERR_INVALID_ARG;
+    if (!ok16(q) || !ok16(out) || !ok4(seq_lens) || !ok4(block_idx) || !ok4(n_sel) || (lse && !ok4(lse)))
+        return BSA_ERR_INVALID_ARG;
+    if ((st = check_ws(*P, ws, ws_bytes)) != BSA_OK) return st;
+    *smem = select ? prefill_select_smem_bytes(P->G, P->nc_cap, P->nb_cap, P->sel_cap) : 1;
+    if (*smem == 0) return BSA_ERR_UNSUPPORTED;
+    memset(a, 0, sizeof *a);
+    a->q = q;
+    a->seq_lens = seq_lens;
+    a->block_idx = const_cast<int32_t*>(block_idx);
+    a->n_sel = const_cast<int32_t*>(n_sel);
+    a->out = out;
+    a->lse = lse;
+    a->err = ws_at<uint32_t>(ws, P->off_err);
+    a->chunk = chunk;
+    a->tiles_cap = (chunk + P->BS - 1) / P->BS + 1;
+    a->Hq = P->Hq;
+    a->Hkv = P->Hkv;
+    a->G = P->G;
+    a->n_init = P->n_init;
+    a->n_local = P->n_local;
+    a->top_k = P->top_k;
+    a->sel_cap = P->sel_cap;
+    a->pairs = P->pairs;
+    a->BS = P->BS;
+    a->l = P->l;
+    a->s = P->s;
+    a->T_cap = P->T_cap;
+    a->nc_cap = P->nc_cap;
+    a->nb_cap = P->nb_cap;
+    a->score_log2 = P->score_log2;
+    a->scale_log2 = P->scale_log2;
+    if ((int64_t)P->pairs * a->tiles_cap > 0x7fffffffLL / 2) return BSA_ERR_UNSUPPORTED;
+    return BSA_OK;
+}
+struct PrefillMapCache {
+    CUtensorMap ck, k, v;
+    MapKey kck, kk, kv;
+};
+}  // namespace
+}  // namespace bsa
+
+extern "C" {
+
+int32_t bsa_prefill_tiles(int32_t chunk, int32_t block_size) {
+    return chunk < 1 || block_size < 1 ? 0 : (chunk + block_size - 1) / block_size + 1;
+}
+
+bsa_status_t bsa_prefill(const bsa_params_t* params, int32_t chunk, const void* q, const void* k_cache,
+                         const void* v_cache, const void* ck, const int32_t* seq_lens, int32_t* block_idx,
+                         int32_t* n_sel, void* out, float* lse, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    Plan P;
+    PrefillArgs a;
+    size_t smem = 0;
+    bsa_status_t st = prefill_args(params, chunk, q, seq_lens, block_idx, n_sel, out, lse, ws, ws_bytes, true, &P,
+                                   &a, &smem);
+    if (st != BSA_OK) return st;
+    if (!ok16(k_cache) || !ok16(v_cache) || (P.nc_cap > 0 && !ok16(ck))) return BSA_ERR_INVALID_ARG;
+    static thread_local PrefillMapCache c;
+    if ((P.nc_cap > 0 &&
+         !encode_kv_map_cached(&c.ck, &c.kck, ck, (uint64_t)P.pairs * P.nc_cap, P.D, 128)) ||
+        !encode_kv_map_cached(&c.k, &c.kk, k_cache, (uint64_t)P.pairs * P.T_cap, P.D, 64) ||
+        !encode_kv_map_cached(&c.v, &c.kv, v_cache, (uint64_t)P.pairs * P.T_cap, P.D, 64))
+        return BSA_ERR_CUDA;
+    const int64_t items = (int64_t)P.pairs * a.tiles_cap;
+    const int ctas = (int)(items < kNumSMs ? items : kNumSMs);
+    cudaError_t e = launch_prefill_select(a, &c.ck, smem, ctas, stream);
+    if (e != cudaSuccess) return BSA_ERR_CUDA;
+    return from_cuda(launch_prefill_attend(a, &c.k, &c.v, stream));
+}
+
+bsa_status_t bsa_prefill_attend(const bsa_params_t* params, int32_t chunk, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* seq_lens, const int32_t* block_idx,
+                                const int32_t* n_sel, void* out, float* lse, void* ws, size_t ws_bytes,
+                                cudaStream_t stream) {
+    Plan P;
+    PrefillArgs a;
+    size_t smem = 0;
+    bsa_status_t st = prefill_args(params, chunk, q, seq_lens, block_idx, n_sel, out, lse, ws, ws_bytes, false, &P,
+                                   &a, &smem);
+    if (st != BSA_OK) return st;
+    if (!ok16(k_cache) || !ok16(v_cache)) return BSA_ERR_INVALID_ARG;
+    static thread_local PrefillMapCache c;
+    if (!encode_kv_map_cached(&c.k, &c.kk, k_cache, (uint64_t)P.pairs * P.T_cap, P.D, 64) ||
+        !encode_kv_map_cached(&c.v, &c.kv, v_cache, (uint64_t)P.pairs * P.T_cap, P.D, 64))
+        return BSA_ERR_CUDA;
+    return from_cuda(launch_prefill_attend(a, &c.k, &c.v, stream));
+}
+
 bsa_status_t bsa_decode_step_info(const bsa_params_t* params, int32_t append, int32_t* fused,
                                   int32_t* launches) {
     Plan P;

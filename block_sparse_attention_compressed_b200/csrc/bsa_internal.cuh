@@ -156,6 +156,26 @@ struct StepArgs {
     uint32_t tmem_cols;
     float score_log2, scale_log2;
 };
+// Block-sparse prefill of a chunk of `chunk` queries per sequence (positions T - chunk .. T - 1).
+struct PrefillArgs {
+    const void* q;          // [B][chunk][Hq][D]
+    const int32_t* seq_lens;
+    int32_t* block_idx;     // [pairs][tiles_cap][sel_cap] per query tile
+    int32_t* n_sel;         // [pairs][tiles_cap]
+    void* out;              // [B][chunk][Hq][D]
+    float* lse;             // [B][chunk][Hq] or null
+    uint32_t* err;
+    int chunk, tiles_cap, Hq, Hkv, G, n_init, n_local, top_k, sel_cap, pairs, BS, l, s;
+    int64_t T_cap, nc_cap, nb_cap;
+    float score_log2, scale_log2;
+};
+cudaError_t launch_prefill_select(const PrefillArgs& a, const CUtensorMap* ck_map, size_t smem, int ctas,
+                                  cudaStream_t st);
+cudaError_t launch_prefill_attend(const PrefillArgs& a, const CUtensorMap* k_map, const CUtensorMap* v_map,
+                                  cudaStream_t st);
+// Dynamic shared memory of the prefill selection kernel, or 0 when it does not fit one CTA.
+size_t prefill_select_smem_bytes(int G, int64_t nc_cap, int64_t nb_cap, int sel_cap);
+
 // TMA descriptors of the step: compressed keys (boxes of 64 rows), K and V (boxes of 32 rows).
 struct alignas(64) StepMaps {
     CUtensorMap ck, k, v;

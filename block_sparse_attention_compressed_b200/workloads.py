@@ -48,6 +48,7 @@ class Workload:
     needle_shift: float = 2.0
     forecast: bool = False  # select with one Forecast vector per GQA group (f = the group's mean q)
     lookahead: bool = False  # (two layers, forecast) layer 0 attends given blocks and selects layer 1's
+    prefill_chunk: int = 0   # >0: block-sparse prefill of the last prefill_chunk positions
     anchors: tuple = (0,)   # multi-layer: layers that select; the others reuse the last anchor's
 
     @property
@@ -66,7 +67,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The decode workloads: one small parity case and seven throughput cases.
+# The workloads: one small parity case, seven decode throughput cases and one prefill case.
 WORKLOADS: dict[str, Workload] = {
     w.name: w
     for w in [
@@ -92,6 +93,9 @@ WORKLOADS: dict[str, Workload] = {
         Workload("lookahead-bf16-128k-b16", batch=16, num_q_heads=32, num_kv_heads=8, head_dim=128,
                  seq_len=131072, dtype="bf16", n_init=1, n_local=4, top_k=64, needles=16,
                  seed=1008, layers=2, forecast=True, lookahead=True),
+        Workload("prefill-bf16-32k-b4", batch=4, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                 seq_len=32768, dtype="bf16", n_init=1, n_local=4, top_k=64, needles=8, seed=1009,
+                 prefill_chunk=4096),
     ]
 }
 DEFAULT_WORKLOAD = "gqa4-bf16-128k-b16"

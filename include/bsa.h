@@ -277,6 +277,43 @@ bsa_status_t bsa_decode_step_lookahead(const bsa_params_t* params, const void* q
                                        float* lse, void* workspace, size_t workspace_bytes,
                                        cudaStream_t stream);
 
+/* Block-sparse prefill of a chunk (page "SparDA: Sparse Decoupled Attention for Efficient
+ * Long-Context LLM Inference", Theoretical Foundation, Eq. 1, and the prefill workload of its
+ * Efficiency Results; one selection per query tile, as the tile-level operations of the page "CoSA:
+ * Accelerating Long-Context Inference via Proxy-Kernel Co-Designed Sparse Attention", Kascade
+ * abstract). The last `chunk` positions of every sequence are queried: q is
+ * [batch][chunk][num_q_heads][head_dim] (query c of sequence b at position seq_lens[b] - chunk + c),
+ * the chunk's keys and values are already in k_cache / v_cache and ck holds the compressed keys of
+ * the whole sequences (bsa_compress_keys after the chunk was written). Query tile i of a
+ * (batch, kv head) pair holds the chunk's positions inside block (seq_lens[b] - chunk) / block_size
+ * + i; per tile and kv head the group's heads score, over every position of the tile, the windows
+ * complete before the tile's block begins (softmax per position and head, summed), the block
+ * scores are the maxima over overlapping windows, and the blocks of Eq. 1 among blocks 0 .. the
+ * tile's own are written to block_idx [batch][num_kv_heads][tiles][n_init + n_local + top_k]
+ * (ascending, -1 padded; tiles = bsa_prefill_tiles(chunk, block_size); tiles past a chunk's last are
+ * empty) and n_sel [batch][num_kv_heads][tiles]. Each query then attends the tokens of its tile's
+ * blocks at or before its own position: out [batch][chunk][num_q_heads][head_dim], lse
+ * [batch][chunk][num_q_heads] (natural log; may be NULL). seq_lens[b] must be in
+ * [chunk, max_seq_len]. Supported: bf16, head_dim 128, 2 or 4 query heads per kv head, blocks of
+ * 64 tokens, windows of 32 with stride 16 and compressed keys whose window scores fit the selection
+ * kernel's shared memory (max_seq_len up to about 128K tokens); others return BSA_ERR_UNSUPPORTED.
+ * The scoring runs on the tensor cores (tcgen05) with accumulators in tensor memory. */
+bsa_status_t bsa_prefill(const bsa_params_t* params, int32_t chunk, const void* q, const void* k_cache,
+                         const void* v_cache, const void* ck, const int32_t* seq_lens, int32_t* block_idx,
+                         int32_t* n_sel, void* out, float* lse, void* workspace, size_t workspace_bytes,
+                         cudaStream_t stream);
+
+/* The attention of bsa_prefill alone, with the tiles' blocks given (block_idx / n_sel laid out as
+ * bsa_prefill writes them; entries outside blocks 0 .. the tile's own are skipped). */
+bsa_status_t bsa_prefill_attend(const bsa_params_t* params, int32_t chunk, const void* q, const void* k_cache,
+                                const void* v_cache, const int32_t* seq_lens, const int32_t* block_idx,
+                                const int32_t* n_sel, void* out, float* lse, void* workspace,
+                                size_t workspace_bytes, cudaStream_t stream);
+
+/* Query tiles per (batch, kv head) pair of a prefill chunk: ceil(chunk / block_size) + 1 (a chunk
+ * that starts inside a block spans one more); 0 for non-positive arguments. Host only. */
+int32_t bsa_prefill_tiles(int32_t chunk, int32_t block_size);
+
 /* How bsa_decode_step runs for these parameters (host only, no CUDA call): *fused is 1 when it
  * runs the one-kernel step of bsa_decode_step_fused, 0 when it chains the scoring, selection,
  * attention and combine kernels; *launches is the number of kernel launches of one call, counting
