@@ -44,6 +44,7 @@ sys.path.insert(0, ROOT)
 METRIC = "block-sparse decode steps/s & achieved HBM GB/s (select+attn) at 128K ctx"
 # the library kernel behind each single-launch phase of a step, by dtype
 KERNEL_OF_PHASE = {"step": {"bf16": "step_kernel"},
+                   "prefill": {"bf16": "prefill_select_kernel+prefill_attend_kernel"},
                    "decode": {"bf16": "decode_tma_kernel+combine_kernel", "f32": "decode_f32_kernel"},
                    "append": {"bf16": "append_kernel", "f32": "append_kernel"},
                    "select": {"bf16": "score_tma_kernel+select_kernel",
@@ -209,6 +210,19 @@ class Bench:
         self.path = path if single else "auto"
         self.fused = single and (path == "fused" or (path == "auto" and bsa.bsa_decode_step_info(self.p)[0]))
         self.lookahead = bool(w.lookahead)
+        self.prefill = w.prefill_chunk > 0
+        if self.prefill:
+            # block-sparse prefill of the last prefill_chunk positions: queries drawn like q
+            C = w.prefill_chunk
+            g = torch.Generator(device=device).manual_seed(w.seed + 7 + seed_offset)
+            self.q_chunk = torch.randn(B, C, w.num_q_heads, d, generator=g, device=device).to(dt)
+            self.data["q_chunk"] = self.q_chunk
+            self.tiles = bsa.bsa_prefill_tiles(C, w.block_size)
+            self.p_idx = torch.zeros(B, Hkv, self.tiles, s.sel_cap, dtype=torch.int32, device=device)
+            self.p_ns = torch.zeros(B, Hkv, self.tiles, dtype=torch.int32, device=device)
+            self.out = [torch.zeros(B, C, w.num_q_heads, d, dtype=dt, device=device)]
+            self.lse = [torch.zeros(B, C, w.num_q_heads, dtype=torch.float32, device=device)]
+            self.fused = True
         if self.lookahead:
             # layer 0 attends blocks chosen beforehand (here by its own queries, outside the timed
             # region) while layer 1's are chosen from the Forecast vectors: one kernel per step
@@ -224,6 +238,8 @@ class Bench:
         torch.cuda.synchronize()
 
     def q_of(self, i):
+        if self.prefill:
+            return self.q_chunk
         return self.data["q_steps"][i] if self.append else self.data["q"][0]
 
     # the library calls of one step, on `stream`; `events` (optional) brackets every launch
@@ -231,6 +247,13 @@ class Bench:
         bsa, d = self.bsa, self.data
         q = self.q_of(i) if q is None else q
         ev = (lambda k: events[k].record(stream)) if events is not None else (lambda k: None)
+        if self.prefill:
+            ev(0)
+            bsa.bsa_prefill(self.p, self.w.prefill_chunk, self.q_chunk, d["k"][0], d["v"][0], self.ck,
+                            d["seq_lens"], self.p_idx, self.p_ns, self.out[0], self.lse[0], self.ws,
+                            stream=stream)
+            ev(1)
+            return
         if self.lookahead:
             ev(0)
             bsa.bsa_decode_step_lookahead(self.p, q, d["k"][0], d["v"][0], self.block_idx, self.n_sel,
@@ -303,6 +326,10 @@ class Bench:
     # Forecast-indexer workloads qs is [q, f]
     def step_io(self, qs, outs, lses, stream, k_new=None, v_new=None):
         bsa, d = self.bsa, self.data
+        if self.prefill:
+            bsa.bsa_prefill(self.p, self.w.prefill_chunk, qs[0], d["k"][0], d["v"][0], self.ck, d["seq_lens"],
+                            self.p_idx, self.p_ns, outs[0], lses[0], self.ws, stream=stream)
+            return
         if self.lookahead:
             bsa.bsa_decode_step_lookahead(self.p, qs[0], d["k"][0], d["v"][0], self.block_idx, self.n_sel,
                                           qs[1], self.ck_next, d["seq_lens"], self.idx_next,
@@ -340,12 +367,16 @@ class Bench:
 
     def kernel_names(self):
         """The phases pass B brackets with events, in launch order."""
+        if self.prefill:
+            return ["prefill"]
         if self.fused:
             return (["append"] if self.append else []) + ["step"]
         names = ["select", "decode"] * (len(self.w.anchors) if self.w.layers > 1 else 1)
         return (["append"] + names) if (self.append and self.w.layers == 1) else names
 
     def launches_per_step(self):
+        if self.prefill:
+            return 2  # the selection (tcgen05) and the attention
         if self.fused:
             return 1 + (1 if self.append else 0)
         # bsa_select_blocks launches two kernels (scoring, selection), the bf16 sparse attention two
@@ -360,6 +391,16 @@ class Bench:
 def algorithmic(w, T):
     from block_sparse_attention_compressed_b200.workloads import algorithmic_bytes
     return algorithmic_bytes(w, T)
+
+
+def load_tensor_peak():
+    """Measured dense bf16 GEMM throughput (burst, TFLOP/s), else the fallback figure."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return 1590.0, "fallback"
 
 
 def load_peaks():
@@ -465,8 +506,11 @@ def cpu_oracle_sample(w, data, seconds: float):
     pairs = [divmod(p, Hkv) for p in range(n0)]
 
     def layer_arrays(L):
-        q = data["q_steps"][0] if ("q_steps" in data and L == 0) else data["q"][L]
-        qs = torch.stack([q[b, h * G:(h + 1) * G] for b, h in pairs])
+        if w.prefill_chunk:
+            qs = torch.stack([data["q_chunk"][b, :, h * G:(h + 1) * G] for b, h in pairs])
+        else:
+            q = data["q_steps"][0] if ("q_steps" in data and L == 0) else data["q"][L]
+            qs = torch.stack([q[b, h * G:(h + 1) * G] for b, h in pairs])
         ks = torch.stack([data["k"][L][b, h:h + 1] for b, h in pairs])
         vs = torch.stack([data["v"][L][b, h:h + 1] for b, h in pairs])
         return oracle.raw(qs)[0], oracle.raw(ks)[0], oracle.raw(vs)[0]
@@ -479,10 +523,10 @@ def cpu_oracle_sample(w, data, seconds: float):
     f_arr = (oracle.raw(torch.stack([data["f"][b, h:h + 1] for b, h in pairs]))[0]
              if w.forecast else None)
     # A1, the compression of every scoring layer's keys (once per cache; timed apart)
-    scored = [1] if w.lookahead else list(w.anchors)
+    scored = [1] if w.lookahead else ([] if w.prefill_chunk else list(w.anchors))
     t0 = time.perf_counter()
     cks = {L: oracle.compress_cache(P, arrays[L][1], lens) for L in scored}
-    compress_s = (time.perf_counter() - t0) * (total / n0) / len(scored)
+    compress_s = (time.perf_counter() - t0) * (total / n0) / max(len(scored), 1)
     # lookahead: layer 0's blocks, chosen beforehand (by its own queries; untimed)
     sel0 = oracle.decode(P, *arrays[0], lens) if w.lookahead else None
 
@@ -497,6 +541,11 @@ def cpu_oracle_sample(w, data, seconds: float):
                 sub, G, 1, w.head_dim, T_cap, P.dtype, w.n_init, w.n_local, w.top_k, w.cmp_kernel,
                 w.cmp_stride, w.block_size)
             ln = lens if sub is None else lens[:sub]
+            if w.prefill_chunk:
+                # the chunk's block-sparse prefill (its compression included: the chunk's keys
+                # complete new windows)
+                oracle.prefill(Ps, q_, k_, v_, ln, w.prefill_chunk)
+                return
             if w.lookahead:
                 # layer 0 attends its blocks, layer 1's are chosen from the Forecast vectors
                 oracle.lookahead_step(Ps, q_, k_, v_, sel0["idx"][idx], sel0["n_sel"][idx], f_arr[idx],
@@ -544,6 +593,12 @@ def run_bsa(args, w, world, rank, local):
     ab = algorithmic(w, T_run)
     stream = torch.cuda.Stream(device=dev)
     per_step_bytes = ab["total"]
+    if w.prefill_chunk:
+        # prefill: the chunk's queries and outputs, the compressed keys and (at least once) the K
+        # and V rows of the whole prefix; the roofline of this workload is the tensor one
+        e, d, pairs = w.elem_bytes, w.head_dim, w.batch * w.num_kv_heads
+        per_step_bytes = (2 * w.batch * w.prefill_chunk * w.num_q_heads * d * e + ab["ck"]
+                          + 2 * pairs * w.seq_len * d * e)
     flush = per_step_bytes < 4 * L2_BYTES
     flush_buf = torch.empty(256 * 1024 * 1024, dtype=torch.uint8, device=dev) if flush else None
     use_graph = not args.no_graph and not bench.append
@@ -739,15 +794,28 @@ def run_bsa(args, w, world, rank, local):
     dom = max(single, key=single.get)
     kname = KERNEL_OF_PHASE[dom][w.dtype]
     n_calls = names.count(dom)  # launches of that phase per step (one per anchor)
-    achieved = kbytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
-    traffic = profile_traffic(kname, w.name)
-    roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
-                "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                "peak_kind": peak_kind + " copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
-                "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
-                "traffic": traffic, "algorithmic_bytes_per_launch": kbytes[dom] / n_calls,
-                "kernel_ms": round(kern_ms[dom] / n_calls, 5),
-                "launches_timed": "one" if "+" not in kname else "the attention kernel and its combine"}
+    if bench.prefill:
+        # a contraction: algorithmic FLOPs (scoring + attention) over the measured bf16 GEMM peak
+        from block_sparse_attention_compressed_b200.workloads import prefill_flops
+        fl = prefill_flops(w)
+        tpeak, tkind = load_tensor_peak()
+        achieved = fl["total"] / (kern_ms[dom] * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "kernel": kname, "achieved": round(achieved, 2), "peak": tpeak,
+                    "unit": "TFLOP/s", "frac": round(achieved / tpeak, 4),
+                    "peak_kind": tkind + " bf16 GEMM throughput (MEASURED_PEAKS.json bf16_tflops)",
+                    "traffic": profile_traffic(kname, w.name), "algorithmic_flops_per_launch": fl["total"],
+                    "algorithmic_flops": fl, "kernel_ms": round(kern_ms[dom], 5),
+                    "launches_timed": "the selection and the attention kernels of one bsa_prefill call"}
+    else:
+        achieved = kbytes[dom] / (kern_ms[dom] * 1e-3) / 1e9
+        traffic = profile_traffic(kname, w.name)
+        roofline = {"bound": "hbm", "kernel": kname, "achieved": round(achieved, 1),
+                    "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
+                    "peak_kind": peak_kind + " copy bandwidth (MEASURED_PEAKS.json hbm_gbs)",
+                    "frac_of_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                    "traffic": traffic, "algorithmic_bytes_per_launch": kbytes[dom] / n_calls,
+                    "kernel_ms": round(kern_ms[dom] / n_calls, 5),
+                    "launches_timed": "one" if "+" not in kname else "the attention kernel and its combine"}
 
     steps_per_s = world * K / (total_ms * 1e-3)
     gbs = per_step_bytes * world * K / (total_ms * 1e-3) / 1e9
@@ -779,13 +847,13 @@ def run_bsa(args, w, world, rank, local):
                            "a one-step graph replayed per step" if graph is not None else False),
             "step_path": "fused" if bench.fused else "chained",
         },
-        "tokens_per_s": round(steps_per_s * w.batch, 1),
+        "tokens_per_s": round(steps_per_s * w.batch * (w.prefill_chunk or 1), 1),
         "hbm_gbs": round(gbs / world, 1),
         "frac_of_8tbs": round(gbs / world / NOMINAL_HBM_GBS, 4),
-        "north_star": {"basis": "compressed keys + selected K/V + q + out bytes of the whole step "
-                                "over 8 TB/s, device-timed step", "frac_of_8tbs":
-                       round(gbs / world / NOMINAL_HBM_GBS, 4), "target": NORTH_STAR_FRAC,
-                       "met": bool(gbs / world / NOMINAL_HBM_GBS >= NORTH_STAR_FRAC)},
+        "north_star": None if bench.prefill else {
+            "basis": "compressed keys + selected K/V + q + out bytes of the whole step over 8 TB/s, "
+                     "device-timed step", "frac_of_8tbs": round(gbs / world / NOMINAL_HBM_GBS, 4),
+            "target": NORTH_STAR_FRAC, "met": bool(gbs / world / NOMINAL_HBM_GBS >= NORTH_STAR_FRAC)},
         "ms_per_step_one_step_graphs": (round(one_step_graphs_ms, 5) if one_step_graphs_ms is not None
                                         else None),
         "fused_step": bool(bench.fused),

@@ -193,6 +193,26 @@ def generate(w: Workload, device="cpu", seq_cap: int | None = None, steps: int |
     return res
 
 
+def prefill_flops(w: Workload) -> dict:
+    """FLOPs of one block-sparse prefill of the last ``prefill_chunk`` positions (every sequence at
+    seq_len): the scoring of every (position, head) against the windows complete before its tile's
+    block (2 d per product), and the attention of every (position, head) over its tile's selected
+    tokens up to itself (4 d per key: the score and the weighted value)."""
+    C, T, d, BS = w.prefill_chunk, w.seq_len, w.head_dim, w.block_size
+    heads = w.batch * w.num_q_heads
+    score = attn = 0
+    for pos in range(T - C, T):
+        r = pos // BS
+        start = BS * r
+        nc = 0 if start < w.cmp_kernel else (start - w.cmp_kernel) // w.cmp_stride + 1
+        score += nc
+        nsel = min(w.n_init + w.n_local + w.top_k, r + 1)
+        keys = BS * (nsel - 1) + (pos - start + 1) if w.n_local > 0 else BS * nsel
+        attn += keys
+    return dict(score=2 * d * heads * score, attend=4 * d * heads * attn,
+                total=2 * d * heads * score + 4 * d * heads * attn)
+
+
 def algorithmic_bytes(w: Workload, T: int | None = None) -> dict:
     """Minimum bytes one decode step moves: the compressed keys of the scored layer, the K and V
     rows of the selected blocks of every layer, q read and the output written, and for the

@@ -65,13 +65,18 @@ def test_algorithmic_bytes(name):
 
 
 @pytest.mark.parametrize("name", ["forecast-bf16-128k-b16", "anchors-2of4-64k-b8", "gqa4-bf16-32k-b1",
-                                  "lookahead-bf16-128k-b16"])
+                                  "lookahead-bf16-128k-b16", "prefill-bf16-32k-b4"])
 def test_cpu_oracle_leg_runs(name):
     """The bench's CPU-baseline / reference leg (the oracle on a bounded sample of pairs) for the
-    Forecast-indexer, anchored and plain workloads, on a shortened copy of each."""
+    Forecast-indexer, anchored, lookahead, prefill and plain workloads, on a shortened copy of each."""
+    import torch
     from block_sparse_attention_compressed_b200.workloads import generate
     w = WORKLOADS[name].replace(batch=1, seq_len=4096, needles=2)
+    if w.prefill_chunk:
+        w = w.replace(prefill_chunk=96)
     data = generate(w, device="cpu")
+    if w.prefill_chunk:
+        data["q_chunk"] = torch.randn(w.batch, w.prefill_chunk, w.num_q_heads, w.head_dim).to(w.torch_dtype)
     c = bench.cpu_oracle_sample(w, data, seconds=0.05)
     assert c["value"] > 0 and c["single_thread_value"] > 0 and c["cores"] >= 1
     assert c["compress_s_per_cache"] >= 0
