@@ -106,6 +106,7 @@ def _bind(path: str):
                                                  _P, _P, _P, _P]),
         "bsa_oracle_prefill": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _INT, _P, _INT, _INT,
                                       _P, _P, _P, _P, _P]),
+        "bsa_oracle_token_select": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _INT, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -443,6 +444,42 @@ def prefill(P: Problem, q, k_cache, v_cache, seq_lens, chunk: int, pairs=None) -
     if rc != 0:
         raise ValueError("bsa_oracle_prefill rejected its arguments")
     return res
+
+
+def token_select(P: Problem, q, k_cache, seq_lens, pairs=None) -> dict:
+    """CLSA's token-level index (``bsa_oracle_token_select``): idx [n][tok_cap] (ascending tokens,
+    -1 padded; tok_cap = (n_init + n_local + top_k) * block_size), n_sel [n], boundary [n][2]."""
+    q = _raw_check(q, P.dtype)
+    k_cache = _raw_check(k_cache, P.dtype)
+    seq_lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
+    if pairs is None:
+        pairs = np.arange(P.batch * P.num_kv_heads, dtype=np.int32)
+    pairs = np.ascontiguousarray(np.asarray(pairs, dtype=np.int32))
+    n = pairs.size
+    tok_cap = (P.n_init + P.n_local + P.top_k) * P.block_size
+    res = dict(idx=np.full((n, tok_cap), -1, dtype=np.int32), n_sel=np.zeros(n, dtype=np.int32),
+               boundary=np.full((n, 2), np.nan, dtype=np.float64))
+    rc = _load().bsa_oracle_token_select(ctypes.byref(P), _ptr(q), _ptr(k_cache), _ptr(seq_lens), _ptr(pairs),
+                                         n, _ptr(res["idx"]), _ptr(res["n_sel"]), _ptr(res["boundary"]))
+    if rc != 0:
+        raise ValueError("bsa_oracle_token_select rejected its arguments")
+    return res
+
+
+def clsa(P: Problem, qs, k_caches, v_caches, seq_lens, pairs=None) -> dict:
+    """CLSA decode over the layers of qs / k_caches / v_caches (lists, layer 0 the index layer):
+    the token index of layer 0, attended by every layer (tokens as blocks of one). Returns idx,
+    n_sel, boundary and out [L][n][G][d], lse [L][n][G]."""
+    sel = token_select(P, qs[0], k_caches[0], seq_lens, pairs)
+    P1 = Problem.from_buffer_copy(P)  # tokens as blocks of one; the index is given
+    P1.top_k = (P.n_init + P.n_local + P.top_k) * P.block_size
+    P1.block_size, P1.n_init, P1.n_local = 1, 0, 0
+    outs, lses = [], []
+    for q, k, v in zip(qs, k_caches, v_caches):
+        r = attend_pairs(P1, q, k, v, seq_lens, sel["idx"], sel["n_sel"], pairs)
+        outs.append(r["out"])
+        lses.append(r["lse"])
+    return dict(sel, out=np.stack(outs), lse=np.stack(lses))
 
 
 def attend_pairs(P: Problem, q, k_cache, v_cache, seq_lens, idx, n_sel, pairs=None) -> dict:

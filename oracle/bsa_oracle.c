@@ -464,6 +464,50 @@ int bsa_oracle_prefill(const orc_problem_t* P, const void* q, const void* k_cach
     return 0;
 }
 
+/* The token-level index of the CLSA abstract (page "HySparse2: Hybrid Sparse Attention with
+ * Two-Level KV Sharing"): one indexer selects tokens once and every layer sharing it attends them.
+ * The indexer is the base selector (Eq. 6 of the SparDA page's Indexer Training) at token
+ * granularity: S[t] = sum over the group's heads of softmax_t(q_h . K_t / tau) over the tokens
+ * t < T of the index layer's keys. The first n_init * BS and the last n_local * BS tokens are always
+ * taken, and top_k * BS more by score (ties to the lower token), ascending: Eq. 1 with blocks of one
+ * token and the block configuration's token budget. idx [n][tok_cap] (-1 padded, tok_cap =
+ * (n_init + n_local + top_k) * BS), n_sel [n], boundary [n][2] (may be NULL). */
+int bsa_oracle_token_select(const orc_problem_t* P, const void* q, const void* k_cache, const int32_t* seq_lens,
+                            const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel, double* boundary) {
+    if (!orc_problem_ok(P) || n_pairs < 0) return -1;
+    const int G = P->num_q_heads / P->num_kv_heads, d = P->head_dim, BS = P->block_size;
+    const int tok_cap = (P->n_init + P->n_local + P->top_k) * BS;
+    for (int i = 0; i < n_pairs; ++i) {
+        if (pairs[i] < 0 || pairs[i] >= P->batch * P->num_kv_heads) return -1;
+        const int64_t T = seq_lens[pairs[i] / P->num_kv_heads];
+        if (T < 0 || T > P->max_seq_len) return -1;
+    }
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int i = 0; i < n_pairs; ++i) {
+        const int pair = pairs[i], b = pair / P->num_kv_heads, kvh = pair % P->num_kv_heads;
+        const int64_t T = seq_lens[b];
+        const void* kp = orc_pair_rows(P, k_cache, pair);
+        double* keys = (double*)malloc((size_t)(T > 0 ? T : 1) * d * sizeof(double));
+        for (int64_t t = 0; t < T * d; ++t) keys[t] = bsa_oracle_load(kp, P->dtype, t);
+        double* qg = (double*)malloc((size_t)G * d * sizeof(double));
+        orc_group_q(P, q, b, kvh, qg);
+        double* S = (double*)malloc((size_t)(T > 0 ? T : 1) * sizeof(double));
+        bsa_oracle_group_scores(qg, keys, T, G, d, P->tau, S);
+        int32_t* my_idx = idx + (int64_t)i * tok_cap;
+        for (int r = 0; r < tok_cap; ++r) my_idx[r] = -1;
+        double bnd[2];
+        n_sel[i] = bsa_oracle_select(S, T, P->n_init * BS, P->n_local * BS, P->top_k * BS, my_idx, bnd);
+        if (boundary) {
+            boundary[2 * i] = bnd[0];
+            boundary[2 * i + 1] = bnd[1];
+        }
+        free(keys);
+        free(qg);
+        free(S);
+    }
+    return 0;
+}
+
 int bsa_oracle_attend_pairs(const orc_problem_t* P, const void* q, const void* k_cache,
                             const void* v_cache, const int32_t* seq_lens, const int32_t* pairs,
                             int n_pairs, const int32_t* idx, const int32_t* n_sel, double* out,

@@ -587,6 +587,35 @@ def pin_prefill_tile_selection_brute_force():
         assert got == want, (r, got, want)
 
 
+def pin_clsa_token_index_brute_force():
+    """CLSA's token index: per pair the sum over the group's heads of a softmax (torch) over every
+    token's key, the first and last tokens of the budget always taken and the rest by a plain sort
+    (ties to the lower token); every layer's output is SDPA over exactly those tokens."""
+    B, Hq, Hkv, d, T, BS = 1, 4, 2, 8, 200, 16
+    n_init, n_local, top_k = 1, 1, 3
+    L = 2
+    qs = [_randn((B, Hq, d), 111 + 3 * l) for l in range(L)]
+    ks = [_randn((B, Hkv, T, d), 112 + 3 * l) for l in range(L)]
+    vs = [_randn((B, Hkv, T, d), 113 + 3 * l) for l in range(L)]
+    P = oracle.make_problem(B, Hq, Hkv, d, T, oracle.F32, n_init, n_local, top_k, block_size=BS)
+    Tn = 170
+    res = oracle.clsa(P, [q.numpy() for q in qs], [k.numpy() for k in ks], [v.numpy() for v in vs], [Tn])
+    G = Hq // Hkv
+    for kvh in range(Hkv):
+        S = sum(torch.softmax(ks[0][0, kvh, :Tn].double() @ qs[0][0, kvh * G + h].double() / math.sqrt(d), dim=0)
+                for h in range(G))
+        fixed = set(range(n_init * BS)) | set(range(Tn - n_local * BS, Tn))
+        cand = sorted((t for t in range(Tn) if t not in fixed), key=lambda t: (-float(S[t]), t))
+        want = sorted(fixed | set(cand[:top_k * BS]))
+        assert res["idx"][kvh, :res["n_sel"][kvh]].tolist() == want
+        assert (res["idx"][kvh, res["n_sel"][kvh]:] == -1).all()
+        for l in range(L):
+            ro, rl = _sdpa(qs[l][0, kvh * G:(kvh + 1) * G].double().numpy(), ks[l][0, kvh, want].double().numpy(),
+                           vs[l][0, kvh, want].double().numpy(), 1.0 / math.sqrt(d))
+            np.testing.assert_allclose(res["out"][l, kvh], ro, rtol=1e-12, atol=1e-13)
+            np.testing.assert_allclose(res["lse"][l, kvh], rl, rtol=1e-12, atol=1e-13)
+
+
 ALL_PINS = [
     pin_round_bf16_matches_torch, pin_round_ties_even, pin_round_f32_matches_numpy,
     pin_compress_matches_avg_pool, pin_compress_constant_windows, pin_window_and_block_counts,
@@ -603,5 +632,5 @@ ALL_PINS = [
     pin_forecast_decode_composes, pin_forecast_one_head_matches_base_selector,
     pin_lookahead_step_brute_force,
     pin_prefill_single_position_is_decode, pin_prefill_all_blocks_is_causal_dense,
-    pin_prefill_tile_selection_brute_force,
+    pin_prefill_tile_selection_brute_force, pin_clsa_token_index_brute_force,
 ]
