@@ -106,7 +106,7 @@ def _bind(path: str):
                                                  _P, _P, _P, _P]),
         "bsa_oracle_prefill": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _INT, _P, _INT, _INT,
                                       _P, _P, _P, _P, _P]),
-        "bsa_oracle_token_select": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _INT, _P, _P, _P]),
+        "bsa_oracle_token_select": (_INT, [ctypes.POINTER(Problem), _P, _P, _P, _P, _INT, _P, _P, _P, _P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -448,7 +448,8 @@ def prefill(P: Problem, q, k_cache, v_cache, seq_lens, chunk: int, pairs=None) -
 
 def token_select(P: Problem, q, k_cache, seq_lens, pairs=None) -> dict:
     """CLSA's token-level index (``bsa_oracle_token_select``): idx [n][tok_cap] (ascending tokens,
-    -1 padded; tok_cap = (n_init + n_local + top_k) * block_size), n_sel [n], boundary [n][2]."""
+    -1 padded; tok_cap = (n_init + n_local + top_k) * block_size), n_sel [n], boundary [n][2] and
+    the token scores [n][max_seq_len] (-inf past each sequence)."""
     q = _raw_check(q, P.dtype)
     k_cache = _raw_check(k_cache, P.dtype)
     seq_lens = np.ascontiguousarray(np.asarray(seq_lens, dtype=np.int32))
@@ -458,9 +459,11 @@ def token_select(P: Problem, q, k_cache, seq_lens, pairs=None) -> dict:
     n = pairs.size
     tok_cap = (P.n_init + P.n_local + P.top_k) * P.block_size
     res = dict(idx=np.full((n, tok_cap), -1, dtype=np.int32), n_sel=np.zeros(n, dtype=np.int32),
-               boundary=np.full((n, 2), np.nan, dtype=np.float64))
+               boundary=np.full((n, 2), np.nan, dtype=np.float64),
+               scores=np.full((n, P.max_seq_len), -np.inf, dtype=np.float64))
     rc = _load().bsa_oracle_token_select(ctypes.byref(P), _ptr(q), _ptr(k_cache), _ptr(seq_lens), _ptr(pairs),
-                                         n, _ptr(res["idx"]), _ptr(res["n_sel"]), _ptr(res["boundary"]))
+                                         n, _ptr(res["idx"]), _ptr(res["n_sel"]), _ptr(res["boundary"]),
+                                         _ptr(res["scores"]))
     if rc != 0:
         raise ValueError("bsa_oracle_token_select rejected its arguments")
     return res

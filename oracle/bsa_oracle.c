@@ -471,9 +471,11 @@ int bsa_oracle_prefill(const orc_problem_t* P, const void* q, const void* k_cach
  * t < T of the index layer's keys. The first n_init * BS and the last n_local * BS tokens are always
  * taken, and top_k * BS more by score (ties to the lower token), ascending: Eq. 1 with blocks of one
  * token and the block configuration's token budget. idx [n][tok_cap] (-1 padded, tok_cap =
- * (n_init + n_local + top_k) * BS), n_sel [n], boundary [n][2] (may be NULL). */
+ * (n_init + n_local + top_k) * BS), n_sel [n], boundary [n][2] and the token scores
+ * scores [n][max_seq_len] (-inf past T) (both may be NULL). */
 int bsa_oracle_token_select(const orc_problem_t* P, const void* q, const void* k_cache, const int32_t* seq_lens,
-                            const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel, double* boundary) {
+                            const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel, double* boundary,
+                            double* scores) {
     if (!orc_problem_ok(P) || n_pairs < 0) return -1;
     const int G = P->num_q_heads / P->num_kv_heads, d = P->head_dim, BS = P->block_size;
     const int tok_cap = (P->n_init + P->n_local + P->top_k) * BS;
@@ -501,6 +503,8 @@ int bsa_oracle_token_select(const orc_problem_t* P, const void* q, const void* k
             boundary[2 * i] = bnd[0];
             boundary[2 * i + 1] = bnd[1];
         }
+        if (scores)
+            for (int64_t t = 0; t < P->max_seq_len; ++t) scores[(int64_t)i * P->max_seq_len + t] = t < T ? S[t] : -INFINITY;
         free(keys);
         free(qg);
         free(S);

@@ -175,10 +175,12 @@ int bsa_oracle_prefill(const orc_problem_t* P, const void* q, const void* k_cach
                        int32_t* idx, int32_t* n_sel, double* boundary, double* out, double* lse);
 /* CLSA token-level index (see bsa_oracle.c): the tokens of each listed pair that the base selector,
  * at token granularity, picks with the block configuration's token budget. idx [n][tok_cap]
- * (tok_cap = (n_init + n_local + top_k) * block_size), n_sel [n], boundary [n][2] (may be NULL).
+ * (tok_cap = (n_init + n_local + top_k) * block_size), n_sel [n], boundary [n][2] and the token
+ * scores [n][max_seq_len] (both may be NULL).
  * Every layer sharing the index attends them: bsa_oracle_attend_pairs with block_size 1. */
 int bsa_oracle_token_select(const orc_problem_t* P, const void* q, const void* k_cache, const int32_t* seq_lens,
-                            const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel, double* boundary);
+                            const int32_t* pairs, int n_pairs, int32_t* idx, int32_t* n_sel, double* boundary,
+                            double* scores);
 int bsa_oracle_select_forecast_ck(const orc_problem_t* P, const void* f, const double* ck,
                                   const int32_t* seq_lens, const int32_t* pairs, int n_pairs,
                                   int32_t* idx, int32_t* n_sel, double* block_scores, double* boundary);
