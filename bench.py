@@ -45,6 +45,7 @@ METRIC = "block-sparse decode steps/s & achieved HBM GB/s (select+attn) at 128K 
 # the library kernel behind each single-launch phase of a step, by dtype
 KERNEL_OF_PHASE = {"step": {"bf16": "step_kernel"},
                    "prefill": {"bf16": "prefill_select_kernel+prefill_attend_kernel"},
+                   "clsa": {"bf16": "score_tma_kernel+token_topk_kernel+token_decode_kernel"},
                    "decode": {"bf16": "decode_tma_kernel+combine_kernel", "f32": "decode_f32_kernel"},
                    "append": {"bf16": "append_kernel", "f32": "append_kernel"},
                    "select": {"bf16": "score_tma_kernel+select_kernel",
@@ -210,6 +211,14 @@ class Bench:
         self.path = path if single else "auto"
         self.fused = single and (path == "fused" or (path == "auto" and bsa.bsa_decode_step_info(self.p)[0]))
         self.lookahead = bool(w.lookahead)
+        self.clsa = bool(w.token_index)
+        if self.clsa:
+            # CLSA: layer 0's token-level index, attended by every layer (three launches per step)
+            self.ws = bsa.alloc_clsa_workspace(self.p, device)
+            self.tok_cap = (w.n_init + w.n_local + w.top_k) * w.block_size
+            self.tok_idx = torch.zeros(B, Hkv, self.tok_cap, dtype=torch.int32, device=device)
+            self.n_tok = torch.zeros(B, Hkv, dtype=torch.int32, device=device)
+            self.fused = True
         self.prefill = w.prefill_chunk > 0
         if self.prefill:
             # block-sparse prefill of the last prefill_chunk positions: queries drawn like q
@@ -247,6 +256,13 @@ class Bench:
         bsa, d = self.bsa, self.data
         q = self.q_of(i) if q is None else q
         ev = (lambda k: events[k].record(stream)) if events is not None else (lambda k: None)
+        if self.clsa:
+            ev(0)
+            bsa.bsa_decode_step_clsa(self.p, [q] + [d["q"][L] for L in range(1, self.w.layers)], d["k"], d["v"],
+                                     d["seq_lens"], self.tok_idx, self.n_tok, self.out, self.lse, self.ws,
+                                     stream=stream)
+            ev(1)
+            return
         if self.prefill:
             ev(0)
             bsa.bsa_prefill(self.p, self.w.prefill_chunk, self.q_chunk, d["k"][0], d["v"][0], self.ck,
@@ -326,6 +342,10 @@ class Bench:
     # Forecast-indexer workloads qs is [q, f]
     def step_io(self, qs, outs, lses, stream, k_new=None, v_new=None):
         bsa, d = self.bsa, self.data
+        if self.clsa:
+            bsa.bsa_decode_step_clsa(self.p, qs, d["k"], d["v"], d["seq_lens"], self.tok_idx, self.n_tok, outs, lses,
+                                     self.ws, stream=stream)
+            return
         if self.prefill:
             bsa.bsa_prefill(self.p, self.w.prefill_chunk, qs[0], d["k"][0], d["v"][0], self.ck, d["seq_lens"],
                             self.p_idx, self.p_ns, outs[0], lses[0], self.ws, stream=stream)
@@ -369,6 +389,8 @@ class Bench:
         """The phases pass B brackets with events, in launch order."""
         if self.prefill:
             return ["prefill"]
+        if self.clsa:
+            return ["clsa"]
         if self.fused:
             return (["append"] if self.append else []) + ["step"]
         names = ["select", "decode"] * (len(self.w.anchors) if self.w.layers > 1 else 1)
@@ -377,6 +399,8 @@ class Bench:
     def launches_per_step(self):
         if self.prefill:
             return 2  # the selection (tcgen05) and the attention
+        if self.clsa:
+            return 3  # token scoring, token top-k, token attention (all layers)
         if self.fused:
             return 1 + (1 if self.append else 0)
         # bsa_select_blocks launches two kernels (scoring, selection), the bf16 sparse attention two
@@ -523,7 +547,7 @@ def cpu_oracle_sample(w, data, seconds: float):
     f_arr = (oracle.raw(torch.stack([data["f"][b, h:h + 1] for b, h in pairs]))[0]
              if w.forecast else None)
     # A1, the compression of every scoring layer's keys (once per cache; timed apart)
-    scored = [1] if w.lookahead else ([] if w.prefill_chunk else list(w.anchors))
+    scored = [1] if w.lookahead else ([] if (w.prefill_chunk or w.token_index) else list(w.anchors))
     t0 = time.perf_counter()
     cks = {L: oracle.compress_cache(P, arrays[L][1], lens) for L in scored}
     compress_s = (time.perf_counter() - t0) * (total / n0) / max(len(scored), 1)
@@ -541,6 +565,11 @@ def cpu_oracle_sample(w, data, seconds: float):
                 sub, G, 1, w.head_dim, T_cap, P.dtype, w.n_init, w.n_local, w.top_k, w.cmp_kernel,
                 w.cmp_stride, w.block_size)
             ln = lens if sub is None else lens[:sub]
+            if w.token_index:
+                if L == 0:
+                    oracle.clsa(Ps, [a[0][idx] for a in arrays], [a[1][idx] for a in arrays],
+                                [a[2][idx] for a in arrays], ln)
+                return
             if w.prefill_chunk:
                 # the chunk's block-sparse prefill (its compression included: the chunk's keys
                 # complete new windows)
@@ -787,6 +816,7 @@ def run_bsa(args, w, world, rank, local):
     kbytes = {"select": ab["ck"] + (fv if w.forecast else q_bytes),  # compressed keys + q (or f)
               "decode": ab["kv"] + ab["qo"],         # selected K/V rows + q + out, every layer
               "step": ab["ck"] + ab["kv"] + ab["qo"] + fv,  # the fused step: all of them
+              "clsa": ab["ck"] + ab["kv"] + ab["qo"],       # the index layer's keys + every layer's tokens
               "append": ab["append"]}
     # the selection phase is two launches (scoring, then selection): the roofline is taken on the
     # largest phase that is one launch, or one launch and its combine

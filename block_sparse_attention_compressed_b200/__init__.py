@@ -12,7 +12,7 @@ from ._abi import (  # noqa: F401
     DEVERR_N_SEL, DEVERR_SEQ_LEN, LIB_PATH, BsaError, Params, Sizes, alloc_workspace,
     bsa_abi_version, bsa_check_params, bsa_compress_append, bsa_compress_keys, bsa_decode_step,
     bsa_decode_step_anchored, bsa_decode_step_info, bsa_decode_step_lookahead, bsa_prefill,
-    bsa_prefill_attend, bsa_prefill_tiles,
+    bsa_prefill_attend, bsa_prefill_tiles, bsa_decode_step_clsa, bsa_clsa_workspace_size, alloc_clsa_workspace,
     bsa_get_sizes, bsa_read_device_error, bsa_select_blocks, bsa_select_blocks_forecast,
     bsa_sparse_decode, bsa_sparse_decode_layers, bsa_sparse_decode_noalloc, bsa_workspace_init,
     bsa_workspace_size, lib, make_params, status_string,

@@ -83,6 +83,8 @@ _SIGS = {
                                    ctypes.c_size_t, _P]),
     "bsa_decode_step_lookahead": (_S, [_PP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                        ctypes.c_size_t, _P]),
+    "bsa_decode_step_clsa": (_S, [_PP, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
+    "bsa_clsa_workspace_size": (ctypes.c_size_t, [_PP]),
     "bsa_prefill": (_S, [_PP, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t, _P]),
     "bsa_prefill_attend": (_S, [_PP, ctypes.c_int32, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_size_t,
                                 _P]),
@@ -312,6 +314,42 @@ def bsa_sparse_decode_layers(p: Params, qs, k_caches, v_caches, seq_lens, block_
         _ptr(n_sel, "n_sel", torch.int32, n["pairs"]), o_a, l_a, _ptr(ws, "workspace"),
         ws.numel() * ws.element_size(), _stream(stream)),
         "bsa_sparse_decode_layers")
+
+
+def bsa_clsa_workspace_size(p: Params) -> int:
+    """Workspace bytes of bsa_decode_step_clsa (0 when unsupported)."""
+    return int(lib().bsa_clsa_workspace_size(ctypes.byref(p)))
+
+
+def alloc_clsa_workspace(p: Params, device="cuda"):
+    """A zero-initialised workspace of bsa_clsa_workspace_size bytes (torch allocates it)."""
+    import torch
+    n = bsa_clsa_workspace_size(p)
+    if n == 0:
+        raise BsaError(BSA_ERR_UNSUPPORTED, "bsa_clsa_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def bsa_decode_step_clsa(p: Params, qs, k_caches, v_caches, seq_lens, tok_idx, n_tok, outs, lses, ws,
+                         stream=None):
+    """bsa_decode_step_clsa: layer 0's token-level index, attended by every layer of the lists."""
+    import torch
+    n, e = _shapes(p), _elem(p)
+    L = len(qs)
+    if not (len(k_caches) == len(v_caches) == len(outs) == L) or (lses is not None and len(lses) != L):
+        raise ValueError("per-layer lists must have the same length")
+    arr = ctypes.c_void_p * L
+    tok_cap = (p.n_init + p.n_local + p.top_k) * p.block_size
+    q_a = arr(*[_ptr(t, "q", e, n["q"]) for t in qs])
+    k_a = arr(*[_ptr(t, "k_cache", e, n["cache"]) for t in k_caches])
+    v_a = arr(*[_ptr(t, "v_cache", e, n["cache"]) for t in v_caches])
+    o_a = arr(*[_ptr(t, "out", e, n["q"]) for t in outs])
+    l_a = None if lses is None else arr(*[_ptr(t, "lse", torch.float32, n["lse"], optional=True) for t in lses])
+    _check(lib().bsa_decode_step_clsa(
+        ctypes.byref(p), L, q_a, k_a, v_a, _ptr(seq_lens, "seq_lens", torch.int32, p.batch),
+        _ptr(tok_idx, "tok_idx", torch.int32, n["pairs"] * tok_cap), _ptr(n_tok, "n_tok", torch.int32, n["pairs"]),
+        o_a, l_a, _ptr(ws, "workspace"), ws.numel() * ws.element_size(), _stream(stream)),
+        "bsa_decode_step_clsa")
 
 
 def bsa_decode_step_anchored(p: Params, anchors, qs, k_caches, v_caches, cks, seq_lens, block_idx,

@@ -796,6 +796,87 @@ struct PrefillMapCache {
 
 extern "C" {
 
+}  // extern "C"
+
+namespace bsa {
+namespace {
+// CLSA: the plan of the token scorer (windows of one token over the index layer's keys).
+bsa_status_t clsa_plan(const bsa_params_t* params, Plan* P, Plan* F) {
+    bsa_status_t st = make_plan(params, P);
+    if (st != BSA_OK) return st;
+    if (P->dtype != BSA_BF16) return BSA_ERR_UNSUPPORTED;
+    bsa_params_t pt = *params;
+    pt.cmp_kernel = 1;
+    pt.cmp_stride = 1;
+    if ((st = make_plan(&pt, F)) != BSA_OK) return st;
+    const int64_t tok_cap = (int64_t)P->sel_cap * P->BS;
+    if (tok_cap > 0x7fffffff / 2 || token_topk_smem_bytes(F->T_cap, F->nstat, F->Gp) == 0) return BSA_ERR_UNSUPPORTED;
+    return BSA_OK;
+}
+}  // namespace
+}  // namespace bsa
+
+extern "C" {
+
+size_t bsa_clsa_workspace_size(const bsa_params_t* params) {
+    Plan P, F;
+    return clsa_plan(params, &P, &F) == BSA_OK ? F.ws_bytes : 0;
+}
+
+bsa_status_t bsa_decode_step_clsa(const bsa_params_t* params, int32_t num_layers, const void* const* q,
+                                  const void* const* k_caches, const void* const* v_caches,
+                                  const int32_t* seq_lens, int32_t* tok_idx, int32_t* n_tok, void* const* outs,
+                                  float* const* lses, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    Plan P, F;
+    bsa_status_t st = clsa_plan(params, &P, &F);
+    if (st != BSA_OK) return st;
+    if (!q || !k_caches || !v_caches || !outs) return BSA_ERR_INVALID_ARG;
+    if (num_layers < 1 || num_layers > BSA_MAX_LAYERS || num_layers > P.layers) return BSA_ERR_INVALID_ARG;
+    if (!ok4(seq_lens) || !ok4(tok_idx) || !ok4(n_tok)) return BSA_ERR_INVALID_ARG;
+    TokenLayers L;
+    memset(&L, 0, sizeof L);
+    for (int i = 0; i < num_layers; ++i) {
+        if (!ok16(q[i]) || !ok16(k_caches[i]) || !ok16(v_caches[i]) || !ok16(outs[i])) return BSA_ERR_INVALID_ARG;
+        if (lses && lses[i] && !ok4(lses[i])) return BSA_ERR_INVALID_ARG;
+        L.q[i] = q[i];
+        L.k[i] = k_caches[i];
+        L.v[i] = v_caches[i];
+        L.out[i] = outs[i];
+        L.lse[i] = lses ? lses[i] : nullptr;
+    }
+    if ((st = check_ws(F, ws, ws_bytes)) != BSA_OK) return st;
+    // token scoring of the index layer (layer 0): its K cache is the scorer's "compressed keys"
+    ScoreArgs sa = score_args(F, q[0], k_caches[0], seq_lens, ws);
+    static thread_local CUtensorMap k_map;
+    static thread_local MapKey k_key;
+    if (!encode_kv_map_cached(&k_map, &k_key, k_caches[0], (uint64_t)F.pairs * F.nc_cap, F.D, 64))
+        return BSA_ERR_CUDA;
+    if (launch_score(F, sa, &k_map, stream) != cudaSuccess) return BSA_ERR_CUDA;
+    TokenArgs a;
+    memset(&a, 0, sizeof a);
+    a.seq_lens = seq_lens;
+    a.logits = ws_at<float>(ws, F.off_logits);
+    a.stats = ws_at<float2>(ws, F.off_stats);
+    a.tok_idx = tok_idx;
+    a.n_tok = n_tok;
+    a.err = ws_at<uint32_t>(ws, F.off_err);
+    a.Hq = P.Hq;
+    a.Hkv = P.Hkv;
+    a.G = P.G;
+    a.pairs = P.pairs;
+    a.n_init_tok = P.n_init * P.BS;
+    a.n_local_tok = P.n_local * P.BS;
+    a.top_k_tok = P.top_k * P.BS;
+    a.tok_cap = P.sel_cap * P.BS;
+    a.T_cap = F.T_cap;
+    a.lg_stride = F.lg_stride;
+    a.nstat = F.nstat;
+    a.scale_log2 = P.scale_log2;
+    if (launch_token_topk(a, F.Gp, token_topk_smem_bytes(F.T_cap, F.nstat, F.Gp), stream) != cudaSuccess)
+        return BSA_ERR_CUDA;
+    return from_cuda(launch_token_decode(a, L, num_layers, P.D, stream));
+}
+
 int32_t bsa_prefill_tiles(int32_t chunk, int32_t block_size) {
     return chunk < 1 || block_size < 1 ? 0 : (chunk + block_size - 1) / block_size + 1;
 }

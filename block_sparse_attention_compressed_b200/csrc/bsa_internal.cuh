@@ -176,6 +176,30 @@ cudaError_t launch_prefill_attend(const PrefillArgs& a, const CUtensorMap* k_map
 // Dynamic shared memory of the prefill selection kernel, or 0 when it does not fit one CTA.
 size_t prefill_select_smem_bytes(int G, int64_t nc_cap, int64_t nb_cap, int sel_cap);
 
+// Token-level shared index (CLSA): the window terms and statistics of the token scorer, the token
+// lists, and the layers that attend them.
+struct TokenArgs {
+    const int32_t* seq_lens;
+    const float* logits;    // [pairs][lg_stride][Gp] window terms of the token scorer (one token per window)
+    const float2* stats;    // [pairs][nstat][Gp]
+    int32_t* tok_idx;       // [pairs][tok_cap] ascending, -1 padded
+    int32_t* n_tok;         // [pairs]
+    uint32_t* err;
+    int Hq, Hkv, G, pairs, n_init_tok, n_local_tok, top_k_tok, tok_cap;
+    int64_t T_cap, lg_stride, nstat;
+    float scale_log2;
+};
+struct TokenLayers {
+    const void* q[BSA_MAX_LAYERS];
+    const void* k[BSA_MAX_LAYERS];
+    const void* v[BSA_MAX_LAYERS];
+    void* out[BSA_MAX_LAYERS];
+    float* lse[BSA_MAX_LAYERS];
+};
+cudaError_t launch_token_topk(const TokenArgs& a, int Gp, size_t smem, cudaStream_t st);
+cudaError_t launch_token_decode(const TokenArgs& a, const TokenLayers& L, int layers, int D, cudaStream_t st);
+size_t token_topk_smem_bytes(int64_t T_cap, int64_t nstat, int Gp);
+
 // TMA descriptors of the step: compressed keys (boxes of 64 rows), K and V (boxes of 32 rows).
 struct alignas(64) StepMaps {
     CUtensorMap ck, k, v;

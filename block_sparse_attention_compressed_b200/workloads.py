@@ -49,6 +49,7 @@ class Workload:
     forecast: bool = False  # select with one Forecast vector per GQA group (f = the group's mean q)
     lookahead: bool = False  # (two layers, forecast) layer 0 attends given blocks and selects layer 1's
     prefill_chunk: int = 0   # >0: block-sparse prefill of the last prefill_chunk positions
+    token_index: bool = False  # (several layers) CLSA: layer 0's token-level index, reused by every layer
     anchors: tuple = (0,)   # multi-layer: layers that select; the others reuse the last anchor's
 
     @property
@@ -67,7 +68,7 @@ class Workload:
         return dataclasses.replace(self, **kw)
 
 
-# The workloads: one small parity case, seven decode throughput cases and one prefill case.
+# The workloads: one small parity case, eight decode throughput cases and one prefill case.
 WORKLOADS: dict[str, Workload] = {
     w.name: w
     for w in [
@@ -96,6 +97,9 @@ WORKLOADS: dict[str, Workload] = {
         Workload("prefill-bf16-32k-b4", batch=4, num_q_heads=32, num_kv_heads=8, head_dim=128,
                  seq_len=32768, dtype="bf16", n_init=1, n_local=4, top_k=64, needles=8, seed=1009,
                  prefill_chunk=4096),
+        Workload("clsa-4x32k-b8", batch=8, num_q_heads=32, num_kv_heads=8, head_dim=128,
+                 seq_len=32768, dtype="bf16", n_init=1, n_local=2, top_k=48, needles=8, seed=1010,
+                 layers=4, token_index=True),
     ]
 }
 DEFAULT_WORKLOAD = "gqa4-bf16-128k-b16"
@@ -229,6 +233,10 @@ def algorithmic_bytes(w: Workload, T: int | None = None) -> dict:
         sel_tokens -= nb * w.block_size - T
     ck = pairs * nc * d * e * len(w.anchors)   # every anchor layer scores its compressed keys
     attended = 1 if w.lookahead else w.layers  # lookahead: one layer attends, the next one is scored
+    if w.token_index:
+        # CLSA: the index layer's every key is scored; each layer reads the taken tokens' rows
+        ck = pairs * T * d * e
+        sel_tokens = min((w.n_init + w.n_local + w.top_k) * w.block_size, T)
     kv = attended * pairs * sel_tokens * d * e * 2
     qo = attended * w.batch * w.num_q_heads * d * e * 2
     app = 0

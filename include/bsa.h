@@ -277,6 +277,31 @@ bsa_status_t bsa_decode_step_lookahead(const bsa_params_t* params, const void* q
                                        float* lse, void* workspace, size_t workspace_bytes,
                                        cudaStream_t stream);
 
+/* Token-level shared index (page "HySparse2: Hybrid Sparse Attention with Two-Level KV Sharing",
+ * CLSA abstract: one indexer computes a token-level top-k once and the layers reuse it). The index
+ * is the base selector at token granularity on layer 0: per (batch, kv head),
+ * S[t] = sum over the group's query heads of softmax_t(q_h . K_t / tau) over the tokens t < T of
+ * k_caches[0] (no compression). The first n_init * block_size and the last n_local * block_size
+ * tokens are always taken, and top_k * block_size more by score (ties to the lower token); the
+ * ascending token list goes to tok_idx [batch][num_kv_heads][(n_init + n_local + top_k) *
+ * block_size] (-1 padded) with its length in n_tok [batch][num_kv_heads]. Every layer
+ * i < num_layers (<= params->num_layers, <= BSA_MAX_LAYERS) then attends exactly those tokens with
+ * its own q[i] [batch][num_q_heads][head_dim], k_caches[i] and v_caches[i] (as bsa_sparse_decode's)
+ * into outs[i] and lses[i] (lses, or an entry of it, may be NULL). q, k_caches, v_caches, outs and
+ * lses are HOST arrays of device pointers. The workspace must hold bsa_clsa_workspace_size(params)
+ * bytes (the token scorer's terms: about 4 * num_kv_heads * max_seq_len * 4 B per sequence).
+ * Supported: bf16, max_seq_len up to about 50K tokens (the token keys of a sequence, 4 bytes each,
+ * sit in one CTA's shared memory); others return BSA_ERR_UNSUPPORTED. Queued on `stream`, no host
+ * sync. */
+bsa_status_t bsa_decode_step_clsa(const bsa_params_t* params, int32_t num_layers, const void* const* q,
+                                  const void* const* k_caches, const void* const* v_caches,
+                                  const int32_t* seq_lens, int32_t* tok_idx, int32_t* n_tok, void* const* outs,
+                                  float* const* lses, void* workspace, size_t workspace_bytes,
+                                  cudaStream_t stream);
+
+/* Workspace bytes of bsa_decode_step_clsa for these parameters (host only); 0 when unsupported. */
+size_t bsa_clsa_workspace_size(const bsa_params_t* params);
+
 /* Block-sparse prefill of a chunk (page "SparDA: Sparse Decoupled Attention for Efficient
  * Long-Context LLM Inference", Theoretical Foundation, Eq. 1, and the prefill workload of its
  * Efficiency Results; one selection per query tile, as the tile-level operations of the page "CoSA:

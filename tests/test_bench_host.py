@@ -58,14 +58,17 @@ def test_algorithmic_bytes(name):
     assert ab["total"] == pytest.approx(ab["ck"] + ab["kv"] + ab["qo"] + ab["append"] + ab["f"])
     pairs, e, d = w.batch * w.num_kv_heads, w.elem_bytes, w.head_dim
     nc = (w.seq_len - w.cmp_kernel) // w.cmp_stride + 1
-    assert ab["ck"] == pairs * nc * d * e * len(w.anchors)
+    if w.token_index:
+        assert ab["ck"] == pairs * w.seq_len * d * e  # every key of the index layer is scored
+    else:
+        assert ab["ck"] == pairs * nc * d * e * len(w.anchors)
     assert ab["f"] == (pairs * d * e if w.forecast else 0)
     if name == "gqa4-bf16-128k-b16":
         assert ab["total"] == 558071808   # 268.40 MB of compressed keys + 289.41 MB of K/V + q, out
 
 
 @pytest.mark.parametrize("name", ["forecast-bf16-128k-b16", "anchors-2of4-64k-b8", "gqa4-bf16-32k-b1",
-                                  "lookahead-bf16-128k-b16", "prefill-bf16-32k-b4"])
+                                  "lookahead-bf16-128k-b16", "prefill-bf16-32k-b4", "clsa-4x32k-b8"])
 def test_cpu_oracle_leg_runs(name):
     """The bench's CPU-baseline / reference leg (the oracle on a bounded sample of pairs) for the
     Forecast-indexer, anchored, lookahead, prefill and plain workloads, on a shortened copy of each."""
