@@ -441,7 +441,8 @@ def load_peaks():
 # the host side that plans the launch.
 KERNEL_SOURCES = {"step": "step_kernels.cu", "decode": "decode_kernels.cu", "combine": "decode_kernels.cu",
                   "score": "select_kernels.cu", "select": "select_kernels.cu",
-                  "compress": "compress_kernels.cu", "append": "compress_kernels.cu"}
+                  "compress": "compress_kernels.cu", "append": "compress_kernels.cu",
+                  "prefill": "prefill_kernels.cu", "token": "clsa_kernels.cu"}
 
 
 def _code_only(text: str) -> str:
@@ -478,8 +479,17 @@ def kernel_source_hash(kernel: str | None = None) -> str:
         paths = sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh")))
     else:
         own = next(f for k, f in KERNEL_SOURCES.items() if kernel.startswith(k))
-        # the kernel's own file and the device headers (the host-side launch code is left out)
-        paths = [os.path.join(csrc, n) for n in (own, "bsa_internal.cuh", "tiles.cuh", "topk.cuh")]
+        # the kernel's own file and the headers it includes, transitively (the host-side launch
+        # code is left out)
+        names, todo = [], [own]
+        while todo:
+            n = todo.pop(0)
+            if n in names or not os.path.exists(os.path.join(csrc, n)):
+                continue  # (the public header lies outside csrc/)
+            names.append(n)
+            with open(os.path.join(csrc, n), encoding="utf-8") as f:
+                todo += re.findall(r'^#include "([^"]+)"', f.read(), flags=re.M)
+        paths = [os.path.join(csrc, n) for n in names if os.path.exists(os.path.join(csrc, n))]
     h = hashlib.sha256()
     for p in paths:
         with open(p, encoding="utf-8") as f:

@@ -213,7 +213,8 @@ __device__ void topk_union(const SelectArgs& a, int nb, uint32_t* keys, TopkSmem
                     }
                 }
             } else {
-                for (int i = seg_lo; i < seg_hi; ++i) {
+                // keys in shared memory: a strided walk (consecutive lanes, consecutive words)
+                for (int i = clo + tid; i < chi; i += NT) {
                     kand &= keys[i];
                     kor |= keys[i];
                 }
@@ -247,7 +248,7 @@ __device__ void topk_union(const SelectArgs& a, int nb, uint32_t* keys, TopkSmem
                     for (int e = 0; e < kKeysPerThread; ++e)
                         if (seg_lo + e < seg_hi && (kr[e] & mask) == prefix) atomicAdd(&hist[(kr[e] >> shift) & dmask], 1);
                 } else {
-                    for (int i = seg_lo; i < seg_hi; ++i) {
+                    for (int i = clo + tid; i < chi; i += NT) {
                         const uint32_t u = keys[i];
                         if ((u & mask) == prefix) atomicAdd(&hist[(u >> shift) & dmask], 1);
                     }
@@ -368,30 +369,60 @@ __device__ void topk_union(const SelectArgs& a, int nb, uint32_t* keys, TopkSmem
         return;
     }
 
-    // streamed candidates: mark the taken ones in keys[] (1 / 0), ties at thr in block order
+    // streamed candidates (keys in shared memory): the warps walk 32-block chunks, lane l taking
+    // block 32c + l, so every read is conflict-free; block order comes from per-chunk counts
+    // (ballots) and a scan over the chunks. The bins are free now and hold those counts.
     {
-        int cnt = 0;
-        for (int i = seg_lo; i < seg_hi; ++i) cnt += (keys[i] == thr);
-        int tot;
-        int r = block_exclusive_scan(cnt, s_warp, &tot, gp);
-        for (int i = seg_lo; i < seg_hi; ++i) {
-            const uint32_t u = keys[i];
-            const bool take = kk > 0 && (take_all || u > thr || (u == thr && r < need));
-            r += (u == thr);
-            keys[i] = take ? 1u : 0u;
+        const int lane = tid & 31, warp = tid >> 5, nwarps = NT >> 5;
+        const int nch = (nb + 31) / 32;
+        const unsigned lt = (1u << lane) - 1u;
+        int* eqc = hist;                   // [nch] keys equal to thr, then their exclusive prefix
+        int* tkc = hist + kHistBins / 2;   // [nch] blocks in the union, then their exclusive prefix
+        // in-place exclusive prefix over arr[0 .. n), in chunk order; returns the total
+        auto chunk_scan = [&](int* arr, int n) -> int {
+            const int cpt = (n + NT - 1) / NT;
+            const int lo = tid * cpt, hi = min(lo + cpt, n);
+            int sum = 0;
+            for (int c = lo; c < hi; ++c) sum += arr[c];
+            int tot;
+            int base = block_exclusive_scan(sum, s_warp, &tot, gp);
+            for (int c = lo; c < hi; ++c) {
+                const int v = arr[c];
+                arr[c] = base;
+                base += v;
+            }
+            gp.sync();
+            return tot;
+        };
+        for (int c = warp; c < nch; c += nwarps) {
+            const int i = 32 * c + lane;
+            const bool eq = i >= clo && i < chi && keys[i] == thr;
+            const unsigned m = __ballot_sync(0xffffffffu, eq);
+            if (lane == 0) eqc[c] = __popc(m);
         }
-    }
-    gp.sync();
-    // union with init and local blocks, emitted in ascending block order
-    {
-        const int per2 = (nb + NT - 1) / NT;
-        const int lo = tid * per2, hi = min(lo + per2, nb);
-        int cnt = 0;
-        for (int i = lo; i < hi; ++i) cnt += (i < init_end || i >= chi || keys[i] != 0u);
-        int total;
-        int pos = block_exclusive_scan(cnt, s_warp, &total, gp);
-        for (int i = lo; i < hi; ++i)
-            if (i < init_end || i >= chi || keys[i] != 0u) out[pos++] = i;
+        gp.sync();
+        chunk_scan(eqc, nch);
+        // taken flags into keys[] (1 / 0): init and local blocks, candidates above thr, and the
+        // first `need` candidates equal to thr in block order
+        for (int c = warp; c < nch; c += nwarps) {
+            const int i = 32 * c + lane;
+            const bool cand = i >= clo && i < chi;
+            const uint32_t u = cand ? keys[i] : 0u;
+            const unsigned m = __ballot_sync(0xffffffffu, cand && u == thr);
+            const int r = eqc[c] + __popc(m & lt);  // candidates equal to thr before block i
+            const bool fl = i < nb && (!cand || (kk > 0 && (take_all || u > thr || (u == thr && r < need))));
+            const unsigned fm = __ballot_sync(0xffffffffu, fl);
+            if (lane == 0) tkc[c] = __popc(fm);
+            if (i < nb) keys[i] = fl ? 1u : 0u;
+        }
+        gp.sync();
+        const int total = chunk_scan(tkc, nch);
+        for (int c = warp; c < nch; c += nwarps) {
+            const int i = 32 * c + lane;
+            const bool fl = i < nb && keys[i] != 0u;
+            const unsigned fm = __ballot_sync(0xffffffffu, fl);
+            if (fl) out[tkc[c] + __popc(fm & lt)] = i;
+        }
         for (int i = total + tid; i < a.sel_cap; i += NT) out[i] = -1;
         if (tid == 0) *n_out = total;
     }
