@@ -21,8 +21,15 @@
 // buffers), read back with tcgen05.ld by four epilogue warps; one warp issues the TMA copies and one
 // thread the MMAs (tcgen05.mma, completion through tcgen05.commit on shared-memory barriers).
 //
-// Attention kernel (mma.m16n8k16): a CTA per (pair, tile, pair of heads), four warps of 16 query
-// positions per head; the selected blocks' K and V rows stream through a TMA ring.
+// Attention kernel (tcgen05): a CTA per (pair, tile) holds the tile's R rows in shared memory as
+// 128-row halves; the selected blocks' K and V rows stream through a TMA ring. For each block one
+// thread issues S = Q K^T (M = 128 rows, N = 64 keys) into a double-buffered TMEM accumulator per
+// half; four warps per half read it back (one row per thread), take the online softmax in the log2
+// domain and write P as bf16 into shared memory in the operand layout; the same thread then issues
+// O += P V (N = 128, V read MN-major from its TMA rows) into a TMEM accumulator. S of the next block
+// is issued ahead of P V of this one, so the tensor cores work while the softmax runs. A row's
+// reference maximum moves only when the block maximum exceeds it by more than 8 (log2), so P stays
+// below 2^8 and O is rescaled in TMEM rarely; O / sum is exact either way.
 #include "bsa_internal.cuh"
 #include "topk.cuh"
 
@@ -344,35 +351,65 @@ __global__ void __launch_bounds__(kPsThreads, 1)
 }
 
 // ------------------------------------------------------------------------------ attention kernel
-constexpr int kPaWarps = 8;              // two heads x four warps of 16 positions
-constexpr int kPaThreads = (kPaWarps + 1) * 32;
-constexpr int kPaSlots = 4;              // K + V block stages in flight
-constexpr uint32_t kPaBox = 64u * 128u;  // 64 rows x 64 columns
-constexpr uint32_t kPaStage = 4u * kPaBox;  // K (two boxes) and V (two boxes) of one 64-token block
+constexpr int kPaSlots = 3;                    // K + V block stages in flight
+constexpr uint32_t kPaBox = 64u * 128u;        // 64 rows x 64 columns of bf16
+constexpr uint32_t kPaStage = 4u * kPaBox;     // K (two boxes) and V (two boxes) of one 64-token block
+constexpr uint32_t kPaPBytes = 128u * 128u;    // P of one 128-row half: 128 rows x 64 keys of bf16
 constexpr uint32_t kPaPolls = 1u << 26;
+constexpr float kPaHeadroom = 8.f;             // log2 growth of a row maximum absorbed without rescaling O
 
-__global__ void __launch_bounds__(kPaThreads, 1)
+// Shared-memory descriptor of an MN-major operand in the 128-byte swizzle: 64 values of the N
+// dimension per 128-byte row, one row per K index, 8-row groups 1024 bytes apart and the next 64
+// values of N `lbo` bytes further (V as the B operand of P V: N = d, K = keys).
+__device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t saddr, uint32_t lbo) {
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) | (64ull << 32) |
+           (1ull << 46) | (2ull << 61);
+}
+// P V: bf16 x bf16 -> fp32, M = 128 rows, N = 128 values of d, A (P) K-major, B (V) MN-major.
+constexpr uint32_t kPaIdescPV = umma_idesc_bf16(128, 128) | (1u << 16);
+
+// H: 128-row halves of the tile (G = 2: one; G = 4: two). Warp 0 issues the TMA copies, warp 1
+// allocates tensor memory and one of its threads issues the MMAs; warps 2 .. 2 + 4H - 1 run the
+// softmax of half (warp - 2) / 4, one tile row per thread (its TMEM lane).
+template <int H>
+__global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
     prefill_attend_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap k_map,
                           const __grid_constant__ CUtensorMap v_map) {
+    constexpr int R = 128 * H;
     extern __shared__ uint8_t dsm_raw[];
-    __shared__ __align__(8) uint64_t full[kPaSlots], empty[kPaSlots];
-    uint8_t* ring = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);
+    __shared__ __align__(8) uint64_t full[kPaSlots], empty[kPaSlots], qready, fin;
+    __shared__ __align__(8) uint64_t s_full[H][2], p_full[H][2], p_free[H][2], o_done[H];
+    __shared__ uint32_t s_tmem;
+    uint8_t* qt = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);  // 2 boxes x R rows x 128 B
+    uint8_t* ring = qt + 2 * R * 128;
+    uint8_t* pbuf = ring + kPaSlots * kPaStage;  // [H][2] x 128 rows x 128 B
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    // item: (pair, tile, head pair)
-    const int hp_n = (a.G + 1) / 2;
-    const int item = blockIdx.x;
-    const int hp = item % hp_n;
-    const int g = item / hp_n;  // pair * tiles_cap + tile
+    const int g = blockIdx.x;  // pair * tiles_cap + tile
     const int pair = g / a.tiles_cap, ti = g - pair * a.tiles_cap;
     const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kPaSlots; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], kPaWarps);
+            mbar_init(&empty[i], 1);
+        }
+        mbar_init(&qready, 128 * H);
+        mbar_init(&fin, 1);
+        for (int h = 0; h < H; ++h) {
+            for (int u = 0; u < 2; ++u) {
+                mbar_init(&s_full[h][u], 1);
+                mbar_init(&p_full[h][u], 128);
+                mbar_init(&p_free[h][u], 1);
+            }
+            mbar_init(&o_done[h], 1);
         }
         mbar_fence_init();
     }
+    if (warp == 1) tmem_alloc(&s_tmem, 256 * H);
+    tmem_fence_before_sync();
     __syncthreads();
+    tmem_fence_after_sync();
+    // TMEM columns: S of half h, buffer u at 64 (2h + u); O of half h at 128 H + 128 h
+    const uint32_t tbase = s_tmem;
     pdl_trigger();
     pdl_wait();
     const int64_t T = a.seq_lens[b];
@@ -381,185 +418,241 @@ __global__ void __launch_bounds__(kPaThreads, 1)
     const bool live = ok && r <= (T - 1) / a.BS;
     const int nsel = live ? min(max(a.n_sel[g], 0), a.sel_cap) : 0;
     const int32_t* idx = a.block_idx + (size_t)g * a.sel_cap;
+    // entries outside blocks 0 .. r are skipped by every role alike; j counts the others
 
-    if (warp == kPaWarps) {
-        // ---- producer: the selected blocks' K and V rows
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
         if (lane == 0) {
-            const uint64_t pol = l2_evict_first_policy();
-            int kk = 0;  // stages issued (entries outside blocks 0 .. r are skipped by every warp alike)
+            int j = 0;
             for (int i = 0; i < nsel; ++i) {
                 const int blk = idx[i];
                 if (blk < 0 || blk > r) continue;
-                const int slot = kk % kPaSlots;
-                if (kk >= kPaSlots && !mbar_wait(&empty[slot], (uint32_t)((kk / kPaSlots) - 1) & 1u, kPaPolls)) {
+                const int slot = j % kPaSlots;
+                if (j >= kPaSlots && !mbar_wait(&empty[slot], (uint32_t)((j / kPaSlots) - 1) & 1u, kPaPolls)) {
                     atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
                     break;
                 }
                 uint8_t* dst = ring + (size_t)slot * kPaStage;
                 mbar_arrive_expect_tx(&full[slot], kPaStage);
                 const int y = (int)((int64_t)pair * a.T_cap + (int64_t)blk * a.BS);
-                tma_load_2d_hint(dst, &k_map, 0, y, &full[slot], pol);
-                tma_load_2d_hint(dst + kPaBox, &k_map, 64, y, &full[slot], pol);
-                tma_load_2d_hint(dst + 2 * kPaBox, &v_map, 0, y, &full[slot], pol);
-                tma_load_2d_hint(dst + 3 * kPaBox, &v_map, 64, y, &full[slot], pol);
-                ++kk;
+                tma_load_2d(dst, &k_map, 0, y, &full[slot]);
+                tma_load_2d(dst + kPaBox, &k_map, 64, y, &full[slot]);
+                tma_load_2d(dst + 2 * kPaBox, &v_map, 0, y, &full[slot]);
+                tma_load_2d(dst + 3 * kPaBox, &v_map, 64, y, &full[slot]);
+                ++j;
             }
+            // every copy issued has landed before the CTA ends (they already have, unless a wait gave up)
+            for (int jj = max(j - kPaSlots, 0); jj < j; ++jj)
+                if (!mbar_wait(&full[jj % kPaSlots], (uint32_t)(jj / kPaSlots) & 1u, kPaPolls)) {
+                    atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                    break;
+                }
         }
-        return;
-    }
-    // ---- consumers: warp w takes head 2 hp + (w >> 2), positions 16 (w & 3) .. + 15 of the tile
-    const int h = 2 * hp + (warp >> 2);
-    const bool hvalid = h < a.G;
-    const int g8 = lane >> 2, tq = lane & 3;
-    const int prow0 = 16 * (warp & 3);            // first position (within the block) of the warp
-    const int64_t blk_start = (int64_t)a.BS * r;
-    // positions of this thread's two rows (g8 and g8 + 8 of the warp's 16)
-    const int64_t pa = blk_start + prow0 + g8, pb = pa + 8;
-    const bool va = live && hvalid && pa >= t0 && pa < T, vb = live && hvalid && pb >= t0 && pb < T;
-    // Q fragments (A operand, rows g8 / g8 + 8, columns 16 ks + 2 tq (+1), + 8)
-    uint32_t qf[8][4];
-    {
-        const uint16_t* q16 = reinterpret_cast<const uint16_t*>(a.q);
-        const size_t hq = (size_t)kvh * a.G + (hvalid ? h : 0);
-        const uint32_t* ra = va ? reinterpret_cast<const uint32_t*>(q16 + (((size_t)b * a.chunk + (size_t)(pa - t0)) * a.Hq + hq) * 128) : nullptr;
-        const uint32_t* rb = vb ? reinterpret_cast<const uint32_t*>(q16 + (((size_t)b * a.chunk + (size_t)(pb - t0)) * a.Hq + hq) * 128) : nullptr;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            qf[ks][0] = ra ? ra[8 * ks + tq] : 0u;
-            qf[ks][1] = rb ? rb[8 * ks + tq] : 0u;
-            qf[ks][2] = ra ? ra[8 * ks + 4 + tq] : 0u;
-            qf[ks][3] = rb ? rb[8 * ks + 4 + tq] : 0u;
-        }
-    }
-    float o[16][4];
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.f;
-    float mrow[2] = {-INFINITY, -INFINITY}, lrow[2] = {0.f, 0.f};
-    const float sl = a.scale_log2;
-    const int mi = lane >> 3, ri = lane & 7;
-    bool dead = false;
-    int ns_ = 0;  // stages consumed
-    for (int i = 0; i < nsel; ++i) {
-        const int blk = idx[i];
-        if (blk < 0 || blk > r) continue;
-        const int slot = ns_ % kPaSlots;
-        if (!dead && !mbar_wait(&full[slot], (uint32_t)(ns_ / kPaSlots) & 1u, kPaPolls)) {
-            if (lane == 0) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
-            dead = true;
-        }
-        const uint8_t* kst = ring + (size_t)slot * kPaStage;
-        const uint8_t* vst = kst + 2 * kPaBox;
-        // S = Q K^T: 16 rows x 64 keys (eight 8-key tiles), fp32
-        float sc[8][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {  // two 8-key tiles per ldmatrix.x4
-                const int key = 16 * np + ri + 8 * (mi >> 1);
-                const int ch = (ks & 3) * 2 + (mi & 1);
-                uint32_t bf[4];
-                ldmatrix_x4(bf, smem_u32(kst + (ks >> 2) * kPaBox + key * 128 + ((ch ^ (key & 7)) << 4)));
-                mma_bf16_16816(sc[2 * np], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], bf[0], bf[1]);
-                mma_bf16_16816(sc[2 * np + 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], bf[2], bf[3]);
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            int n = 0;
+            for (int i = 0; i < nsel; ++i) {
+                const int blk = idx[i];
+                n += (blk >= 0 && blk <= r) ? 1 : 0;
             }
-        }
-        // causal mask on the tile's own block; scale to the log2 domain
-        const int64_t kbase = (int64_t)blk * a.BS;
-        float mx[2] = {-INFINITY, -INFINITY};
+            const uint32_t qt_a = smem_u32(qt), ring_a = smem_u32(ring), p_a = smem_u32(pbuf);
+            // S_h(j) = Q_h K_j^T into buffer j & 1 of half h
+            auto issue_s = [&](int j) -> bool {
+                const int slot = j % kPaSlots;
+                if (!mbar_wait(&full[slot], (uint32_t)(j / kPaSlots) & 1u, kPaPolls)) return false;
+                tmem_fence_after_sync();
+                const uint32_t st_a = ring_a + (uint32_t)slot * kPaStage;
+                for (int h = 0; h < H; ++h) {
+                    const uint32_t d = tbase + (uint32_t)(64 * (2 * h + (j & 1)));
 #pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t off = (uint32_t)((ks & 3) * 32);
+                        umma_bf16(d, umma_desc_k_sw128(qt_a + (uint32_t)((ks >> 2) * R * 128 + h * 128 * 128) + off),
+                                  umma_desc_k_sw128(st_a + (uint32_t)((ks >> 2) * kPaBox) + off),
+                                  umma_idesc_bf16(128, 64), ks > 0);
+                    }
+                    umma_commit(&s_full[h][j & 1]);
+                }
+                return true;
+            };
+            bool stop = n > 0 && (!mbar_wait(&qready, 0, kPaPolls) || !issue_s(0));
+            for (int j = 0; j < n && !stop; ++j) {
+                // S of the next block goes ahead of this block's P V (its buffer was read by the
+                // softmax of block j - 1, which P V of block j - 1 waited for)
+                if (j + 1 < n && !issue_s(j + 1)) {
+                    stop = true;
+                    break;
+                }
+                const uint32_t v_a = ring_a + (uint32_t)(j % kPaSlots) * kPaStage + 2 * kPaBox;
+                for (int h = 0; h < H && !stop; ++h) {
+                    if (!mbar_wait(&p_full[h][j & 1], (uint32_t)(j >> 1) & 1u, kPaPolls)) {
+                        stop = true;
+                        break;
+                    }
+                    tmem_fence_after_sync();
+                    const uint32_t pa = p_a + (uint32_t)((2 * h + (j & 1)) * kPaPBytes);
+                    const uint32_t d = tbase + (uint32_t)(128 * H + 128 * h);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int64_t key = kbase + 8 * nt + 2 * tq + (e & 1);
-                const int64_t pos = (e < 2) ? pa : pb;
-                const float x = (key <= pos && key < T) ? sc[nt][e] * sl : -INFINITY;
-                sc[nt][e] = x;
-                mx[e >> 1] = fmaxf(mx[e >> 1], x);
+                    for (int kk = 0; kk < 4; ++kk)  // 16 keys per MMA
+                        umma_bf16(d, umma_desc_k_sw128(pa + (uint32_t)(kk * 32)),
+                                  umma_desc_mn_sw128(v_a + (uint32_t)(kk * 2048), kPaBox), kPaIdescPV,
+                                  (j > 0 || kk > 0) ? 1u : 0u);
+                    umma_commit(&p_free[h][j & 1]);
+                    umma_commit(&o_done[h]);
+                }
+                if (!stop) umma_commit(&empty[j % kPaSlots]);
             }
+            if (stop) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+            // every MMA issued has completed before the tensor memory is released
+            umma_commit(&fin);
+            if (!mbar_wait(&fin, 0, kPaPolls)) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
         }
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-            mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 1));
-            mx[rr] = fmaxf(mx[rr], __shfl_xor_sync(0xffffffffu, mx[rr], 2));
-        }
-        float alpha[2], ref[2];
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-            const float mn = fmaxf(mrow[rr], mx[rr]);
-            alpha[rr] = mn == -INFINITY ? 1.f : exp2f(mrow[rr] - mn);
-            ref[rr] = mn == -INFINITY ? 0.f : mn;
-            mrow[rr] = mn;
-        }
-        float ps[2] = {0.f, 0.f};
-        // P as the A operand of P V (four 16-key steps), split into bf16 hi + lo parts so that the
-        // products keep about 16 significant bits
-        uint32_t pf[4][4], pl[4][4];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            const float p0 = exp2f(sc[nt][0] - ref[0]), p1 = exp2f(sc[nt][1] - ref[0]);
-            const float p2 = exp2f(sc[nt][2] - ref[1]), p3 = exp2f(sc[nt][3] - ref[1]);
-            ps[0] += p0 + p1;
-            ps[1] += p2 + p3;
-            const int kq = nt >> 1, hi = nt & 1;
-            const uint32_t h01 = pack_bf16x2(p0, p1), h23 = pack_bf16x2(p2, p3);
-            pf[kq][2 * hi] = h01;
-            pf[kq][2 * hi + 1] = h23;
-            pl[kq][2 * hi] = pack_bf16x2(p0 - bf16_lo(h01), p1 - bf16_hi(h01));
-            pl[kq][2 * hi + 1] = pack_bf16x2(p2 - bf16_lo(h23), p3 - bf16_hi(h23));
-        }
-#pragma unroll
-        for (int rr = 0; rr < 2; ++rr) lrow[rr] = lrow[rr] * alpha[rr] + ps[rr];
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            o[nt][0] *= alpha[0];
-            o[nt][1] *= alpha[0];
-            o[nt][2] *= alpha[1];
-            o[nt][3] *= alpha[1];
-        }
-        // O += P V: V^T fragments from the swizzled V rows (ldmatrix.trans)
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-#pragma unroll
-            for (int dp = 0; dp < 8; ++dp) {  // two 8-column tiles of d per ldmatrix.x4
-                const int key = 16 * kk + ri + 8 * (mi & 1);
-                const int ch = 2 * dp + (mi >> 1);
-                uint32_t vf[4];
-                ldmatrix_x4_trans(vf, smem_u32(vst + (ch >> 3) * kPaBox + key * 128 + (((ch & 7) ^ (key & 7)) << 4)));
-                mma_bf16_16816(o[2 * dp], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], vf[0], vf[1]);
-                mma_bf16_16816(o[2 * dp + 1], pf[kk][0], pf[kk][1], pf[kk][2], pf[kk][3], vf[2], vf[3]);
-                mma_bf16_16816(o[2 * dp], pl[kk][0], pl[kk][1], pl[kk][2], pl[kk][3], vf[0], vf[1]);
-                mma_bf16_16816(o[2 * dp + 1], pl[kk][0], pl[kk][1], pl[kk][2], pl[kk][3], vf[2], vf[3]);
+    } else {
+        // ---------------------------------------------------------------- softmax warps
+        const int h = (warp - 2) >> 2;                  // half of the tile
+        const int quarter = warp & 3;                   // TMEM lanes 32 * quarter ..
+        const int m = 32 * quarter + lane;              // row within the half (TMEM lane)
+        const int row = 128 * h + m;                    // tile row: position-in-block * G + head
+        const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+        const int G = a.G;
+        // the tile's rows into shared memory, K-major with the 128-byte swizzle; rows outside the
+        // chunk are zero
+        if (live) {
+            for (int e = threadIdx.x - 64; e < R * 16; e += 128 * H) {
+                const int rr = e >> 4, ch = e & 15;
+                const int cp = rr / G, hh = rr - cp * G;
+                const int64_t p = (int64_t)a.BS * r + cp;
+                uint4 v = make_uint4(0, 0, 0, 0);
+                if (rr < 64 * G && p >= t0 && p < T)
+                    v = *reinterpret_cast<const uint4*>(reinterpret_cast<const uint16_t*>(a.q) +
+                                                        (((size_t)b * a.chunk + (size_t)(p - t0)) * a.Hq +
+                                                         (size_t)kvh * G + hh) * 128 + ch * 8);
+                *reinterpret_cast<uint4*>(qt + (ch >> 3) * R * 128 + rr * 128 + (((ch & 7) ^ (rr & 7)) << 4)) = v;
             }
+            fence_proxy_async_smem();
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[slot]);
-        ++ns_;
-    }
-    // row sums across the quad, then O / l
+        mbar_arrive(&qready);
+        const int cpos = row / G, hd = row - cpos * G;
+        const int64_t pos = (int64_t)a.BS * r + cpos;
+        const bool valid = live && row < 64 * G && pos >= t0 && pos < T;
+        const float sl = a.scale_log2;
+        const uint32_t t_o = tbase + lane_off + (uint32_t)(128 * H + 128 * h);
+        float m_used = -INFINITY, lsum = 0.f;  // log2-domain reference maximum and sum of the row
+        bool dead = false;
+        int j = 0;
+        for (int i = 0; i < nsel; ++i) {
+            const int blk = idx[i];
+            if (blk < 0 || blk > r) continue;
+            const int u = j & 1;
+            if (!dead && !mbar_wait(&s_full[h][u], (uint32_t)(j >> 1) & 1u, kPaPolls)) {
+                atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                dead = true;
+            }
+            tmem_fence_after_sync();
+            float x0[32], x1[32];
+            const uint32_t t_s = tbase + lane_off + (uint32_t)(64 * (2 * h + u));
+            tmem_ld<32>(t_s, x0);
+            tmem_ld<32>(t_s + 32, x1);
+            tmem_wait_ld();
+            // causal mask inside the tile's own block; log2 domain
+            const int lim = blk == r ? cpos : 63;
+            float mx = -INFINITY;
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        lrow[rr] += __shfl_xor_sync(0xffffffffu, lrow[rr], 1);
-        lrow[rr] += __shfl_xor_sync(0xffffffffu, lrow[rr], 2);
-    }
-    __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out);
+            for (int c = 0; c < 32; ++c) {
+                x0[c] = c <= lim ? x0[c] * sl : -INFINITY;
+                x1[c] = c + 32 <= lim ? x1[c] * sl : -INFINITY;
+                mx = fmaxf(mx, fmaxf(x0[c], x1[c]));
+            }
+            // the reference maximum moves (and O and the sum are rescaled) only when the row's
+            // maximum exceeds it by more than the headroom: P stays below 2^8
+            const bool need = mx > m_used + kPaHeadroom;
+            if (__any_sync(0xffffffffu, need)) {
+                const float mn = need ? mx : m_used;
+                const float alpha = m_used == -INFINITY ? 0.f : exp2f(m_used - mn);
+                if (j > 0) {
+                    // O holds P V of blocks 0 .. j - 1 once the last of them has completed
+                    if (!dead && !mbar_wait(&o_done[h], (uint32_t)(j - 1) & 1u, kPaPolls)) {
+                        atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                        dead = true;
+                    }
+                    tmem_fence_after_sync();
+#pragma unroll 1
+                    for (int cc = 0; cc < 4; ++cc) {
+                        float o[32];
+                        tmem_ld<32>(t_o + (uint32_t)(32 * cc), o);
+                        tmem_wait_ld();
 #pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-        const bool v = rr == 0 ? va : vb;
-        if (!v) continue;
-        const int64_t pos = rr == 0 ? pa : pb;
-        const size_t row = ((size_t)b * a.chunk + (size_t)(pos - t0)) * a.Hq + (size_t)kvh * a.G + h;
-        const float inv = lrow[rr] > 0.f ? 1.f / lrow[rr] : 0.f;
+                        for (int e = 0; e < 32; ++e) o[e] *= alpha;
+                        tmem_st<32>(t_o + (uint32_t)(32 * cc), o);
+                    }
+                    tmem_wait_st();
+                }
+                lsum *= alpha;
+                m_used = mn;
+            }
+            uint32_t pk[32];
+            float ps = 0.f;
+            const float mref = m_used == -INFINITY ? 0.f : m_used;  // a row with no finite score so far
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-            const int d0 = 8 * nt + 2 * tq;
-            const uint32_t pk = pack_bf16x2(o[nt][2 * rr] * inv, o[nt][2 * rr + 1] * inv);
-            *reinterpret_cast<uint32_t*>(out + row * 128 + d0) = pk;
+            for (int c = 0; c < 16; ++c) {
+                const float p0 = exp2f(x0[2 * c] - mref), p1 = exp2f(x0[2 * c + 1] - mref);
+                const float p2 = exp2f(x1[2 * c] - mref), p3 = exp2f(x1[2 * c + 1] - mref);
+                ps += (p0 + p1) + (p2 + p3);
+                pk[c] = pack_bf16x2(p0, p1);
+                pk[16 + c] = pack_bf16x2(p2, p3);
+            }
+            lsum += ps;
+            // P buffer u was last read by P V of block j - 2
+            if (j >= 2 && !dead && !mbar_wait(&p_free[h][u], (uint32_t)((j >> 1) - 1) & 1u, kPaPolls)) {
+                atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                dead = true;
+            }
+            uint8_t* prow = pbuf + (size_t)(2 * h + u) * kPaPBytes + (size_t)m * 128;
+#pragma unroll
+            for (int ch = 0; ch < 8; ++ch)
+                *reinterpret_cast<uint4*>(prow + ((ch ^ (m & 7)) << 4)) =
+                    make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+            fence_proxy_async_smem();
+            tmem_fence_before_sync();
+            mbar_arrive(&p_full[h][u]);
+            ++j;
         }
-        if (a.lse && tq == 0)
-            a.lse[row] = lrow[rr] > 0.f ? (mrow[rr] + log2f(lrow[rr])) * 0.69314718055994531f : -INFINITY;
+        // ---- O / sum of the row
+        const size_t orow = ((size_t)b * a.chunk + (size_t)(valid ? pos - t0 : 0)) * a.Hq + (size_t)kvh * G + hd;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + orow * 128;
+        if (j > 0) {
+            if (!dead && !mbar_wait(&o_done[h], (uint32_t)(j - 1) & 1u, kPaPolls)) {
+                atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
+                dead = true;
+            }
+            tmem_fence_after_sync();
+            const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+#pragma unroll 1
+            for (int cc = 0; cc < 4; ++cc) {
+                float o[32];
+                tmem_ld<32>(t_o + (uint32_t)(32 * cc), o);
+                tmem_wait_ld();
+                if (valid) {
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4)
+                        *reinterpret_cast<uint4*>(out + 32 * cc + 8 * q4) =
+                            make_uint4(pack_bf16x2(o[8 * q4] * inv, o[8 * q4 + 1] * inv),
+                                       pack_bf16x2(o[8 * q4 + 2] * inv, o[8 * q4 + 3] * inv),
+                                       pack_bf16x2(o[8 * q4 + 4] * inv, o[8 * q4 + 5] * inv),
+                                       pack_bf16x2(o[8 * q4 + 6] * inv, o[8 * q4 + 7] * inv));
+                }
+            }
+        } else if (valid) {
+            for (int q4 = 0; q4 < 16; ++q4) *reinterpret_cast<uint4*>(out + 8 * q4) = make_uint4(0, 0, 0, 0);
+        }
+        if (valid && a.lse)
+            a.lse[orow] = lsum > 0.f ? (m_used + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
     }
+    tmem_fence_before_sync();
+    __syncthreads();
+    tmem_fence_after_sync();
+    if (warp == 1) tmem_dealloc(tbase, 256 * H);
 }
 
 }  // namespace
@@ -572,7 +665,10 @@ size_t prefill_select_smem_bytes(int G, int64_t nc_cap, int64_t nb_cap, int sel_
     return bytes <= limit ? bytes : 0;
 }
 
-size_t prefill_attend_smem_bytes() { return 1024 + (size_t)kPaSlots * kPaStage; }
+size_t prefill_attend_smem_bytes(int G) {
+    const int H = G > 2 ? 2 : 1;
+    return 1024 + (size_t)2 * 128 * H * 128 + (size_t)kPaSlots * kPaStage + (size_t)2 * H * kPaPBytes;
+}
 
 cudaError_t launch_prefill_select(const PrefillArgs& a, const CUtensorMap* ck_map, size_t smem, int ctas,
                                   cudaStream_t st) {
@@ -589,12 +685,17 @@ cudaError_t launch_prefill_select(const PrefillArgs& a, const CUtensorMap* ck_ma
 
 cudaError_t launch_prefill_attend(const PrefillArgs& a, const CUtensorMap* k_map, const CUtensorMap* v_map,
                                   cudaStream_t st) {
-    const int64_t items = (int64_t)a.pairs * a.tiles_cap * ((a.G + 1) / 2);
+    const int64_t items = (int64_t)a.pairs * a.tiles_cap;
     if (items <= 0) return cudaSuccess;
-    const size_t smem = prefill_attend_smem_bytes();
-    cudaError_t e = ensure_smem<prefill_attend_kernel>(smem);
+    const size_t smem = prefill_attend_smem_bytes(a.G);
+    if (a.G == 2) {
+        cudaError_t e = ensure_smem<prefill_attend_kernel<1>>(smem);
+        if (e != cudaSuccess) return e;
+        return launch_pdl(prefill_attend_kernel<1>, dim3((unsigned)items), dim3(6 * 32), smem, st, a, *k_map, *v_map);
+    }
+    cudaError_t e = ensure_smem<prefill_attend_kernel<2>>(smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(prefill_attend_kernel, dim3((unsigned)items), dim3(kPaThreads), smem, st, a, *k_map, *v_map);
+    return launch_pdl(prefill_attend_kernel<2>, dim3((unsigned)items), dim3(10 * 32), smem, st, a, *k_map, *v_map);
 }
 
 }  // namespace bsa
