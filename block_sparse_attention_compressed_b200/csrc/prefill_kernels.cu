@@ -18,8 +18,9 @@
 // gives each row its softmax maximum and sum (one row per TMEM lane: no cross-thread reduction);
 // pass 2, windows x rows (M = 128 windows, N = R), gives each window the sum over the rows of its
 // probability (one window per TMEM lane). The accumulators live in tensor memory (two 256-column
-// buffers), read back with tcgen05.ld by four epilogue warps; one warp issues the TMA copies and one
-// thread the MMAs (tcgen05.mma, completion through tcgen05.commit on shared-memory barriers).
+// buffers), read back with tcgen05.ld by eight epilogue warps, two per TMEM lane quarter, each
+// taking half of the columns; one warp issues the TMA copies and one thread the MMAs (tcgen05.mma,
+// completion through tcgen05.commit on shared-memory barriers).
 //
 // Attention kernel (tcgen05): a CTA per (pair, tile) holds the tile's R rows in shared memory as
 // 128-row halves; the selected blocks' K and V rows stream through a TMA ring. For each block one
@@ -63,7 +64,9 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 }
 
 // ------------------------------------------------------------------------------ selection kernel
-constexpr int kPsWarps = 6;             // producer, MMA issuer, four epilogue warps
+constexpr int kPsEpiWarps = 8;          // two groups of four epilogue warps
+constexpr int kPsEpiThreads = kPsEpiWarps * 32;
+constexpr int kPsWarps = 2 + kPsEpiWarps;  // producer, MMA issuer, epilogue
 constexpr int kPsThreads = kPsWarps * 32;
 constexpr int kPsSlots = 3;             // compressed-key stages in flight
 constexpr int kPsChunk = 128;           // windows per stage
@@ -110,8 +113,9 @@ __global__ void __launch_bounds__(kPsThreads, 1)
     __shared__ int s_nsel;
     uint8_t* qt = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);  // 2 boxes x R rows x 128 B
     uint8_t* ring = qt + 2 * R * 128;
-    float2* stats = reinterpret_cast<float2*>(ring + kPsSlots * kPsSlotBytes);  // [R] (max, 1/sum), log2 domain
-    float* S = reinterpret_cast<float*>(stats + R);                            // [nc_cap] window scores
+    float2* part = reinterpret_cast<float2*>(ring + kPsSlots * kPsSlotBytes);  // [2][128] (max, sum) per group
+    float* mz = reinterpret_cast<float*>(part + 256);  // [R] max + log2(sum) of each row, log2 domain
+    float* S = mz + R;                                 // [nc_cap] window scores
     uint32_t* keys = reinterpret_cast<uint32_t*>(S + ((a.nc_cap + 3) & ~int64_t(3)));  // [nb_cap]
     int32_t* sel = reinterpret_cast<int32_t*>(keys + ((a.nb_cap + 3) & ~int64_t(3)));
 
@@ -123,9 +127,9 @@ __global__ void __launch_bounds__(kPsThreads, 1)
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&accf[i], 1);
-            mbar_init(&acce[i], 4);
+            mbar_init(&acce[i], kPsEpiWarps);
         }
-        mbar_init(&qready, 128);
+        mbar_init(&qready, kPsEpiThreads);
         mbar_fence_init();
     }
     if (warp == 1) tmem_alloc(&s_tmem, 512);
@@ -214,9 +218,15 @@ __global__ void __launch_bounds__(kPsThreads, 1)
         }
     } else {
         // ---------------------------------------------------------------- epilogue warps
-        const int et = threadIdx.x - 64;                    // 0..127
-        const Grp grp{et, 128, kPsEpiBar};
+        // Group eg (warps 2 + 4 eg .. 5 + 4 eg) reads NL = R / 2 columns of each accumulator: in
+        // pass 1 the windows of its half (R = 128) or all 128 windows of row block eg (R = 256); in
+        // pass 2 the rows eg NL .. eg NL + NL - 1.
+        constexpr int NL = R / 2;
+        const int et = threadIdx.x - 64;                    // 0 .. 255
+        const int eg = et >> 7;
+        const Grp grp{et, kPsEpiThreads, kPsEpiBar};
         const int quarter = warp & 3;                       // TMEM lanes 32 * quarter ..
+        const int ml = 32 * quarter + lane;                 // this thread's TMEM lane
         const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
         SelectArgs sa;
         memset(&sa, 0, sizeof sa);
@@ -231,7 +241,7 @@ __global__ void __launch_bounds__(kPsThreads, 1)
             const PsItem it = ps_item(a, g);
             int32_t* oidx = a.block_idx + (size_t)g * a.sel_cap;
             if (!it.live || dead) {
-                for (int i = et; i < a.sel_cap; i += 128) oidx[i] = -1;
+                for (int i = et; i < a.sel_cap; i += kPsEpiThreads) oidx[i] = -1;
                 if (et == 0) a.n_sel[g] = 0;
                 continue;
             }
@@ -239,7 +249,7 @@ __global__ void __launch_bounds__(kPsThreads, 1)
             // the tile's rows into shared memory (row = position-in-block * G + head), K-major with
             // the 128-byte swizzle; rows outside the chunk are zero
             const int G = a.G;
-            for (int e = et; e < R * 16; e += 128) {
+            for (int e = et; e < R * 16; e += kPsEpiThreads) {
                 const int row = e >> 4, ch = e & 15;
                 const int cpos = row / G, h = row - cpos * G;
                 const int64_t p = (int64_t)a.BS * it.r + cpos;
@@ -252,10 +262,9 @@ __global__ void __launch_bounds__(kPsThreads, 1)
             }
             fence_proxy_async_smem();
             mbar_arrive(&qready);
-            // ---- pass 1: each thread's rows (one per 128-row block): softmax maximum and sum
-            float m[MB], z[MB];
-#pragma unroll
-            for (int mb = 0; mb < MB; ++mb) m[mb] = -INFINITY, z[mb] = 0.f;
+            // ---- pass 1: the softmax maximum and sum of row (R = 256: eg * 128 +) ml over the
+            // group's windows
+            float m = -INFINITY, z = 0.f;
             for (int c = 0; c < it.nch; ++c, ++n) {
                 const int buf = (int)(n & 1);
                 if (!dead && !mbar_wait(&accf[buf], (uint32_t)(n >> 1) & 1u, kPsPolls)) {
@@ -263,46 +272,50 @@ __global__ void __launch_bounds__(kPsThreads, 1)
                     dead = true;
                 }
                 tmem_fence_after_sync();
+                float v[NL];
 #pragma unroll
-                for (int mb = 0; mb < MB; ++mb) {
-#pragma unroll
-                    for (int pc = 0; pc < kPsChunk / 32; ++pc) {
-                        float v[32];
-                        tmem_ld<32>(tbase + lane_off + (uint32_t)(buf * 256 + mb * 128 + pc * 32), v);
-                        tmem_wait_ld();
-                        const int j0 = kPsChunk * c + 32 * pc;
-                        const int nv = min(32, it.nc - j0);  // valid windows of this piece
-                        float mx = -INFINITY;
-#pragma unroll
-                        for (int e = 0; e < 32; ++e) {
-                            v[e] *= sl;
-                            if (e < nv) mx = fmaxf(mx, v[e]);
-                        }
-                        if (nv > 0) {
-                            const float mn = fmaxf(m[mb], mx);
-                            float acc = 0.f;
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                if (e < nv) acc += exp2f(v[e] - mn);
-                            z[mb] = (m[mb] == -INFINITY ? 0.f : z[mb] * exp2f(m[mb] - mn)) + acc;
-                            m[mb] = mn;
-                        }
-                    }
-                }
+                for (int pc = 0; pc < NL / 32; ++pc)
+                    tmem_ld<32>(tbase + lane_off + (uint32_t)(buf * 256 + eg * NL + pc * 32),
+                                *reinterpret_cast<float(*)[32]>(v + 32 * pc));
+                tmem_wait_ld();
                 tmem_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acce[buf]);
-            }
+                const int nv = min(NL, it.nc - (kPsChunk * c + (R == 128 ? eg * NL : 0)));  // valid windows
+                if (nv > 0) {
+                    float mx = -INFINITY;
 #pragma unroll
-            for (int mb = 0; mb < MB; ++mb) {
-                const int row = mb * 128 + 32 * quarter + lane;
-                const int cpos = row / G;
-                const int64_t p = (int64_t)a.BS * it.r + cpos;
-                const bool valid = row < 64 * G && p >= it.t0 && p < it.T && z[mb] > 0.f;
-                stats[row] = valid ? make_float2(m[mb], 1.f / z[mb]) : make_float2(0.f, 0.f);
+                    for (int e = 0; e < NL; ++e)
+                        if (e < nv) mx = fmaxf(mx, v[e]);
+                    const float mn = fmaxf(m, mx * sl);  // sl > 0: max(v) sl = max(v sl)
+                    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int e = 0; e < NL; ++e)
+                        if (e < nv) acc[e & 3] += exp2f(fmaf(v[e], sl, -mn));
+                    z = (m == -INFINITY ? 0.f : z * exp2f(m - mn)) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+                    m = mn;
+                }
             }
+            part[eg * 128 + ml] = make_float2(m, z);
             grp.sync();
-            // ---- pass 2: each thread's window of every stage: the sum over the rows of exp2(x - max) / sum
+            // merge the groups' halves (R = 128) and form max + log2(sum) per row; zero the scores
+            for (int row = et; row < R; row += kPsEpiThreads) {
+                float2 mzr = part[row];
+                if (R == 128) {
+                    const float2 o = part[128 + row];
+                    const float mn = fmaxf(mzr.x, o.x);
+                    if (mn != -INFINITY)
+                        mzr = make_float2(mn, (mzr.y > 0.f ? mzr.y * exp2f(mzr.x - mn) : 0.f) +
+                                                  (o.y > 0.f ? o.y * exp2f(o.x - mn) : 0.f));
+                }
+                const int64_t p = (int64_t)a.BS * it.r + row / G;
+                const bool valid = row < 64 * G && p >= it.t0 && p < it.T && mzr.y > 0.f;
+                mz[row] = valid ? mzr.x + log2f(mzr.y) : INFINITY;  // a row outside the chunk adds 0
+            }
+            for (int j = et; j < it.nc; j += kPsEpiThreads) S[j] = 0.f;
+            grp.sync();
+            // ---- pass 2: window kPsChunk c + ml of each stage: the sum over the group's rows of
+            // exp2(x - max - log2 sum); the two groups' sums meet in S (0 + a + b is exact in either order)
             for (int c = 0; c < it.nch; ++c, ++n) {
                 const int buf = (int)(n & 1);
                 if (!dead && !mbar_wait(&accf[buf], (uint32_t)(n >> 1) & 1u, kPsPolls)) {
@@ -310,28 +323,32 @@ __global__ void __launch_bounds__(kPsThreads, 1)
                     dead = true;
                 }
                 tmem_fence_after_sync();
-                float acc = 0.f;
-#pragma unroll 1
-                for (int pc = 0; pc < R / 32; ++pc) {
-                    float v[32];
-                    tmem_ld<32>(tbase + lane_off + (uint32_t)(buf * 256 + pc * 32), v);
-                    tmem_wait_ld();
+                float v[NL];
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        const float2 st = stats[32 * pc + e];
-                        if (st.y > 0.f) acc += exp2f(v[e] * sl - st.x) * st.y;
-                    }
-                }
+                for (int pc = 0; pc < NL / 32; ++pc)
+                    tmem_ld<32>(tbase + lane_off + (uint32_t)(buf * 256 + eg * NL + pc * 32),
+                                *reinterpret_cast<float(*)[32]>(v + 32 * pc));
+                tmem_wait_ld();
                 tmem_fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&acce[buf]);
-                const int j = kPsChunk * c + 32 * quarter + lane;
-                if (j < it.nc) S[j] = acc;
+                const float4* mz4 = reinterpret_cast<const float4*>(mz + eg * NL);
+                float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int e4 = 0; e4 < NL / 4; ++e4) {
+                    const float4 w = mz4[e4];
+                    acc[0] += exp2f(fmaf(v[4 * e4], sl, -w.x));
+                    acc[1] += exp2f(fmaf(v[4 * e4 + 1], sl, -w.y));
+                    acc[2] += exp2f(fmaf(v[4 * e4 + 2], sl, -w.z));
+                    acc[3] += exp2f(fmaf(v[4 * e4 + 3], sl, -w.w));
+                }
+                const int j = kPsChunk * c + ml;
+                if (j < it.nc) atomicAdd(&S[j], (acc[0] + acc[1]) + (acc[2] + acc[3]));
             }
             grp.sync();
             // ---- block maxima over blocks 0 .. r: block b's windows are 4b - 1 .. 4b + 3
             const int nb = (int)it.r + 1;
-            for (int bb = et; bb < nb; bb += 128) {
+            for (int bb = et; bb < nb; bb += kPsEpiThreads) {
                 float mx = -INFINITY;
                 for (int j = max(4 * bb - 1, 0); j <= 4 * bb + 3 && j < it.nc; ++j) mx = fmaxf(mx, S[j]);
                 keys[bb] = order_key(mx);
@@ -339,9 +356,9 @@ __global__ void __launch_bounds__(kPsThreads, 1)
             grp.sync();
             topk_union(sa, nb, keys, tk, false, grp, sel, &s_nsel);
             grp.sync();
-            for (int i = et; i < a.sel_cap; i += 128) oidx[i] = sel[i];
+            for (int i = et; i < a.sel_cap; i += kPsEpiThreads) oidx[i] = sel[i];
             if (et == 0) a.n_sel[g] = s_nsel;
-            grp.sync();  // sel, keys and stats are rewritten by the next item
+            grp.sync();  // sel, keys, mz and S are rewritten by the next item
         }
     }
     tmem_fence_before_sync();
@@ -659,7 +676,7 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
 
 size_t prefill_select_smem_bytes(int G, int64_t nc_cap, int64_t nb_cap, int sel_cap) {
     const int R = 64 * G;
-    size_t bytes = 1024 + (size_t)2 * R * 128 + (size_t)kPsSlots * kPsSlotBytes + (size_t)R * sizeof(float2);
+    size_t bytes = 1024 + (size_t)2 * R * 128 + (size_t)kPsSlots * kPsSlotBytes + 256 * sizeof(float2) + (size_t)R * 4;
     bytes += (size_t)((nc_cap + 3) & ~int64_t(3)) * 4 + (size_t)((nb_cap + 3) & ~int64_t(3)) * 4 + (size_t)sel_cap * 4;
     const size_t limit = 227 * 1024 - sizeof(TopkSmem) - 256;
     return bytes <= limit ? bytes : 0;
