@@ -63,6 +63,14 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
                  : "memory");
 }
 
+// 2^x by the special-function unit (PTX ex2.approx.ftz: relative error about 2^-22, results below
+// 2^-126 flushed to zero, 2^-inf = 0).
+__device__ __forceinline__ float ex2_ftz(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
 // ------------------------------------------------------------------------------ selection kernel
 constexpr int kPsEpiWarps = 8;          // two groups of four epilogue warps
 constexpr int kPsEpiThreads = kPsEpiWarps * 32;
@@ -283,16 +291,16 @@ __global__ void __launch_bounds__(kPsThreads, 1)
                 if (lane == 0) mbar_arrive(&acce[buf]);
                 const int nv = min(NL, it.nc - (kPsChunk * c + (R == 128 ? eg * NL : 0)));  // valid windows
                 if (nv > 0) {
-                    float mx = -INFINITY;
+                    float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
                     for (int e = 0; e < NL; ++e)
-                        if (e < nv) mx = fmaxf(mx, v[e]);
-                    const float mn = fmaxf(m, mx * sl);  // sl > 0: max(v) sl = max(v sl)
+                        if (e < nv) mq[e & 3] = fmaxf(mq[e & 3], v[e]);
+                    const float mn = fmaxf(m, fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl);  // sl > 0
                     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int e = 0; e < NL; ++e)
-                        if (e < nv) acc[e & 3] += exp2f(fmaf(v[e], sl, -mn));
-                    z = (m == -INFINITY ? 0.f : z * exp2f(m - mn)) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
+                        if (e < nv) acc[e & 3] += ex2_ftz(fmaf(v[e], sl, -mn));
+                    z = (m == -INFINITY ? 0.f : z * ex2_ftz(m - mn)) + ((acc[0] + acc[1]) + (acc[2] + acc[3]));
                     m = mn;
                 }
             }
@@ -337,10 +345,10 @@ __global__ void __launch_bounds__(kPsThreads, 1)
 #pragma unroll
                 for (int e4 = 0; e4 < NL / 4; ++e4) {
                     const float4 w = mz4[e4];
-                    acc[0] += exp2f(fmaf(v[4 * e4], sl, -w.x));
-                    acc[1] += exp2f(fmaf(v[4 * e4 + 1], sl, -w.y));
-                    acc[2] += exp2f(fmaf(v[4 * e4 + 2], sl, -w.z));
-                    acc[3] += exp2f(fmaf(v[4 * e4 + 3], sl, -w.w));
+                    acc[0] += ex2_ftz(fmaf(v[4 * e4], sl, -w.x));
+                    acc[1] += ex2_ftz(fmaf(v[4 * e4 + 1], sl, -w.y));
+                    acc[2] += ex2_ftz(fmaf(v[4 * e4 + 2], sl, -w.z));
+                    acc[3] += ex2_ftz(fmaf(v[4 * e4 + 3], sl, -w.w));
                 }
                 const int j = kPsChunk * c + ml;
                 if (j < it.nc) atomicAdd(&S[j], (acc[0] + acc[1]) + (acc[2] + acc[3]));
@@ -414,7 +422,7 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
         for (int h = 0; h < H; ++h) {
             for (int u = 0; u < 2; ++u) {
                 mbar_init(&s_full[h][u], 1);
-                mbar_init(&p_full[h][u], 128);
+                mbar_init(&p_full[h][u], 4);
                 mbar_init(&p_free[h][u], 1);
             }
             mbar_init(&o_done[h], 1);
@@ -572,21 +580,29 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
             tmem_ld<32>(t_s, x0);
             tmem_ld<32>(t_s + 32, x1);
             tmem_wait_ld();
-            // causal mask inside the tile's own block; log2 domain
-            const int lim = blk == r ? cpos : 63;
-            float mx = -INFINITY;
+            // causal mask inside the tile's own block
+            if (blk == r) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) {
-                x0[c] = c <= lim ? x0[c] * sl : -INFINITY;
-                x1[c] = c + 32 <= lim ? x1[c] * sl : -INFINITY;
-                mx = fmaxf(mx, fmaxf(x0[c], x1[c]));
+                for (int c = 0; c < 32; ++c) {
+                    x0[c] = c <= cpos ? x0[c] : -INFINITY;
+                    x1[c] = c + 32 <= cpos ? x1[c] : -INFINITY;
+                }
             }
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int c = 0; c < 32; c += 2) {
+                mq[0] = fmaxf(mq[0], x0[c]);
+                mq[1] = fmaxf(mq[1], x0[c + 1]);
+                mq[2] = fmaxf(mq[2], x1[c]);
+                mq[3] = fmaxf(mq[3], x1[c + 1]);
+            }
+            const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl;  // log2 domain (sl > 0)
             // the reference maximum moves (and O and the sum are rescaled) only when the row's
             // maximum exceeds it by more than the headroom: P stays below 2^8
             const bool need = mx > m_used + kPaHeadroom;
             if (__any_sync(0xffffffffu, need)) {
                 const float mn = need ? mx : m_used;
-                const float alpha = m_used == -INFINITY ? 0.f : exp2f(m_used - mn);
+                const float alpha = m_used == -INFINITY ? 0.f : ex2_ftz(m_used - mn);
                 if (j > 0) {
                     // O holds P V of blocks 0 .. j - 1 once the last of them has completed
                     if (!dead && !mbar_wait(&o_done[h], (uint32_t)(j - 1) & 1u, kPaPolls)) {
@@ -609,17 +625,20 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
                 m_used = mn;
             }
             uint32_t pk[32];
-            float ps = 0.f;
-            const float mref = m_used == -INFINITY ? 0.f : m_used;  // a row with no finite score so far
+            float ps[4] = {0.f, 0.f, 0.f, 0.f};
+            const float nref = m_used == -INFINITY ? 0.f : -m_used;  // a row with no finite score so far
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                const float p0 = exp2f(x0[2 * c] - mref), p1 = exp2f(x0[2 * c + 1] - mref);
-                const float p2 = exp2f(x1[2 * c] - mref), p3 = exp2f(x1[2 * c + 1] - mref);
-                ps += (p0 + p1) + (p2 + p3);
+                const float p0 = ex2_ftz(fmaf(x0[2 * c], sl, nref)), p1 = ex2_ftz(fmaf(x0[2 * c + 1], sl, nref));
+                const float p2 = ex2_ftz(fmaf(x1[2 * c], sl, nref)), p3 = ex2_ftz(fmaf(x1[2 * c + 1], sl, nref));
+                ps[0] += p0;
+                ps[1] += p1;
+                ps[2] += p2;
+                ps[3] += p3;
                 pk[c] = pack_bf16x2(p0, p1);
                 pk[16 + c] = pack_bf16x2(p2, p3);
             }
-            lsum += ps;
+            lsum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
             // P buffer u was last read by P V of block j - 2
             if (j >= 2 && !dead && !mbar_wait(&p_free[h][u], (uint32_t)((j >> 1) - 1) & 1u, kPaPolls)) {
                 atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
@@ -632,7 +651,8 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
                     make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
             fence_proxy_async_smem();
             tmem_fence_before_sync();
-            mbar_arrive(&p_full[h][u]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[h][u]);
             ++j;
         }
         // ---- O / sum of the row
