@@ -25,10 +25,11 @@
 // Attention kernel (tcgen05): a CTA per (pair, tile) holds the tile's R rows in shared memory as
 // 128-row halves; the selected blocks' K and V rows stream through a TMA ring. For each block one
 // thread issues S = Q K^T (M = 128 rows, N = 64 keys) into a double-buffered TMEM accumulator per
-// half; four warps per half read it back (one row per thread), take the online softmax in the log2
-// domain and write P as bf16 into shared memory in the operand layout; the same thread then issues
-// O += P V (N = 128, V read MN-major from its TMA rows) into a TMEM accumulator. S of the next block
-// is issued ahead of P V of this one, so the tensor cores work while the softmax runs. A row's
+// half; eight warps per half read it back (two threads per row, 32 scores each), take the online
+// softmax in the log2 domain and write P as bf16 over S in TMEM; the same thread then issues
+// O += P V (A = P from TMEM, N = 128, V read MN-major from its TMA rows) into a TMEM accumulator.
+// The issuing thread takes whichever is ready first, S of a later block or P V of a half whose P is
+// written, so the tensor cores work while the softmax runs. A row's
 // reference maximum moves only when the block maximum exceeds it by more than 8 (log2), so P stays
 // below 2^8 and O is rescaled in TMEM rarely; O / sum is exact either way.
 #include "bsa_internal.cuh"
@@ -376,10 +377,9 @@ __global__ void __launch_bounds__(kPsThreads, 1)
 }
 
 // ------------------------------------------------------------------------------ attention kernel
-constexpr int kPaSlots = 3;                    // K + V block stages in flight
+constexpr int kPaSlots = 4;                    // K + V block stages in flight
 constexpr uint32_t kPaBox = 64u * 128u;        // 64 rows x 64 columns of bf16
 constexpr uint32_t kPaStage = 4u * kPaBox;     // K (two boxes) and V (two boxes) of one 64-token block
-constexpr uint32_t kPaPBytes = 128u * 128u;    // P of one 128-row half: 128 rows x 64 keys of bf16
 constexpr uint32_t kPaPolls = 1u << 26;
 constexpr float kPaHeadroom = 8.f;             // log2 growth of a row maximum absorbed without rescaling O
 
@@ -390,40 +390,60 @@ __device__ __forceinline__ uint64_t umma_desc_mn_sw128(uint32_t saddr, uint32_t 
     return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) | (64ull << 32) |
            (1ull << 46) | (2ull << 61);
 }
-// P V: bf16 x bf16 -> fp32, M = 128 rows, N = 128 values of d, A (P) K-major, B (V) MN-major.
+// P V: bf16 x bf16 -> fp32, M = 128 rows, N = 128 values of d, A (P, in TMEM) K-major, B (V) MN-major.
 constexpr uint32_t kPaIdescPV = umma_idesc_bf16(128, 128) | (1u << 16);
+// D (TMEM) = A (TMEM: row i in lane i, two bf16 per 32-bit column) * B^T (+ D when acc).
+__device__ __forceinline__ void umma_bf16_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t bdesc, uint32_t idesc,
+                                             uint32_t acc) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+        " tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n}\n" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(bdesc), "r"(idesc), "r"(acc)
+        : "memory");
+}
+// Non-blocking test of a barrier phase (true once the phase with the given parity has completed).
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+        " selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
 
 // H: 128-row halves of the tile (G = 2: one; G = 4: two). Warp 0 issues the TMA copies, warp 1
-// allocates tensor memory and one of its threads issues the MMAs; warps 2 .. 2 + 4H - 1 run the
-// softmax of half (warp - 2) / 4, one tile row per thread (its TMEM lane).
+// allocates tensor memory and one of its threads issues the MMAs; warps 2 .. 2 + 8H - 1 run the
+// softmax of half (warp - 2) / 8, two threads per tile row (its TMEM lane), 32 scores each.
 template <int H>
-__global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
+__global__ void __launch_bounds__((2 + 8 * H) * 32, 1)
     prefill_attend_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap k_map,
                           const __grid_constant__ CUtensorMap v_map) {
     constexpr int R = 128 * H;
     extern __shared__ uint8_t dsm_raw[];
-    __shared__ __align__(8) uint64_t full[kPaSlots], empty[kPaSlots], qready, fin;
-    __shared__ __align__(8) uint64_t s_full[H][2], p_full[H][2], p_free[H][2], o_done[H];
+    __shared__ __align__(8) uint64_t full_k[kPaSlots], full_v[kPaSlots], empty[kPaSlots], qready, fin;
+    __shared__ __align__(8) uint64_t s_full[H][2], p_full[H][2], o_done[H];
+    __shared__ float xm[2][H][2][128];  // [block parity][half][column group][row]: partial maxima
     __shared__ uint32_t s_tmem;
     uint8_t* qt = dsm_raw + ((1024u - (smem_u32(dsm_raw) & 1023u)) & 1023u);  // 2 boxes x R rows x 128 B
     uint8_t* ring = qt + 2 * R * 128;
-    uint8_t* pbuf = ring + kPaSlots * kPaStage;  // [H][2] x 128 rows x 128 B
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int g = blockIdx.x;  // pair * tiles_cap + tile
     const int pair = g / a.tiles_cap, ti = g - pair * a.tiles_cap;
     const int b = pair / a.Hkv, kvh = pair - b * a.Hkv;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kPaSlots; ++i) {
-            mbar_init(&full[i], 1);
+            mbar_init(&full_k[i], 1);
+            mbar_init(&full_v[i], 1);
             mbar_init(&empty[i], 1);
         }
-        mbar_init(&qready, 128 * H);
+        mbar_init(&qready, 256 * H);
         mbar_init(&fin, 1);
         for (int h = 0; h < H; ++h) {
             for (int u = 0; u < 2; ++u) {
                 mbar_init(&s_full[h][u], 1);
-                mbar_init(&p_full[h][u], 4);
-                mbar_init(&p_free[h][u], 1);
+                mbar_init(&p_full[h][u], 8);
             }
             mbar_init(&o_done[h], 1);
         }
@@ -458,17 +478,19 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
                     break;
                 }
                 uint8_t* dst = ring + (size_t)slot * kPaStage;
-                mbar_arrive_expect_tx(&full[slot], kPaStage);
                 const int y = (int)((int64_t)pair * a.T_cap + (int64_t)blk * a.BS);
-                tma_load_2d(dst, &k_map, 0, y, &full[slot]);
-                tma_load_2d(dst + kPaBox, &k_map, 64, y, &full[slot]);
-                tma_load_2d(dst + 2 * kPaBox, &v_map, 0, y, &full[slot]);
-                tma_load_2d(dst + 3 * kPaBox, &v_map, 64, y, &full[slot]);
+                mbar_arrive_expect_tx(&full_k[slot], 2 * kPaBox);
+                tma_load_2d(dst, &k_map, 0, y, &full_k[slot]);
+                tma_load_2d(dst + kPaBox, &k_map, 64, y, &full_k[slot]);
+                mbar_arrive_expect_tx(&full_v[slot], 2 * kPaBox);
+                tma_load_2d(dst + 2 * kPaBox, &v_map, 0, y, &full_v[slot]);
+                tma_load_2d(dst + 3 * kPaBox, &v_map, 64, y, &full_v[slot]);
                 ++j;
             }
             // every copy issued has landed before the CTA ends (they already have, unless a wait gave up)
             for (int jj = max(j - kPaSlots, 0); jj < j; ++jj)
-                if (!mbar_wait(&full[jj % kPaSlots], (uint32_t)(jj / kPaSlots) & 1u, kPaPolls)) {
+                if (!mbar_wait(&full_k[jj % kPaSlots], (uint32_t)(jj / kPaSlots) & 1u, kPaPolls) ||
+                    !mbar_wait(&full_v[jj % kPaSlots], (uint32_t)(jj / kPaSlots) & 1u, kPaPolls)) {
                     atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
                     break;
                 }
@@ -481,52 +503,65 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
                 const int blk = idx[i];
                 n += (blk >= 0 && blk <= r) ? 1 : 0;
             }
-            const uint32_t qt_a = smem_u32(qt), ring_a = smem_u32(ring), p_a = smem_u32(pbuf);
-            // S_h(j) = Q_h K_j^T into buffer j & 1 of half h
-            auto issue_s = [&](int j) -> bool {
-                const int slot = j % kPaSlots;
-                if (!mbar_wait(&full[slot], (uint32_t)(j / kPaSlots) & 1u, kPaPolls)) return false;
-                tmem_fence_after_sync();
-                const uint32_t st_a = ring_a + (uint32_t)slot * kPaStage;
-                for (int h = 0; h < H; ++h) {
-                    const uint32_t d = tbase + (uint32_t)(64 * (2 * h + (j & 1)));
+            const uint32_t qt_a = smem_u32(qt), ring_a = smem_u32(ring);
+            // Whichever is ready first: S of the next block (its K landed; its TMEM buffer free once
+            // every half's P V of two blocks back is issued: that P V needed the softmax to have read
+            // the S, and it reads the P written over it before the later S, in issue order) or P V of
+            // a half whose P is written (its V landed). A K/V stage is released once every half's P V
+            // of its block is issued (the commit fires when they complete).
+            int ns = 0, npv[H], nmin = 0, ne = 0;
 #pragma unroll
-                    for (int ks = 0; ks < 8; ++ks) {
-                        const uint32_t off = (uint32_t)((ks & 3) * 32);
-                        umma_bf16(d, umma_desc_k_sw128(qt_a + (uint32_t)((ks >> 2) * R * 128 + h * 128 * 128) + off),
-                                  umma_desc_k_sw128(st_a + (uint32_t)((ks >> 2) * kPaBox) + off),
-                                  umma_idesc_bf16(128, 64), ks > 0);
-                    }
-                    umma_commit(&s_full[h][j & 1]);
-                }
-                return true;
-            };
-            bool stop = n > 0 && (!mbar_wait(&qready, 0, kPaPolls) || !issue_s(0));
-            for (int j = 0; j < n && !stop; ++j) {
-                // S of the next block goes ahead of this block's P V (its buffer was read by the
-                // softmax of block j - 1, which P V of block j - 1 waited for)
-                if (j + 1 < n && !issue_s(j + 1)) {
-                    stop = true;
-                    break;
-                }
-                const uint32_t v_a = ring_a + (uint32_t)(j % kPaSlots) * kPaStage + 2 * kPaBox;
-                for (int h = 0; h < H && !stop; ++h) {
-                    if (!mbar_wait(&p_full[h][j & 1], (uint32_t)(j >> 1) & 1u, kPaPolls)) {
-                        stop = true;
-                        break;
-                    }
+            for (int h = 0; h < H; ++h) npv[h] = 0;
+            bool stop = n > 0 && !mbar_wait(&qready, 0, kPaPolls);
+            uint32_t idle = 0;
+            while (!stop && nmin < n) {
+                bool progress = false;
+                if (ns < n && ns <= nmin + 1 &&
+                    mbar_test(&full_k[ns % kPaSlots], (uint32_t)(ns / kPaSlots) & 1u)) {
                     tmem_fence_after_sync();
-                    const uint32_t pa = p_a + (uint32_t)((2 * h + (j & 1)) * kPaPBytes);
+                    const uint32_t k_a = ring_a + (uint32_t)(ns % kPaSlots) * kPaStage;
+                    for (int h = 0; h < H; ++h) {
+                        const uint32_t d = tbase + (uint32_t)(64 * (2 * h + (ns & 1)));
+#pragma unroll
+                        for (int ks = 0; ks < 8; ++ks) {
+                            const uint32_t off = (uint32_t)((ks & 3) * 32);
+                            umma_bf16(d,
+                                      umma_desc_k_sw128(qt_a + (uint32_t)((ks >> 2) * R * 128 + h * 128 * 128) + off),
+                                      umma_desc_k_sw128(k_a + (uint32_t)((ks >> 2) * kPaBox) + off),
+                                      umma_idesc_bf16(128, 64), ks > 0);
+                        }
+                        umma_commit(&s_full[h][ns & 1]);
+                    }
+                    ++ns;
+                    progress = true;
+                }
+                for (int h = 0; h < H; ++h) {
+                    const int j = npv[h];
+                    // P of block j sits in S buffer j & 1; its barrier completes once per two blocks,
+                    // and the softmax cannot write P of block j + 2 before S of block j + 2, which
+                    // waits for this P V
+                    if (j >= ns || !mbar_test(&p_full[h][j & 1], (uint32_t)(j >> 1) & 1u) ||
+                        !mbar_test(&full_v[j % kPaSlots], (uint32_t)(j / kPaSlots) & 1u))
+                        continue;
+                    tmem_fence_after_sync();
+                    const uint32_t v_a = ring_a + (uint32_t)(j % kPaSlots) * kPaStage + 2 * kPaBox;
+                    const uint32_t pa = tbase + (uint32_t)(64 * (2 * h + (j & 1)));  // P over S of block j
                     const uint32_t d = tbase + (uint32_t)(128 * H + 128 * h);
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)  // 16 keys per MMA
-                        umma_bf16(d, umma_desc_k_sw128(pa + (uint32_t)(kk * 32)),
-                                  umma_desc_mn_sw128(v_a + (uint32_t)(kk * 2048), kPaBox), kPaIdescPV,
-                                  (j > 0 || kk > 0) ? 1u : 0u);
-                    umma_commit(&p_free[h][j & 1]);
+                    for (int kk = 0; kk < 4; ++kk)  // 16 keys (8 columns of P) per MMA
+                        umma_bf16_ts(d, pa + (uint32_t)(kk * 8),
+                                     umma_desc_mn_sw128(v_a + (uint32_t)(kk * 2048), kPaBox), kPaIdescPV,
+                                     (j > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&o_done[h]);
+                    npv[h] = j + 1;
+                    progress = true;
                 }
-                if (!stop) umma_commit(&empty[j % kPaSlots]);
+                nmin = npv[0];
+#pragma unroll
+                for (int h = 1; h < H; ++h) nmin = min(nmin, npv[h]);
+                for (; ne < nmin; ++ne) umma_commit(&empty[ne % kPaSlots]);
+                if (progress) idle = 0;
+                else if (++idle > 4 * kPaPolls) stop = true;
             }
             if (stop) atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
             // every MMA issued has completed before the tensor memory is released
@@ -535,16 +570,22 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
         }
     } else {
         // ---------------------------------------------------------------- softmax warps
-        const int h = (warp - 2) >> 2;                  // half of the tile
+        // Row m of half h is shared by the threads of column groups cg = 0 and 1 (scores 32 cg ..
+        // 32 cg + 31, O columns 64 cg .. 64 cg + 63), lane m % 32 of two warps that reach the same
+        // TMEM lanes; the pair exchanges its maxima (and at the end its sums) through shared memory
+        // behind a named barrier of its 64 threads, so both take the same rescaling decisions.
+        const int sw = warp - 2;
+        const int h = sw >> 3, cg = (sw >> 2) & 1;      // half, column group
         const int quarter = warp & 3;                   // TMEM lanes 32 * quarter ..
         const int m = 32 * quarter + lane;              // row within the half (TMEM lane)
         const int row = 128 * h + m;                    // tile row: position-in-block * G + head
         const uint32_t lane_off = (uint32_t)(32 * quarter) << 16;
+        const uint32_t pair_bar = (uint32_t)(1 + 4 * h + quarter);
         const int G = a.G;
         // the tile's rows into shared memory, K-major with the 128-byte swizzle; rows outside the
         // chunk are zero
         if (live) {
-            for (int e = threadIdx.x - 64; e < R * 16; e += 128 * H) {
+            for (int e = threadIdx.x - 64; e < R * 16; e += 256 * H) {
                 const int rr = e >> 4, ch = e & 15;
                 const int cp = rr / G, hh = rr - cp * G;
                 const int64_t p = (int64_t)a.BS * r + cp;
@@ -562,8 +603,8 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
         const int64_t pos = (int64_t)a.BS * r + cpos;
         const bool valid = live && row < 64 * G && pos >= t0 && pos < T;
         const float sl = a.scale_log2;
-        const uint32_t t_o = tbase + lane_off + (uint32_t)(128 * H + 128 * h);
-        float m_used = -INFINITY, lsum = 0.f;  // log2-domain reference maximum and sum of the row
+        const uint32_t t_o = tbase + lane_off + (uint32_t)(128 * H + 128 * h + 64 * cg);
+        float m_used = -INFINITY, lsum = 0.f;  // log2-domain reference maximum and (partial) sum of the row
         bool dead = false;
         int j = 0;
         for (int i = 0; i < nsel; ++i) {
@@ -575,28 +616,21 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
                 dead = true;
             }
             tmem_fence_after_sync();
-            float x0[32], x1[32];
-            const uint32_t t_s = tbase + lane_off + (uint32_t)(64 * (2 * h + u));
-            tmem_ld<32>(t_s, x0);
-            tmem_ld<32>(t_s + 32, x1);
+            float x[32];
+            tmem_ld<32>(tbase + lane_off + (uint32_t)(64 * (2 * h + u) + 32 * cg), x);
             tmem_wait_ld();
             // causal mask inside the tile's own block
             if (blk == r) {
 #pragma unroll
-                for (int c = 0; c < 32; ++c) {
-                    x0[c] = c <= cpos ? x0[c] : -INFINITY;
-                    x1[c] = c + 32 <= cpos ? x1[c] : -INFINITY;
-                }
+                for (int c = 0; c < 32; ++c) x[c] = 32 * cg + c <= cpos ? x[c] : -INFINITY;
             }
             float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int c = 0; c < 32; c += 2) {
-                mq[0] = fmaxf(mq[0], x0[c]);
-                mq[1] = fmaxf(mq[1], x0[c + 1]);
-                mq[2] = fmaxf(mq[2], x1[c]);
-                mq[3] = fmaxf(mq[3], x1[c + 1]);
-            }
-            const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl;  // log2 domain (sl > 0)
+            for (int c = 0; c < 32; ++c) mq[c & 3] = fmaxf(mq[c & 3], x[c]);
+            const float pm = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3]));
+            xm[u][h][cg][m] = pm;
+            asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+            const float mx = fmaxf(pm, xm[u][h][cg ^ 1][m]) * sl;  // log2 domain (sl > 0)
             // the reference maximum moves (and O and the sum are rescaled) only when the row's
             // maximum exceeds it by more than the headroom: P stays below 2^8
             const bool need = mx > m_used + kPaHeadroom;
@@ -611,7 +645,7 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
                     }
                     tmem_fence_after_sync();
 #pragma unroll 1
-                    for (int cc = 0; cc < 4; ++cc) {
+                    for (int cc = 0; cc < 2; ++cc) {
                         float o[32];
                         tmem_ld<32>(t_o + (uint32_t)(32 * cc), o);
                         tmem_wait_ld();
@@ -624,40 +658,33 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
                 lsum *= alpha;
                 m_used = mn;
             }
-            uint32_t pk[32];
+            uint32_t pk[16];
             float ps[4] = {0.f, 0.f, 0.f, 0.f};
             const float nref = m_used == -INFINITY ? 0.f : -m_used;  // a row with no finite score so far
 #pragma unroll
             for (int c = 0; c < 16; ++c) {
-                const float p0 = ex2_ftz(fmaf(x0[2 * c], sl, nref)), p1 = ex2_ftz(fmaf(x0[2 * c + 1], sl, nref));
-                const float p2 = ex2_ftz(fmaf(x1[2 * c], sl, nref)), p3 = ex2_ftz(fmaf(x1[2 * c + 1], sl, nref));
-                ps[0] += p0;
-                ps[1] += p1;
-                ps[2] += p2;
-                ps[3] += p3;
+                const float p0 = ex2_ftz(fmaf(x[2 * c], sl, nref)), p1 = ex2_ftz(fmaf(x[2 * c + 1], sl, nref));
+                ps[(2 * c) & 3] += p0;
+                ps[(2 * c + 1) & 3] += p1;
                 pk[c] = pack_bf16x2(p0, p1);
-                pk[16 + c] = pack_bf16x2(p2, p3);
             }
             lsum += (ps[0] + ps[1]) + (ps[2] + ps[3]);
-            // P buffer u was last read by P V of block j - 2
-            if (j >= 2 && !dead && !mbar_wait(&p_free[h][u], (uint32_t)((j >> 1) - 1) & 1u, kPaPolls)) {
-                atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
-                dead = true;
-            }
-            uint8_t* prow = pbuf + (size_t)(2 * h + u) * kPaPBytes + (size_t)m * 128;
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch)
-                *reinterpret_cast<uint4*>(prow + ((ch ^ (m & 7)) << 4)) =
-                    make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-            fence_proxy_async_smem();
+            // P over the row's S in TMEM (keys 32 cg .. 32 cg + 31 -> columns 16 cg .. 16 cg + 15; both
+            // threads of the row have read their S before the pair barrier above)
+            tmem_st<16>(tbase + lane_off + (uint32_t)(64 * (2 * h + u) + 16 * cg), *reinterpret_cast<float(*)[16]>(pk));
+            tmem_wait_st();
             tmem_fence_before_sync();
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[h][u]);
             ++j;
         }
-        // ---- O / sum of the row
+        // ---- the row's sum from both threads (in the maxima buffer the last block did not use),
+        // then O / sum
+        xm[j & 1][h][cg][m] = lsum;
+        asm volatile("bar.sync %0, 64;" ::"r"(pair_bar) : "memory");
+        lsum += xm[j & 1][h][cg ^ 1][m];
         const size_t orow = ((size_t)b * a.chunk + (size_t)(valid ? pos - t0 : 0)) * a.Hq + (size_t)kvh * G + hd;
-        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + orow * 128;
+        __nv_bfloat16* out = reinterpret_cast<__nv_bfloat16*>(a.out) + orow * 128 + 64 * cg;
         if (j > 0) {
             if (!dead && !mbar_wait(&o_done[h], (uint32_t)(j - 1) & 1u, kPaPolls)) {
                 atomicOr(a.err, (uint32_t)BSA_DEVERR_TIMEOUT);
@@ -666,7 +693,7 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
             tmem_fence_after_sync();
             const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
 #pragma unroll 1
-            for (int cc = 0; cc < 4; ++cc) {
+            for (int cc = 0; cc < 2; ++cc) {
                 float o[32];
                 tmem_ld<32>(t_o + (uint32_t)(32 * cc), o);
                 tmem_wait_ld();
@@ -681,9 +708,9 @@ __global__ void __launch_bounds__((2 + 4 * H) * 32, 1)
                 }
             }
         } else if (valid) {
-            for (int q4 = 0; q4 < 16; ++q4) *reinterpret_cast<uint4*>(out + 8 * q4) = make_uint4(0, 0, 0, 0);
+            for (int q4 = 0; q4 < 8; ++q4) *reinterpret_cast<uint4*>(out + 8 * q4) = make_uint4(0, 0, 0, 0);
         }
-        if (valid && a.lse)
+        if (valid && cg == 0 && a.lse)
             a.lse[orow] = lsum > 0.f ? (m_used + log2f(lsum)) * 0.69314718055994531f : -INFINITY;
     }
     tmem_fence_before_sync();
@@ -704,7 +731,7 @@ size_t prefill_select_smem_bytes(int G, int64_t nc_cap, int64_t nb_cap, int sel_
 
 size_t prefill_attend_smem_bytes(int G) {
     const int H = G > 2 ? 2 : 1;
-    return 1024 + (size_t)2 * 128 * H * 128 + (size_t)kPaSlots * kPaStage + (size_t)2 * H * kPaPBytes;
+    return 1024 + (size_t)2 * 128 * H * 128 + (size_t)kPaSlots * kPaStage;
 }
 
 cudaError_t launch_prefill_select(const PrefillArgs& a, const CUtensorMap* ck_map, size_t smem, int ctas,
@@ -728,11 +755,11 @@ cudaError_t launch_prefill_attend(const PrefillArgs& a, const CUtensorMap* k_map
     if (a.G == 2) {
         cudaError_t e = ensure_smem<prefill_attend_kernel<1>>(smem);
         if (e != cudaSuccess) return e;
-        return launch_pdl(prefill_attend_kernel<1>, dim3((unsigned)items), dim3(6 * 32), smem, st, a, *k_map, *v_map);
+        return launch_pdl(prefill_attend_kernel<1>, dim3((unsigned)items), dim3(10 * 32), smem, st, a, *k_map, *v_map);
     }
     cudaError_t e = ensure_smem<prefill_attend_kernel<2>>(smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(prefill_attend_kernel<2>, dim3((unsigned)items), dim3(10 * 32), smem, st, a, *k_map, *v_map);
+    return launch_pdl(prefill_attend_kernel<2>, dim3((unsigned)items), dim3(18 * 32), smem, st, a, *k_map, *v_map);
 }
 
 }  // namespace bsa
