@@ -414,10 +414,11 @@ __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
 }
 
 // H: 128-row halves of the tile (G = 2: one; G = 4: two). Warp 0 issues the TMA copies, warp 1
-// allocates tensor memory and one of its threads issues the MMAs; warps 2 .. 2 + 8H - 1 run the
-// softmax of half (warp - 2) / 8, two threads per tile row (its TMEM lane), 32 scores each.
+// allocates tensor memory; one thread per half issues that half's MMAs (warp 1 for half 0, warp
+// 2 + 8H for half 1); warps 2 .. 2 + 8H - 1 run the softmax of half (warp - 2) / 8, two threads per
+// tile row (its TMEM lane), 32 scores each.
 template <int H>
-__global__ void __launch_bounds__((2 + 8 * H) * 32, 1)
+__global__ void __launch_bounds__((2 + 9 * H - 1) * 32, 1)
     prefill_attend_kernel(const PrefillArgs a, const __grid_constant__ CUtensorMap k_map,
                           const __grid_constant__ CUtensorMap v_map) {
     constexpr int R = 128 * H;
@@ -436,10 +437,10 @@ __global__ void __launch_bounds__((2 + 8 * H) * 32, 1)
         for (int i = 0; i < kPaSlots; ++i) {
             mbar_init(&full_k[i], 1);
             mbar_init(&full_v[i], 1);
-            mbar_init(&empty[i], 1);
+            mbar_init(&empty[i], H);  // one release per half
         }
         mbar_init(&qready, 256 * H);
-        mbar_init(&fin, 1);
+        mbar_init(&fin, H);
         for (int h = 0; h < H; ++h) {
             for (int u = 0; u < 2; ++u) {
                 mbar_init(&s_full[h][u], 1);
@@ -495,71 +496,62 @@ __global__ void __launch_bounds__((2 + 8 * H) * 32, 1)
                     break;
                 }
         }
-    } else if (warp == 1) {
-        // ---------------------------------------------------------------- MMA issuer
+    } else if (warp == 1 || warp == 2 + 8 * H) {
+        // ---------------------------------------------------------------- MMA issuers
+        // One thread per half takes whichever is ready first: S of its next block (the K landed;
+        // the half's TMEM buffer is free once its P V of two blocks back is issued: that P V needed
+        // the softmax to have read the S, and it reads the P written over it before the later S, in
+        // issue order) or P V of its next block (the half's P written, the V landed). Each half
+        // releases a K/V stage after its P V of that block (the commit fires when its MMAs complete).
         if (lane == 0) {
+            const int h = warp == 1 ? 0 : 1;
             int n = 0;
             for (int i = 0; i < nsel; ++i) {
                 const int blk = idx[i];
                 n += (blk >= 0 && blk <= r) ? 1 : 0;
             }
             const uint32_t qt_a = smem_u32(qt), ring_a = smem_u32(ring);
-            // Whichever is ready first: S of the next block (its K landed; its TMEM buffer free once
-            // every half's P V of two blocks back is issued: that P V needed the softmax to have read
-            // the S, and it reads the P written over it before the later S, in issue order) or P V of
-            // a half whose P is written (its V landed). A K/V stage is released once every half's P V
-            // of its block is issued (the commit fires when they complete).
-            int ns = 0, npv[H], nmin = 0, ne = 0;
-#pragma unroll
-            for (int h = 0; h < H; ++h) npv[h] = 0;
+            const uint32_t q_a = qt_a + (uint32_t)(h * 128 * 128);
+            const uint32_t d_o = tbase + (uint32_t)(128 * H + 128 * h);
+            int ns = 0, npv = 0;
             bool stop = n > 0 && !mbar_wait(&qready, 0, kPaPolls);
             uint32_t idle = 0;
-            while (!stop && nmin < n) {
+            while (!stop && npv < n) {
                 bool progress = false;
-                if (ns < n && ns <= nmin + 1 &&
-                    mbar_test(&full_k[ns % kPaSlots], (uint32_t)(ns / kPaSlots) & 1u)) {
+                if (ns < n && ns <= npv + 1 && mbar_test(&full_k[ns % kPaSlots], (uint32_t)(ns / kPaSlots) & 1u)) {
                     tmem_fence_after_sync();
                     const uint32_t k_a = ring_a + (uint32_t)(ns % kPaSlots) * kPaStage;
-                    for (int h = 0; h < H; ++h) {
-                        const uint32_t d = tbase + (uint32_t)(64 * (2 * h + (ns & 1)));
+                    const uint32_t d = tbase + (uint32_t)(64 * (2 * h + (ns & 1)));
 #pragma unroll
-                        for (int ks = 0; ks < 8; ++ks) {
-                            const uint32_t off = (uint32_t)((ks & 3) * 32);
-                            umma_bf16(d,
-                                      umma_desc_k_sw128(qt_a + (uint32_t)((ks >> 2) * R * 128 + h * 128 * 128) + off),
-                                      umma_desc_k_sw128(k_a + (uint32_t)((ks >> 2) * kPaBox) + off),
-                                      umma_idesc_bf16(128, 64), ks > 0);
-                        }
-                        umma_commit(&s_full[h][ns & 1]);
+                    for (int ks = 0; ks < 8; ++ks) {
+                        const uint32_t off = (uint32_t)((ks & 3) * 32);
+                        umma_bf16(d, umma_desc_k_sw128(q_a + (uint32_t)((ks >> 2) * R * 128) + off),
+                                  umma_desc_k_sw128(k_a + (uint32_t)((ks >> 2) * kPaBox) + off),
+                                  umma_idesc_bf16(128, 64), ks > 0);
                     }
+                    umma_commit(&s_full[h][ns & 1]);
                     ++ns;
                     progress = true;
                 }
-                for (int h = 0; h < H; ++h) {
-                    const int j = npv[h];
-                    // P of block j sits in S buffer j & 1; its barrier completes once per two blocks,
-                    // and the softmax cannot write P of block j + 2 before S of block j + 2, which
-                    // waits for this P V
-                    if (j >= ns || !mbar_test(&p_full[h][j & 1], (uint32_t)(j >> 1) & 1u) ||
-                        !mbar_test(&full_v[j % kPaSlots], (uint32_t)(j / kPaSlots) & 1u))
-                        continue;
+                const int j = npv;
+                // P of block j sits in S buffer j & 1; its barrier completes once per two blocks, and
+                // the softmax cannot write P of block j + 2 before S of block j + 2, which waits for
+                // this P V
+                if (j < ns && mbar_test(&p_full[h][j & 1], (uint32_t)(j >> 1) & 1u) &&
+                    mbar_test(&full_v[j % kPaSlots], (uint32_t)(j / kPaSlots) & 1u)) {
                     tmem_fence_after_sync();
                     const uint32_t v_a = ring_a + (uint32_t)(j % kPaSlots) * kPaStage + 2 * kPaBox;
                     const uint32_t pa = tbase + (uint32_t)(64 * (2 * h + (j & 1)));  // P over S of block j
-                    const uint32_t d = tbase + (uint32_t)(128 * H + 128 * h);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)  // 16 keys (8 columns of P) per MMA
-                        umma_bf16_ts(d, pa + (uint32_t)(kk * 8),
+                        umma_bf16_ts(d_o, pa + (uint32_t)(kk * 8),
                                      umma_desc_mn_sw128(v_a + (uint32_t)(kk * 2048), kPaBox), kPaIdescPV,
                                      (j > 0 || kk > 0) ? 1u : 0u);
                     umma_commit(&o_done[h]);
-                    npv[h] = j + 1;
+                    umma_commit(&empty[j % kPaSlots]);
+                    npv = j + 1;
                     progress = true;
                 }
-                nmin = npv[0];
-#pragma unroll
-                for (int h = 1; h < H; ++h) nmin = min(nmin, npv[h]);
-                for (; ne < nmin; ++ne) umma_commit(&empty[ne % kPaSlots]);
                 if (progress) idle = 0;
                 else if (++idle > 4 * kPaPolls) stop = true;
             }
@@ -759,7 +751,7 @@ cudaError_t launch_prefill_attend(const PrefillArgs& a, const CUtensorMap* k_map
     }
     cudaError_t e = ensure_smem<prefill_attend_kernel<2>>(smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(prefill_attend_kernel<2>, dim3((unsigned)items), dim3(18 * 32), smem, st, a, *k_map, *v_map);
+    return launch_pdl(prefill_attend_kernel<2>, dim3((unsigned)items), dim3(19 * 32), smem, st, a, *k_map, *v_map);
 }
 
 }  // namespace bsa
