@@ -37,7 +37,7 @@ def oracle_problem(w: Workload, n: int, T_cap: int):
                                w.top_k, w.cmp_kernel, w.cmp_stride, w.block_size)
 
 
-class GpuRun:
+class GpuCase:
     """Buffers of one workload on the GPU, and the library calls on them."""
 
     def __init__(self, w: Workload, device="cuda", seq_lens=None, T_cap=None, steps=None):
@@ -112,7 +112,7 @@ def sample_pairs(w: Workload, n: int, seed: int = 0) -> list[int]:
     return sorted(picks)
 
 
-def oracle_on_pairs(run: GpuRun, pairs: list[int], layer=0, given_idx=None, given_n_sel=None,
+def oracle_on_pairs(run: GpuCase, pairs: list[int], layer=0, given_idx=None, given_n_sel=None,
                     q=None) -> dict:
     """Oracle over a sub-batch made of the listed pairs (one kv head each, its G query heads)."""
     w = run.w
@@ -142,7 +142,7 @@ def near_tie(boundary) -> bool:
     return abs(a - b) <= NEAR_TIE_REL * max(abs(a), abs(b))
 
 
-def check_selection(run: GpuRun, pairs: list[int], orc: dict, score_atol=None) -> list[int]:
+def check_selection(run: GpuCase, pairs: list[int], orc: dict, score_atol=None) -> list[int]:
     """Compare the GPU selection of the listed pairs with the oracle. Returns the indices (into
     ``pairs``) of near-tie pairs whose GPU selection may legitimately differ.
 
@@ -207,7 +207,7 @@ def topk_union_of(scores: np.ndarray, nb: int, n_init: int, n_local: int, top_k:
     return list(range(init_end)) + sorted(order[:kk].tolist()) + list(range(chi, nb))
 
 
-def check_output(run: GpuRun, pairs: list[int], orc: dict, layer=0, skip=()):
+def check_output(run: GpuCase, pairs: list[int], orc: dict, layer=0, skip=()):
     w = run.w
     G, Hkv = w.group, w.num_kv_heads
     out = run.out[layer].float().cpu().numpy().astype(np.float64)
@@ -228,7 +228,7 @@ def check_output(run: GpuRun, pairs: list[int], orc: dict, layer=0, skip=()):
             assert lerr <= ltol, f"pair {pr}: lse err {lerr:.3g} > {ltol}"
 
 
-def oracle_idx_tensor(run: GpuRun, pairs: list[int], orc: dict):
+def oracle_idx_tensor(run: GpuCase, pairs: list[int], orc: dict):
     """GPU block_idx/n_sel with the listed pairs' rows replaced by the oracle's selection."""
     idx = run.block_idx.clone()
     ns = run.n_sel.clone()
@@ -239,7 +239,7 @@ def oracle_idx_tensor(run: GpuRun, pairs: list[int], orc: dict):
     return idx, ns
 
 
-def forecast_check(run: GpuRun, pairs: list[int], f: torch.Tensor):
+def forecast_check(run: GpuCase, pairs: list[int], f: torch.Tensor):
     """Forecast-indexer selection on the GPU (already run into run.block_idx / block_scores) and
     the decode of q over it, vs the oracle on the sampled pairs. Block scores are raw fp32 dot
     products f . K~_j: their tolerance is 1e-5 * |f|_1 * max|K| of the pair (fp32 accumulation of
@@ -271,7 +271,7 @@ def forecast_check(run: GpuRun, pairs: list[int], f: torch.Tensor):
     return orc, ties
 
 
-def full_check(run: GpuRun, pairs: list[int], layer=0):
+def full_check(run: GpuCase, pairs: list[int], layer=0):
     """Select + decode on the GPU vs the oracle for the sampled pairs, with the near-tie rule."""
     orc = oracle_on_pairs(run, pairs, layer)
     ties = check_selection(run, pairs, orc)

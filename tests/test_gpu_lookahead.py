@@ -14,7 +14,7 @@ import torch
 import block_sparse_attention_compressed_b200 as bsa
 import oracle
 from block_sparse_attention_compressed_b200.workloads import WORKLOADS
-from gpu_helpers import (GpuRun, check_output, check_selection, oracle_problem, sample_pairs)
+from gpu_helpers import (GpuCase, check_output, check_selection, oracle_problem, sample_pairs)
 
 pytestmark = pytest.mark.gpu
 
@@ -45,11 +45,11 @@ def _forecast(w, seed):
 
 
 class Lookahead:
-    """A GpuRun with the next layer's selection buffers and the lookahead call."""
+    """A GpuCase with the next layer's selection buffers and the lookahead call."""
 
     def __init__(self, case):
         w, lens = CASES[case]
-        self.w, self.run = w, GpuRun(w, seq_lens=lens)
+        self.w, self.run = w, GpuCase(w, seq_lens=lens)
         self.run.compress()
         s = self.run.sizes
         B, Hkv = w.batch, w.num_kv_heads

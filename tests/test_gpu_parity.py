@@ -10,7 +10,7 @@ import torch
 import block_sparse_attention_compressed_b200 as bsa
 import oracle
 from block_sparse_attention_compressed_b200.workloads import WORKLOADS, Workload
-from gpu_helpers import (GpuRun, check_output, check_selection, forecast_check, full_check,
+from gpu_helpers import (GpuCase, check_output, check_selection, forecast_check, full_check,
                          near_tie, oracle_on_pairs, sample_pairs)
 
 pytestmark = pytest.mark.gpu
@@ -43,7 +43,7 @@ SMALL = {
 @pytest.mark.parametrize("case", sorted(SMALL))
 def test_small_select_and_decode(case, cuda_device):
     w = SMALL[case]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     run.select()
     run.decode()
@@ -55,7 +55,7 @@ def test_small_select_and_decode(case, cuda_device):
                                   "bf16-g2-d64-bs32-l16s8"])
 def test_compress_bit_exact(case, cuda_device):
     w = SMALL[case]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     P = oracle.make_problem(w.batch, w.num_q_heads, w.num_kv_heads, w.head_dim, run.T_cap,
                             oracle.F32 if w.dtype == "f32" else oracle.BF16, w.n_init, w.n_local,
@@ -69,7 +69,7 @@ def test_compress_bit_exact(case, cuda_device):
 def test_ragged_batch_lengths(cuda_device):
     """Sequences of different lengths in one batch, down to no window (T < l) and empty (T = 0)."""
     w = BASE.replace(name="x", batch=5, seq_len=5000, top_k=9, needles=3)
-    run = GpuRun(w, seq_lens=[5000, 64, 31, 0, 4097])
+    run = GpuCase(w, seq_lens=[5000, 64, 31, 0, 4097])
     # rows past each sequence's length hold random data here; the kernels must never read them
     run.data["k"][0].view(-1)[:] = run.data["k"][0].view(-1).flip(0)
     run.compress()
@@ -89,7 +89,7 @@ def test_equal_scores_take_lowest_blocks(cuda_device):
     candidate blocks are taken."""
     w = BASE.replace(name="x", batch=1, num_q_heads=4, num_kv_heads=1, seq_len=5000, top_k=8,
                      needles=0)
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.data["q"][0].zero_()
     run.compress()
     run.select()
@@ -109,7 +109,7 @@ def test_periodic_keys_many_ties(seq_len, cuda_device):
     largest sits in a group of equal scores (about 80 or 160 of them), ranked by block index."""
     w = BASE.replace(name="x", batch=1, num_q_heads=8, num_kv_heads=2, seq_len=seq_len, top_k=50,
                      needles=0)
-    run = GpuRun(w)
+    run = GpuCase(w)
     k = run.data["k"][0]
     period = 256
     reps = -(-seq_len // period)
@@ -126,7 +126,7 @@ def test_long_context_large_block_count(cuda_device):
     """nb_cap = 16384 blocks: the selection keeps 64 KB of keys in shared memory."""
     w = BASE.replace(name="x", batch=1, num_q_heads=4, num_kv_heads=1, seq_len=300000, top_k=40,
                      needles=10)
-    run = GpuRun(w, T_cap=1 << 20)
+    run = GpuCase(w, T_cap=1 << 20)
     run.compress()
     run.select()
     run.decode()
@@ -142,7 +142,7 @@ def test_one_cta_per_pair_selection_every_group_size(q_heads, kv_heads, d, cuda_
     B = -(-80 // kv_heads)
     w = BASE.replace(name="x", batch=B, num_q_heads=q_heads, num_kv_heads=kv_heads, head_dim=d,
                      seq_len=3000 + 11, top_k=9, needles=3)
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     run.select()
     run.decode()
@@ -155,7 +155,7 @@ def test_select_streams_rows_longer_than_the_ring(cuda_device):
     """80 pairs get one selection CTA each; at T = 150000 a pair's 9374 windows of window terms
     (150 KB) exceed the 128 KB shared-memory ring, so the stages are refilled as they are read."""
     w = BASE.replace(name="x", batch=10, seq_len=150000, top_k=16, needles=4)
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     run.select()
     run.decode()
@@ -169,7 +169,7 @@ def test_decode_with_given_indices_any_order(cuda_device):
     """Eq. 5 only depends on the set of blocks: shuffled indices and -1 holes give the same
     output as the oracle on the same set."""
     w = SMALL["bf16-g4-d128-ragged"]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     run.select()
     pairs = list(range(w.batch * w.num_kv_heads))
@@ -188,7 +188,7 @@ def test_decode_with_given_indices_any_order(cuda_device):
 
 def test_deterministic(cuda_device):
     w = SMALL["bf16-g4-d128-ragged"]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     outs = []
     for _ in range(2):
@@ -206,7 +206,7 @@ def test_decode_step_entry_point(cuda_device):
     a pair's blocks in one softmax pass: its output rounds differently from the split partials of
     bsa_sparse_decode, so outputs are checked against the oracle's tolerance, not bit for bit.)"""
     w = SMALL["bf16-g4-d128-ragged"]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     run.select()
     ref = (run.block_idx.clone(), run.n_sel.clone(), run.block_scores.clone())
@@ -224,7 +224,7 @@ def test_decode_step_entry_point(cuda_device):
 def test_cuda_graph_replay(cuda_device):
     """The step can be captured in a CUDA graph (launch attributes included) and replayed."""
     w = SMALL["bf16-g4-d128-ragged"]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     run.step()
     ref = run.out[0].clone()
@@ -249,7 +249,7 @@ def test_append_matches_full_compression(cuda_device):
     """Appending tokens one by one (new windows completed on the fly) gives the same compressed keys
     as compressing the final cache, bit for bit, and as the oracle."""
     w = BASE.replace(name="x", batch=3, seq_len=100, top_k=2, needles=0)
-    run = GpuRun(w, T_cap=200, steps=0)
+    run = GpuCase(w, T_cap=200, steps=0)
     run.data["seq_lens"] = torch.tensor([100, 31, 47], dtype=torch.int32, device="cuda")
     run.compress()
     g = torch.Generator(device="cuda").manual_seed(9)
@@ -272,7 +272,7 @@ def test_append_matches_full_compression(cuda_device):
 
 def test_append_capacity_flag(cuda_device):
     w = BASE.replace(name="x", batch=2, seq_len=64, top_k=1, needles=0)
-    run = GpuRun(w, T_cap=65, steps=0)
+    run = GpuCase(w, T_cap=65, steps=0)
     run.data["seq_lens"] = torch.tensor([64, 65], dtype=torch.int32, device="cuda")
     kn = torch.ones(w.batch, w.num_kv_heads, w.head_dim, dtype=w.torch_dtype, device="cuda")
     bsa.bsa_compress_append(run.p, run.data["k"][0], run.data["v"][0], kn, kn,
@@ -284,7 +284,7 @@ def test_append_capacity_flag(cuda_device):
 
 def test_device_error_flags(cuda_device):
     w = BASE.replace(name="x", batch=2, seq_len=640, top_k=2, needles=0)
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     run.data["seq_lens"][1] = run.T_cap + 5          # beyond capacity: pair skipped, flagged
     run.select()
@@ -302,7 +302,7 @@ def test_device_error_flags(cuda_device):
 # ------------------------------------------------------------------------------- full workloads
 def _full_run(name):
     w = WORKLOADS[name]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     return w, run
 
@@ -333,7 +333,7 @@ def test_back_to_back_calls_are_stable(cuda_device):
     through programmatic dependent launch and the persistent rings run at full speed) give the
     first call's results bit for bit and raise no device error: pipeline races show up here."""
     w = WORKLOADS["gqa4-bf16-128k-b16"]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     run.select()
     run.decode()
@@ -386,7 +386,7 @@ def test_full_append_workload(cuda_device):
     completion; then the compressed keys and the last step are checked against the oracle."""
     w = WORKLOADS["append-bf16-16k-b128"]
     steps = 20
-    run = GpuRun(w, steps=steps)
+    run = GpuCase(w, steps=steps)
     run.compress()
     d = run.data
     for i in range(steps):
@@ -437,7 +437,7 @@ def test_forecast_select_and_decode(case, cuda_device):
     """Blocks chosen by one Forecast vector per group (raw scores f . K~, no softmax), attended by
     the group's queries."""
     w = FORECAST[case]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     f = run.data["f"]
     bsa.bsa_select_blocks_forecast(run.p, f, run.ck[0], run.data["seq_lens"], run.block_idx,
@@ -450,7 +450,7 @@ def test_forecast_select_and_decode(case, cuda_device):
 def test_forecast_ragged_lengths(cuda_device):
     """Different lengths in one batch, down to no window and an empty sequence."""
     w = BASE.replace(name="x", batch=5, seq_len=5000, top_k=9, needles=3, forecast=True)
-    run = GpuRun(w, seq_lens=[5000, 64, 31, 0, 4097])
+    run = GpuCase(w, seq_lens=[5000, 64, 31, 0, 4097])
     run.compress()
     bsa.bsa_select_blocks_forecast(run.p, run.data["f"], run.ck[0], run.data["seq_lens"],
                                    run.block_idx, run.n_sel, run.block_scores, run.ws)
@@ -462,7 +462,7 @@ def test_forecast_ragged_lengths(cuda_device):
 @pytest.mark.slow
 def test_forecast_full_workload(cuda_device):
     w = WORKLOADS["forecast-bf16-128k-b16"]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     bsa.bsa_select_blocks_forecast(run.p, run.data["f"], run.ck[0], run.data["seq_lens"],
                                    run.block_idx, run.n_sel, run.block_scores, run.ws)
@@ -486,7 +486,7 @@ def test_anchored_reuse(anchors, dtype, cuda_device):
     attend those blocks."""
     w = BASE.replace(name="x", batch=2, seq_len=3000 + 29, top_k=6, needles=3, layers=4,
                      anchors=anchors, dtype=dtype)
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     A, s = len(anchors), run.sizes
     idx = torch.full((A, w.batch, w.num_kv_heads, s.sel_cap), -7, dtype=torch.int32, device="cuda")

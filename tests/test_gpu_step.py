@@ -17,7 +17,7 @@ import torch
 
 import block_sparse_attention_compressed_b200 as bsa
 from block_sparse_attention_compressed_b200.workloads import WORKLOADS
-from gpu_helpers import GpuRun, full_check, sample_pairs
+from gpu_helpers import GpuCase, full_check, sample_pairs
 
 pytestmark = pytest.mark.gpu
 
@@ -61,7 +61,7 @@ STEP = {
 
 def _run(case):
     w, lens = STEP[case]
-    run = GpuRun(w, seq_lens=lens)
+    run = GpuCase(w, seq_lens=lens)
     if lens is not None:
         # rows past each sequence's length hold other data here; they must never be read
         run.data["k"][0].view(-1)[:] = run.data["k"][0].view(-1).flip(0)

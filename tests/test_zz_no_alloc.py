@@ -9,7 +9,7 @@ import torch
 
 import block_sparse_attention_compressed_b200 as bsa
 from block_sparse_attention_compressed_b200.workloads import WORKLOADS
-from gpu_helpers import LSE_ATOL, OUT_ATOL, GpuRun
+from gpu_helpers import LSE_ATOL, OUT_ATOL, GpuCase
 
 CASES = {
     "gqa4-bf16-128k-b16": WORKLOADS["gqa4-bf16-128k-b16"],
@@ -23,7 +23,7 @@ CASES = {
 @pytest.mark.parametrize("name", list(CASES))
 def test_noalloc_matches_workspace_decode(name, cuda_device):
     w = CASES[name]
-    run = GpuRun(w)
+    run = GpuCase(w)
     run.compress()
     run.select()
     run.decode()  # the workspace entry point
