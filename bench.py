@@ -15,7 +15,7 @@ copied in from pinned host memory and its outputs (every layer) copied back. The
 double-buffered on two copy streams, so a step's transfers overlap its neighbours' compute.
 ``roofline`` is for the largest single launch of the step (the fused step kernel where
 bsa_decode_step runs one, else the sparse attention with its combine), from a second, identical pass
-that brackets every library call with CUDA events; the benchmark spec is the whole step's algorithmic
+that brackets every library call with CUDA events; ``hbm_target`` is the whole step's algorithmic
 bytes over 8 TB/s against the 0.70 target. ``cpu_baseline`` (rank 0, one GPU only) and ``--impl
 reference`` time the CPU oracle's decode step (keys compressed beforehand, as at decode time) on a
 bounded sample of the same workload, on all host cores and on one.
@@ -50,7 +50,7 @@ KERNEL_OF_PHASE = {"step": {"bf16": "step_kernel"},
                    "append": {"bf16": "append_kernel", "f32": "append_kernel"},
                    "select": {"bf16": "score_tma_kernel+select_kernel",
                               "f32": "score_f32_kernel+select_kernel"}}
-NORTH_STAR_FRAC = 0.70  # of 8 TB/s, for the fused select + sparse attention at 128K
+TARGET_FRAC_OF_8TBS = 0.70  # of 8 TB/s, for the fused select + sparse attention at 128K
 L2_BYTES = 126 * 1024 * 1024
 NOMINAL_HBM_GBS = 8000.0
 
@@ -890,10 +890,10 @@ def run_bsa(args, w, world, rank, local):
         "tokens_per_s": round(steps_per_s * w.batch * (w.prefill_chunk or 1), 1),
         "hbm_gbs": round(gbs / world, 1),
         "frac_of_8tbs": round(gbs / world / NOMINAL_HBM_GBS, 4),
-        "north_star": None if bench.prefill else {
+        "hbm_target": None if bench.prefill else {
             "basis": "compressed keys + selected K/V + q + out bytes of the whole step over 8 TB/s, "
                      "device-timed step", "frac_of_8tbs": round(gbs / world / NOMINAL_HBM_GBS, 4),
-            "target": NORTH_STAR_FRAC, "met": bool(gbs / world / NOMINAL_HBM_GBS >= NORTH_STAR_FRAC)},
+            "target": TARGET_FRAC_OF_8TBS, "met": bool(gbs / world / NOMINAL_HBM_GBS >= TARGET_FRAC_OF_8TBS)},
         "ms_per_step_one_step_graphs": (round(one_step_graphs_ms, 5) if one_step_graphs_ms is not None
                                         else None),
         "fused_step": bool(bench.fused),
